@@ -1,0 +1,97 @@
+"""Chunkwise-parallel (WY / UT-transform) evaluation of the gated delta rule, NumPy fp64.
+
+TEST INFRASTRUCTURE ONLY. This is not the oracle the GPU is compared against;
+it shows, on small inputs, that the chunk algebra reproduces the sequential
+definition (``oracle.fwd``). The pages name the chunk-parallel scheme (FG2-GDN
+page, section 2.A: the rank-1 structure that the WY representation needs, and
+section 3 item 2: the diagonal-plus-low-rank structure reused by KDA's chunk
+algorithm; OSDN page, section 2.1: only K -> K~ changes in the block Gram matrix
+and the intra-block scores) but print no formulas for it; the algebra below is
+derived from the recurrence.
+
+Within one chunk of n tokens (t = 1..n), with start state S and per-key-channel
+log-decay prefix g_t = sum_{s<=t} log alpha_s (g_0 = 0), pick a reference point
+m in {0..n} and write e(x) = exp(x) elementwise:
+
+  K+_t = k_t (.) e(g_t - g_m)          Q+_t = q_t (.) e(g_t - g_m)
+  W-_t = w_t (.) e(g_m - g_t)          V~_t = beta^v_t (.) v_t,  w_t = beta^k_t (.) d_t (.) k_t
+  S_m  = Diag(e(g_m)) S                (state decayed to the reference point)
+  L    = strictly-lower(K+ W-^T)       T = (I + L)^{-1}       (the UT transform)
+  U    = T (V~ - K+ S_m)               (all residuals u_t of the chunk)
+  O    = Q+ S_m + lower-incl(Q+ W-^T) U
+  S'   = Diag(e(g_n - g_m)) (S_m + W-^T U)
+
+m = 0 is the chunk-start reference; m = n // 2 (the midpoint) keeps every
+exponent within half a chunk of decay, which is the form the kernels use.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _gate(x, t0, t1, width):
+    """Gate values for tokens [t0, t1) of one head, broadcast to [n, width]."""
+    if x is None:
+        return np.ones((t1 - t0, width))
+    x = np.asarray(x, dtype=np.float64)
+    if x.ndim == 1:
+        return np.repeat(x[t0:t1, None], width, axis=1)
+    return x[t0:t1]
+
+
+def head_fwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, C: int, ref: str = "mid"):
+    """One head. q, k [T,dk]; v [T,dv]; gates [T] or [T,n] or None; S [dk,dv] (copied).
+
+    Returns (o [T,dv], S_T [dk,dv]).
+    """
+    T, dk = q.shape
+    dv = v.shape[1]
+    S = np.array(S, dtype=np.float64, copy=True)
+    o = np.zeros((T, dv))
+    for c0 in range(0, T, C):
+        c1 = min(T, c0 + C)
+        n = c1 - c0
+        a = _gate(alpha, c0, c1, dk)
+        g = np.concatenate([np.zeros((1, dk)), np.cumsum(np.log(a), axis=0)])  # g[0..n]
+        m = n // 2 if ref == "mid" else 0
+        gt = g[1:]                                                              # g_t, t = 1..n
+        w = _gate(beta_k, c0, c1, dk) * _gate(key_scale, c0, c1, dk) * k[c0:c1]
+        Kp = k[c0:c1] * np.exp(gt - g[m])
+        Qp = q[c0:c1] * np.exp(gt - g[m])
+        Wm = w * np.exp(g[m] - gt)
+        Vt = _gate(beta_v, c0, c1, dv) * v[c0:c1]
+        Sm = np.exp(g[m])[:, None] * S
+        L = np.tril(Kp @ Wm.T, k=-1)
+        Tm = np.linalg.inv(np.eye(n) + L)
+        U = Tm @ (Vt - Kp @ Sm)
+        P = np.tril(Qp @ Wm.T)
+        o[c0:c1] = Qp @ Sm + P @ U
+        S = np.exp(g[n] - g[m])[:, None] * (Sm + Wm.T @ U)
+    return o, S
+
+
+def fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, C: int = 64,
+        ref: str = "mid"):
+    """All heads, public layouts (q [B,T,H,dk] ...), fp64 inputs. Returns (o, S_T)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+
+    def sl(x, b, h):
+        if x is None:
+            return None
+        x = np.asarray(x, dtype=np.float64)
+        return x[b, :, h] if x.ndim == 3 else x[b, :, h, :]
+
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float64)[b, h]
+            ob, Sb = head_fwd(q[b, :, h], k[b, :, h], v[b, :, h], sl(alpha, b, h), sl(beta_k, b, h),
+                              sl(beta_v, b, h), sl(key_scale, b, h), S, C, ref)
+            o[b, :, h] = ob
+            ST[b, h] = Sb
+    return o, ST

@@ -1,0 +1,145 @@
+/*
+ * fp64 CPU oracle of the gated delta-rule recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library. It shares no code with
+ * the CUDA path and is deliberately plain: one sequential loop over tokens per
+ * (batch, head), in double precision, written straight from the definitions.
+ *
+ * Definitions followed (key-major state S in R^{dk x dv}):
+ *   decay     S_bar = Diag(alpha_t) S_{t-1}
+ *             scalar alpha: Gated DeltaNet forget gate (FG2-GDN page, section 1;
+ *             Sparse Delta Memory page, "Gated Delta Updates", forget gate applied
+ *             before the delta step); vector alpha in R^dk: KDA channel-wise decay
+ *             (FG2-GDN page, section 1).
+ *   write key w_t = beta^k_t (.) d_t (.) k_t
+ *             vector beta^k: FG2-GDN+ erase strength (FG2-GDN page, section 2.B);
+ *             d_t: OSDN preconditioner applied as a write-key scaling
+ *             (OSDN page, section 2.1, the right-preconditioning identity).
+ *   residual  u_t = beta^v_t (.) v_t - S_bar^T k_t
+ *             the prediction uses the raw key k_t (OSDN page, section 2.1: the
+ *             residual v - S k keeps the unscaled key); beta^v is the FG2-GDN+
+ *             write strength (FG2-GDN page, section 2.B).
+ *   update    S_t = S_bar + w_t u_t^T
+ *             = (I - w_t k_t^T) Diag(alpha_t) S_{t-1} + w_t (beta^v_t (.) v_t)^T,
+ *             the delta rule as one online-gradient step on 0.5 ||S k - v||^2
+ *             (OSDN page, section 1), transposed to the key-major orientation.
+ *   readout   o_t = S_t^T q_t  (after the update, no 1/sqrt(dk) scaling)
+ *
+ * Gate widths: 0 = absent (the gate is 1), 1 = one value per token, n = one value
+ * per channel (n = dk for alpha, beta^k, d; n = dv for beta^v).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static inline double gate(const double* g, int width, int t, int i) {
+  if (width == 0) return 1.0;
+  if (width == 1) return g[t];
+  return g[(int64_t)t * width + i];
+}
+
+/*
+ * One (batch, head) sequence.
+ *   q, k: [T][dk]   v: [T][dv]   gates: [T][width]
+ *   S:    [dk][dv]  in: initial state, out: final state
+ *   o:    [T][dv]
+ * Returns 0, or -1 on a bad argument / allocation failure.
+ */
+int dn_oracle_head(int T, int dk, int dv, const double* q, const double* k, const double* v,
+                   const double* alpha, int alpha_w, const double* beta_k, int bk_w,
+                   const double* beta_v, int bv_w, const double* key_scale, int d_w, double* S,
+                   double* o) {
+  if (T < 0 || dk <= 0 || dv <= 0 || !S) return -1;
+  if (!(alpha_w == 0 || alpha_w == 1 || alpha_w == dk)) return -1;
+  if (!(bk_w == 0 || bk_w == 1 || bk_w == dk)) return -1;
+  if (!(bv_w == 0 || bv_w == 1 || bv_w == dv)) return -1;
+  if (!(d_w == 0 || d_w == 1 || d_w == dk)) return -1;
+  double* w = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* u = (double*)malloc(sizeof(double) * (size_t)dv);
+  if (!w || !u) {
+    free(w);
+    free(u);
+    return -1;
+  }
+  for (int t = 0; t < T; ++t) {
+    const double* kt = k + (int64_t)t * dk;
+    const double* qt = q + (int64_t)t * dk;
+    const double* vt = v + (int64_t)t * dv;
+    /* S_bar = Diag(alpha_t) S_{t-1}: row i of S scales by alpha_t[i] */
+    for (int i = 0; i < dk; ++i) {
+      double a = gate(alpha, alpha_w, t, i);
+      double* Si = S + (int64_t)i * dv;
+      for (int j = 0; j < dv; ++j) Si[j] *= a;
+    }
+    /* w_t = beta^k (.) d (.) k */
+    for (int i = 0; i < dk; ++i) w[i] = gate(beta_k, bk_w, t, i) * gate(key_scale, d_w, t, i) * kt[i];
+    /* u_t = beta^v (.) v - S_bar^T k */
+    for (int j = 0; j < dv; ++j) u[j] = gate(beta_v, bv_w, t, j) * vt[j];
+    for (int i = 0; i < dk; ++i) {
+      const double* Si = S + (int64_t)i * dv;
+      double ki = kt[i];
+      for (int j = 0; j < dv; ++j) u[j] -= Si[j] * ki;
+    }
+    /* S_t = S_bar + w u^T */
+    for (int i = 0; i < dk; ++i) {
+      double* Si = S + (int64_t)i * dv;
+      double wi = w[i];
+      for (int j = 0; j < dv; ++j) Si[j] += wi * u[j];
+    }
+    /* o_t = S_t^T q_t */
+    double* ot = o + (int64_t)t * dv;
+    for (int j = 0; j < dv; ++j) ot[j] = 0.0;
+    for (int i = 0; i < dk; ++i) {
+      const double* Si = S + (int64_t)i * dv;
+      double qi = qt[i];
+      for (int j = 0; j < dv; ++j) ot[j] += Si[j] * qi;
+    }
+  }
+  free(w);
+  free(u);
+  return 0;
+}
+
+/*
+ * NH independent heads, each laid out contiguously ([NH][T][...], [NH][dk][dv]).
+ * A gate pointer may be NULL exactly when its width is 0. Heads run in parallel
+ * on `nthreads` OpenMP threads (<= 0: the OpenMP default). Returns 0 or -1.
+ */
+int dn_oracle_heads(int NH, int T, int dk, int dv, const double* q, const double* k,
+                    const double* v, const double* alpha, int alpha_w, const double* beta_k,
+                    int bk_w, const double* beta_v, int bv_w, const double* key_scale, int d_w,
+                    double* S, double* o, int nthreads) {
+  if (NH < 0) return -1;
+  int bad = 0;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int h = 0; h < NH; ++h) {
+    int64_t tk = (int64_t)h * T * dk, tv = (int64_t)h * T * dv;
+    int rc = dn_oracle_head(
+        T, dk, dv, q + tk, k + tk, v + tv, alpha ? alpha + (int64_t)h * T * alpha_w : NULL, alpha_w,
+        beta_k ? beta_k + (int64_t)h * T * bk_w : NULL, bk_w,
+        beta_v ? beta_v + (int64_t)h * T * bv_w : NULL, bv_w,
+        key_scale ? key_scale + (int64_t)h * T * d_w : NULL, d_w, S + (int64_t)h * dk * dv, o + tv);
+    bad |= (rc != 0);
+  }
+  return bad ? -1 : 0;
+}
+
+/* Number of threads an OpenMP parallel region would use (for reporting). */
+int dn_oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
