@@ -1,0 +1,407 @@
+"""Benchmark of the gated delta-rule hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-decode]
+
+One step = one dn_chunk_fwd over the GDN prefill workload (B=8, H=16, T=4096,
+d_k=d_v=128, bf16 q/k/v, scalar fp32 gates, chunk 64) with inputs resident in
+HBM. The same run also times the decode workload (1024 sequences x 32 heads,
+d=128, fp32 state of 2 GiB updated in place, 100 consecutive steps) and reports
+its HBM throughput. Prints ONE JSON line on rank 0.
+
+Multi-GPU (torchrun): heads are independent, so every rank runs its own full
+workload with no collective on the data path (weak scaling); the time is the
+max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores over a bounded
+sample of the same workload (there is no upstream code to run).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dn_inputs as di  # noqa: E402
+
+METRIC = "tokens/s gated-delta chunk fwd (H=16,d=128,T=4096); decode GB/s; % roofline"
+WORKLOAD = "gdn_prefill"
+DECODE = "decode"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def algorithmic_bytes(w: di.Workload) -> int:
+    """HBM bytes one dn_chunk_fwd must move: read q, k, v, gates, S0; write o, S_T."""
+    es = 2 if w.io == "bf16" else 4
+    ntok = w.B * w.T * w.H
+    b = ntok * (2 * w.dk + w.dv) * es + ntok * w.dv * es
+    for mode, width in ((w.alpha, w.dk), (w.beta_k, w.dk), (w.beta_v, w.dv), (w.key_scale, w.dk)):
+        if mode == di.GATE_SCALAR:
+            b += ntok * 4
+        elif mode == di.GATE_CHANNEL:
+            b += ntok * width * 4
+    sbytes = w.B * w.H * w.dk * w.dv * 4
+    b += sbytes * (2 if w.s0_std > 0 else 1)
+    return b
+
+
+def decode_bytes(w: di.Workload) -> int:
+    """HBM bytes of one decode step: S read + written once, plus the token's vectors and o."""
+    nh = w.B * w.H
+    b = 2 * nh * w.dk * w.dv * 4
+    b += nh * (2 * w.dk + w.dv) * 2 + nh * w.dv * 2
+    b += nh * (w.dk + w.dk + w.dv) * 4  # alpha, beta_k, beta_v (channel)
+    return b
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_linear_attention_dn_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(w: di.Workload, x: dict, budget_s: float, nthreads: int, heads_cap: int = 10 ** 9):
+    """Run the fp64 oracle over whole heads of `w` until ~budget_s of CPU work; returns
+    (head_tokens, seconds, heads)."""
+    import oracle
+    allh = [(b, h) for b in range(w.B) for h in range(w.H)]
+    done, t_total = 0, 0.0
+    step = max(1, nthreads)
+    while done < min(len(allh), heads_cap) and t_total < budget_s:
+        batch = allh[done:done + step]
+        t0 = time.perf_counter()
+        oracle.fwd(**x, heads=batch, nthreads=nthreads)
+        t_total += time.perf_counter() - t0
+        done += len(batch)
+    return done * w.T, t_total, done
+
+
+def run_reference(args, rank: int, world: int):
+    """CPU oracle arm: each step times the oracle on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import oracle
+    w = di.WORKLOADS[WORKLOAD]
+    oracle.build()
+    nthreads = oracle.max_threads()
+    # a sample of whole heads: sequences are independent, so per-head cost is exact
+    ws = w.scaled(B=1)
+    x = di.make_inputs(ws)
+    per_step_heads = max(1, nthreads)
+    for _ in range(args.warmup):
+        oracle.fwd(**x, heads=[(0, h % ws.H) for h in range(min(per_step_heads, ws.H))], nthreads=nthreads)
+    times = []
+    for s in range(args.steps):
+        hs = [(0, h % ws.H) for h in range(min(per_step_heads, ws.H))]
+        t0 = time.perf_counter()
+        oracle.fwd(**x, heads=hs, nthreads=nthreads)
+        times.append(time.perf_counter() - t0)
+    nheads = min(per_step_heads, ws.H)
+    tok_per_s = nheads * w.T / statistics.mean(times) / w.H  # sequence tokens (all H heads) per second
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "gdn_prefill B=8 H=16 T=4096 d_k=d_v=128 bf16, scalar gates",
+                   "global_batch": w.B, "seq_len": w.T, "parallelism": "cpu-oracle"},
+        "cpu_baseline": {"value": tok_per_s, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{nheads} whole heads of T={w.T} per step (all heads are independent); "
+                                   "tokens/s = head-tokens/s / H"},
+        "e2e": {"value": tok_per_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=100)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import gated_linear_attention_dn_b200 as dn
+    from gated_linear_attention_dn_b200 import build as dnbuild
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if not os.path.exists(dnbuild.LIB):
+        dnbuild.build()
+    dn.load()
+    peaks = measured_peaks()
+
+    w = di.WORKLOADS[WORKLOAD]
+    x = di.make_inputs(w)
+
+    def to_dev(a):
+        if a is None:
+            return None
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.cuda()
+
+    xd = {n: to_dev(a) for n, a in x.items()}
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device="cuda")
+    ST = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dn.dn_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                        xd["S0"], o=o, S_T=ST, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dn.dn_stream_status(stream) != dn.DN_OK:
+        raise RuntimeError("device status after warm-up")
+
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        evs[0].record(stream)
+        for i in range(args.steps):
+            step()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    per_launch_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    if dn.dn_stream_status(stream) != dn.DN_OK:
+        raise RuntimeError("device status after timed region")
+    t_max = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+    ms_per_step = total_ms / args.steps
+    tokens = B * T * world * args.steps
+    value = tokens / (total_ms * 1e-3)
+    kern_ms = statistics.mean(per_launch_ms)
+    alg = algorithmic_bytes(w)
+    achieved = alg / (kern_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic("chunk_fwd"),
+                "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg,
+                "kernel_ms": kern_ms}
+
+    # ---- end to end: pinned host buffers, H2D of the step's inputs, D2H of o and S_T
+    pin = {n: (None if t is None else t.cpu().pin_memory()) for n, t in xd.items()}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_h = torch.empty(ST.shape, dtype=ST.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values() if t is not None)
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
+
+    def e2e_step():
+        for n, t in pin.items():
+            if t is not None:
+                xd[n].copy_(t, non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        S_h.copy_(ST, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 10))
+    barrier()
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+    e2e = {"value": B * T * world * e_steps / (float(e_ms.item()) * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del pin
+
+    # ---- decode workload
+    decode = None
+    launches = args.steps
+    if not args.no_decode:
+        wd = di.WORKLOADS[DECODE]
+        nd = args.decode_steps
+        xs = [di.make_inputs(wd, step=s) for s in range(nd)]
+        S = to_dev(xs[0]["S0"])
+        steps_dev = [{n: to_dev(a) for n, a in xx.items() if n != "S0"} for xx in xs]
+        del xs
+        od = torch.empty((wd.B, 1, wd.H, wd.dv), dtype=torch.bfloat16, device="cuda")
+
+        def dstep(s):
+            z = steps_dev[s]
+            dn.dn_decode_step(z["q"], z["k"], z["v"], z["alpha"], z["beta_k"], z["beta_v"], z["key_scale"],
+                              S=S, o=od, stream=stream)
+
+        for s in range(3):
+            dstep(s)
+        torch.cuda.synchronize()
+        devs = [torch.cuda.Event(enable_timing=True) for _ in range(nd + 1)]
+        barrier()
+        devs[0].record(stream)
+        for s in range(nd):
+            dstep(s)
+            devs[s + 1].record(stream)
+        torch.cuda.synchronize()
+        if dn.dn_stream_status(stream) != dn.DN_OK:
+            raise RuntimeError("device status after decode")
+        dms = [devs[i].elapsed_time(devs[i + 1]) for i in range(nd)]
+        d_ms = statistics.mean(dms)
+        db = decode_bytes(wd)
+        gbs = db / (d_ms * 1e-3) / 1e9
+        decode = {"workload": "decode 1024 seq x 32 heads, d=128, fp32 state 2 GiB in place, channel gates",
+                  "steps": nd, "ms_per_step": d_ms, "tokens_per_s": wd.B * world / (d_ms * 1e-3),
+                  "GB/s": gbs * world,
+                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("decode"),
+                               "algorithmic_bytes_per_launch": db}}
+        launches += nd
+        del steps_dev, S
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        nthreads = oracle.max_threads()
+        head_tokens, secs, nheads = oracle_sample(w, x, budget_s=12.0, nthreads=nthreads)
+        cpu = {"value": head_tokens / secs / w.H, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+               "sample": f"{nheads} of {w.B * w.H} heads of the same workload, whole T={w.T} each "
+                         f"({secs:.1f} s); tokens/s = head-tokens/s / H"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "gdn_prefill B=8 H=16 T=4096 d_k=d_v=128 bf16 q/k/v, scalar fp32 gates, "
+                                   "chunk 64, S0=0",
+                       "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
+                       "l2": f"inputs {alg / 1e6:.0f} MB per step > {L2_BYTES / 1e6:.0f} MB L2 (no flush)"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode,
+            "kernel_source": kernel_source_hash(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

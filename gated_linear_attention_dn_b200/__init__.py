@@ -1,0 +1,179 @@
+"""Python binding of libdn.so, the B200 (sm_100a) gated delta-rule library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/dn.h. PyTorch supplies device
+memory and streams. There is no CPU path: if libdn.so is missing or cannot be
+loaded, every call raises.
+
+Entry points (same names as the C ABI):
+    dn_chunk_fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None,
+                 S0=None, o=None, S_T=None, stream=None) -> (o, S_T)
+    dn_decode_step(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None,
+                   S=..., o=None, stream=None) -> o          (S updated in place)
+    dn_stream_status(stream=None) -> int
+    dn_status_string(code) -> str
+
+Layouts: q, k [B,T,H,d_k]; v [B,T,H,d_v]; gates [B,T,H] (one per token),
+[B,T,H,n] (one per channel) or None (absent = 1); states [B,H,d_k,d_v] fp32.
+q/k/v/o are bf16 or fp32 CUDA tensors; gates fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdn.so")
+
+DN_OK, DN_ERR_INVALID_ARGUMENT, DN_ERR_UNSUPPORTED, DN_ERR_MISALIGNED = 0, 1, 2, 3
+DN_ERR_WORKSPACE_TOO_SMALL, DN_ERR_CUDA, DN_ERR_DEVICE_TIMEOUT = 4, 5, 6
+DN_F32, DN_BF16 = 0, 1
+DN_GATE_ONE, DN_GATE_SCALAR, DN_GATE_CHANNEL = 0, 1, 2
+
+EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_stream_status",
+            "dn_status_string", "dn_version")
+
+
+class DnDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
+                ("d_v", ctypes.c_int), ("chunk", ctypes.c_int), ("io_dtype", ctypes.c_int),
+                ("alpha", ctypes.c_int), ("beta_k", ctypes.c_int), ("beta_v", ctypes.c_int),
+                ("key_scale", ctypes.c_int)]
+
+
+class DnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {dn_status_string(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libdn.so (raises if it is absent: there is no fallback path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libdn.so not built at {path}; run `python -m gated_linear_attention_dn_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    D = ctypes.POINTER(DnDesc)
+    lib.dn_chunk_fwd_workspace_bytes.argtypes = [D]
+    lib.dn_chunk_fwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.dn_chunk_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.dn_chunk_fwd.restype = I
+    lib.dn_decode_step.argtypes = [D, P, P, P, P, P, P, P, P, P, P]
+    lib.dn_decode_step.restype = I
+    lib.dn_stream_status.argtypes = [P]
+    lib.dn_stream_status.restype = I
+    lib.dn_status_string.argtypes = [I]
+    lib.dn_status_string.restype = ctypes.c_char_p
+    lib.dn_version.restype = I
+    _lib = lib
+    return lib
+
+
+def dn_status_string(code: int) -> str:
+    return load().dn_status_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _gate_mode(g, B, T, H, width, name):
+    if g is None:
+        return DN_GATE_ONE
+    if g.dtype != torch.float32 or not g.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous float32 tensor")
+    if tuple(g.shape) == (B, T, H):
+        return DN_GATE_SCALAR
+    if tuple(g.shape) == (B, T, H, width):
+        return DN_GATE_CHANNEL
+    raise ValueError(f"{name} has shape {tuple(g.shape)}; expected {(B, T, H)} or {(B, T, H, width)}")
+
+
+def make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk: int = 0) -> DnDesc:
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype == torch.bfloat16:
+        io = DN_BF16
+    elif q.dtype == torch.float32:
+        io = DN_F32
+    else:
+        raise TypeError("q/k/v must be bfloat16 or float32")
+    return DnDesc(B, T, H, dk, dv, chunk, io,
+                  _gate_mode(alpha, B, T, H, dk, "alpha"), _gate_mode(beta_k, B, T, H, dk, "beta_k"),
+                  _gate_mode(beta_v, B, T, H, dv, "beta_v"), _gate_mode(key_scale, B, T, H, dk, "key_scale"))
+
+
+def _check_io(q, k, v):
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise TypeError(f"{n} must be contiguous")
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v must share a dtype")
+    if k.shape != q.shape or v.shape[:3] != q.shape[:3]:
+        raise ValueError("q, k, v shapes disagree")
+
+
+def dn_chunk_fwd_workspace_bytes(desc: DnDesc) -> int:
+    return int(load().dn_chunk_fwd_workspace_bytes(ctypes.byref(desc)))
+
+
+def dn_chunk_fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, o=None,
+                 S_T=None, stream=None, chunk: int = 0, workspace=None):
+    """Chunked prefill. Returns (o [B,T,H,d_v] io dtype, S_T [B,H,d_k,d_v] fp32)."""
+    lib = load()
+    _check_io(q, k, v)
+    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    ws_bytes = dn_chunk_fwd_workspace_bytes(desc)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    rc = lib.dn_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                          _ptr(beta_v), _ptr(key_scale), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
+                          ws_bytes if workspace is not None else 0, _stream_handle(stream))
+    if rc != DN_OK:
+        raise DnError(rc, "dn_chunk_fwd")
+    return o, S_T
+
+
+def dn_decode_step(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S=None, o=None,
+                   stream=None):
+    """One recurrent step; S [B,H,d_k,d_v] fp32 is updated in place. Returns o [B,1,H,d_v]."""
+    lib = load()
+    _check_io(q, k, v)
+    if S is None:
+        raise ValueError("decode needs the resident state S")
+    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale)
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    rc = lib.dn_decode_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
+                            _ptr(beta_v), _ptr(key_scale), _ptr(S), _ptr(o), _stream_handle(stream))
+    if rc != DN_OK:
+        raise DnError(rc, "dn_decode_step")
+    return o
+
+
+def dn_stream_status(stream=None) -> int:
+    return int(load().dn_stream_status(_stream_handle(stream)))
+
+
+def dn_version() -> int:
+    return int(load().dn_version())

@@ -1,0 +1,202 @@
+// C ABI shim: argument validation, the per-GPU status word, and dispatch to
+// the kernels. Nothing here allocates device memory.
+#include <stdint.h>
+#include <string.h>
+
+#include "dn_common.cuh"
+
+// One status word per GPU that loads the library; kernels set it when a
+// bounded wait gives up.
+__device__ int g_dn_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+
+dn_status status_ptr(int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DN_ERR_CUDA;
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dn_status) != cudaSuccess) return DN_ERR_CUDA;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return DN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool gate_ok(int mode) { return mode == DN_GATE_ONE || mode == DN_GATE_SCALAR || mode == DN_GATE_CHANNEL; }
+
+dn_status check_desc(const dn_desc* d, bool decode) {
+  if (!d) return DN_ERR_INVALID_ARGUMENT;
+  if (d->B < 1 || d->H < 1 || d->T < 0) return DN_ERR_INVALID_ARGUMENT;
+  if (decode && d->T != 1) return DN_ERR_INVALID_ARGUMENT;
+  if (d->d_k <= 0 || d->d_v <= 0) return DN_ERR_INVALID_ARGUMENT;
+  if (d->io_dtype != DN_F32 && d->io_dtype != DN_BF16) return DN_ERR_INVALID_ARGUMENT;
+  if (!gate_ok(d->alpha) || !gate_ok(d->beta_k) || !gate_ok(d->beta_v) || !gate_ok(d->key_scale))
+    return DN_ERR_INVALID_ARGUMENT;
+  if (d->chunk < 0) return DN_ERR_INVALID_ARGUMENT;
+  if (!((d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128))) return DN_ERR_UNSUPPORTED;
+  if (!(d->chunk == 0 || d->chunk == 64)) return DN_ERR_UNSUPPORTED;
+  // sizes must stay addressable with 32-bit grid math and 64-bit offsets
+  const int64_t heads = (int64_t)d->B * d->H;
+  if (heads * 2 >= (int64_t)1 << 31) return DN_ERR_UNSUPPORTED;
+  if ((int64_t)d->B * d->T * d->H * (d->d_k > d->d_v ? d->d_k : d->d_v) >= ((int64_t)1 << 46))
+    return DN_ERR_UNSUPPORTED;
+  return DN_OK;
+}
+
+// A gate pointer is present exactly when its mode is not DN_GATE_ONE (for T == 0
+// no token data is read and gate pointers may be anything, NULL included).
+dn_status check_gate_ptr(int mode, const void* p, int T) {
+  if (T > 0 && (mode == DN_GATE_ONE) != (p == nullptr)) return DN_ERR_INVALID_ARGUMENT;
+  // per-channel gates are read in 16-byte vectors; per-token gates only need fp32 alignment
+  if (p && mode == DN_GATE_CHANNEL && !aligned16(p)) return DN_ERR_MISALIGNED;
+  if (p && (reinterpret_cast<uintptr_t>(p) & 3u) != 0) return DN_ERR_MISALIGNED;
+  return DN_OK;
+}
+
+dn_status fill_args(const dn_desc* d, const void* q, const void* k, const void* v, const float* alpha,
+                    const float* beta_k, const float* beta_v, const float* key_scale, dn::Args* a) {
+  dn_status st;
+  if ((st = check_gate_ptr(d->alpha, alpha, d->T)) != DN_OK) return st;
+  if ((st = check_gate_ptr(d->beta_k, beta_k, d->T)) != DN_OK) return st;
+  if ((st = check_gate_ptr(d->beta_v, beta_v, d->T)) != DN_OK) return st;
+  if ((st = check_gate_ptr(d->key_scale, key_scale, d->T)) != DN_OK) return st;
+  if (d->T > 0) {
+    if (!q || !k || !v) return DN_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return DN_ERR_MISALIGNED;
+  }
+  memset(a, 0, sizeof(*a));
+  a->B = d->B;
+  a->T = d->T;
+  a->H = d->H;
+  a->dk = d->d_k;
+  a->dv = d->d_v;
+  a->chunk = d->chunk == 0 ? 64 : d->chunk;
+  a->io_bf16 = d->io_dtype == DN_BF16;
+  a->alpha = d->alpha;
+  a->beta_k = d->beta_k;
+  a->beta_v = d->beta_v;
+  a->key_scale = d->key_scale;
+  a->q = q;
+  a->k = k;
+  a->v = v;
+  a->alpha_p = alpha;
+  a->beta_k_p = beta_k;
+  a->beta_v_p = beta_v;
+  a->key_scale_p = key_scale;
+  return DN_OK;
+}
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dn_version(void) { return 100; }
+
+const char* dn_status_string(dn_status s) {
+  switch (s) {
+    case DN_OK: return "DN_OK";
+    case DN_ERR_INVALID_ARGUMENT: return "DN_ERR_INVALID_ARGUMENT";
+    case DN_ERR_UNSUPPORTED: return "DN_ERR_UNSUPPORTED";
+    case DN_ERR_MISALIGNED: return "DN_ERR_MISALIGNED";
+    case DN_ERR_WORKSPACE_TOO_SMALL: return "DN_ERR_WORKSPACE_TOO_SMALL";
+    case DN_ERR_CUDA: return "DN_ERR_CUDA";
+    case DN_ERR_DEVICE_TIMEOUT: return "DN_ERR_DEVICE_TIMEOUT";
+  }
+  return "DN_ERR_UNKNOWN";
+}
+
+size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc) {
+  (void)desc;
+  return 0;
+}
+
+dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta_k, const float* beta_v,
+                       const float* key_scale, const float* S0, void* o, float* S_T,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  dn_status st = check_desc(desc, false);
+  if (st != DN_OK) return st;
+  dn::Args a;
+  if ((st = fill_args(desc, q, k, v, alpha, beta_k, beta_v, key_scale, &a)) != DN_OK) return st;
+  if (!S_T) return DN_ERR_INVALID_ARGUMENT;
+  if (!aligned16(S_T) || (S0 && !aligned16(S0))) return DN_ERR_MISALIGNED;
+  if (desc->T > 0) {
+    if (!o) return DN_ERR_INVALID_ARGUMENT;
+    if (!aligned16(o)) return DN_ERR_MISALIGNED;
+    const size_t es = desc->io_dtype == DN_BF16 ? 2 : 4;
+    const size_t n_o = (size_t)desc->B * desc->T * desc->H * desc->d_v * es;
+    const size_t n_qk = (size_t)desc->B * desc->T * desc->H * desc->d_k * es;
+    const size_t n_S = (size_t)desc->B * desc->H * desc->d_k * desc->d_v * 4;
+    if (ranges_overlap(o, n_o, q, n_qk) || ranges_overlap(o, n_o, k, n_qk) ||
+        ranges_overlap(o, n_o, v, n_o) || ranges_overlap(o, n_o, S_T, n_S))
+      return DN_ERR_INVALID_ARGUMENT;
+  }
+  if ((st = status_ptr(&a.status)) != DN_OK) return st;
+  a.S0 = S0;
+  a.S = S_T;
+  a.o = o;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const size_t n_S = (size_t)desc->B * desc->H * desc->d_k * desc->d_v * sizeof(float);
+  if (desc->T == 0) {
+    cudaError_t e = S0 ? (S0 == S_T ? cudaSuccess : cudaMemcpyAsync(S_T, S0, n_S, cudaMemcpyDeviceToDevice, s))
+                       : cudaMemsetAsync(S_T, 0, n_S, s);
+    return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
+  }
+  cudaError_t e;
+  if (a.io_bf16 && dn::chunk_tc_supported(a)) {
+    e = dn::launch_chunk_tc(a, s);
+  } else {
+    e = dn::launch_seq_fwd(a, s);
+  }
+  return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
+}
+
+dn_status dn_decode_step(const dn_desc* desc, const void* q, const void* k, const void* v,
+                         const float* alpha, const float* beta_k, const float* beta_v,
+                         const float* key_scale, float* S, void* o, void* cuda_stream) {
+  dn_status st = check_desc(desc, true);
+  if (st != DN_OK) return st;
+  dn::Args a;
+  if ((st = fill_args(desc, q, k, v, alpha, beta_k, beta_v, key_scale, &a)) != DN_OK) return st;
+  if (!S || !o) return DN_ERR_INVALID_ARGUMENT;
+  if (!aligned16(S) || !aligned16(o)) return DN_ERR_MISALIGNED;
+  if ((st = status_ptr(&a.status)) != DN_OK) return st;
+  a.S0 = S;
+  a.S = S;
+  a.o = o;
+  cudaError_t e = dn::launch_decode(a, static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
+}
+
+dn_status dn_stream_status(void* cuda_stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return DN_ERR_CUDA;
+  int* p = nullptr;
+  dn_status st = status_ptr(&p);
+  if (st != DN_OK) return st;
+  int word = 0;
+  if (cudaMemcpy(&word, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DN_ERR_CUDA;
+  if (word != dn::kDevOk) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DN_ERR_CUDA;
+    return DN_ERR_DEVICE_TIMEOUT;
+  }
+  return DN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+// Shared device helpers and the host-side launch interface between the ABI
+// shim (dn_abi.cu) and the kernels (one .cu file per kernel family).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dn.h"
+
+namespace dn {
+
+// Device status codes written to the per-GPU status word (0 = fine).
+enum : int { kDevOk = 0, kDevTimeout = 1 };
+
+// Everything a kernel launch needs, already validated by the ABI shim.
+struct Args {
+  int B, T, H, dk, dv, chunk;
+  int io_bf16;                    // 1: q/k/v/o are bf16, 0: fp32
+  int alpha, beta_k, beta_v, key_scale;   // dn_gate modes
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* alpha_p;
+  const float* beta_k_p;
+  const float* beta_v_p;
+  const float* key_scale_p;
+  const float* S0;                // may be null (zero state)
+  void* o;
+  float* S;                       // S_T (chunk fwd) or the in/out state (decode)
+  int* status;                    // device status word of the current GPU
+};
+
+// Launchers (host). Each returns cudaSuccess or the launch error.
+cudaError_t launch_decode(const Args& a, cudaStream_t s);
+cudaError_t launch_seq_fwd(const Args& a, cudaStream_t s);
+cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s);
+// Largest dynamic shared memory the tensor-core chunk kernel asks for (for validation).
+bool chunk_tc_supported(const Args& a);
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ float io_load(const void* p, int64_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  return reinterpret_cast<const float*>(p)[i];
+}
+
+__device__ __forceinline__ void io_store(void* p, int64_t i, float x, int bf16) {
+  if (bf16) {
+    reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(x);
+  } else {
+    reinterpret_cast<float*>(p)[i] = x;
+  }
+}
+
+// Gate value for (row, token, channel): mode 0 -> 1, 1 -> one per token, 2 -> one per channel.
+__device__ __forceinline__ float gate_load(const float* g, int mode, int64_t tok, int width, int ch) {
+  if (mode == DN_GATE_ONE) return 1.0f;
+  if (mode == DN_GATE_SCALAR) return g[tok];
+  return g[tok * width + ch];
+}
+
+// Streaming 16-byte global load that does not allocate in L1 (the state is touched once).
+// Not the non-coherent path: the decode kernel writes the same addresses later.
+__device__ __forceinline__ float4 ld_stream_f4(const float* p) {
+  float4 r;
+  asm volatile("ld.global.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// Streaming 16-byte global store (evict-first / cache-streaming).
+__device__ __forceinline__ void st_stream_f4(float* p, float4 v) {
+  asm volatile("st.global.cs.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+
+}  // namespace dn

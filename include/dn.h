@@ -1,0 +1,144 @@
+/*
+ * dn.h -- C ABI of the B200 (sm_100a) gated delta-rule library (libdn.so).
+ *
+ * The recurrence (key-major state S in R^{d_k x d_v}, fp32), per batch b,
+ * head h and token t:
+ *
+ *   S_bar_t = Diag(alpha_t) S_{t-1}
+ *   w_t     = beta^k_t (.) d_t (.) k_t
+ *   u_t     = beta^v_t (.) v_t - S_bar_t^T k_t
+ *   S_t     = S_bar_t + w_t u_t^T
+ *           = (I - w_t k_t^T) Diag(alpha_t) S_{t-1} + w_t (beta^v_t (.) v_t)^T
+ *   o_t     = S_t^T q_t                       (read-out after the update, no 1/sqrt(d_k))
+ *
+ * Sources of each term:
+ *   - the delta rule as one online-gradient step on 0.5 ||S k - v||^2, with a
+ *     scalar write gate beta (OSDN page, section 1; delta-mem page, section 2.A);
+ *   - scalar forget gate alpha_t (Gated DeltaNet) and per-key-channel decay
+ *     alpha_t in R^{d_k} (KDA) (FG2-GDN page, section 1); decay is applied to the
+ *     state before the delta step (Sparse Delta Memory page, "Gated Delta Updates");
+ *   - vector beta^k (erase strength) and beta^v (write strength) of FG2-GDN+
+ *     (FG2-GDN page, section 2.B); FG2-GDN's symmetric form with k~ = sqrt(beta) (.) k,
+ *     v~ = sqrt(beta) (.) v (section 2.A) is this recurrence fed k' = k~,
+ *     beta^k = 1, beta^v = sqrt(beta);
+ *   - OSDN preconditioned write key k~ = d (.) k, where the residual keeps the raw
+ *     key (OSDN page, section 2.1, right-preconditioning identity).
+ *
+ * dn_chunk_fwd evaluates a whole sequence in chunkwise-parallel (WY / UT
+ * transform) form, the chunk algorithm the FG2-GDN page (sections 2.A and 3
+ * item 2) and the OSDN page (section 2.1) rely on; dn_decode_step advances a
+ * resident state by one token.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory and keeps no per-call state. The only global
+ *     state is one device status word per GPU (see dn_stream_status).
+ *   - Row-major layouts, innermost dimension last:
+ *       q, k      [B, T, H, d_k]        io dtype
+ *       v, o      [B, T, H, d_v]        io dtype
+ *       alpha     [B, T, H] (DN_GATE_SCALAR) or [B, T, H, d_k] (DN_GATE_CHANNEL), fp32
+ *       beta_k    [B, T, H] or [B, T, H, d_k], fp32
+ *       beta_v    [B, T, H] or [B, T, H, d_v], fp32
+ *       key_scale [B, T, H] or [B, T, H, d_k], fp32   (OSDN d_t)
+ *       S0, S_T, S [B, H, d_k, d_v], fp32
+ *     A gate whose mode is DN_GATE_ONE is absent (every value 1) and its pointer
+ *     must be NULL. With T == 0 no token data is read: q, k, v, o and the gate
+ *     pointers are ignored (they may be NULL).
+ *   - q, k, v, o, S0, S_T, S and per-channel gates must be 16-byte aligned;
+ *     per-token (DN_GATE_SCALAR) gates need only 4-byte alignment, so a gate
+ *     tensor sliced at any token offset is accepted.
+ *   - Calls are asynchronous on `cuda_stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Argument errors are returned synchronously before any
+ *     launch; a failed launch returns DN_ERR_CUDA. A device-side bounded wait
+ *     that gives up is reported later by dn_stream_status.
+ *   - Numerics: fp32 state, fp32 accumulation. bf16 io runs the tensor-core
+ *     chunk kernel (bf16 operands; the state-update product uses a hi/lo bf16
+ *     split); fp32 io runs an fp32 CUDA-core kernel.
+ */
+#ifndef DN_H_
+#define DN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DN_OK = 0,
+  DN_ERR_INVALID_ARGUMENT = 1,   /* null/inconsistent pointer or size, bad enum */
+  DN_ERR_UNSUPPORTED = 2,        /* valid but not implemented (d_k, d_v, chunk, dtype) */
+  DN_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+  DN_ERR_WORKSPACE_TOO_SMALL = 4,
+  DN_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+  DN_ERR_DEVICE_TIMEOUT = 6      /* a kernel's bounded wait gave up (reported by dn_stream_status) */
+} dn_status;
+
+typedef enum { DN_F32 = 0, DN_BF16 = 1 } dn_dtype;
+
+/* How a gate is given: absent (1), one value per (b, t, h), or one per channel. */
+typedef enum { DN_GATE_ONE = 0, DN_GATE_SCALAR = 1, DN_GATE_CHANNEL = 2 } dn_gate;
+
+typedef struct {
+  int B, T, H;        /* batch, tokens per sequence, heads; B, H >= 1, T >= 0 */
+  int d_k, d_v;       /* head dims; supported: d_k, d_v in {64, 128} */
+  int chunk;          /* chunk length of the WY form; 0 selects the default, 64 (the only value supported) */
+  dn_dtype io_dtype;  /* dtype of q, k, v and o */
+  dn_gate alpha;      /* forget gate: scalar (GDN) or per key channel (KDA) */
+  dn_gate beta_k;     /* erase / write strength on the key side (GDN beta; FG2-GDN+ beta^k) */
+  dn_gate beta_v;     /* write strength on the value side (FG2-GDN+ beta^v); CHANNEL means d_v wide */
+  dn_gate key_scale;  /* OSDN preconditioner d_t on the write key; CHANNEL means d_k wide */
+} dn_desc;
+
+/*
+ * Bytes of workspace dn_chunk_fwd needs for this descriptor. The current
+ * kernels keep every intermediate on chip and need none (returns 0); the
+ * argument is kept so a future path (e.g. a segment-parallel state scan) can
+ * ask for scratch without an ABI change. Returns 0 for an invalid descriptor.
+ */
+size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc);
+
+/*
+ * Chunked prefill (FG2-GDN page, sections 2.A and 3 item 2: the DPLR update that
+ * keeps the WY chunk-parallel algorithm; OSDN page, section 2.1: only K -> d (.) K
+ * changes in the block Gram matrix and intra-block scores).
+ *
+ * In:  q, k, v, gates as laid out above; S0 = initial state or NULL (zero).
+ * Out: o [B,T,H,d_v] (io dtype), S_T [B,H,d_k,d_v] fp32 (final state).
+ * S_T may alias S0 (in-place resume). q, k, v, o must not overlap each other or
+ * S_T. `workspace` may be NULL when dn_chunk_fwd_workspace_bytes() is 0.
+ * T == 0 copies S0 (or zeros) into S_T and writes no o.
+ */
+dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta_k, const float* beta_v,
+                       const float* key_scale, const float* S0, void* o, float* S_T,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * One recurrent step (desc->T must be 1): S <- S_1, o <- S_1^T q, in place.
+ * In:  q, k [B,1,H,d_k], v [B,1,H,d_v], gates for one token, S [B,H,d_k,d_v] fp32.
+ * Out: S updated in place, o [B,1,H,d_v] (io dtype).
+ * Each (b, h) state is read once and written once (HBM-streaming kernel).
+ */
+dn_status dn_decode_step(const dn_desc* desc, const void* q, const void* k, const void* v,
+                         const float* alpha, const float* beta_k, const float* beta_v,
+                         const float* key_scale, float* S, void* o, void* cuda_stream);
+
+/*
+ * Synchronises `cuda_stream`, then reports (and clears) the device status word
+ * that kernels set when a bounded wait gives up (DN_ERR_DEVICE_TIMEOUT), or
+ * DN_ERR_CUDA if the stream holds a CUDA error. DN_OK otherwise.
+ */
+dn_status dn_stream_status(void* cuda_stream);
+
+/* Static, human-readable name of a status code. Never NULL. */
+const char* dn_status_string(dn_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int dn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DN_H_ */

@@ -1,0 +1,133 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared
+entry point, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import gated_linear_attention_dn_b200 as dn
+from gated_linear_attention_dn_b200 import build as dnbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dnbuild.build()
+    return dn.load()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(dn_[a-z_0-9]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert {"dn_chunk_fwd", "dn_decode_step", "dn_stream_status", "dn_status_string"} <= names
+    for n in names:
+        assert hasattr(lib, n), f"libdn.so does not export {n}"
+    for n in dn.EXPORTED:
+        assert n in names
+
+
+def test_status_strings(lib):
+    assert dn.dn_status_string(0) == "DN_OK"
+    assert dn.dn_status_string(6) == "DN_ERR_DEVICE_TIMEOUT"
+    assert dn.dn_status_string(99) == "DN_ERR_UNKNOWN"
+    assert dn.dn_version() >= 100
+
+
+class _Buf:
+    """16-byte aligned host scratch whose address stands in for a device pointer;
+    validation failures return before any pointer is dereferenced or any CUDA call."""
+
+    def __init__(self, n=4096):
+        self.raw = np.zeros(n + 64, dtype=np.uint8)
+        base = self.raw.ctypes.data
+        self.addr = (base + 15) & ~15
+
+    def p(self, off=0):
+        return ctypes.c_void_p(self.addr + off)
+
+
+def _desc(**kw):
+    d = dict(B=1, T=8, H=2, d_k=64, d_v=64, chunk=0, io_dtype=dn.DN_BF16, alpha=dn.DN_GATE_SCALAR,
+             beta_k=dn.DN_GATE_SCALAR, beta_v=dn.DN_GATE_ONE, key_scale=dn.DN_GATE_ONE)
+    d.update(kw)
+    return dn.DnDesc(**d)
+
+
+def _call(lib, desc, off=None, **ptrs):
+    bufs = {n: _Buf() for n in ("q", "k", "v", "a", "bk", "bv", "d", "s0", "o", "st")}
+    p = {n: b.p() for n, b in bufs.items()}
+    p["bv"] = None
+    p["d"] = None
+    p.update(ptrs)
+    return lib.dn_chunk_fwd(ctypes.byref(desc) if desc is not None else None, p["q"], p["k"], p["v"],
+                            p["a"], p["bk"], p["bv"], p["d"], p["s0"], p["o"], p["st"], None, 0, None)
+
+
+def test_rejects_bad_descriptors(lib):
+    assert _call(lib, None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(B=0)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(T=-1)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(io_dtype=7)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(alpha=5)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(d_k=96)) == dn.DN_ERR_UNSUPPORTED
+    assert _call(lib, _desc(d_v=256)) == dn.DN_ERR_UNSUPPORTED
+    assert _call(lib, _desc(chunk=32)) == dn.DN_ERR_UNSUPPORTED
+
+
+def test_rejects_bad_pointers(lib):
+    b = _Buf()
+    # gate present iff its mode is not DN_GATE_ONE
+    assert _call(lib, _desc(), a=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(), bv=b.p()) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(), q=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(), o=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(), st=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(), k=b.p(4)) == dn.DN_ERR_MISALIGNED
+    assert _call(lib, _desc(), a=b.p(2)) == dn.DN_ERR_MISALIGNED
+    assert _call(lib, _desc(alpha=dn.DN_GATE_CHANNEL), a=b.p(8)) == dn.DN_ERR_MISALIGNED
+    assert _call(lib, _desc(), o=b.p(2)) == dn.DN_ERR_MISALIGNED
+    # o overlapping q
+    q = _Buf()
+    assert _call(lib, _desc(), q=q.p(), o=q.p(16)) == dn.DN_ERR_INVALID_ARGUMENT
+
+
+def test_decode_rejects_bad_arguments(lib):
+    b = _Buf()
+    d = _desc(T=2)
+    args = [b.p(), b.p(), b.p(), b.p(), b.p(), None, None, b.p(), b.p(), None]
+    assert lib.dn_decode_step(ctypes.byref(d), *args) == dn.DN_ERR_INVALID_ARGUMENT  # T must be 1
+    d = _desc(T=1)
+    bad = list(args)
+    bad[7] = b.p(4)  # misaligned S
+    assert lib.dn_decode_step(ctypes.byref(d), *bad) == dn.DN_ERR_MISALIGNED
+    bad = list(args)
+    bad[7] = None
+    assert lib.dn_decode_step(ctypes.byref(d), *bad) == dn.DN_ERR_INVALID_ARGUMENT
+
+
+def test_workspace_query(lib):
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc()) == 0
+    assert lib.dn_chunk_fwd_workspace_bytes(None) == 0
+
+
+def test_binding_has_no_cpu_path(tmp_path):
+    with pytest.raises(RuntimeError):
+        dn.load.__wrapped__ if hasattr(dn.load, "__wrapped__") else None
+        saved = dn._lib
+        try:
+            dn._lib = None
+            dn.load(str(tmp_path / "missing.so"))
+        finally:
+            dn._lib = saved
