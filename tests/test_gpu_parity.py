@@ -125,10 +125,13 @@ def test_decode_one_step_equals_chunk_T1():
     o_dec = dn.dn_decode_step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"],
                               xd["key_scale"], S=S)
     o_chk, S_chk = run_chunk(xd)
-    torch.testing.assert_close(o_dec.float(), o_chk.float(), rtol=2e-2, atol=2e-2)
-    assert oracle.rel_l2(host_f64(S), host_f64(S_chk)) < 1e-5
+    # the decode step is fp32 on CUDA cores; the chunked kernel uses bf16 tensor-core operands,
+    # so the two agree to the bf16 tolerances, and each matches the oracle on its own
+    assert oracle.rel_l2(host_f64(o_dec), host_f64(o_chk)) < TOL["bf16"]["o"]
+    assert oracle.rel_l2(host_f64(S), host_f64(S_chk)) < TOL["bf16"]["S"]
     o_ref, S_ref = oracle.fwd(**x)
     check(o_dec, S, o_ref, S_ref, "bf16")
+    check(o_chk, S_chk, o_ref, S_ref, "bf16")
 
 
 @pytest.mark.parametrize("B,steps", [(4, 100), (1024, 3)])
