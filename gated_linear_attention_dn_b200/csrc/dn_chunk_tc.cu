@@ -2,8 +2,8 @@
 //
 // One CTA (256 threads) owns one (b, h) sequence and walks its chunks of C = 64
 // tokens in order, keeping the fp32 state in tensor memory. Per chunk, with the
-// log-decay prefix referenced to the chunk midpoint m (after token 31), so that
-// every exponent spans at most half a chunk of decay:
+// decay referenced to the chunk midpoint m (after token 31), so that every
+// decay factor spans at most half a chunk:
 //
 //   r_t = gamma_t / gamma_m  (per key channel; products of alpha, no exp/log)
 //   K+ = k (.) r,  Q+ = q (.) r,  W- = beta^k (.) d (.) k / r,  V~ = beta^v (.) v
@@ -19,18 +19,29 @@
 // matrix and intra-block scores take the preconditioned key under OSDN (OSDN
 // page, section 2.1); the algebra is derived from the recurrence in dn.h.
 //
+// Two gate classes share the kernel:
+//  * per-token gates only (GDN: scalar alpha, beta^k, beta^v, d): every decay and
+//    write factor is a scalar per token, so they move onto the 64x64 and 64xN
+//    matrices (A_ti = (k_t.k_i) beta_i r_t / r_i, T K+ = (T Diag(r)) K,
+//    W-^T U = K^T (Diag(beta / r) U), O_t = r_t (Q S_m + P_raw U')_t) and the raw
+//    TMA tiles of q, k, v feed the tensor cores directly, with no elementwise pass;
+//  * any per-channel gate (KDA decay, FG2-GDN+ vector beta, OSDN d): the CUDA
+//    cores build K+, Q+, W- (hi/lo) and V~ (hi/lo) tiles per chunk, with all gate
+//    loads of a chunk in flight at once.
+//
 // Precision plan (bf16 operands, fp32 accumulation everywhere): the state update
-// W-^T U is the product whose rounding reaches S_T directly, so both operands
-// are split hi + lo in bf16 (three MMAs: hi*hi + hi*lo + lo*hi); V~ is split the
-// same way when beta^v is present. All other operands are single bf16.
+// W-^T U is the product whose rounding reaches S_T directly, so its operands are
+// split hi + lo in bf16 (raw k is exact in bf16, so the per-token path splits
+// only U); V~ is split the same way when beta^v is a vector. All other operands
+// are single bf16.
 //
 // Shared-memory operand tiles use the 128-byte-swizzled canonical layout (see
 // canon()); q/k/v tiles arrive by TMA (4-D tensor maps over [B, T, H, d], boxes of
 // 64 channels x 64 tokens, zero fill past the end of the sequence).
 //
 // Tensor memory (512 columns): S_acc [0, NV) | D1 [NV, 2NV) | U0 [2NV, 3NV) | scratch (Gram, Wk).
-// Every wait on an mbarrier is bounded; on expiry the CTA sets the status word,
-// drains what it issued (again bounded), frees its tensor memory and exits.
+// Every wait on an mbarrier is bounded in time; on expiry the CTA sets the status
+// word, drains what it issued (again bounded), frees its tensor memory and exits.
 #include <cudaTypedefs.h>
 
 #include "dn_common.cuh"
@@ -49,7 +60,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, far above any legi
 template <int DK, int NV>
 struct Layout {
   static constexpr int STK = 0;                       // raw k  [C][DK]   (TMA)
-  static constexpr int STQ = STK + C * DK * 2;        // raw q  [C][DK]   (TMA)
+  static constexpr int STQ = STK + C * DK * 2;        // raw q  [C][DK]   (TMA); per-token path: T~ tile
   static constexpr int STV = STQ + C * DK * 2;        // raw v  [C][NV]   (TMA), V~ hi after prep
   static constexpr int VLO = STV + C * NV * 2;        // V~ lo  [C][NV]
   static constexpr int KQ = VLO + C * NV * 2;         // [K+ ; Q+] then [Wk ; Q+]   [128][DK]
@@ -67,49 +78,167 @@ struct Layout {
   static_assert(TM_SCR + (DK > 64 ? DK : 64) <= (int)kTmemCols, "tensor memory budget");
 };
 
-// rotated index into a 64x64 fp32 array: row r's columns start at bank r, so
-// column-wise access by 32 consecutive rows is conflict-free
-__device__ __forceinline__ int ri(int r, int c) { return (r << 6) | ((c + r) & 63); }
+// Index into a 64x64 fp32 array: rows of 64, columns XOR-permuted in groups of 4
+// by (row mod 8), so float4 accesses stay aligned and column walks by
+// consecutive rows spread over the banks.
+__device__ __forceinline__ int xi(int r, int c) { return (r << 6) | (c ^ ((r & 7) << 2)); }
 
-__device__ __forceinline__ float2 gate2(const float* g, int mode, int64_t tok, int width, int ch) {
-  if (mode == DN_GATE_ONE) return make_float2(1.f, 1.f);
-  if (mode == DN_GATE_SCALAR) {
-    const float x = g[tok];
-    return make_float2(x, x);
-  }
-  return *reinterpret_cast<const float2*>(g + tok * width + ch);
+__device__ __forceinline__ float4 f4(float x) { return make_float4(x, x, x, x); }
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+__device__ __forceinline__ float4 rcp4(float4 a) {
+  return make_float4(__fdividef(1.f, a.x), __fdividef(1.f, a.y), __fdividef(1.f, a.z), __fdividef(1.f, a.w));
 }
 
-// X = sum_{k=j}^{i-1} L_ik T_kj for block (i, j) of the 16x16 blocking; element (r, cc).
-__device__ __forceinline__ float block_lt(const float* sL, const float* sT, int i, int j, int r, int cc) {
-  float s = 0.f;
-  for (int k = j; k < i; ++k) {
+// gate values of four consecutive channels (mode ONE -> 1, SCALAR -> broadcast)
+__device__ __forceinline__ float4 gate4(const float* g, int mode, int64_t tok, int width, int ch) {
+  if (mode == DN_GATE_ONE) return f4(1.f);
+  if (mode == DN_GATE_SCALAR) return f4(g[tok]);
+  return *reinterpret_cast<const float4*>(g + tok * width + ch);
+}
+
+__device__ __forceinline__ float4 lds4(const float* p, int idx) { return *reinterpret_cast<const float4*>(p + idx); }
+__device__ __forceinline__ void sts4(float* p, int idx, float4 v) { *reinterpret_cast<float4*>(p + idx) = v; }
+
+__device__ __forceinline__ uint2 pack4(float4 v) { return make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w)); }
+__device__ __forceinline__ float4 unpack4(uint2 u) {
+  const float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void split4(float4 v, uint2& hi, uint2& lo) {
+  split_bf16(v.x, v.y, hi.x, lo.x);
+  split_bf16(v.z, v.w, hi.y, lo.y);
+}
+
+// Warp-level tensor-core product (mma.sync, TF32 inputs, fp32 accumulation), used only for the
+// small block products inside the 64x64 triangular inverse; T is rounded to bf16 afterwards, so
+// TF32 (10-bit mantissa) operands here add an error well below that rounding. Fragment layouts
+// of m16n8k8 row.col (g = lane / 4, t = lane % 4): A 16x8: (g, t) (g+8, t) (g, t+4) (g+8, t+4);
+// B 8x8: (t, g) (t+4, g); C 16x8: (g, 2t) (g, 2t+1) (g+8, 2t) (g+8, 2t+1).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// d[16x8] += X[16 x K] * Y[K x 8] for one warp; X(i, k), Y(k, n) fetch elements.
+template <int K, class FX, class FY>
+__device__ __forceinline__ void warp_mm(float* d, FX X, FY Y, int lane) {
+  const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) s = fmaf(sL[ri(16 * i + r, 16 * k + m)], sT[ri(16 * k + m, 16 * j + cc)], s);
+  for (int k = 0; k < K; k += 8) {
+    const uint32_t av[4] = {to_tf32(X(g, k + t)), to_tf32(X(g + 8, k + t)), to_tf32(X(g, k + t + 4)),
+                            to_tf32(X(g + 8, k + t + 4))};
+    const uint32_t bv[2] = {to_tf32(Y(k + t, g)), to_tf32(Y(k + t + 4, g))};
+    mma_tf32(d, av, bv);
   }
-  return s;
 }
 
-// T_ij = -T_ii X for block (i, j); element (r, cc); X is 16x16 row-major.
-__device__ __forceinline__ float block_tx(const float* sT, const float* X, int i, int r, int cc) {
-  float s = 0.f;
+// writes the 16x8 accumulator fragment through W(i, n, value)
+template <class FW>
+__device__ __forceinline__ void warp_store(const float* d, FW W, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  W(g, 2 * t, d[0]);
+  W(g, 2 * t + 1, d[1]);
+  W(g + 8, 2 * t, d[2]);
+  W(g + 8, 2 * t + 1, d[3]);
+}
+
+// T = (I + L)^{-1} for the 64x64 strictly lower L in sL (zeros on and above the diagonal), into
+// sT. Blocking: the four 16x16 diagonal blocks by forward substitution (one column per thread);
+// the two 32x32 diagonal blocks by T_{i,i-1} = -T_ii L_{i,i-1} T_{i-1,i-1}; the lower-left 32x32
+// block by T21 = -T2 L21 T1. scr: 2048 floats of scratch. All 256 threads call this.
+__device__ __forceinline__ void unit_lower_inverse(const float* sL, float* sT, float* scr, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid < 64) {
+    const int blk = tid >> 4, j = tid & 15, base = 16 * blk;
+    float x[16];
 #pragma unroll
-  for (int m = 0; m < 16; ++m) s = fmaf(sT[ri(16 * i + r, 16 * i + m)], X[m * 16 + cc], s);
-  return -s;
+    for (int r = 0; r < 16; ++r) {
+      float s0 = (r == j) ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < r; ++i) {
+        const float l = sL[xi(base + r, base + i)];
+        if (i & 1)
+          s1 = fmaf(-l, x[i], s1);
+        else
+          s0 = fmaf(-l, x[i], s0);
+      }
+      x[r] = s0 + s1;
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) sT[xi(base + r, base + j)] = x[r];
+  } else {
+    // the upper off-diagonal 16x16 blocks inside the two 32x32 diagonal blocks are zero
+    for (int e = tid - 64; e < 512; e += 192) {
+      const int q = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+      sT[xi(32 * q + r, 32 * q + 16 + cc)] = 0.f;
+    }
+  }
+  __syncthreads();
+  if (warp < 2) {
+    const int bi = 1 + 2 * warp, bk = bi - 1;  // (1,0) and (3,2)
+    float* Y = scr + 1152 + warp * 384;        // 16 x 24 (padded) dense scratch of this warp
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      warp_mm<16>(d, [&](int i, int k) { return sL[xi(16 * bi + i, 16 * bk + k)]; },
+                  [&](int k, int n) { return sT[xi(16 * bk + k, 16 * bk + 8 * nt + n)]; }, lane);
+      warp_store(d, [&](int i, int n, float v) { Y[i * 24 + 8 * nt + n] = v; }, lane);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      warp_mm<16>(d, [&](int i, int k) { return sT[xi(16 * bi + i, 16 * bi + k)]; },
+                  [&](int k, int n) { return Y[k * 24 + 8 * nt + n]; }, lane);
+      warp_store(d, [&](int i, int n, float v) { sT[xi(16 * bi + i, 16 * bk + 8 * nt + n)] = -v; }, lane);
+    }
+  }
+  __syncthreads();
+  // X = L21 T1: warp w computes rows 16 (w / 4) .. +16, columns 8 (w % 4) .. +8
+  float* X = scr;  // 32 x 36 (padded) dense
+  {
+    const int mt = warp >> 2, nt = warp & 3;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    warp_mm<32>(d, [&](int i, int k) { return sL[xi(32 + 16 * mt + i, k)]; },
+                [&](int k, int n) { return sT[xi(k, 8 * nt + n)]; }, lane);
+    warp_store(d, [&](int i, int n, float v) { X[(16 * mt + i) * 36 + 8 * nt + n] = v; }, lane);
+  }
+  __syncthreads();
+  {
+    const int mt = warp >> 2, nt = warp & 3;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    warp_mm<32>(d, [&](int i, int k) { return sT[xi(32 + 16 * mt + i, 32 + k)]; },
+                [&](int k, int n) { return X[k * 36 + 8 * nt + n]; }, lane);
+    warp_store(d, [&](int i, int n, float v) { sT[xi(32 + 16 * mt + i, 8 * nt + n)] = -v; }, lane);
+  }
+  __syncthreads();
 }
 
-template <int DK, int NV>
+template <int DK, int NV, bool SC>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Args a) {
   using Ly = Layout<DK, NV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bar_qk, bar_v, bar_mma;
+  __shared__ __align__(8) uint64_t bar_qk, bar_k, bar_v, bar_mma;
   __shared__ uint32_t s_tmem;
-  __shared__ float s_lam[2][DK];
-  __shared__ float s_gm[DK];
-  __shared__ float s_X[3][256];
+  __shared__ __align__(16) float s_lam[2][DK];   // gamma_C / gamma_m per key channel (per-channel path)
+  __shared__ __align__(16) float s_gm[DK];       // gamma_m per key channel
+  __shared__ __align__(16) float s_grp[8][DK];   // per-8-token decay products (per-channel path)
+  __shared__ __align__(16) float s_Y[2048];
+  __shared__ float s_r[C], s_ri[C], s_ws[C], s_bv[C];  // per-token path: r_t, 1/r_t, beta^k d, beta^v
+  __shared__ float s_lam1[2], s_gm1;
+  __shared__ float s_nx[2][4][C];  // per-token path: gates of the next chunk (alpha, beta^k, d, beta^v)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, ch = warp >> 2;
@@ -119,24 +248,48 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&bar_qk, 1);
+    mbar_init(&bar_k, 1);
     mbar_init(&bar_v, 1);
     mbar_init(&bar_mma, 1);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
+  if (SC) {
+    // rows 64..127 of the T~ tile are never meaningful; keep them finite
+    for (int i = tid; i < 64 * 128 / 16; i += kThreads)
+      reinterpret_cast<uint4*>(sm + Ly::STQ + 64 * 128)[i] = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
 
+  // Operand buffers. Per-channel path: raw k, q staging (STK, STQ) feeds the prep,
+  // which writes [K+; Q+] into KQ. Per-token path: the raw [K; Q] tile (Gram operand,
+  // later [Wk; Q]) is double-buffered in KQ and in the W- region it does not use, so
+  // the next chunk's tile loads during this chunk; a separate raw k tile (STK) serves
+  // the state update at the end of the chunk and reloads after it.
+  auto kq_buf = [&](int c) -> uint8_t* { return (SC && (c & 1)) ? sm + Ly::WHI : sm + Ly::KQ; };
   auto issue_qk = [&](int c) {
     mbar_expect_tx(&bar_qk, 2u * C * DK * 2);
 #pragma unroll
     for (int x = 0; x < DK / 64; ++x) {
-      tma_load_4d(sm + Ly::STK + x * C * 128, &tm_k, &bar_qk, 64 * x, h, c * C, b);
-      tma_load_4d(sm + Ly::STQ + x * C * 128, &tm_q, &bar_qk, 64 * x, h, c * C, b);
+      if (SC) {
+        uint8_t* kq = kq_buf(c);
+        tma_load_4d(kq + x * 128 * 128, &tm_k, &bar_qk, 64 * x, h, c * C, b);
+        tma_load_4d(kq + x * 128 * 128 + 64 * 128, &tm_q, &bar_qk, 64 * x, h, c * C, b);
+      } else {
+        tma_load_4d(sm + Ly::STK + x * C * 128, &tm_k, &bar_qk, 64 * x, h, c * C, b);
+        tma_load_4d(sm + Ly::STQ + x * C * 128, &tm_q, &bar_qk, 64 * x, h, c * C, b);
+      }
     }
+  };
+  auto issue_k = [&](int c) {  // per-token path only
+    mbar_expect_tx(&bar_k, (uint32_t)C * DK * 2);
+#pragma unroll
+    for (int x = 0; x < DK / 64; ++x) tma_load_4d(sm + Ly::STK + x * C * 128, &tm_k, &bar_k, 64 * x, h, c * C, b);
   };
   auto issue_v = [&](int c) {
     mbar_expect_tx(&bar_v, (uint32_t)C * NV * 2);
@@ -144,22 +297,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < NV / 64; ++x) tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, 64 * x, h, c * C, b);
   };
 
-  uint32_t ph_qk = 0, ph_v = 0, ph_mma = 0;
-  bool qk_pending = false, v_pending = false, mma_pending = false;
+  uint32_t ph_qk = 0, ph_k = 0, ph_v = 0, ph_mma = 0;
+  bool qk_pending = false, k_pending = false, v_pending = false, mma_pending = false;
   bool failed = false;
   if (tid == 0 && nchunks > 0) {
     issue_qk(0);
+    if (SC) issue_k(0);
     issue_v(0);
   }
   if (nchunks > 0) qk_pending = v_pending = true;
+  if (SC && nchunks > 0) k_pending = true;
 
   const uint32_t id_gram = idesc_bf16(128, 64, 0, 0);
   const uint32_t id_wk = idesc_bf16(128, DK, 0, 1);
   const uint32_t id_nv = idesc_bf16(128, NV, 0, 1);
   const uint32_t id_state = idesc_bf16(128, NV, 1, 1);
-  const bool bv_split = a.beta_v != DN_GATE_ONE;
+  const bool bv_split = !SC && a.beta_v != DN_GATE_ONE;
   float* sL = reinterpret_cast<float*>(sm + Ly::INV);
   float* sT = sL + C * C;
+
+  // per-token path: thread j < 64 copies token j's gates of the next chunk into shared memory
+  // one chunk ahead with cp.async (absent gates and tokens past the end are written directly)
+  auto prefetch_token_gates = [&](int cn) {
+    const int j = tid, t0n = cn * C;
+    float* dst = &s_nx[cn & 1][0][j];
+    const float* src[4] = {a.alpha_p, a.beta_k_p, a.key_scale_p, a.beta_v_p};
+    const int mode[4] = {a.alpha, a.beta_k, a.key_scale, a.beta_v};
+    const bool valid = j < T - t0n;
+    const int64_t tok = ((int64_t)b * T + t0n + j) * H + h;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (valid && mode[g] == DN_GATE_SCALAR)
+        cp_async_4(dst + g * C, src[g] + tok);
+      else
+        dst[g * C] = valid ? 1.f : (g == 0 ? 1.f : 0.f);
+    }
+    cp_async_commit();
+  };
+  if (SC && tid < 64 && nchunks > 0) prefetch_token_gates(0);
 
   for (int c = 0; c < nchunks; ++c) {
     const int t0 = c * C;
@@ -177,88 +352,131 @@ __global__ void __launch_bounds__(kThreads, 1)
       ph_v ^= 1;
       qk_pending = v_pending = false;
     }
+    uint8_t* const kq = kq_buf(c);
+    // per-token path: the other [K; Q] buffer was last read by the previous chunk's D1 MMA
+    if (SC && tid == 0 && c + 1 < nchunks) issue_qk(c + 1);
+    if (SC && c + 1 < nchunks) qk_pending = true;
 
-    // ---- P1: gate prefix products and operand tiles
-    if (tid < 128) {
-      const int c0 = 2 * (tid & 63);
-      const int half = tid >> 6;
-      float2 r = make_float2(1.f, 1.f), rinv = make_float2(1.f, 1.f), rho = make_float2(1.f, 1.f);
-      const int jbeg = half ? 32 : 31, jend = half ? 64 : -1, jstep = half ? 1 : -1;
-      for (int j = jbeg; j != jend; j += jstep) {
+    // ---- P1: decay factors (and, per-channel path, the operand tiles)
+    if (SC) {
+      if (tid < 64) {
+        const int j = tid;
+        cp_async_wait_all();
+        const float al = s_nx[cur][0][j], ws = s_nx[cur][1][j] * s_nx[cur][2][j], bv = s_nx[cur][3][j];
+        if (c + 1 < nchunks) prefetch_token_gates(c + 1);
+        float p = al;
+        if (warp == 1) {  // tokens 32..63: r_j = prod_{s=32..j} alpha_s (inclusive prefix over lanes)
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, p, off);
+            if (lane >= off) p *= y;
+          }
+          s_r[j] = p;
+          s_ri[j] = __fdividef(1.f, p);
+          if (lane == 31) s_lam1[cur] = p;
+        } else {  // tokens 0..31: 1/r_j = prod_{s=j+1..31} alpha_s (exclusive suffix over lanes)
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_down_sync(0xffffffffu, p, off);
+            if (lane + off < 32) p *= y;
+          }
+          const float nxt = __shfl_down_sync(0xffffffffu, p, 1);
+          const float ri = lane == 31 ? 1.f : nxt;
+          s_ri[j] = ri;
+          s_r[j] = __fdividef(1.f, ri);
+          if (lane == 0) s_gm1 = p;
+        }
+        s_ws[j] = ws;
+        s_bv[j] = bv;
+      }
+    } else {
+      // per-channel path: thread (g4, tg) owns channels 4g4..4g4+3 of tokens 8tg..8tg+7
+      const int g4 = lane, tg = warp, cb0 = 4 * g4;
+      float4 al[8], ws[8];
+      uint2 kr[8], qr[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = 8 * tg + i;
         const bool valid = j < n;
         const int64_t tok = ((int64_t)b * T + t0 + j) * H + h;
-        float2 al = make_float2(1.f, 1.f), ws = make_float2(0.f, 0.f);
-        if (valid) {
-          al = gate2(a.alpha_p, a.alpha, tok, DK, c0);
-          const float2 bk = gate2(a.beta_k_p, a.beta_k, tok, DK, c0);
-          const float2 dd = gate2(a.key_scale_p, a.key_scale, tok, DK, c0);
-          ws = make_float2(bk.x * dd.x, bk.y * dd.y);
-        }
-        const float2 ial = make_float2(__fdividef(1.f, al.x), __fdividef(1.f, al.y));
-        if (half) {  // forward from the midpoint: r_j = prod_{s=32..j} alpha_s
-          r.x *= al.x;
-          r.y *= al.y;
-          rinv.x *= ial.x;
-          rinv.y *= ial.y;
-        }
-        const float2 kk = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + Ly::STK + canon(j, c0, C)));
-        const float2 qq = unpack_bf16(*reinterpret_cast<const uint32_t*>(sm + Ly::STQ + canon(j, c0, C)));
-        *reinterpret_cast<uint32_t*>(sm + Ly::KQ + canon(j, c0, 128)) = pack_bf16(kk.x * r.x, kk.y * r.y);
-        *reinterpret_cast<uint32_t*>(sm + Ly::KQ + canon(64 + j, c0, 128)) = pack_bf16(qq.x * r.x, qq.y * r.y);
-        uint32_t whi, wlo;
-        split_bf16(ws.x * kk.x * rinv.x, ws.y * kk.y * rinv.y, whi, wlo);
-        *reinterpret_cast<uint32_t*>(sm + Ly::WHI + canon(j, c0, C)) = whi;
-        *reinterpret_cast<uint32_t*>(sm + Ly::WLO + canon(j, c0, C)) = wlo;
-        if (!half) {  // backward from the midpoint: r_{j-1} = r_j / alpha_j
-          r.x *= ial.x;
-          r.y *= ial.y;
-          rinv.x *= al.x;
-          rinv.y *= al.y;
-          rho.x *= al.x;
-          rho.y *= al.y;
-        }
+        al[i] = valid ? gate4(a.alpha_p, a.alpha, tok, DK, cb0) : f4(1.f);
+        ws[i] = valid ? mul4(gate4(a.beta_k_p, a.beta_k, tok, DK, cb0),
+                             gate4(a.key_scale_p, a.key_scale, tok, DK, cb0))
+                      : f4(0.f);
+        kr[i] = *reinterpret_cast<const uint2*>(sm + Ly::STK + canon(j, cb0, C));
+        qr[i] = *reinterpret_cast<const uint2*>(sm + Ly::STQ + canon(j, cb0, C));
       }
-      if (half) {
-        s_lam[cur][c0] = r.x;
-        s_lam[cur][c0 + 1] = r.y;
+      // products inside the group: prefix (second half) or exclusive suffix (first half)
+      float4 loc[8];
+      float4 grp;
+      if (tg >= 4) {
+        float4 p = f4(1.f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          p = mul4(p, al[i]);
+          loc[i] = p;
+        }
+        grp = p;
       } else {
-        s_gm[c0] = rho.x;
-        s_gm[c0 + 1] = rho.y;
+        float4 p = f4(1.f);
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          loc[i] = p;
+          p = mul4(p, al[i]);
+        }
+        grp = p;
       }
-    } else if (bv_split) {
-      // V~ = beta^v (.) v, split hi (in place) / lo
-      const int u = tid - 128;
-      const int j = u >> 1;
-      const bool valid = j < n;
-      const int64_t tok = ((int64_t)b * T + t0 + j) * H + h;
-      constexpr int CH8 = NV / 16;  // 16-byte chunks per thread (half a row)
+      sts4(&s_grp[tg][0], cb0, grp);
+      __syncthreads();
+      float4 off = f4(1.f);
+      if (tg >= 4) {
+        for (int g = 4; g < tg; ++g) off = mul4(off, lds4(&s_grp[g][0], cb0));
+      } else {
+        for (int g = tg + 1; g < 4; ++g) off = mul4(off, lds4(&s_grp[g][0], cb0));
+      }
+      if (tg == 0) {
+        float4 gm = f4(1.f), lm = f4(1.f);
 #pragma unroll
-      for (int i = 0; i < CH8; ++i) {
-        const int x8 = (u & 1) * CH8 + i;
-        const uint32_t off = canon_chunk(j, x8, C);
-        uint4 raw = *reinterpret_cast<const uint4*>(sm + Ly::STV + off);
-        float bv[8];
-        if (!valid) {
+        for (int g = 0; g < 4; ++g) gm = mul4(gm, lds4(&s_grp[g][0], cb0));
 #pragma unroll
-          for (int e = 0; e < 8; ++e) bv[e] = 0.f;
-        } else if (a.beta_v == DN_GATE_SCALAR) {
-          const float x = a.beta_v_p[tok];
+        for (int g = 4; g < 8; ++g) lm = mul4(lm, lds4(&s_grp[g][0], cb0));
+        sts4(s_gm, cb0, gm);
+        sts4(&s_lam[cur][0], cb0, lm);
+      }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) bv[e] = x;
+      for (int i = 0; i < 8; ++i) {
+        const int j = 8 * tg + i;
+        float4 r, rinv;
+        if (tg >= 4) {
+          r = mul4(off, loc[i]);
+          rinv = rcp4(r);
         } else {
-          const float4 lo4 = *reinterpret_cast<const float4*>(a.beta_v_p + tok * dv + 8 * x8);
-          const float4 hi4 = *reinterpret_cast<const float4*>(a.beta_v_p + tok * dv + 8 * x8 + 4);
-          bv[0] = lo4.x, bv[1] = lo4.y, bv[2] = lo4.z, bv[3] = lo4.w;
-          bv[4] = hi4.x, bv[5] = hi4.y, bv[6] = hi4.z, bv[7] = hi4.w;
+          rinv = mul4(off, loc[i]);
+          r = rcp4(rinv);
         }
-        uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w}, hi[4], lo[4];
+        const float4 kk = unpack4(kr[i]), qq = unpack4(qr[i]);
+        *reinterpret_cast<uint2*>(kq + canon(j, cb0, 128)) = pack4(mul4(kk, r));
+        *reinterpret_cast<uint2*>(kq + canon(64 + j, cb0, 128)) = pack4(mul4(qq, r));
+        uint2 hi, lo;
+        split4(mul4(mul4(ws[i], kk), rinv), hi, lo);
+        *reinterpret_cast<uint2*>(sm + Ly::WHI + canon(j, cb0, C)) = hi;
+        *reinterpret_cast<uint2*>(sm + Ly::WLO + canon(j, cb0, C)) = lo;
+      }
+      if (bv_split && cb0 < NV) {
+        // V~ = beta^v (.) v, split hi (in place) / lo
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 vv = unpack_bf16(w[e]);
-          split_bf16(vv.x * bv[2 * e], vv.y * bv[2 * e + 1], hi[e], lo[e]);
+        for (int i = 0; i < 8; ++i) {
+          const int j = 8 * tg + i;
+          const bool valid = j < n;
+          const int64_t tok = ((int64_t)b * T + t0 + j) * H + h;
+          const float4 bv = valid ? gate4(a.beta_v_p, a.beta_v, tok, dv, cb0) : f4(0.f);
+          const uint32_t off2 = canon(j, cb0, C);
+          const float4 vv = unpack4(*reinterpret_cast<const uint2*>(sm + Ly::STV + off2));
+          uint2 hi, lo;
+          split4(mul4(vv, bv), hi, lo);
+          *reinterpret_cast<uint2*>(sm + Ly::STV + off2) = hi;
+          *reinterpret_cast<uint2*>(sm + Ly::VLO + off2) = lo;
         }
-        *reinterpret_cast<uint4*>(sm + Ly::STV + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(sm + Ly::VLO + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
     __syncthreads();
@@ -266,7 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- P1.5: bring the state into this chunk's frame: S_m = Diag(lambda_prev * gamma_m) S
     {
       const int k = 32 * q4 + lane;
-      const float mu = (c == 0) ? s_gm[k] : s_lam[prev][k] * s_gm[k];
+      const float mu = SC ? ((c == 0) ? s_gm1 : s_lam1[prev] * s_gm1)
+                          : ((c == 0) ? s_gm[k] : s_lam[prev][k] * s_gm[k]);
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {
         const int col = ch * (NV / 2) + 32 * cb;
@@ -302,18 +521,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
 
-    // ---- P2: prefetch next q/k; Gram [K+; Q+] W-^T -> scratch
+    // ---- P2: Gram [K+; Q+] W-^T (per-token path: [K; Q] K^T) -> scratch
     if (tid == 0) {
-      if (c + 1 < nchunks) issue_qk(c + 1);
+      // per-channel path: the raw q, k staging was consumed by the prep; prefetch the next chunk
+      if (!SC && c + 1 < nchunks) {
+        fence_proxy_async();
+        issue_qk(c + 1);
+      }
+      const uint8_t* gb = SC ? kq : sm + Ly::WHI;
+      const uint32_t gb_blk = SC ? 128 * 128 : C * 128;
 #pragma unroll
       for (int kk = 0; kk < DK; kk += 16) {
-        const uint64_t ad = sdesc(smem_u32(sm + Ly::KQ) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
-        const uint64_t bd = sdesc(smem_u32(sm + Ly::WHI) + (kk >> 6) * (C * 128) + (kk & 63) * 2, 16, 1024);
+        const uint64_t ad = sdesc(smem_u32(kq) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+        const uint64_t bd = sdesc(smem_u32(gb) + (kk >> 6) * gb_blk + (kk & 63) * 2, 16, 1024);
         mma_bf16(tmem + Ly::TM_SCR, ad, bd, id_gram, kk > 0);
       }
       mma_commit(&bar_mma);
     }
-    if (c + 1 < nchunks) qk_pending = true;
+    if (!SC && c + 1 < nchunks) qk_pending = true;
     mma_pending = true;
     {
       bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
@@ -333,8 +558,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = 32 * ch;
       if (q4 < 2) {
         const int t = 32 * q4 + lane;
+        const float rt = SC ? s_r[t] : 1.f;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sL[ri(t, i0 + e)] = (i0 + e < t) ? x[e] : 0.f;
+        for (int e4 = 0; e4 < 8; ++e4) {
+          float y[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = i0 + 4 * e4 + e;
+            float v = x[4 * e4 + e];
+            if (SC) v *= s_ws[i] * rt * s_ri[i];
+            y[e] = (i < t) ? v : 0.f;
+          }
+          sts4(sL, xi(t, i0 + 4 * e4), make_float4(y[0], y[1], y[2], y[3]));
+        }
       } else {
         const int t = 32 * (q4 - 2) + lane;
 #pragma unroll
@@ -350,58 +586,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    // inverse of the unit lower-triangular (I + A), 16x16 blocking
-    if (tid < 64) {
-      const int blk = tid >> 4, j = tid & 15;
-      float xv[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float s = (r == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int i = 0; i < r; ++i) s = fmaf(-sL[ri(16 * blk + r, 16 * blk + i)], xv[i], s);
-        xv[r] = s;
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) sT[ri(16 * blk + r, 16 * blk + j)] = xv[r];
-    }
-    __syncthreads();
-    {
-      const int r = tid >> 4, cc = tid & 15;
-      // level 1: (1,0) (2,1) (3,2)
-#pragma unroll
-      for (int bi = 1; bi < 4; ++bi) s_X[bi - 1][tid] = block_lt(sL, sT, bi, bi - 1, r, cc);
-      __syncthreads();
-#pragma unroll
-      for (int bi = 1; bi < 4; ++bi) sT[ri(16 * bi + r, 16 * (bi - 1) + cc)] = block_tx(sT, s_X[bi - 1], bi, r, cc);
-      __syncthreads();
-      // level 2: (2,0) (3,1)
-#pragma unroll
-      for (int bi = 2; bi < 4; ++bi) s_X[bi - 2][tid] = block_lt(sL, sT, bi, bi - 2, r, cc);
-      __syncthreads();
-#pragma unroll
-      for (int bi = 2; bi < 4; ++bi) sT[ri(16 * bi + r, 16 * (bi - 2) + cc)] = block_tx(sT, s_X[bi - 2], bi, r, cc);
-      __syncthreads();
-      // level 3: (3,0)
-      s_X[0][tid] = block_lt(sL, sT, 3, 0, r, cc);
-      __syncthreads();
-      sT[ri(48 + r, cc)] = block_tx(sT, s_X[0], 3, r, cc);
-      __syncthreads();
-    }
-    // T -> bf16 TP rows 0..63
+    unit_lower_inverse(sL, sT, s_Y, tid);
+    // T -> bf16: TP rows 0..63 (per-token path: T Diag(r) for Wk), and T Diag(beta^v) into the T~ tile
     {
       const int t = tid >> 2;
       const int i0 = 16 * (tid & 3);
 #pragma unroll
       for (int q8 = 0; q8 < 2; ++q8) {
-        float y[8];
+        float y[8], z[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int i = i0 + 8 * q8 + e;
-          y[e] = ((i >> 4) > (t >> 4)) ? 0.f : sT[ri(t, i)];
+        for (int e4 = 0; e4 < 2; ++e4) {
+          const int i = i0 + 8 * q8 + 4 * e4;
+          const float4 v = ((i >> 4) > (t >> 4)) ? f4(0.f) : lds4(sT, xi(t, i));
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            y[4 * e4 + e] = SC ? vv[e] * s_r[i + e] : vv[e];
+            z[4 * e4 + e] = SC ? vv[e] * s_bv[i + e] : 0.f;
+          }
         }
         uint4 pk = make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
                               pack_bf16(y[6], y[7]));
         *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, i0 / 8 + q8, 128)) = pk;
+        if (SC) {
+          uint4 pz = make_uint4(pack_bf16(z[0], z[1]), pack_bf16(z[2], z[3]), pack_bf16(z[4], z[5]),
+                                pack_bf16(z[6], z[7]));
+          *reinterpret_cast<uint4*>(sm + Ly::STQ + canon_chunk(t, i0 / 8 + q8, 128)) = pz;
+        }
       }
     }
     fence_proxy_async();
@@ -409,17 +620,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
 
-    // ---- P4: Wk = [T; P] K+ -> scratch;  U0 = [T; P] V~ -> U0
+    // ---- P4: Wk = [T; P] K+ -> scratch;  U0 = [T; P] V~ (per-token path: T~ V) -> U0
     if (tid == 0) {
+      const uint8_t* ta = SC ? sm + Ly::STQ : sm + Ly::TP;
 #pragma unroll
       for (int kk = 0; kk < C; kk += 16) {
         const uint64_t ad = sdesc(smem_u32(sm + Ly::TP) + kk * 2, 16, 1024);
-        const uint64_t bk = sdesc(smem_u32(sm + Ly::KQ) + kk * 128, 128 * 128, 1024);
+        const uint64_t bk = sdesc(smem_u32(kq) + kk * 128, 128 * 128, 1024);
         mma_bf16(tmem + Ly::TM_SCR, ad, bk, id_wk, kk > 0);
       }
 #pragma unroll
       for (int kk = 0; kk < C; kk += 16) {
-        const uint64_t ad = sdesc(smem_u32(sm + Ly::TP) + kk * 2, 16, 1024);
+        const uint64_t ad = sdesc(smem_u32(ta) + kk * 2, 16, 1024);
         const uint64_t bv = sdesc(smem_u32(sm + Ly::STV) + kk * 128, C * 128, 1024);
         mma_bf16(tmem + Ly::TM_U0, ad, bv, id_nv, kk > 0);
       }
@@ -450,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (c + 1 < nchunks) v_pending = true;
 
-    // ---- P5: Wk -> bf16 into KQ rows 0..63 (K+ is dead now)
+    // ---- P5: Wk -> bf16 into KQ rows 0..63 (K+ / raw K there is dead now)
     if (q4 < 2) {
       const int t = 32 * q4 + lane;
 #pragma unroll
@@ -462,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q8 = 0; q8 < 4; ++q8) {
           uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
                                 pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
-          *reinterpret_cast<uint4*>(sm + Ly::KQ + canon_chunk(t, col / 8 + q8, 128)) = pk;
+          *reinterpret_cast<uint4*>(kq + canon_chunk(t, col / 8 + q8, 128)) = pk;
         }
       }
     }
@@ -475,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
 #pragma unroll
       for (int kk = 0; kk < DK; kk += 16) {
-        const uint64_t ad = sdesc(smem_u32(sm + Ly::KQ) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+        const uint64_t ad = sdesc(smem_u32(kq) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
         const uint64_t bd = sdesc(smem_u32(sm + Ly::SM) + kk * 128, DK * 128, 1024);
         mma_bf16(tmem + Ly::TM_D1, ad, bd, id_nv, kk > 0);
       }
@@ -493,9 +705,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
     }
 
-    // ---- P7: U = U0 - Wk S_m -> hi / lo tiles
+    // ---- P7: U = U0 - Wk S_m (per-token path: U' = beta_t / r_t * U) -> hi / lo tiles
     if (q4 < 2) {
       const int t = 32 * q4 + lane;
+      const float us = SC ? s_ws[t] * s_ri[t] : 1.f;
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {
         const int col = ch * (NV / 2) + 32 * cb;
@@ -508,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = 8 * q8 + 2 * e;
-            split_bf16(u0[i] - d1[i], u0[i + 1] - d1[i + 1], hi[e], lo[e]);
+            split_bf16(us * (u0[i] - d1[i]), us * (u0[i + 1] - d1[i + 1]), hi[e], lo[e]);
           }
           const uint32_t off = canon_chunk(t, col / 8 + q8, C);
           *reinterpret_cast<uint4*>(sm + Ly::UHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -522,6 +735,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     // ---- P8: O = Q+ S_m + P U (rows 64..127 of D1); S_acc += W-^T U (split)
+    if (SC) {
+      bool ok = mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
+      }
+      ph_k ^= 1;
+      k_pending = false;
+    }
     if (tid == 0) {
 #pragma unroll
       for (int kk = 0; kk < C; kk += 16) {
@@ -531,13 +753,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int kk = 0; kk < C; kk += 16) {
-        const uint64_t awh = sdesc(smem_u32(sm + Ly::WHI) + kk * 128, C * 128, 1024);
-        const uint64_t awl = sdesc(smem_u32(sm + Ly::WLO) + kk * 128, C * 128, 1024);
         const uint64_t buh = sdesc(smem_u32(sm + Ly::UHI) + kk * 128, C * 128, 1024);
         const uint64_t bul = sdesc(smem_u32(sm + Ly::ULO) + kk * 128, C * 128, 1024);
-        mma_bf16(tmem + Ly::TM_S, awh, buh, id_state, 1);
-        mma_bf16(tmem + Ly::TM_S, awh, bul, id_state, 1);
-        mma_bf16(tmem + Ly::TM_S, awl, buh, id_state, 1);
+        if (SC) {
+          const uint64_t ak = sdesc(smem_u32(sm + Ly::STK) + kk * 128, C * 128, 1024);
+          mma_bf16(tmem + Ly::TM_S, ak, buh, id_state, 1);
+          mma_bf16(tmem + Ly::TM_S, ak, bul, id_state, 1);
+        } else {
+          const uint64_t awh = sdesc(smem_u32(sm + Ly::WHI) + kk * 128, C * 128, 1024);
+          const uint64_t awl = sdesc(smem_u32(sm + Ly::WLO) + kk * 128, C * 128, 1024);
+          mma_bf16(tmem + Ly::TM_S, awh, buh, id_state, 1);
+          mma_bf16(tmem + Ly::TM_S, awh, bul, id_state, 1);
+          mma_bf16(tmem + Ly::TM_S, awl, buh, id_state, 1);
+        }
       }
       mma_commit(&bar_mma);
     }
@@ -552,11 +780,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_pending = false;
       tc_fence_after();
     }
+    // per-token path: the raw k tile of the state update is free now: load the next chunk's
+    if (SC && tid == 0 && c + 1 < nchunks) {
+      fence_proxy_async();
+      issue_k(c + 1);
+    }
+    if (SC && c + 1 < nchunks) k_pending = true;
 
     // ---- P9: o rows of this chunk
     if (q4 >= 2) {
       // the TMEM load is warp-collective: every lane loads, only rows of real tokens store
       const int t = 32 * (q4 - 2) + lane;
+      const float os = SC ? s_r[t] : 1.f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0 + t) * H + h) * dv;
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {
@@ -566,8 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t < n) {
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
-            uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
-                                  pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
+            uint4 pk = make_uint4(pack_bf16(os * x[8 * q8], os * x[8 * q8 + 1]),
+                                  pack_bf16(os * x[8 * q8 + 2], os * x[8 * q8 + 3]),
+                                  pack_bf16(os * x[8 * q8 + 4], os * x[8 * q8 + 5]),
+                                  pack_bf16(os * x[8 * q8 + 6], os * x[8 * q8 + 7]));
             *reinterpret_cast<uint4*>(orow + col + 8 * q8) = pk;
           }
         }
@@ -581,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!failed && nchunks > 0) {
     // S_T = Diag(gamma_C / gamma_m) S_acc of the last chunk
     const int k = 32 * q4 + lane;
-    const float lam = s_lam[(nchunks - 1) & 1][k];
+    const float lam = SC ? s_lam1[(nchunks - 1) & 1] : s_lam[(nchunks - 1) & 1][k];
 #pragma unroll
     for (int cb = 0; cb < NV / 64; ++cb) {
       const int col = ch * (NV / 2) + 32 * cb;
@@ -596,6 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (failed) {
     // drain whatever this CTA still has in flight (bounded), then report
     if (qk_pending) mbar_wait_bounded(&bar_qk, ph_qk, kWaitNs);
+    if (k_pending) mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
     if (v_pending) mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
     if (mma_pending) mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
     if (tid == 0) atomicExch(a.status, kDevTimeout);
@@ -632,19 +870,20 @@ bool make_map(CUtensorMap* m, const void* base, int d, int H, int T, int B) {
   return r == CUDA_SUCCESS;
 }
 
-template <int DK, int NV>
+template <int DK, int NV, bool SC>
 cudaError_t launch_impl(const Args& a, cudaStream_t s) {
   using Ly = Layout<DK, NV>;
   const int smem = Ly::TOTAL + 1024;
   // per call: the attribute is per device, and the call is cheap next to the kernel
-  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<DK, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(chunk_tc_kernel<DK, NV, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   CUtensorMap mq, mk, mv;
   if (!get_encode()) return cudaErrorNotSupported;
   if (!make_map(&mq, a.q, DK, a.H, a.T, a.B) || !make_map(&mk, a.k, DK, a.H, a.T, a.B) ||
       !make_map(&mv, a.v, NV, a.H, a.T, a.B))
     return cudaErrorInvalidValue;
-  chunk_tc_kernel<DK, NV><<<a.B * a.H, kThreads, smem, s>>>(mq, mk, mv, a);
+  chunk_tc_kernel<DK, NV, SC><<<a.B * a.H, kThreads, smem, s>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -655,8 +894,11 @@ bool chunk_tc_supported(const Args& a) {
 }
 
 cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s) {
-  if (a.dv == 128) return launch_impl<128, 128>(a, s);
-  return launch_impl<128, 64>(a, s);
+  // per-token gates only -> the raw-tile path
+  const bool sc = a.alpha != DN_GATE_CHANNEL && a.beta_k != DN_GATE_CHANNEL && a.beta_v != DN_GATE_CHANNEL &&
+                  a.key_scale != DN_GATE_CHANNEL;
+  if (a.dv == 128) return sc ? launch_impl<128, 128, true>(a, s) : launch_impl<128, 128, false>(a, s);
+  return sc ? launch_impl<128, 64, true>(a, s) : launch_impl<128, 64, false>(a, s);
 }
 
 }  // namespace dn
