@@ -141,6 +141,14 @@ __device__ __forceinline__ void warp_mm(float* d, FX X, FY Y, int lane) {
   }
 }
 
+// writes the 16x8 accumulator fragment as column pairs through W(i, n, v_n, v_n+1)
+template <class FW>
+__device__ __forceinline__ void warp_store2(const float* d, FW W, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  W(g, 2 * t, d[0], d[1]);
+  W(g + 8, 2 * t, d[2], d[3]);
+}
+
 // writes the 16x8 accumulator fragment through W(i, n, value)
 template <class FW>
 __device__ __forceinline__ void warp_store(const float* d, FW W, int lane) {
@@ -151,12 +159,28 @@ __device__ __forceinline__ void warp_store(const float* d, FW W, int lane) {
   W(g + 8, 2 * t + 1, d[3]);
 }
 
-// T = (I + L)^{-1} for the 64x64 strictly lower L in sL (zeros on and above the diagonal), into
-// sT. Blocking: the four 16x16 diagonal blocks by forward substitution (one column per thread);
+// T = (I + L)^{-1} for the 64x64 strictly lower L in sL (zeros on and above the diagonal).
+// Blocking: the four 16x16 diagonal blocks by forward substitution (one column per thread);
 // the two 32x32 diagonal blocks by T_{i,i-1} = -T_ii L_{i,i-1} T_{i-1,i-1}; the lower-left 32x32
-// block by T21 = -T2 L21 T1. scr: 2048 floats of scratch. All 256 threads call this.
-__device__ __forceinline__ void unit_lower_inverse(const float* sL, float* sT, float* scr, int tid) {
+// block by T21 = -T2 L21 T1. fp32 blocks that later stages read are kept in sT; every element
+// of the lower block triangle is written as bf16 straight into rows 0..63 of the 128-row tile tp
+// (scaled by column factor cs_c[i] when SC) and, when SC, T Diag(cs_v) into tile tt. Blocks
+// strictly above the block diagonal are not written (their zeros are set once by the caller).
+// scr: 2048 floats of scratch. Not inlined: it gets its own register budget. All 256 threads call it.
+template <bool SC>
+__device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, float* scr, uint8_t* tp, uint8_t* tt,
+                                                const float* cs_c, const float* cs_v, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
+  auto emit1 = [&](int t, int i, float v) {
+    const uint32_t off = canon(t, i, 128);
+    *reinterpret_cast<__nv_bfloat16*>(tp + off) = __float2bfloat16_rn(SC ? v * cs_c[i] : v);
+    if (SC) *reinterpret_cast<__nv_bfloat16*>(tt + off) = __float2bfloat16_rn(v * cs_v[i]);
+  };
+  auto emit2 = [&](int t, int i, float v0, float v1) {  // columns i, i + 1 (i even)
+    const uint32_t off = canon(t, i, 128);
+    *reinterpret_cast<uint32_t*>(tp + off) = pack_bf16(SC ? v0 * cs_c[i] : v0, SC ? v1 * cs_c[i + 1] : v1);
+    if (SC) *reinterpret_cast<uint32_t*>(tt + off) = pack_bf16(v0 * cs_v[i], v1 * cs_v[i + 1]);
+  };
   if (tid < 64) {
     const int blk = tid >> 4, j = tid & 15, base = 16 * blk;
     float x[16];
@@ -174,7 +198,10 @@ __device__ __forceinline__ void unit_lower_inverse(const float* sL, float* sT, f
       x[r] = s0 + s1;
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) sT[xi(base + r, base + j)] = x[r];
+    for (int r = 0; r < 16; ++r) {
+      sT[xi(base + r, base + j)] = x[r];
+      emit1(base + r, base + j, x[r]);
+    }
   } else {
     // the upper off-diagonal 16x16 blocks inside the two 32x32 diagonal blocks are zero
     for (int e = tid - 64; e < 512; e += 192) {
@@ -199,7 +226,11 @@ __device__ __forceinline__ void unit_lower_inverse(const float* sL, float* sT, f
       float d[4] = {0.f, 0.f, 0.f, 0.f};
       warp_mm<16>(d, [&](int i, int k) { return sT[xi(16 * bi + i, 16 * bi + k)]; },
                   [&](int k, int n) { return Y[k * 24 + 8 * nt + n]; }, lane);
-      warp_store(d, [&](int i, int n, float v) { sT[xi(16 * bi + i, 16 * bk + 8 * nt + n)] = -v; }, lane);
+      warp_store2(d, [&](int i, int n, float v0, float v1) {
+        sT[xi(16 * bi + i, 16 * bk + 8 * nt + n)] = -v0;
+        sT[xi(16 * bi + i, 16 * bk + 8 * nt + n + 1)] = -v1;
+        emit2(16 * bi + i, 16 * bk + 8 * nt + n, -v0, -v1);
+      }, lane);
     }
   }
   __syncthreads();
@@ -218,7 +249,8 @@ __device__ __forceinline__ void unit_lower_inverse(const float* sL, float* sT, f
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     warp_mm<32>(d, [&](int i, int k) { return sT[xi(32 + 16 * mt + i, 32 + k)]; },
                 [&](int k, int n) { return X[k * 36 + 8 * nt + n]; }, lane);
-    warp_store(d, [&](int i, int n, float v) { sT[xi(32 + 16 * mt + i, 8 * nt + n)] = -v; }, lane);
+    warp_store2(d, [&](int i, int n, float v0, float v1) { emit2(32 + 16 * mt + i, 8 * nt + n, -v0, -v1); },
+                lane);
   }
   __syncthreads();
 }
@@ -236,8 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(16) float s_gm[DK];       // gamma_m per key channel
   __shared__ __align__(16) float s_grp[8][DK];   // per-8-token decay products (per-channel path)
   __shared__ __align__(16) float s_Y[2048];
-  __shared__ float s_r[C], s_ri[C], s_ws[C], s_bv[C];  // per-token path: r_t, 1/r_t, beta^k d, beta^v
-  __shared__ float s_lam1[2], s_gm1;
+  // per-token path, by chunk parity: r_t, 1/r_t, beta^k d, beta^v; gamma_C / gamma_m; gamma_m
+  __shared__ float s_r[2][C], s_ri[2][C], s_ws[2][C], s_bv[2][C];
+  __shared__ float s_lam1[2], s_gm1[2];
   __shared__ float s_nx[2][4][C];  // per-token path: gates of the next chunk (alpha, beta^k, d, beta^v)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -254,6 +287,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
+  // rows 0..63 of the [T; P] tile (and of the T~ tile): the 16x16 blocks above the block
+  // diagonal of T are zero and nothing else writes them; set them once
+  for (int e = tid; e < 64 * 8; e += kThreads) {
+    const int t = e >> 3, x8 = e & 7;
+    if ((x8 >> 1) > (t >> 4)) {
+      *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
+      if (SC) *reinterpret_cast<uint4*>(sm + Ly::STQ + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
+    }
+  }
   if (SC) {
     // rows 64..127 of the T~ tile are never meaningful; keep them finite
     for (int i = tid; i < 64 * 128 / 16; i += kThreads)
@@ -334,7 +376,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_commit();
   };
-  if (SC && tid < 64 && nchunks > 0) prefetch_token_gates(0);
+  // per-token path, threads 0..63 (token j): decay factors of chunk cn from its prefetched gates;
+  // warp 1 (tokens 32..63) forms r_j = prod_{s=32..j} alpha_s by an inclusive product scan,
+  // warp 0 (tokens 0..31) forms 1/r_j = prod_{s=j+1..31} alpha_s by an exclusive suffix scan
+  auto token_prep = [&](int cn) {
+    const int j = tid, par = cn & 1;
+    cp_async_wait_all();
+    const float al = s_nx[par][0][j], ws = s_nx[par][1][j] * s_nx[par][2][j], bv = s_nx[par][3][j];
+    if (cn + 1 < nchunks) prefetch_token_gates(cn + 1);
+    float p = al;
+    if (warp == 1) {
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, p, off);
+        if (lane >= off) p *= y;
+      }
+      s_r[par][j] = p;
+      s_ri[par][j] = __fdividef(1.f, p);
+      if (lane == 31) s_lam1[par] = p;
+    } else {
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_down_sync(0xffffffffu, p, off);
+        if (lane + off < 32) p *= y;
+      }
+      const float nxt = __shfl_down_sync(0xffffffffu, p, 1);
+      const float ri = lane == 31 ? 1.f : nxt;
+      s_ri[par][j] = ri;
+      s_r[par][j] = __fdividef(1.f, ri);
+      if (lane == 0) s_gm1[par] = p;
+    }
+    s_ws[par][j] = ws;
+    s_bv[par][j] = bv;
+  };
+  if (SC && tid < 64 && nchunks > 0) {
+    prefetch_token_gates(0);
+    token_prep(0);
+  }
 
   for (int c = 0; c < nchunks; ++c) {
     const int t0 = c * C;
@@ -359,36 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- P1: decay factors (and, per-channel path, the operand tiles)
     if (SC) {
-      if (tid < 64) {
-        const int j = tid;
-        cp_async_wait_all();
-        const float al = s_nx[cur][0][j], ws = s_nx[cur][1][j] * s_nx[cur][2][j], bv = s_nx[cur][3][j];
-        if (c + 1 < nchunks) prefetch_token_gates(c + 1);
-        float p = al;
-        if (warp == 1) {  // tokens 32..63: r_j = prod_{s=32..j} alpha_s (inclusive prefix over lanes)
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, p, off);
-            if (lane >= off) p *= y;
-          }
-          s_r[j] = p;
-          s_ri[j] = __fdividef(1.f, p);
-          if (lane == 31) s_lam1[cur] = p;
-        } else {  // tokens 0..31: 1/r_j = prod_{s=j+1..31} alpha_s (exclusive suffix over lanes)
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const float y = __shfl_down_sync(0xffffffffu, p, off);
-            if (lane + off < 32) p *= y;
-          }
-          const float nxt = __shfl_down_sync(0xffffffffu, p, 1);
-          const float ri = lane == 31 ? 1.f : nxt;
-          s_ri[j] = ri;
-          s_r[j] = __fdividef(1.f, ri);
-          if (lane == 0) s_gm1 = p;
-        }
-        s_ws[j] = ws;
-        s_bv[j] = bv;
-      }
+      // per-token factors of this chunk were computed during the previous chunk (token_prep)
     } else {
       // per-channel path: thread (g4, tg) owns channels 4g4..4g4+3 of tokens 8tg..8tg+7
       const int g4 = lane, tg = warp, cb0 = 4 * g4;
@@ -484,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- P1.5: bring the state into this chunk's frame: S_m = Diag(lambda_prev * gamma_m) S
     {
       const int k = 32 * q4 + lane;
-      const float mu = SC ? ((c == 0) ? s_gm1 : s_lam1[prev] * s_gm1)
+      const float mu = SC ? ((c == 0) ? s_gm1[cur] : s_lam1[prev] * s_gm1[cur])
                           : ((c == 0) ? s_gm[k] : s_lam[prev][k] * s_gm[k]);
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {
@@ -558,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = 32 * ch;
       if (q4 < 2) {
         const int t = 32 * q4 + lane;
-        const float rt = SC ? s_r[t] : 1.f;
+        const float rt = SC ? s_r[cur][t] : 1.f;
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           float y[4];
@@ -566,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int i = i0 + 4 * e4 + e;
             float v = x[4 * e4 + e];
-            if (SC) v *= s_ws[i] * rt * s_ri[i];
+            if (SC) v *= s_ws[cur][i] * rt * s_ri[cur][i];
             y[e] = (i < t) ? v : 0.f;
           }
           sts4(sL, xi(t, i0 + 4 * e4), make_float4(y[0], y[1], y[2], y[3]));
@@ -586,35 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
-    unit_lower_inverse(sL, sT, s_Y, tid);
-    // T -> bf16: TP rows 0..63 (per-token path: T Diag(r) for Wk), and T Diag(beta^v) into the T~ tile
-    {
-      const int t = tid >> 2;
-      const int i0 = 16 * (tid & 3);
-#pragma unroll
-      for (int q8 = 0; q8 < 2; ++q8) {
-        float y[8], z[8];
-#pragma unroll
-        for (int e4 = 0; e4 < 2; ++e4) {
-          const int i = i0 + 8 * q8 + 4 * e4;
-          const float4 v = ((i >> 4) > (t >> 4)) ? f4(0.f) : lds4(sT, xi(t, i));
-          const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            y[4 * e4 + e] = SC ? vv[e] * s_r[i + e] : vv[e];
-            z[4 * e4 + e] = SC ? vv[e] * s_bv[i + e] : 0.f;
-          }
-        }
-        uint4 pk = make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
-                              pack_bf16(y[6], y[7]));
-        *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, i0 / 8 + q8, 128)) = pk;
-        if (SC) {
-          uint4 pz = make_uint4(pack_bf16(z[0], z[1]), pack_bf16(z[2], z[3]), pack_bf16(z[4], z[5]),
-                                pack_bf16(z[6], z[7]));
-          *reinterpret_cast<uint4*>(sm + Ly::STQ + canon_chunk(t, i0 / 8 + q8, 128)) = pz;
-        }
-      }
-    }
+    unit_lower_inverse<SC>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], tid);
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -708,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- P7: U = U0 - Wk S_m (per-token path: U' = beta_t / r_t * U) -> hi / lo tiles
     if (q4 < 2) {
       const int t = 32 * q4 + lane;
-      const float us = SC ? s_ws[t] * s_ri[t] : 1.f;
+      const float us = SC ? s_ws[cur][t] * s_ri[cur][t] : 1.f;
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {
         const int col = ch * (NV / 2) + 32 * cb;
@@ -787,11 +808,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (SC && c + 1 < nchunks) k_pending = true;
 
-    // ---- P9: o rows of this chunk
+    // ---- P9: o rows of this chunk (per-token path: threads 0..63 meanwhile prepare the next chunk)
+    if (SC && tid < 64 && c + 1 < nchunks) token_prep(c + 1);
     if (q4 >= 2) {
       // the TMEM load is warp-collective: every lane loads, only rows of real tokens store
       const int t = 32 * (q4 - 2) + lane;
-      const float os = SC ? s_r[t] : 1.f;
+      const float os = SC ? s_r[cur][t] : 1.f;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0 + t) * H + h) * dv;
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {

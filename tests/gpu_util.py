@@ -37,6 +37,7 @@ def check(o_gpu, S_gpu, o_ref, S_ref, io):
     eo = oracle.rel_l2(host_f64(o_gpu), o_ref)
     eS = oracle.rel_l2(host_f64(S_gpu), S_ref)
     tol = TOL[io]
+    print(f"[parity] o rel-L2 {eo:.3e} (tol {tol['o']:.0e}), S rel-L2 {eS:.3e} (tol {tol['S']:.0e})")
     assert eo <= tol["o"], f"o rel-L2 {eo:.3e} > {tol['o']}"
     assert eS <= tol["S"], f"S_T rel-L2 {eS:.3e} > {tol['S']}"
     return eo, eS
