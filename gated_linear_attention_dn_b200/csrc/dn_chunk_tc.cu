@@ -160,17 +160,19 @@ __device__ __forceinline__ void warp_store(const float* d, FW W, int lane) {
 }
 
 // T = (I + L)^{-1} for the 64x64 strictly lower L in sL (zeros on and above the diagonal).
-// Blocking: the four 16x16 diagonal blocks by forward substitution (one column per thread);
-// the two 32x32 diagonal blocks by T_{i,i-1} = -T_ii L_{i,i-1} T_{i-1,i-1}; the lower-left 32x32
-// block by T21 = -T2 L21 T1. fp32 blocks that later stages read are kept in sT; every element
-// of the lower block triangle is written as bf16 straight into rows 0..63 of the 128-row tile tp
-// (scaled by column factor cs_c[i] when SC) and, when SC, T Diag(cs_v) into tile tt. Blocks
-// strictly above the block diagonal are not written (their zeros are set once by the caller).
-// scr: 2048 floats of scratch. Not inlined: it gets its own register budget. All 256 threads call it.
+// Blocking by doubling: the eight 8x8 diagonal blocks by forward substitution (one column per
+// thread, chains of at most seven steps); then three merge levels with warp mma.sync, each using
+// [[A, 0], [C, B]]^{-1} = [[A^-1, 0], [-B^-1 C A^-1, B^-1]]:
+//   8 -> 16 (warps 0..3), 16 -> 32 (warps 0..1), 32 -> 64 (all 8 warps).
+// fp32 blocks that later levels read are kept in sT; every element of the lower triangle is also
+// written as bf16 straight into rows 0..63 of the 128-row tile tp (scaled by column factor
+// cs_c[i] when SC) and, when SC, T Diag(cs_v) into tile tt. Elements above the 8x8 block diagonal
+// are not written (their zeros are set once by the caller). scr: 2048 floats of scratch.
+// Not inlined: it gets its own register budget. All 256 threads call it.
 template <bool SC>
 __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, float* scr, uint8_t* tp, uint8_t* tt,
                                                 const float* cs_c, const float* cs_v, int tid) {
-  const int warp = tid >> 5, lane = tid & 31;
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
   auto emit1 = [&](int t, int i, float v) {
     const uint32_t off = canon(t, i, 128);
     *reinterpret_cast<__nv_bfloat16*>(tp + off) = __float2bfloat16_rn(SC ? v * cs_c[i] : v);
@@ -182,10 +184,10 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
     if (SC) *reinterpret_cast<uint32_t*>(tt + off) = pack_bf16(v0 * cs_v[i], v1 * cs_v[i + 1]);
   };
   if (tid < 64) {
-    const int blk = tid >> 4, j = tid & 15, base = 16 * blk;
-    float x[16];
+    const int base = 8 * (tid >> 3), j = tid & 7;
+    float x[8];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
+    for (int r = 0; r < 8; ++r) {
       float s0 = (r == j) ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
       for (int i = 0; i < r; ++i) {
@@ -198,34 +200,60 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
       x[r] = s0 + s1;
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
+    for (int r = 0; r < 8; ++r) {
       sT[xi(base + r, base + j)] = x[r];
       emit1(base + r, base + j, x[r]);
     }
   } else {
-    // the upper off-diagonal 16x16 blocks inside the two 32x32 diagonal blocks are zero
-    for (int e = tid - 64; e < 512; e += 192) {
-      const int q = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-      sT[xi(32 * q + r, 32 * q + 16 + cc)] = 0.f;
+    // zero, inside each 32x32 diagonal block, the 8x8 and 16x16 blocks above the diagonal that the
+    // merge levels read: rows 16p..+8 x cols 16p+8..+8 (p < 4); rows 32q..+16 x cols 32q+16..+16 (q < 2)
+    for (int e = tid - 64; e < 768; e += 192) {
+      if (e < 256) {
+        const int p = e >> 6, r = (e >> 3) & 7, cc = e & 7;
+        sT[xi(16 * p + r, 16 * p + 8 + cc)] = 0.f;
+      } else {
+        const int e2 = e - 256, q = e2 >> 8, r = (e2 >> 4) & 15, cc = e2 & 15;
+        sT[xi(32 * q + r, 32 * q + 16 + cc)] = 0.f;
+      }
     }
   }
   __syncthreads();
-  if (warp < 2) {
-    const int bi = 1 + 2 * warp, bk = bi - 1;  // (1,0) and (3,2)
-    float* Y = scr + 1152 + warp * 384;        // 16 x 24 (padded) dense scratch of this warp
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+  // 8 -> 16: T_ba = -T_bb (L_ba T_aa) in each 16x16 diagonal block (rows 8..15 of the 16-row
+  // mma operands repeat rows 0..7 and their results are ignored)
+  if (warp < 4) {
+    const int a0 = 16 * warp, b0 = a0 + 8;
+    float* Y = scr + warp * 96;  // 8 x 12 (padded)
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    warp_mm<8>(d, [&](int i, int k) { return sL[xi(b0 + (i & 7), a0 + k)]; },
+               [&](int k, int n) { return sT[xi(a0 + k, a0 + n)]; }, lane);
+    Y[g * 12 + 2 * t4] = d[0];
+    Y[g * 12 + 2 * t4 + 1] = d[1];
+    __syncwarp();
+    float e[4] = {0.f, 0.f, 0.f, 0.f};
+    warp_mm<8>(e, [&](int i, int k) { return sT[xi(b0 + (i & 7), b0 + k)]; },
+               [&](int k, int n) { return Y[k * 12 + n]; }, lane);
+    sT[xi(b0 + g, a0 + 2 * t4)] = -e[0];
+    sT[xi(b0 + g, a0 + 2 * t4 + 1)] = -e[1];
+    emit2(b0 + g, a0 + 2 * t4, -e[0], -e[1]);
+  }
+  __syncthreads();
+  // 16 -> 32: T_{i,i-1} = -T_ii (L_{i,i-1} T_{i-1,i-1}) for (i, i-1) = (1, 0), (3, 2); warp w < 4
+  // owns pair w / 2 and the 8-column tile w % 2 (a column tile of the result needs only the
+  // same column tile of L T)
+  if (warp < 4) {
+    const int bi = 1 + 2 * (warp >> 1), bk = bi - 1, nt = warp & 1;
+    float* Y = scr + 1152 + warp * 192;  // 16 x 12 (padded) dense scratch of this warp
+    {
       float d[4] = {0.f, 0.f, 0.f, 0.f};
       warp_mm<16>(d, [&](int i, int k) { return sL[xi(16 * bi + i, 16 * bk + k)]; },
                   [&](int k, int n) { return sT[xi(16 * bk + k, 16 * bk + 8 * nt + n)]; }, lane);
-      warp_store(d, [&](int i, int n, float v) { Y[i * 24 + 8 * nt + n] = v; }, lane);
+      warp_store(d, [&](int i, int n, float v) { Y[i * 12 + n] = v; }, lane);
     }
     __syncwarp();
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    {
       float d[4] = {0.f, 0.f, 0.f, 0.f};
       warp_mm<16>(d, [&](int i, int k) { return sT[xi(16 * bi + i, 16 * bi + k)]; },
-                  [&](int k, int n) { return Y[k * 24 + 8 * nt + n]; }, lane);
+                  [&](int k, int n) { return Y[k * 12 + n]; }, lane);
       warp_store2(d, [&](int i, int n, float v0, float v1) {
         sT[xi(16 * bi + i, 16 * bk + 8 * nt + n)] = -v0;
         sT[xi(16 * bi + i, 16 * bk + 8 * nt + n + 1)] = -v1;
@@ -234,10 +262,10 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
     }
   }
   __syncthreads();
-  // X = L21 T1: warp w computes rows 16 (w / 4) .. +16, columns 8 (w % 4) .. +8
+  // 32 -> 64: X = L21 T1, then T21 = -T2 X; warp w owns rows 16 (w / 4) .. +16, columns 8 (w % 4) .. +8
   float* X = scr;  // 32 x 36 (padded) dense
+  const int mt = warp >> 2, nt = warp & 3;
   {
-    const int mt = warp >> 2, nt = warp & 3;
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     warp_mm<32>(d, [&](int i, int k) { return sL[xi(32 + 16 * mt + i, k)]; },
                 [&](int k, int n) { return sT[xi(k, 8 * nt + n)]; }, lane);
@@ -245,7 +273,6 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
   }
   __syncthreads();
   {
-    const int mt = warp >> 2, nt = warp & 3;
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     warp_mm<32>(d, [&](int i, int k) { return sT[xi(32 + 16 * mt + i, 32 + k)]; },
                 [&](int k, int n) { return X[k * 36 + 8 * nt + n]; }, lane);
@@ -262,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Ly = Layout<DK, NV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bar_qk, bar_k, bar_v, bar_mma;
+  __shared__ __align__(8) uint64_t bar_qk, bar_k, bar_v, bar_mma, bar_gram;
+  __shared__ int s_gram_ready;  // per-token path: the next chunk's Gram MMA was issued early
   __shared__ uint32_t s_tmem;
   __shared__ __align__(16) float s_lam[2][DK];   // gamma_C / gamma_m per key channel (per-channel path)
   __shared__ __align__(16) float s_gm[DK];       // gamma_m per key channel
@@ -284,14 +312,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bar_k, 1);
     mbar_init(&bar_v, 1);
     mbar_init(&bar_mma, 1);
+    mbar_init(&bar_gram, 1);
+    s_gram_ready = 0;
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
-  // rows 0..63 of the [T; P] tile (and of the T~ tile): the 16x16 blocks above the block
-  // diagonal of T are zero and nothing else writes them; set them once
+  // rows 0..63 of the [T; P] tile (and of the T~ tile): the 8x8 blocks above the block diagonal
+  // of T are zero and nothing else writes them; set them once
   for (int e = tid; e < 64 * 8; e += kThreads) {
     const int t = e >> 3, x8 = e & 7;
-    if ((x8 >> 1) > (t >> 4)) {
+    if (x8 > (t >> 3)) {
       *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
       if (SC) *reinterpret_cast<uint4*>(sm + Ly::STQ + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
     }
@@ -339,8 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < NV / 64; ++x) tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, 64 * x, h, c * C, b);
   };
 
-  uint32_t ph_qk = 0, ph_k = 0, ph_v = 0, ph_mma = 0;
-  bool qk_pending = false, k_pending = false, v_pending = false, mma_pending = false;
+  uint32_t ph_qk = 0, ph_k = 0, ph_v = 0, ph_mma = 0, ph_gram = 0;
+  bool qk_pending = false, k_pending = false, v_pending = false, mma_pending = false, gram_pending = false;
   bool failed = false;
   if (tid == 0 && nchunks > 0) {
     issue_qk(0);
@@ -360,8 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // per-token path: thread j < 64 copies token j's gates of the next chunk into shared memory
   // one chunk ahead with cp.async (absent gates and tokens past the end are written directly)
-  auto prefetch_token_gates = [&](int cn) {
-    const int j = tid, t0n = cn * C;
+  auto prefetch_token_gates = [&](int cn, int j) {
+    const int t0n = cn * C;
     float* dst = &s_nx[cn & 1][0][j];
     const float* src[4] = {a.alpha_p, a.beta_k_p, a.key_scale_p, a.beta_v_p};
     const int mode[4] = {a.alpha, a.beta_k, a.key_scale, a.beta_v};
@@ -379,13 +409,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // per-token path, threads 0..63 (token j): decay factors of chunk cn from its prefetched gates;
   // warp 1 (tokens 32..63) forms r_j = prod_{s=32..j} alpha_s by an inclusive product scan,
   // warp 0 (tokens 0..31) forms 1/r_j = prod_{s=j+1..31} alpha_s by an exclusive suffix scan
-  auto token_prep = [&](int cn) {
-    const int j = tid, par = cn & 1;
+  auto token_prep = [&](int cn, int j, bool upper) {
+    const int par = cn & 1;
     cp_async_wait_all();
     const float al = s_nx[par][0][j], ws = s_nx[par][1][j] * s_nx[par][2][j], bv = s_nx[par][3][j];
-    if (cn + 1 < nchunks) prefetch_token_gates(cn + 1);
+    if (cn + 1 < nchunks) prefetch_token_gates(cn + 1, j);
     float p = al;
-    if (warp == 1) {
+    if (upper) {
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const float y = __shfl_up_sync(0xffffffffu, p, off);
@@ -410,9 +440,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     s_bv[par][j] = bv;
   };
   if (SC && tid < 64 && nchunks > 0) {
-    prefetch_token_gates(0);
-    token_prep(0);
+    prefetch_token_gates(0, tid);
+    token_prep(0, tid, warp == 1);
   }
+
+  // S_m = Diag(lambda_prev * gamma_m) S for rows 32 q4 .. +32, columns of half ch: the state in
+  // chunk c's frame, in TMEM (fp32) and as the bf16 operand tile
+  auto state_to_frame = [&](int c) {
+    const int cur = c & 1, prev = cur ^ 1;
+    const int k = 32 * q4 + lane;
+    const float mu = SC ? ((c == 0) ? s_gm1[cur] : s_lam1[prev] * s_gm1[cur])
+                        : ((c == 0) ? s_gm[k] : s_lam[prev][k] * s_gm[k]);
+#pragma unroll
+    for (int cb = 0; cb < NV / 64; ++cb) {
+      const int col = ch * (NV / 2) + 32 * cb;
+      float x[32];
+      if (c == 0) {
+        if (a.S0) {
+          const float* src = a.S0 + ((int64_t)bh * DK + k) * dv + col;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 f = *reinterpret_cast<const float4*>(src + e);
+            x[e] = f.x, x[e + 1] = f.y, x[e + 2] = f.z, x[e + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = 0.f;
+        }
+      } else {
+        tmem_ld32(tmem + lane_base + Ly::TM_S + col, x);
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] *= mu;
+      tmem_st32(tmem + lane_base + Ly::TM_S + col, x);
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
+                              pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
+        *reinterpret_cast<uint4*>(sm + Ly::SM + canon_chunk(k, col / 8 + q8, DK)) = pk;
+      }
+    }
+  };
+  // o rows of chunk c from rows 64..127 of D1 (warps of quadrants 2 and 3, columns of half ch); the
+  // TMEM load is warp-collective: every lane loads, only rows of real tokens store
+  auto store_o = [&](int c) {
+    const int t = 32 * (q4 - 2) + lane, t0c = c * C, nc = min(C, T - t0c);
+    const float os = SC ? s_r[c & 1][t] : 1.f;
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0c + t) * H + h) * dv;
+#pragma unroll
+    for (int cb = 0; cb < NV / 64; ++cb) {
+      const int col = ch * (NV / 2) + 32 * cb;
+      float x[32];
+      tmem_ld32(tmem + lane_base + Ly::TM_D1 + col, x);
+      if (t < nc) {
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint4 pk = make_uint4(pack_bf16(os * x[8 * q8], os * x[8 * q8 + 1]),
+                                pack_bf16(os * x[8 * q8 + 2], os * x[8 * q8 + 3]),
+                                pack_bf16(os * x[8 * q8 + 4], os * x[8 * q8 + 5]),
+                                pack_bf16(os * x[8 * q8 + 6], os * x[8 * q8 + 7]));
+          *reinterpret_cast<uint4*>(orow + col + 8 * q8) = pk;
+        }
+      }
+    }
+  };
+
+  // Gram [K+; Q+] W-^T (per-token path: [K; Q] K^T) of chunk c -> TMEM scratch; thread 0 only
+  auto issue_gram = [&](int c) {
+    uint8_t* kqc = kq_buf(c);
+    const uint8_t* gb = SC ? kqc : sm + Ly::WHI;
+    const uint32_t gb_blk = SC ? 128 * 128 : C * 128;
+#pragma unroll
+    for (int kk = 0; kk < DK; kk += 16) {
+      const uint64_t ad = sdesc(smem_u32(kqc) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+      const uint64_t bd = sdesc(smem_u32(gb) + (kk >> 6) * gb_blk + (kk & 63) * 2, 16, 1024);
+      mma_bf16(tmem + Ly::TM_SCR, ad, bd, id_gram, kk > 0);
+    }
+  };
 
   for (int c = 0; c < nchunks; ++c) {
     const int t0 = c * C;
@@ -530,66 +634,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    // ---- P1.5: bring the state into this chunk's frame: S_m = Diag(lambda_prev * gamma_m) S
-    {
-      const int k = 32 * q4 + lane;
-      const float mu = SC ? ((c == 0) ? s_gm1[cur] : s_lam1[prev] * s_gm1[cur])
-                          : ((c == 0) ? s_gm[k] : s_lam[prev][k] * s_gm[k]);
-#pragma unroll
-      for (int cb = 0; cb < NV / 64; ++cb) {
-        const int col = ch * (NV / 2) + 32 * cb;
-        float x[32];
-        if (c == 0) {
-          if (a.S0) {
-            const float* src = a.S0 + ((int64_t)bh * DK + k) * dv + col;
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 f = *reinterpret_cast<const float4*>(src + e);
-              x[e] = f.x, x[e + 1] = f.y, x[e + 2] = f.z, x[e + 3] = f.w;
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = 0.f;
-          }
-        } else {
-          tmem_ld32(tmem + lane_base + Ly::TM_S + col, x);
-        }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] *= mu;
-        tmem_st32(tmem + lane_base + Ly::TM_S + col, x);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
-                                pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
-          *reinterpret_cast<uint4*>(sm + Ly::SM + canon_chunk(k, col / 8 + q8, DK)) = pk;
-        }
-      }
-    }
+    // ---- P1.5: (the state is brought into this chunk's frame while the T MMAs run, below)
     fence_proxy_async();
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
 
     // ---- P2: Gram [K+; Q+] W-^T (per-token path: [K; Q] K^T) -> scratch
-    if (tid == 0) {
-      // per-channel path: the raw q, k staging was consumed by the prep; prefetch the next chunk
-      if (!SC && c + 1 < nchunks) {
-        fence_proxy_async();
-        issue_qk(c + 1);
+    const bool gram_early = SC && s_gram_ready;  // uniform: written before the last barrier
+    if (gram_early) {
+      bool ok = mbar_wait_bounded(&bar_gram, ph_gram, kWaitNs);
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
       }
-      const uint8_t* gb = SC ? kq : sm + Ly::WHI;
-      const uint32_t gb_blk = SC ? 128 * 128 : C * 128;
-#pragma unroll
-      for (int kk = 0; kk < DK; kk += 16) {
-        const uint64_t ad = sdesc(smem_u32(kq) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
-        const uint64_t bd = sdesc(smem_u32(gb) + (kk >> 6) * gb_blk + (kk & 63) * 2, 16, 1024);
-        mma_bf16(tmem + Ly::TM_SCR, ad, bd, id_gram, kk > 0);
+      ph_gram ^= 1;
+      gram_pending = false;
+      tc_fence_after();
+    } else {
+      if (tid == 0) {
+        // per-channel path: the raw q, k staging was consumed by the prep; prefetch the next chunk
+        if (!SC && c + 1 < nchunks) {
+          fence_proxy_async();
+          issue_qk(c + 1);
+        }
+        issue_gram(c);
+        mma_commit(&bar_mma);
       }
-      mma_commit(&bar_mma);
-    }
-    if (!SC && c + 1 < nchunks) qk_pending = true;
-    mma_pending = true;
-    {
+      if (!SC && c + 1 < nchunks) qk_pending = true;
+      mma_pending = true;
       bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
       if (__syncthreads_or(!ok)) {
         failed = true;
@@ -635,6 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    tc_fence_after();
     unit_lower_inverse<SC>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], tid);
     fence_proxy_async();
     tc_fence_before();
@@ -667,6 +739,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bar_mma);
     }
     mma_pending = true;
+    // while those MMAs run: the previous chunk's outputs (D1 rows 64..127) and the state in this
+    // chunk's frame (S_acc columns; no overlap with the TMEM the MMAs write)
+    if (!SC && c > 0 && q4 >= 2) store_o(c - 1);
+    state_to_frame(c);
     {
       bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
       if (__syncthreads_or(!ok)) {
@@ -727,6 +803,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- P7: U = U0 - Wk S_m (per-token path: U' = beta_t / r_t * U) -> hi / lo tiles
+    // (per-token path: warps 2, 3 meanwhile compute the next chunk's decay factors)
+    if (SC && (warp == 2 || warp == 3) && c + 1 < nchunks) token_prep(c + 1, tid - 64, warp == 3);
     if (q4 < 2) {
       const int t = 32 * q4 + lane;
       const float us = SC ? s_ws[cur][t] * s_ri[cur][t] : 1.f;
@@ -789,6 +867,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       mma_commit(&bar_mma);
+      // per-token path: the next chunk's [K; Q] tile has its own buffer; once it has landed, its
+      // Gram can follow these MMAs on the tensor core right away
+      int ready = 0;
+      if (SC && c + 1 < nchunks && mbar_wait_bounded(&bar_qk, ph_qk, kWaitNs)) {
+        issue_gram(c + 1);
+        mma_commit(&bar_gram);
+        ready = 1;
+      }
+      s_gram_ready = ready;
     }
     mma_pending = true;
     {
@@ -801,43 +888,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_pending = false;
       tc_fence_after();
     }
+    if (SC && s_gram_ready) gram_pending = true;
     // per-token path: the raw k tile of the state update is free now: load the next chunk's
     if (SC && tid == 0 && c + 1 < nchunks) {
       fence_proxy_async();
       issue_k(c + 1);
     }
     if (SC && c + 1 < nchunks) k_pending = true;
+    // per-token path: this chunk's outputs, while the next chunk's Gram runs
+    if (SC && q4 >= 2) store_o(c);
 
-    // ---- P9: o rows of this chunk (per-token path: threads 0..63 meanwhile prepare the next chunk)
-    if (SC && tid < 64 && c + 1 < nchunks) token_prep(c + 1);
-    if (q4 >= 2) {
-      // the TMEM load is warp-collective: every lane loads, only rows of real tokens store
-      const int t = 32 * (q4 - 2) + lane;
-      const float os = SC ? s_r[cur][t] : 1.f;
-      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0 + t) * H + h) * dv;
-#pragma unroll
-      for (int cb = 0; cb < NV / 64; ++cb) {
-        const int col = ch * (NV / 2) + 32 * cb;
-        float x[32];
-        tmem_ld32(tmem + lane_base + Ly::TM_D1 + col, x);
-        if (t < n) {
-#pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {
-            uint4 pk = make_uint4(pack_bf16(os * x[8 * q8], os * x[8 * q8 + 1]),
-                                  pack_bf16(os * x[8 * q8 + 2], os * x[8 * q8 + 3]),
-                                  pack_bf16(os * x[8 * q8 + 4], os * x[8 * q8 + 5]),
-                                  pack_bf16(os * x[8 * q8 + 6], os * x[8 * q8 + 7]));
-            *reinterpret_cast<uint4*>(orow + col + 8 * q8) = pk;
-          }
-        }
-      }
-    }
+    // ---- P9: (this chunk's outputs are stored during the next chunk's inverse, or after the loop)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
   }
 
   if (!failed && nchunks > 0) {
+    if (!SC && q4 >= 2) store_o(nchunks - 1);
     // S_T = Diag(gamma_C / gamma_m) S_acc of the last chunk
     const int k = 32 * q4 + lane;
     const float lam = SC ? s_lam1[(nchunks - 1) & 1] : s_lam[(nchunks - 1) & 1][k];
@@ -858,6 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (k_pending) mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
     if (v_pending) mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
     if (mma_pending) mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+    if (gram_pending) mbar_wait_bounded(&bar_gram, ph_gram, kWaitNs);
     if (tid == 0) atomicExch(a.status, kDevTimeout);
   }
   tc_fence_before();
