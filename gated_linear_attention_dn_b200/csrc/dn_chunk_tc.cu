@@ -96,6 +96,33 @@ __device__ __forceinline__ float4 gate4(const float* g, int mode, int64_t tok, i
   return *reinterpret_cast<const float4*>(g + tok * width + ch);
 }
 
+// Gate values of 8 tokens (rows tok0 + i * tstride, i < 8) for 4 consecutive channels, with every
+// load issued before any is used: the mode branch is uniform and outside the loads, and tokens past
+// the end (i >= nvalid) re-read row tok0 + (nvalid - 1) * tstride, or row tok0 when nvalid == 0
+// (the caller points tok0 at a real token then); their values are replaced by `dflt`.
+__device__ __forceinline__ void gate4x8(float4* out, const float* g, int mode, int64_t tok0, int64_t tstride,
+                                        int width, int ch, int nvalid, float dflt) {
+  if (mode == DN_GATE_CHANNEL) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ic = i < nvalid ? i : max(nvalid - 1, 0);
+      out[i] = __ldg(reinterpret_cast<const float4*>(g + (tok0 + ic * tstride) * width + ch));
+    }
+  } else if (mode == DN_GATE_SCALAR) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ic = i < nvalid ? i : max(nvalid - 1, 0);
+      out[i] = f4(__ldg(g + tok0 + ic * tstride));
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = f4(1.f);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (i >= nvalid) out[i] = f4(dflt);
+}
+
 __device__ __forceinline__ float4 lds4(const float* p, int idx) { return *reinterpret_cast<const float4*>(p + idx); }
 __device__ __forceinline__ void sts4(float* p, int idx, float4 v) { *reinterpret_cast<float4*>(p + idx) = v; }
 
@@ -545,20 +572,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       // per-channel path: thread (g4, tg) owns channels 4g4..4g4+3 of tokens 8tg..8tg+7
       const int g4 = lane, tg = warp, cb0 = 4 * g4;
-      float4 al[8], ws[8];
+      float4 al[8], ws[8], dd[8];
       uint2 kr[8], qr[8];
+      // tokens 8 tg .. 8 tg + 7 of this chunk; a group wholly past the end reads token 0 of the
+      // chunk (always a real token) and discards it
+      const int nvalid = max(0, min(8, n - 8 * tg));
+      const int64_t tok0 = ((int64_t)b * T + t0 + (nvalid > 0 ? 8 * tg : 0)) * H + h;
+      gate4x8(al, a.alpha_p, a.alpha, tok0, H, DK, cb0, nvalid, 1.f);
+      gate4x8(ws, a.beta_k_p, a.beta_k, tok0, H, DK, cb0, nvalid, 0.f);
+      gate4x8(dd, a.key_scale_p, a.key_scale, tok0, H, DK, cb0, nvalid, 0.f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int j = 8 * tg + i;
-        const bool valid = j < n;
-        const int64_t tok = ((int64_t)b * T + t0 + j) * H + h;
-        al[i] = valid ? gate4(a.alpha_p, a.alpha, tok, DK, cb0) : f4(1.f);
-        ws[i] = valid ? mul4(gate4(a.beta_k_p, a.beta_k, tok, DK, cb0),
-                             gate4(a.key_scale_p, a.key_scale, tok, DK, cb0))
-                      : f4(0.f);
         kr[i] = *reinterpret_cast<const uint2*>(sm + Ly::STK + canon(j, cb0, C));
         qr[i] = *reinterpret_cast<const uint2*>(sm + Ly::STQ + canon(j, cb0, C));
       }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ws[i] = mul4(ws[i], dd[i]);
       // products inside the group: prefix (second half) or exclusive suffix (first half)
       float4 loc[8];
       float4 grp;
@@ -617,12 +647,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (bv_split && cb0 < NV) {
         // V~ = beta^v (.) v, split hi (in place) / lo
+        float4 bvs[8];
+        gate4x8(bvs, a.beta_v_p, a.beta_v, tok0, H, dv, cb0, nvalid, 0.f);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int j = 8 * tg + i;
-          const bool valid = j < n;
-          const int64_t tok = ((int64_t)b * T + t0 + j) * H + h;
-          const float4 bv = valid ? gate4(a.beta_v_p, a.beta_v, tok, dv, cb0) : f4(0.f);
+          const float4 bv = bvs[i];
           const uint32_t off2 = canon(j, cb0, C);
           const float4 vv = unpack4(*reinterpret_cast<const uint2*>(sm + Ly::STV + off2));
           uint2 hi, lo;
