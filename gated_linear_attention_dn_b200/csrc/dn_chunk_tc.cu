@@ -331,7 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, ch = warp >> 2;
   const int T = a.T, H = a.H, dv = a.dv;
-  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+  // one CTA per (b, h) and slice of NV value columns (columns of the state evolve independently)
+  const int nslices = dv / NV;
+  const int bh = blockIdx.x / nslices, b = bh / H, h = bh % H;
+  const int col0 = (blockIdx.x % nslices) * NV;
   const int nchunks = (T + C - 1) / C;
 
   if (tid == 0) {
@@ -393,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto issue_v = [&](int c) {
     mbar_expect_tx(&bar_v, (uint32_t)C * NV * 2);
 #pragma unroll
-    for (int x = 0; x < NV / 64; ++x) tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, 64 * x, h, c * C, b);
+    for (int x = 0; x < NV / 64; ++x)
+      tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, col0 + 64 * x, h, c * C, b);
   };
 
   uint32_t ph_qk = 0, ph_k = 0, ph_v = 0, ph_mma = 0, ph_gram = 0;
@@ -484,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float x[32];
       if (c == 0) {
         if (a.S0) {
-          const float* src = a.S0 + ((int64_t)bh * DK + k) * dv + col;
+          const float* src = a.S0 + ((int64_t)bh * DK + k) * dv + col0 + col;
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const float4 f = *reinterpret_cast<const float4*>(src + e);
@@ -513,7 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto store_o = [&](int c) {
     const int t = 32 * (q4 - 2) + lane, t0c = c * C, nc = min(C, T - t0c);
     const float os = SC ? s_r[c & 1][t] : 1.f;
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0c + t) * H + h) * dv;
+    __nv_bfloat16* orow =
+        reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0c + t) * H + h) * dv + col0;
 #pragma unroll
     for (int cb = 0; cb < NV / 64; ++cb) {
       const int col = ch * (NV / 2) + 32 * cb;
@@ -648,7 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bv_split && cb0 < NV) {
         // V~ = beta^v (.) v, split hi (in place) / lo
         float4 bvs[8];
-        gate4x8(bvs, a.beta_v_p, a.beta_v, tok0, H, dv, cb0, nvalid, 0.f);
+        gate4x8(bvs, a.beta_v_p, a.beta_v, tok0, H, dv, col0 + cb0, nvalid, 0.f);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int j = 8 * tg + i;
@@ -944,7 +949,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int col = ch * (NV / 2) + 32 * cb;
       float x[32];
       tmem_ld32(tmem + lane_base + Ly::TM_S + col, x);
-      float* dst = a.S + ((int64_t)bh * DK + k) * dv + col;
+      float* dst = a.S + ((int64_t)bh * DK + k) * dv + col0 + col;
 #pragma unroll
       for (int e = 0; e < 32; e += 4)
         *reinterpret_cast<float4*>(dst + e) = make_float4(lam * x[e], lam * x[e + 1], lam * x[e + 2], lam * x[e + 3]);
@@ -1002,9 +1007,9 @@ cudaError_t launch_impl(const Args& a, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   if (!get_encode()) return cudaErrorNotSupported;
   if (!make_map(&mq, a.q, DK, a.H, a.T, a.B) || !make_map(&mk, a.k, DK, a.H, a.T, a.B) ||
-      !make_map(&mv, a.v, NV, a.H, a.T, a.B))
+      !make_map(&mv, a.v, a.dv, a.H, a.T, a.B))
     return cudaErrorInvalidValue;
-  chunk_tc_kernel<DK, NV, SC><<<a.B * a.H, kThreads, smem, s>>>(mq, mk, mv, a);
+  chunk_tc_kernel<DK, NV, SC><<<a.B * a.H * (a.dv / NV), kThreads, smem, s>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -1018,7 +1023,12 @@ cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s) {
   // per-token gates only -> the raw-tile path
   const bool sc = a.alpha != DN_GATE_CHANNEL && a.beta_k != DN_GATE_CHANNEL && a.beta_v != DN_GATE_CHANNEL &&
                   a.key_scale != DN_GATE_CHANNEL;
-  if (a.dv == 128) return sc ? launch_impl<128, 128, true>(a, s) : launch_impl<128, 128, false>(a, s);
+  // few sequences: split the 128 value columns into two 64-column CTAs when that still fits in one
+  // wave (each CTA repeats the column-independent prep, Gram and inverse)
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const bool split = a.dv == 128 && (int64_t)a.B * a.H * 2 <= sms;
+  if (a.dv == 128 && !split) return sc ? launch_impl<128, 128, true>(a, s) : launch_impl<128, 128, false>(a, s);
   return sc ? launch_impl<128, 64, true>(a, s) : launch_impl<128, 64, false>(a, s);
 }
 
