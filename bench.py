@@ -104,8 +104,9 @@ class ClockSampler:
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, interval_ms: int = 100):
         self.index = index
+        self.interval_ms = interval_ms
         self.proc = None
         self.lines = []
         self.t = None
@@ -113,7 +114,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -170,6 +171,15 @@ def oracle_sample(w: di.Workload, x: dict, budget_s: float, nthreads: int, heads
     return done * w.T, t_total, done
 
 
+def bench_config(world: int) -> dict:
+    """The workload description both arms print (the reference arm times the oracle on it)."""
+    w = di.WORKLOADS[WORKLOAD]
+    alg = algorithmic_bytes(w)
+    return {"workload": "gdn_prefill B=8 H=16 T=4096 d_k=d_v=128 bf16 q/k/v, scalar fp32 gates, chunk 64, S0=0",
+            "global_batch": w.B * world, "seq_len": w.T, "parallelism": f"dp{world}",
+            "l2": f"inputs {alg / 1e6:.0f} MB per step > {L2_BYTES / 1e6:.0f} MB L2 (no flush)"}
+
+
 def run_reference(args, rank: int, world: int):
     """CPU oracle arm: each step times the oracle on a bounded sample of the workload."""
     if rank != 0:
@@ -196,14 +206,63 @@ def run_reference(args, rank: int, world: int):
         "impl": "reference", "metric": METRIC, "value": tok_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "gdn_prefill B=8 H=16 T=4096 d_k=d_v=128 bf16, scalar gates",
-                   "global_batch": w.B, "seq_len": w.T, "parallelism": "cpu-oracle"},
+        "config": bench_config(world),
         "cpu_baseline": {"value": tok_per_s, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
                          "sample": f"{nheads} whole heads of T={w.T} per step (all heads are independent); "
                                    "tokens/s = head-tokens/s / H"},
         "e2e": {"value": tok_per_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_single_kernel(args):
+    """Profiling mode: warm-up + timed launches of one kernel on a (smaller) batch of a workload.
+
+    Used for the ncu captures summarised in profiles/: the same code path as the bench, with a
+    batch that keeps the capture small while the inputs stay larger than L2."""
+    import torch
+
+    import gated_linear_attention_dn_b200 as dn
+    from gated_linear_attention_dn_b200 import build as dnbuild
+
+    if not os.path.exists(dnbuild.LIB):
+        dnbuild.build()
+    name = WORKLOAD if args.only == "chunk" else DECODE
+    w = di.WORKLOADS[name]
+    if args.batch:
+        w = w.scaled(B=args.batch)
+    x = di.make_inputs(w)
+
+    def to_dev(a):
+        if a is None:
+            return None
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+        return t.cuda()
+
+    xd = {n: to_dev(a) for n, a in x.items()}
+    S = xd["S0"].clone() if xd["S0"] is not None else None
+
+    def launch():
+        if args.only == "chunk":
+            dn.dn_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                            xd["S0"])
+        else:
+            dn.dn_decode_step(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"],
+                              xd["key_scale"], S=S)
+
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        launch()
+    e1.record()
+    torch.cuda.synchronize()
+    if dn.dn_stream_status() != dn.DN_OK:
+        raise RuntimeError("device status")
+    print(json.dumps({"only": args.only, "workload": name, "batch": w.B, "steps": args.steps,
+                      "ms_per_launch": e0.elapsed_time(e1) / max(1, args.steps)}))
 
 
 def main():
@@ -215,6 +274,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=100)
+    ap.add_argument("--only", choices=["chunk", "decode"], default=None,
+                    help="profiling mode: run just one kernel on the workload with batch --batch")
+    ap.add_argument("--batch", type=int, default=0, help="with --only: batch size of the scaled workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -225,6 +287,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.only:
+        run_single_kernel(args)
         return
 
     import torch
@@ -265,6 +330,11 @@ def main():
         if world > 1:
             dist.barrier()
 
+    # clocks are sampled from before the warm-up to the end of the decode timing: the timed regions
+    # alone are often shorter than one nvidia-smi sampling interval
+    clocks = ClockSampler(local)
+    clocks.__enter__()
+    time.sleep(0.3)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -272,15 +342,14 @@ def main():
         raise RuntimeError("device status after warm-up")
 
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    with ClockSampler(local) as clocks:
-        barrier()
-        torch.cuda.synchronize()
-        evs[0].record(stream)
-        for i in range(args.steps):
-            step()
-            evs[i + 1].record(stream)
-        torch.cuda.synchronize()
-        barrier()
+    barrier()
+    torch.cuda.synchronize()
+    evs[0].record(stream)
+    for i in range(args.steps):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
     per_launch_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
     total_ms = evs[0].elapsed_time(evs[-1])
     if dn.dn_stream_status(stream) != dn.DN_OK:
@@ -375,6 +444,8 @@ def main():
         launches += nd
         del steps_dev, S
 
+    clocks.__exit__(None, None, None)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -390,10 +461,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "gdn_prefill B=8 H=16 T=4096 d_k=d_v=128 bf16 q/k/v, scalar fp32 gates, "
-                                   "chunk 64, S0=0",
-                       "global_batch": B * world, "seq_len": T, "parallelism": f"dp{world}",
-                       "l2": f"inputs {alg / 1e6:.0f} MB per step > {L2_BYTES / 1e6:.0f} MB L2 (no flush)"},
+            "config": bench_config(world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode,
             "kernel_source": kernel_source_hash(),
