@@ -1,0 +1,628 @@
+// Tensor-core chunked prefill for per-token gates (GDN: scalar alpha, beta^k, beta^v, d; bf16 io,
+// d_k = 128, d_v in {64, 128}) for sm_100a, with the chunk-local UT transform pipelined one chunk
+// ahead of the state recurrence.
+//
+// One CTA owns one (b, h) sequence (and a slice of NV value columns) and walks its chunks of
+// C = 64 tokens. Per chunk, with decays referenced to the chunk midpoint m (after token 31) and
+// every gate a scalar per token:
+//
+//   r_t = gamma_t / gamma_m,  A_ti = (k_t . k_i) beta_i d_i r_t / r_i  (i < t),  T = (I + A)^{-1}
+//   Wk = (T Diag(r)) K,  U0 = (T Diag(beta^v)) V,  S_m = Diag(gamma_m) S
+//   U' = Diag(beta d / r) (U0 - Wk S_m)
+//   O_t = r_t (Q S_m + P U')_t,  P_ti = q_t . k_i (i <= t)
+//   S' = (gamma_C / gamma_m) (S_m + K^T U')
+//
+// (the chunk-parallel WY / UT evaluation of the gated delta rule: FG2-GDN page, sections 2.A and
+// 3 item 2; the scalar-gate rewriting of it keeps the raw TMA tiles of q, k, v as tensor-core
+// operands with no elementwise pass).
+//
+// Only the last four lines depend on the state. Two warp groups therefore work one chunk apart:
+//  * the state group (warps 0..7) runs the state chain of chunk c: the Wk and U0 products, S_m,
+//    D1 = [Wk; Q] S_m, U', the O and state-update products and the o store;
+//  * the transform group (warps 8..15) meanwhile prepares chunk c + 1: its decay factors, A and P
+//    from the Gram product [K; Q] K^T (issued by the state group right after chunk c's Wk / U0
+//    products), and the inverse T, emitted as the bf16 operand tiles T Diag(r) and T Diag(beta^v).
+// Hand-offs are mbarriers: the transform group arrives on `tready` once chunk c + 1's tiles are in
+// shared memory; the Gram of chunk c + 1 is committed after chunk c's Wk / U0 products, so its
+// completion also tells the transform group that the T tiles of chunk c are no longer read.
+// P is double-buffered by chunk parity; the per-token factors are kept for four chunks.
+//
+// Precision: bf16 operands, fp32 accumulation; U' is split hi + lo for the state update (raw k is
+// exact in bf16); T is inverted in fp32 (TF32 block merges) and rounded to bf16 once.
+//
+// Tensor memory (512 columns): S_acc | D1 | U0 | (Wk, d_v = 64 only) | Gram; Wk shares D1's columns
+// when d_v = 128 (D1 is written only after Wk has been read).
+// Every mbarrier wait is bounded in time; on expiry both groups leave their loops, the state group
+// drains what it issued (bounded), the CTA sets the status word and frees its tensor memory.
+#include "dn_common.cuh"
+#include "dn_tc_ptx.cuh"
+#include "dn_ut_inverse.cuh"
+
+namespace dn {
+namespace {
+
+using namespace tc;
+using namespace ut;
+
+constexpr int C = 64;
+constexpr int DK = 128;
+constexpr int kStateThreads = 256;   // warps 0..7
+constexpr int kXformThreads = 256;   // warps 8..15
+constexpr int kThreads = kStateThreads + kXformThreads;
+constexpr int kBarState = 1, kBarXform = 2;   // hardware barriers of the two groups (0 = whole CTA)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, far above any legitimate wait
+
+template <int NV>
+struct ScLayout {
+  static constexpr int STK = 0;                   // raw k [C][DK] (TMA): state-update operand
+  static constexpr int STQ = STK + C * DK * 2;    // T Diag(beta^v) [128][C] (rows 64..127 zero)
+  static constexpr int STV = STQ + 128 * C * 2;   // raw v [C][NV] (TMA)
+  static constexpr int KQ0 = STV + C * NV * 2;    // [K; Q] (TMA), then [Wk; Q]: even chunks
+  static constexpr int KQ1 = KQ0 + 128 * DK * 2;  //                               odd chunks
+  static constexpr int TP = KQ1 + 128 * DK * 2;   // T Diag(r) | P (even chunks) | P (odd chunks), 64 rows each
+  static constexpr int SMU = TP + 3 * C * C * 2;  // S_m bf16 [DK][NV]; after D1: U' hi, U' lo [C][NV]
+  static constexpr int SMU_BYTES = (DK * NV * 2 > 2 * C * NV * 2) ? DK * NV * 2 : 2 * C * NV * 2;
+  static constexpr int INV = SMU + SMU_BYTES;     // fp32 L and T of the inverse (64 x 64 each)
+  static constexpr int TOTAL = INV + 2 * C * C * 4;
+  static constexpr int TM_S = 0, TM_D1 = NV, TM_U0 = 2 * NV;
+  static constexpr int TM_WK = (NV == 128) ? TM_D1 : 3 * NV;
+  static constexpr int TM_GR = (NV == 128) ? 3 * NV : 3 * NV + DK;
+  static_assert(TM_GR + 64 <= (int)kTmemCols, "tensor memory budget");
+  // dynamic (plus 1 KB for alignment) and about 15 KB of static shared memory per CTA
+  static_assert(TOTAL + 1024 + 16 * 1024 <= 227 * 1024, "shared memory budget");
+};
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int NV>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_sc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const Args a) {
+  using Ly = ScLayout<NV>;
+  constexpr int NCB = NV / 64;  // 32-column TMEM loads per thread per NV-wide tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_qk[2], bar_k, bar_v, bar_mma, bar_gram, bar_tready, bar_drain;
+  __shared__ uint32_t s_tmem;
+  __shared__ __align__(16) float s_Y[2048];  // inverse scratch
+  // per-token factors by chunk index mod 4: r_t, 1/r_t, beta^k d, beta^v; gamma_C / gamma_m; gamma_m
+  __shared__ float s_r[4][C], s_ri[4][C], s_ws[4][C], s_bv[4][C];
+  __shared__ float s_lam[4], s_gm[4];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
+  const int T = a.T, H = a.H, dv = a.dv;
+  const int nslices = dv / NV;
+  const int bh = blockIdx.x / nslices, b = bh / H, h = bh % H;
+  const int col0 = (blockIdx.x % nslices) * NV;
+  const int nchunks = (T + C - 1) / C;
+
+  if (tid == 0) {
+    mbar_init(&bar_qk[0], 1);
+    mbar_init(&bar_qk[1], 1);
+    mbar_init(&bar_k, 1);
+    mbar_init(&bar_v, 1);
+    mbar_init(&bar_mma, 1);
+    mbar_init(&bar_gram, 1);
+    mbar_init(&bar_tready, 1);
+    mbar_init(&bar_drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
+  // rows 0..63 of the T Diag(r) and T Diag(beta^v) tiles: the 8x8 blocks above the block diagonal
+  // stay zero (the inverse never writes them); rows 64..127 of the T Diag(beta^v) tile are zero
+  for (int e = tid; e < 64 * 8; e += kThreads) {
+    const int t = e >> 3, x8 = e & 7;
+    if (x8 > (t >> 3)) {
+      *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 64)) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(sm + Ly::STQ + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  for (int i = tid; i < 64 * 128 / 16; i += kThreads)
+    reinterpret_cast<uint4*>(sm + Ly::STQ + 64 * 128)[i] = make_uint4(0, 0, 0, 0);
+  // the inverse's fp32 scratch (L, T): the blocks of T above the diagonal stay zero
+  for (int i = tid; i < 2 * C * C * 4 / 16; i += kThreads)
+    reinterpret_cast<uint4*>(sm + Ly::INV)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+
+  auto kq_buf = [&](int c) -> uint8_t* { return sm + ((c & 1) ? Ly::KQ1 : Ly::KQ0); };
+  // [K; Q] tile of chunk c (one thread)
+  auto issue_qk = [&](int c) {
+    uint64_t* bar = &bar_qk[c & 1];
+    uint8_t* kq = kq_buf(c);
+    mbar_expect_tx(bar, 2u * C * DK * 2);
+#pragma unroll
+    for (int x = 0; x < DK / 64; ++x) {
+      tma_load_4d(kq + x * 128 * 128, &tm_k, bar, 64 * x, h, c * C, b);
+      tma_load_4d(kq + x * 128 * 128 + 64 * 128, &tm_q, bar, 64 * x, h, c * C, b);
+    }
+  };
+  auto issue_k = [&](int c) {
+    mbar_expect_tx(&bar_k, (uint32_t)C * DK * 2);
+#pragma unroll
+    for (int x = 0; x < DK / 64; ++x) tma_load_4d(sm + Ly::STK + x * C * 128, &tm_k, &bar_k, 64 * x, h, c * C, b);
+  };
+  auto issue_v = [&](int c) {
+    mbar_expect_tx(&bar_v, (uint32_t)C * NV * 2);
+#pragma unroll
+    for (int x = 0; x < NV / 64; ++x)
+      tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, col0 + 64 * x, h, c * C, b);
+  };
+  // Gram [K; Q] K^T of chunk c -> TM_GR (one thread)
+  auto issue_gram = [&](int c) {
+    const uint8_t* kq = kq_buf(c);
+    const uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < DK; kk += 16) {
+      const uint64_t d = sdesc(smem_u32(kq) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+      mma_bf16(tmem + Ly::TM_GR, d, d, id, kk > 0);
+    }
+  };
+
+  bool failed = false;
+  if (warp < 8) {
+    // ======================================================= state group
+    const int ch = warp >> 2;  // column half of the TMEM tiles this warp covers
+    uint32_t ph_qk[2] = {0, 0}, ph_k = 0, ph_v = 0, ph_mma = 0, ph_tr = 0;
+    bool pend_qk[2] = {false, false}, pend_k = false, pend_v = false;
+    bool ok0 = true;  // thread 0: its own waits (the [K; Q] tiles before a Gram) succeeded
+    if (tid == 0 && nchunks > 0) {
+      issue_qk(0);
+      pend_qk[0] = true;
+      if (nchunks > 1) {
+        issue_qk(1);
+        pend_qk[1] = true;
+      }
+      issue_k(0);
+      issue_v(0);
+      pend_k = pend_v = true;
+      if (mbar_wait_bounded(&bar_qk[0], ph_qk[0], kWaitNs)) {
+        ph_qk[0] ^= 1;
+        pend_qk[0] = false;
+        tc_fence_after();
+        issue_gram(0);
+        mma_commit(&bar_gram);
+      } else {
+        ok0 = false;
+      }
+    }
+    const uint32_t id_wk = idesc_bf16(128, DK, 0, 1);
+    const uint32_t id_nv = idesc_bf16(128, NV, 0, 1);
+    const uint32_t id_state = idesc_bf16(128, NV, 1, 1);
+
+    for (int c = 0; c < nchunks; ++c) {
+      const int t0 = c * C, cur = c & 3, prev = (c + 3) & 3;
+      uint8_t* const kq = kq_buf(c);
+
+      // ---- M0: chunk c's T tiles, P and factors are ready; its v tile has landed
+      {
+        const bool ok = ok0 && mbar_wait_bounded(&bar_tready, ph_tr, kWaitNs) &&
+                        mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
+        if (group_or(kBarState, kStateThreads, !ok)) {
+          failed = true;
+          break;
+        }
+        ph_tr ^= 1;
+        ph_v ^= 1;
+        pend_v = false;
+        tc_fence_after();
+      }
+
+      // ---- M1: Wk = (T Diag r) K -> TM_WK, U0 = (T Diag beta^v) V -> TM_U0; then chunk c + 1's Gram
+      // (its completion also tells the transform group that chunk c's T tiles are no longer read)
+      if (tid == 0) {
+#pragma unroll
+        for (int kk = 0; kk < C; kk += 16) {
+          const uint64_t ad = sdesc(smem_u32(sm + Ly::TP) + kk * 2, 16, 1024);
+          const uint64_t bk = sdesc(smem_u32(kq) + kk * 128, 128 * 128, 1024);
+          mma_bf16(tmem + Ly::TM_WK, ad, bk, id_wk, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < C; kk += 16) {
+          const uint64_t ad = sdesc(smem_u32(sm + Ly::STQ) + kk * 2, 16, 1024);
+          const uint64_t bv = sdesc(smem_u32(sm + Ly::STV) + kk * 128, C * 128, 1024);
+          mma_bf16(tmem + Ly::TM_U0, ad, bv, id_nv, kk > 0);
+        }
+        mma_commit(&bar_mma);
+        if (c + 1 < nchunks) {
+          const int j = (c + 1) & 1;
+          if (mbar_wait_bounded(&bar_qk[j], ph_qk[j], kWaitNs)) {
+            ph_qk[j] ^= 1;
+            pend_qk[j] = false;
+            issue_gram(c + 1);
+            mma_commit(&bar_gram);
+          } else {
+            ok0 = false;
+          }
+        }
+      }
+      // meanwhile: S_m = Diag(lambda_{c-1} gamma_m) S -> TM_S (fp32) and the bf16 tile in SMU; rows
+      // 32 q4 .. +32, columns of half ch
+      {
+        const int k = 32 * q4 + lane;
+        const float mu = (c == 0) ? s_gm[cur] : s_lam[prev] * s_gm[cur];
+        uint32_t xr[NCB][32];  // all TMEM loads of this thread in flight at once
+        if (c == 0) {
+#pragma unroll
+          for (int cb = 0; cb < NCB; ++cb) {
+            const int col = ch * (NV / 2) + 32 * cb;
+            const float* src = a.S0 ? a.S0 + ((int64_t)bh * DK + k) * dv + col0 + col : nullptr;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 f = src ? *reinterpret_cast<const float4*>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+              xr[cb][e] = __float_as_uint(f.x), xr[cb][e + 1] = __float_as_uint(f.y);
+              xr[cb][e + 2] = __float_as_uint(f.z), xr[cb][e + 3] = __float_as_uint(f.w);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_S + ch * (NV / 2) + 32 * cb, xr[cb]);
+#pragma unroll
+          for (int cb = 0; cb < NCB; ++cb) tmem_wait_ld(xr[cb]);
+        }
+#pragma unroll
+        for (int cb = 0; cb < NCB; ++cb) {
+          const int col = ch * (NV / 2) + 32 * cb;
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(xr[cb][e]) * mu;
+          tmem_st32_issue(tmem + lane_base + Ly::TM_S + col, x);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
+                                  pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
+            *reinterpret_cast<uint4*>(sm + Ly::SMU + canon_chunk(k, col / 8 + q8, DK)) = pk;
+          }
+        }
+        tmem_wait_st();
+      }
+      {
+        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+        if (group_or(kBarState, kStateThreads, !ok)) {
+          failed = true;
+          break;
+        }
+        ph_mma ^= 1;
+        tc_fence_after();
+      }
+      if (tid == 0 && c + 1 < nchunks) {
+        issue_v(c + 1);
+        pend_v = true;
+      }
+
+      // ---- M2: Wk -> bf16 into rows 0..63 of the [K; Q] tile (K is not read again)
+      if (q4 < 2) {
+        const int t = 32 * q4 + lane;
+        uint32_t xr[DK / 64][32];
+#pragma unroll
+        for (int cb = 0; cb < DK / 64; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_WK + ch * (DK / 2) + 32 * cb, xr[cb]);
+#pragma unroll
+        for (int cb = 0; cb < DK / 64; ++cb) tmem_wait_ld(xr[cb]);
+#pragma unroll
+        for (int cb = 0; cb < DK / 64; ++cb) {
+          const int col = ch * (DK / 2) + 32 * cb;
+          const uint32_t* x = xr[cb];
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint4 pk = make_uint4(pack_bf16(__uint_as_float(x[8 * q8]), __uint_as_float(x[8 * q8 + 1])),
+                                  pack_bf16(__uint_as_float(x[8 * q8 + 2]), __uint_as_float(x[8 * q8 + 3])),
+                                  pack_bf16(__uint_as_float(x[8 * q8 + 4]), __uint_as_float(x[8 * q8 + 5])),
+                                  pack_bf16(__uint_as_float(x[8 * q8 + 6]), __uint_as_float(x[8 * q8 + 7])));
+            *reinterpret_cast<uint4*>(kq + canon_chunk(t, col / 8 + q8, 128)) = pk;
+          }
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      group_sync(kBarState, kStateThreads);
+      tc_fence_after();
+
+      // ---- M3: D1 = [Wk; Q] S_m -> TM_D1
+      if (tid == 0) {
+#pragma unroll
+        for (int kk = 0; kk < DK; kk += 16) {
+          const uint64_t ad = sdesc(smem_u32(kq) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+          const uint64_t bd = sdesc(smem_u32(sm + Ly::SMU) + kk * 128, DK * 128, 1024);
+          mma_bf16(tmem + Ly::TM_D1, ad, bd, id_nv, kk > 0);
+        }
+        mma_commit(&bar_mma);
+      }
+      {
+        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+        if (group_or(kBarState, kStateThreads, !ok)) {
+          failed = true;
+          break;
+        }
+        ph_mma ^= 1;
+        tc_fence_after();
+      }
+      // this chunk's [K; Q] buffer is free: load chunk c + 2's into it
+      if (tid == 0 && c + 2 < nchunks) {
+        issue_qk(c + 2);
+        pend_qk[c & 1] = true;
+      }
+
+      // ---- M4: U' = (beta d / r) (U0 - Wk S_m), rows 0..63 -> hi / lo tiles (S_m is dead)
+      if (q4 < 2) {
+        const int t = 32 * q4 + lane;
+        const float us = s_ws[cur][t] * s_ri[cur][t];
+#pragma unroll
+        for (int cb = 0; cb < NV / 64; ++cb) {
+          const int col = ch * (NV / 2) + 32 * cb;
+          uint32_t u0r[32], d1r[32];
+          tmem_ld32_issue(tmem + lane_base + Ly::TM_U0 + col, u0r);
+          tmem_ld32_issue(tmem + lane_base + Ly::TM_D1 + col, d1r);
+          tmem_wait_ld(u0r);
+          tmem_wait_ld(d1r);
+          float u0[32], d1[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) u0[e] = __uint_as_float(u0r[e]), d1[e] = __uint_as_float(d1r[e]);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 8 * q8 + 2 * e;
+              split_bf16(us * (u0[i] - d1[i]), us * (u0[i + 1] - d1[i + 1]), hi[e], lo[e]);
+            }
+            const uint32_t off = canon_chunk(t, col / 8 + q8, C);
+            *reinterpret_cast<uint4*>(sm + Ly::SMU + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(sm + Ly::SMU + C * NV * 2 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
+      }
+      fence_proxy_async();
+      {
+        // the raw k tile of the state update (loaded during the previous chunk)
+        const bool ok = mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
+        tc_fence_before();
+        if (group_or(kBarState, kStateThreads, !ok)) {
+          failed = true;
+          break;
+        }
+        ph_k ^= 1;
+        pend_k = false;
+        tc_fence_after();
+      }
+
+      // ---- M5: D1 rows 64..127 += P U' (O); S_acc += K^T U' (hi and lo)
+      if (tid == 0) {
+        const uint32_t pa = smem_u32(sm + Ly::TP) + (uint32_t)(c & 1) * (C * C * 2);  // rows 64..127 = P
+#pragma unroll
+        for (int kk = 0; kk < C; kk += 16) {
+          const uint64_t ad = sdesc(pa + kk * 2, 16, 1024);
+          const uint64_t bd = sdesc(smem_u32(sm + Ly::SMU) + kk * 128, C * 128, 1024);
+          mma_bf16(tmem + Ly::TM_D1, ad, bd, id_nv, 1);
+        }
+#pragma unroll
+        for (int kk = 0; kk < C; kk += 16) {
+          const uint64_t ak = sdesc(smem_u32(sm + Ly::STK) + kk * 128, C * 128, 1024);
+          const uint64_t buh = sdesc(smem_u32(sm + Ly::SMU) + kk * 128, C * 128, 1024);
+          const uint64_t bul = sdesc(smem_u32(sm + Ly::SMU + C * NV * 2) + kk * 128, C * 128, 1024);
+          mma_bf16(tmem + Ly::TM_S, ak, buh, id_state, 1);
+          mma_bf16(tmem + Ly::TM_S, ak, bul, id_state, 1);
+        }
+        mma_commit(&bar_mma);
+      }
+      {
+        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+        if (group_or(kBarState, kStateThreads, !ok)) {
+          failed = true;
+          break;
+        }
+        ph_mma ^= 1;
+        tc_fence_after();
+      }
+      if (tid == 0 && c + 1 < nchunks) {
+        issue_k(c + 1);
+        pend_k = true;
+      }
+
+      // ---- M6: o rows of chunk c = r_t (rows 64..127 of D1), warps of quadrants 2 and 3; the TMEM
+      // load is warp-collective: every lane loads, only rows of real tokens store
+      if (q4 >= 2) {
+        const int t = 32 * (q4 - 2) + lane, nc = min(C, T - t0);
+        const float os = s_r[cur][t];
+        __nv_bfloat16* orow =
+            reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0 + t) * H + h) * dv + col0;
+        uint32_t xr[NCB][32];
+#pragma unroll
+        for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_D1 + ch * (NV / 2) + 32 * cb, xr[cb]);
+#pragma unroll
+        for (int cb = 0; cb < NCB; ++cb) tmem_wait_ld(xr[cb]);
+        if (t < nc) {
+#pragma unroll
+          for (int cb = 0; cb < NCB; ++cb) {
+            const int col = ch * (NV / 2) + 32 * cb;
+            float x[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = os * __uint_as_float(xr[cb][e]);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
+                                    pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
+              *reinterpret_cast<uint4*>(orow + col + 8 * q8) = pk;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      group_sync(kBarState, kStateThreads);
+      tc_fence_after();
+    }
+
+    if (!failed && nchunks > 0) {
+      // S_T = (gamma_C / gamma_m) S_acc of the last chunk
+      const int k = 32 * q4 + lane;
+      const float lam = s_lam[(nchunks - 1) & 3];
+#pragma unroll
+      for (int cb = 0; cb < NV / 64; ++cb) {
+        const int col = ch * (NV / 2) + 32 * cb;
+        float x[32];
+        tmem_ld32(tmem + lane_base + Ly::TM_S + col, x);
+        float* dst = a.S + ((int64_t)bh * DK + k) * dv + col0 + col;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(lam * x[e], lam * x[e + 1], lam * x[e + 2], lam * x[e + 3]);
+      }
+    }
+    if (failed && tid == 0) {
+      // drain: every tensor-core op this thread issued (a commit tracks all earlier ones), then
+      // every TMA load still in flight (bounded)
+      mma_commit(&bar_drain);
+      mbar_wait_bounded(&bar_drain, 0, kWaitNs);
+      for (int j = 0; j < 2; ++j)
+        if (pend_qk[j]) mbar_wait_bounded(&bar_qk[j], ph_qk[j], kWaitNs);
+      if (pend_k) mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
+      if (pend_v) mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
+    }
+  } else {
+    // ======================================================= transform group
+    const int gt = tid - kStateThreads, gw = gt >> 5, gch = gw >> 2;  // q4 == gw & 3
+    uint32_t ph_gr = 0;
+    // Thread j < 64 (warps 8, 9) loads token j's gates (alpha, beta^k, d, beta^v) of chunk cn into
+    // registers, one chunk ahead of their use; absent gates read as 1, tokens past the end as
+    // alpha 1 and 0 for the others (no decay, no write).
+    float gx[4];
+    auto load_gates = [&](int cn, int j) {
+      const bool valid = j < T - cn * C;
+      const int64_t tok = ((int64_t)b * T + cn * C + j) * H + h;
+      gx[0] = (valid && a.alpha == DN_GATE_SCALAR) ? __ldg(a.alpha_p + tok) : 1.f;
+      gx[1] = (valid && a.beta_k == DN_GATE_SCALAR) ? __ldg(a.beta_k_p + tok) : (valid ? 1.f : 0.f);
+      gx[2] = (valid && a.key_scale == DN_GATE_SCALAR) ? __ldg(a.key_scale_p + tok) : 1.f;
+      gx[3] = (valid && a.beta_v == DN_GATE_SCALAR) ? __ldg(a.beta_v_p + tok) : (valid ? 1.f : 0.f);
+    };
+    // Decay factors of chunk cn from its gates in gx (then the next chunk's are loaded). Warp 9
+    // (tokens 32..63) forms r_j = prod_{s=32..j} alpha_s by an inclusive product scan, warp 8
+    // (tokens 0..31) 1/r_j = prod_{s=j+1..31} alpha_s by an exclusive suffix scan;
+    // gamma_m = prod_{s<32} alpha_s, gamma_C / gamma_m = prod_{s>=32} alpha_s.
+    auto token_prep = [&](int cn, int j) {
+      const int slot = cn & 3;
+      const float al = gx[0], ws = gx[1] * gx[2], bv = gx[3];
+      if (cn + 1 < nchunks) load_gates(cn + 1, j);
+      float p = al;
+      if (j >= 32) {
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, p, off);
+          if (lane >= off) p *= y;
+        }
+        s_r[slot][j] = p;
+        s_ri[slot][j] = __fdividef(1.f, p);
+        if (lane == 31) s_lam[slot] = p;
+      } else {
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_down_sync(0xffffffffu, p, off);
+          if (lane + off < 32) p *= y;
+        }
+        const float nxt = __shfl_down_sync(0xffffffffu, p, 1);
+        const float ri = lane == 31 ? 1.f : nxt;
+        s_ri[slot][j] = ri;
+        s_r[slot][j] = __fdividef(1.f, ri);
+        if (lane == 0) s_gm[slot] = p;
+      }
+      s_ws[slot][j] = ws;
+      s_bv[slot][j] = bv;
+    };
+    if (gt < 64 && nchunks > 0) load_gates(0, gt);
+
+    for (int n = 0; n < nchunks; ++n) {
+      const int cur = n & 3;
+      if (gt < 64) token_prep(n, gt);
+      // ---- X1: the Gram of chunk n has completed, and with it chunk n - 1's Wk / U0 products
+      {
+        const bool ok = mbar_wait_bounded(&bar_gram, ph_gr, kWaitNs);
+        if (group_or(kBarXform, kXformThreads, !ok)) {
+          failed = true;
+          break;
+        }
+        ph_gr ^= 1;
+        tc_fence_after();
+      }
+      // ---- X2: A (strict lower, scaled) -> fp32 L; P (lower incl., raw q.k) -> bf16 P tile of parity
+      // n & 1 (last read by chunk n - 2's O product, long complete)
+      float* sL = reinterpret_cast<float*>(sm + Ly::INV);
+      float* sT = sL + C * C;
+      if (q4 < 2) {
+        const int t = 32 * q4 + lane;
+        const float rt = s_r[cur][t];
+        float x[32];
+        tmem_ld32(tmem + lane_base + Ly::TM_GR + 32 * gch, x);
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          float y[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 32 * gch + 4 * e4 + e;
+            y[e] = (i < t) ? x[4 * e4 + e] * s_ws[cur][i] * rt * s_ri[cur][i] : 0.f;
+          }
+          *reinterpret_cast<float4*>(sL + xi(t, 32 * gch + 4 * e4)) = make_float4(y[0], y[1], y[2], y[3]);
+        }
+      } else {
+        const int t = 32 * (q4 - 2) + lane;
+        uint8_t* pt = sm + Ly::TP + (1 + (n & 1)) * (C * C * 2);
+        float x[32];
+        tmem_ld32(tmem + lane_base + Ly::TM_GR + 32 * gch, x);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = (32 * gch + 8 * q8 + e <= t) ? x[8 * q8 + e] : 0.f;
+          *reinterpret_cast<uint4*>(pt + canon_chunk(t, 4 * gch + q8, 64)) =
+              make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]));
+        }
+      }
+      tc_fence_before();
+      // ---- X3: T = (I + A)^{-1} -> T Diag(r) (TP rows 0..63) and T Diag(beta^v) (STQ rows 0..63)
+      unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt, kBarXform);
+      fence_proxy_async();
+      group_sync(kBarXform, kXformThreads);
+      if (gt == 0) mbar_arrive(&bar_tready);
+    }
+  }
+
+  if (failed && tid == 0) atomicExch(a.status, kDevTimeout);
+  if (failed && tid == kStateThreads) atomicExch(a.status, kDevTimeout);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------- host side
+template <int NV>
+cudaError_t launch_impl(const Args& a, cudaStream_t s) {
+  using Ly = ScLayout<NV>;
+  const int smem = Ly::TOTAL + 1024;
+  cudaError_t e = cudaFuncSetAttribute(chunk_sc_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mq, mk, mv;
+  if (!make_bthd_map(&mq, a.q, DK, a.H, a.T, a.B, C) || !make_bthd_map(&mk, a.k, DK, a.H, a.T, a.B, C) ||
+      !make_bthd_map(&mv, a.v, a.dv, a.H, a.T, a.B, C))
+    return cudaErrorInvalidValue;
+  chunk_sc_kernel<NV><<<a.B * a.H * (a.dv / NV), kThreads, smem, s>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_sc(const Args& a, cudaStream_t s) {
+  // few sequences: split the 128 value columns into two 64-column CTAs when that still fits in one
+  // wave (each CTA repeats the column-independent transform)
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const bool split = a.dv == 128 && (int64_t)a.B * a.H * 2 <= sms;
+  if (a.dv == 128 && !split) return launch_impl<128>(a, s);
+  return launch_impl<64>(a, s);
+}
+
+}  // namespace dn

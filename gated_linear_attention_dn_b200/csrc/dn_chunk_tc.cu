@@ -1,4 +1,6 @@
-// Tensor-core chunked prefill (bf16 io, d_k = 128, d_v in {64, 128}) for sm_100a.
+// Tensor-core chunked prefill for gates with a per-channel part (KDA channel decay, FG2-GDN+
+// vector beta, OSDN key scale d), bf16 io, d_k = 128, d_v in {64, 128}, sm_100a. (Problems whose
+// gates are all per-token scalars take the pipelined kernel in dn_chunk_sc.cu.)
 //
 // One CTA (256 threads) owns one (b, h) sequence and walks its chunks of C = 64
 // tokens in order, keeping the fp32 state in tensor memory. Per chunk, with the
@@ -18,22 +20,13 @@
 // says the DPLR update keeps (sections 2.A and 3 item 2) and whose block Gram
 // matrix and intra-block scores take the preconditioned key under OSDN (OSDN
 // page, section 2.1); the algebra is derived from the recurrence in dn.h.
-//
-// Two gate classes share the kernel:
-//  * per-token gates only (GDN: scalar alpha, beta^k, beta^v, d): every decay and
-//    write factor is a scalar per token, so they move onto the 64x64 and 64xN
-//    matrices (A_ti = (k_t.k_i) beta_i r_t / r_i, T K+ = (T Diag(r)) K,
-//    W-^T U = K^T (Diag(beta / r) U), O_t = r_t (Q S_m + P_raw U')_t) and the raw
-//    TMA tiles of q, k, v feed the tensor cores directly, with no elementwise pass;
-//  * any per-channel gate (KDA decay, FG2-GDN+ vector beta, OSDN d): the CUDA
-//    cores build K+, Q+, W- (hi/lo) and V~ (hi/lo) tiles per chunk, with all gate
-//    loads of a chunk in flight at once.
+// The CUDA cores build the K+, Q+, W- (hi/lo) and V~ (hi/lo) tiles per chunk from the raw
+// TMA tiles and the gates, with all gate loads of a chunk in flight at once.
 //
 // Precision plan (bf16 operands, fp32 accumulation everywhere): the state update
 // W-^T U is the product whose rounding reaches S_T directly, so its operands are
-// split hi + lo in bf16 (raw k is exact in bf16, so the per-token path splits
-// only U); V~ is split the same way when beta^v is a vector. All other operands
-// are single bf16.
+// split hi + lo in bf16; V~ is split the same way when beta^v is a vector. All
+// other operands are single bf16.
 //
 // Shared-memory operand tiles use the 128-byte-swizzled canonical layout (see
 // canon()); q/k/v tiles arrive by TMA (4-D tensor maps over [B, T, H, d], boxes of
@@ -42,15 +35,15 @@
 // Tensor memory (512 columns): S_acc [0, NV) | D1 [NV, 2NV) | U0 [2NV, 3NV) | scratch (Gram, Wk).
 // Every wait on an mbarrier is bounded in time; on expiry the CTA sets the status
 // word, drains what it issued (again bounded), frees its tensor memory and exits.
-#include <cudaTypedefs.h>
-
 #include "dn_common.cuh"
 #include "dn_tc_ptx.cuh"
+#include "dn_ut_inverse.cuh"
 
 namespace dn {
 namespace {
 
 using namespace tc;
+using namespace ut;
 
 constexpr int C = 64;
 constexpr int kThreads = 256;
@@ -60,7 +53,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, far above any legi
 template <int DK, int NV>
 struct Layout {
   static constexpr int STK = 0;                       // raw k  [C][DK]   (TMA)
-  static constexpr int STQ = STK + C * DK * 2;        // raw q  [C][DK]   (TMA); per-token path: T~ tile
+  static constexpr int STQ = STK + C * DK * 2;        // raw q  [C][DK]   (TMA)
   static constexpr int STV = STQ + C * DK * 2;        // raw v  [C][NV]   (TMA), V~ hi after prep
   static constexpr int VLO = STV + C * NV * 2;        // V~ lo  [C][NV]
   static constexpr int KQ = VLO + C * NV * 2;         // [K+ ; Q+] then [Wk ; Q+]   [128][DK]
@@ -78,22 +71,10 @@ struct Layout {
   static_assert(TM_SCR + (DK > 64 ? DK : 64) <= (int)kTmemCols, "tensor memory budget");
 };
 
-// Index into a 64x64 fp32 array: rows of 64, columns XOR-permuted in groups of 4
-// by (row mod 8), so float4 accesses stay aligned and column walks by
-// consecutive rows spread over the banks.
-__device__ __forceinline__ int xi(int r, int c) { return (r << 6) | (c ^ ((r & 7) << 2)); }
-
 __device__ __forceinline__ float4 f4(float x) { return make_float4(x, x, x, x); }
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
 __device__ __forceinline__ float4 rcp4(float4 a) {
   return make_float4(__fdividef(1.f, a.x), __fdividef(1.f, a.y), __fdividef(1.f, a.z), __fdividef(1.f, a.w));
-}
-
-// gate values of four consecutive channels (mode ONE -> 1, SCALAR -> broadcast)
-__device__ __forceinline__ float4 gate4(const float* g, int mode, int64_t tok, int width, int ch) {
-  if (mode == DN_GATE_ONE) return f4(1.f);
-  if (mode == DN_GATE_SCALAR) return f4(g[tok]);
-  return *reinterpret_cast<const float4*>(g + tok * width + ch);
 }
 
 // Gate values of 8 tokens (rows tok0 + i * tstride, i < 8) for 4 consecutive channels, with every
@@ -136,197 +117,19 @@ __device__ __forceinline__ void split4(float4 v, uint2& hi, uint2& lo) {
   split_bf16(v.z, v.w, hi.y, lo.y);
 }
 
-// Warp-level tensor-core product (mma.sync, TF32 inputs, fp32 accumulation), used only for the
-// small block products inside the 64x64 triangular inverse; T is rounded to bf16 afterwards, so
-// TF32 (10-bit mantissa) operands here add an error well below that rounding. Fragment layouts
-// of m16n8k8 row.col (g = lane / 4, t = lane % 4): A 16x8: (g, t) (g+8, t) (g, t+4) (g+8, t+4);
-// B 8x8: (t, g) (t+4, g); C 16x8: (g, 2t) (g, 2t+1) (g+8, 2t) (g+8, 2t+1).
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-
-__device__ __forceinline__ void mma_tf32(float* d, const uint32_t* a, const uint32_t* b) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-// d[16x8] += X[16 x K] * Y[K x 8] for one warp; X(i, k), Y(k, n) fetch elements.
-template <int K, class FX, class FY>
-__device__ __forceinline__ void warp_mm(float* d, FX X, FY Y, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int k = 0; k < K; k += 8) {
-    const uint32_t av[4] = {to_tf32(X(g, k + t)), to_tf32(X(g + 8, k + t)), to_tf32(X(g, k + t + 4)),
-                            to_tf32(X(g + 8, k + t + 4))};
-    const uint32_t bv[2] = {to_tf32(Y(k + t, g)), to_tf32(Y(k + t + 4, g))};
-    mma_tf32(d, av, bv);
-  }
-}
-
-// writes the 16x8 accumulator fragment as column pairs through W(i, n, v_n, v_n+1)
-template <class FW>
-__device__ __forceinline__ void warp_store2(const float* d, FW W, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  W(g, 2 * t, d[0], d[1]);
-  W(g + 8, 2 * t, d[2], d[3]);
-}
-
-// writes the 16x8 accumulator fragment through W(i, n, value)
-template <class FW>
-__device__ __forceinline__ void warp_store(const float* d, FW W, int lane) {
-  const int g = lane >> 2, t = lane & 3;
-  W(g, 2 * t, d[0]);
-  W(g, 2 * t + 1, d[1]);
-  W(g + 8, 2 * t, d[2]);
-  W(g + 8, 2 * t + 1, d[3]);
-}
-
-// T = (I + L)^{-1} for the 64x64 strictly lower L in sL (zeros on and above the diagonal).
-// Blocking by doubling: the eight 8x8 diagonal blocks by forward substitution (one column per
-// thread, chains of at most seven steps); then three merge levels with warp mma.sync, each using
-// [[A, 0], [C, B]]^{-1} = [[A^-1, 0], [-B^-1 C A^-1, B^-1]]:
-//   8 -> 16 (warps 0..3), 16 -> 32 (warps 0..1), 32 -> 64 (all 8 warps).
-// fp32 blocks that later levels read are kept in sT; every element of the lower triangle is also
-// written as bf16 straight into rows 0..63 of the 128-row tile tp (scaled by column factor
-// cs_c[i] when SC) and, when SC, T Diag(cs_v) into tile tt. Elements above the 8x8 block diagonal
-// are not written (their zeros are set once by the caller). scr: 2048 floats of scratch.
-// Not inlined: it gets its own register budget. All 256 threads call it.
-template <bool SC>
-__device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, float* scr, uint8_t* tp, uint8_t* tt,
-                                                const float* cs_c, const float* cs_v, int tid) {
-  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
-  auto emit1 = [&](int t, int i, float v) {
-    const uint32_t off = canon(t, i, 128);
-    *reinterpret_cast<__nv_bfloat16*>(tp + off) = __float2bfloat16_rn(SC ? v * cs_c[i] : v);
-    if (SC) *reinterpret_cast<__nv_bfloat16*>(tt + off) = __float2bfloat16_rn(v * cs_v[i]);
-  };
-  auto emit2 = [&](int t, int i, float v0, float v1) {  // columns i, i + 1 (i even)
-    const uint32_t off = canon(t, i, 128);
-    *reinterpret_cast<uint32_t*>(tp + off) = pack_bf16(SC ? v0 * cs_c[i] : v0, SC ? v1 * cs_c[i + 1] : v1);
-    if (SC) *reinterpret_cast<uint32_t*>(tt + off) = pack_bf16(v0 * cs_v[i], v1 * cs_v[i + 1]);
-  };
-  if (tid < 64) {
-    const int base = 8 * (tid >> 3), j = tid & 7;
-    float x[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      float s0 = (r == j) ? 1.f : 0.f, s1 = 0.f;
-#pragma unroll
-      for (int i = 0; i < r; ++i) {
-        const float l = sL[xi(base + r, base + i)];
-        if (i & 1)
-          s1 = fmaf(-l, x[i], s1);
-        else
-          s0 = fmaf(-l, x[i], s0);
-      }
-      x[r] = s0 + s1;
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      sT[xi(base + r, base + j)] = x[r];
-      emit1(base + r, base + j, x[r]);
-    }
-  } else {
-    // zero, inside each 32x32 diagonal block, the 8x8 and 16x16 blocks above the diagonal that the
-    // merge levels read: rows 16p..+8 x cols 16p+8..+8 (p < 4); rows 32q..+16 x cols 32q+16..+16 (q < 2)
-    for (int e = tid - 64; e < 768; e += 192) {
-      if (e < 256) {
-        const int p = e >> 6, r = (e >> 3) & 7, cc = e & 7;
-        sT[xi(16 * p + r, 16 * p + 8 + cc)] = 0.f;
-      } else {
-        const int e2 = e - 256, q = e2 >> 8, r = (e2 >> 4) & 15, cc = e2 & 15;
-        sT[xi(32 * q + r, 32 * q + 16 + cc)] = 0.f;
-      }
-    }
-  }
-  __syncthreads();
-  // 8 -> 16: T_ba = -T_bb (L_ba T_aa) in each 16x16 diagonal block (rows 8..15 of the 16-row
-  // mma operands repeat rows 0..7 and their results are ignored)
-  if (warp < 4) {
-    const int a0 = 16 * warp, b0 = a0 + 8;
-    float* Y = scr + warp * 96;  // 8 x 12 (padded)
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    warp_mm<8>(d, [&](int i, int k) { return sL[xi(b0 + (i & 7), a0 + k)]; },
-               [&](int k, int n) { return sT[xi(a0 + k, a0 + n)]; }, lane);
-    Y[g * 12 + 2 * t4] = d[0];
-    Y[g * 12 + 2 * t4 + 1] = d[1];
-    __syncwarp();
-    float e[4] = {0.f, 0.f, 0.f, 0.f};
-    warp_mm<8>(e, [&](int i, int k) { return sT[xi(b0 + (i & 7), b0 + k)]; },
-               [&](int k, int n) { return Y[k * 12 + n]; }, lane);
-    sT[xi(b0 + g, a0 + 2 * t4)] = -e[0];
-    sT[xi(b0 + g, a0 + 2 * t4 + 1)] = -e[1];
-    emit2(b0 + g, a0 + 2 * t4, -e[0], -e[1]);
-  }
-  __syncthreads();
-  // 16 -> 32: T_{i,i-1} = -T_ii (L_{i,i-1} T_{i-1,i-1}) for (i, i-1) = (1, 0), (3, 2); warp w < 4
-  // owns pair w / 2 and the 8-column tile w % 2 (a column tile of the result needs only the
-  // same column tile of L T)
-  if (warp < 4) {
-    const int bi = 1 + 2 * (warp >> 1), bk = bi - 1, nt = warp & 1;
-    float* Y = scr + 1152 + warp * 192;  // 16 x 12 (padded) dense scratch of this warp
-    {
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      warp_mm<16>(d, [&](int i, int k) { return sL[xi(16 * bi + i, 16 * bk + k)]; },
-                  [&](int k, int n) { return sT[xi(16 * bk + k, 16 * bk + 8 * nt + n)]; }, lane);
-      warp_store(d, [&](int i, int n, float v) { Y[i * 12 + n] = v; }, lane);
-    }
-    __syncwarp();
-    {
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      warp_mm<16>(d, [&](int i, int k) { return sT[xi(16 * bi + i, 16 * bi + k)]; },
-                  [&](int k, int n) { return Y[k * 12 + n]; }, lane);
-      warp_store2(d, [&](int i, int n, float v0, float v1) {
-        sT[xi(16 * bi + i, 16 * bk + 8 * nt + n)] = -v0;
-        sT[xi(16 * bi + i, 16 * bk + 8 * nt + n + 1)] = -v1;
-        emit2(16 * bi + i, 16 * bk + 8 * nt + n, -v0, -v1);
-      }, lane);
-    }
-  }
-  __syncthreads();
-  // 32 -> 64: X = L21 T1, then T21 = -T2 X; warp w owns rows 16 (w / 4) .. +16, columns 8 (w % 4) .. +8
-  float* X = scr;  // 32 x 36 (padded) dense
-  const int mt = warp >> 2, nt = warp & 3;
-  {
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    warp_mm<32>(d, [&](int i, int k) { return sL[xi(32 + 16 * mt + i, k)]; },
-                [&](int k, int n) { return sT[xi(k, 8 * nt + n)]; }, lane);
-    warp_store(d, [&](int i, int n, float v) { X[(16 * mt + i) * 36 + 8 * nt + n] = v; }, lane);
-  }
-  __syncthreads();
-  {
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    warp_mm<32>(d, [&](int i, int k) { return sT[xi(32 + 16 * mt + i, 32 + k)]; },
-                [&](int k, int n) { return X[k * 36 + 8 * nt + n]; }, lane);
-    warp_store2(d, [&](int i, int n, float v0, float v1) { emit2(32 + 16 * mt + i, 8 * nt + n, -v0, -v1); },
-                lane);
-  }
-  __syncthreads();
-}
-
-template <int DK, int NV, bool SC>
+template <int DK, int NV>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Args a) {
   using Ly = Layout<DK, NV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bar_qk, bar_k, bar_v, bar_mma, bar_gram;
-  __shared__ int s_gram_ready;  // per-token path: the next chunk's Gram MMA was issued early
+  __shared__ __align__(8) uint64_t bar_qk, bar_v, bar_mma;
   __shared__ uint32_t s_tmem;
-  __shared__ __align__(16) float s_lam[2][DK];   // gamma_C / gamma_m per key channel (per-channel path)
+  __shared__ __align__(16) float s_lam[2][DK];   // gamma_C / gamma_m per key channel
   __shared__ __align__(16) float s_gm[DK];       // gamma_m per key channel
-  __shared__ __align__(16) float s_grp[8][DK];   // per-8-token decay products (per-channel path)
+  __shared__ __align__(16) float s_grp[8][DK];   // per-8-token decay products
   __shared__ __align__(16) float s_Y[2048];
-  // per-token path, by chunk parity: r_t, 1/r_t, beta^k d, beta^v; gamma_C / gamma_m; gamma_m
-  __shared__ float s_r[2][C], s_ri[2][C], s_ws[2][C], s_bv[2][C];
-  __shared__ float s_lam1[2], s_gm1[2];
-  __shared__ float s_nx[2][4][C];  // per-token path: gates of the next chunk (alpha, beta^k, d, beta^v)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, ch = warp >> 2;
@@ -339,27 +142,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&bar_qk, 1);
-    mbar_init(&bar_k, 1);
     mbar_init(&bar_v, 1);
     mbar_init(&bar_mma, 1);
-    mbar_init(&bar_gram, 1);
-    s_gram_ready = 0;
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
-  // rows 0..63 of the [T; P] tile (and of the T~ tile): the 8x8 blocks above the block diagonal
-  // of T are zero and nothing else writes them; set them once
+  // rows 0..63 of the [T; P] tile: the 8x8 blocks above the block diagonal of T are zero and
+  // nothing else writes them; set them once
   for (int e = tid; e < 64 * 8; e += kThreads) {
     const int t = e >> 3, x8 = e & 7;
-    if (x8 > (t >> 3)) {
-      *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
-      if (SC) *reinterpret_cast<uint4*>(sm + Ly::STQ + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
-    }
-  }
-  if (SC) {
-    // rows 64..127 of the T~ tile are never meaningful; keep them finite
-    for (int i = tid; i < 64 * 128 / 16; i += kThreads)
-      reinterpret_cast<uint4*>(sm + Ly::STQ + 64 * 128)[i] = make_uint4(0, 0, 0, 0);
+    if (x8 > (t >> 3)) *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async();
   tc_fence_before();
@@ -368,30 +160,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
 
-  // Operand buffers. Per-channel path: raw k, q staging (STK, STQ) feeds the prep,
-  // which writes [K+; Q+] into KQ. Per-token path: the raw [K; Q] tile (Gram operand,
-  // later [Wk; Q]) is double-buffered in KQ and in the W- region it does not use, so
-  // the next chunk's tile loads during this chunk; a separate raw k tile (STK) serves
-  // the state update at the end of the chunk and reloads after it.
-  auto kq_buf = [&](int c) -> uint8_t* { return (SC && (c & 1)) ? sm + Ly::WHI : sm + Ly::KQ; };
+  // Raw k, q staging (STK, STQ) by TMA feeds the prep, which writes [K+; Q+] into KQ.
+  uint8_t* const kq = sm + Ly::KQ;
   auto issue_qk = [&](int c) {
     mbar_expect_tx(&bar_qk, 2u * C * DK * 2);
 #pragma unroll
     for (int x = 0; x < DK / 64; ++x) {
-      if (SC) {
-        uint8_t* kq = kq_buf(c);
-        tma_load_4d(kq + x * 128 * 128, &tm_k, &bar_qk, 64 * x, h, c * C, b);
-        tma_load_4d(kq + x * 128 * 128 + 64 * 128, &tm_q, &bar_qk, 64 * x, h, c * C, b);
-      } else {
-        tma_load_4d(sm + Ly::STK + x * C * 128, &tm_k, &bar_qk, 64 * x, h, c * C, b);
-        tma_load_4d(sm + Ly::STQ + x * C * 128, &tm_q, &bar_qk, 64 * x, h, c * C, b);
-      }
+      tma_load_4d(sm + Ly::STK + x * C * 128, &tm_k, &bar_qk, 64 * x, h, c * C, b);
+      tma_load_4d(sm + Ly::STQ + x * C * 128, &tm_q, &bar_qk, 64 * x, h, c * C, b);
     }
-  };
-  auto issue_k = [&](int c) {  // per-token path only
-    mbar_expect_tx(&bar_k, (uint32_t)C * DK * 2);
-#pragma unroll
-    for (int x = 0; x < DK / 64; ++x) tma_load_4d(sm + Ly::STK + x * C * 128, &tm_k, &bar_k, 64 * x, h, c * C, b);
   };
   auto issue_v = [&](int c) {
     mbar_expect_tx(&bar_v, (uint32_t)C * NV * 2);
@@ -400,88 +177,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, col0 + 64 * x, h, c * C, b);
   };
 
-  uint32_t ph_qk = 0, ph_k = 0, ph_v = 0, ph_mma = 0, ph_gram = 0;
-  bool qk_pending = false, k_pending = false, v_pending = false, mma_pending = false, gram_pending = false;
+  uint32_t ph_qk = 0, ph_v = 0, ph_mma = 0;
+  bool qk_pending = false, v_pending = false, mma_pending = false;
   bool failed = false;
   if (tid == 0 && nchunks > 0) {
     issue_qk(0);
-    if (SC) issue_k(0);
     issue_v(0);
   }
   if (nchunks > 0) qk_pending = v_pending = true;
-  if (SC && nchunks > 0) k_pending = true;
 
   const uint32_t id_gram = idesc_bf16(128, 64, 0, 0);
   const uint32_t id_wk = idesc_bf16(128, DK, 0, 1);
   const uint32_t id_nv = idesc_bf16(128, NV, 0, 1);
   const uint32_t id_state = idesc_bf16(128, NV, 1, 1);
-  const bool bv_split = !SC && a.beta_v != DN_GATE_ONE;
+  const bool bv_split = a.beta_v != DN_GATE_ONE;
   float* sL = reinterpret_cast<float*>(sm + Ly::INV);
   float* sT = sL + C * C;
-
-  // per-token path: thread j < 64 copies token j's gates of the next chunk into shared memory
-  // one chunk ahead with cp.async (absent gates and tokens past the end are written directly)
-  auto prefetch_token_gates = [&](int cn, int j) {
-    const int t0n = cn * C;
-    float* dst = &s_nx[cn & 1][0][j];
-    const float* src[4] = {a.alpha_p, a.beta_k_p, a.key_scale_p, a.beta_v_p};
-    const int mode[4] = {a.alpha, a.beta_k, a.key_scale, a.beta_v};
-    const bool valid = j < T - t0n;
-    const int64_t tok = ((int64_t)b * T + t0n + j) * H + h;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      if (valid && mode[g] == DN_GATE_SCALAR)
-        cp_async_4(dst + g * C, src[g] + tok);
-      else
-        dst[g * C] = valid ? 1.f : (g == 0 ? 1.f : 0.f);
-    }
-    cp_async_commit();
-  };
-  // per-token path, threads 0..63 (token j): decay factors of chunk cn from its prefetched gates;
-  // warp 1 (tokens 32..63) forms r_j = prod_{s=32..j} alpha_s by an inclusive product scan,
-  // warp 0 (tokens 0..31) forms 1/r_j = prod_{s=j+1..31} alpha_s by an exclusive suffix scan
-  auto token_prep = [&](int cn, int j, bool upper) {
-    const int par = cn & 1;
-    cp_async_wait_all();
-    const float al = s_nx[par][0][j], ws = s_nx[par][1][j] * s_nx[par][2][j], bv = s_nx[par][3][j];
-    if (cn + 1 < nchunks) prefetch_token_gates(cn + 1, j);
-    float p = al;
-    if (upper) {
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, p, off);
-        if (lane >= off) p *= y;
-      }
-      s_r[par][j] = p;
-      s_ri[par][j] = __fdividef(1.f, p);
-      if (lane == 31) s_lam1[par] = p;
-    } else {
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y = __shfl_down_sync(0xffffffffu, p, off);
-        if (lane + off < 32) p *= y;
-      }
-      const float nxt = __shfl_down_sync(0xffffffffu, p, 1);
-      const float ri = lane == 31 ? 1.f : nxt;
-      s_ri[par][j] = ri;
-      s_r[par][j] = __fdividef(1.f, ri);
-      if (lane == 0) s_gm1[par] = p;
-    }
-    s_ws[par][j] = ws;
-    s_bv[par][j] = bv;
-  };
-  if (SC && tid < 64 && nchunks > 0) {
-    prefetch_token_gates(0, tid);
-    token_prep(0, tid, warp == 1);
-  }
 
   // S_m = Diag(lambda_prev * gamma_m) S for rows 32 q4 .. +32, columns of half ch: the state in
   // chunk c's frame, in TMEM (fp32) and as the bf16 operand tile
   auto state_to_frame = [&](int c) {
     const int cur = c & 1, prev = cur ^ 1;
     const int k = 32 * q4 + lane;
-    const float mu = SC ? ((c == 0) ? s_gm1[cur] : s_lam1[prev] * s_gm1[cur])
-                        : ((c == 0) ? s_gm[k] : s_lam[prev][k] * s_gm[k]);
+    const float mu = (c == 0) ? s_gm[k] : s_lam[prev][k] * s_gm[k];
 #pragma unroll
     for (int cb = 0; cb < NV / 64; ++cb) {
       const int col = ch * (NV / 2) + 32 * cb;
@@ -516,7 +234,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // TMEM load is warp-collective: every lane loads, only rows of real tokens store
   auto store_o = [&](int c) {
     const int t = 32 * (q4 - 2) + lane, t0c = c * C, nc = min(C, T - t0c);
-    const float os = SC ? s_r[c & 1][t] : 1.f;
     __nv_bfloat16* orow =
         reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0c + t) * H + h) * dv + col0;
 #pragma unroll
@@ -527,25 +244,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t < nc) {
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
-          uint4 pk = make_uint4(pack_bf16(os * x[8 * q8], os * x[8 * q8 + 1]),
-                                pack_bf16(os * x[8 * q8 + 2], os * x[8 * q8 + 3]),
-                                pack_bf16(os * x[8 * q8 + 4], os * x[8 * q8 + 5]),
-                                pack_bf16(os * x[8 * q8 + 6], os * x[8 * q8 + 7]));
+          uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
+                                pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
           *reinterpret_cast<uint4*>(orow + col + 8 * q8) = pk;
         }
       }
     }
   };
 
-  // Gram [K+; Q+] W-^T (per-token path: [K; Q] K^T) of chunk c -> TMEM scratch; thread 0 only
-  auto issue_gram = [&](int c) {
-    uint8_t* kqc = kq_buf(c);
-    const uint8_t* gb = SC ? kqc : sm + Ly::WHI;
-    const uint32_t gb_blk = SC ? 128 * 128 : C * 128;
+  // Gram [K+; Q+] W-^T of the current chunk -> TMEM scratch; thread 0 only
+  auto issue_gram = [&]() {
 #pragma unroll
     for (int kk = 0; kk < DK; kk += 16) {
-      const uint64_t ad = sdesc(smem_u32(kqc) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
-      const uint64_t bd = sdesc(smem_u32(gb) + (kk >> 6) * gb_blk + (kk & 63) * 2, 16, 1024);
+      const uint64_t ad = sdesc(smem_u32(kq) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+      const uint64_t bd = sdesc(smem_u32(sm + Ly::WHI) + (kk >> 6) * (C * 128) + (kk & 63) * 2, 16, 1024);
       mma_bf16(tmem + Ly::TM_SCR, ad, bd, id_gram, kk > 0);
     }
   };
@@ -553,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int c = 0; c < nchunks; ++c) {
     const int t0 = c * C;
     const int n = min(C, T - t0);
-    const int cur = c & 1, prev = cur ^ 1;
+    const int cur = c & 1;
 
     // ---- P0: this chunk's q, k, v have landed
     {
@@ -566,15 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ph_v ^= 1;
       qk_pending = v_pending = false;
     }
-    uint8_t* const kq = kq_buf(c);
-    // per-token path: the other [K; Q] buffer was last read by the previous chunk's D1 MMA
-    if (SC && tid == 0 && c + 1 < nchunks) issue_qk(c + 1);
-    if (SC && c + 1 < nchunks) qk_pending = true;
 
-    // ---- P1: decay factors (and, per-channel path, the operand tiles)
-    if (SC) {
-      // per-token factors of this chunk were computed during the previous chunk (token_prep)
-    } else {
+    // ---- P1: decay factors and the operand tiles
+    {
       // per-channel path: thread (g4, tg) owns channels 4g4..4g4+3 of tokens 8tg..8tg+7
       const int g4 = lane, tg = warp, cb0 = 4 * g4;
       float4 al[8], ws[8], dd[8];
@@ -673,28 +379,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async();
     __syncthreads();
 
-    // ---- P2: Gram [K+; Q+] W-^T (per-token path: [K; Q] K^T) -> scratch
-    const bool gram_early = SC && s_gram_ready;  // uniform: written before the last barrier
-    if (gram_early) {
-      bool ok = mbar_wait_bounded(&bar_gram, ph_gram, kWaitNs);
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-      ph_gram ^= 1;
-      gram_pending = false;
-      tc_fence_after();
-    } else {
+    // ---- P2: Gram [K+; Q+] W-^T -> scratch
+    {
       if (tid == 0) {
-        // per-channel path: the raw q, k staging was consumed by the prep; prefetch the next chunk
-        if (!SC && c + 1 < nchunks) {
+        // the raw q, k staging was consumed by the prep; prefetch the next chunk's
+        if (c + 1 < nchunks) {
           fence_proxy_async();
           issue_qk(c + 1);
         }
-        issue_gram(c);
+        issue_gram();
         mma_commit(&bar_mma);
       }
-      if (!SC && c + 1 < nchunks) qk_pending = true;
+      if (c + 1 < nchunks) qk_pending = true;
       mma_pending = true;
       bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
       if (__syncthreads_or(!ok)) {
@@ -713,16 +409,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = 32 * ch;
       if (q4 < 2) {
         const int t = 32 * q4 + lane;
-        const float rt = SC ? s_r[cur][t] : 1.f;
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           float y[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = i0 + 4 * e4 + e;
-            float v = x[4 * e4 + e];
-            if (SC) v *= s_ws[cur][i] * rt * s_ri[cur][i];
-            y[e] = (i < t) ? v : 0.f;
+            y[e] = (i < t) ? x[4 * e4 + e] : 0.f;
           }
           sts4(sL, xi(t, i0 + 4 * e4), make_float4(y[0], y[1], y[2], y[3]));
         }
@@ -742,15 +435,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    unit_lower_inverse<SC>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], tid);
+    unit_lower_inverse<false, 8>(sL, sT, s_Y, sm + Ly::TP, nullptr, nullptr, nullptr, tid, 0);
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    // ---- P4: Wk = [T; P] K+ -> scratch;  U0 = [T; P] V~ (per-token path: T~ V) -> U0
+    // ---- P4: Wk = [T; P] K+ -> scratch;  U0 = [T; P] V~ -> U0
     if (tid == 0) {
-      const uint8_t* ta = SC ? sm + Ly::STQ : sm + Ly::TP;
 #pragma unroll
       for (int kk = 0; kk < C; kk += 16) {
         const uint64_t ad = sdesc(smem_u32(sm + Ly::TP) + kk * 2, 16, 1024);
@@ -759,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int kk = 0; kk < C; kk += 16) {
-        const uint64_t ad = sdesc(smem_u32(ta) + kk * 2, 16, 1024);
+        const uint64_t ad = sdesc(smem_u32(sm + Ly::TP) + kk * 2, 16, 1024);
         const uint64_t bv = sdesc(smem_u32(sm + Ly::STV) + kk * 128, C * 128, 1024);
         mma_bf16(tmem + Ly::TM_U0, ad, bv, id_nv, kk > 0);
       }
@@ -776,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_pending = true;
     // while those MMAs run: the previous chunk's outputs (D1 rows 64..127) and the state in this
     // chunk's frame (S_acc columns; no overlap with the TMEM the MMAs write)
-    if (!SC && c > 0 && q4 >= 2) store_o(c - 1);
+    if (c > 0 && q4 >= 2) store_o(c - 1);
     state_to_frame(c);
     {
       bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
@@ -837,12 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
     }
 
-    // ---- P7: U = U0 - Wk S_m (per-token path: U' = beta_t / r_t * U) -> hi / lo tiles
-    // (per-token path: warps 2, 3 meanwhile compute the next chunk's decay factors)
-    if (SC && (warp == 2 || warp == 3) && c + 1 < nchunks) token_prep(c + 1, tid - 64, warp == 3);
+    // ---- P7: U = U0 - Wk S_m -> hi / lo tiles
     if (q4 < 2) {
       const int t = 32 * q4 + lane;
-      const float us = SC ? s_ws[cur][t] * s_ri[cur][t] : 1.f;
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {
         const int col = ch * (NV / 2) + 32 * cb;
@@ -855,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = 8 * q8 + 2 * e;
-            split_bf16(us * (u0[i] - d1[i]), us * (u0[i + 1] - d1[i + 1]), hi[e], lo[e]);
+            split_bf16(u0[i] - d1[i], u0[i + 1] - d1[i + 1], hi[e], lo[e]);
           }
           const uint32_t off = canon_chunk(t, col / 8 + q8, C);
           *reinterpret_cast<uint4*>(sm + Ly::UHI + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -869,15 +558,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     // ---- P8: O = Q+ S_m + P U (rows 64..127 of D1); S_acc += W-^T U (split)
-    if (SC) {
-      bool ok = mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-      ph_k ^= 1;
-      k_pending = false;
-    }
     if (tid == 0) {
 #pragma unroll
       for (int kk = 0; kk < C; kk += 16) {
@@ -889,28 +569,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kk = 0; kk < C; kk += 16) {
         const uint64_t buh = sdesc(smem_u32(sm + Ly::UHI) + kk * 128, C * 128, 1024);
         const uint64_t bul = sdesc(smem_u32(sm + Ly::ULO) + kk * 128, C * 128, 1024);
-        if (SC) {
-          const uint64_t ak = sdesc(smem_u32(sm + Ly::STK) + kk * 128, C * 128, 1024);
-          mma_bf16(tmem + Ly::TM_S, ak, buh, id_state, 1);
-          mma_bf16(tmem + Ly::TM_S, ak, bul, id_state, 1);
-        } else {
-          const uint64_t awh = sdesc(smem_u32(sm + Ly::WHI) + kk * 128, C * 128, 1024);
-          const uint64_t awl = sdesc(smem_u32(sm + Ly::WLO) + kk * 128, C * 128, 1024);
-          mma_bf16(tmem + Ly::TM_S, awh, buh, id_state, 1);
-          mma_bf16(tmem + Ly::TM_S, awh, bul, id_state, 1);
-          mma_bf16(tmem + Ly::TM_S, awl, buh, id_state, 1);
-        }
+        const uint64_t awh = sdesc(smem_u32(sm + Ly::WHI) + kk * 128, C * 128, 1024);
+        const uint64_t awl = sdesc(smem_u32(sm + Ly::WLO) + kk * 128, C * 128, 1024);
+        mma_bf16(tmem + Ly::TM_S, awh, buh, id_state, 1);
+        mma_bf16(tmem + Ly::TM_S, awh, bul, id_state, 1);
+        mma_bf16(tmem + Ly::TM_S, awl, buh, id_state, 1);
       }
       mma_commit(&bar_mma);
-      // per-token path: the next chunk's [K; Q] tile has its own buffer; once it has landed, its
-      // Gram can follow these MMAs on the tensor core right away
-      int ready = 0;
-      if (SC && c + 1 < nchunks && mbar_wait_bounded(&bar_qk, ph_qk, kWaitNs)) {
-        issue_gram(c + 1);
-        mma_commit(&bar_gram);
-        ready = 1;
-      }
-      s_gram_ready = ready;
     }
     mma_pending = true;
     {
@@ -923,27 +588,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_pending = false;
       tc_fence_after();
     }
-    if (SC && s_gram_ready) gram_pending = true;
-    // per-token path: the raw k tile of the state update is free now: load the next chunk's
-    if (SC && tid == 0 && c + 1 < nchunks) {
-      fence_proxy_async();
-      issue_k(c + 1);
-    }
-    if (SC && c + 1 < nchunks) k_pending = true;
-    // per-token path: this chunk's outputs, while the next chunk's Gram runs
-    if (SC && q4 >= 2) store_o(c);
 
-    // ---- P9: (this chunk's outputs are stored during the next chunk's inverse, or after the loop)
+    // ---- P9: (this chunk's outputs are stored during the next chunk's P4 products, or after the loop)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
   }
 
   if (!failed && nchunks > 0) {
-    if (!SC && q4 >= 2) store_o(nchunks - 1);
+    if (q4 >= 2) store_o(nchunks - 1);
     // S_T = Diag(gamma_C / gamma_m) S_acc of the last chunk
     const int k = 32 * q4 + lane;
-    const float lam = SC ? s_lam1[(nchunks - 1) & 1] : s_lam[(nchunks - 1) & 1][k];
+    const float lam = s_lam[(nchunks - 1) & 1][k];
 #pragma unroll
     for (int cb = 0; cb < NV / 64; ++cb) {
       const int col = ch * (NV / 2) + 32 * cb;
@@ -958,10 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (failed) {
     // drain whatever this CTA still has in flight (bounded), then report
     if (qk_pending) mbar_wait_bounded(&bar_qk, ph_qk, kWaitNs);
-    if (k_pending) mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
     if (v_pending) mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
     if (mma_pending) mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
-    if (gram_pending) mbar_wait_bounded(&bar_gram, ph_gram, kWaitNs);
     if (tid == 0) atomicExch(a.status, kDevTimeout);
   }
   tc_fence_before();
@@ -971,45 +625,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-bool get_encode() {
-  if (g_encode) return true;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-      q != cudaDriverEntryPointSuccess || !fn)
-    return false;
-  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  return true;
-}
-
-// 4-D map over a [B, T, H, d] bf16 tensor; box = 64 channels x 1 head x 64 tokens x 1 batch.
-bool make_map(CUtensorMap* m, const void* base, int d, int H, int T, int B) {
-  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-template <int DK, int NV, bool SC>
+template <int DK, int NV>
 cudaError_t launch_impl(const Args& a, cudaStream_t s) {
   using Ly = Layout<DK, NV>;
   const int smem = Ly::TOTAL + 1024;
   // per call: the attribute is per device, and the call is cheap next to the kernel
   cudaError_t e =
-      cudaFuncSetAttribute(chunk_tc_kernel<DK, NV, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      cudaFuncSetAttribute(chunk_tc_kernel<DK, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   CUtensorMap mq, mk, mv;
-  if (!get_encode()) return cudaErrorNotSupported;
-  if (!make_map(&mq, a.q, DK, a.H, a.T, a.B) || !make_map(&mk, a.k, DK, a.H, a.T, a.B) ||
-      !make_map(&mv, a.v, a.dv, a.H, a.T, a.B))
+  if (!make_bthd_map(&mq, a.q, DK, a.H, a.T, a.B, C) || !make_bthd_map(&mk, a.k, DK, a.H, a.T, a.B, C) ||
+      !make_bthd_map(&mv, a.v, a.dv, a.H, a.T, a.B, C))
     return cudaErrorInvalidValue;
-  chunk_tc_kernel<DK, NV, SC><<<a.B * a.H * (a.dv / NV), kThreads, smem, s>>>(mq, mk, mv, a);
+  chunk_tc_kernel<DK, NV><<<a.B * a.H * (a.dv / NV), kThreads, smem, s>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -1020,16 +648,17 @@ bool chunk_tc_supported(const Args& a) {
 }
 
 cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s) {
-  // per-token gates only -> the raw-tile path
+  // per-token gates only -> the pipelined raw-tile kernel (dn_chunk_sc.cu)
   const bool sc = a.alpha != DN_GATE_CHANNEL && a.beta_k != DN_GATE_CHANNEL && a.beta_v != DN_GATE_CHANNEL &&
                   a.key_scale != DN_GATE_CHANNEL;
+  if (sc) return launch_chunk_sc(a, s);
   // few sequences: split the 128 value columns into two 64-column CTAs when that still fits in one
   // wave (each CTA repeats the column-independent prep, Gram and inverse)
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const bool split = a.dv == 128 && (int64_t)a.B * a.H * 2 <= sms;
-  if (a.dv == 128 && !split) return sc ? launch_impl<128, 128, true>(a, s) : launch_impl<128, 128, false>(a, s);
-  return sc ? launch_impl<128, 64, true>(a, s) : launch_impl<128, 64, false>(a, s);
+  if (a.dv == 128 && !split) return launch_impl<128, 128>(a, s);
+  return launch_impl<128, 64>(a, s);
 }
 
 }  // namespace dn

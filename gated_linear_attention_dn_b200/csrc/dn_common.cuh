@@ -2,6 +2,7 @@
 // shim (dn_abi.cu) and the kernels (one .cu file per kernel family).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -35,8 +36,13 @@ struct Args {
 cudaError_t launch_decode(const Args& a, cudaStream_t s);
 cudaError_t launch_seq_fwd(const Args& a, cudaStream_t s);
 cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s);
-// Largest dynamic shared memory the tensor-core chunk kernel asks for (for validation).
+// per-token gates only (called by launch_chunk_tc)
+cudaError_t launch_chunk_sc(const Args& a, cudaStream_t s);
+// Whether the tensor-core chunk kernels take this problem (else the sequential kernel does).
 bool chunk_tc_supported(const Args& a);
+// TMA tensor map over a [B, T, H, d] bf16 tensor, 128-byte swizzle, box of 64 channels x 1 head x
+// box_tokens tokens x 1 sequence, zero fill past the end (dn_tma.cu). False if encoding fails.
+bool make_bthd_map(CUtensorMap* m, const void* base, int d, int H, int T, int B, int box_tokens);
 
 // ---------------------------------------------------------------- device helpers
 __device__ __forceinline__ float io_load(const void* p, int64_t i, int bf16) {
