@@ -73,14 +73,20 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+# sources each timed kernel is built from (its recorded DRAM traffic is void once any changes)
+KERNEL_SOURCES = {
+    "chunk_fwd": ["dn_chunk_sc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
+    "decode": ["dn_decode.cu", "dn_common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_linear_attention_dn_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode())
-                h.update(f.read())
+    for fn in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -92,7 +98,7 @@ def recorded_traffic(kernel: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
@@ -464,7 +470,7 @@ def main():
             "config": bench_config(world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode,
-            "kernel_source": kernel_source_hash(),
+            "kernel_source": {k: kernel_source_hash(k) for k in KERNEL_SOURCES},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
