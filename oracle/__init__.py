@@ -4,11 +4,13 @@ TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
 CPU-baseline leg are the only callers. Nothing here is shared with the CUDA
 path, and nothing here imports it.
 
-Two independent evaluations live here:
+Three evaluations live here, each independent of the CUDA path:
 
 * ``fwd`` -- the definition itself: a sequential fp64 loop over tokens per
   (batch, head), in plain C (``dn_oracle.c``), OpenMP across heads. This is the
   oracle that parity tests compare the GPU against.
+* ``osdn_precond`` -- OSDN phase 1, the preconditioner sequence d_t that the
+  OSDN key scale takes (sequential fp64 loop in the same C file).
 * ``chunked.fwd`` -- the chunkwise-parallel (WY / UT-transform) evaluation of
   the same recurrence in NumPy fp64, following the chunk algebra the kernels
   use. It is never compared against the GPU; it exists so that tests can show
@@ -54,6 +56,8 @@ def _load():
             lib.dn_oracle_heads.argtypes = [I, I, I, I, P, P, P, P, I, P, I, P, I, P, I, P, P, I]
             lib.dn_oracle_heads.restype = I
             lib.dn_oracle_max_threads.restype = I
+            lib.dn_oracle_osdn_heads.argtypes = [I, I, I, P, P, P, ctypes.c_double, P, P, I]
+            lib.dn_oracle_osdn_heads.restype = I
             _lib = lib
     return _lib
 
@@ -129,6 +133,45 @@ def fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None,
         o_full[b, :, h, :] = o[n]
         S_full[b, h] = S[n]
     return o_full, S_full
+
+
+def osdn_precond(k, beta, retention=None, d0=None, eta: float = 0.5, heads=None, nthreads: int = 0):
+    """OSDN phase 1 in fp64: the preconditioner d_t used by every token, and the final d_T.
+
+    k [B,T,H,dk] (bf16 bits or float), beta [B,T,H] (the scalar write strength), retention
+    [B,T,H] or None (no forgetting, r = 1), d0 [B,H,dk] or None (ones). Returns (d [B,T,H,dk],
+    d_T [B,H,dk]); with ``heads=[(b, h), ...]`` only those run and the shapes are [NH,T,dk],
+    [NH,dk].
+    """
+    k = np.asarray(k)
+    B, T, H, dk = k.shape
+    all_heads = heads is None
+    if all_heads:
+        heads = [(b, h) for b in range(B) for h in range(H)]
+    NH = len(heads)
+    kh = np.ascontiguousarray(np.stack([widen(k[b, :, h]) for (b, h) in heads])).reshape(NH, T, dk)
+    bh = np.ascontiguousarray(np.stack([widen(np.asarray(beta)[b, :, h]) for (b, h) in heads]))
+    rh = None
+    if retention is not None:
+        rh = np.ascontiguousarray(np.stack([widen(np.asarray(retention)[b, :, h]) for (b, h) in heads]))
+    if d0 is None:
+        d = np.ones((NH, dk), dtype=np.float64)
+    else:
+        d = np.ascontiguousarray(np.stack([widen(np.asarray(d0)[b, h]) for (b, h) in heads]))
+    dseq = np.zeros((NH, T, dk), dtype=np.float64)
+    rc = _load().dn_oracle_osdn_heads(NH, T, dk, kh.ctypes.data, bh.ctypes.data,
+                                      None if rh is None else rh.ctypes.data, float(eta), d.ctypes.data,
+                                      dseq.ctypes.data, nthreads)
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    if not all_heads:
+        return dseq, d
+    d_full = np.empty((B, T, H, dk), dtype=np.float64)
+    dT_full = np.empty((B, H, dk), dtype=np.float64)
+    for n, (b, h) in enumerate(heads):
+        d_full[b, :, h, :] = dseq[n]
+        dT_full[b, h] = d[n]
+    return d_full, dT_full
 
 
 def rel_l2(x, ref) -> float:

@@ -135,6 +135,66 @@ int dn_oracle_heads(int NH, int T, int dk, int dv, const double* q, const double
   return bad ? -1 : 0;
 }
 
+/*
+ * OSDN phase 1: the diagonal preconditioner sequence of one (batch, head)
+ * (OSDN page, section 2.2 "decoupled hypergradient feedback" and section 2.3
+ * "adaptive preconditioner forgetting").
+ *
+ * The per-token surrogate of the preconditioner is, in closed form,
+ *   h_t(d) = ((1 - beta_t <d, k_t (.) k_t>)^2 - 1) / (2 ||k_t||^2),
+ * whose gradient in d is
+ *   grad h_t(d) = -beta_t (1 - beta_t <d, k_t (.) k_t>) (k_t (.) k_t) / ||k_t||^2.
+ * Token t is written with the preconditioner d_t (the key scale d of the main
+ * recurrence), then one online-gradient-descent step with retention r_t follows:
+ *   d_{t+1} = r_t d_t - eta grad h_t(d_t)
+ * (r_t = 1 without retention). A token with k_t = 0 has no gradient and leaves
+ * d unchanged apart from the retention.
+ *
+ *   k: [T][dk]  beta: [T]  r: [T] or NULL  d: [dk] in: d_0, out: d_T
+ *   dseq: [T][dk] out: d_t for every token
+ */
+int dn_oracle_osdn_head(int T, int dk, const double* k, const double* beta, const double* r,
+                        double eta, double* d, double* dseq) {
+  if (T < 0 || dk <= 0 || !d || !dseq || (T > 0 && (!k || !beta))) return -1;
+  for (int t = 0; t < T; ++t) {
+    const double* kt = k + (int64_t)t * dk;
+    double* out = dseq + (int64_t)t * dk;
+    double dot = 0.0, nrm = 0.0;
+    for (int i = 0; i < dk; ++i) {
+      out[i] = d[i];
+      dot += d[i] * kt[i] * kt[i];
+      nrm += kt[i] * kt[i];
+    }
+    const double rt = r ? r[t] : 1.0;
+    const double g = 1.0 - beta[t] * dot;
+    for (int i = 0; i < dk; ++i) {
+      const double grad = nrm > 0.0 ? -beta[t] * g * kt[i] * kt[i] / nrm : 0.0;
+      d[i] = rt * d[i] - eta * grad;
+    }
+  }
+  return 0;
+}
+
+/* NH heads of OSDN phase 1, laid out contiguously ([NH][T][dk], [NH][T], [NH][dk]). */
+int dn_oracle_osdn_heads(int NH, int T, int dk, const double* k, const double* beta, const double* r,
+                         double eta, double* d, double* dseq, int nthreads) {
+  if (NH < 0) return -1;
+  int bad = 0;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int h = 0; h < NH; ++h) {
+    int rc = dn_oracle_osdn_head(T, dk, k + (int64_t)h * T * dk, beta + (int64_t)h * T,
+                                 r ? r + (int64_t)h * T : NULL, eta, d + (int64_t)h * dk,
+                                 dseq + (int64_t)h * T * dk);
+    bad |= (rc != 0);
+  }
+  return bad ? -1 : 0;
+}
+
 /* Number of threads an OpenMP parallel region would use (for reporting). */
 int dn_oracle_max_threads(void) {
 #ifdef _OPENMP
