@@ -19,6 +19,9 @@ GDN scalar gates, KDA channel decay, FG2-GDN+ with OSDN preconditioner, decode):
                                                  preconditioner d=1+0.1*N per key channel, S0~N(0,0.02^2)
   decode           1024 sequences, H=32, d=128: resident S~N(0,0.02^2) fp32, one bf16 token per step,
                    channel alpha, beta_k, beta_v as in fg2_osdn_long, 100 steps
+  osdn_phase1      the OSDN preconditioner scan on fg2_osdn_long's keys (same seed): B=2 H=16 T=32768
+                   d_k=128 bf16 k, beta=sigmoid(N) per token, retention r~U(0.95,1) per token, eta=0.5,
+                   d_0 = 1
 
 q and k are drawn N(0,1) per element and L2-normalised per (b, t, h) row in fp64
 before rounding to the storage dtype; v ~ N(0,1).
@@ -45,7 +48,8 @@ OUT_F64, OUT_F32, OUT_BF16 = 0, 1, 2
 GATE_ONE, GATE_SCALAR, GATE_CHANNEL = 0, 1, 2
 
 SEED_BASE = 20260000
-TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "alpha": 3, "beta_k": 4, "beta_v": 5, "key_scale": 6, "S0": 7}
+TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "alpha": 3, "beta_k": 4, "beta_v": 5, "key_scale": 6, "S0": 7,
+              "beta": 8, "retention": 9}
 
 
 def build(force: bool = False) -> str:
@@ -163,6 +167,11 @@ WORKLOADS = {
                        alpha=GATE_CHANNEL, alpha_kind=(GEN_EXP_NEG_SOFTPLUS, 0.05, 0.0),
                        beta_k=GATE_CHANNEL, beta_v=GATE_CHANNEL, key_scale=GATE_ONE,
                        s0_std=0.02, steps=100, cfg_index=5),
+    "osdn_phase1": Workload("osdn_phase1", B=2, T=32768, H=16, dk=128, dv=128, io="bf16",
+                            alpha=GATE_ONE, alpha_kind=(GEN_UNIFORM, 1.0, 1.0),
+                            beta_k=GATE_SCALAR, beta_v=GATE_ONE, key_scale=GATE_ONE,
+                            s0_std=0.0, cfg_index=4,
+                            extra={"eta": 0.5, "retention": (GEN_UNIFORM, 0.95, 1.0)}),
 }
 
 
@@ -213,4 +222,18 @@ def make_inputs(w: Workload, step: int = 0) -> dict:
             out["S0"] = None  # decode steps after the first continue from the resident state
     else:
         out["S0"] = None
+    return out
+
+
+def make_osdn_inputs(w: Workload) -> dict:
+    """Inputs of the OSDN preconditioner scan: k (as make_inputs draws it for the same seed block),
+    beta [B,T,H] = sigmoid(N(0,1)), retention [B,T,H] (None when the recipe has none), eta."""
+    shp = (w.B, w.T, w.H)
+    out = {"k": fill((w.B, w.T, w.H, w.dk), w.seed("k"), GEN_L2ROWS, dtype=w.io, row=w.dk),
+           "beta": fill(shp, w.seed("beta"), GEN_SIGMOID, dtype="f32"),
+           "retention": None, "eta": float(w.extra.get("eta", 0.5))}
+    rk = w.extra.get("retention")
+    if rk is not None:
+        kind, p0, p1 = rk
+        out["retention"] = fill(shp, w.seed("retention"), kind, p0, p1, dtype="f32")
     return out

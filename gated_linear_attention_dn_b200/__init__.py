@@ -10,6 +10,8 @@ Entry points (same names as the C ABI):
                  S0=None, o=None, S_T=None, stream=None) -> (o, S_T)
     dn_decode_step(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None,
                    S=..., o=None, stream=None) -> o          (S updated in place)
+    dn_osdn_precond(k, beta, retention=None, d0=None, eta=0.5, d=None, d_T=None,
+                    workspace=None, stream=None) -> (d, d_T)   (OSDN phase 1)
     dn_stream_status(stream=None) -> int
     dn_status_string(code) -> str
 
@@ -32,8 +34,8 @@ DN_ERR_WORKSPACE_TOO_SMALL, DN_ERR_CUDA, DN_ERR_DEVICE_TIMEOUT = 4, 5, 6
 DN_F32, DN_BF16 = 0, 1
 DN_GATE_ONE, DN_GATE_SCALAR, DN_GATE_CHANNEL = 0, 1, 2
 
-EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_stream_status",
-            "dn_status_string", "dn_version")
+EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_osdn_precond_workspace_bytes",
+            "dn_osdn_precond", "dn_stream_status", "dn_status_string", "dn_version")
 
 
 class DnDesc(ctypes.Structure):
@@ -41,6 +43,11 @@ class DnDesc(ctypes.Structure):
                 ("d_v", ctypes.c_int), ("chunk", ctypes.c_int), ("io_dtype", ctypes.c_int),
                 ("alpha", ctypes.c_int), ("beta_k", ctypes.c_int), ("beta_v", ctypes.c_int),
                 ("key_scale", ctypes.c_int)]
+
+
+class DnOsdnDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
+                ("io_dtype", ctypes.c_int), ("eta", ctypes.c_float)]
 
 
 class DnError(RuntimeError):
@@ -68,6 +75,11 @@ def load(path: str = LIB_PATH):
     lib.dn_chunk_fwd.restype = I
     lib.dn_decode_step.argtypes = [D, P, P, P, P, P, P, P, P, P, P]
     lib.dn_decode_step.restype = I
+    O = ctypes.POINTER(DnOsdnDesc)
+    lib.dn_osdn_precond_workspace_bytes.argtypes = [O]
+    lib.dn_osdn_precond_workspace_bytes.restype = ctypes.c_size_t
+    lib.dn_osdn_precond.argtypes = [O, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+    lib.dn_osdn_precond.restype = I
     lib.dn_stream_status.argtypes = [P]
     lib.dn_stream_status.restype = I
     lib.dn_status_string.argtypes = [I]
@@ -169,6 +181,45 @@ def dn_decode_step(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None
     if rc != DN_OK:
         raise DnError(rc, "dn_decode_step")
     return o
+
+
+def dn_osdn_precond_workspace_bytes(desc: DnOsdnDesc) -> int:
+    return int(load().dn_osdn_precond_workspace_bytes(ctypes.byref(desc)))
+
+
+def dn_osdn_precond(k, beta, retention=None, d0=None, eta: float = 0.5, d=None, d_T=None, workspace=None,
+                    stream=None):
+    """OSDN phase 1: the preconditioner d_t of every token. Returns (d [B,T,H,d_k], d_T [B,H,d_k]) fp32.
+
+    k [B,T,H,d_k] bf16 or fp32; beta [B,T,H] fp32; retention [B,T,H] fp32 or None; d0 [B,H,d_k] fp32 or
+    None (ones). The workspace (dn_osdn_precond_workspace_bytes) is allocated here when not given.
+    """
+    lib = load()
+    if not k.is_contiguous():
+        raise TypeError("k must be contiguous")
+    B, T, H, dk = k.shape
+    io = DN_BF16 if k.dtype == torch.bfloat16 else DN_F32 if k.dtype == torch.float32 else None
+    if io is None:
+        raise TypeError("k must be bfloat16 or float32")
+    for n, g, shape in (("beta", beta, (B, T, H)), ("retention", retention, (B, T, H)), ("d0", d0, (B, H, dk))):
+        if g is None:
+            continue
+        if g.dtype != torch.float32 or not g.is_contiguous() or tuple(g.shape) != shape:
+            raise ValueError(f"{n} must be a contiguous float32 tensor of shape {shape}")
+    desc = DnOsdnDesc(B, T, H, dk, io, float(eta))
+    if d is None:
+        d = torch.empty((B, T, H, dk), dtype=torch.float32, device=k.device)
+    if d_T is None:
+        d_T = torch.empty((B, H, dk), dtype=torch.float32, device=k.device)
+    ws_bytes = dn_osdn_precond_workspace_bytes(desc)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=k.device)
+    rc = lib.dn_osdn_precond(ctypes.byref(desc), _ptr(k), _ptr(beta), _ptr(retention), _ptr(d0), _ptr(d),
+                             _ptr(d_T), _ptr(workspace), ws_bytes if workspace is not None else 0,
+                             _stream_handle(stream))
+    if rc != DN_OK:
+        raise DnError(rc, "dn_osdn_precond")
+    return d, d_T
 
 
 def dn_stream_status(stream=None) -> int:

@@ -1,5 +1,6 @@
 // C ABI shim: argument validation, the per-GPU status word, and dispatch to
 // the kernels. Nothing here allocates device memory.
+#include <math.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -179,6 +180,59 @@ dn_status dn_decode_step(const dn_desc* desc, const void* q, const void* k, cons
   a.S = S;
   a.o = o;
   cudaError_t e = dn::launch_decode(a, static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+dn_status check_osdn_desc(const dn_osdn_desc* d) {
+  if (!d) return DN_ERR_INVALID_ARGUMENT;
+  if (d->B < 1 || d->H < 1 || d->T < 0) return DN_ERR_INVALID_ARGUMENT;
+  if (d->io_dtype != DN_F32 && d->io_dtype != DN_BF16) return DN_ERR_INVALID_ARGUMENT;
+  if (!isfinite(d->eta) || d->eta < 0.f) return DN_ERR_INVALID_ARGUMENT;
+  if (d->d_k != 64 && d->d_k != 128) return DN_ERR_UNSUPPORTED;
+  const int64_t heads = (int64_t)d->B * d->H;
+  const int64_t blocks = heads * ((d->T + 31) / 32);
+  if (heads >= ((int64_t)1 << 31) || blocks >= ((int64_t)1 << 32)) return DN_ERR_UNSUPPORTED;
+  if ((int64_t)d->B * d->T * d->H * d->d_k >= ((int64_t)1 << 46)) return DN_ERR_UNSUPPORTED;
+  return DN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dn_osdn_precond_workspace_bytes(const dn_osdn_desc* desc) {
+  if (check_osdn_desc(desc) != DN_OK) return 0;
+  return dn::osdn_workspace_bytes(desc->B, desc->T, desc->H);
+}
+
+dn_status dn_osdn_precond(const dn_osdn_desc* desc, const void* k, const float* beta,
+                          const float* retention, const float* d0, float* d, float* d_T,
+                          void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  dn_status st = check_osdn_desc(desc);
+  if (st != DN_OK) return st;
+  if (!aligned4(retention) || !aligned4(d0) || !aligned4(d_T)) return DN_ERR_MISALIGNED;
+  if (desc->T > 0) {
+    if (!k || !beta || !d) return DN_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k)) return DN_ERR_MISALIGNED;
+    if (!aligned4(beta) || !aligned4(d)) return DN_ERR_MISALIGNED;
+    const size_t need = dn::osdn_workspace_bytes(desc->B, desc->T, desc->H);
+    if (!workspace || workspace_bytes < need) return DN_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return DN_ERR_MISALIGNED;
+    const size_t n_d = (size_t)desc->B * desc->T * desc->H * desc->d_k * sizeof(float);
+    const size_t n_k = (size_t)desc->B * desc->T * desc->H * desc->d_k * (desc->io_dtype == DN_BF16 ? 2 : 4);
+    if (ranges_overlap(d, n_d, workspace, need) || ranges_overlap(d, n_d, k, n_k)) return DN_ERR_INVALID_ARGUMENT;
+  } else if (!d_T) {
+    return DN_OK;  // nothing to compute, nothing to write
+  }
+  cudaError_t e = dn::launch_osdn(k, beta, retention, d0, desc->eta, desc->B, desc->T, desc->H, desc->d_k,
+                                  desc->io_dtype == DN_BF16, static_cast<float*>(workspace), d, d_T,
+                                  static_cast<cudaStream_t>(cuda_stream));
   return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
 

@@ -1,0 +1,299 @@
+// OSDN phase 1: the diagonal preconditioner sequence d_t of every (b, h) (OSDN page, section 2.2
+// "decoupled hypergradient feedback", two-phase implementation item 1, and section 2.3 "adaptive
+// preconditioner forgetting"). Token t is written with d_t (the key scale d of the main
+// recurrence); then, with a_t = k_t (.) k_t,
+//   e_t = c_t (1 - beta_t <d_t, a_t>),  c_t = eta beta_t / ||k_t||^2   (0 when k_t = 0)
+//   d_{t+1} = r_t d_t + e_t a_t
+// which is d_{t+1} = r_t d_t - eta grad h_t(d_t) for the closed-form surrogate
+// h_t(d) = ((1 - beta_t <d, a_t>)^2 - 1) / (2 ||k_t||^2) (r_t = 1 without forgetting).
+//
+// The only sequential dependence is the scalar <d_t, a_t>. Over a block of m = 32 tokens
+// starting at t0, with rho_t = prod_{t0<=j<t} r_j, R(i+1, t) = prod_{i<j<t} r_j, G = Gram of the a_t,
+// W_ti = R(i+1, t) G_ti (i < t) and P_t = <d_{t0}, a_t>:
+//   <d_t, a_t> = rho_t P_t + sum_{i<t} W_ti e_i
+//   => (I + Diag(c beta) W) e = c - Diag(c beta rho) P
+//   => e = u0 - B P,  u0 = T c,  B = T Diag(c beta rho),  T = (I + Diag(c beta) W)^{-1}.
+// u0 and B do not depend on d, so they are formed for all blocks of all heads at once
+// (osdn_block_kernel, one warp per block, into the caller's workspace). The scan
+// (osdn_scan_kernel, one CTA per (b, h), one thread per key channel) then needs per block only
+// P (a transposed warp reduction), e = u0 - B P (one warp), and the per-channel recurrence that
+// writes d_t for the 32 tokens; the block's k tile, B and u0 are loaded one block ahead.
+#include "dn_common.cuh"
+
+namespace dn {
+namespace {
+
+constexpr int kM = 32;              // tokens per block
+constexpr int kBlockFloats = kM * kM + kM;  // B (row-major, row = token) then u0
+
+__device__ __forceinline__ float load_k(const void* k, int64_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(k)[i]);
+  return reinterpret_cast<const float*>(k)[i];
+}
+
+// ------------------------------------------------------------------ block kernel
+// 4 warps per CTA, one block of 32 tokens per warp; lane t = token t0 + t.
+template <int DK>
+struct BlockSmem {
+  static constexpr int AP = DK + 4;  // padded row of a (16-byte aligned, spreads rows over banks)
+  static constexpr int A = kM * AP, L = kM * (kM + 1);
+  static constexpr int BYTES = 4 * (A + L) * (int)sizeof(float);  // 4 warps
+};
+
+template <int DK>
+__global__ void __launch_bounds__(128) osdn_block_kernel(const void* k, const float* beta, const float* ret,
+                                                         float eta, int B, int T, int H, int io_bf16,
+                                                         float* ws) {
+  using Sm = BlockSmem<DK>;
+  constexpr int AP = Sm::AP;
+  extern __shared__ __align__(16) float smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nblk = (T + kM - 1) / kM;
+  const int64_t blk = (int64_t)blockIdx.x * 4 + warp;
+  if (blk >= (int64_t)B * H * nblk) return;  // whole warps only: no barrier below spans warps
+  const int bh = (int)(blk / nblk), j = (int)(blk % nblk), b = bh / H, h = bh % H;
+  const int t = j * kM + lane;
+  const bool valid = t < T;
+  float (*a)[AP] = reinterpret_cast<float (*)[AP]>(smem + warp * Sm::A);
+  float (*L)[kM + 1] = reinterpret_cast<float (*)[kM + 1]>(smem + 4 * Sm::A + warp * Sm::L);
+
+  // a_t = k_t (.) k_t, ||k_t||^2, c_t, beta_t, r_t (padding tokens: a = 0, c = 0, r = 1)
+  float nrm = 0.f;
+  const int64_t row = (((int64_t)b * T + t) * H + h) * DK;
+  if (valid && io_bf16) {
+    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(k) + row);
+#pragma unroll 4
+    for (int c8 = 0; c8 < DK / 8; ++c8) {
+      const uint4 u = __ldg(src + c8);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __uint_as_float(w[e] << 16);
+        v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float sq = v[e] * v[e];
+        nrm += sq;
+        a[lane][8 * c8 + e] = sq;
+      }
+    }
+  } else {
+    for (int c = 0; c < DK; ++c) {
+      const float x = valid ? load_k(k, row + c, io_bf16) : 0.f;
+      nrm += x * x;
+      a[lane][c] = x * x;
+    }
+  }
+  const int64_t tok = ((int64_t)b * T + t) * H + h;
+  const float bt = valid ? beta[tok] : 0.f;
+  const float rt = valid && ret ? ret[tok] : 1.f;
+  const float ct = (valid && nrm > 0.f) ? eta * bt / nrm : 0.f;
+  // rho_t = prod_{s<t} r_s within the block (exclusive product scan)
+  float incl = rt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl *= y;
+  }
+  const float prev_incl = __shfl_up_sync(0xffffffffu, incl, 1);  // every lane takes part in the shuffle
+  const float rho = lane == 0 ? 1.f : prev_incl;
+  __syncwarp();
+
+  // Gram row t: g[i] = <a_t, a_i>
+  float g[kM];
+#pragma unroll
+  for (int i = 0; i < kM; ++i) g[i] = 0.f;
+  for (int c4 = 0; c4 < DK; c4 += 4) {
+    const float4 at = *reinterpret_cast<const float4*>(&a[lane][c4]);
+#pragma unroll
+    for (int i = 0; i < kM; ++i) {
+      const float4 ai = *reinterpret_cast<const float4*>(&a[i][c4]);
+      g[i] = fmaf(at.x, ai.x, fmaf(at.y, ai.y, fmaf(at.z, ai.z, fmaf(at.w, ai.w, g[i]))));
+    }
+  }
+  // L_ti = c_t beta_t R(i+1, t) G_ti for i < t; R built from i = t - 1 downwards
+  {
+    const float cb = ct * bt;
+    float R = 1.f;
+#pragma unroll
+    for (int i = kM - 1; i >= 0; --i) {
+      const float ri = __shfl_sync(0xffffffffu, rt, i);
+      if (i < lane) {
+        L[lane][i] = cb * R * g[i];
+        R *= ri;
+      } else {
+        L[lane][i] = 0.f;
+      }
+    }
+  }
+  __syncwarp();
+  // T = (I + L)^{-1}: lane s forms column s by forward substitution
+  float x[kM];
+#pragma unroll
+  for (int r = 0; r < kM; ++r) {
+    float s0 = (r == lane) ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < r; ++i) {
+      if (i & 1)
+        s1 = fmaf(-L[r][i], x[i], s1);
+      else
+        s0 = fmaf(-L[r][i], x[i], s0);
+    }
+    x[r] = s0 + s1;
+  }
+  // B[:, s] = T[:, s] c_s beta_s rho_s (lane s); u0 = T c (row sums, through shared memory)
+  float* out = ws + blk * kBlockFloats;
+  const float colscale = ct * bt * rho;
+  __syncwarp();
+#pragma unroll
+  for (int r = 0; r < kM; ++r) {
+    out[r * kM + lane] = x[r] * colscale;  // row r: lanes write consecutive columns
+    L[r][lane] = x[r] * ct;                // reuse L for T Diag(c)
+  }
+  __syncwarp();
+  float u0 = 0.f;
+#pragma unroll
+  for (int s = 0; s < kM; ++s) u0 += L[lane][s];
+  out[kM * kM + lane] = u0;
+}
+
+// ------------------------------------------------------------------ scan kernel
+// One CTA of DK threads per (b, h); thread ch owns key channel ch of d.
+template <int DK>
+__global__ void __launch_bounds__(DK) osdn_scan_kernel(const void* k, const float* ret, const float* d0, int B,
+                                                       int T, int H, int io_bf16, const float* ws, float* dout,
+                                                       float* dT) {
+  constexpr int NW = DK / 32;
+  __shared__ float s_B[2][kM][kM + 1];
+  __shared__ float s_u0[2][kM];
+  __shared__ float s_r[2][kM];
+  __shared__ float s_part[NW][kM];
+  __shared__ float s_P[kM];
+  __shared__ float s_e[kM];
+  const int ch = threadIdx.x, lane = ch & 31, warp = ch >> 5;
+  const int bh = blockIdx.x, b = bh / H, h = bh % H;
+  const int nblk = (T + kM - 1) / kM;
+  float d = d0 ? d0[(int64_t)bh * DK + ch] : 1.f;
+
+  // block j's k column of this channel (a = k^2), retentions, B and u0 -> registers / shared memory
+  float a_nx[kM];
+  float bu_nx[(kBlockFloats + DK - 1) / DK];
+  float r_nx = 1.f;
+  auto fetch = [&](int j) {
+#pragma unroll
+    for (int t = 0; t < kM; ++t) {
+      const int tt = j * kM + t;
+      const float x = tt < T ? load_k(k, (((int64_t)b * T + tt) * H + h) * DK + ch, io_bf16) : 0.f;
+      a_nx[t] = x * x;
+    }
+    const float* src = ws + ((int64_t)bh * nblk + j) * kBlockFloats;
+#pragma unroll
+    for (int i = 0; i < (kBlockFloats + DK - 1) / DK; ++i) {
+      const int idx = i * DK + ch;
+      bu_nx[i] = idx < kBlockFloats ? src[idx] : 0.f;
+    }
+    if (ch < kM) {
+      const int tt = j * kM + ch;
+      r_nx = (tt < T && ret) ? ret[((int64_t)b * T + tt) * H + h] : 1.f;
+    }
+  };
+  auto stage = [&](int par) {
+#pragma unroll
+    for (int i = 0; i < (kBlockFloats + DK - 1) / DK; ++i) {
+      const int idx = i * DK + ch;
+      if (idx < kM * kM)
+        s_B[par][idx / kM][idx % kM] = bu_nx[i];
+      else if (idx < kBlockFloats)
+        s_u0[par][idx - kM * kM] = bu_nx[i];
+    }
+    if (ch < kM) s_r[par][ch] = r_nx;
+  };
+
+  float a[kM];
+  if (nblk > 0) fetch(0);
+  for (int j = 0; j < nblk; ++j) {
+    const int par = j & 1, t0 = j * kM, nb = min(kM, T - t0);
+#pragma unroll
+    for (int t = 0; t < kM; ++t) a[t] = a_nx[t];
+    stage(par);
+    if (j + 1 < nblk) fetch(j + 1);  // in flight during this block
+    // P_t = <d_{t0}, a_t>: per-warp partials by a transposed butterfly (lane t ends with token t)
+    {
+      float v[kM];
+#pragma unroll
+      for (int t = 0; t < kM; ++t) v[t] = d * a[t];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const bool upper = (lane & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+          const float send = upper ? v[i] : v[i + off];
+          const float keep = upper ? v[i + off] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      s_part[warp][lane] = v[0];
+    }
+    __syncthreads();
+    // e = u0 - B P (warp 0, lane t)
+    if (warp == 0) {
+      float P = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) P += s_part[w][lane];
+      s_P[lane] = P;
+      __syncwarp();
+      float e = s_u0[par][lane];
+#pragma unroll
+      for (int s = 0; s < kM; ++s) e = fmaf(-s_B[par][lane][s], s_P[s], e);
+      s_e[lane] = e;
+    }
+    __syncthreads();
+    // d_t for the block's tokens, then d_{t0 + 32}
+    float* o = dout + (((int64_t)b * T + t0) * H + h) * DK + ch;
+#pragma unroll
+    for (int t = 0; t < kM; ++t) {
+      if (t < nb) o[(int64_t)t * H * DK] = d;
+      d = fmaf(s_r[par][t], d, s_e[t] * a[t]);
+    }
+  }
+  if (dT) dT[(int64_t)bh * DK + ch] = d;
+}
+
+}  // namespace
+
+size_t osdn_workspace_bytes(int B, int T, int H) {
+  const int64_t nblk = (T + kM - 1) / kM;
+  return (size_t)B * H * nblk * kBlockFloats * sizeof(float);
+}
+
+cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, const float* d0, float eta, int B,
+                        int T, int H, int dk, int io_bf16, float* ws, float* dout, float* dT, cudaStream_t s) {
+  if ((int64_t)B * H == 0) return cudaSuccess;
+  const int64_t nblk_all = (int64_t)B * H * ((T + kM - 1) / kM);
+  if (nblk_all > 0) {
+    const unsigned grid = (unsigned)((nblk_all + 3) / 4);
+    cudaError_t e;
+    if (dk == 128) {
+      e = cudaFuncSetAttribute(osdn_block_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BlockSmem<128>::BYTES);
+      if (e != cudaSuccess) return e;
+      osdn_block_kernel<128><<<grid, 128, BlockSmem<128>::BYTES, s>>>(k, beta, ret, eta, B, T, H, io_bf16, ws);
+    } else {
+      e = cudaFuncSetAttribute(osdn_block_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BlockSmem<64>::BYTES);
+      if (e != cudaSuccess) return e;
+      osdn_block_kernel<64><<<grid, 128, BlockSmem<64>::BYTES, s>>>(k, beta, ret, eta, B, T, H, io_bf16, ws);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (dk == 128)
+    osdn_scan_kernel<128><<<B * H, 128, 0, s>>>(k, ret, d0, B, T, H, io_bf16, ws, dout, dT);
+  else
+    osdn_scan_kernel<64><<<B * H, 64, 0, s>>>(k, ret, d0, B, T, H, io_bf16, ws, dout, dT);
+  return cudaGetLastError();
+}
+
+}  // namespace dn

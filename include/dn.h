@@ -125,6 +125,43 @@ dn_status dn_decode_step(const dn_desc* desc, const void* q, const void* k, cons
                          const float* key_scale, float* S, void* o, void* cuda_stream);
 
 /*
+ * OSDN phase 1 (OSDN page, section 2.2 "decoupled hypergradient feedback", the
+ * first of its two phases, and section 2.3 "adaptive preconditioner
+ * forgetting"): the per-token diagonal preconditioner d_t of every (b, h), which
+ * dn_chunk_fwd / dn_decode_step then take as the key scale (DN_GATE_CHANNEL).
+ * Token t is written with d_t; then one online-gradient-descent step on the
+ * closed-form surrogate h_t(d) = ((1 - beta_t <d, k_t (.) k_t>)^2 - 1) / (2 ||k_t||^2):
+ *
+ *   d_{t+1} = r_t d_t + eta beta_t (1 - beta_t <d_t, k_t (.) k_t>) (k_t (.) k_t) / ||k_t||^2
+ *
+ * (r_t = 1 without forgetting; a token with k_t = 0 only applies r_t). The page
+ * prints the forgetting variant with "+ eta grad h"; this is the descent reading.
+ *
+ * In:  k [B,T,H,d_k] (io dtype); beta [B,T,H] fp32 (the scalar write strength);
+ *      retention [B,T,H] fp32 or NULL (r = 1); d0 [B,H,d_k] fp32 or NULL (ones).
+ * Out: d [B,T,H,d_k] fp32 (d_t of every token); d_T [B,H,d_k] fp32 or NULL
+ *      (the preconditioner after the last token, for a later call's d0; may
+ *      alias d0).
+ * Scratch: `workspace` of at least dn_osdn_precond_workspace_bytes() bytes,
+ * 16-byte aligned, owned by the caller; its contents on entry do not matter.
+ * Supported: d_k in {64, 128}; k 16-byte aligned; beta, retention, d0, d, d_T
+ * 4-byte aligned. T == 0 copies d0 (or ones) into d_T. Asynchronous on the stream.
+ */
+typedef struct {
+  int B, T, H;        /* batch, tokens per sequence, heads; B, H >= 1, T >= 0 */
+  int d_k;            /* key head dim: 64 or 128 */
+  dn_dtype io_dtype;  /* dtype of k */
+  float eta;          /* step size of the preconditioner's online-gradient descent (finite, >= 0) */
+} dn_osdn_desc;
+
+/* Bytes of workspace dn_osdn_precond needs: 4224 per head per 32 tokens. 0 for an invalid descriptor. */
+size_t dn_osdn_precond_workspace_bytes(const dn_osdn_desc* desc);
+
+dn_status dn_osdn_precond(const dn_osdn_desc* desc, const void* k, const float* beta,
+                          const float* retention, const float* d0, float* d, float* d_T,
+                          void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reports (and clears) the device status word
  * that kernels set when a bounded wait gives up (DN_ERR_DEVICE_TIMEOUT), or
  * DN_ERR_CUDA if the stream holds a CUDA error. DN_OK otherwise.

@@ -131,3 +131,39 @@ def test_binding_has_no_cpu_path(tmp_path):
             dn.load(str(tmp_path / "missing.so"))
         finally:
             dn._lib = saved
+
+
+def _odesc(B=1, T=64, H=2, dk=128, io=dn.DN_BF16, eta=0.5):
+    return dn.DnOsdnDesc(B, T, H, dk, io, eta)
+
+
+def test_osdn_workspace_and_validation(lib):
+    # 4224 bytes per head per 32 tokens (a 32x32 fp32 matrix and a 32-vector)
+    assert dn.dn_osdn_precond_workspace_bytes(_odesc(B=2, T=65, H=3)) == 2 * 3 * 3 * 4224
+    assert dn.dn_osdn_precond_workspace_bytes(_odesc(dk=96)) == 0
+    assert lib.dn_osdn_precond_workspace_bytes(None) == 0
+    P = ctypes.c_void_p
+    good = P(1 << 20)  # a 16-byte-aligned address the library only inspects, never touches here
+    ws = dn.dn_osdn_precond_workspace_bytes(_odesc())
+
+    def call(desc, k=good, beta=good, ret=None, d0=None, d=P(1 << 30), dT=None, w=P(1 << 24), wb=ws):
+        return lib.dn_osdn_precond(ctypes.byref(desc), k, beta, ret, d0, d, dT, w, wb, None)
+
+    assert call(_odesc(B=0)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(T=-1)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(eta=float("nan"))) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(eta=-1.0)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(io=7)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(dk=96)) == dn.DN_ERR_UNSUPPORTED
+    assert call(_odesc(), k=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(), beta=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(), d=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert call(_odesc(), k=P((1 << 20) + 8)) == dn.DN_ERR_MISALIGNED
+    assert call(_odesc(), beta=P((1 << 20) + 2)) == dn.DN_ERR_MISALIGNED
+    assert call(_odesc(), ret=P((1 << 20) + 1)) == dn.DN_ERR_MISALIGNED
+    assert call(_odesc(), w=None) == dn.DN_ERR_WORKSPACE_TOO_SMALL
+    assert call(_odesc(), wb=ws - 1) == dn.DN_ERR_WORKSPACE_TOO_SMALL
+    assert call(_odesc(), w=P((1 << 24) + 4)) == dn.DN_ERR_MISALIGNED
+    assert call(_odesc(), d=P(1 << 24)) == dn.DN_ERR_INVALID_ARGUMENT  # output overlaps the workspace
+    # T == 0 with no d_T: nothing to do
+    assert call(_odesc(T=0), k=None, beta=None, d=None, w=None, wb=0) == dn.DN_OK
