@@ -18,6 +18,8 @@
 // (osdn_scan_kernel, one CTA per (b, h), one thread per key channel) then needs per block only
 // P (a transposed warp reduction), e = u0 - B P (one warp), and the per-channel recurrence that
 // writes d_t for the 32 tokens; the block's k tile, B and u0 are loaded one block ahead.
+#include <mutex>
+
 #include "dn_common.cuh"
 
 namespace dn {
@@ -296,4 +298,51 @@ cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, cons
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ allocation-free entry point
+// Some callers cannot allocate device memory at the moment they need this scan: a serving
+// process whose allocator has handed out all of the GPU's memory up front, a host framework
+// that forbids allocations inside its compute callbacks, or a latency-critical loop where an
+// allocation's implicit device synchronisation is not allowed. dn_osdn_precond_noalloc serves
+// them with a fixed scratch buffer that is part of the library's device image: every GPU that
+// loads the library holds these 32 MiB until the process exits. Problems that need more
+// (more than 7,943 blocks of 32 tokens over all heads) are rejected.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_osdn_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+std::mutex g_scratch_mu;
+
+// Device address of the scratch buffer on the current device (host code cannot use the
+// array's name as a device pointer). Looked up once per device, on that device's first call.
+dn_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_osdn_scratch) != cudaSuccess || !p) return DN_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return DN_OK;
+}
+
+}  // namespace
 }  // namespace dn
+
+extern "C" dn_status dn_osdn_precond_noalloc(const dn_osdn_desc* desc, const void* k, const float* beta,
+                                             const float* retention, const float* d0, float* d, float* d_T,
+                                             void* cuda_stream) {
+  const size_t need = dn_osdn_precond_workspace_bytes(desc);
+  if (!desc) return DN_ERR_INVALID_ARGUMENT;
+  if (need > dn::kNoAllocScratchBytes) return DN_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  if (need > 0) {
+    const dn_status st = dn::scratch_address(&scratch);
+    if (st != DN_OK) return st;
+  }
+  return dn_osdn_precond(desc, k, beta, retention, d0, d, d_T, scratch, dn::kNoAllocScratchBytes, cuda_stream);
+}

@@ -162,6 +162,32 @@ dn_status dn_osdn_precond(const dn_osdn_desc* desc, const void* k, const float* 
                           void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * dn_osdn_precond without a caller-provided workspace: the same computation and
+ * results, with the scratch taken from a fixed 32 MiB buffer built into the
+ * library. The pages have no counterpart to this entry point; it exists for
+ * callers that cannot allocate device memory when they run the scan -- e.g. a
+ * serving process whose allocator reserved the whole GPU at start-up, or a host
+ * framework that forbids allocations inside its compute callbacks.
+ *
+ *  - Nothing is allocated: the buffer is a static device array that every GPU
+ *    which loads libdn.so holds until the process exits.
+ *  - Limit: problems whose dn_osdn_precond_workspace_bytes() exceeds 32 MiB (more
+ *    than 7,943 blocks of 32 tokens summed over all (b, h)) are rejected with
+ *    DN_ERR_WORKSPACE_TOO_SMALL before anything runs.
+ *  - The first call on each device looks up the buffer's device address on the
+ *    current device (one cudaGetSymbolAddress); make that first call before any
+ *    stream capture.
+ *  - All calls share the one buffer. Calls whose executions overlap on the GPU
+ *    (different streams, or different host threads) race on it and give wrong
+ *    results: serialise them. Its contents between calls do not matter; nothing
+ *    needs clearing.
+ * Arguments and errors are otherwise those of dn_osdn_precond.
+ */
+dn_status dn_osdn_precond_noalloc(const dn_osdn_desc* desc, const void* k, const float* beta,
+                                  const float* retention, const float* d0, float* d, float* d_T,
+                                  void* cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reports (and clears) the device status word
  * that kernels set when a bounded wait gives up (DN_ERR_DEVICE_TIMEOUT), or
  * DN_ERR_CUDA if the stream holds a CUDA error. DN_OK otherwise.
