@@ -64,6 +64,13 @@ def decode_bytes(w: di.Workload) -> int:
     return b
 
 
+def osdn_bytes(w: di.Workload) -> int:
+    """HBM bytes the OSDN preconditioner scan must move: read k, beta, retention; write d and d_T."""
+    es = 2 if w.io == "bf16" else 4
+    ntok = w.B * w.T * w.H
+    return ntok * w.dk * es + 2 * ntok * 4 + ntok * w.dk * 4 + w.B * w.H * w.dk * 4
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -77,6 +84,7 @@ def measured_peaks() -> dict:
 KERNEL_SOURCES = {
     "chunk_fwd": ["dn_chunk_sc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
     "decode": ["dn_decode.cu", "dn_common.cuh"],
+    "osdn": ["dn_osdn.cu", "dn_common.cuh"],
 }
 
 
@@ -279,6 +287,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-osdn", action="store_true", help="skip the OSDN preconditioner scan leg")
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--only", choices=["chunk", "decode"], default=None,
                     help="profiling mode: run just one kernel on the workload with batch --batch")
@@ -450,6 +459,59 @@ def main():
         launches += nd
         del steps_dev, S
 
+    # ---- OSDN phase 1 (the preconditioner scan), next to the chunked pass it feeds
+    osdn = None
+    if not args.no_osdn:
+        wo = di.WORKLOADS["osdn_phase1"]
+        xo = di.make_osdn_inputs(wo)
+        ko, bo, ro = to_dev(xo["k"]), to_dev(xo["beta"]), to_dev(xo["retention"])
+        do = torch.empty((wo.B, wo.T, wo.H, wo.dk), dtype=torch.float32, device="cuda")
+        dTo = torch.empty((wo.B, wo.H, wo.dk), dtype=torch.float32, device="cuda")
+        desc = dn.DnOsdnDesc(wo.B, wo.T, wo.H, wo.dk, dn.DN_BF16, xo["eta"])
+        wso = torch.empty(dn.dn_osdn_precond_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+
+        def ostep():
+            dn.dn_osdn_precond(ko, bo, ro, None, eta=xo["eta"], d=do, d_T=dTo, workspace=wso, stream=stream)
+
+        # the chunked pass over the same keys (fg2_osdn_long), with the scan's d as its key scale
+        wf = di.WORKLOADS["fg2_osdn_long"]
+        xf = {n: to_dev(a) for n, a in di.make_inputs(wf).items()}
+        Sf = torch.empty((wf.B, wf.H, wf.dk, wf.dv), dtype=torch.float32, device="cuda")
+        of = torch.empty((wf.B, wf.T, wf.H, wf.dv), dtype=torch.bfloat16, device="cuda")
+
+        def fstep():
+            dn.dn_chunk_fwd(xf["q"], xf["k"], xf["v"], xf["alpha"], xf["beta_k"], xf["beta_v"], do, xf["S0"],
+                            o=of, S_T=Sf, stream=stream)
+
+        def timed(fn, n):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            a0.record(stream)
+            for _ in range(n):
+                fn()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            return a0.elapsed_time(a1) / n
+
+        o_ms = timed(ostep, 10)
+        f_ms = timed(fstep, 3)
+        if dn.dn_stream_status(stream) != dn.DN_OK:
+            raise RuntimeError("device status after the OSDN scan")
+        ob = osdn_bytes(wo)
+        ogbs = ob / (o_ms * 1e-3) / 1e9
+        osdn = {"workload": "OSDN preconditioner scan, B=2 H=16 T=32768 d_k=128 (fg2_osdn_long's keys), "
+                            "scalar beta, retention, eta=0.5",
+                "ms_per_call": o_ms, "tokens_per_s": wo.B * wo.T * world / (o_ms * 1e-3),
+                "chunk_fwd_ms_same_keys": f_ms, "scan_over_chunk_fwd": o_ms / f_ms,
+                "roofline": {"bound": "hbm", "achieved": ogbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": ogbs / peaks["hbm_gbs"], "traffic": recorded_traffic("osdn"),
+                             "algorithmic_bytes_per_launch": ob}}
+        launches += 2 * 10 + 3  # timed: 10 scans of two kernels, 3 chunked passes
+        del ko, bo, ro, do, dTo, wso, xf, Sf, of
+
     clocks.__exit__(None, None, None)
 
     cpu = None
@@ -469,7 +531,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": bench_config(world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode,
+            "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode, "osdn_phase1": osdn,
             "kernel_source": {k: kernel_source_hash(k) for k in KERNEL_SOURCES},
         }
         print(json.dumps(line), flush=True)

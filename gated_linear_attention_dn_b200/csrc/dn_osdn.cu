@@ -21,12 +21,13 @@
 #include <mutex>
 
 #include "dn_common.cuh"
+#include "dn_tc_ptx.cuh"
 
 namespace dn {
 namespace {
 
 constexpr int kM = 32;              // tokens per block
-constexpr int kBlockFloats = kM * kM + kM;  // B (row-major, row = token) then u0
+constexpr int kBlockFloats = kM * kM + kM;  // B (column-major: element (t, s) at s * 32 + t), then u0
 
 __device__ __forceinline__ float load_k(const void* k, int64_t i, int bf16) {
   if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(k)[i]);
@@ -48,7 +49,8 @@ __global__ void __launch_bounds__(128) osdn_block_kernel(const void* k, const fl
                                                          float* ws) {
   using Sm = BlockSmem<DK>;
   constexpr int AP = Sm::AP;
-  extern __shared__ __align__(16) float smem[];
+  extern __shared__ __align__(16) float smem_raw[];
+  float* const smem = smem_raw;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nblk = (T + kM - 1) / kM;
   const int64_t blk = (int64_t)blockIdx.x * 4 + warp;
@@ -64,9 +66,12 @@ __global__ void __launch_bounds__(128) osdn_block_kernel(const void* k, const fl
   const int64_t row = (((int64_t)b * T + t) * H + h) * DK;
   if (valid && io_bf16) {
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(k) + row);
-#pragma unroll 4
+    uint4 raw[DK / 8];  // the whole row in flight before any of it is used
+#pragma unroll
+    for (int c8 = 0; c8 < DK / 8; ++c8) raw[c8] = __ldg(src + c8);
+#pragma unroll
     for (int c8 = 0; c8 < DK / 8; ++c8) {
-      const uint4 u = __ldg(src + c8);
+      const uint4 u = raw[c8];
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
       float v[8];
 #pragma unroll
@@ -145,15 +150,17 @@ __global__ void __launch_bounds__(128) osdn_block_kernel(const void* k, const fl
     }
     x[r] = s0 + s1;
   }
-  // B[:, s] = T[:, s] c_s beta_s rho_s (lane s); u0 = T c (row sums, through shared memory)
+  // B[:, s] = T[:, s] c_s beta_s rho_s (lane s writes column s, stored column-major so that the
+  // scan's lanes read rows without bank conflicts); u0 = T c (row sums, through shared memory)
   float* out = ws + blk * kBlockFloats;
   const float colscale = ct * bt * rho;
   __syncwarp();
 #pragma unroll
-  for (int r = 0; r < kM; ++r) {
-    out[r * kM + lane] = x[r] * colscale;  // row r: lanes write consecutive columns
-    L[r][lane] = x[r] * ct;                // reuse L for T Diag(c)
-  }
+  for (int r = 0; r < kM; r += 4)
+    *reinterpret_cast<float4*>(out + lane * kM + r) =
+        make_float4(x[r] * colscale, x[r + 1] * colscale, x[r + 2] * colscale, x[r + 3] * colscale);
+#pragma unroll
+  for (int r = 0; r < kM; ++r) L[r][lane] = x[r] * ct;  // reuse L for T Diag(c)
   __syncwarp();
   float u0 = 0.f;
 #pragma unroll
@@ -162,15 +169,31 @@ __global__ void __launch_bounds__(128) osdn_block_kernel(const void* k, const fl
 }
 
 // ------------------------------------------------------------------ scan kernel
-// One CTA of DK threads per (b, h); thread ch owns key channel ch of d.
-template <int DK>
+// One CTA of DK threads per (b, h); thread ch owns key channel ch of d. A ring of kStages shared-
+// memory stages holds the k tile, B, u0 and retentions of the next blocks, copied with cp.async
+// kStages - 1 blocks ahead (one commit group per block, empty past the end, so that a fixed
+// wait_group count always means "this block's copies have landed").
+constexpr int kStages = 4;
+
+template <int DK, bool BF16>
+struct ScanSmem {
+  static constexpr int KT = kM * DK * (BF16 ? 2 : 4);  // k tile bytes
+  static constexpr int BU = kBlockFloats * 4;          // B and u0
+  static constexpr int RT = kM * 4;                    // retentions
+  static constexpr int STAGE = KT + BU + RT;
+  static constexpr int BYTES = kStages * STAGE;
+  static_assert(KT % 16 == 0 && BU % 16 == 0 && STAGE % 16 == 0, "16-byte cp.async granularity");
+};
+
+template <int DK, bool BF16>
 __global__ void __launch_bounds__(DK) osdn_scan_kernel(const void* k, const float* ret, const float* d0, int B,
-                                                       int T, int H, int io_bf16, const float* ws, float* dout,
-                                                       float* dT) {
+                                                       int T, int H, const float* ws, float* dout, float* dT) {
+  using namespace tc;
+  using Sm = ScanSmem<DK, BF16>;
   constexpr int NW = DK / 32;
-  __shared__ float s_B[2][kM][kM + 1];
-  __shared__ float s_u0[2][kM];
-  __shared__ float s_r[2][kM];
+  constexpr int ES = BF16 ? 2 : 4, ROW = DK * ES, ROW_CHUNKS = ROW / 16;
+  extern __shared__ __align__(16) float smem_raw[];  // same declaration type as the block kernel's
+  uint8_t* const smem = reinterpret_cast<uint8_t*>(smem_raw);
   __shared__ float s_part[NW][kM];
   __shared__ float s_P[kM];
   __shared__ float s_e[kM];
@@ -178,49 +201,45 @@ __global__ void __launch_bounds__(DK) osdn_scan_kernel(const void* k, const floa
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const int nblk = (T + kM - 1) / kM;
   float d = d0 ? d0[(int64_t)bh * DK + ch] : 1.f;
+  auto s_k = [&](int st) { return smem + st * Sm::STAGE; };
+  auto s_bu = [&](int st) { return reinterpret_cast<float*>(smem + st * Sm::STAGE + Sm::KT); };
+  auto s_r = [&](int st) { return reinterpret_cast<float*>(smem + st * Sm::STAGE + Sm::KT + Sm::BU); };
 
-  // block j's k column of this channel (a = k^2), retentions, B and u0 -> registers / shared memory
-  float a_nx[kM];
-  float bu_nx[(kBlockFloats + DK - 1) / DK];
-  float r_nx = 1.f;
-  auto fetch = [&](int j) {
+  // copies of block j into stage j % kStages, committed as one group (an empty group past the end)
+  auto issue = [&](int j) {
+    if (j < nblk) {
+      const int st = j % kStages, t0 = j * kM, nb = min(kM, T - t0);
+      const uint8_t* kb = static_cast<const uint8_t*>(k);
+      for (int c = ch; c < kM * ROW_CHUNKS; c += DK) {
+        const int t = c / ROW_CHUNKS, part = c % ROW_CHUNKS;
+        const bool v = t < nb;
+        const uint8_t* src = v ? kb + (((int64_t)b * T + t0 + t) * H + h) * ROW + part * 16 : kb;
+        cp_async_16_zfill(s_k(st) + t * ROW + part * 16, src, v ? 16u : 0u);
+      }
+      const float* wb = ws + ((int64_t)bh * nblk + j) * kBlockFloats;
+      for (int c = ch; c < kBlockFloats / 4; c += DK) cp_async_16_zfill(s_bu(st) + 4 * c, wb + 4 * c, 16u);
+      if (ret && ch < nb) cp_async_4(s_r(st) + ch, ret + ((int64_t)b * T + t0 + ch) * H + h);
+    }
+    cp_async_commit();
+  };
+
+#pragma unroll
+  for (int j = 0; j < kStages - 1; ++j) issue(j);
+  for (int j = 0; j < nblk; ++j) {
+    const int st = j % kStages, t0 = j * kM, nb = min(kM, T - t0);
+    cp_async_wait_group<kStages - 2>();
+    __syncthreads();             // block j's tiles have landed, and every thread is done with block j - 1
+    issue(j + kStages - 1);      // into the stage block j - 1 used
+    float a[kM];
 #pragma unroll
     for (int t = 0; t < kM; ++t) {
-      const int tt = j * kM + t;
-      const float x = tt < T ? load_k(k, (((int64_t)b * T + tt) * H + h) * DK + ch, io_bf16) : 0.f;
-      a_nx[t] = x * x;
+      float x;
+      if (BF16)
+        x = __uint_as_float((uint32_t)reinterpret_cast<const unsigned short*>(s_k(st))[t * DK + ch] << 16);
+      else
+        x = reinterpret_cast<const float*>(s_k(st))[t * DK + ch];
+      a[t] = x * x;
     }
-    const float* src = ws + ((int64_t)bh * nblk + j) * kBlockFloats;
-#pragma unroll
-    for (int i = 0; i < (kBlockFloats + DK - 1) / DK; ++i) {
-      const int idx = i * DK + ch;
-      bu_nx[i] = idx < kBlockFloats ? src[idx] : 0.f;
-    }
-    if (ch < kM) {
-      const int tt = j * kM + ch;
-      r_nx = (tt < T && ret) ? ret[((int64_t)b * T + tt) * H + h] : 1.f;
-    }
-  };
-  auto stage = [&](int par) {
-#pragma unroll
-    for (int i = 0; i < (kBlockFloats + DK - 1) / DK; ++i) {
-      const int idx = i * DK + ch;
-      if (idx < kM * kM)
-        s_B[par][idx / kM][idx % kM] = bu_nx[i];
-      else if (idx < kBlockFloats)
-        s_u0[par][idx - kM * kM] = bu_nx[i];
-    }
-    if (ch < kM) s_r[par][ch] = r_nx;
-  };
-
-  float a[kM];
-  if (nblk > 0) fetch(0);
-  for (int j = 0; j < nblk; ++j) {
-    const int par = j & 1, t0 = j * kM, nb = min(kM, T - t0);
-#pragma unroll
-    for (int t = 0; t < kM; ++t) a[t] = a_nx[t];
-    stage(par);
-    if (j + 1 < nblk) fetch(j + 1);  // in flight during this block
     // P_t = <d_{t0}, a_t>: per-warp partials by a transposed butterfly (lane t ends with token t)
     {
       float v[kM];
@@ -239,28 +258,44 @@ __global__ void __launch_bounds__(DK) osdn_scan_kernel(const void* k, const floa
       s_part[warp][lane] = v[0];
     }
     __syncthreads();
-    // e = u0 - B P (warp 0, lane t)
+    // e = u0 - B P (warp 0, lane t; B column-major)
     if (warp == 0) {
       float P = 0.f;
 #pragma unroll
       for (int w = 0; w < NW; ++w) P += s_part[w][lane];
       s_P[lane] = P;
       __syncwarp();
-      float e = s_u0[par][lane];
+      const float* bu = s_bu(st);
+      float e = bu[kM * kM + lane];
 #pragma unroll
-      for (int s = 0; s < kM; ++s) e = fmaf(-s_B[par][lane][s], s_P[s], e);
+      for (int s2 = 0; s2 < kM; ++s2) e = fmaf(-bu[s2 * kM + lane], s_P[s2], e);
       s_e[lane] = e;
     }
     __syncthreads();
-    // d_t for the block's tokens, then d_{t0 + 32}
+    // d_t for the block's tokens, then d_{t0 + nb}
     float* o = dout + (((int64_t)b * T + t0) * H + h) * DK + ch;
+    const float* rr = s_r(st);
 #pragma unroll
     for (int t = 0; t < kM; ++t) {
-      if (t < nb) o[(int64_t)t * H * DK] = d;
-      d = fmaf(s_r[par][t], d, s_e[t] * a[t]);
+      if (t < nb) {
+        o[(int64_t)t * H * DK] = d;
+        d = fmaf(ret ? rr[t] : 1.f, d, s_e[t] * a[t]);
+      }
     }
   }
+  cp_async_wait_all();
   if (dT) dT[(int64_t)bh * DK + ch] = d;
+}
+
+template <int DK, bool BF16>
+cudaError_t launch_scan(const void* k, const float* ret, const float* d0, int B, int T, int H, const float* ws,
+                        float* dout, float* dT, cudaStream_t s) {
+  using Sm = ScanSmem<DK, BF16>;
+  cudaError_t e = cudaFuncSetAttribute(osdn_scan_kernel<DK, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Sm::BYTES);
+  if (e != cudaSuccess) return e;
+  osdn_scan_kernel<DK, BF16><<<B * H, DK, Sm::BYTES, s>>>(k, ret, d0, B, T, H, ws, dout, dT);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -292,10 +327,10 @@ cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, cons
     if (e != cudaSuccess) return e;
   }
   if (dk == 128)
-    osdn_scan_kernel<128><<<B * H, 128, 0, s>>>(k, ret, d0, B, T, H, io_bf16, ws, dout, dT);
-  else
-    osdn_scan_kernel<64><<<B * H, 64, 0, s>>>(k, ret, d0, B, T, H, io_bf16, ws, dout, dT);
-  return cudaGetLastError();
+    return io_bf16 ? launch_scan<128, true>(k, ret, d0, B, T, H, ws, dout, dT, s)
+                   : launch_scan<128, false>(k, ret, d0, B, T, H, ws, dout, dT, s);
+  return io_bf16 ? launch_scan<64, true>(k, ret, d0, B, T, H, ws, dout, dT, s)
+                 : launch_scan<64, false>(k, ret, d0, B, T, H, ws, dout, dT, s);
 }
 
 // ------------------------------------------------------------------ allocation-free entry point
