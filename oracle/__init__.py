@@ -53,7 +53,7 @@ def _load():
             lib = ctypes.CDLL(_LIB_PATH)
             P = ctypes.c_void_p
             I = ctypes.c_int
-            lib.dn_oracle_heads.argtypes = [I, I, I, I, P, P, P, P, I, P, I, P, I, P, I, P, P, I]
+            lib.dn_oracle_heads.argtypes = [I, I, I, I, P, P, P, P, I, P, I, P, I, P, I, P, P, I, I]
             lib.dn_oracle_heads.restype = I
             lib.dn_oracle_max_threads.restype = I
             lib.dn_oracle_osdn_heads.argtypes = [I, I, I, P, P, P, ctypes.c_double, P, P, I]
@@ -90,8 +90,10 @@ def _per_head(x, heads, width_expected):
 
 
 def fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None,
-        heads=None, nthreads: int = 0):
+        heads=None, nthreads: int = 0, readout: str = "post"):
     """Sequential fp64 recurrence. Returns (o, S_T).
+
+    readout="post": o_t = S_t^T q_t (after the token's update); "pre": o_t = S_{t-1}^T q_t.
 
     With ``heads=None`` every (b, h) runs and o is [B,T,H,dv], S_T [B,H,dk,dv].
     With ``heads=[(b, h), ...]`` only those run and o is [NH,T,dv], S_T [NH,dk,dv].
@@ -121,8 +123,11 @@ def fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None,
     def ptr(a):
         return None if a is None else a.ctypes.data
 
+    if readout not in ("post", "pre"):
+        raise ValueError("readout must be 'post' or 'pre'")
     rc = _load().dn_oracle_heads(NH, T, dk, dv, ptr(qh), ptr(kh), ptr(vh), ptr(ah), aw, ptr(bkh), bkw,
-                                 ptr(bvh), bvw, ptr(dh), dw, S.ctypes.data, o.ctypes.data, nthreads)
+                                 ptr(bvh), bvw, ptr(dh), dw, S.ctypes.data, o.ctypes.data,
+                                 int(readout == "pre"), nthreads)
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     if not all_heads:

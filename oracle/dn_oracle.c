@@ -24,7 +24,9 @@
  *             = (I - w_t k_t^T) Diag(alpha_t) S_{t-1} + w_t (beta^v_t (.) v_t)^T,
  *             the delta rule as one online-gradient step on 0.5 ||S k - v||^2
  *             (OSDN page, section 1), transposed to the key-major orientation.
- *   readout   o_t = S_t^T q_t  (after the update, no 1/sqrt(dk) scaling)
+ *   readout   o_t = S_t^T q_t  (after the update, no 1/sqrt(dk) scaling), or, with pre_read,
+ *             o_t = S_{t-1}^T q_t: the state before token t's decay and write (the read of the
+ *             delta-mem page, section 2.C, r_t = S_{t-1} q_t, transposed to key-major).
  *
  * Gate widths: 0 = absent (the gate is 1), 1 = one value per token, n = one value
  * per channel (n = dk for alpha, beta^k, d; n = dv for beta^v).
@@ -54,7 +56,7 @@ static inline double gate(const double* g, int width, int t, int i) {
 int dn_oracle_head(int T, int dk, int dv, const double* q, const double* k, const double* v,
                    const double* alpha, int alpha_w, const double* beta_k, int bk_w,
                    const double* beta_v, int bv_w, const double* key_scale, int d_w, double* S,
-                   double* o) {
+                   double* o, int pre_read) {
   if (T < 0 || dk <= 0 || dv <= 0 || !S) return -1;
   if (!(alpha_w == 0 || alpha_w == 1 || alpha_w == dk)) return -1;
   if (!(bk_w == 0 || bk_w == 1 || bk_w == dk)) return -1;
@@ -71,6 +73,16 @@ int dn_oracle_head(int T, int dk, int dv, const double* q, const double* k, cons
     const double* kt = k + (int64_t)t * dk;
     const double* qt = q + (int64_t)t * dk;
     const double* vt = v + (int64_t)t * dv;
+    double* ot = o + (int64_t)t * dv;
+    if (pre_read) {
+      /* o_t = S_{t-1}^T q_t, before this token's decay and write */
+      for (int j = 0; j < dv; ++j) ot[j] = 0.0;
+      for (int i = 0; i < dk; ++i) {
+        const double* Si = S + (int64_t)i * dv;
+        const double qpre = qt[i];
+        for (int j = 0; j < dv; ++j) ot[j] += Si[j] * qpre;
+      }
+    }
     /* S_bar = Diag(alpha_t) S_{t-1}: row i of S scales by alpha_t[i] */
     for (int i = 0; i < dk; ++i) {
       double a = gate(alpha, alpha_w, t, i);
@@ -92,8 +104,8 @@ int dn_oracle_head(int T, int dk, int dv, const double* q, const double* k, cons
       double wi = w[i];
       for (int j = 0; j < dv; ++j) Si[j] += wi * u[j];
     }
+    if (pre_read) continue;
     /* o_t = S_t^T q_t */
-    double* ot = o + (int64_t)t * dv;
     for (int j = 0; j < dv; ++j) ot[j] = 0.0;
     for (int i = 0; i < dk; ++i) {
       const double* Si = S + (int64_t)i * dv;
@@ -114,7 +126,7 @@ int dn_oracle_head(int T, int dk, int dv, const double* q, const double* k, cons
 int dn_oracle_heads(int NH, int T, int dk, int dv, const double* q, const double* k,
                     const double* v, const double* alpha, int alpha_w, const double* beta_k,
                     int bk_w, const double* beta_v, int bv_w, const double* key_scale, int d_w,
-                    double* S, double* o, int nthreads) {
+                    double* S, double* o, int pre_read, int nthreads) {
   if (NH < 0) return -1;
   int bad = 0;
 #ifdef _OPENMP
@@ -129,7 +141,8 @@ int dn_oracle_heads(int NH, int T, int dk, int dv, const double* q, const double
         T, dk, dv, q + tk, k + tk, v + tv, alpha ? alpha + (int64_t)h * T * alpha_w : NULL, alpha_w,
         beta_k ? beta_k + (int64_t)h * T * bk_w : NULL, bk_w,
         beta_v ? beta_v + (int64_t)h * T * bv_w : NULL, bv_w,
-        key_scale ? key_scale + (int64_t)h * T * d_w : NULL, d_w, S + (int64_t)h * dk * dv, o + tv);
+        key_scale ? key_scale + (int64_t)h * T * d_w : NULL, d_w, S + (int64_t)h * dk * dv, o + tv,
+        pre_read);
     bad |= (rc != 0);
   }
   return bad ? -1 : 0;

@@ -54,7 +54,7 @@ def test_pins_catch_planted_mistake(name, tmp_path, monkeypatch):
                    check=True)
     lib = ctypes.CDLL(str(so))
     P, I = ctypes.c_void_p, ctypes.c_int
-    lib.dn_oracle_heads.argtypes = [I, I, I, I, P, P, P, P, I, P, I, P, I, P, I, P, P, I]
+    lib.dn_oracle_heads.argtypes = [I, I, I, I, P, P, P, P, I, P, I, P, I, P, I, P, P, I, I]
     lib.dn_oracle_heads.restype = I
     oracle._load()
     monkeypatch.setattr(oracle, "_lib", lib)
