@@ -33,6 +33,8 @@ DN_OK, DN_ERR_INVALID_ARGUMENT, DN_ERR_UNSUPPORTED, DN_ERR_MISALIGNED = 0, 1, 2,
 DN_ERR_WORKSPACE_TOO_SMALL, DN_ERR_CUDA, DN_ERR_DEVICE_TIMEOUT = 4, 5, 6
 DN_F32, DN_BF16 = 0, 1
 DN_GATE_ONE, DN_GATE_SCALAR, DN_GATE_CHANNEL = 0, 1, 2
+DN_READ_POST, DN_READ_PRE = 0, 1
+_READOUT = {"post": DN_READ_POST, "pre": DN_READ_PRE}
 
 EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_osdn_precond_workspace_bytes",
             "dn_osdn_precond", "dn_stream_status", "dn_status_string", "dn_version")
@@ -42,7 +44,7 @@ class DnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
                 ("d_v", ctypes.c_int), ("chunk", ctypes.c_int), ("io_dtype", ctypes.c_int),
                 ("alpha", ctypes.c_int), ("beta_k", ctypes.c_int), ("beta_v", ctypes.c_int),
-                ("key_scale", ctypes.c_int)]
+                ("key_scale", ctypes.c_int), ("readout", ctypes.c_int)]
 
 
 class DnOsdnDesc(ctypes.Structure):
@@ -115,7 +117,7 @@ def _gate_mode(g, B, T, H, width, name):
     raise ValueError(f"{name} has shape {tuple(g.shape)}; expected {(B, T, H)} or {(B, T, H, width)}")
 
 
-def make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk: int = 0) -> DnDesc:
+def make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk: int = 0, readout: str = "post") -> DnDesc:
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     if q.dtype == torch.bfloat16:
@@ -126,7 +128,8 @@ def make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk: int = 0) -> DnDesc:
         raise TypeError("q/k/v must be bfloat16 or float32")
     return DnDesc(B, T, H, dk, dv, chunk, io,
                   _gate_mode(alpha, B, T, H, dk, "alpha"), _gate_mode(beta_k, B, T, H, dk, "beta_k"),
-                  _gate_mode(beta_v, B, T, H, dv, "beta_v"), _gate_mode(key_scale, B, T, H, dk, "key_scale"))
+                  _gate_mode(beta_v, B, T, H, dv, "beta_v"), _gate_mode(key_scale, B, T, H, dk, "key_scale"),
+                  _READOUT[readout])
 
 
 def _check_io(q, k, v):
@@ -144,11 +147,13 @@ def dn_chunk_fwd_workspace_bytes(desc: DnDesc) -> int:
 
 
 def dn_chunk_fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, o=None,
-                 S_T=None, stream=None, chunk: int = 0, workspace=None):
-    """Chunked prefill. Returns (o [B,T,H,d_v] io dtype, S_T [B,H,d_k,d_v] fp32)."""
+                 S_T=None, stream=None, chunk: int = 0, workspace=None, readout: str = "post"):
+    """Chunked prefill. Returns (o [B,T,H,d_v] io dtype, S_T [B,H,d_k,d_v] fp32).
+
+    readout="post": o_t = S_t^T q_t; "pre": o_t = S_{t-1}^T q_t (before the token's update)."""
     lib = load()
     _check_io(q, k, v)
-    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk)
+    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk, readout)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     if o is None:
@@ -167,13 +172,14 @@ def dn_chunk_fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, 
 
 
 def dn_decode_step(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S=None, o=None,
-                   stream=None):
-    """One recurrent step; S [B,H,d_k,d_v] fp32 is updated in place. Returns o [B,1,H,d_v]."""
+                   stream=None, readout: str = "post"):
+    """One recurrent step; S [B,H,d_k,d_v] fp32 is updated in place. Returns o [B,1,H,d_v]
+    (readout="pre": o = S^T q from the state before this step)."""
     lib = load()
     _check_io(q, k, v)
     if S is None:
         raise ValueError("decode needs the resident state S")
-    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale)
+    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, 0, readout)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     rc = lib.dn_decode_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),

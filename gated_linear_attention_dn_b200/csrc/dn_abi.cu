@@ -40,6 +40,7 @@ dn_status check_desc(const dn_desc* d, bool decode) {
   if (!gate_ok(d->alpha) || !gate_ok(d->beta_k) || !gate_ok(d->beta_v) || !gate_ok(d->key_scale))
     return DN_ERR_INVALID_ARGUMENT;
   if (d->chunk < 0) return DN_ERR_INVALID_ARGUMENT;
+  if (d->readout != DN_READ_POST && d->readout != DN_READ_PRE) return DN_ERR_INVALID_ARGUMENT;
   if (!((d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128))) return DN_ERR_UNSUPPORTED;
   if (!(d->chunk == 0 || d->chunk == 64)) return DN_ERR_UNSUPPORTED;
   // sizes must stay addressable with 32-bit grid math and 64-bit offsets
@@ -83,6 +84,7 @@ dn_status fill_args(const dn_desc* d, const void* q, const void* k, const void* 
   a->beta_k = d->beta_k;
   a->beta_v = d->beta_v;
   a->key_scale = d->key_scale;
+  a->pre_read = d->readout == DN_READ_PRE;
   a->q = q;
   a->k = k;
   a->v = v;

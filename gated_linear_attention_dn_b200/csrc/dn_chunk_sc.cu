@@ -56,7 +56,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, far above any legi
 template <int NV>
 struct ScLayout {
   static constexpr int STK = 0;                   // raw k [C][DK] (TMA): state-update operand
-  static constexpr int STQ = STK + C * DK * 2;    // T Diag(beta^v) [128][C] (rows 64..127 zero)
+  static constexpr int STQ = STK + C * DK * 2;    // T Diag(beta^v) [128][C]: rows 0..63 bf16 hi, 64..127 lo (or 0)
   static constexpr int STV = STQ + 128 * C * 2;   // raw v [C][NV] (TMA)
   static constexpr int KQ0 = STV + C * NV * 2;    // [K; Q] (TMA), then [Wk; Q]: even chunks
   static constexpr int KQ1 = KQ0 + 128 * DK * 2;  //                               odd chunks
@@ -89,11 +89,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ __align__(16) float s_Y[2048];  // inverse scratch
   // per-token factors by chunk index mod 4: r_t, 1/r_t, beta^k d, beta^v; gamma_C / gamma_m; gamma_m
-  __shared__ float s_r[4][C], s_ri[4][C], s_ws[4][C], s_bv[4][C];
+  __shared__ float s_r[4][C], s_ri[4][C], s_ws[4][C], s_bv[4][C], s_al[4][C];
   __shared__ float s_lam[4], s_gm[4];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
+  const int pre = a.pre_read ? 1 : 0;  // o_t before the token's update: strictly causal P, scale r_{t-1}
+  // a per-token beta^v is folded into T Diag(beta^v), kept as bf16 hi + lo (U0 = T~_hi V + T~_lo V)
+  const bool bv_split = a.beta_v != DN_GATE_ONE;
   const int T = a.T, H = a.H, dv = a.dv;
   const int nslices = dv / NV;
   const int bh = blockIdx.x / nslices, b = bh / H, h = bh % H;
@@ -230,6 +233,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t ad = sdesc(smem_u32(sm + Ly::STQ) + kk * 2, 16, 1024);
           const uint64_t bv = sdesc(smem_u32(sm + Ly::STV) + kk * 128, C * 128, 1024);
           mma_bf16(tmem + Ly::TM_U0, ad, bv, id_nv, kk > 0);
+        }
+        if (bv_split) {
+          // + (lo part of T Diag(beta^v)) V: the lo rows sit in rows 64..127 of the tile, so this
+          // 128-row operand starts there; its other 64 rows only reach unused rows of U0
+#pragma unroll
+          for (int kk = 0; kk < C; kk += 16) {
+            const uint64_t ad = sdesc(smem_u32(sm + Ly::STQ) + 64 * 128 + kk * 2, 16, 1024);
+            const uint64_t bv = sdesc(smem_u32(sm + Ly::STV) + kk * 128, C * 128, 1024);
+            mma_bf16(tmem + Ly::TM_U0, ad, bv, id_nv, 1);
+          }
         }
         mma_commit(&bar_mma);
         if (c + 1 < nchunks) {
@@ -430,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // load is warp-collective: every lane loads, only rows of real tokens store
       if (q4 >= 2) {
         const int t = 32 * (q4 - 2) + lane, nc = min(C, T - t0);
-        const float os = s_r[cur][t];
+        // post-update read-out: r_t; pre-update: r_{t-1} = r_t / alpha_t
+        const float os = pre ? __fdividef(s_r[cur][t], s_al[cur][t]) : s_r[cur][t];
         __nv_bfloat16* orow =
             reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0 + t) * H + h) * dv + col0;
         uint32_t xr[NCB][32];
@@ -532,6 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       s_ws[slot][j] = ws;
       s_bv[slot][j] = bv;
+      s_al[slot][j] = al;
     };
     if (gt < 64 && nchunks > 0) load_gates(0, gt);
 
@@ -576,14 +591,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q8 = 0; q8 < 4; ++q8) {
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = (32 * gch + 8 * q8 + e <= t) ? x[8 * q8 + e] : 0.f;
+          for (int e = 0; e < 8; ++e) y[e] = (32 * gch + 8 * q8 + e <= t - pre) ? x[8 * q8 + e] : 0.f;
           *reinterpret_cast<uint4*>(pt + canon_chunk(t, 4 * gch + q8, 64)) =
               make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]));
         }
       }
       tc_fence_before();
       // ---- X3: T = (I + A)^{-1} -> T Diag(r) (TP rows 0..63) and T Diag(beta^v) (STQ rows 0..63)
-      unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt, kBarXform);
+      unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt, kBarXform,
+                                         bv_split);
       fence_proxy_async();
       group_sync(kBarXform, kXformThreads);
       if (gt == 0) mbar_arrive(&bar_tready);

@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, ch = warp >> 2;
+  const int pre = a.pre_read ? 1 : 0;  // o_t before the token's update: strictly causal P, Q+ with r_{t-1}
   const int T = a.T, H = a.H, dv = a.dv;
   // one CTA per (b, h) and slice of NV value columns (columns of the state evolve independently)
   const int nslices = dv / NV;
@@ -350,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float4 kk = unpack4(kr[i]), qq = unpack4(qr[i]);
         *reinterpret_cast<uint2*>(kq + canon(j, cb0, 128)) = pack4(mul4(kk, r));
-        *reinterpret_cast<uint2*>(kq + canon(64 + j, cb0, 128)) = pack4(mul4(qq, r));
+        // Q+ = q (.) r_t; for the pre-update read-out q (.) r_{t-1} = q (.) r_t / alpha_t
+        *reinterpret_cast<uint2*>(kq + canon(64 + j, cb0, 128)) = pack4(pre ? mul4(qq, mul4(r, rcp4(al[i]))) : mul4(qq, r));
         uint2 hi, lo;
         split4(mul4(mul4(ws[i], kk), rinv), hi, lo);
         *reinterpret_cast<uint2*>(sm + Ly::WHI + canon(j, cb0, C)) = hi;
@@ -425,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q8 = 0; q8 < 4; ++q8) {
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = (i0 + 8 * q8 + e <= t) ? x[8 * q8 + e] : 0.f;
+          for (int e = 0; e < 8; ++e) y[e] = (i0 + 8 * q8 + e <= t - pre) ? x[8 * q8 + e] : 0.f;
           uint4 pk = make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
                                 pack_bf16(y[6], y[7]));
           *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(64 + t, i0 / 8 + q8, 128)) = pk;

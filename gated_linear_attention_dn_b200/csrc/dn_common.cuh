@@ -19,6 +19,7 @@ struct Args {
   int B, T, H, dk, dv, chunk;
   int io_bf16;                    // 1: q/k/v/o are bf16, 0: fp32
   int alpha, beta_k, beta_v, key_scale;   // dn_gate modes
+  int pre_read;                   // 1: o_t = S_{t-1}^T q_t (before the token's update)
   const void* q;
   const void* k;
   const void* v;

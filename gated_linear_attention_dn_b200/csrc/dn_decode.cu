@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Args a) {
   const int col0 = (blockIdx.x % slices) * kCols;
   const int tid = threadIdx.x;
   const int c4 = tid & 15;
+  const bool pre = a.pre_read != 0;
   const int rg = tid >> 4;
 
   __shared__ float s_alpha[DK], s_k[DK], s_q[DK], s_w[DK];
@@ -70,6 +71,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Args a) {
   for (int j = 0; j < RPT; ++j) {
     const int i = rg + 16 * j;
     const float al = s_alpha[i], kk = s_k[i], qq = s_q[i];
+    // s = S^T q from the state before the decay (pre-update read-out) or after it
+    const float sq = pre ? qq : qq * al;
+    s[0] = fmaf(x[j].x, sq, s[0]);
+    s[1] = fmaf(x[j].y, sq, s[1]);
+    s[2] = fmaf(x[j].z, sq, s[2]);
+    s[3] = fmaf(x[j].w, sq, s[3]);
     x[j].x *= al;
     x[j].y *= al;
     x[j].z *= al;
@@ -78,10 +85,6 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Args a) {
     r[1] = fmaf(x[j].y, kk, r[1]);
     r[2] = fmaf(x[j].z, kk, r[2]);
     r[3] = fmaf(x[j].w, kk, r[3]);
-    s[0] = fmaf(x[j].x, qq, s[0]);
-    s[1] = fmaf(x[j].y, qq, s[1]);
-    s[2] = fmaf(x[j].z, qq, s[2]);
-    s[3] = fmaf(x[j].w, qq, s[3]);
   }
   // reduce the two row groups that share a warp, then across the 8 warps
 #pragma unroll
@@ -114,7 +117,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Args a) {
     const float bv = gate_load(a.beta_v_p, a.beta_v, bh, dv, col);
     const float u = bv * vv - rr;
     s_u[j] = u;
-    io_store(a.o, (int64_t)bh * dv + col, fmaf(u, wq, ss), a.io_bf16);
+    io_store(a.o, (int64_t)bh * dv + col, pre ? ss : fmaf(u, wq, ss), a.io_bf16);
   }
   __syncthreads();
   const float u0 = s_u[4 * c4 + 0], u1 = s_u[4 * c4 + 1], u2 = s_u[4 * c4 + 2], u3 = s_u[4 * c4 + 3];

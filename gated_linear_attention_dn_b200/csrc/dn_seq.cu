@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(kThreads) seq_fwd_kernel(Args a) {
   const int col0 = (blockIdx.x % slices) * kCols;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c4 = tid & 7, rg = tid >> 3;
+  const bool pre = a.pre_read != 0;
 
   __shared__ float s_k[kTT][DK], s_q[kTT][DK], s_al[kTT][DK], s_w[kTT][DK];
   __shared__ float s_v[kTT][kCols];
@@ -80,6 +81,12 @@ __global__ void __launch_bounds__(kThreads) seq_fwd_kernel(Args a) {
       for (int j = 0; j < RPT; ++j) {
         const int i = rg + 32 * j;
         const float al = s_al[t][i], kk = s_k[t][i], qq = s_q[t][i];
+        // s = S^T q from the state before the decay (pre-update read-out) or after it
+        const float sq = pre ? qq : qq * al;
+        s[0] = fmaf(x[j].x, sq, s[0]);
+        s[1] = fmaf(x[j].y, sq, s[1]);
+        s[2] = fmaf(x[j].z, sq, s[2]);
+        s[3] = fmaf(x[j].w, sq, s[3]);
         x[j].x *= al;
         x[j].y *= al;
         x[j].z *= al;
@@ -88,10 +95,6 @@ __global__ void __launch_bounds__(kThreads) seq_fwd_kernel(Args a) {
         r[1] = fmaf(x[j].y, kk, r[1]);
         r[2] = fmaf(x[j].z, kk, r[2]);
         r[3] = fmaf(x[j].w, kk, r[3]);
-        s[0] = fmaf(x[j].x, qq, s[0]);
-        s[1] = fmaf(x[j].y, qq, s[1]);
-        s[2] = fmaf(x[j].z, qq, s[2]);
-        s[3] = fmaf(x[j].w, qq, s[3]);
       }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kThreads) seq_fwd_kernel(Args a) {
         const float u = s_v[t][tid] - rr;
         s_u[tid] = u;
         const int64_t tok = ((int64_t)b * T + t0 + t) * H + h;
-        io_store(a.o, tok * dv + col0 + tid, fmaf(u, s_wq[t], ss), a.io_bf16);
+        io_store(a.o, tok * dv + col0 + tid, pre ? ss : fmaf(u, s_wq[t], ss), a.io_bf16);
       }
       __syncthreads();
       const float u0 = s_u[4 * c4], u1 = s_u[4 * c4 + 1], u2 = s_u[4 * c4 + 2], u3 = s_u[4 * c4 + 3];

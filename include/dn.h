@@ -79,6 +79,16 @@ typedef enum { DN_F32 = 0, DN_BF16 = 1 } dn_dtype;
 /* How a gate is given: absent (1), one value per (b, t, h), or one per channel. */
 typedef enum { DN_GATE_ONE = 0, DN_GATE_SCALAR = 1, DN_GATE_CHANNEL = 2 } dn_gate;
 
+/*
+ * When o_t reads the state. DN_READ_POST: o_t = S_t^T q_t, after the token's update (the
+ * default). DN_READ_PRE: o_t = S_{t-1}^T q_t, before the token's decay and write -- the read of
+ * the delta-mem page (section 2.C, r_t = S_{t-1} q^m_t). delta-mem's update
+ * S_t = lambda_t S_{t-1} + beta_t (v_t - S_{t-1} k_t) k_t^T (section 2.A; undecayed residual) is
+ * this recurrence with alpha = lambda, beta^k = beta / lambda, beta^v = lambda (lambda > 0).
+ * DN_READ_PRE needs alpha > 0 on the chunk path (it divides by the token's own decay).
+ */
+typedef enum { DN_READ_POST = 0, DN_READ_PRE = 1 } dn_readout;
+
 typedef struct {
   int B, T, H;        /* batch, tokens per sequence, heads; B, H >= 1, T >= 0 */
   int d_k, d_v;       /* head dims; supported: d_k, d_v in {64, 128} */
@@ -88,6 +98,7 @@ typedef struct {
   dn_gate beta_k;     /* erase / write strength on the key side (GDN beta; FG2-GDN+ beta^k) */
   dn_gate beta_v;     /* write strength on the value side (FG2-GDN+ beta^v); CHANNEL means d_v wide */
   dn_gate key_scale;  /* OSDN preconditioner d_t on the write key; CHANNEL means d_k wide */
+  dn_readout readout; /* read-out after (default, 0) or before the token's update */
 } dn_desc;
 
 /*

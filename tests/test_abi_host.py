@@ -84,6 +84,7 @@ def test_rejects_bad_descriptors(lib):
     assert _call(lib, _desc(d_k=96)) == dn.DN_ERR_UNSUPPORTED
     assert _call(lib, _desc(d_v=256)) == dn.DN_ERR_UNSUPPORTED
     assert _call(lib, _desc(chunk=32)) == dn.DN_ERR_UNSUPPORTED
+    assert _call(lib, _desc(readout=2)) == dn.DN_ERR_INVALID_ARGUMENT
 
 
 def test_rejects_bad_pointers(lib):
