@@ -71,6 +71,22 @@ def osdn_bytes(w: di.Workload) -> int:
     return ntok * w.dk * es + 2 * ntok * 4 + ntok * w.dk * 4 + w.B * w.H * w.dk * 4
 
 
+def reduce_max(value: float, world: int, device: str = "cuda") -> float:
+    """Max over ranks of a per-rank time: the slowest rank sets a multi-rank step's time."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput when every rank processes `units_per_rank` in (max-over-ranks) `ms`."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -369,13 +385,9 @@ def main():
     total_ms = evs[0].elapsed_time(evs[-1])
     if dn.dn_stream_status(stream) != dn.DN_OK:
         raise RuntimeError("device status after timed region")
-    t_max = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms = float(t_max.item())
+    total_ms = reduce_max(total_ms, world)
     ms_per_step = total_ms / args.steps
-    tokens = B * T * world * args.steps
-    value = tokens / (total_ms * 1e-3)
+    value = weak_scaling_rate(B * T * args.steps, world, total_ms)
     kern_ms = statistics.mean(per_launch_ms)
     alg = algorithmic_bytes(w)
     achieved = alg / (kern_ms * 1e-3) / 1e9
@@ -410,10 +422,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-    e2e = {"value": B * T * world * e_steps / (float(e_ms.item()) * 1e-3), "unit": "tokens/s",
+    e_ms = reduce_max(e0.elapsed_time(e1), world)
+    e2e = {"value": weak_scaling_rate(B * T * e_steps, world, e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del pin
 
@@ -447,11 +457,11 @@ def main():
         if dn.dn_stream_status(stream) != dn.DN_OK:
             raise RuntimeError("device status after decode")
         dms = [devs[i].elapsed_time(devs[i + 1]) for i in range(nd)]
-        d_ms = statistics.mean(dms)
+        d_ms = reduce_max(statistics.mean(dms), world)
         db = decode_bytes(wd)
         gbs = db / (d_ms * 1e-3) / 1e9
         decode = {"workload": "decode 1024 seq x 32 heads, d=128, fp32 state 2 GiB in place, channel gates",
-                  "steps": nd, "ms_per_step": d_ms, "tokens_per_s": wd.B * world / (d_ms * 1e-3),
+                  "steps": nd, "ms_per_step": d_ms, "tokens_per_s": weak_scaling_rate(wd.B, world, d_ms),
                   "GB/s": gbs * world,
                   "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                "frac": gbs / peaks["hbm_gbs"], "traffic": recorded_traffic("decode"),
@@ -494,7 +504,7 @@ def main():
                 fn()
             a1.record(stream)
             torch.cuda.synchronize()
-            return a0.elapsed_time(a1) / n
+            return reduce_max(a0.elapsed_time(a1) / n, world)
 
         o_ms = timed(ostep, 10)
         f_ms = timed(fstep, 3)
@@ -504,7 +514,7 @@ def main():
         ogbs = ob / (o_ms * 1e-3) / 1e9
         osdn = {"workload": "OSDN preconditioner scan, B=2 H=16 T=32768 d_k=128 (fg2_osdn_long's keys), "
                             "scalar beta, retention, eta=0.5",
-                "ms_per_call": o_ms, "tokens_per_s": wo.B * wo.T * world / (o_ms * 1e-3),
+                "ms_per_call": o_ms, "tokens_per_s": weak_scaling_rate(wo.B * wo.T, world, o_ms),
                 "chunk_fwd_ms_same_keys": f_ms, "scan_over_chunk_fwd": o_ms / f_ms,
                 "roofline": {"bound": "hbm", "achieved": ogbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": ogbs / peaks["hbm_gbs"], "traffic": recorded_traffic("osdn"),
