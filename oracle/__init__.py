@@ -189,3 +189,4 @@ def rel_l2(x, ref) -> float:
 
 
 from . import chunked  # noqa: E402  (NumPy chunked evaluation, test-only)
+from . import memcache  # noqa: E402  (Memory Caching over the recurrence, test-only)
