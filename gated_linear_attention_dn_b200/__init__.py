@@ -12,6 +12,8 @@ Entry points (same names as the C ABI):
                    S=..., o=None, stream=None) -> o          (S updated in place)
     dn_osdn_precond(k, beta, retention=None, d0=None, eta=0.5, d=None, d_T=None,
                     workspace=None, stream=None) -> (d, d_T)   (OSDN phase 1)
+    dn_mc_readout(q, M, gates=None, o=..., seg_len=L, stream=None) -> o     (Memory Caching read-out)
+    mc_fwd(q, k, v, ..., seg_len=L, gates=None) -> (o, M)   (segments + cached read-out)
     dn_stream_status(stream=None) -> int
     dn_status_string(code) -> str
 
@@ -37,7 +39,7 @@ DN_READ_POST, DN_READ_PRE = 0, 1
 _READOUT = {"post": DN_READ_POST, "pre": DN_READ_PRE}
 
 EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_osdn_precond_workspace_bytes",
-            "dn_osdn_precond", "dn_stream_status", "dn_status_string", "dn_version")
+            "dn_osdn_precond", "dn_mc_readout", "dn_stream_status", "dn_status_string", "dn_version")
 
 
 class DnDesc(ctypes.Structure):
@@ -50,6 +52,11 @@ class DnDesc(ctypes.Structure):
 class DnOsdnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
                 ("io_dtype", ctypes.c_int), ("eta", ctypes.c_float)]
+
+
+class DnMcDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
+                ("d_v", ctypes.c_int), ("seg_len", ctypes.c_int), ("io_dtype", ctypes.c_int)]
 
 
 class DnError(RuntimeError):
@@ -82,6 +89,8 @@ def load(path: str = LIB_PATH):
     lib.dn_osdn_precond_workspace_bytes.restype = ctypes.c_size_t
     lib.dn_osdn_precond.argtypes = [O, P, P, P, P, P, P, P, ctypes.c_size_t, P]
     lib.dn_osdn_precond.restype = I
+    lib.dn_mc_readout.argtypes = [ctypes.POINTER(DnMcDesc), P, P, P, P, P]
+    lib.dn_mc_readout.restype = I
     lib.dn_stream_status.argtypes = [P]
     lib.dn_stream_status.restype = I
     lib.dn_status_string.argtypes = [I]
@@ -226,6 +235,49 @@ def dn_osdn_precond(k, beta, retention=None, d0=None, eta: float = 0.5, d=None, 
     if rc != DN_OK:
         raise DnError(rc, "dn_osdn_precond")
     return d, d_T
+
+
+def dn_mc_readout(q, M, gates=None, o=None, seg_len: int = 64, stream=None):
+    """o [B,T,H,d_v] += sum_{s < t // seg_len} gates[b,t,h,s] M[b,s,h]^T q_t, in place (gates None: 1)."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = M.shape[-1]
+    io = DN_BF16 if q.dtype == torch.bfloat16 else DN_F32
+    if o is None or not o.is_contiguous() or o.dtype != q.dtype or tuple(o.shape) != (B, T, H, dv):
+        raise ValueError("o must be a contiguous [B,T,H,d_v] tensor of q's dtype (it is accumulated into)")
+    N = (T + seg_len - 1) // seg_len
+    if M.dtype != torch.float32 or not M.is_contiguous() or tuple(M.shape) != (B, N, H, dk, dv):
+        raise ValueError(f"M must be a contiguous float32 tensor of shape {(B, N, H, dk, dv)}")
+    if gates is not None and (gates.dtype != torch.float32 or not gates.is_contiguous()
+                              or tuple(gates.shape) != (B, T, H, N)):
+        raise ValueError(f"gates must be a contiguous float32 tensor of shape {(B, T, H, N)}")
+    desc = DnMcDesc(B, T, H, dk, dv, seg_len, io)
+    rc = lib.dn_mc_readout(ctypes.byref(desc), _ptr(q), _ptr(M), _ptr(gates), _ptr(o), _stream_handle(stream))
+    if rc != DN_OK:
+        raise DnError(rc, "dn_mc_readout")
+    return o
+
+
+def mc_fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, seg_len: int = 64,
+           gates=None, readout: str = "post", stream=None):
+    """Memory Caching over the recurrence: every segment of seg_len tokens runs from S0 (or zero)
+    and its final state is cached; each token adds the gated read of the earlier segments'
+    memories. Returns (o [B,T,H,d_v], M [B,N,H,d_k,d_v]). T must be a multiple of seg_len."""
+    B, T, H, dk = q.shape
+    if seg_len <= 0 or T % seg_len:
+        raise ValueError("T must be a positive multiple of seg_len")
+    N = T // seg_len
+
+    def seg(x):  # [B, T, ...] -> [B*N, L, ...], the same memory
+        return None if x is None else x.view(B * N, seg_len, *x.shape[2:])
+
+    S0r = None if S0 is None else S0.repeat_interleave(N, dim=0).contiguous()
+    o, M = dn_chunk_fwd(seg(q), seg(k), seg(v), seg(alpha), seg(beta_k), seg(beta_v), seg(key_scale), S0r,
+                        stream=stream, readout=readout)
+    o = o.view(B, T, H, -1)
+    M = M.view(B, N, H, dk, -1)
+    dn_mc_readout(q, M, gates, o, seg_len, stream)
+    return o, M
 
 
 def dn_stream_status(stream=None) -> int:

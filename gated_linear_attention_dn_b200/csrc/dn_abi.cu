@@ -238,6 +238,29 @@ dn_status dn_osdn_precond(const dn_osdn_desc* desc, const void* k, const float* 
   return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
 
+dn_status dn_mc_readout(const dn_mc_desc* d, const void* q, const float* M, const float* gates, void* o,
+                        void* cuda_stream) {
+  if (!d) return DN_ERR_INVALID_ARGUMENT;
+  if (d->B < 1 || d->H < 1 || d->T < 0 || d->seg_len < 1) return DN_ERR_INVALID_ARGUMENT;
+  if (d->io_dtype != DN_F32 && d->io_dtype != DN_BF16) return DN_ERR_INVALID_ARGUMENT;
+  if (!((d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128))) return DN_ERR_UNSUPPORTED;
+  const int64_t tiles = (int64_t)d->B * d->H * ((d->T + 63) / 64);
+  if (tiles >= ((int64_t)1 << 31) || (int64_t)d->B * d->T * d->H * d->d_v >= ((int64_t)1 << 46))
+    return DN_ERR_UNSUPPORTED;
+  if (d->T <= d->seg_len) return DN_OK;  // no token has an earlier segment
+  if (!q || !M || !o) return DN_ERR_INVALID_ARGUMENT;
+  if (!aligned16(M)) return DN_ERR_MISALIGNED;
+  const size_t es = d->io_dtype == DN_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(o)) & (es - 1)) return DN_ERR_MISALIGNED;
+  if (gates && !aligned4(gates)) return DN_ERR_MISALIGNED;
+  const size_t n_o = (size_t)d->B * d->T * d->H * d->d_v * es;
+  const size_t n_q = (size_t)d->B * d->T * d->H * d->d_k * es;
+  if (ranges_overlap(o, n_o, q, n_q)) return DN_ERR_INVALID_ARGUMENT;
+  cudaError_t e = dn::launch_mc_readout(q, M, gates, o, d->B, d->T, d->H, d->d_k, d->d_v, d->seg_len,
+                                        d->io_dtype == DN_BF16, static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
+}
+
 dn_status dn_stream_status(void* cuda_stream) {
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return DN_ERR_CUDA;

@@ -43,6 +43,9 @@ cudaError_t launch_chunk_sc(const Args& a, cudaStream_t s);
 size_t osdn_workspace_bytes(int B, int T, int H);
 cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, const float* d0, float eta, int B,
                         int T, int H, int dk, int io_bf16, float* ws, float* dout, float* dT, cudaStream_t s);
+// Memory Caching read-out (dn_memcache.cu).
+cudaError_t launch_mc_readout(const void* q, const float* M, const float* gates, void* o, int B, int T, int H,
+                              int dk, int dv, int L, int bf16, cudaStream_t s);
 // Whether the tensor-core chunk kernels take this problem (else the sequential kernel does).
 bool chunk_tc_supported(const Args& a);
 // TMA tensor map over a [B, T, H, d] bf16 tensor, 128-byte swizzle, box of 64 channels x 1 head x

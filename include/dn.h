@@ -199,6 +199,33 @@ dn_status dn_osdn_precond_noalloc(const dn_osdn_desc* desc, const void* k, const
                                   void* cuda_stream);
 
 /*
+ * Memory Caching read-out (Memory Caching page, section 2 "retrieval" and section 3: the
+ * residual memory and the gated residual memory): the sequence is cut into segments of L
+ * tokens, every segment's memory runs the recurrence from the initial state, and its final
+ * state M_s is cached; a token t of segment j = t / L adds the gated read of the earlier
+ * segments' memories to its own output:
+ *
+ *   o_t += sum_{s < j} g[b, t, h, s] M_s^T q_t          (g = 1 when gates is NULL)
+ *
+ * The online part and the cache come from dn_chunk_fwd on the sequence viewed as B * N
+ * sequences of L tokens (q, k, v, gates as [B*N, L, H, d] views of the same memory when T is a
+ * multiple of L): its o is the online read-out and its S_T is M [B, N, H, d_k, d_v].
+ *
+ * In:  q [B,T,H,d_k] (io dtype), M [B,N,H,d_k,d_v] fp32 (N = ceil(T / seg_len)), gates
+ *      [B,T,H,N] fp32 or NULL.   In/out: o [B,T,H,d_v] (io dtype), accumulated in place.
+ * Supported: d_k, d_v in {64, 128}; M 16-byte aligned. fp32 arithmetic.
+ */
+typedef struct {
+  int B, T, H;        /* B, H >= 1, T >= 0 */
+  int d_k, d_v;       /* 64 or 128 each */
+  int seg_len;        /* L >= 1 */
+  dn_dtype io_dtype;  /* dtype of q and o */
+} dn_mc_desc;
+
+dn_status dn_mc_readout(const dn_mc_desc* desc, const void* q, const float* M, const float* gates, void* o,
+                        void* cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reports (and clears) the device status word
  * that kernels set when a bounded wait gives up (DN_ERR_DEVICE_TIMEOUT), or
  * DN_ERR_CUDA if the stream holds a CUDA error. DN_OK otherwise.

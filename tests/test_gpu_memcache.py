@@ -1,0 +1,62 @@
+"""GPU parity of Memory Caching (segment memories by dn_chunk_fwd on the segment view, cached
+read-out by dn_mc_readout) against the fp64 oracle (oracle/memcache.py), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import dn_inputs as di
+import gated_linear_attention_dn_b200 as dn
+import oracle
+from tests.gpu_util import TOL, dev, host_f64, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(name, L, gated, **kw):
+    w = di.WORKLOADS[name].scaled(**kw)
+    x = di.make_inputs(w)
+    N = w.T // L
+    g = None
+    if gated:
+        g = np.random.default_rng(7).uniform(0.0, 1.0, (w.B, w.T, w.H, N)).astype(np.float32)
+    return w, x, g
+
+
+@pytest.mark.parametrize("name,L,gated,kw", [
+    ("gdn_prefill", 256, True, dict(B=1, H=2, T=1024)),
+    ("gdn_prefill", 128, False, dict(B=2, H=2, T=512)),
+    ("kda", 192, True, dict(B=1, H=2, T=576)),
+    ("gdn_fp32_small", 64, True, dict(T=256)),
+])
+def test_mc_fwd_matches_oracle(name, L, gated, kw):
+    w, x, g = _case(name, L, gated, **kw)
+    xd = to_device(x)
+    o, M = dn.mc_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"], xd["S0"],
+                     seg_len=L, gates=dev(g))
+    assert dn.dn_stream_status() == dn.DN_OK
+    o_ref, M_ref = oracle.memcache.mc_fwd(**x, seg_len=L, gates=g)
+    tol = TOL[w.io]
+    eo, eM = oracle.rel_l2(host_f64(o), o_ref), oracle.rel_l2(host_f64(M), M_ref)
+    print(f"[parity] mc o rel-L2 {eo:.3e} (tol {tol['o']:.0e}), M rel-L2 {eM:.3e} (tol {tol['S']:.0e})")
+    assert eo <= tol["o"] and eM <= tol["S"]
+
+
+def test_readout_alone_fp32():
+    """The cached read-out by itself, on exact fp32 memories, against the sum written out."""
+    r = np.random.default_rng(3)
+    B, T, H, dk, dv, L = 2, 320, 3, 128, 64, 64
+    N = T // L
+    q = r.standard_normal((B, T, H, dk)).astype(np.float32)
+    M = r.standard_normal((B, N, H, dk, dv)).astype(np.float32) * 0.1
+    g = r.uniform(0, 1, (B, T, H, N)).astype(np.float32)
+    o0 = r.standard_normal((B, T, H, dv)).astype(np.float32)
+    o = dev(o0.copy())
+    dn.dn_mc_readout(dev(q), dev(M), dev(g), o, seg_len=L)
+    assert dn.dn_stream_status() == dn.DN_OK
+    ref = o0.astype(np.float64)
+    for t in range(T):
+        for s in range(t // L):
+            ref[:, t] += g[:, t, :, s][..., None] * np.einsum("bhk,bhkv->bhv", q[:, t].astype(np.float64), M[:, s])
+    err = oracle.rel_l2(host_f64(o), ref)
+    print(f"[parity] mc read-out rel-L2 {err:.3e}")
+    assert err <= 1e-5
