@@ -304,6 +304,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-osdn", action="store_true", help="skip the OSDN preconditioner scan leg")
+    ap.add_argument("--no-mc", action="store_true", help="skip the Memory Caching leg")
     ap.add_argument("--decode-steps", type=int, default=100)
     ap.add_argument("--only", choices=["chunk", "decode"], default=None,
                     help="profiling mode: run just one kernel on the workload with batch --batch")
@@ -522,6 +523,55 @@ def main():
         launches += 2 * 10 + 3  # timed: 10 scans of two kernels, 3 chunked passes
         del ko, bo, ro, do, dTo, wso, xf, Sf, of
 
+    # ---- Memory Caching on the prefill workload: 4 segments of 1024 tokens, residual memory
+    mc = None
+    if not args.no_mc:
+        L = 1024
+        nseg = T // L
+        Mc = torch.empty((B * nseg, H, dk, dv), dtype=torch.float32, device="cuda")
+
+        def seg(t):
+            return None if t is None else t.view(B * nseg, L, *t.shape[2:])
+
+        def mc_online():
+            dn.dn_chunk_fwd(seg(xd["q"]), seg(xd["k"]), seg(xd["v"]), seg(xd["alpha"]), seg(xd["beta_k"]),
+                            seg(xd["beta_v"]), seg(xd["key_scale"]), None, o=o.view(B * nseg, L, H, dv),
+                            S_T=Mc, stream=stream)
+
+        def mc_read():
+            dn.dn_mc_readout(xd["q"], Mc.view(B, nseg, H, dk, dv), None, o, seg_len=L, stream=stream)
+
+        def timed2(fn, n):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            a0.record(stream)
+            for _ in range(n):
+                fn()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            return reduce_max(a0.elapsed_time(a1) / n, world)
+
+        on_ms = timed2(mc_online, 10)
+        rd_ms = timed2(mc_read, 10)
+        if dn.dn_stream_status(stream) != dn.DN_OK:
+            raise RuntimeError("device status after Memory Caching")
+        # cached reads: a token of segment j reads j memories, 2 d_k d_v flops each
+        flops = B * H * sum(j * L for j in range(nseg)) * 2 * dk * dv
+        fp32_peak = 148 * 4 * 32 * 2 * 1.965e9 / 1e12  # FFMA lanes x 2 flops x max clock, TFLOP/s
+        tf = flops / (rd_ms * 1e-3) / 1e12
+        mc = {"workload": "Memory Caching on gdn_prefill: 4 segments of 1024 tokens, residual memory",
+              "online_ms": on_ms, "readout_ms": rd_ms, "total_ms": on_ms + rd_ms,
+              "tokens_per_s": weak_scaling_rate(B * T, world, on_ms + rd_ms),
+              "readout_roofline": {"bound": "alu", "achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s",
+                                   "frac": tf / fp32_peak, "traffic": None,
+                                   "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flops x 1.965 GHz",
+                                   "algorithmic_flops_per_launch": flops}}
+        launches += 10 + 10
+        del Mc
+
     clocks.__exit__(None, None, None)
 
     cpu = None
@@ -542,6 +592,7 @@ def main():
             "config": bench_config(world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode, "osdn_phase1": osdn,
+            "memory_caching": mc,
             "kernel_source": {k: kernel_source_hash(k) for k in KERNEL_SOURCES},
         }
         print(json.dumps(line), flush=True)

@@ -598,8 +598,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       // ---- X3: T = (I + A)^{-1} -> T Diag(r) (TP rows 0..63) and T Diag(beta^v) (STQ rows 0..63)
-      unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt, kBarXform,
-                                         bv_split);
+      if (bv_split)
+        unit_lower_inverse<true, 8, false, true>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt,
+                                                 kBarXform);
+      else
+        unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt,
+                                           kBarXform);
       fence_proxy_async();
       group_sync(kBarXform, kXformThreads);
       if (gt == 0) mbar_arrive(&bar_tready);

@@ -98,14 +98,13 @@ __device__ __forceinline__ void warp_store(const float* d, FW W, int lane) {
 // cs_c[i] when SC) and, when SC, T Diag(cs_v) into tile tt. Elements above the 8x8 block diagonal
 // are not written (their zeros are set once by the caller). The fp32 blocks above the diagonal
 // that the merges read are zeroed here when ZERO (sT shares memory with other data), else the
-// caller keeps them zero. When SC and tt_lo, the bf16 rounding residue of T Diag(cs_v) is written
+// caller keeps them zero. When SC and TT_LO, the bf16 rounding residue of T Diag(cs_v) is written
 // too, into rows 64..127 of tile tt (so that hi + lo carries about 16 mantissa bits). scr: 2048
 // floats of scratch.
 // Not inlined: it gets its own register budget.
-template <bool SC, int NW, bool ZERO = true>
+template <bool SC, int NW, bool ZERO = true, bool TT_LO = false>
 __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, float* scr, uint8_t* tp, uint8_t* tt,
-                                                const float* cs_c, const float* cs_v, int tid, int bar_id,
-                                                bool tt_lo = false) {
+                                                const float* cs_c, const float* cs_v, int tid, int bar_id) {
   static_assert(NW >= 4 && NW <= 8, "warp count");
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
   auto sync = [&] { group_sync(bar_id, 32 * NW); };
@@ -117,17 +116,19 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
       const float x = v * cs_v[i];
       const __nv_bfloat16 hi = __float2bfloat16_rn(x);
       *reinterpret_cast<__nv_bfloat16*>(tt + off) = hi;
-      if (tt_lo) *reinterpret_cast<__nv_bfloat16*>(tt + kLoRows + off) = __float2bfloat16_rn(x - __bfloat162float(hi));
+      if (TT_LO) *reinterpret_cast<__nv_bfloat16*>(tt + kLoRows + off) = __float2bfloat16_rn(x - __bfloat162float(hi));
     }
   };
   auto emit2 = [&](int t, int i, float v0, float v1) {  // columns i, i + 1 (i even)
     const uint32_t off = canon(t, i, 128);
     *reinterpret_cast<uint32_t*>(tp + off) = pack_bf16(SC ? v0 * cs_c[i] : v0, SC ? v1 * cs_c[i + 1] : v1);
-    if (SC) {
+    if (SC && TT_LO) {
       uint32_t hi, lo;
       tc::split_bf16(v0 * cs_v[i], v1 * cs_v[i + 1], hi, lo);
       *reinterpret_cast<uint32_t*>(tt + off) = hi;
-      if (tt_lo) *reinterpret_cast<uint32_t*>(tt + kLoRows + off) = lo;
+      *reinterpret_cast<uint32_t*>(tt + kLoRows + off) = lo;
+    } else if (SC) {
+      *reinterpret_cast<uint32_t*>(tt + off) = pack_bf16(v0 * cs_v[i], v1 * cs_v[i + 1]);
     }
   };
   if (tid < 64) {
