@@ -100,7 +100,7 @@ def measured_peaks() -> dict:
 KERNEL_SOURCES = {
     "chunk_fwd": ["dn_chunk_sc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
     "decode": ["dn_decode.cu", "dn_common.cuh"],
-    "osdn": ["dn_osdn.cu", "dn_common.cuh"],
+    "osdn": ["dn_osdn.cu", "dn_tc_ptx.cuh", "dn_common.cuh"],
 }
 
 
