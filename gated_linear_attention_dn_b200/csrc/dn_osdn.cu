@@ -15,9 +15,10 @@
 //   => e = u0 - B P,  u0 = T c,  B = T Diag(c beta rho),  T = (I + Diag(c beta) W)^{-1}.
 // u0 and B do not depend on d, so they are formed for all blocks of all heads at once
 // (osdn_block_kernel, one warp per block, into the caller's workspace). The scan
-// (osdn_scan_kernel, one CTA per (b, h), one thread per key channel) then needs per block only
-// P (a transposed warp reduction), e = u0 - B P (one warp), and the per-channel recurrence that
-// writes d_t for the 32 tokens; the block's k tile, B and u0 are loaded one block ahead.
+// (osdn_scan_kernel, one CTA per (b, h), two threads per key channel) then needs per block only
+// P (transposed warp reductions), e = u0 - B P (one warp), and the per-channel recurrences that
+// write d_t for the 32 tokens, in two halves of 16 that run at once; the next blocks' k tiles,
+// B and u0 arrive ahead through a cp.async ring.
 #include <mutex>
 
 #include "dn_common.cuh"
@@ -169,7 +170,9 @@ __global__ void __launch_bounds__(128) osdn_block_kernel(const void* k, const fl
 }
 
 // ------------------------------------------------------------------ scan kernel
-// One CTA of DK threads per (b, h); thread ch owns key channel ch of d. A ring of kStages shared-
+// One CTA of 2 DK threads per (b, h): thread (half, ch) owns key channel ch of d over tokens
+// 16 half .. +16 of every block (the second half starts from d at token 16, formed directly from the
+// block's start state, the first half's e and its k rows). A ring of kStages shared-
 // memory stages holds the k tile, B, u0 and retentions of the next blocks, copied with cp.async
 // kStages - 1 blocks ahead (one commit group per block, empty past the end, so that a fixed
 // wait_group count always means "this block's copies have landed").
@@ -186,67 +189,78 @@ struct ScanSmem {
 };
 
 template <int DK, bool BF16>
-__global__ void __launch_bounds__(DK) osdn_scan_kernel(const void* k, const float* ret, const float* d0, int B,
-                                                       int T, int H, const float* ws, float* dout, float* dT) {
+__global__ void __launch_bounds__(2 * DK) osdn_scan_kernel(const void* k, const float* ret, const float* d0, int B,
+                                                           int T, int H, const float* ws, float* dout, float* dT) {
   using namespace tc;
   using Sm = ScanSmem<DK, BF16>;
-  constexpr int NW = DK / 32;
+  constexpr int NT = 2 * DK;   // two threads per key channel: tokens 0..15 and 16..31 of a block
+  constexpr int NW = DK / 32;  // warps per half
+  constexpr int HM = kM / 2;
   constexpr int ES = BF16 ? 2 : 4, ROW = DK * ES, ROW_CHUNKS = ROW / 16;
   extern __shared__ __align__(16) float smem_raw[];  // same declaration type as the block kernel's
   uint8_t* const smem = reinterpret_cast<uint8_t*>(smem_raw);
-  __shared__ float s_part[NW][kM];
+  __shared__ float s_part[2][NW][HM];
   __shared__ float s_P[kM];
   __shared__ float s_e[kM];
-  const int ch = threadIdx.x, lane = ch & 31, warp = ch >> 5;
+  __shared__ float s_coef[HM];  // R(i + 1, 16) e_i: the first half's writes as seen at token 16
+  __shared__ float s_rho16;     // prod_{j < 16} r_j
+  __shared__ __align__(16) float s_d[DK];
+  const int tid = threadIdx.x, ch = tid % DK, half = tid / DK, lane = tid & 31, wih = (tid % DK) >> 5;
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   const int nblk = (T + kM - 1) / kM;
-  float d = d0 ? d0[(int64_t)bh * DK + ch] : 1.f;
   auto s_k = [&](int st) { return smem + st * Sm::STAGE; };
   auto s_bu = [&](int st) { return reinterpret_cast<float*>(smem + st * Sm::STAGE + Sm::KT); };
   auto s_r = [&](int st) { return reinterpret_cast<float*>(smem + st * Sm::STAGE + Sm::KT + Sm::BU); };
+  auto k_at = [&](int st, int t) -> float {
+    float x;
+    if (BF16)
+      x = __uint_as_float((uint32_t)reinterpret_cast<const unsigned short*>(s_k(st))[t * DK + ch] << 16);
+    else
+      x = reinterpret_cast<const float*>(s_k(st))[t * DK + ch];
+    return x;
+  };
 
   // copies of block j into stage j % kStages, committed as one group (an empty group past the end)
   auto issue = [&](int j) {
     if (j < nblk) {
       const int st = j % kStages, t0 = j * kM, nb = min(kM, T - t0);
       const uint8_t* kb = static_cast<const uint8_t*>(k);
-      for (int c = ch; c < kM * ROW_CHUNKS; c += DK) {
+      for (int c = tid; c < kM * ROW_CHUNKS; c += NT) {
         const int t = c / ROW_CHUNKS, part = c % ROW_CHUNKS;
         const bool v = t < nb;
         const uint8_t* src = v ? kb + (((int64_t)b * T + t0 + t) * H + h) * ROW + part * 16 : kb;
         cp_async_16_zfill(s_k(st) + t * ROW + part * 16, src, v ? 16u : 0u);
       }
       const float* wb = ws + ((int64_t)bh * nblk + j) * kBlockFloats;
-      for (int c = ch; c < kBlockFloats / 4; c += DK) cp_async_16_zfill(s_bu(st) + 4 * c, wb + 4 * c, 16u);
-      if (ret && ch < nb) cp_async_4(s_r(st) + ch, ret + ((int64_t)b * T + t0 + ch) * H + h);
+      for (int c = tid; c < kBlockFloats / 4; c += NT) cp_async_16_zfill(s_bu(st) + 4 * c, wb + 4 * c, 16u);
+      if (ret && tid < nb) cp_async_4(s_r(st) + tid, ret + ((int64_t)b * T + t0 + tid) * H + h);
     }
     cp_async_commit();
   };
 
+  if (half == 0) s_d[ch] = d0 ? d0[(int64_t)bh * DK + ch] : 1.f;
 #pragma unroll
   for (int j = 0; j < kStages - 1; ++j) issue(j);
   for (int j = 0; j < nblk; ++j) {
-    const int st = j % kStages, t0 = j * kM, nb = min(kM, T - t0);
+    const int st = j % kStages, t0 = j * kM, nb = min(kM, T - t0), tb = half * HM;
     cp_async_wait_group<kStages - 2>();
-    __syncthreads();             // block j's tiles have landed, and every thread is done with block j - 1
-    issue(j + kStages - 1);      // into the stage block j - 1 used
-    float a[kM];
+    __syncthreads();         // block j's tiles have landed; block j - 1 is done (its d_end is in s_d)
+    issue(j + kStages - 1);  // into the stage block j - 1 used
+    const float dstart = s_d[ch];
+    float a[HM];
 #pragma unroll
-    for (int t = 0; t < kM; ++t) {
-      float x;
-      if (BF16)
-        x = __uint_as_float((uint32_t)reinterpret_cast<const unsigned short*>(s_k(st))[t * DK + ch] << 16);
-      else
-        x = reinterpret_cast<const float*>(s_k(st))[t * DK + ch];
+    for (int t = 0; t < HM; ++t) {
+      const float x = k_at(st, tb + t);
       a[t] = x * x;
     }
-    // P_t = <d_{t0}, a_t>: per-warp partials by a transposed butterfly (lane t ends with token t)
+    // P_t = <d_{t0}, a_t> for this half's 16 tokens: a transposed butterfly over lanes 0..15's bit
+    // pattern, then one exchange across lane bit 4; lane t (mod 16) ends with token t
     {
-      float v[kM];
+      float v[HM];
 #pragma unroll
-      for (int t = 0; t < kM; ++t) v[t] = d * a[t];
+      for (int t = 0; t < HM; ++t) v[t] = dstart * a[t];
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
+      for (int off = 8; off >= 1; off >>= 1) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < off; ++i) {
@@ -255,14 +269,15 @@ __global__ void __launch_bounds__(DK) osdn_scan_kernel(const void* k, const floa
           v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
         }
       }
-      s_part[warp][lane] = v[0];
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+      if (lane < HM) s_part[half][wih][lane] = v[0];
     }
     __syncthreads();
-    // e = u0 - B P (warp 0, lane t; B column-major)
-    if (warp == 0) {
+    // e = u0 - B P (warp 0, lane t; B column-major), then the second half's start: R(i+1,16) e_i
+    if (tid < 32) {
       float P = 0.f;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) P += s_part[w][lane];
+      for (int w = 0; w < NW; ++w) P += s_part[lane / HM][w][lane % HM];
       s_P[lane] = P;
       __syncwarp();
       const float* bu = s_bu(st);
@@ -270,21 +285,47 @@ __global__ void __launch_bounds__(DK) osdn_scan_kernel(const void* k, const floa
 #pragma unroll
       for (int s2 = 0; s2 < kM; ++s2) e = fmaf(-bu[s2 * kM + lane], s_P[s2], e);
       s_e[lane] = e;
+      // suffix products over lanes 0..15: suf_i = prod_{i<j<16} r_j (exclusive), rho16 = prod_{j<16} r_j
+      const float rl = (ret && lane < HM) ? s_r(st)[lane] : 1.f;
+      float incl = lane < HM ? rl : 1.f;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_down_sync(0xffffffffu, incl, off);
+        if (lane + off < 32) incl *= y;
+      }
+      const float nxt = __shfl_down_sync(0xffffffffu, incl, 1);  // every lane takes part
+      const float suf = lane == 31 ? 1.f : nxt;
+      if (lane < HM) s_coef[lane] = suf * e;
+      if (lane == 0) s_rho16 = incl;
     }
     __syncthreads();
-    // d_t for the block's tokens, then d_{t0 + nb}
-    float* o = dout + (((int64_t)b * T + t0) * H + h) * DK + ch;
-    const float* rr = s_r(st);
+    // d_t for this half's tokens; the second half starts from d_{t0 + 16}
+    float d;
+    if (half == 0) {
+      d = dstart;
+    } else {
+      d = s_rho16 * dstart;
 #pragma unroll
-    for (int t = 0; t < kM; ++t) {
-      if (t < nb) {
-        o[(int64_t)t * H * DK] = d;
-        d = fmaf(ret ? rr[t] : 1.f, d, s_e[t] * a[t]);
+      for (int i = 0; i < HM; ++i) {
+        const float x = k_at(st, i);
+        d = fmaf(s_coef[i], x * x, d);
       }
     }
+    float* o = dout + (((int64_t)b * T + t0 + tb) * H + h) * DK + ch;
+    const float* rr = s_r(st);
+#pragma unroll
+    for (int t = 0; t < HM; ++t) {
+      if (tb + t < nb) {
+        o[(int64_t)t * H * DK] = d;
+        d = fmaf(ret ? rr[tb + t] : 1.f, d, s_e[tb + t] * a[t]);
+      }
+    }
+    // the block's final d: from the second half, or from the first when the block ends by token 16
+    if ((half == 1 && nb > HM) || (half == 0 && nb <= HM)) s_d[ch] = d;
   }
   cp_async_wait_all();
-  if (dT) dT[(int64_t)bh * DK + ch] = d;
+  __syncthreads();
+  if (dT && half == 0) dT[(int64_t)bh * DK + ch] = s_d[ch];
 }
 
 template <int DK, bool BF16>
@@ -294,7 +335,7 @@ cudaError_t launch_scan(const void* k, const float* ret, const float* d0, int B,
   cudaError_t e = cudaFuncSetAttribute(osdn_scan_kernel<DK, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Sm::BYTES);
   if (e != cudaSuccess) return e;
-  osdn_scan_kernel<DK, BF16><<<B * H, DK, Sm::BYTES, s>>>(k, ret, d0, B, T, H, ws, dout, dT);
+  osdn_scan_kernel<DK, BF16><<<B * H, 2 * DK, Sm::BYTES, s>>>(k, ret, d0, B, T, H, ws, dout, dT);
   return cudaGetLastError();
 }
 
