@@ -41,7 +41,9 @@ dn_status check_desc(const dn_desc* d, bool decode) {
     return DN_ERR_INVALID_ARGUMENT;
   if (d->chunk < 0) return DN_ERR_INVALID_ARGUMENT;
   if (d->readout != DN_READ_POST && d->readout != DN_READ_PRE) return DN_ERR_INVALID_ARGUMENT;
-  if (!((d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128))) return DN_ERR_UNSUPPORTED;
+  const bool big = (d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128);
+  const bool small = (d->d_k == 8 || d->d_k == 16) && (d->d_v == 8 || d->d_v == 16);
+  if (!big && !small) return DN_ERR_UNSUPPORTED;
   if (!(d->chunk == 0 || d->chunk == 64)) return DN_ERR_UNSUPPORTED;
   // sizes must stay addressable with 32-bit grid math and 64-bit offsets
   const int64_t heads = (int64_t)d->B * d->H;
@@ -160,7 +162,9 @@ dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const 
     return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
   }
   cudaError_t e;
-  if (a.io_bf16 && dn::chunk_tc_supported(a)) {
+  if (dn::small_state_supported(a)) {
+    e = dn::launch_small_state(a, s);
+  } else if (a.io_bf16 && dn::chunk_tc_supported(a)) {
     e = dn::launch_chunk_tc(a, s);
   } else {
     e = dn::launch_seq_fwd(a, s);
@@ -181,7 +185,8 @@ dn_status dn_decode_step(const dn_desc* desc, const void* q, const void* k, cons
   a.S0 = S;
   a.S = S;
   a.o = o;
-  cudaError_t e = dn::launch_decode(a, static_cast<cudaStream_t>(cuda_stream));
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = dn::small_state_supported(a) ? dn::launch_small_state(a, s) : dn::launch_decode(a, s);
   return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
 

@@ -46,6 +46,9 @@ cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, cons
 // Memory Caching read-out (dn_memcache.cu).
 cudaError_t launch_mc_readout(const void* q, const float* M, const float* gates, void* o, int B, int T, int H,
                               int dk, int dv, int L, int bf16, cudaStream_t s);
+// Small states (d_k, d_v in {8, 16}; dn_small.cu): chunk fwd and decode alike.
+bool small_state_supported(const Args& a);
+cudaError_t launch_small_state(const Args& a, cudaStream_t s);
 // Whether the tensor-core chunk kernels take this problem (else the sequential kernel does).
 bool chunk_tc_supported(const Args& a);
 // TMA tensor map over a [B, T, H, d] bf16 tensor, 128-byte swizzle, box of 64 channels x 1 head x

@@ -53,7 +53,9 @@
  *     that gives up is reported later by dn_stream_status.
  *   - Numerics: fp32 state, fp32 accumulation. bf16 io runs the tensor-core
  *     chunk kernel (bf16 operands; the state-update product uses a hi/lo bf16
- *     split); fp32 io runs an fp32 CUDA-core kernel.
+ *     split); fp32 io runs an fp32 CUDA-core kernel. Small states (d_k, d_v in
+ *     {8, 16}, e.g. the delta-mem page's 8 x 8 memory) run an fp32 CUDA-core
+ *     kernel with one warp per head, for the chunked call and the decode step.
  */
 #ifndef DN_H_
 #define DN_H_
@@ -91,7 +93,7 @@ typedef enum { DN_READ_POST = 0, DN_READ_PRE = 1 } dn_readout;
 
 typedef struct {
   int B, T, H;        /* batch, tokens per sequence, heads; B, H >= 1, T >= 0 */
-  int d_k, d_v;       /* head dims; supported: d_k, d_v in {64, 128} */
+  int d_k, d_v;       /* head dims; supported: d_k, d_v in {64, 128}, or both in {8, 16} (small states) */
   int chunk;          /* chunk length of the WY form; 0 selects the default, 64 (the only value supported) */
   dn_dtype io_dtype;  /* dtype of q, k, v and o */
   dn_gate alpha;      /* forget gate: scalar (GDN) or per key channel (KDA) */

@@ -85,6 +85,8 @@ def test_rejects_bad_descriptors(lib):
     assert _call(lib, _desc(d_v=256)) == dn.DN_ERR_UNSUPPORTED
     assert _call(lib, _desc(chunk=32)) == dn.DN_ERR_UNSUPPORTED
     assert _call(lib, _desc(readout=2)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(d_k=8, d_v=64)) == dn.DN_ERR_UNSUPPORTED  # small and large dims do not mix
+    assert _call(lib, _desc(d_k=32, d_v=32)) == dn.DN_ERR_UNSUPPORTED
 
 
 def test_rejects_bad_pointers(lib):
