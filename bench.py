@@ -257,11 +257,12 @@ def run_single_kernel(args):
 
     if not os.path.exists(dnbuild.LIB):
         dnbuild.build()
-    name = WORKLOAD if args.only == "chunk" else DECODE
+    name = {"chunk": WORKLOAD, "decode": DECODE, "osdn": "osdn_phase1"}[args.only]
     w = di.WORKLOADS[name]
     if args.batch:
         w = w.scaled(B=args.batch)
-    x = di.make_inputs(w)
+    x = di.make_osdn_inputs(w) if args.only == "osdn" else di.make_inputs(w)
+    eta = x.pop("eta", None)
 
     def to_dev(a):
         if a is None:
@@ -270,10 +271,12 @@ def run_single_kernel(args):
         return t.cuda()
 
     xd = {n: to_dev(a) for n, a in x.items()}
-    S = xd["S0"].clone() if xd["S0"] is not None else None
+    S = xd["S0"].clone() if xd.get("S0") is not None else None
 
     def launch():
-        if args.only == "chunk":
+        if args.only == "osdn":
+            dn.dn_osdn_precond(xd["k"], xd["beta"], xd["retention"], None, eta=eta)
+        elif args.only == "chunk":
             dn.dn_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
                             xd["S0"])
         else:
@@ -306,7 +309,7 @@ def main():
     ap.add_argument("--no-osdn", action="store_true", help="skip the OSDN preconditioner scan leg")
     ap.add_argument("--no-mc", action="store_true", help="skip the Memory Caching leg")
     ap.add_argument("--decode-steps", type=int, default=100)
-    ap.add_argument("--only", choices=["chunk", "decode"], default=None,
+    ap.add_argument("--only", choices=["chunk", "decode", "osdn"], default=None,
                     help="profiling mode: run just one kernel on the workload with batch --batch")
     ap.add_argument("--batch", type=int, default=0, help="with --only: batch size of the scaled workload")
     args = ap.parse_args()

@@ -8,7 +8,9 @@
 // One CTA (256 threads) per (b, h) and tile of 64 tokens: the tile's q rows sit in shared memory
 // as fp32; each memory M_s streams through shared memory in slabs of 16 rows; thread (ty, tx)
 // accumulates 4 tokens x (d_v / 16) columns in registers and weights each memory's contribution
-// by its tokens' gates (0 for a memory of the token's own or a later segment). fp32 throughout.
+// by its tokens' gates (0 for a memory of the token's own or a later segment). For the residual
+// memory on a tile inside one segment, the memories are summed while they are loaded and one
+// product serves them all. fp32 throughout.
 #include "dn_common.cuh"
 
 namespace dn {
@@ -47,14 +49,19 @@ __global__ void __launch_bounds__(256) mc_readout_kernel(const void* q, const fl
 #pragma unroll
     for (int c = 0; c < CPT; ++c) acc[r][c] = 0.f;
 
-  for (int s = 0; s < jmax; ++s) {
+  // residual memory over a tile that lies in one segment: every token reads the same memories,
+  // so their sum is formed while loading and one product serves them all
+  const bool summed = gates == nullptr && t0 / L == jmax;
+  const int passes = summed ? 1 : jmax;
+  for (int s = 0; s < passes; ++s) {
     __syncthreads();  // every thread is done with the previous memory's gates
     if (tid < kTok) {
       const int t = t0 + tid;
-      const bool reads = tid < nt && s < t / L;
+      const bool reads = tid < nt && (summed || s < t / L);
       s_g[tid] = reads ? (gates ? gates[(((int64_t)b * T + t) * H + h) * N + s] : 1.f) : 0.f;
     }
     const float* Ms = M + (((int64_t)b * N + s) * H + h) * DK * DV;
+    const int64_t mstride = (int64_t)H * DK * DV;  // from memory s to s + 1
     float tmp[4][CPT];
 #pragma unroll
     for (int r = 0; r < 4; ++r)
@@ -62,8 +69,16 @@ __global__ void __launch_bounds__(256) mc_readout_kernel(const void* q, const fl
       for (int c = 0; c < CPT; ++c) tmp[r][c] = 0.f;
     for (int k0 = 0; k0 < DK; k0 += kSlab) {
       __syncthreads();  // the previous slab (and, at k0 = 0, the q tile and gates) is settled
-      for (int e = tid; e < kSlab * DV / 4; e += 256)
-        reinterpret_cast<float4*>(&s_m[0][0])[e] = reinterpret_cast<const float4*>(Ms + (int64_t)k0 * DV)[e];
+      for (int e = tid; e < kSlab * DV / 4; e += 256) {
+        float4 m4 = reinterpret_cast<const float4*>(Ms + (int64_t)k0 * DV)[e];
+        if (summed) {
+          for (int s2 = 1; s2 < jmax; ++s2) {
+            const float4 y = reinterpret_cast<const float4*>(Ms + s2 * mstride + (int64_t)k0 * DV)[e];
+            m4.x += y.x, m4.y += y.y, m4.z += y.z, m4.w += y.w;
+          }
+        }
+        reinterpret_cast<float4*>(&s_m[0][0])[e] = m4;
+      }
       __syncthreads();
 #pragma unroll 4
       for (int kk = 0; kk < kSlab; ++kk) {
