@@ -11,6 +11,9 @@ Three evaluations live here, each independent of the CUDA path:
   oracle that parity tests compare the GPU against.
 * ``osdn_precond`` -- OSDN phase 1, the preconditioner sequence d_t that the
   OSDN key scale takes (sequential fp64 loop in the same C file).
+* ``bwd`` -- the reverse mode of the definition: the gradients of
+  sum <dO, o> + <dS_T, S_T> with respect to every input, by the chain rule
+  walked token by token from the end (same C file).
 * ``chunked.fwd`` -- the chunkwise-parallel (WY / UT-transform) evaluation of
   the same recurrence in NumPy fp64, following the chunk algebra the kernels
   use. It is never compared against the GPU; it exists so that tests can show
@@ -58,6 +61,9 @@ def _load():
             lib.dn_oracle_max_threads.restype = I
             lib.dn_oracle_osdn_heads.argtypes = [I, I, I, P, P, P, ctypes.c_double, P, P, I]
             lib.dn_oracle_osdn_heads.restype = I
+            lib.dn_oracle_bwd_heads.argtypes = [I, I, I, I, P, P, P, P, I, P, I, P, I, P, I, P, P, P, I,
+                                                P, P, P, P, P, P, P, P, I]
+            lib.dn_oracle_bwd_heads.restype = I
             _lib = lib
     return _lib
 
@@ -138,6 +144,79 @@ def fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None,
         o_full[b, :, h, :] = o[n]
         S_full[b, h] = S[n]
     return o_full, S_full
+
+
+def bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, dO=None, dS_T=None,
+        heads=None, nthreads: int = 0, readout: str = "post"):
+    """Reverse mode in fp64: the gradients of L = sum <dO, o> + <dS_T, S_T> (dS_T None: zero).
+
+    Returns a dict with the gradient of every input under its own name ("q", "k", "v", "alpha",
+    "beta_k", "beta_v", "key_scale", "S0"), each shaped like that input (None for an absent gate;
+    "S0" is always [B,H,dk,dv]). With ``heads=[(b, h), ...]`` only those run and the leading
+    [B,...,H] axes become one [NH] axis, as in ``fwd``.
+    """
+    q = np.asarray(q)
+    B, T, H, dk = q.shape
+    dv = np.asarray(v).shape[-1]
+    all_heads = heads is None
+    if all_heads:
+        heads = [(b, h) for b in range(B) for h in range(H)]
+    NH = len(heads)
+    qh, _ = _per_head(q, heads, dk)
+    kh, _ = _per_head(k, heads, dk)
+    vh, _ = _per_head(v, heads, dv)
+    dOh, _ = _per_head(dO, heads, dv)
+    qh, kh, vh, dOh = (x.reshape(NH, T, -1) for x in (qh, kh, vh, dOh))
+    gates = {}
+    for name, x, n in (("alpha", alpha, dk), ("beta_k", beta_k, dk), ("beta_v", beta_v, dv),
+                       ("key_scale", key_scale, dk)):
+        gates[name] = _per_head(x, heads, n)
+
+    def mats(x):
+        if x is None:
+            return None
+        x = np.asarray(x)
+        return np.ascontiguousarray(np.stack([widen(x[b, h]) for (b, h) in heads]))
+
+    S0h, dSTh = mats(S0), mats(dS_T)
+    out = {"q": np.zeros((NH, T, dk)), "k": np.zeros((NH, T, dk)), "v": np.zeros((NH, T, dv)),
+           "S0": np.zeros((NH, dk, dv))}
+    for name, (g, w) in gates.items():
+        out[name] = None if g is None else np.zeros((NH, T, w))
+
+    def ptr(a):
+        return None if a is None else a.ctypes.data
+
+    if readout not in ("post", "pre"):
+        raise ValueError("readout must be 'post' or 'pre'")
+    (ah, aw), (bkh, bkw), (bvh, bvw), (dh, dw) = (gates[n] for n in ("alpha", "beta_k", "beta_v", "key_scale"))
+    rc = _load().dn_oracle_bwd_heads(NH, T, dk, dv, ptr(qh), ptr(kh), ptr(vh), ptr(ah), aw, ptr(bkh), bkw,
+                                     ptr(bvh), bvw, ptr(dh), dw, ptr(S0h), ptr(dOh), ptr(dSTh),
+                                     int(readout == "pre"), ptr(out["q"]), ptr(out["k"]), ptr(out["v"]),
+                                     ptr(out["alpha"]), ptr(out["beta_k"]), ptr(out["beta_v"]),
+                                     ptr(out["key_scale"]), ptr(out["S0"]), nthreads)
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    for name, x in (("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v), ("key_scale", key_scale)):
+        if x is not None and np.asarray(x).ndim == 3:
+            out[name] = out[name][..., 0]
+    if not all_heads:
+        return out
+    full = {}
+    for name, g in out.items():
+        if g is None:
+            full[name] = None
+            continue
+        if name == "S0":
+            f = np.empty((B, H) + g.shape[1:])
+            for n, (b, h) in enumerate(heads):
+                f[b, h] = g[n]
+        else:
+            f = np.empty((B, T, H) + g.shape[2:])
+            for n, (b, h) in enumerate(heads):
+                f[b, :, h] = g[n]
+        full[name] = f
+    return full
 
 
 def osdn_precond(k, beta, retention=None, d0=None, eta: float = 0.5, heads=None, nthreads: int = 0):

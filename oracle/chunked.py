@@ -95,3 +95,113 @@ def fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, 
             o[b, :, h] = ob
             ST[b, h] = Sb
     return o, ST
+
+
+def head_bwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, dO, dS_T, C: int):
+    """Reverse mode of ``head_fwd`` (post read-out) in the same chunk algebra.
+
+    The chain rule through the chunk equations gives, with dS' the adjoint of the chunk-end state
+    and lam = e(g_n - g_m):
+      dX  = Diag(lam) dS'                          (adjoint of X = S_m + W-^T U)
+      dU  = lower-incl(Q+ W-^T)^T dO + W- dX
+      dV~ = T^T dU                                  (adjoint of V~ - K+ S_m, as U = T (V~ - K+ S_m))
+      dS_m = Q+^T dO + dX - K+^T dV~,    dS = Diag(e(g_m)) dS_m
+      dP  = lower-incl(dO U^T),          dL = -strictly-lower(dV~ U^T)
+      dQ+ = dO S_m^T + dP W-,    dK+ = -dV~ S_m^T + dL W-,    dW- = U dX^T + dP^T Q+ + dL^T K+
+    (dL uses T^T dT T^T with dT = dU ((I + L) U)^T, so T^T dT T^T = dV~ U^T.) The outputs do not
+    depend on the reference point g_m, so its adjoint terms cancel and g_m is held fixed: the
+    log-decay adjoint of token t is dh_t = Q+ (.) dQ+ + K+ (.) dK+ - W- (.) dW- (every channel), plus
+    rowsum(dX (.) X) at the chunk's last token, and d log alpha_s is the sum over t >= s in the chunk.
+
+    Returns a dict of per-token gradients shaped [T, n] for every gate (channel form) and
+    dS0 [dk, dv].
+    """
+    T, dk = q.shape
+    dv = v.shape[1]
+    S = np.array(S, dtype=np.float64, copy=True)
+    nc = (T + C - 1) // C
+    keep = []
+    for c in range(nc):  # forward, keeping what the reverse needs
+        c0, c1 = c * C, min(T, c * C + C)
+        n = c1 - c0
+        a = _gate(alpha, c0, c1, dk)
+        g = np.cumsum(np.log(a), axis=0)                  # g_t, t = 0..n-1 (after token t)
+        r = g[(n - 1) // 2]                               # the reference point, held fixed
+        eh = np.exp(g - r)
+        bkd = _gate(beta_k, c0, c1, dk) * _gate(key_scale, c0, c1, dk)
+        w = bkd * k[c0:c1]
+        Kp, Qp, Wm = k[c0:c1] * eh, q[c0:c1] * eh, w / eh
+        Vt = _gate(beta_v, c0, c1, dv) * v[c0:c1]
+        Sm = np.exp(r)[:, None] * S
+        Tm = np.linalg.inv(np.eye(n) + np.tril(Kp @ Wm.T, k=-1))
+        U = Tm @ (Vt - Kp @ Sm)
+        X = Sm + Wm.T @ U
+        lam = np.exp(g[-1] - r)
+        keep.append((c0, c1, a, eh, bkd, Kp, Qp, Wm, Tm, U, Sm, X, lam, r))
+        S = lam[:, None] * X
+    out = {n: np.zeros((T, w)) for n, w in (("q", dk), ("k", dk), ("v", dv), ("alpha", dk),
+                                               ("beta_k", dk), ("beta_v", dv), ("key_scale", dk))}
+    dS = np.zeros((dk, dv)) if dS_T is None else np.array(dS_T, dtype=np.float64)
+    for c in reversed(range(nc)):
+        c0, c1, a, eh, bkd, Kp, Qp, Wm, Tm, U, Sm, X, lam, r = keep[c]
+        dOc = dO[c0:c1]
+        dX = lam[:, None] * dS
+        P = np.tril(Qp @ Wm.T)
+        dU = P.T @ dOc + Wm @ dX
+        dVt = Tm.T @ dU
+        dS = np.exp(r)[:, None] * (Qp.T @ dOc + dX - Kp.T @ dVt)
+        dP = np.tril(dOc @ U.T)
+        dL = -np.tril(dVt @ U.T, k=-1)
+        dQp = dOc @ Sm.T + dP @ Wm
+        dKp = -dVt @ Sm.T + dL @ Wm
+        dWm = U @ dX.T + dP.T @ Qp + dL.T @ Kp
+        dh = Qp * dQp + Kp * dKp - Wm * dWm
+        dh[-1] += np.sum(dX * X, axis=1)
+        dlog = np.cumsum(dh[::-1], axis=0)[::-1]
+        dw = dWm / eh
+        kc, vc = k[c0:c1], v[c0:c1]
+        out["q"][c0:c1] = dQp * eh
+        out["k"][c0:c1] = dKp * eh + bkd * dw
+        out["alpha"][c0:c1] = dlog / a
+        out["beta_k"][c0:c1] = _gate(key_scale, c0, c1, dk) * kc * dw
+        out["key_scale"][c0:c1] = _gate(beta_k, c0, c1, dk) * kc * dw
+        out["v"][c0:c1] = _gate(beta_v, c0, c1, dv) * dVt
+        out["beta_v"][c0:c1] = vc * dVt
+    out["S0"] = dS
+    return out
+
+
+def bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, dO=None, dS_T=None,
+        C: int = 64):
+    """All heads, public layouts, post read-out: the gradients as ``oracle.bwd`` returns them."""
+    q = np.asarray(q, dtype=np.float64)
+    B, T, H, dk = q.shape
+    dv = np.asarray(v).shape[-1]
+
+    def sl(x, b, h):
+        if x is None:
+            return None
+        x = np.asarray(x, dtype=np.float64)
+        return x[b, :, h] if x.ndim == 3 else x[b, :, h, :]
+
+    gates = dict(alpha=alpha, beta_k=beta_k, beta_v=beta_v, key_scale=key_scale)
+    res = {"q": np.zeros((B, T, H, dk)), "k": np.zeros((B, T, H, dk)), "v": np.zeros((B, T, H, dv)),
+           "S0": np.zeros((B, H, dk, dv))}
+    for n, x in gates.items():
+        res[n] = None if x is None else np.zeros(np.shape(x))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float64)[b, h]
+            g = head_bwd(q[b, :, h], np.asarray(k, dtype=np.float64)[b, :, h],
+                         np.asarray(v, dtype=np.float64)[b, :, h], *(sl(gates[n], b, h) for n in gates), S,
+                         np.asarray(dO, dtype=np.float64)[b, :, h],
+                         None if dS_T is None else np.asarray(dS_T, dtype=np.float64)[b, h], C)
+            for n in ("q", "k", "v"):
+                res[n][b, :, h] = g[n]
+            res["S0"][b, h] = g["S0"]
+            for n, x in gates.items():
+                if x is None:
+                    continue
+                gn = g[n]
+                res[n][b, :, h] = gn.sum(axis=1) if np.ndim(x) == 3 else gn
+    return res
