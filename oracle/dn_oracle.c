@@ -243,11 +243,14 @@ static void fwd_token(int dk, int dv, const double* qt, const double* kt, const 
                       const double* S_prev, double* S_bar, double* w, double* u, double* S_t) {
   (void)qt;
   for (int i = 0; i < dk; ++i) {
-    const double a = gate(alpha, alpha_w, t, i);
-    for (int j = 0; j < dv; ++j) S_bar[(int64_t)i * dv + j] = a * S_prev[(int64_t)i * dv + j];
+    const double decay = gate(alpha, alpha_w, t, i);
+    for (int j = 0; j < dv; ++j) S_bar[(int64_t)i * dv + j] = decay * S_prev[(int64_t)i * dv + j];
   }
-  for (int i = 0; i < dk; ++i) w[i] = gate(beta_k, bk_w, t, i) * gate(key_scale, d_w, t, i) * kt[i];
-  for (int j = 0; j < dv; ++j) u[j] = gate(beta_v, bv_w, t, j) * vt[j];
+  for (int i = 0; i < dk; ++i) {
+    const double bkd = gate(beta_k, bk_w, t, i) * gate(key_scale, d_w, t, i);
+    w[i] = bkd * kt[i];
+  }
+  for (int j = 0; j < dv; ++j) u[j] = vt[j] * gate(beta_v, bv_w, t, j);
   for (int i = 0; i < dk; ++i)
     for (int j = 0; j < dv; ++j) u[j] -= S_bar[(int64_t)i * dv + j] * kt[i];
   for (int i = 0; i < dk; ++i)
@@ -363,12 +366,12 @@ int dn_oracle_bwd_head(int T, int dk, int dv, const double* q, const double* k, 
       }
       /* dS_bar = dS - k du^T; dalpha_i = <row i of dS_bar, row i of S_prev>; dS_prev = Diag(alpha) dS_bar */
       for (int i = 0; i < dk; ++i) {
-        const double a = gate(alpha, alpha_w, t, i);
+        const double decay = gate(alpha, alpha_w, t, i);
         double da = 0.0;
         for (int j = 0; j < dv; ++j) {
           const double dsb = dS[(int64_t)i * dv + j] - kt[i] * du[j];
           da += dsb * S_prev[(int64_t)i * dv + j];
-          dS[(int64_t)i * dv + j] = a * dsb;
+          dS[(int64_t)i * dv + j] = decay * dsb;
         }
         gate_grad(dalpha, alpha_w, t, i, da);
       }

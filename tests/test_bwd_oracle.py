@@ -186,7 +186,7 @@ MUTATIONS = {
     "value_gradient_without_beta_v": ("dvt[j] = gate(beta_v, bv_w, t, j) * du[j];", "dvt[j] = du[j];"),
     "post_read_uses_old_state": ("const double* S_read = pre_read ? S_prev : S_t;",
                                  "const double* S_read = S_prev;"),
-    "adjoint_not_decayed": ("dS[(int64_t)i * dv + j] = a * dsb;", "dS[(int64_t)i * dv + j] = dsb;"),
+    "adjoint_not_decayed": ("dS[(int64_t)i * dv + j] = decay * dsb;", "dS[(int64_t)i * dv + j] = dsb;"),
     "beta_k_gradient_without_d": ("gate_grad(dbeta_k, bk_w, t, i, dd * kt[i] * dw[i]);",
                                   "gate_grad(dbeta_k, bk_w, t, i, kt[i] * dw[i]);"),
 }
