@@ -71,6 +71,18 @@ def osdn_bytes(w: di.Workload) -> int:
     return ntok * w.dk * es + 2 * ntok * 4 + ntok * w.dk * 4 + w.B * w.H * w.dk * 4
 
 
+def bwd_flops(w: di.Workload, C: int = 64) -> int:
+    """Flops of one dn_chunk_bwd as its chunk algorithm states them (2 per multiply-add, every product
+    counted in full, triangular ones included), per chunk of C tokens:
+      9 C dk dv  (K+ S_m, W-^T U, W- dX, Q+^T dO, K+^T dV~, dO S_m^T, dV~ S_m^T, U dX^T, W-^T U for X)
+      6 C^2 dk   (K+ W-^T, Q+ W-^T, dP W-, dL W-, dP^T Q+, dL^T K+)
+      5 C^2 dv   (T R, P^T dO, T^T dU, dO U^T, dV~ U^T)
+      C^3 / 6    (the unit-lower inverse)."""
+    nc = (w.T + C - 1) // C
+    per = 9 * C * w.dk * w.dv + 6 * C * C * w.dk + 5 * C * C * w.dv + C ** 3 // 6
+    return 2 * per * nc * w.B * w.H
+
+
 def reduce_max(value: float, world: int, device: str = "cuda") -> float:
     """Max over ranks of a per-rank time: the slowest rank sets a multi-rank step's time."""
     if world <= 1:
@@ -101,6 +113,7 @@ KERNEL_SOURCES = {
     "chunk_fwd": ["dn_chunk_sc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
     "decode": ["dn_decode.cu", "dn_common.cuh"],
     "osdn": ["dn_osdn.cu", "dn_tc_ptx.cuh", "dn_common.cuh"],
+    "chunk_bwd": ["dn_bwd.cu", "dn_bwd.cuh", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_common.cuh"],
 }
 
 
@@ -257,7 +270,7 @@ def run_single_kernel(args):
 
     if not os.path.exists(dnbuild.LIB):
         dnbuild.build()
-    name = {"chunk": WORKLOAD, "decode": DECODE, "osdn": "osdn_phase1"}[args.only]
+    name = {"chunk": WORKLOAD, "decode": DECODE, "osdn": "osdn_phase1", "bwd": WORKLOAD}[args.only]
     w = di.WORKLOADS[name]
     if args.batch:
         w = w.scaled(B=args.batch)
@@ -272,9 +285,18 @@ def run_single_kernel(args):
 
     xd = {n: to_dev(a) for n, a in x.items()}
     S = xd["S0"].clone() if xd.get("S0") is not None else None
+    if args.only == "bwd":
+        gb = {n: to_dev(a) for n, a in di.make_bwd_inputs(w).items()}
+        desc = dn.make_desc(xd["q"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"])
+        wsb = torch.empty(dn.dn_chunk_bwd_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+        gout = dn.dn_chunk_bwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                               xd["S0"], dO=gb["dO"], dS_T=gb["dS_T"], workspace=wsb)
 
     def launch():
-        if args.only == "osdn":
+        if args.only == "bwd":
+            dn.dn_chunk_bwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                            xd["S0"], dO=gb["dO"], dS_T=gb["dS_T"], workspace=wsb, out=gout)
+        elif args.only == "osdn":
             dn.dn_osdn_precond(xd["k"], xd["beta"], xd["retention"], None, eta=eta)
         elif args.only == "chunk":
             dn.dn_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
@@ -308,8 +330,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-osdn", action="store_true", help="skip the OSDN preconditioner scan leg")
     ap.add_argument("--no-mc", action="store_true", help="skip the Memory Caching leg")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the chunked backward leg")
     ap.add_argument("--decode-steps", type=int, default=100)
-    ap.add_argument("--only", choices=["chunk", "decode", "osdn"], default=None,
+    ap.add_argument("--only", choices=["chunk", "decode", "osdn", "bwd"], default=None,
                     help="profiling mode: run just one kernel on the workload with batch --batch")
     ap.add_argument("--batch", type=int, default=0, help="with --only: batch size of the scaled workload")
     args = ap.parse_args()
@@ -575,6 +598,48 @@ def main():
         launches += 10 + 10
         del Mc
 
+    # ---- chunked backward on the prefill workload (the training pass of the same recurrence)
+    bwd = None
+    if not args.no_bwd:
+        gb = {n: to_dev(a) for n, a in di.make_bwd_inputs(w).items()}
+        desc_b = dn.make_desc(xd["q"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"])
+        wsb = torch.empty(dn.dn_chunk_bwd_workspace_bytes(desc_b), dtype=torch.uint8, device="cuda")
+        gout = dn.dn_chunk_bwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                               xd["S0"], dO=gb["dO"], dS_T=gb["dS_T"], workspace=wsb, stream=stream)
+
+        def bstep():
+            dn.dn_chunk_bwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                            xd["S0"], dO=gb["dO"], dS_T=gb["dS_T"], workspace=wsb, out=gout, stream=stream)
+
+        for _ in range(3):
+            bstep()
+        torch.cuda.synchronize()
+        nb = 5
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        b0.record(stream)
+        for _ in range(nb):
+            bstep()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        if dn.dn_stream_status(stream) != dn.DN_OK:
+            raise RuntimeError("device status after the backward")
+        b_ms = reduce_max(b0.elapsed_time(b1) / nb, world)
+        fl = bwd_flops(w)
+        tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25  # nominal dense tf32 : bf16 ratio
+        btf = fl / (b_ms * 1e-3) / 1e12
+        bwd = {"workload": "chunked backward of gdn_prefill (B=8 H=16 T=4096 d=128 bf16, scalar gates); "
+                           "dO ~ N(0,1) bf16, dS_T ~ N(0,0.1^2)",
+               "ms_per_call": b_ms, "tokens_per_s": weak_scaling_rate(B * T, world, b_ms),
+               "fwd_ms": kern_ms, "bwd_over_fwd": b_ms / kern_ms, "kernels_per_call": 4,
+               "roofline": {"bound": "tensor", "achieved": btf, "peak": tf32_peak, "unit": "TFLOP/s",
+                            "frac": btf / tf32_peak, "traffic": recorded_traffic("chunk_bwd"),
+                            "peak_source": f"{peaks['source']} bf16 x 1.1/2.25 (dense tf32 : bf16)",
+                            "scope": "the whole call (4 kernels); flops as bwd_flops counts them",
+                            "algorithmic_flops_per_launch": fl}}
+        launches += 4 * nb
+        del gb, wsb, gout
+
     clocks.__exit__(None, None, None)
 
     cpu = None
@@ -595,7 +660,7 @@ def main():
             "config": bench_config(world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode, "osdn_phase1": osdn,
-            "memory_caching": mc,
+            "memory_caching": mc, "chunk_bwd": bwd,
             "kernel_source": {k: kernel_source_hash(k) for k in KERNEL_SOURCES},
         }
         print(json.dumps(line), flush=True)

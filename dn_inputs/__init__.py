@@ -19,6 +19,8 @@ GDN scalar gates, KDA channel decay, FG2-GDN+ with OSDN preconditioner, decode):
                                                  preconditioner d=1+0.1*N per key channel, S0~N(0,0.02^2)
   decode           1024 sequences, H=32, d=128: resident S~N(0,0.02^2) fp32, one bf16 token per step,
                    channel alpha, beta_k, beta_v as in fg2_osdn_long, 100 steps
+  (backward)       every workload above also draws the backward's cotangents: dO ~ N(0,1) like o,
+                   dS_T ~ N(0, 0.1^2) fp32 (make_bwd_inputs)
   osdn_phase1      the OSDN preconditioner scan on fg2_osdn_long's keys (same seed): B=2 H=16 T=32768
                    d_k=128 bf16 k, beta=sigmoid(N) per token, retention r~U(0.95,1) per token, eta=0.5,
                    d_0 = 1
@@ -49,7 +51,7 @@ GATE_ONE, GATE_SCALAR, GATE_CHANNEL = 0, 1, 2
 
 SEED_BASE = 20260000
 TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "alpha": 3, "beta_k": 4, "beta_v": 5, "key_scale": 6, "S0": 7,
-              "beta": 8, "retention": 9}
+              "beta": 8, "retention": 9, "dO": 10, "dS_T": 11}
 
 
 def build(force: bool = False) -> str:
@@ -223,6 +225,14 @@ def make_inputs(w: Workload, step: int = 0) -> dict:
     else:
         out["S0"] = None
     return out
+
+
+def make_bwd_inputs(w: Workload, ds_std: float = 0.1) -> dict:
+    """Cotangents of the backward pass for workload w: dO [B,T,H,dv] ~ N(0,1) in the storage dtype
+    (the gradient of the loss with respect to o) and dS_T [B,H,dk,dv] ~ N(0, ds_std^2) fp32 (with
+    respect to the final state)."""
+    return {"dO": fill((w.B, w.T, w.H, w.dv), w.seed("dO"), GEN_NORMAL, 0.0, 1.0, dtype=w.io),
+            "dS_T": fill((w.B, w.H, w.dk, w.dv), w.seed("dS_T"), GEN_NORMAL, 0.0, ds_std, dtype="f32")}
 
 
 def make_osdn_inputs(w: Workload) -> dict:

@@ -10,6 +10,8 @@ Entry points (same names as the C ABI):
                  S0=None, o=None, S_T=None, stream=None) -> (o, S_T)
     dn_decode_step(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None,
                    S=..., o=None, stream=None) -> o          (S updated in place)
+    dn_chunk_bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None,
+                 dO=..., dS_T=None, workspace=None, stream=None) -> dict of gradients
     dn_osdn_precond(k, beta, retention=None, d0=None, eta=0.5, d=None, d_T=None,
                     workspace=None, stream=None) -> (d, d_T)   (OSDN phase 1)
     dn_mc_readout(q, M, gates=None, o=..., seg_len=L, stream=None) -> o     (Memory Caching read-out)
@@ -38,8 +40,9 @@ DN_GATE_ONE, DN_GATE_SCALAR, DN_GATE_CHANNEL = 0, 1, 2
 DN_READ_POST, DN_READ_PRE = 0, 1
 _READOUT = {"post": DN_READ_POST, "pre": DN_READ_PRE}
 
-EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_osdn_precond_workspace_bytes",
-            "dn_osdn_precond", "dn_mc_readout", "dn_stream_status", "dn_status_string", "dn_version")
+EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_chunk_bwd_workspace_bytes",
+            "dn_chunk_bwd", "dn_osdn_precond_workspace_bytes", "dn_osdn_precond", "dn_osdn_precond_noalloc",
+            "dn_mc_readout", "dn_stream_status", "dn_status_string", "dn_version")
 
 
 class DnDesc(ctypes.Structure):
@@ -84,6 +87,10 @@ def load(path: str = LIB_PATH):
     lib.dn_chunk_fwd.restype = I
     lib.dn_decode_step.argtypes = [D, P, P, P, P, P, P, P, P, P, P]
     lib.dn_decode_step.restype = I
+    lib.dn_chunk_bwd_workspace_bytes.argtypes = [D]
+    lib.dn_chunk_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.dn_chunk_bwd.argtypes = [D] + [P] * 19 + [ctypes.c_size_t, P]
+    lib.dn_chunk_bwd.restype = I
     O = ctypes.POINTER(DnOsdnDesc)
     lib.dn_osdn_precond_workspace_bytes.argtypes = [O]
     lib.dn_osdn_precond_workspace_bytes.restype = ctypes.c_size_t
@@ -196,6 +203,56 @@ def dn_decode_step(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None
     if rc != DN_OK:
         raise DnError(rc, "dn_decode_step")
     return o
+
+
+def dn_chunk_bwd_workspace_bytes(desc: DnDesc) -> int:
+    return int(load().dn_chunk_bwd_workspace_bytes(ctypes.byref(desc)))
+
+
+def dn_chunk_bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, dO=None, dS_T=None,
+                 workspace=None, want_dS0: bool = True, out=None, stream=None):
+    """Chunked backward of dn_chunk_fwd (post-update read-out): the gradients of
+    sum <dO, o> + <dS_T, S_T>. dO [B,T,H,d_v] in the io dtype; dS_T [B,H,d_k,d_v] fp32 or None (zero).
+
+    Returns {"q", "k", "v"} (io dtype, shaped like the inputs), {"alpha", "beta_k", "beta_v",
+    "key_scale"} (fp32, shaped like each gate; None for an absent gate) and "S0" (fp32
+    [B,H,d_k,d_v], or None when want_dS0 is False). The workspace (dn_chunk_bwd_workspace_bytes)
+    is allocated here when not given; so are the outputs, unless `out` (a dict returned by an
+    earlier call of the same shapes) is passed to be written again.
+    """
+    lib = load()
+    _check_io(q, k, v)
+    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, 0, "post")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if dO is None or not dO.is_contiguous() or dO.dtype != q.dtype or tuple(dO.shape) != (B, T, H, dv):
+        raise ValueError("dO must be a contiguous [B,T,H,d_v] tensor of q's dtype")
+    if dS_T is not None and (dS_T.dtype != torch.float32 or not dS_T.is_contiguous()
+                             or tuple(dS_T.shape) != (B, H, dk, dv)):
+        raise ValueError("dS_T must be a contiguous float32 [B,H,d_k,d_v] tensor")
+    if out is None:
+        out = {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v)}
+        for name, g in (("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v), ("key_scale", key_scale)):
+            out[name] = None if g is None else torch.empty_like(g)
+        out["S0"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if want_dS0 else None
+    else:
+        for name, ref in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta_k", beta_k), ("beta_v", beta_v),
+                          ("key_scale", key_scale)):
+            t = out.get(name)
+            if (t is None) != (ref is None) or (t is not None and (t.shape != ref.shape or t.dtype != ref.dtype
+                                                                   or not t.is_contiguous())):
+                raise ValueError(f"out[{name!r}] does not match {name}")
+    ws_bytes = dn_chunk_bwd_workspace_bytes(desc)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    rc = lib.dn_chunk_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k), _ptr(beta_v),
+                          _ptr(key_scale), _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(out["q"]), _ptr(out["k"]),
+                          _ptr(out["v"]), _ptr(out["alpha"]), _ptr(out["beta_k"]), _ptr(out["beta_v"]),
+                          _ptr(out["key_scale"]), _ptr(out["S0"]), _ptr(workspace),
+                          ws_bytes if workspace is not None else 0, _stream_handle(stream))
+    if rc != DN_OK:
+        raise DnError(rc, "dn_chunk_bwd")
+    return out
 
 
 def dn_osdn_precond_workspace_bytes(desc: DnOsdnDesc) -> int:

@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "dn_bwd.cuh"
 #include "dn_common.cuh"
 
 // One status word per GPU that loads the library; kernels set it when a
@@ -263,6 +264,85 @@ dn_status dn_mc_readout(const dn_mc_desc* d, const void* q, const float* M, cons
   if (ranges_overlap(o, n_o, q, n_q)) return DN_ERR_INVALID_ARGUMENT;
   cudaError_t e = dn::launch_mc_readout(q, M, gates, o, d->B, d->T, d->H, d->d_k, d->d_v, d->seg_len,
                                         d->io_dtype == DN_BF16, static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+
+// The backward covers the tensor-core sizes with the post-update read-out.
+dn_status check_bwd_desc(const dn_desc* d) {
+  dn_status st = check_desc(d, false);
+  if (st != DN_OK) return st;
+  if (d->readout != DN_READ_POST) return DN_ERR_UNSUPPORTED;
+  if (!((d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128))) return DN_ERR_UNSUPPORTED;
+  const int64_t blocks = (int64_t)d->B * d->H * ((d->T + 63) / 64);
+  if (blocks >= ((int64_t)1 << 31)) return DN_ERR_UNSUPPORTED;
+  return DN_OK;
+}
+
+// A gate gradient is given exactly when its gate is.
+dn_status check_grad_ptr(int mode, const float* g) {
+  if ((mode == DN_GATE_ONE) != (g == nullptr)) return DN_ERR_INVALID_ARGUMENT;
+  if (g && !aligned4(g)) return DN_ERR_MISALIGNED;
+  return DN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t dn_chunk_bwd_workspace_bytes(const dn_desc* desc) {
+  if (check_bwd_desc(desc) != DN_OK) return 0;
+  return dn::chunk_bwd_workspace_bytes(desc->B, desc->T, desc->H, desc->d_k, desc->d_v);
+}
+
+dn_status dn_chunk_bwd(const dn_desc* desc, const void* q, const void* k, const void* v, const float* alpha,
+                       const float* beta_k, const float* beta_v, const float* key_scale, const float* S0,
+                       const void* dO, const float* dS_T, void* dq, void* dk, void* dv, float* d_alpha,
+                       float* d_beta_k, float* d_beta_v, float* d_key_scale, float* dS0, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream) {
+  dn_status st = check_bwd_desc(desc);
+  if (st != DN_OK) return st;
+  dn::Args a;
+  if ((st = fill_args(desc, q, k, v, alpha, beta_k, beta_v, key_scale, &a)) != DN_OK) return st;
+  if ((S0 && !aligned16(S0)) || (dS_T && !aligned16(dS_T)) || (dS0 && !aligned16(dS0))) return DN_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const size_t n_S = (size_t)desc->B * desc->H * desc->d_k * desc->d_v * sizeof(float);
+  if (desc->T == 0) {  // no tokens: dS0 = dS_T
+    if (!dS0) return DN_OK;
+    cudaError_t e = dS_T ? (dS_T == dS0 ? cudaSuccess : cudaMemcpyAsync(dS0, dS_T, n_S, cudaMemcpyDeviceToDevice, s))
+                         : cudaMemsetAsync(dS0, 0, n_S, s);
+    return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
+  }
+  if (!dO || !dq || !dk || !dv) return DN_ERR_INVALID_ARGUMENT;
+  if (!aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DN_ERR_MISALIGNED;
+  if ((st = check_grad_ptr(desc->alpha, d_alpha)) != DN_OK) return st;
+  if ((st = check_grad_ptr(desc->beta_k, d_beta_k)) != DN_OK) return st;
+  if ((st = check_grad_ptr(desc->beta_v, d_beta_v)) != DN_OK) return st;
+  if ((st = check_grad_ptr(desc->key_scale, d_key_scale)) != DN_OK) return st;
+  const size_t need = dn::chunk_bwd_workspace_bytes(desc->B, desc->T, desc->H, desc->d_k, desc->d_v);
+  if (!workspace || workspace_bytes < need) return DN_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(workspace)) return DN_ERR_MISALIGNED;
+  {  // the gradients of q, k, v are written while every input, dO and the workspace are still read
+    const size_t es = desc->io_dtype == DN_BF16 ? 2 : 4;
+    const size_t n_k = (size_t)desc->B * desc->T * desc->H * desc->d_k * es;
+    const size_t n_v = (size_t)desc->B * desc->T * desc->H * desc->d_v * es;
+    const void* outs[3] = {dq, dk, dv};
+    const size_t out_n[3] = {n_k, n_k, n_v};
+    const void* ins[6] = {q, k, v, dO, workspace, S0};
+    const size_t in_n[6] = {n_k, n_k, n_v, n_v, need, S0 ? n_S : 0};
+    for (int i = 0; i < 3; ++i) {
+      for (int j = 0; j < 6; ++j)
+        if (ranges_overlap(outs[i], out_n[i], ins[j], in_n[j])) return DN_ERR_INVALID_ARGUMENT;
+      for (int j = i + 1; j < 3; ++j)
+        if (ranges_overlap(outs[i], out_n[i], outs[j], out_n[j])) return DN_ERR_INVALID_ARGUMENT;
+    }
+  }
+  a.S0 = S0;
+  cudaError_t e = dn::launch_chunk_bwd(a, dO, dS_T, dq, dk, dv, d_alpha, d_beta_k, d_beta_v, d_key_scale, dS0,
+                                       static_cast<float*>(workspace), s);
   return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
 

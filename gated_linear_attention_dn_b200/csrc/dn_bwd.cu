@@ -1,0 +1,719 @@
+// Chunked backward (training pass) of the recurrence with the post-update read-out: the gradients
+// of sum <dO, o> + <dS_T, S_T> with respect to q, k, v, every gate and S0. The pages name
+// chunk-parallel training (FG2-GDN page, section 3 item 2) but print no backward; the equations
+// below are the chain rule through the chunk form of the forward.
+//
+// Chunk form (C = 64 tokens, local t = 0..C-1; g_t = sum_{s<=t} log alpha_s per key channel; r = g at
+// token (n-1)/2 of the chunk's n valid tokens, a reference held fixed; h_t = g_t - r):
+//   K+ = k e^h,  Q+ = q e^h,  W- = w e^-h (w = beta^k d k),  V~ = beta^v v,  S_m = Diag(e^r) S
+//   T = (I + strictly-lower(K+ W-^T))^-1,  P = lower-incl(Q+ W-^T)
+//   U = T (V~ - K+ S_m),  O = Q+ S_m + P U,  S' = Diag(lam) X,  X = S_m + W-^T U,  lam = e^{g_last - r}
+// Reverse, given dO and the chunk-end adjoint dS':
+//   dX = Diag(lam) dS',  dU = P^T dO + W- dX,  dV~ = T^T dU,  dS = Diag(e^r)(dX + Q+^T dO - K+^T dV~)
+//   dP = lower-incl(dO U^T),  dL = -strictly-lower(dV~ U^T)
+//   dQ+ = dO S_m^T + dP W-,  dK+ = -dV~ S_m^T + dL W-,  dW- = U dX^T + dP^T Q+ + dL^T K+
+//   dh_t = Q+ dQ+ + K+ dK+ - W- dW- (per channel), plus rowsum(dX (.) X) at the last token;
+//   d log alpha_s = sum_{t >= s in the chunk} dh_t; then the products back to q, k, w, gates.
+// (The outputs do not depend on r, so its own adjoint terms cancel and r is held fixed.)
+//
+// Four kernels, all fp32 with the dense per-chunk products on warp tensor cores (mma.sync TF32 with
+// a three-product hi/lo split, so each product keeps about fp32 accuracy):
+//   bwd_prep   one CTA per chunk:                 T and P of every chunk          -> workspace
+//   bwd_state  one CTA per (b, h, 32 columns of d_v), chunks in order:   S_m, U  -> workspace
+//   bwd_dstate one CTA per (b, h, 32 columns of d_v), chunks in reverse: dX, dV~ -> workspace; dS0
+//   bwd_local  one CTA per chunk: dq, dk, dv and the gate gradients (key channels in slices of 32)
+#include "dn_bwd.cuh"
+#include "dn_ut_inverse.cuh"
+
+namespace dn {
+namespace {
+
+constexpr int kC = 64;     // chunk length
+constexpr int kNT = 256;   // threads per CTA (8 warps)
+constexpr int kDVS = 32;   // value columns per chain CTA
+constexpr int kDKS = 32;   // key channels per slice of the local-gradient kernel
+
+struct BwdArgs {
+  Args f;  // forward inputs and sizes
+  const void* dO;
+  const float* dS_T;
+  void* gq;
+  void* gk;
+  void* gv;
+  float* galpha;
+  float* gbeta_k;
+  float* gbeta_v;
+  float* gkey_scale;
+  float* gS0;
+  float* wT;    // [BH][nc][C][C]
+  float* wP;    // [BH][nc][C][C]
+  float* wSm;   // [BH][nc][dk][dv]
+  float* wU;    // [BH][nc][C][dv]
+  float* wdX;   // [BH][nc][dk][dv]
+  float* wdVt;  // [BH][nc][C][dv]
+  int nc;
+};
+
+// ------------------------------------------------------------------ warp tensor-core products
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = ut::to_tf32(x);
+  lo = ut::to_tf32(x - __uint_as_float(hi));
+}
+
+// acc[MI][NI] (16 x 8 fragments) += sum_{k < K} A(m, k) B(k, n) over the warp tile of 16 MI rows and
+// 8 NI columns, with x = hi + lo split operands: a b ~ a_lo b_hi + a_hi b_lo + a_hi b_hi.
+template <int MI, int NI, int K, class FA, class FB>
+__device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t ah[MI][4], al[MI][4];
+#pragma unroll
+    for (int mi = 0; mi < MI; ++mi) {
+      split_tf32(A(16 * mi + g, k0 + t), ah[mi][0], al[mi][0]);
+      split_tf32(A(16 * mi + g + 8, k0 + t), ah[mi][1], al[mi][1]);
+      split_tf32(A(16 * mi + g, k0 + t + 4), ah[mi][2], al[mi][2]);
+      split_tf32(A(16 * mi + g + 8, k0 + t + 4), ah[mi][3], al[mi][3]);
+    }
+#pragma unroll
+    for (int ni = 0; ni < NI; ++ni) {
+      uint32_t bh[2], bl[2];
+      split_tf32(B(k0 + t, 8 * ni + g), bh[0], bl[0]);
+      split_tf32(B(k0 + t + 4, 8 * ni + g), bh[1], bl[1]);
+#pragma unroll
+      for (int mi = 0; mi < MI; ++mi) {
+        ut::mma_tf32(acc[mi][ni], al[mi], bh);
+        ut::mma_tf32(acc[mi][ni], ah[mi], bl);
+        ut::mma_tf32(acc[mi][ni], ah[mi], bh);
+      }
+    }
+  }
+}
+
+// E(m, n, value) for every element of the warp tile's accumulator.
+template <int MI, int NI, class FE>
+__device__ __forceinline__ void warp_epilogue(const float (&acc)[MI][NI][4], FE E, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+    for (int ni = 0; ni < NI; ++ni) {
+      E(16 * mi + g, 8 * ni + 2 * t, acc[mi][ni][0]);
+      E(16 * mi + g, 8 * ni + 2 * t + 1, acc[mi][ni][1]);
+      E(16 * mi + g + 8, 8 * ni + 2 * t, acc[mi][ni][2]);
+      E(16 * mi + g + 8, 8 * ni + 2 * t + 1, acc[mi][ni][3]);
+    }
+}
+
+// ------------------------------------------------------------------ chunk quantities
+__device__ __forceinline__ int64_t token(const Args& a, int b, int h, int t) {
+  return ((int64_t)b * a.T + t) * a.H + h;
+}
+
+// Key channels [i0, i0 + NCH) of the chunk starting at token t0 (n valid tokens) of head (b, h), into
+// [C][NCH + 4] arrays: hb = h_t, Kp = k e^h, Qp = q e^h, Wm = w e^-h (Kp, Qp may be null; hb may be
+// Wm itself), er = e^r, lam = e^{g_last - r}. Tokens past the end have k = q = w = 0 and alpha = 1.
+// Called by all kNT threads; returns after a barrier.
+template <int NCH>
+__device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, float* hb, float* Kp, float* Qp,
+                           float* Wm, float* er, float* lam, int tid) {
+  constexpr int LD = NCH + 4;
+  for (int e = tid; e < kC * NCH; e += kNT) {
+    const int t = e / NCH, i = e % NCH;
+    float la = 0.f;
+    if (t < n) la = logf(gate_load(a.alpha_p, a.alpha, token(a, b, h, t0 + t), a.dk, i0 + i));
+    hb[t * LD + i] = la;
+  }
+  __syncthreads();
+  const int tr = (n - 1) / 2;
+  for (int i = tid; i < NCH; i += kNT) {
+    float run = 0.f, r = 0.f;
+    for (int t = 0; t < kC; ++t) {
+      run += hb[t * LD + i];
+      hb[t * LD + i] = run;
+      if (t == tr) r = run;
+    }
+    for (int t = 0; t < kC; ++t) hb[t * LD + i] -= r;
+    er[i] = expf(r);
+    lam[i] = expf(run - r);
+  }
+  __syncthreads();
+  for (int e = tid; e < kC * NCH; e += kNT) {
+    const int t = e / NCH, i = e % NCH;
+    const float hv = hb[t * LD + i];
+    float kk = 0.f, qq = 0.f, w = 0.f;
+    if (t < n) {
+      const int64_t tok = token(a, b, h, t0 + t);
+      kk = io_load(a.k, tok * a.dk + i0 + i, a.io_bf16);
+      if (Qp) qq = io_load(a.q, tok * a.dk + i0 + i, a.io_bf16);
+      w = gate_load(a.beta_k_p, a.beta_k, tok, a.dk, i0 + i) * gate_load(a.key_scale_p, a.key_scale, tok, a.dk, i0 + i) *
+          kk;
+    }
+    const float eh = expf(hv);
+    if (Kp) Kp[t * LD + i] = kk * eh;
+    if (Qp) Qp[t * LD + i] = qq * eh;
+    Wm[t * LD + i] = w / eh;
+  }
+  __syncthreads();
+}
+
+// T = (I + L)^-1 for the strictly lower 64 x 64 L in Lm (row stride LDC) into Tm (same stride), fp32.
+// The four 16 x 16 diagonal blocks by forward substitution (one column per thread), then the blocks
+// below the diagonal by block distance d: T_ij = -T_ii sum_{j <= k < i} L_ik T_kj. scr: 768 floats.
+constexpr int kLDC = kC + 4;
+__device__ void inverse64(const float* Lm, float* Tm, float* scr, int tid) {
+  for (int e = tid; e < kC * kC; e += kNT) Tm[(e / kC) * kLDC + e % kC] = 0.f;
+  __syncthreads();
+  if (tid < 64) {
+    const int o = (tid >> 4) * 16, j = tid & 15;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = i == j ? 1.f : 0.f;
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < i; ++k) s = fmaf(Lm[(o + i) * kLDC + o + k], x[k], s);
+      if (i > j) x[i] = -s;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) Tm[(o + i) * kLDC + o + j] = x[i];
+  }
+  __syncthreads();
+  for (int d = 1; d < 4; ++d) {
+    const int np = 4 - d;
+    for (int e = tid; e < np * 256; e += kNT) {
+      const int bj = e >> 8, bi = bj + d, r = (e >> 4) & 15, col = e & 15;
+      float s = 0.f;
+      for (int k = bj * 16; k < bi * 16; ++k) s = fmaf(Lm[(bi * 16 + r) * kLDC + k], Tm[k * kLDC + bj * 16 + col], s);
+      scr[e] = s;
+    }
+    __syncthreads();
+    for (int e = tid; e < np * 256; e += kNT) {
+      const int bj = e >> 8, bi = bj + d, r = (e >> 4) & 15, col = e & 15;
+      float s = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) s = fmaf(Tm[(bi * 16 + r) * kLDC + bi * 16 + k], scr[(bj << 8) + (k << 4) + col], s);
+      Tm[(bi * 16 + r) * kLDC + bj * 16 + col] = -s;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ kernel 1: T and P per chunk
+template <int DK>
+__global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
+  extern __shared__ float4 smem4[];
+  constexpr int LDK = DK + 4;
+  float* Kp = reinterpret_cast<float*>(smem4);
+  float* Qp = Kp + kC * LDK;
+  float* Wm = Qp + kC * LDK;
+  float* Lm = Wm + kC * LDK;
+  float* Tm = Lm + kC * kLDC;
+  float* scr = Tm + kC * kLDC;
+  float* er = scr + 768;
+  float* lam = er + DK;
+  const Args& a = p.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x % p.nc, bh = blockIdx.x / p.nc, b = bh / a.H, h = bh % a.H;
+  const int t0 = c * kC, n = min(kC, a.T - t0);
+  prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, tid);
+
+  const int64_t cb = (int64_t)bh * p.nc + c;
+  {  // warps 0-3: L = strictly-lower(K+ W-^T); warps 4-7: P = lower-incl(Q+ W-^T); 32 x 32 tiles
+    const int m0 = ((warp & 3) >> 1) * 32, n0 = (warp & 1) * 32;
+    const float* X = warp < 4 ? Kp : Qp;
+    float acc[2][4][4] = {};
+    warp_gemm<2, 4, DK>(
+        acc, [&](int m, int k) { return X[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return Wm[(n0 + nn) * LDK + k]; },
+        lane);
+    if (warp < 4) {
+      warp_epilogue(acc, [&](int m, int nn, float v) { Lm[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? v : 0.f; }, lane);
+    } else {
+      float* P = p.wP + cb * kC * kC;
+      warp_epilogue(acc, [&](int m, int nn, float v) { P[(m0 + m) * kC + n0 + nn] = n0 + nn <= m0 + m ? v : 0.f; }, lane);
+    }
+  }
+  __syncthreads();
+  inverse64(Lm, Tm, scr, tid);
+  float* Tg = p.wT + cb * kC * kC;
+  for (int e = tid; e < kC * kC; e += kNT) Tg[e] = Tm[(e / kC) * kLDC + e % kC];
+}
+
+// ------------------------------------------------------------------ kernel 2: states, chunks in order
+template <int DK, int DV>
+__global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
+  extern __shared__ float4 smem4[];
+  constexpr int LDK = DK + 4, LDS = kDVS + 4;
+  float* S = reinterpret_cast<float*>(smem4);  // [DK][LDS]
+  float* Kp = S + DK * LDS;                     // [C][LDK]
+  float* Wm = Kp + kC * LDK;                    // [C][LDK]
+  float* Tm = Wm + kC * LDK;                    // [C][kLDC]
+  float* R = Tm + kC * kLDC;                    // [C][LDS]: V~ - K+ S_m, then U
+  float* er = R + kC * LDS;
+  float* lam = er + DK;
+  const Args& a = p.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NS = DV / kDVS;
+  const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * kDVS, b = bh / a.H, h = bh % a.H;
+  for (int e = tid; e < DK * kDVS; e += kNT) {
+    const int i = e / kDVS, j = e % kDVS;
+    S[i * LDS + j] = a.S0 ? a.S0[((int64_t)bh * DK + i) * DV + j0 + j] : 0.f;
+  }
+  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;  // this warp's 16 x 16 tile of a 64 x 32 result
+  for (int c = 0; c < p.nc; ++c) {
+    const int t0 = c * kC, n = min(kC, a.T - t0);
+    const int64_t cb = (int64_t)bh * p.nc + c;
+    __syncthreads();  // the previous chunk is done with every buffer
+    prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, nullptr, Wm, er, lam, tid);
+    const float* Tg = p.wT + cb * kC * kC;
+    for (int e = tid; e < kC * kC; e += kNT) Tm[(e / kC) * kLDC + e % kC] = Tg[e];
+    for (int e = tid; e < kC * kDVS; e += kNT) {
+      const int t = e / kDVS, j = e % kDVS;
+      float x = 0.f;
+      if (t < n) {
+        const int64_t tok = token(a, b, h, t0 + t);
+        x = gate_load(a.beta_v_p, a.beta_v, tok, DV, j0 + j) * io_load(a.v, tok * DV + j0 + j, a.io_bf16);
+      }
+      R[t * LDS + j] = x;
+    }
+    float* Smg = p.wSm + cb * DK * DV;
+    for (int e = tid; e < DK * kDVS; e += kNT) {
+      const int i = e / kDVS, j = e % kDVS;
+      const float x = S[i * LDS + j] * er[i];
+      S[i * LDS + j] = x;
+      Smg[(int64_t)i * DV + j0 + j] = x;
+    }
+    __syncthreads();
+    {  // R = V~ - K+ S_m (each warp updates only its own tile)
+      float acc[1][2][4] = {};
+      warp_gemm<1, 2, DK>(
+          acc, [&](int m, int k) { return Kp[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return S[k * LDS + n0 + nn]; },
+          lane);
+      warp_epilogue(acc, [&](int m, int nn, float v) { R[(m0 + m) * LDS + n0 + nn] -= v; }, lane);
+    }
+    __syncthreads();
+    {  // U = T R
+      float acc[1][2][4] = {};
+      warp_gemm<1, 2, kC>(
+          acc, [&](int m, int k) { return Tm[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return R[k * LDS + n0 + nn]; },
+          lane);
+      __syncthreads();
+      float* Ug = p.wU + cb * kC * DV;
+      warp_epilogue(acc,
+                    [&](int m, int nn, float v) {
+                      R[(m0 + m) * LDS + n0 + nn] = v;
+                      Ug[(int64_t)(m0 + m) * DV + j0 + n0 + nn] = v;
+                    },
+                    lane);
+    }
+    __syncthreads();
+    // S' = Diag(lam) (S_m + W-^T U): DK x 32 in 16 x 16 tiles
+    for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
+      const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * 16;
+      float acc[1][2][4] = {};
+      warp_gemm<1, 2, kC>(
+          acc, [&](int m, int k) { return Wm[k * LDK + r0 + m]; }, [&](int k, int nn) { return R[k * LDS + q0 + nn]; },
+          lane);
+      warp_epilogue(acc,
+                    [&](int m, int nn, float v) {
+                      float* s = &S[(r0 + m) * LDS + q0 + nn];
+                      *s = lam[r0 + m] * (*s + v);
+                    },
+                    lane);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel 3: state adjoints, chunks in reverse
+template <int DK, int DV>
+__global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
+  extern __shared__ float4 smem4[];
+  constexpr int LDK = DK + 4, LDS = kDVS + 4;
+  float* dS = reinterpret_cast<float*>(smem4);  // [DK][LDS]: dS', then dX, then dS
+  float* Qp = dS + DK * LDS;                     // [C][LDK]
+  float* Kp = Qp + kC * LDK;
+  float* Wm = Kp + kC * LDK;
+  float* Tm = Wm + kC * LDK;  // [C][kLDC]
+  float* Pm = Tm + kC * kLDC;
+  float* dOs = Pm + kC * kLDC;  // [C][LDS]
+  float* dU = dOs + kC * LDS;   // [C][LDS]: dU, then dV~
+  float* er = dU + kC * LDS;
+  float* lam = er + DK;
+  const Args& a = p.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int NS = DV / kDVS;
+  const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * kDVS, b = bh / a.H, h = bh % a.H;
+  for (int e = tid; e < DK * kDVS; e += kNT) {
+    const int i = e / kDVS, j = e % kDVS;
+    dS[i * LDS + j] = p.dS_T ? p.dS_T[((int64_t)bh * DK + i) * DV + j0 + j] : 0.f;
+  }
+  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
+  for (int c = p.nc - 1; c >= 0; --c) {
+    const int t0 = c * kC, n = min(kC, a.T - t0);
+    const int64_t cb = (int64_t)bh * p.nc + c;
+    __syncthreads();
+    prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, tid);
+    const float* Tg = p.wT + cb * kC * kC;
+    const float* Pg = p.wP + cb * kC * kC;
+    for (int e = tid; e < kC * kC; e += kNT) {
+      Tm[(e / kC) * kLDC + e % kC] = Tg[e];
+      Pm[(e / kC) * kLDC + e % kC] = Pg[e];
+    }
+    for (int e = tid; e < kC * kDVS; e += kNT) {
+      const int t = e / kDVS, j = e % kDVS;
+      dOs[t * LDS + j] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j0 + j, a.io_bf16) : 0.f;
+    }
+    float* dXg = p.wdX + cb * DK * DV;
+    for (int e = tid; e < DK * kDVS; e += kNT) {
+      const int i = e / kDVS, j = e % kDVS;
+      const float x = dS[i * LDS + j] * lam[i];
+      dS[i * LDS + j] = x;
+      dXg[(int64_t)i * DV + j0 + j] = x;
+    }
+    __syncthreads();
+    {  // dU = P^T dO + W- dX
+      float acc[1][2][4] = {};
+      warp_gemm<1, 2, kC>(
+          acc, [&](int m, int k) { return Pm[k * kLDC + m0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + n0 + nn]; },
+          lane);
+      warp_gemm<1, 2, DK>(
+          acc, [&](int m, int k) { return Wm[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return dS[k * LDS + n0 + nn]; },
+          lane);
+      warp_epilogue(acc, [&](int m, int nn, float v) { dU[(m0 + m) * LDS + n0 + nn] = v; }, lane);
+    }
+    __syncthreads();
+    {  // dV~ = T^T dU
+      float acc[1][2][4] = {};
+      warp_gemm<1, 2, kC>(
+          acc, [&](int m, int k) { return Tm[k * kLDC + m0 + m]; }, [&](int k, int nn) { return dU[k * LDS + n0 + nn]; },
+          lane);
+      __syncthreads();
+      float* dVg = p.wdVt + cb * kC * DV;
+      warp_epilogue(acc,
+                    [&](int m, int nn, float v) {
+                      dU[(m0 + m) * LDS + n0 + nn] = v;
+                      dVg[(int64_t)(m0 + m) * DV + j0 + n0 + nn] = v;
+                    },
+                    lane);
+    }
+    __syncthreads();
+    // dS = Diag(e^r) (dX + Q+^T dO - K+^T dV~): DK x 32 in 16 x 16 tiles
+    for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
+      const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * 16;
+      float acc[1][2][4] = {};
+      warp_gemm<1, 2, kC>(
+          acc, [&](int m, int k) { return Qp[k * LDK + r0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + q0 + nn]; },
+          lane);
+      warp_gemm<1, 2, kC>(
+          acc, [&](int m, int k) { return -Kp[k * LDK + r0 + m]; }, [&](int k, int nn) { return dU[k * LDS + q0 + nn]; },
+          lane);
+      warp_epilogue(acc,
+                    [&](int m, int nn, float v) {
+                      float* s = &dS[(r0 + m) * LDS + q0 + nn];
+                      *s = er[r0 + m] * (*s + v);
+                    },
+                    lane);
+    }
+  }
+  if (p.gS0) {
+    __syncthreads();
+    for (int e = tid; e < DK * kDVS; e += kNT) {
+      const int i = e / kDVS, j = e % kDVS;
+      p.gS0[((int64_t)bh * DK + i) * DV + j0 + j] = dS[i * LDS + j];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel 4: per-token gradients
+template <int DK, int DV>
+__global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
+  extern __shared__ float4 smem4[];
+  constexpr int LDV = DV + 4, LDS = kDKS + 4;
+  float* U = reinterpret_cast<float*>(smem4);  // [C][LDV]
+  float* dVt = U + kC * LDV;
+  float* dOs = dVt + kC * LDV;
+  float* dP = dOs + kC * LDV;   // [C][kLDC]
+  float* dL = dP + kC * kLDC;
+  float* Sm = dL + kC * kLDC;   // [kDKS][LDV]: rows i0.. of S_m
+  float* dX = Sm + kDKS * LDV;  // [kDKS][LDV]
+  float* hb = dX + kDKS * LDV;  // [C][LDS]
+  float* Qp = hb + kC * LDS;    // then the beta^k gradient terms
+  float* Kp = Qp + kC * LDS;    // then the d gradient terms
+  float* Wm = Kp + kC * LDS;    // then dh, then d log alpha
+  float* er = Wm + kC * LDS;
+  float* lam = er + kDKS;
+  float* red = lam + kDKS;    // [4][kDKS]
+  float* acc_a = red + 4 * kDKS;  // [C] per-token sums for gates of width 1
+  float* acc_bk = acc_a + kC;
+  float* acc_d = acc_bk + kC;
+  const Args& a = p.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x % p.nc, bh = blockIdx.x / p.nc, b = bh / a.H, h = bh % a.H;
+  const int t0 = c * kC, n = min(kC, a.T - t0);
+  const int64_t cb = (int64_t)bh * p.nc + c;
+  {
+    const float* Ug = p.wU + cb * kC * DV;
+    const float* dVg = p.wdVt + cb * kC * DV;
+    for (int e = tid; e < kC * DV; e += kNT) {
+      const int t = e / DV, j = e % DV;
+      U[t * LDV + j] = Ug[e];
+      dVt[t * LDV + j] = dVg[e];
+      dOs[t * LDV + j] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j, a.io_bf16) : 0.f;
+    }
+    if (tid < kC) acc_a[tid] = acc_bk[tid] = acc_d[tid] = 0.f;
+  }
+  __syncthreads();
+  // dv = beta^v dV~, and the beta^v gradient v dV~ (summed over channels for a per-token gate)
+  for (int e = tid; e < n * DV; e += kNT) {
+    const int t = e / DV, j = e % DV;
+    const int64_t tok = token(a, b, h, t0 + t);
+    const float dvt = dVt[t * LDV + j];
+    io_store(p.gv, tok * DV + j, gate_load(a.beta_v_p, a.beta_v, tok, DV, j) * dvt, a.io_bf16);
+    if (a.beta_v == DN_GATE_CHANNEL) p.gbeta_v[tok * DV + j] = io_load(a.v, tok * DV + j, a.io_bf16) * dvt;
+  }
+  if (a.beta_v == DN_GATE_SCALAR) {
+    for (int t = warp; t < n; t += kNT / 32) {  // uniform per warp: every lane takes part in the shuffles
+      const int64_t tok = token(a, b, h, t0 + t);
+      float s = 0.f;
+      for (int j = lane; j < DV; j += 32) s = fmaf(io_load(a.v, tok * DV + j, a.io_bf16), dVt[t * LDV + j], s);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) p.gbeta_v[tok] = s;
+    }
+  }
+  {  // warps 0-3: dP = lower-incl(dO U^T); warps 4-7: dL = -strictly-lower(dV~ U^T); 32 x 32 tiles
+    const int m0 = ((warp & 3) >> 1) * 32, n0 = (warp & 1) * 32;
+    const float* X = warp < 4 ? dOs : dVt;
+    float acc[2][4][4] = {};
+    warp_gemm<2, 4, DV>(
+        acc, [&](int m, int k) { return X[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return U[(n0 + nn) * LDV + k]; },
+        lane);
+    if (warp < 4)
+      warp_epilogue(acc, [&](int m, int nn, float v) { dP[(m0 + m) * kLDC + n0 + nn] = n0 + nn <= m0 + m ? v : 0.f; }, lane);
+    else
+      warp_epilogue(acc, [&](int m, int nn, float v) { dL[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? -v : 0.f; }, lane);
+  }
+  __syncthreads();
+
+  const float* Smg = p.wSm + cb * DK * DV;
+  const float* dXg = p.wdX + cb * DK * DV;
+  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;  // 16 x 16 tile of a 64 x 32 (token x channel) result
+  constexpr int XN = DV / 4, NIX = XN / 8;                 // X (32 x DV, channel x column): 16 x XN warp tiles
+  const int mx = (warp >> 2) * 16, nx = (warp & 3) * XN;
+  for (int i0 = 0; i0 < DK; i0 += kDKS) {
+    prep_chunk<kDKS>(a, b, h, t0, n, i0, hb, Kp, Qp, Wm, er, lam, tid);
+    for (int e = tid; e < kDKS * DV; e += kNT) {
+      const int i = e / DV, j = e % DV;
+      Sm[i * LDV + j] = Smg[(int64_t)(i0 + i) * DV + j];
+      dX[i * LDV + j] = dXg[(int64_t)(i0 + i) * DV + j];
+    }
+    __syncthreads();
+    float aq[1][2][4] = {}, ak[1][2][4] = {}, aw[1][2][4] = {}, ax[1][NIX][4] = {};
+    // dQ+ = dO S_m^T + dP W-
+    warp_gemm<1, 2, DV>(
+        aq, [&](int m, int k) { return dOs[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return Sm[(n0 + nn) * LDV + k]; },
+        lane);
+    warp_gemm<1, 2, kC>(
+        aq, [&](int m, int k) { return dP[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return Wm[k * LDS + n0 + nn]; },
+        lane);
+    // dK+ = -dV~ S_m^T + dL W-
+    warp_gemm<1, 2, DV>(
+        ak, [&](int m, int k) { return -dVt[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return Sm[(n0 + nn) * LDV + k]; },
+        lane);
+    warp_gemm<1, 2, kC>(
+        ak, [&](int m, int k) { return dL[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return Wm[k * LDS + n0 + nn]; },
+        lane);
+    // dW- = U dX^T + dP^T Q+ + dL^T K+
+    warp_gemm<1, 2, DV>(
+        aw, [&](int m, int k) { return U[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return dX[(n0 + nn) * LDV + k]; },
+        lane);
+    warp_gemm<1, 2, kC>(
+        aw, [&](int m, int k) { return dP[k * kLDC + m0 + m]; }, [&](int k, int nn) { return Qp[k * LDS + n0 + nn]; },
+        lane);
+    warp_gemm<1, 2, kC>(
+        aw, [&](int m, int k) { return dL[k * kLDC + m0 + m]; }, [&](int k, int nn) { return Kp[k * LDS + n0 + nn]; },
+        lane);
+    // X - S_m = W-^T U for these channels
+    warp_gemm<1, NIX, kC>(
+        ax, [&](int m, int k) { return Wm[k * LDS + mx + m]; }, [&](int k, int nn) { return U[k * LDV + nx + nn]; }, lane);
+    {  // partial rowsum(dX (.) X) over this warp's columns
+      const int g = lane >> 2, t4 = lane & 3;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int ni = 0; ni < NIX; ++ni) {
+        const int j = nx + 8 * ni + 2 * t4;
+        const int r0 = mx + g, r1 = mx + g + 8;
+        s0 += dX[r0 * LDV + j] * (Sm[r0 * LDV + j] + ax[0][ni][0]) + dX[r0 * LDV + j + 1] * (Sm[r0 * LDV + j + 1] + ax[0][ni][1]);
+        s1 += dX[r1 * LDV + j] * (Sm[r1 * LDV + j] + ax[0][ni][2]) + dX[r1 * LDV + j + 1] * (Sm[r1 * LDV + j + 1] + ax[0][ni][3]);
+      }
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+      if (t4 == 0) {
+        red[(warp & 3) * kDKS + mx + g] = s0;
+        red[(warp & 3) * kDKS + mx + g + 8] = s1;
+      }
+    }
+    __syncthreads();  // every product has read Q+, K+, W- before they are overwritten below
+    {
+      // Per (token, channel) of this warp's tiles: dq, dk, the beta^k and d gradients, and dh. Each
+      // thread then reads and writes only its own elements of hb, Qp, Kp, Wm.
+      float gq[2][4], gk[2][4];
+      auto elem = [&](int ni, int q, int m, int nn, float vq, float vk, float vw) {
+        const int t = m0 + m, il = n0 + nn, gi = i0 + il;
+        const float eh = expf(hb[t * LDS + il]);
+        const float dw = vw / eh;
+        float gbk = 0.f, gdd = 0.f, dk = 0.f;
+        if (t < n) {
+          const int64_t tok = token(a, b, h, t0 + t);
+          const float kk = io_load(a.k, tok * DK + gi, a.io_bf16);
+          const float bk = gate_load(a.beta_k_p, a.beta_k, tok, DK, gi);
+          const float dd = gate_load(a.key_scale_p, a.key_scale, tok, DK, gi);
+          dk = vk * eh + bk * dd * dw;
+          gbk = dd * kk * dw;
+          gdd = bk * kk * dw;
+        }
+        gq[ni][q] = vq * eh;
+        gk[ni][q] = dk;
+        const float dh = Qp[t * LDS + il] * vq + Kp[t * LDS + il] * vk - Wm[t * LDS + il] * vw;
+        Qp[t * LDS + il] = gbk;
+        Kp[t * LDS + il] = gdd;
+        Wm[t * LDS + il] = dh;
+      };
+      const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+      for (int ni = 0; ni < 2; ++ni) {
+        elem(ni, 0, g, 8 * ni + 2 * t4, aq[0][ni][0], ak[0][ni][0], aw[0][ni][0]);
+        elem(ni, 1, g, 8 * ni + 2 * t4 + 1, aq[0][ni][1], ak[0][ni][1], aw[0][ni][1]);
+        elem(ni, 2, g + 8, 8 * ni + 2 * t4, aq[0][ni][2], ak[0][ni][2], aw[0][ni][2]);
+        elem(ni, 3, g + 8, 8 * ni + 2 * t4 + 1, aq[0][ni][3], ak[0][ni][3], aw[0][ni][3]);
+      }
+#pragma unroll
+      for (int ni = 0; ni < 2; ++ni)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = m0 + g + (q >> 1) * 8, gi = i0 + n0 + 8 * ni + 2 * t4 + (q & 1);
+          if (t < n) {
+            const int64_t tok = token(a, b, h, t0 + t);
+            io_store(p.gq, tok * DK + gi, gq[ni][q], a.io_bf16);
+            io_store(p.gk, tok * DK + gi, gk[ni][q], a.io_bf16);
+            if (a.beta_k == DN_GATE_CHANNEL) p.gbeta_k[tok * DK + gi] = Qp[t * LDS + gi - i0];
+            if (a.key_scale == DN_GATE_CHANNEL) p.gkey_scale[tok * DK + gi] = Kp[t * LDS + gi - i0];
+          }
+        }
+    }
+    __syncthreads();
+    // d log alpha_s = sum_{t >= s} dh_t + rowsum(dX (.) X) (the last token's share), per channel
+    for (int il = tid; il < kDKS; il += kNT) {
+      float run = red[il] + red[kDKS + il] + red[2 * kDKS + il] + red[3 * kDKS + il];
+      for (int t = kC - 1; t >= 0; --t) {
+        run += Wm[t * LDS + il];
+        if (t < n && a.alpha == DN_GATE_CHANNEL) {
+          const int64_t tok = token(a, b, h, t0 + t);
+          p.galpha[tok * DK + i0 + il] = run / gate_load(a.alpha_p, a.alpha, tok, DK, i0 + il);
+        }
+        Wm[t * LDS + il] = run;
+      }
+    }
+    __syncthreads();
+    // per-token sums over these channels, for gates of width 1
+    if (tid < kC) {
+      float sa = 0.f, sb = 0.f, sd = 0.f;
+      for (int il = 0; il < kDKS; ++il) {
+        sa += Wm[tid * LDS + il];
+        sb += Qp[tid * LDS + il];
+        sd += Kp[tid * LDS + il];
+      }
+      acc_a[tid] += sa;
+      acc_bk[tid] += sb;
+      acc_d[tid] += sd;
+    }
+    __syncthreads();
+  }
+  if (tid < n) {
+    const int64_t tok = token(a, b, h, t0 + tid);
+    if (a.alpha == DN_GATE_SCALAR) p.galpha[tok] = acc_a[tid] / a.alpha_p[tok];
+    if (a.beta_k == DN_GATE_SCALAR) p.gbeta_k[tok] = acc_bk[tid];
+    if (a.key_scale == DN_GATE_SCALAR) p.gkey_scale[tok] = acc_d[tid];
+  }
+}
+
+// ------------------------------------------------------------------ host side
+template <int DK>
+constexpr size_t prep_smem() {
+  return sizeof(float) * (3 * kC * (DK + 4) + 2 * kC * kLDC + 768 + 2 * DK);
+}
+template <int DK>
+constexpr size_t state_smem() {
+  return sizeof(float) * (DK * (kDVS + 4) + 2 * kC * (DK + 4) + kC * kLDC + kC * (kDVS + 4) + 2 * DK);
+}
+template <int DK>
+constexpr size_t dstate_smem() {
+  return sizeof(float) * (DK * (kDVS + 4) + 3 * kC * (DK + 4) + 2 * kC * kLDC + 2 * kC * (kDVS + 4) + 2 * DK);
+}
+template <int DV>
+constexpr size_t local_smem() {
+  return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 4 * kC * (kDKS + 4) + 2 * kDKS +
+                          4 * kDKS + 3 * kC);
+}
+
+template <class K>
+cudaError_t launch(K kernel, unsigned grid, size_t smem, cudaStream_t s, const BwdArgs& p) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kernel<<<grid, kNT, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int DK, int DV>
+cudaError_t launch_dims(const BwdArgs& p, cudaStream_t s) {
+  static_assert(local_smem<DV>() <= 227 * 1024 && dstate_smem<DK>() <= 227 * 1024, "shared memory");
+  const int64_t bh = (int64_t)p.f.B * p.f.H;
+  const unsigned chunks = (unsigned)(bh * p.nc), chains = (unsigned)(bh * (DV / kDVS));
+  cudaError_t e;
+  if ((e = launch(bwd_prep_kernel<DK>, chunks, prep_smem<DK>(), s, p)) != cudaSuccess) return e;
+  if ((e = launch(bwd_state_kernel<DK, DV>, chains, state_smem<DK>(), s, p)) != cudaSuccess) return e;
+  if ((e = launch(bwd_dstate_kernel<DK, DV>, chains, dstate_smem<DK>(), s, p)) != cudaSuccess) return e;
+  return launch(bwd_local_kernel<DK, DV>, chunks, local_smem<DV>(), s, p);
+}
+
+}  // namespace
+
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  const int64_t nc = (T + kC - 1) / kC;
+  const int64_t per = 2LL * kC * kC + 2LL * dk * dv + 2LL * kC * dv;
+  return (size_t)((int64_t)B * H * nc * per) * sizeof(float);
+}
+
+cudaError_t launch_chunk_bwd(const Args& f, const void* dO, const float* dS_T, void* gq, void* gk, void* gv,
+                             float* galpha, float* gbeta_k, float* gbeta_v, float* gkey_scale, float* gS0, float* ws,
+                             cudaStream_t s) {
+  BwdArgs p;
+  p.f = f;
+  p.dO = dO;
+  p.dS_T = dS_T;
+  p.gq = gq;
+  p.gk = gk;
+  p.gv = gv;
+  p.galpha = galpha;
+  p.gbeta_k = gbeta_k;
+  p.gbeta_v = gbeta_v;
+  p.gkey_scale = gkey_scale;
+  p.gS0 = gS0;
+  p.nc = (f.T + kC - 1) / kC;
+  const int64_t blocks = (int64_t)f.B * f.H * p.nc;
+  p.wT = ws;
+  p.wP = p.wT + blocks * kC * kC;
+  p.wSm = p.wP + blocks * kC * kC;
+  p.wU = p.wSm + blocks * f.dk * f.dv;
+  p.wdX = p.wU + blocks * kC * f.dv;
+  p.wdVt = p.wdX + blocks * f.dk * f.dv;
+  if (f.dk == 128 && f.dv == 128) return launch_dims<128, 128>(p, s);
+  if (f.dk == 128 && f.dv == 64) return launch_dims<128, 64>(p, s);
+  if (f.dk == 64 && f.dv == 128) return launch_dims<64, 128>(p, s);
+  return launch_dims<64, 64>(p, s);
+}
+
+}  // namespace dn

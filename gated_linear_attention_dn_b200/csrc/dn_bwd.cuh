@@ -1,0 +1,18 @@
+// Host-side launch interface of the chunked backward (dn_bwd.cu), used by the ABI shim.
+#pragma once
+
+#include "dn_common.cuh"
+
+namespace dn {
+
+// Workspace bytes of the backward: per (b, h) and chunk of 64 tokens, the chunk's UT transform and
+// score matrix (64 x 64 each), S_m and its adjoint (d_k x d_v each), U and dV~ (64 x d_v each), fp32.
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+// Launches the four kernels of the backward on stream s. Gradient pointers of absent gates are null;
+// dS_T and gS0 may be null.
+cudaError_t launch_chunk_bwd(const Args& f, const void* dO, const float* dS_T, void* gq, void* gk, void* gv,
+                             float* galpha, float* gbeta_k, float* gbeta_v, float* gkey_scale, float* gS0, float* ws,
+                             cudaStream_t s);
+
+}  // namespace dn

@@ -228,6 +228,38 @@ dn_status dn_mc_readout(const dn_mc_desc* desc, const void* q, const float* M, c
                         void* cuda_stream);
 
 /*
+ * Chunked backward (training pass) of dn_chunk_fwd: the gradients of the scalar
+ *
+ *   L = sum_{b,t,h} <dO_t, o_t> + sum_{b,h} <dS_T, S_T>
+ *
+ * with respect to q, k, v, every gate given, and S0. The FG2-GDN page (section 3
+ * item 2) names chunk-parallel training for this DPLR update but prints no backward;
+ * this is the chain rule through the same chunk form (C = 64) that the forward uses.
+ *
+ * In:  desc, q, k, v, gates, S0 exactly as given to dn_chunk_fwd (S0 may be NULL);
+ *      dO [B,T,H,d_v] (io dtype); dS_T [B,H,d_k,d_v] fp32 or NULL (zero).
+ * Out: dq, dk [B,T,H,d_k] and dv [B,T,H,d_v] (io dtype); d_alpha, d_beta_k,
+ *      d_beta_v, d_key_scale fp32, each shaped like its gate ([B,T,H] for a
+ *      per-token gate, [B,T,H,n] per channel), given exactly when the gate is
+ *      (NULL when it is DN_GATE_ONE); dS0 [B,H,d_k,d_v] fp32 or NULL (not wanted).
+ * Scratch: `workspace` of at least dn_chunk_bwd_workspace_bytes() bytes, 16-byte
+ * aligned, owned by the caller; its contents on entry do not matter. It holds the
+ * per-chunk states S_m, residuals U, their adjoints and the chunk's UT transform.
+ * Supported: the post-update read-out (DN_READ_PRE returns DN_ERR_UNSUPPORTED),
+ * d_k, d_v in {64, 128}, alpha > 0. dq, dk, dv must not overlap each other, q, k, v,
+ * dO, S0 or the workspace. fp32 arithmetic throughout. T == 0 writes dS0 = dS_T (or
+ * zeros). Asynchronous on the stream.
+ */
+size_t dn_chunk_bwd_workspace_bytes(const dn_desc* desc);
+
+dn_status dn_chunk_bwd(const dn_desc* desc, const void* q, const void* k, const void* v,
+                       const float* alpha, const float* beta_k, const float* beta_v,
+                       const float* key_scale, const float* S0, const void* dO, const float* dS_T,
+                       void* dq, void* dk, void* dv, float* d_alpha, float* d_beta_k, float* d_beta_v,
+                       float* d_key_scale, float* dS0, void* workspace, size_t workspace_bytes,
+                       void* cuda_stream);
+
+/*
  * Synchronises `cuda_stream`, then reports (and clears) the device status word
  * that kernels set when a bounded wait gives up (DN_ERR_DEVICE_TIMEOUT), or
  * DN_ERR_CUDA if the stream holds a CUDA error. DN_OK otherwise.

@@ -170,3 +170,47 @@ def test_osdn_workspace_and_validation(lib):
     assert call(_odesc(), d=P(1 << 24)) == dn.DN_ERR_INVALID_ARGUMENT  # output overlaps the workspace
     # T == 0 with no d_T: nothing to do
     assert call(_odesc(T=0), k=None, beta=None, d=None, w=None, wb=0) == dn.DN_OK
+
+
+def _bwd_call(lib, desc, ws_bytes=None, **ptrs):
+    names = ("q", "k", "v", "a", "bk", "bv", "d", "s0", "dO", "dST", "gq", "gk", "gv", "ga", "gbk", "gbv", "gd",
+             "gs0", "ws")
+    bufs = {n: _Buf() for n in names}
+    p = {n: b.p() for n, b in bufs.items()}
+    for n in ("bv", "d", "gbv", "gd"):  # the default descriptor has no beta^v and no key scale
+        p[n] = None
+    p.update(ptrs)
+    if ws_bytes is None:
+        ws_bytes = lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(desc))
+    return lib.dn_chunk_bwd(ctypes.byref(desc), *(p[n] for n in names), ws_bytes, None)
+
+
+def test_bwd_workspace_bytes(lib):
+    d = _desc(B=2, T=130, H=3, d_k=128, d_v=64)
+    nc = 3  # ceil(130 / 64)
+    per = 2 * 64 * 64 + 2 * 128 * 64 + 2 * 64 * 64
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(d)) == 2 * 3 * nc * per * 4
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(d_k=8, d_v=8))) == 0   # small states: no backward
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(readout=dn.DN_READ_PRE))) == 0
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    assert _bwd_call(lib, _desc(readout=dn.DN_READ_PRE), ws_bytes=1 << 20) == dn.DN_ERR_UNSUPPORTED
+    assert _bwd_call(lib, _desc(d_k=16, d_v=16), ws_bytes=1 << 20) == dn.DN_ERR_UNSUPPORTED
+    assert _bwd_call(lib, _desc(B=0)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _bwd_call(lib, _desc(), dO=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _bwd_call(lib, _desc(), gq=None) == dn.DN_ERR_INVALID_ARGUMENT
+    # a gate gradient is given exactly when its gate is
+    assert _bwd_call(lib, _desc(), ga=None) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _bwd_call(lib, _desc(), gbv=_Buf().p()) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _bwd_call(lib, _desc(), gbk=_Buf().p(2)) == dn.DN_ERR_MISALIGNED
+    assert _bwd_call(lib, _desc(), gq=_Buf().p(8)) == dn.DN_ERR_MISALIGNED
+    assert _bwd_call(lib, _desc(), dST=_Buf().p(4)) == dn.DN_ERR_MISALIGNED
+    need = lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc()))
+    assert _bwd_call(lib, _desc(), ws_bytes=need - 1) == dn.DN_ERR_WORKSPACE_TOO_SMALL
+    assert _bwd_call(lib, _desc(), ws=None) == dn.DN_ERR_WORKSPACE_TOO_SMALL
+    # the q gradient may not overlap q (it is written while q is still read)
+    shared = _Buf(1 << 16)
+    assert _bwd_call(lib, _desc(), q=shared.p(), gq=shared.p(256)) == dn.DN_ERR_INVALID_ARGUMENT
+    # no tokens and no dS0 wanted: nothing to do
+    assert _bwd_call(lib, _desc(T=0), gs0=None) == dn.DN_OK
