@@ -18,10 +18,12 @@
 //
 // Four kernels, all fp32 with the dense per-chunk products on warp tensor cores (mma.sync TF32 with
 // a three-product hi/lo split, so each product keeps about fp32 accuracy):
-//   bwd_prep   one CTA per chunk:                 T and P of every chunk          -> workspace
+//   bwd_prep   one CTA per chunk: the chunk's K+, Q+, W-, e^h, e^r, lam, T and P -> workspace
 //   bwd_state  one CTA per (b, h, 32 columns of d_v), chunks in order:   S_m, U  -> workspace
 //   bwd_dstate one CTA per (b, h, 32 columns of d_v), chunks in reverse: dX, dV~ -> workspace; dS0
 //   bwd_local  one CTA per chunk: dq, dk, dv and the gate gradients (key channels in slices of 32)
+// The two chains are sequential over chunks; all elementwise work (gates, logs, exponentials) is done
+// once per chunk by bwd_prep, so a chain step only copies its operands in (cp.async) and multiplies.
 #include "dn_bwd.cuh"
 #include "dn_ut_inverse.cuh"
 
@@ -32,6 +34,7 @@ constexpr int kC = 64;     // chunk length
 constexpr int kNT = 256;   // threads per CTA (8 warps)
 constexpr int kDVS = 32;   // value columns per chain CTA
 constexpr int kDKS = 32;   // key channels per slice of the local-gradient kernel
+constexpr int kLDS = kDVS + 2;  // row stride of the chain kernels' d_v-slice arrays
 
 struct BwdArgs {
   Args f;  // forward inputs and sizes
@@ -47,6 +50,12 @@ struct BwdArgs {
   float* gS0;
   float* wT;    // [BH][nc][C][C]
   float* wP;    // [BH][nc][C][C]
+  float* wKp;   // [BH][nc][C][dk]: K+
+  float* wQp;   // [BH][nc][C][dk]: Q+
+  float* wWm;   // [BH][nc][C][dk]: W-
+  float* wEh;   // [BH][nc][C][dk]: e^h
+  float* wEr;   // [BH][nc][dk]:    e^r
+  float* wLam;  // [BH][nc][dk]:    lam
   float* wSm;   // [BH][nc][dk][dv]
   float* wU;    // [BH][nc][C][dv]
   float* wdX;   // [BH][nc][dk][dv]
@@ -112,17 +121,28 @@ __device__ __forceinline__ int64_t token(const Args& a, int b, int h, int t) {
 
 // Key channels [i0, i0 + NCH) of the chunk starting at token t0 (n valid tokens) of head (b, h), into
 // [C][NCH + 4] arrays: hb = h_t, Kp = k e^h, Qp = q e^h, Wm = w e^-h (Kp, Qp may be null; hb may be
-// Wm itself), er = e^r, lam = e^{g_last - r}. Tokens past the end have k = q = w = 0 and alpha = 1.
+// Wm itself), er = e^r, lam = e^{g_last - r}; e^h also to global ehg ([C][NCH]) when not null.
+// Tokens past the end have k = q = w = 0 and alpha = 1.
 // Called by all kNT threads; returns after a barrier.
 template <int NCH>
 __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, float* hb, float* Kp, float* Qp,
-                           float* Wm, float* er, float* lam, int tid) {
-  constexpr int LD = NCH + 4;
-  for (int e = tid; e < kC * NCH; e += kNT) {
-    const int t = e / NCH, i = e % NCH;
-    float la = 0.f;
-    if (t < n) la = logf(gate_load(a.alpha_p, a.alpha, token(a, b, h, t0 + t), a.dk, i0 + i));
-    hb[t * LD + i] = la;
+                           float* Wm, float* er, float* lam, float* ehg, int tid) {
+  constexpr int LD = NCH + 4, PER = kC * NCH / kNT, BAT = PER < 8 ? PER : 8;
+  static_assert(PER * kNT == kC * NCH && PER % BAT == 0, "work split");
+  // Every loop below first loads a batch into registers and only then computes and stores to
+  // shared memory, so a thread's global loads are all in flight at once.
+  {
+    float al[PER];
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * kNT, t = e / NCH, i = e % NCH;
+      al[it] = t < n ? gate_load(a.alpha_p, a.alpha, token(a, b, h, t0 + t), a.dk, i0 + i) : 1.f;
+    }
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * kNT, t = e / NCH, i = e % NCH;
+      hb[t * LD + i] = logf(al[it]);
+    }
   }
   __syncthreads();
   const int tr = (n - 1) / 2;
@@ -138,29 +158,50 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
     lam[i] = expf(run - r);
   }
   __syncthreads();
-  for (int e = tid; e < kC * NCH; e += kNT) {
-    const int t = e / NCH, i = e % NCH;
-    const float hv = hb[t * LD + i];
-    float kk = 0.f, qq = 0.f, w = 0.f;
-    if (t < n) {
-      const int64_t tok = token(a, b, h, t0 + t);
-      kk = io_load(a.k, tok * a.dk + i0 + i, a.io_bf16);
-      if (Qp) qq = io_load(a.q, tok * a.dk + i0 + i, a.io_bf16);
-      w = gate_load(a.beta_k_p, a.beta_k, tok, a.dk, i0 + i) * gate_load(a.key_scale_p, a.key_scale, tok, a.dk, i0 + i) *
-          kk;
+  for (int it0 = 0; it0 < PER; it0 += BAT) {
+    float kk[BAT], qq[BAT], ws[BAT];
+#pragma unroll
+    for (int u = 0; u < BAT; ++u) {
+      const int e = tid + (it0 + u) * kNT, t = e / NCH, i = e % NCH;
+      kk[u] = qq[u] = ws[u] = 0.f;
+      if (t < n) {
+        const int64_t tok = token(a, b, h, t0 + t);
+        kk[u] = io_load(a.k, tok * a.dk + i0 + i, a.io_bf16);
+        if (Qp) qq[u] = io_load(a.q, tok * a.dk + i0 + i, a.io_bf16);
+        ws[u] = gate_load(a.beta_k_p, a.beta_k, tok, a.dk, i0 + i) * gate_load(a.key_scale_p, a.key_scale, tok, a.dk, i0 + i);
+      }
     }
-    const float eh = expf(hv);
-    if (Kp) Kp[t * LD + i] = kk * eh;
-    if (Qp) Qp[t * LD + i] = qq * eh;
-    Wm[t * LD + i] = w / eh;
+#pragma unroll
+    for (int u = 0; u < BAT; ++u) {
+      const int e = tid + (it0 + u) * kNT, t = e / NCH, i = e % NCH;
+      const float eh = expf(hb[t * LD + i]);
+      if (ehg) ehg[t * NCH + i] = eh;
+      if (Kp) Kp[t * LD + i] = kk[u] * eh;
+      if (Qp) Qp[t * LD + i] = qq[u] * eh;
+      Wm[t * LD + i] = ws[u] * kk[u] / eh;
+    }
   }
   __syncthreads();
+}
+
+constexpr int kLDC = kC + 4;  // row stride of shared 64 x 64 arrays
+
+// cp.async copy of a ROWS x COLS fp32 block (global row stride gs floats) into shared rows of ss
+// floats; 16-byte granules, so COLS, gs, ss and both bases must be multiples of 4 floats. The caller
+// commits and waits.
+template <int ROWS, int COLS>
+__device__ __forceinline__ void async_rows(float* sm, int ss, const float* g, int64_t gs, int tid) {
+  constexpr int V = COLS / 4;
+  static_assert(COLS % 4 == 0, "16-byte granules");
+  for (int e = tid; e < ROWS * V; e += kNT) {
+    const int r = e / V, c = (e % V) * 4;
+    tc::cp_async_16_zfill(sm + r * ss + c, g + r * gs + c, 16);
+  }
 }
 
 // T = (I + L)^-1 for the strictly lower 64 x 64 L in Lm (row stride LDC) into Tm (same stride), fp32.
 // The four 16 x 16 diagonal blocks by forward substitution (one column per thread), then the blocks
 // below the diagonal by block distance d: T_ij = -T_ii sum_{j <= k < i} L_ik T_kj. scr: 768 floats.
-constexpr int kLDC = kC + 4;
 __device__ void inverse64(const float* Lm, float* Tm, float* scr, int tid) {
   for (int e = tid; e < kC * kC; e += kNT) Tm[(e / kC) * kLDC + e % kC] = 0.f;
   __syncthreads();
@@ -200,7 +241,7 @@ __device__ void inverse64(const float* Lm, float* Tm, float* scr, int tid) {
   }
 }
 
-// ------------------------------------------------------------------ kernel 1: T and P per chunk
+// ------------------------------------------------------------------ kernel 1: per-chunk operands
 template <int DK>
 __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
@@ -208,32 +249,48 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
   float* Kp = reinterpret_cast<float*>(smem4);
   float* Qp = Kp + kC * LDK;
   float* Wm = Qp + kC * LDK;
-  float* Lm = Wm + kC * LDK;
-  float* Tm = Lm + kC * kLDC;
-  float* scr = Tm + kC * kLDC;
+  float* scr = Wm + kC * LDK;
   float* er = scr + 768;
   float* lam = er + DK;
+  float* Lm = Kp;  // once K+ and Q+ are consumed, their space holds L and T
+  float* Tm = Qp;
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x % p.nc, bh = blockIdx.x / p.nc, b = bh / a.H, h = bh % a.H;
   const int t0 = c * kC, n = min(kC, a.T - t0);
-  prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, tid);
-
   const int64_t cb = (int64_t)bh * p.nc + c;
-  {  // warps 0-3: L = strictly-lower(K+ W-^T); warps 4-7: P = lower-incl(Q+ W-^T); 32 x 32 tiles
-    const int m0 = ((warp & 3) >> 1) * 32, n0 = (warp & 1) * 32;
+  prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, p.wEh + cb * kC * DK, tid);
+
+  // warps 0-3: L = strictly-lower(K+ W-^T) (kept in registers); warps 4-7: P = lower-incl(Q+ W-^T)
+  const int m0 = ((warp & 3) >> 1) * 32, n0 = (warp & 1) * 32;
+  float acc[2][4][4] = {};
+  {
     const float* X = warp < 4 ? Kp : Qp;
-    float acc[2][4][4] = {};
     warp_gemm<2, 4, DK>(
         acc, [&](int m, int k) { return X[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return Wm[(n0 + nn) * LDK + k]; },
         lane);
-    if (warp < 4) {
-      warp_epilogue(acc, [&](int m, int nn, float v) { Lm[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? v : 0.f; }, lane);
-    } else {
-      float* P = p.wP + cb * kC * kC;
-      warp_epilogue(acc, [&](int m, int nn, float v) { P[(m0 + m) * kC + n0 + nn] = n0 + nn <= m0 + m ? v : 0.f; }, lane);
-    }
   }
+  if (warp >= 4) {
+    float* P = p.wP + cb * kC * kC;
+    warp_epilogue(acc, [&](int m, int nn, float v) { P[(m0 + m) * kC + n0 + nn] = n0 + nn <= m0 + m ? v : 0.f; }, lane);
+  }
+  if (tid < DK) {
+    p.wEr[cb * DK + tid] = er[tid];
+    p.wLam[cb * DK + tid] = lam[tid];
+  }
+  {  // K+, Q+, W- to the workspace
+    float* dst[3] = {p.wKp + cb * kC * DK, p.wQp + cb * kC * DK, p.wWm + cb * kC * DK};
+    const float* src[3] = {Kp, Qp, Wm};
+#pragma unroll
+    for (int q = 0; q < 3; ++q)
+      for (int e = tid; e < kC * DK / 4; e += kNT) {
+        const int t = e / (DK / 4), i = (e % (DK / 4)) * 4;
+        *reinterpret_cast<float4*>(dst[q] + t * DK + i) = *reinterpret_cast<const float4*>(src[q] + t * LDK + i);
+      }
+  }
+  __syncthreads();  // K+ and Q+ are consumed
+  if (warp < 4)
+    warp_epilogue(acc, [&](int m, int nn, float v) { Lm[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? v : 0.f; }, lane);
   __syncthreads();
   inverse64(Lm, Tm, scr, tid);
   float* Tg = p.wT + cb * kC * kC;
@@ -244,7 +301,7 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDS = kDVS + 4;
+  constexpr int LDK = DK + 4, LDS = kLDS;
   float* S = reinterpret_cast<float*>(smem4);  // [DK][LDS]
   float* Kp = S + DK * LDS;                     // [C][LDK]
   float* Wm = Kp + kC * LDK;                    // [C][LDK]
@@ -265,18 +322,32 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
     const int t0 = c * kC, n = min(kC, a.T - t0);
     const int64_t cb = (int64_t)bh * p.nc + c;
     __syncthreads();  // the previous chunk is done with every buffer
-    prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, nullptr, Wm, er, lam, tid);
-    const float* Tg = p.wT + cb * kC * kC;
-    for (int e = tid; e < kC * kC; e += kNT) Tm[(e / kC) * kLDC + e % kC] = Tg[e];
-    for (int e = tid; e < kC * kDVS; e += kNT) {
-      const int t = e / kDVS, j = e % kDVS;
-      float x = 0.f;
-      if (t < n) {
-        const int64_t tok = token(a, b, h, t0 + t);
-        x = gate_load(a.beta_v_p, a.beta_v, tok, DV, j0 + j) * io_load(a.v, tok * DV + j0 + j, a.io_bf16);
+    async_rows<kC, DK>(Kp, LDK, p.wKp + cb * kC * DK, DK, tid);
+    async_rows<kC, DK>(Wm, LDK, p.wWm + cb * kC * DK, DK, tid);
+    async_rows<kC, kC>(Tm, kLDC, p.wT + cb * kC * kC, kC, tid);
+    async_rows<1, DK>(er, 0, p.wEr + cb * DK, 0, tid);
+    async_rows<1, DK>(lam, 0, p.wLam + cb * DK, 0, tid);
+    tc::cp_async_commit();
+    {
+      constexpr int PER = kC * kDVS / kNT;
+      float x[PER];
+#pragma unroll
+      for (int it = 0; it < PER; ++it) {
+        const int e = tid + it * kNT, t = e / kDVS, j = e % kDVS;
+        x[it] = 0.f;
+        if (t < n) {
+          const int64_t tok = token(a, b, h, t0 + t);
+          x[it] = gate_load(a.beta_v_p, a.beta_v, tok, DV, j0 + j) * io_load(a.v, tok * DV + j0 + j, a.io_bf16);
+        }
       }
-      R[t * LDS + j] = x;
+#pragma unroll
+      for (int it = 0; it < PER; ++it) {
+        const int e = tid + it * kNT;
+        R[(e / kDVS) * LDS + e % kDVS] = x[it];
+      }
     }
+    tc::cp_async_wait_all();
+    __syncthreads();
     float* Smg = p.wSm + cb * DK * DV;
     for (int e = tid; e < DK * kDVS; e += kNT) {
       const int i = e / kDVS, j = e % kDVS;
@@ -329,7 +400,7 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDS = kDVS + 4;
+  constexpr int LDK = DK + 4, LDS = kLDS;
   float* dS = reinterpret_cast<float*>(smem4);  // [DK][LDS]: dS', then dX, then dS
   float* Qp = dS + DK * LDS;                     // [C][LDK]
   float* Kp = Qp + kC * LDK;
@@ -353,17 +424,30 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
     const int t0 = c * kC, n = min(kC, a.T - t0);
     const int64_t cb = (int64_t)bh * p.nc + c;
     __syncthreads();
-    prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, tid);
-    const float* Tg = p.wT + cb * kC * kC;
-    const float* Pg = p.wP + cb * kC * kC;
-    for (int e = tid; e < kC * kC; e += kNT) {
-      Tm[(e / kC) * kLDC + e % kC] = Tg[e];
-      Pm[(e / kC) * kLDC + e % kC] = Pg[e];
+    async_rows<kC, DK>(Qp, LDK, p.wQp + cb * kC * DK, DK, tid);
+    async_rows<kC, DK>(Kp, LDK, p.wKp + cb * kC * DK, DK, tid);
+    async_rows<kC, DK>(Wm, LDK, p.wWm + cb * kC * DK, DK, tid);
+    async_rows<kC, kC>(Tm, kLDC, p.wT + cb * kC * kC, kC, tid);
+    async_rows<kC, kC>(Pm, kLDC, p.wP + cb * kC * kC, kC, tid);
+    async_rows<1, DK>(er, 0, p.wEr + cb * DK, 0, tid);
+    async_rows<1, DK>(lam, 0, p.wLam + cb * DK, 0, tid);
+    tc::cp_async_commit();
+    {
+      constexpr int PER = kC * kDVS / kNT;
+      float x[PER];
+#pragma unroll
+      for (int it = 0; it < PER; ++it) {
+        const int e = tid + it * kNT, t = e / kDVS, j = e % kDVS;
+        x[it] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j0 + j, a.io_bf16) : 0.f;
+      }
+#pragma unroll
+      for (int it = 0; it < PER; ++it) {
+        const int e = tid + it * kNT;
+        dOs[(e / kDVS) * LDS + e % kDVS] = x[it];
+      }
     }
-    for (int e = tid; e < kC * kDVS; e += kNT) {
-      const int t = e / kDVS, j = e % kDVS;
-      dOs[t * LDS + j] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j0 + j, a.io_bf16) : 0.f;
-    }
+    tc::cp_async_wait_all();
+    __syncthreads();
     float* dXg = p.wdX + cb * DK * DV;
     for (int e = tid; e < DK * kDVS; e += kNT) {
       const int i = e / kDVS, j = e % kDVS;
@@ -437,13 +521,11 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   float* dL = dP + kC * kLDC;
   float* Sm = dL + kC * kLDC;   // [kDKS][LDV]: rows i0.. of S_m
   float* dX = Sm + kDKS * LDV;  // [kDKS][LDV]
-  float* hb = dX + kDKS * LDV;  // [C][LDS]
-  float* Qp = hb + kC * LDS;    // then the beta^k gradient terms
+  float* Eh = dX + kDKS * LDV;  // [C][LDS]: e^h
+  float* Qp = Eh + kC * LDS;    // then the beta^k gradient terms
   float* Kp = Qp + kC * LDS;    // then the d gradient terms
   float* Wm = Kp + kC * LDS;    // then dh, then d log alpha
-  float* er = Wm + kC * LDS;
-  float* lam = er + kDKS;
-  float* red = lam + kDKS;    // [4][kDKS]
+  float* red = Wm + kC * LDS;   // [4][kDKS]
   float* acc_a = red + 4 * kDKS;  // [C] per-token sums for gates of width 1
   float* acc_bk = acc_a + kC;
   float* acc_d = acc_bk + kC;
@@ -453,24 +535,60 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   const int t0 = c * kC, n = min(kC, a.T - t0);
   const int64_t cb = (int64_t)bh * p.nc + c;
   {
-    const float* Ug = p.wU + cb * kC * DV;
-    const float* dVg = p.wdVt + cb * kC * DV;
-    for (int e = tid; e < kC * DV; e += kNT) {
-      const int t = e / DV, j = e % DV;
-      U[t * LDV + j] = Ug[e];
-      dVt[t * LDV + j] = dVg[e];
-      dOs[t * LDV + j] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j, a.io_bf16) : 0.f;
+    constexpr int PER4 = kC * DV / 4 / kNT;  // float4 per thread of a C x DV array
+    const float4* Ug = reinterpret_cast<const float4*>(p.wU + cb * kC * DV);
+    const float4* dVg = reinterpret_cast<const float4*>(p.wdVt + cb * kC * DV);
+    float4 xu[PER4], xv[PER4];
+#pragma unroll
+    for (int it = 0; it < PER4; ++it) {
+      xu[it] = Ug[tid + it * kNT];
+      xv[it] = dVg[tid + it * kNT];
+    }
+#pragma unroll
+    for (int it = 0; it < PER4; ++it) {
+      const int e = (tid + it * kNT) * 4, t = e / DV, j = e % DV;
+      *reinterpret_cast<float4*>(&U[t * LDV + j]) = xu[it];
+      *reinterpret_cast<float4*>(&dVt[t * LDV + j]) = xv[it];
+    }
+    for (int it0 = 0; it0 < kC * DV / kNT; it0 += 8) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
+        x[u] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j, a.io_bf16) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = tid + (it0 + u) * kNT;
+        dOs[(e / DV) * LDV + e % DV] = x[u];
+      }
     }
     if (tid < kC) acc_a[tid] = acc_bk[tid] = acc_d[tid] = 0.f;
   }
   __syncthreads();
   // dv = beta^v dV~, and the beta^v gradient v dV~ (summed over channels for a per-token gate)
-  for (int e = tid; e < n * DV; e += kNT) {
-    const int t = e / DV, j = e % DV;
-    const int64_t tok = token(a, b, h, t0 + t);
-    const float dvt = dVt[t * LDV + j];
-    io_store(p.gv, tok * DV + j, gate_load(a.beta_v_p, a.beta_v, tok, DV, j) * dvt, a.io_bf16);
-    if (a.beta_v == DN_GATE_CHANNEL) p.gbeta_v[tok * DV + j] = io_load(a.v, tok * DV + j, a.io_bf16) * dvt;
+  for (int it0 = 0; it0 < kC * DV / kNT; it0 += 8) {
+    float bv[8], vv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
+      bv[u] = vv[u] = 0.f;
+      if (t < n) {
+        const int64_t tok = token(a, b, h, t0 + t);
+        bv[u] = gate_load(a.beta_v_p, a.beta_v, tok, DV, j);
+        if (a.beta_v == DN_GATE_CHANNEL) vv[u] = io_load(a.v, tok * DV + j, a.io_bf16);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
+      if (t < n) {
+        const int64_t tok = token(a, b, h, t0 + t);
+        const float dvt = dVt[t * LDV + j];
+        io_store(p.gv, tok * DV + j, bv[u] * dvt, a.io_bf16);
+        if (a.beta_v == DN_GATE_CHANNEL) p.gbeta_v[tok * DV + j] = vv[u] * dvt;
+      }
+    }
   }
   if (a.beta_v == DN_GATE_SCALAR) {
     for (int t = warp; t < n; t += kNT / 32) {  // uniform per warp: every lane takes part in the shuffles
@@ -502,12 +620,14 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   constexpr int XN = DV / 4, NIX = XN / 8;                 // X (32 x DV, channel x column): 16 x XN warp tiles
   const int mx = (warp >> 2) * 16, nx = (warp & 3) * XN;
   for (int i0 = 0; i0 < DK; i0 += kDKS) {
-    prep_chunk<kDKS>(a, b, h, t0, n, i0, hb, Kp, Qp, Wm, er, lam, tid);
-    for (int e = tid; e < kDKS * DV; e += kNT) {
-      const int i = e / DV, j = e % DV;
-      Sm[i * LDV + j] = Smg[(int64_t)(i0 + i) * DV + j];
-      dX[i * LDV + j] = dXg[(int64_t)(i0 + i) * DV + j];
-    }
+    async_rows<kC, kDKS>(Eh, LDS, p.wEh + cb * kC * DK + i0, DK, tid);
+    async_rows<kC, kDKS>(Qp, LDS, p.wQp + cb * kC * DK + i0, DK, tid);
+    async_rows<kC, kDKS>(Kp, LDS, p.wKp + cb * kC * DK + i0, DK, tid);
+    async_rows<kC, kDKS>(Wm, LDS, p.wWm + cb * kC * DK + i0, DK, tid);
+    async_rows<kDKS, DV>(Sm, LDV, Smg + (int64_t)i0 * DV, DV, tid);
+    async_rows<kDKS, DV>(dX, LDV, dXg + (int64_t)i0 * DV, DV, tid);
+    tc::cp_async_commit();
+    tc::cp_async_wait_all();
     __syncthreads();
     float aq[1][2][4] = {}, ak[1][2][4] = {}, aw[1][2][4] = {}, ax[1][NIX][4] = {};
     // dQ+ = dO S_m^T + dP W-
@@ -560,21 +680,29 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
     {
       // Per (token, channel) of this warp's tiles: dq, dk, the beta^k and d gradients, and dh. Each
       // thread then reads and writes only its own elements of hb, Qp, Kp, Wm.
-      float gq[2][4], gk[2][4];
-      auto elem = [&](int ni, int q, int m, int nn, float vq, float vk, float vw) {
-        const int t = m0 + m, il = n0 + nn, gi = i0 + il;
-        const float eh = expf(hb[t * LDS + il]);
-        const float dw = vw / eh;
-        float gbk = 0.f, gdd = 0.f, dk = 0.f;
-        if (t < n) {
-          const int64_t tok = token(a, b, h, t0 + t);
-          const float kk = io_load(a.k, tok * DK + gi, a.io_bf16);
-          const float bk = gate_load(a.beta_k_p, a.beta_k, tok, DK, gi);
-          const float dd = gate_load(a.key_scale_p, a.key_scale, tok, DK, gi);
-          dk = vk * eh + bk * dd * dw;
-          gbk = dd * kk * dw;
-          gdd = bk * kk * dw;
+      float gq[2][4], gk[2][4], lk[2][4], lb[2][4], ld[2][4];
+      const int g = lane >> 2, t4 = lane & 3;
+#pragma unroll
+      for (int ni = 0; ni < 2; ++ni)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // the inputs of this thread's elements, loaded up front
+          const int t = m0 + g + (q >> 1) * 8, gi = i0 + n0 + 8 * ni + 2 * t4 + (q & 1);
+          lk[ni][q] = 0.f;
+          lb[ni][q] = ld[ni][q] = 1.f;
+          if (t < n) {
+            const int64_t tok = token(a, b, h, t0 + t);
+            lk[ni][q] = io_load(a.k, tok * DK + gi, a.io_bf16);
+            lb[ni][q] = gate_load(a.beta_k_p, a.beta_k, tok, DK, gi);
+            ld[ni][q] = gate_load(a.key_scale_p, a.key_scale, tok, DK, gi);
+          }
         }
+      auto elem = [&](int ni, int q, int m, int nn, float vq, float vk, float vw) {
+        const int t = m0 + m, il = n0 + nn;
+        const float eh = Eh[t * LDS + il];
+        const float dw = vw / eh;
+        const float kk = lk[ni][q], bk = lb[ni][q], dd = ld[ni][q];
+        const float dk = vk * eh + bk * dd * dw;
+        const float gbk = dd * kk * dw, gdd = bk * kk * dw;
         gq[ni][q] = vq * eh;
         gk[ni][q] = dk;
         const float dh = Qp[t * LDS + il] * vq + Kp[t * LDS + il] * vk - Wm[t * LDS + il] * vw;
@@ -582,7 +710,6 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
         Kp[t * LDS + il] = gdd;
         Wm[t * LDS + il] = dh;
       };
-      const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
       for (int ni = 0; ni < 2; ++ni) {
         elem(ni, 0, g, 8 * ni + 2 * t4, aq[0][ni][0], ak[0][ni][0], aw[0][ni][0]);
@@ -643,20 +770,20 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
 // ------------------------------------------------------------------ host side
 template <int DK>
 constexpr size_t prep_smem() {
-  return sizeof(float) * (3 * kC * (DK + 4) + 2 * kC * kLDC + 768 + 2 * DK);
+  return sizeof(float) * (3 * kC * (DK + 4) + 768 + 2 * DK);
 }
 template <int DK>
 constexpr size_t state_smem() {
-  return sizeof(float) * (DK * (kDVS + 4) + 2 * kC * (DK + 4) + kC * kLDC + kC * (kDVS + 4) + 2 * DK);
+  return sizeof(float) * (DK * kLDS + 2 * kC * (DK + 4) + kC * kLDC + kC * kLDS + 2 * DK);
 }
 template <int DK>
 constexpr size_t dstate_smem() {
-  return sizeof(float) * (DK * (kDVS + 4) + 3 * kC * (DK + 4) + 2 * kC * kLDC + 2 * kC * (kDVS + 4) + 2 * DK);
+  return sizeof(float) * (DK * kLDS + 3 * kC * (DK + 4) + 2 * kC * kLDC + 2 * kC * kLDS + 2 * DK);
 }
 template <int DV>
 constexpr size_t local_smem() {
-  return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 4 * kC * (kDKS + 4) + 2 * kDKS +
-                          4 * kDKS + 3 * kC);
+  return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 4 * kC * (kDKS + 4) + 4 * kDKS +
+                          3 * kC);
 }
 
 template <class K>
@@ -683,7 +810,7 @@ cudaError_t launch_dims(const BwdArgs& p, cudaStream_t s) {
 
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
   const int64_t nc = (T + kC - 1) / kC;
-  const int64_t per = 2LL * kC * kC + 2LL * dk * dv + 2LL * kC * dv;
+  const int64_t per = 2LL * kC * kC + 2LL * dk * dv + 2LL * kC * dv + 4LL * kC * dk + 2LL * dk;
   return (size_t)((int64_t)B * H * nc * per) * sizeof(float);
 }
 
@@ -710,6 +837,12 @@ cudaError_t launch_chunk_bwd(const Args& f, const void* dO, const float* dS_T, v
   p.wU = p.wSm + blocks * f.dk * f.dv;
   p.wdX = p.wU + blocks * kC * f.dv;
   p.wdVt = p.wdX + blocks * f.dk * f.dv;
+  p.wKp = p.wdVt + blocks * kC * f.dv;
+  p.wQp = p.wKp + blocks * kC * f.dk;
+  p.wWm = p.wQp + blocks * kC * f.dk;
+  p.wEh = p.wWm + blocks * kC * f.dk;
+  p.wEr = p.wEh + blocks * kC * f.dk;
+  p.wLam = p.wEr + blocks * f.dk;
   if (f.dk == 128 && f.dv == 128) return launch_dims<128, 128>(p, s);
   if (f.dk == 128 && f.dv == 64) return launch_dims<128, 64>(p, s);
   if (f.dk == 64 && f.dv == 128) return launch_dims<64, 128>(p, s);

@@ -188,7 +188,8 @@ def _bwd_call(lib, desc, ws_bytes=None, **ptrs):
 def test_bwd_workspace_bytes(lib):
     d = _desc(B=2, T=130, H=3, d_k=128, d_v=64)
     nc = 3  # ceil(130 / 64)
-    per = 2 * 64 * 64 + 2 * 128 * 64 + 2 * 64 * 64
+    # per chunk: T, P (64 x 64); S_m, dX (d_k x d_v); U, dV~ (64 x d_v); K+, Q+, W-, e^h (64 x d_k); e^r, lam (d_k)
+    per = 2 * 64 * 64 + 2 * 128 * 64 + 2 * 64 * 64 + 4 * 64 * 128 + 2 * 128
     assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(d)) == 2 * 3 * nc * per * 4
     assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(d_k=8, d_v=8))) == 0   # small states: no backward
     assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(readout=dn.DN_READ_PRE))) == 0
