@@ -20,7 +20,7 @@
 // a three-product hi/lo split, so each product keeps about fp32 accuracy):
 //   bwd_prep   one CTA per chunk: the chunk's K+, Q+, W-, e^h, e^r, lam, T and P -> workspace
 //   bwd_state  one CTA per (b, h, 32 columns of d_v), chunks in order:   S_m, U  -> workspace
-//   bwd_dstate one CTA per (b, h, 32 columns of d_v), chunks in reverse: dX, dV~ -> workspace; dS0
+//   bwd_dstate one CTA per (b, h, 64 columns of d_v), chunks in reverse: dX, dV~ -> workspace; dS0
 //   bwd_local  one CTA per chunk: dq, dk, dv and the gate gradients (key channels in slices of 32)
 // The two chains are sequential over chunks; all elementwise work (gates, logs, exponentials) is done
 // once per chunk by bwd_prep, so a chain step only copies its operands in (cp.async) and multiplies.
@@ -32,9 +32,9 @@ namespace {
 
 constexpr int kC = 64;     // chunk length
 constexpr int kNT = 256;   // threads per CTA (8 warps)
-constexpr int kDVS = 32;   // value columns per chain CTA
-constexpr int kDKS = 32;   // key channels per slice of the local-gradient kernel
-constexpr int kLDS = kDVS + 2;  // row stride of the chain kernels' d_v-slice arrays
+constexpr int kDVS_STATE = 32;   // value columns per CTA of the state chain (two CTAs per SM)
+constexpr int kDVS_DSTATE = 64;  // value columns per CTA of the adjoint chain (one CTA per SM, fewer waves)
+constexpr int kDKS = 32;         // key channels per slice of the local-gradient kernel
 
 struct BwdArgs {
   Args f;  // forward inputs and sizes
@@ -298,10 +298,10 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
 }
 
 // ------------------------------------------------------------------ kernel 2: states, chunks in order
-template <int DK, int DV>
+template <int DK, int DV, int DVS>
 __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDS = kLDS;
+  constexpr int LDK = DK + 4, LDS = DVS + 2, NI = DVS / 16;
   float* S = reinterpret_cast<float*>(smem4);  // [DK][LDS]
   float* Kp = S + DK * LDS;                     // [C][LDK]
   float* Wm = Kp + kC * LDK;                    // [C][LDK]
@@ -311,13 +311,13 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   float* lam = er + DK;
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int NS = DV / kDVS;
-  const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * kDVS, b = bh / a.H, h = bh % a.H;
-  for (int e = tid; e < DK * kDVS; e += kNT) {
-    const int i = e / kDVS, j = e % kDVS;
+  constexpr int NS = DV / DVS;
+  const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * DVS, b = bh / a.H, h = bh % a.H;
+  for (int e = tid; e < DK * DVS; e += kNT) {
+    const int i = e / DVS, j = e % DVS;
     S[i * LDS + j] = a.S0 ? a.S0[((int64_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
-  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;  // this warp's 16 x 16 tile of a 64 x 32 result
+  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * (DVS / 2);  // this warp's tile of a 64 x DVS result
   for (int c = 0; c < p.nc; ++c) {
     const int t0 = c * kC, n = min(kC, a.T - t0);
     const int64_t cb = (int64_t)bh * p.nc + c;
@@ -329,11 +329,11 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
     async_rows<1, DK>(lam, 0, p.wLam + cb * DK, 0, tid);
     tc::cp_async_commit();
     {
-      constexpr int PER = kC * kDVS / kNT;
+      constexpr int PER = kC * DVS / kNT;
       float x[PER];
 #pragma unroll
       for (int it = 0; it < PER; ++it) {
-        const int e = tid + it * kNT, t = e / kDVS, j = e % kDVS;
+        const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
         x[it] = 0.f;
         if (t < n) {
           const int64_t tok = token(a, b, h, t0 + t);
@@ -343,30 +343,30 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
 #pragma unroll
       for (int it = 0; it < PER; ++it) {
         const int e = tid + it * kNT;
-        R[(e / kDVS) * LDS + e % kDVS] = x[it];
+        R[(e / DVS) * LDS + e % DVS] = x[it];
       }
     }
     tc::cp_async_wait_all();
     __syncthreads();
     float* Smg = p.wSm + cb * DK * DV;
-    for (int e = tid; e < DK * kDVS; e += kNT) {
-      const int i = e / kDVS, j = e % kDVS;
+    for (int e = tid; e < DK * DVS; e += kNT) {
+      const int i = e / DVS, j = e % DVS;
       const float x = S[i * LDS + j] * er[i];
       S[i * LDS + j] = x;
       Smg[(int64_t)i * DV + j0 + j] = x;
     }
     __syncthreads();
     {  // R = V~ - K+ S_m (each warp updates only its own tile)
-      float acc[1][2][4] = {};
-      warp_gemm<1, 2, DK>(
+      float acc[1][NI][4] = {};
+      warp_gemm<1, NI, DK>(
           acc, [&](int m, int k) { return Kp[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return S[k * LDS + n0 + nn]; },
           lane);
       warp_epilogue(acc, [&](int m, int nn, float v) { R[(m0 + m) * LDS + n0 + nn] -= v; }, lane);
     }
     __syncthreads();
     {  // U = T R
-      float acc[1][2][4] = {};
-      warp_gemm<1, 2, kC>(
+      float acc[1][NI][4] = {};
+      warp_gemm<1, NI, kC>(
           acc, [&](int m, int k) { return Tm[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return R[k * LDS + n0 + nn]; },
           lane);
       __syncthreads();
@@ -379,11 +379,11 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
                     lane);
     }
     __syncthreads();
-    // S' = Diag(lam) (S_m + W-^T U): DK x 32 in 16 x 16 tiles
+    // S' = Diag(lam) (S_m + W-^T U): DK x DVS in 16 x DVS/2 tiles
     for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
-      const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * 16;
-      float acc[1][2][4] = {};
-      warp_gemm<1, 2, kC>(
+      const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * (DVS / 2);
+      float acc[1][NI][4] = {};
+      warp_gemm<1, NI, kC>(
           acc, [&](int m, int k) { return Wm[k * LDK + r0 + m]; }, [&](int k, int nn) { return R[k * LDS + q0 + nn]; },
           lane);
       warp_epilogue(acc,
@@ -397,10 +397,10 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
 }
 
 // ------------------------------------------------------------------ kernel 3: state adjoints, chunks in reverse
-template <int DK, int DV>
+template <int DK, int DV, int DVS>
 __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDS = kLDS;
+  constexpr int LDK = DK + 4, LDS = DVS + 2, NI = DVS / 16;
   float* dS = reinterpret_cast<float*>(smem4);  // [DK][LDS]: dS', then dX, then dS
   float* Qp = dS + DK * LDS;                     // [C][LDK]
   float* Kp = Qp + kC * LDK;
@@ -413,13 +413,13 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   float* lam = er + DK;
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int NS = DV / kDVS;
-  const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * kDVS, b = bh / a.H, h = bh % a.H;
-  for (int e = tid; e < DK * kDVS; e += kNT) {
-    const int i = e / kDVS, j = e % kDVS;
+  constexpr int NS = DV / DVS;
+  const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * DVS, b = bh / a.H, h = bh % a.H;
+  for (int e = tid; e < DK * DVS; e += kNT) {
+    const int i = e / DVS, j = e % DVS;
     dS[i * LDS + j] = p.dS_T ? p.dS_T[((int64_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
-  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * 16;
+  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * (DVS / 2);
   for (int c = p.nc - 1; c >= 0; --c) {
     const int t0 = c * kC, n = min(kC, a.T - t0);
     const int64_t cb = (int64_t)bh * p.nc + c;
@@ -433,43 +433,43 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
     async_rows<1, DK>(lam, 0, p.wLam + cb * DK, 0, tid);
     tc::cp_async_commit();
     {
-      constexpr int PER = kC * kDVS / kNT;
+      constexpr int PER = kC * DVS / kNT;
       float x[PER];
 #pragma unroll
       for (int it = 0; it < PER; ++it) {
-        const int e = tid + it * kNT, t = e / kDVS, j = e % kDVS;
+        const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
         x[it] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j0 + j, a.io_bf16) : 0.f;
       }
 #pragma unroll
       for (int it = 0; it < PER; ++it) {
         const int e = tid + it * kNT;
-        dOs[(e / kDVS) * LDS + e % kDVS] = x[it];
+        dOs[(e / DVS) * LDS + e % DVS] = x[it];
       }
     }
     tc::cp_async_wait_all();
     __syncthreads();
     float* dXg = p.wdX + cb * DK * DV;
-    for (int e = tid; e < DK * kDVS; e += kNT) {
-      const int i = e / kDVS, j = e % kDVS;
+    for (int e = tid; e < DK * DVS; e += kNT) {
+      const int i = e / DVS, j = e % DVS;
       const float x = dS[i * LDS + j] * lam[i];
       dS[i * LDS + j] = x;
       dXg[(int64_t)i * DV + j0 + j] = x;
     }
     __syncthreads();
     {  // dU = P^T dO + W- dX
-      float acc[1][2][4] = {};
-      warp_gemm<1, 2, kC>(
+      float acc[1][NI][4] = {};
+      warp_gemm<1, NI, kC>(
           acc, [&](int m, int k) { return Pm[k * kLDC + m0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + n0 + nn]; },
           lane);
-      warp_gemm<1, 2, DK>(
+      warp_gemm<1, NI, DK>(
           acc, [&](int m, int k) { return Wm[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return dS[k * LDS + n0 + nn]; },
           lane);
       warp_epilogue(acc, [&](int m, int nn, float v) { dU[(m0 + m) * LDS + n0 + nn] = v; }, lane);
     }
     __syncthreads();
     {  // dV~ = T^T dU
-      float acc[1][2][4] = {};
-      warp_gemm<1, 2, kC>(
+      float acc[1][NI][4] = {};
+      warp_gemm<1, NI, kC>(
           acc, [&](int m, int k) { return Tm[k * kLDC + m0 + m]; }, [&](int k, int nn) { return dU[k * LDS + n0 + nn]; },
           lane);
       __syncthreads();
@@ -482,14 +482,14 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
                     lane);
     }
     __syncthreads();
-    // dS = Diag(e^r) (dX + Q+^T dO - K+^T dV~): DK x 32 in 16 x 16 tiles
+    // dS = Diag(e^r) (dX + Q+^T dO - K+^T dV~): DK x DVS in 16 x DVS/2 tiles
     for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
-      const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * 16;
-      float acc[1][2][4] = {};
-      warp_gemm<1, 2, kC>(
+      const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * (DVS / 2);
+      float acc[1][NI][4] = {};
+      warp_gemm<1, NI, kC>(
           acc, [&](int m, int k) { return Qp[k * LDK + r0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + q0 + nn]; },
           lane);
-      warp_gemm<1, 2, kC>(
+      warp_gemm<1, NI, kC>(
           acc, [&](int m, int k) { return -Kp[k * LDK + r0 + m]; }, [&](int k, int nn) { return dU[k * LDS + q0 + nn]; },
           lane);
       warp_epilogue(acc,
@@ -502,8 +502,8 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   }
   if (p.gS0) {
     __syncthreads();
-    for (int e = tid; e < DK * kDVS; e += kNT) {
-      const int i = e / kDVS, j = e % kDVS;
+    for (int e = tid; e < DK * DVS; e += kNT) {
+      const int i = e / DVS, j = e % DVS;
       p.gS0[((int64_t)bh * DK + i) * DV + j0 + j] = dS[i * LDS + j];
     }
   }
@@ -772,13 +772,13 @@ template <int DK>
 constexpr size_t prep_smem() {
   return sizeof(float) * (3 * kC * (DK + 4) + 768 + 2 * DK);
 }
-template <int DK>
+template <int DK, int DVS>
 constexpr size_t state_smem() {
-  return sizeof(float) * (DK * kLDS + 2 * kC * (DK + 4) + kC * kLDC + kC * kLDS + 2 * DK);
+  return sizeof(float) * (DK * (DVS + 2) + 2 * kC * (DK + 4) + kC * kLDC + kC * (DVS + 2) + 2 * DK);
 }
-template <int DK>
+template <int DK, int DVS>
 constexpr size_t dstate_smem() {
-  return sizeof(float) * (DK * kLDS + 3 * kC * (DK + 4) + 2 * kC * kLDC + 2 * kC * kLDS + 2 * DK);
+  return sizeof(float) * (DK * (DVS + 2) + 3 * kC * (DK + 4) + 2 * kC * kLDC + 2 * kC * (DVS + 2) + 2 * DK);
 }
 template <int DV>
 constexpr size_t local_smem() {
@@ -796,13 +796,18 @@ cudaError_t launch(K kernel, unsigned grid, size_t smem, cudaStream_t s, const B
 
 template <int DK, int DV>
 cudaError_t launch_dims(const BwdArgs& p, cudaStream_t s) {
-  static_assert(local_smem<DV>() <= 227 * 1024 && dstate_smem<DK>() <= 227 * 1024, "shared memory");
+  constexpr int S1 = kDVS_STATE, S2 = kDVS_DSTATE < DV ? kDVS_DSTATE : DV;
+  static_assert(DV % S1 == 0 && DV % S2 == 0, "d_v slices");
+  static_assert(local_smem<DV>() <= 227 * 1024 && dstate_smem<DK, S2>() <= 227 * 1024, "shared memory");
   const int64_t bh = (int64_t)p.f.B * p.f.H;
-  const unsigned chunks = (unsigned)(bh * p.nc), chains = (unsigned)(bh * (DV / kDVS));
+  const unsigned chunks = (unsigned)(bh * p.nc);
   cudaError_t e;
   if ((e = launch(bwd_prep_kernel<DK>, chunks, prep_smem<DK>(), s, p)) != cudaSuccess) return e;
-  if ((e = launch(bwd_state_kernel<DK, DV>, chains, state_smem<DK>(), s, p)) != cudaSuccess) return e;
-  if ((e = launch(bwd_dstate_kernel<DK, DV>, chains, dstate_smem<DK>(), s, p)) != cudaSuccess) return e;
+  if ((e = launch(bwd_state_kernel<DK, DV, S1>, (unsigned)(bh * (DV / S1)), state_smem<DK, S1>(), s, p)) != cudaSuccess)
+    return e;
+  if ((e = launch(bwd_dstate_kernel<DK, DV, S2>, (unsigned)(bh * (DV / S2)), dstate_smem<DK, S2>(), s, p)) !=
+      cudaSuccess)
+    return e;
   return launch(bwd_local_kernel<DK, DV>, chunks, local_smem<DV>(), s, p);
 }
 
