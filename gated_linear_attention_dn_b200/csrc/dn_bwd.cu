@@ -84,18 +84,26 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, i
       split_tf32(A(16 * mi + g, k0 + t + 4), ah[mi][2], al[mi][2]);
       split_tf32(A(16 * mi + g + 8, k0 + t + 4), ah[mi][3], al[mi][3]);
     }
+    uint32_t bh[NI][2], bl[NI][2];
 #pragma unroll
     for (int ni = 0; ni < NI; ++ni) {
-      uint32_t bh[2], bl[2];
-      split_tf32(B(k0 + t, 8 * ni + g), bh[0], bl[0]);
-      split_tf32(B(k0 + t + 4, 8 * ni + g), bh[1], bl[1]);
-#pragma unroll
-      for (int mi = 0; mi < MI; ++mi) {
-        ut::mma_tf32(acc[mi][ni], al[mi], bh);
-        ut::mma_tf32(acc[mi][ni], ah[mi], bl);
-        ut::mma_tf32(acc[mi][ni], ah[mi], bh);
-      }
+      split_tf32(B(k0 + t, 8 * ni + g), bh[ni][0], bl[ni][0]);
+      split_tf32(B(k0 + t + 4, 8 * ni + g), bh[ni][1], bl[ni][1]);
     }
+    // the three products of a fragment go to the same accumulator; issuing each round over all
+    // fragments keeps MI * NI independent products in flight instead of one dependent chain
+#pragma unroll
+    for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[mi][ni], al[mi], bh[ni]);
+#pragma unroll
+    for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[mi][ni], ah[mi], bl[ni]);
+#pragma unroll
+    for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[mi][ni], ah[mi], bh[ni]);
   }
 }
 
