@@ -210,9 +210,9 @@ def dn_chunk_bwd_workspace_bytes(desc: DnDesc) -> int:
 
 
 def dn_chunk_bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, dO=None, dS_T=None,
-                 workspace=None, want_dS0: bool = True, out=None, stream=None):
-    """Chunked backward of dn_chunk_fwd (post-update read-out): the gradients of
-    sum <dO, o> + <dS_T, S_T>. dO [B,T,H,d_v] in the io dtype; dS_T [B,H,d_k,d_v] fp32 or None (zero).
+                 workspace=None, want_dS0: bool = True, out=None, stream=None, readout: str = "post"):
+    """Backward of dn_chunk_fwd with the same read-out: the gradients of sum <dO, o> + <dS_T, S_T>.
+    dO [B,T,H,d_v] in the io dtype; dS_T [B,H,d_k,d_v] fp32 or None (zero).
 
     Returns {"q", "k", "v"} (io dtype, shaped like the inputs), {"alpha", "beta_k", "beta_v",
     "key_scale"} (fp32, shaped like each gate; None for an absent gate) and "S0" (fp32
@@ -222,7 +222,7 @@ def dn_chunk_bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, 
     """
     lib = load()
     _check_io(q, k, v)
-    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, 0, "post")
+    desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, 0, readout)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     if dO is None or not dO.is_contiguous() or dO.dtype != q.dtype or tuple(dO.shape) != (B, T, H, dv):

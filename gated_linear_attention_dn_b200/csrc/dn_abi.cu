@@ -271,12 +271,14 @@ dn_status dn_mc_readout(const dn_mc_desc* d, const void* q, const float* M, cons
 
 namespace {
 
-// The backward covers the tensor-core sizes with the post-update read-out.
+bool small_dims(const dn_desc* d) { return (d->d_k == 8 || d->d_k == 16) && (d->d_v == 8 || d->d_v == 16); }
+
+// The backward covers the tensor-core sizes (chunked kernels) and the small states (sequential
+// kernel), either read-out.
 dn_status check_bwd_desc(const dn_desc* d) {
   dn_status st = check_desc(d, false);
   if (st != DN_OK) return st;
-  if (d->readout != DN_READ_POST) return DN_ERR_UNSUPPORTED;
-  if (!((d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128))) return DN_ERR_UNSUPPORTED;
+  if (small_dims(d)) return DN_OK;
   const int64_t blocks = (int64_t)d->B * d->H * ((d->T + 63) / 64);
   if (blocks >= ((int64_t)1 << 31)) return DN_ERR_UNSUPPORTED;
   return DN_OK;
@@ -295,6 +297,7 @@ extern "C" {
 
 size_t dn_chunk_bwd_workspace_bytes(const dn_desc* desc) {
   if (check_bwd_desc(desc) != DN_OK) return 0;
+  if (small_dims(desc)) return dn::small_bwd_workspace_bytes(desc->B, desc->T, desc->H, desc->d_k, desc->d_v);
   return dn::chunk_bwd_workspace_bytes(desc->B, desc->T, desc->H, desc->d_k, desc->d_v);
 }
 
@@ -322,7 +325,7 @@ dn_status dn_chunk_bwd(const dn_desc* desc, const void* q, const void* k, const 
   if ((st = check_grad_ptr(desc->beta_k, d_beta_k)) != DN_OK) return st;
   if ((st = check_grad_ptr(desc->beta_v, d_beta_v)) != DN_OK) return st;
   if ((st = check_grad_ptr(desc->key_scale, d_key_scale)) != DN_OK) return st;
-  const size_t need = dn::chunk_bwd_workspace_bytes(desc->B, desc->T, desc->H, desc->d_k, desc->d_v);
+  const size_t need = dn_chunk_bwd_workspace_bytes(desc);
   if (!workspace || workspace_bytes < need) return DN_ERR_WORKSPACE_TOO_SMALL;
   if (!aligned16(workspace)) return DN_ERR_MISALIGNED;
   {  // the gradients of q, k, v are written while every input, dO and the workspace are still read
@@ -341,8 +344,12 @@ dn_status dn_chunk_bwd(const dn_desc* desc, const void* q, const void* k, const 
     }
   }
   a.S0 = S0;
-  cudaError_t e = dn::launch_chunk_bwd(a, dO, dS_T, dq, dk, dv, d_alpha, d_beta_k, d_beta_v, d_key_scale, dS0,
-                                       static_cast<float*>(workspace), s);
+  cudaError_t e =
+      small_dims(desc)
+          ? dn::launch_small_bwd(a, dO, dS_T, dq, dk, dv, d_alpha, d_beta_k, d_beta_v, d_key_scale, dS0,
+                                 static_cast<float*>(workspace), s)
+          : dn::launch_chunk_bwd(a, dO, dS_T, dq, dk, dv, d_alpha, d_beta_k, d_beta_v, d_key_scale, dS0,
+                                 static_cast<float*>(workspace), s);
   return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
 

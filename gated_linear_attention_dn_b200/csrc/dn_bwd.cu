@@ -1,4 +1,4 @@
-// Chunked backward (training pass) of the recurrence with the post-update read-out: the gradients
+// Chunked backward (training pass) of the recurrence, either read-out: the gradients
 // of sum <dO, o> + <dS_T, S_T> with respect to q, k, v, every gate and S0. The pages name
 // chunk-parallel training (FG2-GDN page, section 3 item 2) but print no backward; the equations
 // below are the chain rule through the chunk form of the forward.
@@ -15,6 +15,8 @@
 //   dh_t = Q+ dQ+ + K+ dK+ - W- dW- (per channel), plus rowsum(dX (.) X) at the last token;
 //   d log alpha_s = sum_{t >= s in the chunk} dh_t; then the products back to q, k, w, gates.
 // (The outputs do not depend on r, so its own adjoint terms cancel and r is held fixed.)
+// Pre-update read-out (o_t = S_{t-1}^T q_t): Q+_t = q_t e^{h_t} / alpha_t and P is strictly lower, so
+// dP is strictly lower, dq = e^h / alpha dQ+, and d log alpha_t also gets -Q+_t dQ+_t (not cumulated).
 //
 // Four kernels, all fp32 with the dense per-chunk products on warp tensor cores (mma.sync TF32 with
 // a three-product hi/lo split, so each product keeps about fp32 accuracy):
@@ -175,7 +177,10 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
       if (t < n) {
         const int64_t tok = token(a, b, h, t0 + t);
         kk[u] = io_load(a.k, tok * a.dk + i0 + i, a.io_bf16);
-        if (Qp) qq[u] = io_load(a.q, tok * a.dk + i0 + i, a.io_bf16);
+        if (Qp) {
+          qq[u] = io_load(a.q, tok * a.dk + i0 + i, a.io_bf16);
+          if (a.pre_read) qq[u] /= gate_load(a.alpha_p, a.alpha, tok, a.dk, i0 + i);  // read before the decay
+        }
         ws[u] = gate_load(a.beta_k_p, a.beta_k, tok, a.dk, i0 + i) * gate_load(a.key_scale_p, a.key_scale, tok, a.dk, i0 + i);
       }
     }
@@ -269,7 +274,8 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
   const int64_t cb = (int64_t)bh * p.nc + c;
   prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, p.wEh + cb * kC * DK, tid);
 
-  // warps 0-3: L = strictly-lower(K+ W-^T) (kept in registers); warps 4-7: P = lower-incl(Q+ W-^T)
+  // warps 0-3: L = strictly-lower(K+ W-^T) (kept in registers); warps 4-7: P = lower(Q+ W-^T), with the
+  // diagonal for the post read-out and without it for the pre read-out
   const int m0 = ((warp & 3) >> 1) * 32, n0 = (warp & 1) * 32;
   float acc[2][4][4] = {};
   {
@@ -280,7 +286,9 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
   }
   if (warp >= 4) {
     float* P = p.wP + cb * kC * kC;
-    warp_epilogue(acc, [&](int m, int nn, float v) { P[(m0 + m) * kC + n0 + nn] = n0 + nn <= m0 + m ? v : 0.f; }, lane);
+    const int diag = a.pre_read ? 0 : 1;  // the pre read-out excludes the token's own write
+    warp_epilogue(acc, [&](int m, int nn, float v) { P[(m0 + m) * kC + n0 + nn] = n0 + nn < m0 + m + diag ? v : 0.f; },
+                  lane);
   }
   if (tid < DK) {
     p.wEr[cb * DK + tid] = er[tid];
@@ -533,7 +541,8 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   float* Qp = Eh + kC * LDS;    // then the beta^k gradient terms
   float* Kp = Qp + kC * LDS;    // then the d gradient terms
   float* Wm = Kp + kC * LDS;    // then dh, then d log alpha
-  float* red = Wm + kC * LDS;   // [4][kDKS]
+  float* Xq = Wm + kC * LDS;    // Q+ (.) dQ+, the pre read-out's own-token decay term
+  float* red = Xq + kC * LDS;   // [4][kDKS]
   float* acc_a = red + 4 * kDKS;  // [C] per-token sums for gates of width 1
   float* acc_bk = acc_a + kC;
   float* acc_d = acc_bk + kC;
@@ -615,8 +624,10 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
     warp_gemm<2, 4, DV>(
         acc, [&](int m, int k) { return X[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return U[(n0 + nn) * LDV + k]; },
         lane);
+    const int diag = a.pre_read ? 0 : 1;
     if (warp < 4)
-      warp_epilogue(acc, [&](int m, int nn, float v) { dP[(m0 + m) * kLDC + n0 + nn] = n0 + nn <= m0 + m ? v : 0.f; }, lane);
+      warp_epilogue(acc, [&](int m, int nn, float v) { dP[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m + diag ? v : 0.f; },
+                    lane);
     else
       warp_epilogue(acc, [&](int m, int nn, float v) { dL[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? -v : 0.f; }, lane);
   }
@@ -688,7 +699,7 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
     {
       // Per (token, channel) of this warp's tiles: dq, dk, the beta^k and d gradients, and dh. Each
       // thread then reads and writes only its own elements of hb, Qp, Kp, Wm.
-      float gq[2][4], gk[2][4], lk[2][4], lb[2][4], ld[2][4];
+      float gq[2][4], gk[2][4], lk[2][4], lb[2][4], ld[2][4], la[2][4];
       const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
       for (int ni = 0; ni < 2; ++ni)
@@ -696,12 +707,13 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
         for (int q = 0; q < 4; ++q) {  // the inputs of this thread's elements, loaded up front
           const int t = m0 + g + (q >> 1) * 8, gi = i0 + n0 + 8 * ni + 2 * t4 + (q & 1);
           lk[ni][q] = 0.f;
-          lb[ni][q] = ld[ni][q] = 1.f;
+          lb[ni][q] = ld[ni][q] = la[ni][q] = 1.f;
           if (t < n) {
             const int64_t tok = token(a, b, h, t0 + t);
             lk[ni][q] = io_load(a.k, tok * DK + gi, a.io_bf16);
             lb[ni][q] = gate_load(a.beta_k_p, a.beta_k, tok, DK, gi);
             ld[ni][q] = gate_load(a.key_scale_p, a.key_scale, tok, DK, gi);
+            if (a.pre_read) la[ni][q] = gate_load(a.alpha_p, a.alpha, tok, DK, gi);
           }
         }
       auto elem = [&](int ni, int q, int m, int nn, float vq, float vk, float vw) {
@@ -711,9 +723,11 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
         const float kk = lk[ni][q], bk = lb[ni][q], dd = ld[ni][q];
         const float dk = vk * eh + bk * dd * dw;
         const float gbk = dd * kk * dw, gdd = bk * kk * dw;
-        gq[ni][q] = vq * eh;
+        gq[ni][q] = vq * eh / la[ni][q];
         gk[ni][q] = dk;
-        const float dh = Qp[t * LDS + il] * vq + Kp[t * LDS + il] * vk - Wm[t * LDS + il] * vw;
+        const float xq = Qp[t * LDS + il] * vq;
+        Xq[t * LDS + il] = xq;
+        const float dh = xq + Kp[t * LDS + il] * vk - Wm[t * LDS + il] * vw;
         Qp[t * LDS + il] = gbk;
         Kp[t * LDS + il] = gdd;
         Wm[t * LDS + il] = dh;
@@ -745,11 +759,12 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
       float run = red[il] + red[kDKS + il] + red[2 * kDKS + il] + red[3 * kDKS + il];
       for (int t = kC - 1; t >= 0; --t) {
         run += Wm[t * LDS + il];
+        const float dlog = a.pre_read ? run - Xq[t * LDS + il] : run;
         if (t < n && a.alpha == DN_GATE_CHANNEL) {
           const int64_t tok = token(a, b, h, t0 + t);
-          p.galpha[tok * DK + i0 + il] = run / gate_load(a.alpha_p, a.alpha, tok, DK, i0 + il);
+          p.galpha[tok * DK + i0 + il] = dlog / gate_load(a.alpha_p, a.alpha, tok, DK, i0 + il);
         }
-        Wm[t * LDS + il] = run;
+        Wm[t * LDS + il] = dlog;
       }
     }
     __syncthreads();
@@ -790,7 +805,7 @@ constexpr size_t dstate_smem() {
 }
 template <int DV>
 constexpr size_t local_smem() {
-  return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 4 * kC * (kDKS + 4) + 4 * kDKS +
+  return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 5 * kC * (kDKS + 4) + 4 * kDKS +
                           3 * kC);
 }
 

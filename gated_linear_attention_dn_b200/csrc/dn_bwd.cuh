@@ -15,4 +15,11 @@ cudaError_t launch_chunk_bwd(const Args& f, const void* dO, const float* dS_T, v
                              float* galpha, float* gbeta_k, float* gbeta_v, float* gkey_scale, float* gS0, float* ws,
                              cudaStream_t s);
 
+// Small states (d_k, d_v in {8, 16}; dn_small_bwd.cu), either read-out: the state entering every
+// token is kept in the workspace (B * H * T * d_k * d_v fp32).
+size_t small_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_small_bwd(const Args& a, const void* dO, const float* dS_T, void* gq, void* gk, void* gv,
+                             float* galpha, float* gbeta_k, float* gbeta_v, float* gkey_scale, float* gS0, float* ws,
+                             cudaStream_t s);
+
 }  // namespace dn

@@ -243,12 +243,14 @@ dn_status dn_mc_readout(const dn_mc_desc* desc, const void* q, const float* M, c
  *      per-token gate, [B,T,H,n] per channel), given exactly when the gate is
  *      (NULL when it is DN_GATE_ONE); dS0 [B,H,d_k,d_v] fp32 or NULL (not wanted).
  * Scratch: `workspace` of at least dn_chunk_bwd_workspace_bytes() bytes, 16-byte
- * aligned, owned by the caller; its contents on entry do not matter. Per (b, h) and
- * chunk of 64 tokens it holds, fp32: the UT transform and score matrix (64 x 64 each), the
+ * aligned, owned by the caller; its contents on entry do not matter. Small states: the
+ * state entering every token (B * H * T * d_k * d_v fp32). Otherwise, per (b, h) and
+ * chunk of 64 tokens, fp32: the UT transform and score matrix (64 x 64 each), the
  * decay-scaled keys, queries and write keys and their decay factors (64 x d_k each), the
  * state and its adjoint (d_k x d_v each), and the residuals and their adjoints (64 x d_v each).
- * Supported: the post-update read-out (DN_READ_PRE returns DN_ERR_UNSUPPORTED),
- * d_k, d_v in {64, 128}, alpha > 0. dq, dk, dv must not overlap each other, q, k, v,
+ * Supported: both read-outs (desc->readout as given to the forward); d_k, d_v in {64, 128}
+ * (chunked kernels) or both in {8, 16} (small states: one warp per head, sequential, the state
+ * entering every token kept in the workspace); alpha > 0. dq, dk, dv must not overlap each other, q, k, v,
  * dO, S0 or the workspace. fp32 arithmetic throughout. T == 0 writes dS0 = dS_T (or
  * zeros). Asynchronous on the stream.
  */

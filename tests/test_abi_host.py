@@ -191,13 +191,14 @@ def test_bwd_workspace_bytes(lib):
     # per chunk: T, P (64 x 64); S_m, dX (d_k x d_v); U, dV~ (64 x d_v); K+, Q+, W-, e^h (64 x d_k); e^r, lam (d_k)
     per = 2 * 64 * 64 + 2 * 128 * 64 + 2 * 64 * 64 + 4 * 64 * 128 + 2 * 128
     assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(d)) == 2 * 3 * nc * per * 4
-    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(d_k=8, d_v=8))) == 0   # small states: no backward
-    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(readout=dn.DN_READ_PRE))) == 0
+    # small states keep the state entering every token: B * H * T * d_k * d_v floats
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(d_k=8, d_v=16))) == 1 * 2 * 8 * 8 * 16 * 4
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(d_k=16, d_v=8, readout=dn.DN_READ_PRE))) == 2 * 8 * 128 * 4
 
 
 def test_bwd_rejects_bad_arguments(lib):
-    assert _bwd_call(lib, _desc(readout=dn.DN_READ_PRE), ws_bytes=1 << 20) == dn.DN_ERR_UNSUPPORTED
-    assert _bwd_call(lib, _desc(d_k=16, d_v=16), ws_bytes=1 << 20) == dn.DN_ERR_UNSUPPORTED
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(readout=dn.DN_READ_PRE))) > 0  # both read-outs
+    assert _bwd_call(lib, _desc(d_k=16, d_v=64), ws_bytes=1 << 20) == dn.DN_ERR_UNSUPPORTED  # mixed small and big
     assert _bwd_call(lib, _desc(B=0)) == dn.DN_ERR_INVALID_ARGUMENT
     assert _bwd_call(lib, _desc(), dO=None) == dn.DN_ERR_INVALID_ARGUMENT
     assert _bwd_call(lib, _desc(), gq=None) == dn.DN_ERR_INVALID_ARGUMENT

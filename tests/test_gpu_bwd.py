@@ -1,5 +1,6 @@
-"""GPU parity of the chunked backward (dn_chunk_bwd, through the C ABI) against the fp64 oracle's
-reverse mode (oracle.bwd), element by element over every gradient.
+"""GPU parity of the backward (dn_chunk_bwd, through the C ABI: the chunked kernels for d in {64, 128},
+the sequential small-state kernel for d in {8, 16}, both read-outs) against the fp64 oracle's reverse
+mode (oracle.bwd), element by element over every gradient.
 
 Tolerances (rel-L2 over the whole tensor): the kernels compute in fp32 throughout (their dense
 products are TF32 tensor-core products with a hi/lo split, about fp32 accuracy), and the same
@@ -24,11 +25,11 @@ TOL_IO = {"f32": 1e-4, "bf16": 1e-2}
 NAMES = ("q", "k", "v", "alpha", "beta_k", "beta_v", "key_scale", "S0")
 
 
-def _run(x, g):
+def _run(x, g, readout="post"):
     xd = to_device(x)
     gd = to_device(g)
     out = dn.dn_chunk_bwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
-                          xd["S0"], dO=gd["dO"], dS_T=gd["dS_T"])
+                          xd["S0"], dO=gd["dO"], dS_T=gd["dS_T"], readout=readout)
     assert dn.dn_stream_status() == dn.DN_OK
     return out
 
@@ -69,6 +70,37 @@ def test_bwd_matches_oracle(name, kw):
     g = di.make_bwd_inputs(w)
     out = _run(x, g)
     ref = oracle.bwd(**x, dO=g["dO"], dS_T=g["dS_T"])
+    _compare(out, ref, w.io)
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("gdn_prefill", dict(B=1, H=2, T=200)),              # bf16 scalar gates, ragged tail
+    ("kda", dict(B=1, H=2, T=130)),                      # channel decay, S0
+    ("fg2_osdn_long", dict(B=1, H=2, T=150)),            # every gate per channel
+    ("gdn_fp32_small", dict(dv=128)),                    # fp32, d_k 64, d_v 128
+])
+def test_bwd_pre_readout_matches_oracle(name, kw):
+    """o_t = S_{t-1}^T q_t (the delta-mem page's read): the same four kernels with Q+ / alpha and a strict P."""
+    w = di.WORKLOADS[name].scaled(**kw)
+    x = di.make_inputs(w)
+    g = di.make_bwd_inputs(w)
+    out = _run(x, g, readout="pre")
+    ref = oracle.bwd(**x, dO=g["dO"], dS_T=g["dS_T"], readout="pre")
+    _compare(out, ref, w.io)
+
+
+@pytest.mark.parametrize("readout", ["post", "pre"])
+@pytest.mark.parametrize("name,kw", [
+    ("gdn_fp32_small", dict(B=2, H=3, T=300, dk=8, dv=8)),         # the delta-mem page's 8 x 8 memory
+    ("fg2_osdn_long", dict(B=1, H=2, T=130, dk=16, dv=8)),        # every gate per channel, bf16
+    ("kda", dict(B=1, H=5, T=77, dk=16, dv=16)),                  # channel decay, S0
+])
+def test_bwd_small_states_match_oracle(name, kw, readout):
+    w = di.WORKLOADS[name].scaled(**kw)
+    x = di.make_inputs(w)
+    g = di.make_bwd_inputs(w)
+    out = _run(x, g, readout=readout)
+    ref = oracle.bwd(**x, dO=g["dO"], dS_T=g["dS_T"], readout=readout)
     _compare(out, ref, w.io)
 
 
