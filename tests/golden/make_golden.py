@@ -1,4 +1,5 @@
-"""Write tests/golden/oracle_tiny.json from the fp64 oracle (and the seeded inputs) only.
+"""Write tests/golden/oracle_tiny.json and oracle_bwd_tiny.json from the fp64 oracle (and the seeded
+inputs) only.
 
 The pages print no worked numeric example for this recurrence, so this fixture is
 a regression anchor of the oracle itself, not a value from the pages: it pins the
@@ -35,3 +36,17 @@ out = {
 with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "oracle_tiny.json"), "w") as f:
     json.dump(out, f, indent=1)
 print("wrote oracle_tiny.json")
+
+# the reverse mode on the same inputs, with the seeded cotangents of the same recipe
+gb = di.make_bwd_inputs(w)
+g = oracle.bwd(**x, dO=gb["dO"], dS_T=gb["dS_T"])
+out = {
+    "what": "fp64 oracle reverse mode on the seeded fg2_osdn_long recipe at tiny sizes (regression anchor)",
+    "workload": WORKLOAD,
+    "sizes": SIZES,
+    "grad_head": {n: [float(v) for v in a.ravel()[:8]] for n, a in g.items() if a is not None},
+    "grad_norm": {n: float(np.linalg.norm(a)) for n, a in g.items() if a is not None},
+}
+with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "oracle_bwd_tiny.json"), "w") as f:
+    json.dump(out, f, indent=1)
+print("wrote oracle_bwd_tiny.json")

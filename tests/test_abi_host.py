@@ -216,3 +216,21 @@ def test_bwd_rejects_bad_arguments(lib):
     assert _bwd_call(lib, _desc(), q=shared.p(), gq=shared.p(256)) == dn.DN_ERR_INVALID_ARGUMENT
     # no tokens and no dS0 wanted: nothing to do
     assert _bwd_call(lib, _desc(T=0), gs0=None) == dn.DN_OK
+
+
+def test_binding_bwd_checks_arguments_before_the_library(lib):
+    """dn_chunk_bwd's argument checks raise before any call into libdn.so (CPU tensors are enough)."""
+    import torch
+    q = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    v = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    a = torch.ones(1, 8, 2)
+    with pytest.raises(ValueError, match="dO"):
+        dn.dn_chunk_bwd(q, q, v, a, a, dO=None)
+    with pytest.raises(ValueError, match="dO"):
+        dn.dn_chunk_bwd(q, q, v, a, a, dO=torch.zeros(1, 8, 2, 64))  # fp32 dO for bf16 inputs
+    with pytest.raises(ValueError, match="dS_T"):
+        dn.dn_chunk_bwd(q, q, v, a, a, dO=v, dS_T=torch.zeros(1, 2, 64, 32))
+    with pytest.raises(ValueError, match="out"):
+        dn.dn_chunk_bwd(q, q, v, a, a, dO=v, out={"q": q, "k": q, "v": v, "alpha": None, "beta_k": a})
+    with pytest.raises(TypeError):
+        dn.dn_chunk_bwd(q, q.float(), v, a, a, dO=v)

@@ -175,6 +175,22 @@ def test_b4_chunked_reverse_matches(T, C, gates):
         np.testing.assert_allclose(gc[name], g[name], rtol=1e-9, atol=1e-11, err_msg=name)
 
 
+def test_golden_fixture_regression():
+    """The committed fixture was written by tests/golden/make_golden.py (oracle and seeded inputs only)."""
+    import json
+    import dn_inputs as di
+    with open(os.path.join(os.path.dirname(__file__), "golden", "oracle_bwd_tiny.json")) as f:
+        gold = json.load(f)
+    w = di.WORKLOADS[gold["workload"]].scaled(**gold["sizes"])
+    x = di.make_inputs(w)
+    gb = di.make_bwd_inputs(w)
+    g = oracle.bwd(**x, dO=gb["dO"], dS_T=gb["dS_T"])
+    assert sorted(gold["grad_norm"]) == sorted(n for n, a in g.items() if a is not None)
+    for n, head in gold["grad_head"].items():
+        np.testing.assert_allclose(g[n].ravel()[: len(head)], head, rtol=1e-12, atol=1e-15, err_msg=n)
+        np.testing.assert_allclose(np.linalg.norm(g[n]), gold["grad_norm"][n], rtol=1e-12, err_msg=n)
+
+
 SRC = os.path.join(os.path.dirname(oracle.__file__), "dn_oracle.c")
 MUTATIONS = {
     "erase_adjoint_dropped": ("const double dsb = dS[(int64_t)i * dv + j] - kt[i] * du[j];",
