@@ -242,6 +242,9 @@ def dn_chunk_bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, 
             if (t is None) != (ref is None) or (t is not None and (t.shape != ref.shape or t.dtype != ref.dtype
                                                                    or not t.is_contiguous())):
                 raise ValueError(f"out[{name!r}] does not match {name}")
+        t = out.get("S0")
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous() or tuple(t.shape) != (B, H, dk, dv)):
+            raise ValueError("out['S0'] must be a contiguous float32 [B,H,d_k,d_v] tensor or None")
     ws_bytes = dn_chunk_bwd_workspace_bytes(desc)
     if workspace is None and ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
