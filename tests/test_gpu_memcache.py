@@ -60,3 +60,23 @@ def test_readout_alone_fp32():
     err = oracle.rel_l2(host_f64(o), ref)
     print(f"[parity] mc read-out rel-L2 {err:.3e}")
     assert err <= 1e-5
+
+
+def test_mc_full_size_sampled_batches():
+    """The configuration the benchmark times (GDN prefill B=8, H=16, T=4096, four segments of 1024,
+    residual memory): the whole batch on the GPU; the first and last batch rows (all heads, the
+    whole sequence) against the oracle. Batch rows are independent, so the oracle runs only those."""
+    w = di.WORKLOADS["gdn_prefill"]
+    x = di.make_inputs(w)
+    xd = to_device(x)
+    o, M = dn.mc_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"], xd["S0"],
+                     seg_len=1024)
+    assert dn.dn_stream_status() == dn.DN_OK
+    sel = [0, w.B - 1]
+    xs = {n: (None if a is None else np.ascontiguousarray(a[sel])) for n, a in x.items()}
+    o_ref, M_ref = oracle.memcache.mc_fwd(**xs, seg_len=1024)
+    tol = TOL[w.io]
+    eo = oracle.rel_l2(host_f64(o)[sel], o_ref)
+    eM = oracle.rel_l2(host_f64(M)[sel], M_ref)
+    print(f"[parity] mc full size o rel-L2 {eo:.3e} (tol {tol['o']:.0e}), M rel-L2 {eM:.3e} (tol {tol['S']:.0e})")
+    assert eo <= tol["o"] and eM <= tol["S"]
