@@ -32,7 +32,8 @@
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
  *     allocates no device memory and keeps no per-call state. The only global
- *     state is one device status word per GPU (see dn_stream_status).
+ *     state is one device status word per GPU (see dn_stream_status) and the
+ *     static scratch buffer of dn_osdn_precond_noalloc.
  *   - Row-major layouts, innermost dimension last:
  *       q, k      [B, T, H, d_k]        io dtype
  *       v, o      [B, T, H, d_v]        io dtype
