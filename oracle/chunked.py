@@ -97,8 +97,8 @@ def fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, 
     return o, ST
 
 
-def head_bwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, dO, dS_T, C: int):
-    """Reverse mode of ``head_fwd`` (post read-out) in the same chunk algebra.
+def head_bwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, dO, dS_T, C: int, readout: str = "post"):
+    """Reverse mode of the chunk algebra, either read-out.
 
     The chain rule through the chunk equations gives, with dS' the adjoint of the chunk-end state
     and lam = e(g_n - g_m):
@@ -112,6 +112,9 @@ def head_bwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, dO, dS_T, C: int):
     depend on the reference point g_m, so its adjoint terms cancel and g_m is held fixed: the
     log-decay adjoint of token t is dh_t = Q+ (.) dQ+ + K+ (.) dK+ - W- (.) dW- (every channel), plus
     rowsum(dX (.) X) at the chunk's last token, and d log alpha_s is the sum over t >= s in the chunk.
+    The pre read-out o_t = S_{t-1}^T q_t reads the state before token t's decay: Q+_t = q_t (.) e(h_t)
+    / alpha_t and P = strictly-lower(Q+ W-^T), so dP is strictly lower, dq = e(h) / alpha (.) dQ+, and
+    d log alpha_t also gets -Q+_t (.) dQ+_t, token t's own term (not summed over later tokens).
 
     Returns a dict of per-token gradients shaped [T, n] for every gate (channel form) and
     dS0 [dk, dv].
@@ -130,27 +133,29 @@ def head_bwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, dO, dS_T, C: int):
         eh = np.exp(g - r)
         bkd = _gate(beta_k, c0, c1, dk) * _gate(key_scale, c0, c1, dk)
         w = bkd * k[c0:c1]
-        Kp, Qp, Wm = k[c0:c1] * eh, q[c0:c1] * eh, w / eh
+        eq = eh / a if readout == "pre" else eh   # the pre read-out stops the decay one token earlier
+        Kp, Qp, Wm = k[c0:c1] * eh, q[c0:c1] * eq, w / eh
         Vt = _gate(beta_v, c0, c1, dv) * v[c0:c1]
         Sm = np.exp(r)[:, None] * S
         Tm = np.linalg.inv(np.eye(n) + np.tril(Kp @ Wm.T, k=-1))
         U = Tm @ (Vt - Kp @ Sm)
         X = Sm + Wm.T @ U
         lam = np.exp(g[-1] - r)
-        keep.append((c0, c1, a, eh, bkd, Kp, Qp, Wm, Tm, U, Sm, X, lam, r))
+        keep.append((c0, c1, a, eh, eq, bkd, Kp, Qp, Wm, Tm, U, Sm, X, lam, r))
         S = lam[:, None] * X
     out = {n: np.zeros((T, w)) for n, w in (("q", dk), ("k", dk), ("v", dv), ("alpha", dk),
                                                ("beta_k", dk), ("beta_v", dv), ("key_scale", dk))}
     dS = np.zeros((dk, dv)) if dS_T is None else np.array(dS_T, dtype=np.float64)
     for c in reversed(range(nc)):
-        c0, c1, a, eh, bkd, Kp, Qp, Wm, Tm, U, Sm, X, lam, r = keep[c]
+        c0, c1, a, eh, eq, bkd, Kp, Qp, Wm, Tm, U, Sm, X, lam, r = keep[c]
         dOc = dO[c0:c1]
         dX = lam[:, None] * dS
-        P = np.tril(Qp @ Wm.T)
+        diag = -1 if readout == "pre" else 0
+        P = np.tril(Qp @ Wm.T, k=diag)
         dU = P.T @ dOc + Wm @ dX
         dVt = Tm.T @ dU
         dS = np.exp(r)[:, None] * (Qp.T @ dOc + dX - Kp.T @ dVt)
-        dP = np.tril(dOc @ U.T)
+        dP = np.tril(dOc @ U.T, k=diag)
         dL = -np.tril(dVt @ U.T, k=-1)
         dQp = dOc @ Sm.T + dP @ Wm
         dKp = -dVt @ Sm.T + dL @ Wm
@@ -158,9 +163,11 @@ def head_bwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, dO, dS_T, C: int):
         dh = Qp * dQp + Kp * dKp - Wm * dWm
         dh[-1] += np.sum(dX * X, axis=1)
         dlog = np.cumsum(dh[::-1], axis=0)[::-1]
+        if readout == "pre":
+            dlog = dlog - Qp * dQp
         dw = dWm / eh
         kc, vc = k[c0:c1], v[c0:c1]
-        out["q"][c0:c1] = dQp * eh
+        out["q"][c0:c1] = dQp * eq
         out["k"][c0:c1] = dKp * eh + bkd * dw
         out["alpha"][c0:c1] = dlog / a
         out["beta_k"][c0:c1] = _gate(key_scale, c0, c1, dk) * kc * dw
@@ -172,8 +179,8 @@ def head_bwd(q, k, v, alpha, beta_k, beta_v, key_scale, S, dO, dS_T, C: int):
 
 
 def bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, dO=None, dS_T=None,
-        C: int = 64):
-    """All heads, public layouts, post read-out: the gradients as ``oracle.bwd`` returns them."""
+        C: int = 64, readout: str = "post"):
+    """All heads, public layouts: the gradients as ``oracle.bwd`` returns them."""
     q = np.asarray(q, dtype=np.float64)
     B, T, H, dk = q.shape
     dv = np.asarray(v).shape[-1]
@@ -195,7 +202,7 @@ def bwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, S0=None, 
             g = head_bwd(q[b, :, h], np.asarray(k, dtype=np.float64)[b, :, h],
                          np.asarray(v, dtype=np.float64)[b, :, h], *(sl(gates[n], b, h) for n in gates), S,
                          np.asarray(dO, dtype=np.float64)[b, :, h],
-                         None if dS_T is None else np.asarray(dS_T, dtype=np.float64)[b, h], C)
+                         None if dS_T is None else np.asarray(dS_T, dtype=np.float64)[b, h], C, readout)
             for n in ("q", "k", "v"):
                 res[n][b, :, h] = g[n]
             res["S0"][b, h] = g["S0"]

@@ -161,13 +161,14 @@ def test_b3_no_writes_closed_form(mode, readout):
     np.testing.assert_allclose(got, da.sum(axis=1) if got.ndim == 1 else da, rtol=1e-11, atol=1e-14)
 
 
-# B4 -- the chunked reverse mode (post read-out) against the sequential one
+# B4 -- the chunked reverse mode against the sequential one, both read-outs
+@pytest.mark.parametrize("readout", ["post", "pre"])
 @pytest.mark.parametrize("T,C", [(1, 4), (5, 4), (64, 16), (65, 16), (130, 64), (37, 8)])
 @pytest.mark.parametrize("gates", ["channel", "scalar", "none"])
-def test_b4_chunked_reverse_matches(T, C, gates):
+def test_b4_chunked_reverse_matches(T, C, gates, readout):
     x, dO, dS_T = _case(T=T, H=2, dk=6, dv=5, seed=T + C, gates=gates)
-    g = oracle.bwd(**x, dO=dO, dS_T=dS_T)
-    gc = chunked.bwd(**x, dO=dO, dS_T=dS_T, C=C)
+    g = oracle.bwd(**x, dO=dO, dS_T=dS_T, readout=readout)
+    gc = chunked.bwd(**x, dO=dO, dS_T=dS_T, C=C, readout=readout)
     for name in NAMES:
         if g[name] is None:
             assert gc[name] is None
