@@ -3,7 +3,6 @@ C ABI through the Python binding."""
 import numpy as np
 import torch
 
-import dn_inputs as di
 import gated_linear_attention_dn_b200 as dn
 import oracle
 

@@ -2,7 +2,6 @@
 read-out by dn_mc_readout) against the fp64 oracle (oracle/memcache.py), through the C ABI."""
 import numpy as np
 import pytest
-import torch
 
 import dn_inputs as di
 import gated_linear_attention_dn_b200 as dn

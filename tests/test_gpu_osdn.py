@@ -12,7 +12,7 @@ import torch
 import dn_inputs as di
 import gated_linear_attention_dn_b200 as dn
 import oracle
-from tests.gpu_util import TOL, check, dev, host_f64, sampled_heads
+from tests.gpu_util import check, dev, host_f64, sampled_heads
 
 pytestmark = pytest.mark.gpu
 

@@ -12,7 +12,7 @@ import torch
 import dn_inputs as di
 import gated_linear_attention_dn_b200 as dn
 import oracle
-from tests.gpu_util import TOL, check, dev, host_f64, run_chunk, sampled_heads, to_device
+from tests.gpu_util import TOL, check, host_f64, run_chunk, sampled_heads, to_device
 
 pytestmark = pytest.mark.gpu
 

@@ -4,12 +4,11 @@ kernel, the per-token-gate and per-channel-gate tensor-core chunk kernels, and t
 plus the delta-mem update (undecayed residual) through its mapping onto the recurrence."""
 import numpy as np
 import pytest
-import torch
 
 import dn_inputs as di
 import gated_linear_attention_dn_b200 as dn
 import oracle
-from tests.gpu_util import TOL, check, dev, host_f64, to_device
+from tests.gpu_util import check, dev, to_device
 
 pytestmark = pytest.mark.gpu
 
