@@ -62,3 +62,21 @@ def test_workload_shapes():
     assert x0["q"].shape == (4, 1, 32, 128)
     assert not np.array_equal(x0["q"], x1["q"])
     assert x0["S0"] is not None and x1["S0"] is None
+
+
+def test_backward_cotangents():
+    """dO ~ N(0,1) in the storage dtype and dS_T ~ N(0, 0.1^2) fp32, deterministic, and drawn from
+    seeds no forward tensor of any workload uses."""
+    w = di.WORKLOADS["gdn_prefill"].scaled(B=2, T=512, H=4)
+    g1, g2 = di.make_bwd_inputs(w), di.make_bwd_inputs(w)
+    assert g1["dO"].dtype == np.uint16 and g1["dO"].shape == (2, 512, 4, 128)
+    assert g1["dS_T"].dtype == np.float32 and g1["dS_T"].shape == (2, 4, 128, 128)
+    np.testing.assert_array_equal(g1["dO"], g2["dO"])
+    np.testing.assert_array_equal(g1["dS_T"], g2["dS_T"])
+    dO = di.to_f64(g1["dO"], "bf16")
+    assert abs(dO.mean()) < 0.01 and abs(dO.std() - 1.0) < 0.01
+    assert abs(g1["dS_T"].std() - 0.1) < 0.002
+    fwd_seeds = {w2.seed(n) for w2 in di.WORKLOADS.values()
+                 for n in ("q", "k", "v", "alpha", "beta_k", "beta_v", "key_scale", "S0", "beta", "retention")}
+    bwd_seeds = {w2.seed(n) for w2 in di.WORKLOADS.values() for n in ("dO", "dS_T")}
+    assert not (fwd_seeds & bwd_seeds)
