@@ -140,6 +140,45 @@ def test_o7_resume_and_zero_key():
     np.testing.assert_allclose(d[0, 4, 1], ret[0, 3, 1] * d[0, 3, 1], rtol=1e-14)
 
 
+# O8 -- the surrogate is quadratic in d, so one step is affine in d:
+#   d_{t+1} = (r_t I - (eta beta_t^2 / ||k_t||^2) a_t a_t^T) d_t + (eta beta_t / ||k_t||^2) a_t,  a_t = k_t (.) k_t.
+# Hence the scan over any segment is an affine map d -> M d + m: affine combinations of start
+# states map to the same combinations of end states, and chaining the segments' maps (each read off
+# the scan itself from basis start states) reproduces the whole sequence -- the composition a
+# segment-parallel scan would use.
+def test_o8_affine_in_d_and_segment_composition():
+    T, dk, L = 48, 8, 12
+    k = _keys(T, 1, dk, seed=8)
+    r = np.random.default_rng(8)
+    beta = r.uniform(0.2, 1.0, (1, T, 1))
+    ret = r.uniform(0.85, 1.0, (1, T, 1))
+    eta = 0.7
+    x, y = r.uniform(0.5, 2.0, (1, 1, dk)), r.uniform(0.5, 2.0, (1, 1, dk))
+    for w in (0.3, -1.7, 2.5):  # affine (not only convex) combinations
+        _, ex = oracle.osdn_precond(k, beta, ret, x, eta=eta)
+        _, ey = oracle.osdn_precond(k, beta, ret, y, eta=eta)
+        _, ez = oracle.osdn_precond(k, beta, ret, w * x + (1 - w) * y, eta=eta)
+        np.testing.assert_allclose(ez, w * ex + (1 - w) * ey, rtol=1e-12, atol=1e-13)
+    d_full, dT_full = oracle.osdn_precond(k, beta, ret, x, eta=eta)
+    d = x[0, 0].copy()
+    for s0 in range(0, T, L):
+        seg = slice(s0, s0 + L)
+        _, m = oracle.osdn_precond(k[:, seg], beta[:, seg], ret[:, seg], np.zeros((1, 1, dk)), eta=eta)
+        M = np.stack([oracle.osdn_precond(k[:, seg], beta[:, seg], ret[:, seg], np.eye(dk)[i][None, None], eta=eta)[1][0, 0]
+                      - m[0, 0] for i in range(dk)], axis=1)
+        # the same map from the per-token matrices written out
+        A, c = np.eye(dk), np.zeros(dk)
+        for t in range(s0, s0 + L):
+            kt = k[0, t, 0]
+            at, nrm = kt * kt, np.sum(kt * kt)
+            At = ret[0, t, 0] * np.eye(dk) - eta * beta[0, t, 0] ** 2 / nrm * np.outer(at, at)
+            A, c = At @ A, At @ c + eta * beta[0, t, 0] / nrm * at
+        np.testing.assert_allclose(M, A, rtol=1e-11, atol=1e-13)
+        np.testing.assert_allclose(m[0, 0], c, rtol=1e-11, atol=1e-13)
+        d = M @ d + m[0, 0]
+    np.testing.assert_allclose(d, dT_full[0, 0], rtol=1e-11)
+
+
 SRC = os.path.join(os.path.dirname(oracle.__file__), "dn_oracle.c")
 MUTATIONS = {
     "ascent": ("d[i] = rt * d[i] - eta * grad;", "d[i] = rt * d[i] + eta * grad;"),
@@ -151,7 +190,8 @@ MUTATIONS = {
 }
 PINS = [test_o1_no_learning_pure_retention, test_o2_newton_fixed_point,
         lambda: test_o3_geometric_contraction(0.5, 0.8), test_o4_step_is_surrogate_gradient,
-        test_o5_descent_on_the_current_surrogate, test_o6_full_forgetting, test_o7_resume_and_zero_key]
+        test_o5_descent_on_the_current_surrogate, test_o6_full_forgetting, test_o7_resume_and_zero_key,
+        test_o8_affine_in_d_and_segment_composition]
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
