@@ -3,32 +3,45 @@
 // ahead of the state recurrence.
 //
 // One CTA owns one (b, h) sequence (and a slice of NV value columns) and walks its chunks of
-// C = 64 tokens. Per chunk, with decays referenced to the chunk midpoint m (after token 31) and
-// every gate a scalar per token:
+// C = 64 tokens. Every gate is a scalar per token, so every decay factor is a scalar per token (or
+// per token pair) and moves onto the small C x C matrices or onto rows of the raw tiles. With
+// gamma_t = prod_{s <= t} alpha_s (from the chunk start, token t included), S the state entering
+// the chunk and w_t = beta^k_t d_t k_t:
 //
-//   r_t = gamma_t / gamma_m,  A_ti = (k_t . k_i) beta_i d_i r_t / r_i  (i < t),  T = (I + A)^{-1}
-//   Wk = (T Diag(r)) K,  U0 = (T Diag(beta^v)) V,  S_m = Diag(gamma_m) S
-//   U' = Diag(beta d / r) (U0 - Wk S_m)
-//   O_t = r_t (Q S_m + P U')_t,  P_ti = q_t . k_i (i <= t)
-//   S' = (gamma_C / gamma_m) (S_m + K^T U')
+//   A_ti = (gamma_t / gamma_i) beta_i d_i (k_t . k_i)  (i < t),   T = (I + A)^{-1}
+//   Wk = (T Diag(gamma)) K,   U0 = (T Diag(beta^v)) V,   U = U0 - Wk S
+//   o_t = gamma_t S^T q_t + sum_{i <= t} (gamma_t / gamma_i) (q_t . w_i) u_i
+//   S'  = gamma_C S + sum_i (gamma_C / gamma_i) w_i u_i^T
 //
 // (the chunk-parallel WY / UT evaluation of the gated delta rule: FG2-GDN page, sections 2.A and
-// 3 item 2; the scalar-gate rewriting of it keeps the raw TMA tiles of q, k, v as tensor-core
-// operands with no elementwise pass).
+// 3 item 2). Every factor above is a ratio of decay products, at most 1 for gates in (0, 1], and
+// the products themselves are carried as mantissa and exponent (split_pow2), so no gate strength
+// can overflow or underflow an intermediate: small factors round to zero, as the recurrence does.
+// The output and the state update read one residual tile between them, U'_i = c_i u_i, and the
+// powers of two that separate their two scalings move, exactly, onto rows of the raw tiles:
 //
-// Only the last four lines depend on the state. Two warp groups therefore work one chunk apart:
-//  * the state group (warps 0..7) runs the state chain of chunk c: the Wk and U0 products, S_m,
-//    D1 = [Wk; Q] S_m, U', the O and state-update products and the o store;
-//  * the transform group (warps 8..15) meanwhile prepares chunk c + 1: its decay factors, A and P
+//   gamma_t = rho_t 2^{e_t},  gamma_C / gamma_i = mu_i 2^{n_i}   (rho, mu in [0.5, 1))
+//   c_i = beta_i d_i mu_i,   K'_i = 2^{n_i} k_i,   Q'_t = 2^{e_t} q_t
+//   P'_ti = (q_t . k_i) 2^{e_t - e_i} / (rho_i mu_i)   (i <= t)
+//   o_t = rho_t (Q' S + P' U')_t,    S' = gamma_C S + K'^T U'
+//
+// (the read-out before the update uses gamma_{t-1} in place of gamma_t and i < t).
+//
+// Only the last lines depend on the state. Two warp groups therefore work one chunk apart:
+//  * the state group (warps 0..7) runs the state chain of chunk c: the Wk and U0 products, the
+//    state framing, D1 = [Wk; Q'] S, U', the O and state-update products and the o store;
+//  * the transform group (warps 8..15) meanwhile prepares chunk c + 1: its decay factors, A and P'
 //    from the Gram product [K; Q] K^T (issued by the state group right after chunk c's Wk / U0
-//    products), and the inverse T, emitted as the bf16 operand tiles T Diag(r) and T Diag(beta^v).
+//    products), and the inverse T, emitted as the bf16 operand tiles T Diag(gamma) and
+//    T Diag(beta^v).
 // Hand-offs are mbarriers: the transform group arrives on `tready` once chunk c + 1's tiles are in
 // shared memory; the Gram of chunk c + 1 is committed after chunk c's Wk / U0 products, so its
 // completion also tells the transform group that the T tiles of chunk c are no longer read.
-// P is double-buffered by chunk parity; the per-token factors are kept for four chunks.
+// P' is double-buffered by chunk parity; the per-token factors are kept for four chunks.
 //
-// Precision: bf16 operands, fp32 accumulation; U' is split hi + lo for the state update (raw k is
-// exact in bf16); T is inverted in fp32 (TF32 block merges) and rounded to bf16 once.
+// Precision: bf16 operands, fp32 accumulation; U' is split hi + lo for the state update (K' is raw k
+// times a power of two, exact in bf16); T is inverted in fp32 (TF32 block merges) and rounded to
+// bf16 once.
 //
 // Tensor memory (512 columns): S_acc | D1 | U0 | (Wk, d_v = 64 only) | Gram; Wk shares D1's columns
 // when d_v = 128 (D1 is written only after Wk has been read).
@@ -51,17 +64,17 @@ constexpr int kXformThreads = 256;   // warps 8..15
 constexpr int kThreads = kStateThreads + kXformThreads;
 constexpr int kBarState = 1, kBarXform = 2;   // hardware barriers of the two groups (0 = whole CTA)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, far above any legitimate wait
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: the bound of the drain waits after a failure
 
 template <int NV>
 struct ScLayout {
-  static constexpr int STK = 0;                   // raw k [C][DK] (TMA): state-update operand
+  static constexpr int STK = 0;                   // raw k [C][DK] (TMA), rows scaled to K': state-update operand
   static constexpr int STQ = STK + C * DK * 2;    // T Diag(beta^v) [128][C]: rows 0..63 bf16 hi, 64..127 lo (or 0)
   static constexpr int STV = STQ + 128 * C * 2;   // raw v [C][NV] (TMA)
   static constexpr int KQ0 = STV + C * NV * 2;    // [K; Q] (TMA), then [Wk; Q]: even chunks
   static constexpr int KQ1 = KQ0 + 128 * DK * 2;  //                               odd chunks
-  static constexpr int TP = KQ1 + 128 * DK * 2;   // T Diag(r) | P (even chunks) | P (odd chunks), 64 rows each
-  static constexpr int SMU = TP + 3 * C * C * 2;  // S_m bf16 [DK][NV]; after D1: U' hi, U' lo [C][NV]
+  static constexpr int TP = KQ1 + 128 * DK * 2;   // T Diag(gamma) | P' (even chunks) | P' (odd chunks), 64 rows each
+  static constexpr int SMU = TP + 3 * C * C * 2;  // S bf16 [DK][NV]; after D1: U' hi, U' lo [C][NV]
   static constexpr int SMU_BYTES = (DK * NV * 2 > 2 * C * NV * 2) ? DK * NV * 2 : 2 * C * NV * 2;
   static constexpr int INV = SMU + SMU_BYTES;     // fp32 L and T of the inverse (64 x 64 each)
   static constexpr int TOTAL = INV + 2 * C * C * 4;
@@ -69,8 +82,8 @@ struct ScLayout {
   static constexpr int TM_WK = (NV == 128) ? TM_D1 : 3 * NV;
   static constexpr int TM_GR = (NV == 128) ? 3 * NV : 3 * NV + DK;
   static_assert(TM_GR + 64 <= (int)kTmemCols, "tensor memory budget");
-  // dynamic (plus 1 KB for alignment) and about 15 KB of static shared memory per CTA
-  static_assert(TOTAL + 1024 + 16 * 1024 <= 227 * 1024, "shared memory budget");
+  // dynamic (plus 1 KB for alignment) and about 20 KB of static shared memory per CTA
+  static_assert(TOTAL + 1024 + 20 * 1024 <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
@@ -88,13 +101,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_qk[2], bar_k, bar_v, bar_mma, bar_gram, bar_tready, bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ __align__(16) float s_Y[2048];  // inverse scratch
-  // per-token factors by chunk index mod 4: r_t, 1/r_t, beta^k d, beta^v; gamma_C / gamma_m; gamma_m
-  __shared__ float s_r[4][C], s_ri[4][C], s_ws[4][C], s_bv[4][C], s_al[4][C];
-  __shared__ float s_lam[4], s_gm[4];
+  // per-token factors by chunk index mod 4 (gamma_t = rho_t 2^{e_t}, gamma_C / gamma_t = mu_t 2^{n_t}):
+  // rho_t, 1 / rho_t, e_t; the read-out's o scale and Q' exponent (those of gamma_t, or of
+  // gamma_{t-1} before the update); 1 / (rho_t mu_t); c_t = beta^k_t d_t mu_t; n_t; beta^k d;
+  // beta^v; gamma_t as a float; and gamma_C per chunk
+  __shared__ float s_rho[4][C], s_rhoi[4][C], s_orho[4][C], s_pinv[4][C], s_c[4][C], s_ws[4][C], s_bv[4][C],
+      s_gam[4][C];
+  __shared__ int s_ex[4][C], s_oex[4][C], s_n[4][C];
+  __shared__ float s_glast[4];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
-  const int pre = a.pre_read ? 1 : 0;  // o_t before the token's update: strictly causal P, scale r_{t-1}
+  const int pre = a.pre_read ? 1 : 0;  // o_t before the token's update: strictly causal P', gamma_{t-1}
   // a per-token beta^v is folded into T Diag(beta^v), kept as bf16 hi + lo (U0 = T~_hi V + T~_lo V)
   const bool bv_split = a.beta_v != DN_GATE_ONE;
   const int T = a.T, H = a.H, dv = a.dv;
@@ -187,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_k(0);
       issue_v(0);
       pend_k = pend_v = true;
-      if (mbar_wait_bounded(&bar_qk[0], ph_qk[0], kWaitNs)) {
+      if (mbar_wait_bounded(&bar_qk[0], ph_qk[0], a.wait_ns)) {
         ph_qk[0] ^= 1;
         pend_qk[0] = false;
         tc_fence_after();
@@ -202,13 +220,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t id_state = idesc_bf16(128, NV, 1, 1);
 
     for (int c = 0; c < nchunks; ++c) {
-      const int t0 = c * C, cur = c & 3, prev = (c + 3) & 3;
+      const int t0 = c * C, cur = c & 3;
       uint8_t* const kq = kq_buf(c);
 
       // ---- M0: chunk c's T tiles, P and factors are ready; its v tile has landed
       {
-        const bool ok = ok0 && mbar_wait_bounded(&bar_tready, ph_tr, kWaitNs) &&
-                        mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
+        const bool ok = ok0 && mbar_wait_bounded(&bar_tready, ph_tr, a.wait_ns) &&
+                        mbar_wait_bounded(&bar_v, ph_v, a.wait_ns);
         if (group_or(kBarState, kStateThreads, !ok)) {
           failed = true;
           break;
@@ -219,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
 
-      // ---- M1: Wk = (T Diag r) K -> TM_WK, U0 = (T Diag beta^v) V -> TM_U0; then chunk c + 1's Gram
+      // ---- M1: Wk = (T Diag gamma) K -> TM_WK, U0 = (T Diag beta^v) V -> TM_U0; then chunk c + 1's Gram
       // (its completion also tells the transform group that chunk c's T tiles are no longer read)
       if (tid == 0) {
 #pragma unroll
@@ -247,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bar_mma);
         if (c + 1 < nchunks) {
           const int j = (c + 1) & 1;
-          if (mbar_wait_bounded(&bar_qk[j], ph_qk[j], kWaitNs)) {
+          if (mbar_wait_bounded(&bar_qk[j], ph_qk[j], a.wait_ns)) {
             ph_qk[j] ^= 1;
             pend_qk[j] = false;
             issue_gram(c + 1);
@@ -257,11 +275,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // meanwhile: S_m = Diag(lambda_{c-1} gamma_m) S -> TM_S (fp32) and the bf16 tile in SMU; rows
-      // 32 q4 .. +32, columns of half ch
+      // meanwhile: the state entering the chunk -> bf16 operand tile in SMU, and gamma_C S -> TM_S
+      // (fp32, where the state update accumulates); rows 32 q4 .. +32, columns of half ch
       {
         const int k = 32 * q4 + lane;
-        const float mu = (c == 0) ? s_gm[cur] : s_lam[prev] * s_gm[cur];
+        const float gl = s_glast[cur];
         uint32_t xr[NCB][32];  // all TMEM loads of this thread in flight at once
         if (c == 0) {
 #pragma unroll
@@ -286,19 +304,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int col = ch * (NV / 2) + 32 * cb;
           float x[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(xr[cb][e]) * mu;
-          tmem_st32_issue(tmem + lane_base + Ly::TM_S + col, x);
+          for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(xr[cb][e]);
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
                                   pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
             *reinterpret_cast<uint4*>(sm + Ly::SMU + canon_chunk(k, col / 8 + q8, DK)) = pk;
           }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= gl;
+          tmem_st32_issue(tmem + lane_base + Ly::TM_S + col, x);
         }
         tmem_wait_st();
       }
       {
-        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
         if (group_or(kBarState, kStateThreads, !ok)) {
           failed = true;
           break;
@@ -311,7 +331,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         pend_v = true;
       }
 
-      // ---- M2: Wk -> bf16 into rows 0..63 of the [K; Q] tile (K is not read again)
+      // ---- M2: Wk -> bf16 into rows 0..63 of the [K; Q] tile (K is not read again); meanwhile the
+      // other warps scale rows 64..127 to Q' = 2^{e_t} q_t (this chunk's Gram is complete: its
+      // transform arrived on tready)
+      if (q4 >= 2) {
+        const int t = 32 * (q4 - 2) + lane;
+        const float sc = pow2f(s_oex[cur][t]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4* p = reinterpret_cast<uint4*>(kq + canon_chunk(64 + t, 8 * ch + j, 128));
+          *p = scale_bf16x8(*p, sc);
+        }
+      }
       if (q4 < 2) {
         const int t = 32 * q4 + lane;
         uint32_t xr[DK / 64][32];
@@ -338,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       group_sync(kBarState, kStateThreads);
       tc_fence_after();
 
-      // ---- M3: D1 = [Wk; Q] S_m -> TM_D1
+      // ---- M3: D1 = [Wk; Q'] S -> TM_D1
       if (tid == 0) {
 #pragma unroll
         for (int kk = 0; kk < DK; kk += 16) {
@@ -349,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bar_mma);
       }
       {
-        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
         if (group_or(kBarState, kStateThreads, !ok)) {
           failed = true;
           break;
@@ -363,10 +394,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         pend_qk[c & 1] = true;
       }
 
-      // ---- M4: U' = (beta d / r) (U0 - Wk S_m), rows 0..63 -> hi / lo tiles (S_m is dead)
+      // ---- M4: U' = c (U0 - Wk S), rows 0..63 -> hi / lo tiles (the S tile is dead); meanwhile the
+      // other warps wait for this chunk's raw k tile and scale its rows to K' = 2^{n_i} k_i
+      bool ok_k = true;
+      if (q4 >= 2) {
+        ok_k = mbar_wait_bounded(&bar_k, ph_k, a.wait_ns);
+        if (ok_k) {
+          const int u = 32 * ((q4 - 2) + 2 * ch) + lane;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int e = u + 128 * it, i = e >> 4;
+            uint4* p = reinterpret_cast<uint4*>(sm + Ly::STK + canon_chunk(i, e & 15, C));
+            *p = scale_bf16x8(*p, pow2f(s_n[cur][i]));
+          }
+        }
+      }
       if (q4 < 2) {
         const int t = 32 * q4 + lane;
-        const float us = s_ws[cur][t] * s_ri[cur][t];
+        const float us = s_c[cur][t];
 #pragma unroll
         for (int cb = 0; cb < NV / 64; ++cb) {
           const int col = ch * (NV / 2) + 32 * cb;
@@ -394,10 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async();
       {
-        // the raw k tile of the state update (loaded during the previous chunk)
-        const bool ok = mbar_wait_bounded(&bar_k, ph_k, kWaitNs);
         tc_fence_before();
-        if (group_or(kBarState, kStateThreads, !ok)) {
+        if (group_or(kBarState, kStateThreads, !ok_k)) {
           failed = true;
           break;
         }
@@ -406,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
 
-      // ---- M5: D1 rows 64..127 += P U' (O); S_acc += K^T U' (hi and lo)
+      // ---- M5: D1 rows 64..127 += P' U' (O); S_acc += K'^T U' (hi and lo)
       if (tid == 0) {
         const uint32_t pa = smem_u32(sm + Ly::TP) + (uint32_t)(c & 1) * (C * C * 2);  // rows 64..127 = P
 #pragma unroll
@@ -426,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bar_mma);
       }
       {
-        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+        const bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
         if (group_or(kBarState, kStateThreads, !ok)) {
           failed = true;
           break;
@@ -439,12 +482,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         pend_k = true;
       }
 
-      // ---- M6: o rows of chunk c = r_t (rows 64..127 of D1), warps of quadrants 2 and 3; the TMEM
-      // load is warp-collective: every lane loads, only rows of real tokens store
+      // ---- M6: o rows of chunk c = rho_t x (rows 64..127 of D1), warps of quadrants 2 and 3; the
+      // TMEM load is warp-collective: every lane loads, only rows of real tokens store
       if (q4 >= 2) {
         const int t = 32 * (q4 - 2) + lane, nc = min(C, T - t0);
-        // post-update read-out: r_t; pre-update: r_{t-1} = r_t / alpha_t
-        const float os = pre ? __fdividef(s_r[cur][t], s_al[cur][t]) : s_r[cur][t];
+        const float os = s_orho[cur][t];  // mantissa of gamma_t (of gamma_{t-1} before the update)
         __nv_bfloat16* orow =
             reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0 + t) * H + h) * dv + col0;
         uint32_t xr[NCB][32];
@@ -474,9 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (!failed && nchunks > 0) {
-      // S_T = (gamma_C / gamma_m) S_acc of the last chunk
+      // S_T = S_acc of the last chunk
       const int k = 32 * q4 + lane;
-      const float lam = s_lam[(nchunks - 1) & 3];
 #pragma unroll
       for (int cb = 0; cb < NV / 64; ++cb) {
         const int col = ch * (NV / 2) + 32 * cb;
@@ -485,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* dst = a.S + ((int64_t)bh * DK + k) * dv + col0 + col;
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + e) = make_float4(lam * x[e], lam * x[e + 1], lam * x[e + 2], lam * x[e + 3]);
+          *reinterpret_cast<float4*>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
       }
     }
     if (failed && tid == 0) {
@@ -502,51 +543,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================================================= transform group
     const int gt = tid - kStateThreads, gw = gt >> 5, gch = gw >> 2;  // q4 == gw & 3
     uint32_t ph_gr = 0;
-    // Thread j < 64 (warps 8, 9) loads token j's gates (alpha, beta^k, d, beta^v) of chunk cn into
-    // registers, one chunk ahead of their use; absent gates read as 1, tokens past the end as
-    // alpha 1 and 0 for the others (no decay, no write).
-    float gx[4];
+    // Thread j < 64 (warps 8, 9) loads token j's gates (alpha, beta^k, d, beta^v) of chunk cn, and
+    // the alpha of token j ^ 32, into registers one chunk ahead of their use; absent gates read as 1,
+    // tokens past the end as alpha 1 and 0 for the others (no decay, no write).
+    float gx[5];
     auto load_gates = [&](int cn, int j) {
-      const bool valid = j < T - cn * C;
+      const int left = T - cn * C;
+      const bool valid = j < left, valid_p = (j ^ 32) < left;
       const int64_t tok = ((int64_t)b * T + cn * C + j) * H + h;
+      const int64_t tok_p = ((int64_t)b * T + cn * C + (j ^ 32)) * H + h;
       gx[0] = (valid && a.alpha == DN_GATE_SCALAR) ? __ldg(a.alpha_p + tok) : 1.f;
       gx[1] = (valid && a.beta_k == DN_GATE_SCALAR) ? __ldg(a.beta_k_p + tok) : (valid ? 1.f : 0.f);
       gx[2] = (valid && a.key_scale == DN_GATE_SCALAR) ? __ldg(a.key_scale_p + tok) : 1.f;
       gx[3] = (valid && a.beta_v == DN_GATE_SCALAR) ? __ldg(a.beta_v_p + tok) : (valid ? 1.f : 0.f);
+      gx[4] = (valid_p && a.alpha == DN_GATE_SCALAR) ? __ldg(a.alpha_p + tok_p) : 1.f;
     };
-    // Decay factors of chunk cn from its gates in gx (then the next chunk's are loaded). Warp 9
-    // (tokens 32..63) forms r_j = prod_{s=32..j} alpha_s by an inclusive product scan, warp 8
-    // (tokens 0..31) 1/r_j = prod_{s=j+1..31} alpha_s by an exclusive suffix scan;
-    // gamma_m = prod_{s<32} alpha_s, gamma_C / gamma_m = prod_{s>=32} alpha_s.
+    // Decay factors of chunk cn from the gates in gx (then the next chunk's are loaded). Each of
+    // warps 8 and 9 scans both halves of the chunk (lane l holds tokens l and 32 + l), so neither
+    // waits for the other: inclusive prefix products in mantissa-exponent form give gamma_t, the
+    // previous token's gamma_{t-1} and gamma_C.
     auto token_prep = [&](int cn, int j) {
       const int slot = cn & 3;
-      const float al = gx[0], ws = gx[1] * gx[2], bv = gx[3];
+      const float ws = gx[1] * gx[2], bv = gx[3];
+      const bool hi = j >= 32;
+      float m1, m2;
+      int e1, e2;
+      split_pow2(hi ? gx[4] : gx[0], m1, e1);  // token lane
+      split_pow2(hi ? gx[0] : gx[4], m2, e2);  // token 32 + lane
       if (cn + 1 < nchunks) load_gates(cn + 1, j);
-      float p = al;
-      if (j >= 32) {
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, p, off);
-          if (lane >= off) p *= y;
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y1 = __shfl_up_sync(0xffffffffu, m1, off), y2 = __shfl_up_sync(0xffffffffu, m2, off);
+        const int f1 = __shfl_up_sync(0xffffffffu, e1, off), f2 = __shfl_up_sync(0xffffffffu, e2, off);
+        if (lane >= off) {
+          mul_pow2(m1, e1, y1, f1);
+          mul_pow2(m2, e2, y2, f2);
         }
-        s_r[slot][j] = p;
-        s_ri[slot][j] = __fdividef(1.f, p);
-        if (lane == 31) s_lam[slot] = p;
-      } else {
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_down_sync(0xffffffffu, p, off);
-          if (lane + off < 32) p *= y;
-        }
-        const float nxt = __shfl_down_sync(0xffffffffu, p, 1);
-        const float ri = lane == 31 ? 1.f : nxt;
-        s_ri[slot][j] = ri;
-        s_r[slot][j] = __fdividef(1.f, ri);
-        if (lane == 0) s_gm[slot] = p;
       }
+      const float t1m = __shfl_sync(0xffffffffu, m1, 31), t2m = __shfl_sync(0xffffffffu, m2, 31);
+      const int t1e = __shfl_sync(0xffffffffu, e1, 31), t2e = __shfl_sync(0xffffffffu, e2, 31);
+      float p1m = __shfl_up_sync(0xffffffffu, m1, 1), p2m = __shfl_up_sync(0xffffffffu, m2, 1);
+      int p1e = __shfl_up_sync(0xffffffffu, e1, 1), p2e = __shfl_up_sync(0xffffffffu, e2, 1);
+      float gm, pm;  // gamma_j and gamma_{j-1}
+      int ge, pe;
+      if (!hi) {
+        gm = m1, ge = e1;
+        if (lane == 0) p1m = 0.5f, p1e = 1;  // gamma_{-1} = 1
+        pm = p1m, pe = p1e;
+      } else {
+        gm = t1m, ge = t1e;
+        mul_pow2(gm, ge, m2, e2);
+        pm = t1m, pe = t1e;
+        if (lane > 0) mul_pow2(pm, pe, p2m, p2e);
+      }
+      float lm = t1m;  // gamma_C
+      int le = t1e;
+      mul_pow2(lm, le, t2m, t2e);
+      float mu = __fdividef(lm, gm);  // gamma_C / gamma_j = mu 2^ne, mu in [0.5, 1)
+      int ne = le - ge;
+      if (mu >= 1.f) mu *= 0.5f, ne += 1;
+      s_rho[slot][j] = gm;
+      s_rhoi[slot][j] = __fdividef(1.f, gm);
+      s_ex[slot][j] = ge;
+      s_orho[slot][j] = pre ? pm : gm;
+      s_oex[slot][j] = pre ? pe : ge;
+      s_pinv[slot][j] = __fdividef(1.f, gm * mu);
+      s_c[slot][j] = ws * mu;
+      s_n[slot][j] = ne;
+      s_gam[slot][j] = gm * pow2f(ge);
       s_ws[slot][j] = ws;
       s_bv[slot][j] = bv;
-      s_al[slot][j] = al;
+      if (j == 63) s_glast[slot] = lm * pow2f(le);
     };
     if (gt < 64 && nchunks > 0) load_gates(0, gt);
 
@@ -555,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (gt < 64) token_prep(n, gt);
       // ---- X1: the Gram of chunk n has completed, and with it chunk n - 1's Wk / U0 products
       {
-        const bool ok = mbar_wait_bounded(&bar_gram, ph_gr, kWaitNs);
+        const bool ok = mbar_wait_bounded(&bar_gram, ph_gr, a.wait_ns);
         if (group_or(kBarXform, kXformThreads, !ok)) {
           failed = true;
           break;
@@ -563,13 +630,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ph_gr ^= 1;
         tc_fence_after();
       }
-      // ---- X2: A (strict lower, scaled) -> fp32 L; P (lower incl., raw q.k) -> bf16 P tile of parity
-      // n & 1 (last read by chunk n - 2's O product, long complete)
+      // ---- X2: A (strict lower) -> fp32 L; P' (lower incl., or strictly lower before the update) ->
+      // bf16 P' tile of parity n & 1 (last read by chunk n - 2's O product, long complete)
       float* sL = reinterpret_cast<float*>(sm + Ly::INV);
       float* sT = sL + C * C;
       if (q4 < 2) {
         const int t = 32 * q4 + lane;
-        const float rt = s_r[cur][t];
+        const float rt = s_rho[cur][t];
+        const int et = s_ex[cur][t];
         float x[32];
         tmem_ld32(tmem + lane_base + Ly::TM_GR + 32 * gch, x);
 #pragma unroll
@@ -578,12 +646,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = 32 * gch + 4 * e4 + e;
-            y[e] = (i < t) ? x[4 * e4 + e] * s_ws[cur][i] * rt * s_ri[cur][i] : 0.f;
+            const float f = s_ws[cur][i] * (rt * s_rhoi[cur][i]) * pow2f(et - s_ex[cur][i]);  // (gamma_t / gamma_i) beta_i d_i
+            y[e] = (i < t) ? x[4 * e4 + e] * f : 0.f;
           }
           *reinterpret_cast<float4*>(sL + xi(t, 32 * gch + 4 * e4)) = make_float4(y[0], y[1], y[2], y[3]);
         }
       } else {
         const int t = 32 * (q4 - 2) + lane;
+        const int et = s_oex[cur][t];
         uint8_t* pt = sm + Ly::TP + (1 + (n & 1)) * (C * C * 2);
         float x[32];
         tmem_ld32(tmem + lane_base + Ly::TM_GR + 32 * gch, x);
@@ -591,18 +661,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q8 = 0; q8 < 4; ++q8) {
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = (32 * gch + 8 * q8 + e <= t - pre) ? x[8 * q8 + e] : 0.f;
+          for (int e = 0; e < 8; ++e) {
+            const int i = 32 * gch + 8 * q8 + e;
+            const float f = s_pinv[cur][i] * pow2f(et - s_ex[cur][i]);  // 2^{e_t - e_i} / (rho_i mu_i)
+            y[e] = (i <= t - pre) ? x[8 * q8 + e] * f : 0.f;
+          }
           *reinterpret_cast<uint4*>(pt + canon_chunk(t, 4 * gch + q8, 64)) =
               make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]));
         }
       }
       tc_fence_before();
-      // ---- X3: T = (I + A)^{-1} -> T Diag(r) (TP rows 0..63) and T Diag(beta^v) (STQ rows 0..63)
+      // ---- X3: T = (I + A)^{-1} -> T Diag(gamma) (TP rows 0..63) and T Diag(beta^v) (STQ rows 0..63)
       if (bv_split)
-        unit_lower_inverse<true, 8, false, true>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt,
+        unit_lower_inverse<true, 8, false, true>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_gam[cur], s_bv[cur], gt,
                                                  kBarXform);
       else
-        unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_r[cur], s_bv[cur], gt,
+        unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_gam[cur], s_bv[cur], gt,
                                            kBarXform);
       fence_proxy_async();
       group_sync(kBarXform, kXformThreads);

@@ -11,8 +11,9 @@
 
 namespace dn {
 
-// Device status codes written to the per-GPU status word (0 = fine).
-enum : int { kDevOk = 0, kDevTimeout = 1 };
+// Device status codes written to the per-GPU status word (0 = fine): a bounded wait gave up, or a
+// chunk's gates were outside the range a kernel's factorisation supports.
+enum : int { kDevOk = 0, kDevTimeout = 1, kDevGateRange = 2 };
 
 // Everything a kernel launch needs, already validated by the ABI shim.
 struct Args {
@@ -31,7 +32,11 @@ struct Args {
   void* o;
   float* S;                       // S_T (chunk fwd) or the in/out state (decode)
   int* status;                    // device status word of the current GPU
+  uint64_t wait_ns;               // bound of each mbarrier wait of the chunk kernels (0: one probe)
 };
+
+// The wait bound the launches take (dn_set_wait_limit_ns; 2 s unless changed).
+uint64_t wait_limit_ns();
 
 // Launchers (host). Each returns cudaSuccess or the launch error.
 cudaError_t launch_decode(const Args& a, cudaStream_t s);
@@ -75,6 +80,43 @@ __device__ __forceinline__ float gate_load(const float* g, int mode, int64_t tok
   if (mode == DN_GATE_SCALAR) return g[tok];
   return g[tok * width + ch];
 }
+
+// ---------------------------------------------------------------- decay products without range limits
+// A product of gates is carried as m * 2^e with m in [0.5, 1) and an integer exponent, so a chunk's
+// cumulative decay never under- or overflows however strong the gates are; only the final factors,
+// which are at most 1 in size, are formed as floats.
+
+// x = m * 2^e for x > 0 (subnormals included). A gate that is 0 (or not positive) becomes
+// 0.5 * 2^-1000: every product that contains it then rounds to zero, as it should.
+__device__ __forceinline__ void split_pow2(float x, float& m, int& e) {
+  if (!(x > 0.f)) {
+    m = 0.5f;
+    e = -1000;
+    return;
+  }
+  int s = 0;
+  if (x < 1.17549435e-38f) {  // subnormal: scale into the normal range first (exact)
+    x *= 18446744073709551616.f;  // 2^64
+    s = 64;
+  }
+  const int bits = __float_as_int(x);
+  e = ((bits >> 23) & 0xff) - 126 - s;
+  m = __int_as_float((bits & 0x007fffff) | 0x3f000000);
+}
+
+// (m, e) *= (m2, e2), renormalised so that m stays in [0.5, 1).
+__device__ __forceinline__ void mul_pow2(float& m, int& e, float m2, int e2) {
+  m *= m2;
+  e += e2;
+  if (m < 0.5f) {
+    m *= 2.f;
+    e -= 1;
+  }
+}
+
+// 2^k as a float: exact for -126 <= k <= 127, 0 below (those factors are negligible next to 1),
+// 2^127 above.
+__device__ __forceinline__ float pow2f(int k) { return __int_as_float(min(max(k + 127, 0), 254) << 23); }
 
 // Streaming 16-byte global load that does not allocate in L1 (the state is touched once).
 // Not the non-coherent path: the decode kernel writes the same addresses later.

@@ -47,10 +47,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Non-blocking probe of the phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: gives up once `limit_ns` of wall-clock time has passed (each
 // try_wait poll may itself suspend the thread for a while, so the bound is on
 // time, not on polls), returning false so the caller can bail out cleanly.
+// limit_ns == 0 probes once without blocking.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (limit_ns == 0) return mbar_test_wait(bar, parity);
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -260,6 +275,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
   return __bfloat1622float2(h);
+}
+
+// Eight packed bf16 values times a float (a power of two in the callers, so the scaling is exact
+// unless a value leaves the bf16 range).
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 u, float s) {
+  float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
+  return make_uint4(pack_bf16(a.x * s, a.y * s), pack_bf16(b.x * s, b.y * s), pack_bf16(c.x * s, c.y * s),
+                    pack_bf16(d.x * s, d.y * s));
 }
 
 // Split x into hi = bf16(x) and lo = bf16(x - hi): hi + lo carries ~16 mantissa bits.
