@@ -163,7 +163,14 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
       hb[t * LD + i] = run;
       if (t == tr) r = run;
     }
-    for (int t = 0; t < kC; ++t) hb[t * LD + i] -= r;
+    // every exponent of the factorisation within +-80 (e^80 ~ 5.5e34), else the chunk's factors
+    // would over- or underflow fp32: report it instead of returning non-finite gradients
+    bool ok = fabsf(r) <= 80.f && fabsf(run - r) <= 80.f;
+    for (int t = 0; t < kC; ++t) {
+      hb[t * LD + i] -= r;
+      ok = ok && fabsf(hb[t * LD + i]) <= 80.f;
+    }
+    if (!ok && a.status) atomicExch(a.status, kDevGateRange);
     er[i] = expf(r);
     lam[i] = expf(run - r);
   }

@@ -32,6 +32,12 @@
 // canon()); q/k/v tiles arrive by TMA (4-D tensor maps over [B, T, H, d], boxes of
 // 64 channels x 64 tokens, zero fill past the end of the sequence).
 //
+// Strong decay: the midpoint-referenced factors stay within 2^-50 .. 2^50 only while the gates of
+// each half chunk multiply to no less than that (mean alpha above ~0.34 per token). A chunk whose
+// factors leave that range (any gate product of a half chunk below 2^-50, per channel) is evaluated
+// exactly instead, token by token on the CUDA cores in fp32 (exact_chunk), from and back to the
+// state in tensor memory; every other chunk keeps the tensor-core path.
+//
 // Tensor memory (512 columns): S_acc [0, NV) | D1 [NV, 2NV) | U0 [2NV, 3NV) | scratch (Gram, Wk).
 // Every wait on an mbarrier is bounded in time; on expiry the CTA sets the status
 // word, drains what it issued (again bounded), frees its tensor memory and exits.
@@ -48,7 +54,7 @@ using namespace ut;
 constexpr int C = 64;
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait, far above any legitimate wait
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: the bound of the drain waits after a failure
 
 template <int DK, int NV>
 struct Layout {
@@ -69,6 +75,8 @@ struct Layout {
   static constexpr int TOTAL = (INV + 2 * C * C * 4 > END) ? INV + 2 * C * C * 4 : END;
   static constexpr int TM_S = 0, TM_D1 = NV, TM_U0 = 2 * NV, TM_SCR = 3 * NV;
   static_assert(TM_SCR + (DK > 64 ? DK : 64) <= (int)kTmemCols, "tensor memory budget");
+  // the exact path's fp32 state transpose (DK x (NV + 1)) overlays [T; P] and what follows it
+  static_assert(TP + DK * (NV + 1) * 4 <= TOTAL, "transpose buffer of the exact path");
 };
 
 __device__ __forceinline__ float4 f4(float x) { return make_float4(x, x, x, x); }
@@ -105,6 +113,12 @@ __device__ __forceinline__ void gate4x8(float4* out, const float* g, int mode, i
 }
 
 __device__ __forceinline__ float4 lds4(const float* p, int idx) { return *reinterpret_cast<const float4*>(p + idx); }
+
+// every component within [2^-50, 2^50] (false for NaN)
+__device__ __forceinline__ bool in_range4(float4 v) {
+  constexpr float lo = 8.8817842e-16f, hi = 1.1258999e15f;
+  return v.x >= lo && v.x <= hi && v.y >= lo && v.y <= hi && v.z >= lo && v.z <= hi && v.w >= lo && v.w <= hi;
+}
 __device__ __forceinline__ void sts4(float* p, int idx, float4 v) { *reinterpret_cast<float4*>(p + idx) = v; }
 
 __device__ __forceinline__ uint2 pack4(float4 v) { return make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w)); }
@@ -115,6 +129,114 @@ __device__ __forceinline__ float4 unpack4(uint2 u) {
 __device__ __forceinline__ void split4(float4 v, uint2& hi, uint2& lo) {
   split_bf16(v.x, v.y, hi.x, lo.x);
   split_bf16(v.z, v.w, hi.y, lo.y);
+}
+
+// Exact evaluation of one chunk, token by token on the CUDA cores in fp32, for a chunk whose decay is
+// too strong for the midpoint-referenced factors of the tensor-core path. In: the chunk's raw k and q
+// tiles, V~ (bf16 hi + lo when beta^v is given, else raw v), alpha and w = beta^k d k per token and
+// key channel as fp32 rows (sAl, sWk, [C][DK]) and w_t . q_t per token (s_wq); the state entering
+// the chunk comes from tensor memory times the previous chunk's pending end factor lam_prev (or from
+// S0 at c == 0). Out: o of the chunk's n tokens straight to global memory, and the chunk-end state
+// back into tensor memory (S_acc, no pending factor). Thread (j, part) owns value column j and DK / TPC
+// key rows of it, so the per-token sums over the rows take TPC - 1 shuffles and no barrier; sX
+// (DK x (NV + 1) fp32) transposes the state between the tensor-memory rows and these columns.
+// Called by all 256 threads.
+template <int DK, int NV>
+__device__ __noinline__ void exact_chunk(const Args& a, const uint8_t* sk, const uint8_t* sq, const uint8_t* svhi,
+                                         const uint8_t* svlo, bool v_split, const float* sAl, const float* sWk,
+                                         const float* s_wq, float* sX, const float* lam_prev, uint32_t tmem_s,
+                                         int c, int n, int b, int h, int bh, int col0, int tid) {
+  constexpr int TPC = kThreads / NV;  // threads per value column
+  constexpr int R = DK / TPC;          // key rows per thread
+  constexpr int LDX = NV + 1;
+  const int warp = tid >> 5, lane = tid & 31, q4 = warp & 3, ch = warp >> 2;
+  const int j = tid / TPC, part = tid % TPC, k0 = part * R;
+  const int T = a.T, H = a.H, dv = a.dv, pre = a.pre_read;
+  {
+    // the state entering the chunk, tensor-memory rows -> sX
+    const int k = 32 * q4 + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+#pragma unroll
+    for (int cb = 0; cb < NV / 64; ++cb) {
+      const int col = ch * (NV / 2) + 32 * cb;
+      float x[32];
+      if (c == 0) {
+        const float* src = a.S0 ? a.S0 + ((int64_t)bh * DK + k) * dv + col0 + col : nullptr;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = src ? src[e] : 0.f;
+      } else {
+        tmem_ld32(tmem_s + lane_base + col, x);
+        const float l = lam_prev[k];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] *= l;
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) sX[k * LDX + col + e] = x[e];
+    }
+  }
+  __syncthreads();
+  float S[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) S[r] = sX[(k0 + r) * LDX + j];
+  __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + c * C) * H + h) * dv + col0 + j;
+  for (int t = 0; t < n; ++t) {
+    const float* al = sAl + t * DK + k0;
+    const float* wr = sWk + t * DK + k0;
+    float rr = 0.f, ss = 0.f;  // (alpha (.) S)^T k and the read-out's S^T q over this thread's rows
+#pragma unroll
+    for (int r8 = 0; r8 < R; r8 += 8) {
+      const uint4 kv = *reinterpret_cast<const uint4*>(sk + canon_chunk(t, (k0 + r8) >> 3, C));
+      const uint4 qv = *reinterpret_cast<const uint4*>(sq + canon_chunk(t, (k0 + r8) >> 3, C));
+      const float2 k01 = unpack_bf16(kv.x), k23 = unpack_bf16(kv.y), k45 = unpack_bf16(kv.z), k67 = unpack_bf16(kv.w);
+      const float2 q01 = unpack_bf16(qv.x), q23 = unpack_bf16(qv.y), q45 = unpack_bf16(qv.z), q67 = unpack_bf16(qv.w);
+      const float kf[8] = {k01.x, k01.y, k23.x, k23.y, k45.x, k45.y, k67.x, k67.y};
+      const float qf[8] = {q01.x, q01.y, q23.x, q23.y, q45.x, q45.y, q67.x, q67.y};
+      const float4 a0 = lds4(al, r8), a1 = lds4(al, r8 + 4);
+      const float af[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float sb = af[e] * S[r8 + e];
+        rr = fmaf(sb, kf[e], rr);
+        ss = fmaf(pre ? S[r8 + e] : sb, qf[e], ss);
+        S[r8 + e] = sb;
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < TPC; off <<= 1) {
+      rr += __shfl_xor_sync(0xffffffffu, rr, off);
+      ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    }
+    const uint32_t voff = canon(t, j, C);
+    float vt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(svhi + voff));
+    if (v_split) vt += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(svlo + voff));
+    const float u = vt - rr;  // u_t = beta^v v_t - S_bar^T k_t
+#pragma unroll
+    for (int r4 = 0; r4 < R; r4 += 4) {
+      const float4 w4 = lds4(wr, r4);
+      S[r4] = fmaf(w4.x, u, S[r4]);
+      S[r4 + 1] = fmaf(w4.y, u, S[r4 + 1]);
+      S[r4 + 2] = fmaf(w4.z, u, S[r4 + 2]);
+      S[r4 + 3] = fmaf(w4.w, u, S[r4 + 3]);
+    }
+    // o_t = S_t^T q_t = S_bar^T q_t + (w . q) u_t; before the update: S_{t-1}^T q_t
+    if (part == 0) orow[(int64_t)t * H * dv] = __float2bfloat16_rn(pre ? ss : fmaf(s_wq[t], u, ss));
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < R; ++r) sX[(k0 + r) * LDX + j] = S[r];
+  __syncthreads();
+  {
+    const int k = 32 * q4 + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+#pragma unroll
+    for (int cb = 0; cb < NV / 64; ++cb) {
+      const int col = ch * (NV / 2) + 32 * cb;
+      float x[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] = sX[k * LDX + col + e];
+      tmem_st32(tmem_s + lane_base + col, x);
+    }
+  }
 }
 
 template <int DK, int NV>
@@ -130,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(16) float s_gm[DK];       // gamma_m per key channel
   __shared__ __align__(16) float s_grp[8][DK];   // per-8-token decay products
   __shared__ __align__(16) float s_Y[2048];
+  __shared__ float s_wq[C];                      // w_t . q_t of a chunk on the exact path
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3, ch = warp >> 2;
@@ -148,12 +271,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
-  // rows 0..63 of the [T; P] tile: the 8x8 blocks above the block diagonal of T are zero and
-  // nothing else writes them; set them once
-  for (int e = tid; e < 64 * 8; e += kThreads) {
-    const int t = e >> 3, x8 = e & 7;
-    if (x8 > (t >> 3)) *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
-  }
+  // rows 0..63 of the [T; P] tile: the 8x8 blocks above the block diagonal of T are zero and the
+  // inverse never writes them; set at the start and again after the exact path has used the tile's
+  // memory
+  auto zero_t_upper = [&]() {
+    for (int e = tid; e < 64 * 8; e += kThreads) {
+      const int t = e >> 3, x8 = e & 7;
+      if (x8 > (t >> 3)) *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
+    }
+  };
+  zero_t_upper();
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
@@ -180,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint32_t ph_qk = 0, ph_v = 0, ph_mma = 0;
   bool qk_pending = false, v_pending = false, mma_pending = false;
+  bool o_pending = false;  // the previous chunk's outputs are still in D1 (stored during this chunk)
   bool failed = false;
   if (tid == 0 && nchunks > 0) {
     issue_qk(0);
@@ -270,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- P0: this chunk's q, k, v have landed
     {
-      bool ok = mbar_wait_bounded(&bar_qk, ph_qk, kWaitNs) && mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
+      bool ok = mbar_wait_bounded(&bar_qk, ph_qk, a.wait_ns) && mbar_wait_bounded(&bar_v, ph_v, a.wait_ns);
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
@@ -280,7 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       qk_pending = v_pending = false;
     }
 
-    // ---- P1: decay factors and the operand tiles
+    // ---- P1: decay factors and the operand tiles (or, for a chunk of too strong a decay, the rows the
+    // exact path reads)
+    bool extreme;
     {
       // per-channel path: thread (g4, tg) owns channels 4g4..4g4+3 of tokens 8tg..8tg+7
       const int g4 = lane, tg = warp, cb0 = 4 * g4;
@@ -329,6 +459,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         for (int g = tg + 1; g < 4; ++g) off = mul4(off, lds4(&s_grp[g][0], cb0));
       }
+      // every factor of the tensor-core path: r_t (second half) or 1 / r_t (first half), gamma_m and
+      // gamma_C / gamma_m; one outside [2^-50, 2^50] sends the chunk to the exact path
+      bool ok = true;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ok = ok && in_range4(mul4(off, loc[i]));
       if (tg == 0) {
         float4 gm = f4(1.f), lm = f4(1.f);
 #pragma unroll
@@ -337,7 +472,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 4; g < 8; ++g) lm = mul4(lm, lds4(&s_grp[g][0], cb0));
         sts4(s_gm, cb0, gm);
         sts4(&s_lam[cur][0], cb0, lm);
+        ok = ok && in_range4(gm) && in_range4(lm);
       }
+      extreme = __syncthreads_or(!ok);
+      if (extreme) {
+        // alpha and w = beta^k d k as fp32 rows [C][DK] over the [K+; Q+] and W- tiles, and w . q
+        float* sAl = reinterpret_cast<float*>(sm + Ly::KQ);
+        float* sWk = reinterpret_cast<float*>(sm + Ly::WHI);
+        float wq[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = 8 * tg + i;
+          const float4 kk = unpack4(kr[i]), qq = unpack4(qr[i]);
+          const float4 wv = mul4(ws[i], kk);
+          sts4(sAl, j * DK + cb0, al[i]);
+          sts4(sWk, j * DK + cb0, wv);
+          wq[i] = wv.x * qq.x + wv.y * qq.y + wv.z * qq.z + wv.w * qq.w;
+        }
+#pragma unroll
+        for (int off2 = 16; off2 > 0; off2 >>= 1)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) wq[i] += __shfl_xor_sync(0xffffffffu, wq[i], off2);
+        if (lane == 0)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) s_wq[8 * tg + i] = wq[i];
+      } else
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int j = 8 * tg + i;
@@ -377,6 +536,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
+    if (extreme) {
+      // ---- exact path for this chunk: the previous chunk's outputs first (they are still in D1)
+      if (o_pending && q4 >= 2) store_o(c - 1);
+      o_pending = false;
+      tc_fence_before();
+      exact_chunk<DK, NV>(a, sm + Ly::STK, sm + Ly::STQ, sm + Ly::STV, sm + Ly::VLO, bv_split,
+                          reinterpret_cast<const float*>(sm + Ly::KQ), reinterpret_cast<const float*>(sm + Ly::WHI),
+                          s_wq, reinterpret_cast<float*>(sm + Ly::TP), &s_lam[cur ^ 1][0], tmem + Ly::TM_S, c, n, b,
+                          h, bh, col0, tid);
+      // the state in tensor memory is now the true state: no pending chunk-end factor
+      if (tid < DK) s_lam[cur][tid] = 1.f;
+      __syncthreads();  // every thread is done with the transpose buffer over the [T; P] tile
+      zero_t_upper();
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      // the staging tiles were read by the exact path: the next chunk's q, k, v may land now
+      if (tid == 0 && c + 1 < nchunks) {
+        issue_qk(c + 1);
+        issue_v(c + 1);
+      }
+      if (c + 1 < nchunks) qk_pending = v_pending = true;
+      continue;
+    }
+
     // ---- P1.5: (the state is brought into this chunk's frame while the T MMAs run, below)
     fence_proxy_async();
     __syncthreads();
@@ -394,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (c + 1 < nchunks) qk_pending = true;
       mma_pending = true;
-      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
@@ -470,10 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_pending = true;
     // while those MMAs run: the previous chunk's outputs (D1 rows 64..127) and the state in this
     // chunk's frame (S_acc columns; no overlap with the TMEM the MMAs write)
-    if (c > 0 && q4 >= 2) store_o(c - 1);
+    if (o_pending && q4 >= 2) store_o(c - 1);
     state_to_frame(c);
     {
-      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
@@ -521,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mma_pending = true;
     {
-      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
@@ -581,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mma_pending = true;
     {
-      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+      bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
@@ -592,13 +777,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- P9: (this chunk's outputs are stored during the next chunk's P4 products, or after the loop)
+    o_pending = true;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
   }
 
   if (!failed && nchunks > 0) {
-    if (q4 >= 2) store_o(nchunks - 1);
+    if (o_pending && q4 >= 2) store_o(nchunks - 1);
     // S_T = Diag(gamma_C / gamma_m) S_acc of the last chunk
     const int k = 32 * q4 + lane;
     const float lam = s_lam[(nchunks - 1) & 1][k];
