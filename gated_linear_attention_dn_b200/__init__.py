@@ -18,6 +18,7 @@ Entry points (same names as the C ABI):
     mc_fwd(q, k, v, ..., seg_len=L, gates=None) -> (o, M)   (segments + cached read-out)
     dn_stream_status(stream=None) -> int
     dn_status_string(code) -> str
+    dn_set_wait_limit_ns(ns)        (diagnostics: bound of the chunk kernels' mbarrier waits)
 
 Layouts: q, k [B,T,H,d_k]; v [B,T,H,d_v]; gates [B,T,H] (one per token),
 [B,T,H,n] (one per channel) or None (absent = 1); states [B,H,d_k,d_v] fp32.
@@ -34,7 +35,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdn.so")
 
 DN_OK, DN_ERR_INVALID_ARGUMENT, DN_ERR_UNSUPPORTED, DN_ERR_MISALIGNED = 0, 1, 2, 3
-DN_ERR_WORKSPACE_TOO_SMALL, DN_ERR_CUDA, DN_ERR_DEVICE_TIMEOUT = 4, 5, 6
+DN_ERR_WORKSPACE_TOO_SMALL, DN_ERR_CUDA, DN_ERR_DEVICE_TIMEOUT, DN_ERR_GATE_RANGE = 4, 5, 6, 7
+DEFAULT_WAIT_NS = 2_000_000_000
 DN_F32, DN_BF16 = 0, 1
 DN_GATE_ONE, DN_GATE_SCALAR, DN_GATE_CHANNEL = 0, 1, 2
 DN_READ_POST, DN_READ_PRE = 0, 1
@@ -42,7 +44,7 @@ _READOUT = {"post": DN_READ_POST, "pre": DN_READ_PRE}
 
 EXPORTED = ("dn_chunk_fwd_workspace_bytes", "dn_chunk_fwd", "dn_decode_step", "dn_chunk_bwd_workspace_bytes",
             "dn_chunk_bwd", "dn_osdn_precond_workspace_bytes", "dn_osdn_precond", "dn_osdn_precond_noalloc",
-            "dn_mc_readout", "dn_stream_status", "dn_status_string", "dn_version")
+            "dn_mc_readout", "dn_stream_status", "dn_status_string", "dn_version", "dn_set_wait_limit_ns")
 
 
 class DnDesc(ctypes.Structure):
@@ -103,12 +105,22 @@ def load(path: str = LIB_PATH):
     lib.dn_status_string.argtypes = [I]
     lib.dn_status_string.restype = ctypes.c_char_p
     lib.dn_version.restype = I
+    lib.dn_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    lib.dn_set_wait_limit_ns.restype = I
     _lib = lib
     return lib
 
 
 def dn_status_string(code: int) -> str:
     return load().dn_status_string(int(code)).decode()
+
+
+def dn_set_wait_limit_ns(ns: int) -> None:
+    """Bound of every mbarrier wait of the tensor-core chunk kernels for later launches (default
+    DEFAULT_WAIT_NS; 0 = one non-blocking probe per wait). A diagnostics hook for the timeout path."""
+    code = load().dn_set_wait_limit_ns(int(ns))
+    if code != DN_OK:
+        raise DnError(code, "dn_set_wait_limit_ns")
 
 
 def _ptr(t):

@@ -4,6 +4,9 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "dn_bwd.cuh"
 #include "dn_common.cuh"
 
@@ -15,10 +18,14 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {nullptr};
+std::mutex g_status_mu;  // guards the first lookup on each device
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
 
+// Device address of the status word on the current device, looked up once per device.
 dn_status status_ptr(int** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_status_mu);
   if (!g_status_ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dn_status) != cudaSuccess) return DN_ERR_CUDA;
@@ -95,6 +102,7 @@ dn_status fill_args(const dn_desc* d, const void* q, const void* k, const void* 
   a->beta_k_p = beta_k;
   a->beta_v_p = beta_v;
   a->key_scale_p = key_scale;
+  a->wait_ns = dn::wait_limit_ns();
   return DN_OK;
 }
 
@@ -106,9 +114,18 @@ bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 }  // namespace
 
+namespace dn {
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+}  // namespace dn
+
 extern "C" {
 
-int dn_version(void) { return 100; }
+int dn_version(void) { return 200; }
+
+dn_status dn_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_ns.store(ns, std::memory_order_relaxed);
+  return DN_OK;
+}
 
 const char* dn_status_string(dn_status s) {
   switch (s) {
@@ -119,6 +136,7 @@ const char* dn_status_string(dn_status s) {
     case DN_ERR_WORKSPACE_TOO_SMALL: return "DN_ERR_WORKSPACE_TOO_SMALL";
     case DN_ERR_CUDA: return "DN_ERR_CUDA";
     case DN_ERR_DEVICE_TIMEOUT: return "DN_ERR_DEVICE_TIMEOUT";
+    case DN_ERR_GATE_RANGE: return "DN_ERR_GATE_RANGE";
   }
   return "DN_ERR_UNKNOWN";
 }
@@ -150,6 +168,19 @@ dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const 
     if (ranges_overlap(o, n_o, q, n_qk) || ranges_overlap(o, n_o, k, n_qk) ||
         ranges_overlap(o, n_o, v, n_o) || ranges_overlap(o, n_o, S_T, n_S))
       return DN_ERR_INVALID_ARGUMENT;
+    // S_T is written while every input is still read
+    const size_t n_tok = (size_t)desc->B * desc->T * desc->H;
+    const void* ins[7] = {q, k, v, alpha, beta_k, beta_v, key_scale};
+    const size_t in_n[7] = {n_qk, n_qk, n_o, n_tok * 4 * (desc->alpha == DN_GATE_CHANNEL ? desc->d_k : 1),
+                            n_tok * 4 * (desc->beta_k == DN_GATE_CHANNEL ? desc->d_k : 1),
+                            n_tok * 4 * (desc->beta_v == DN_GATE_CHANNEL ? desc->d_v : 1),
+                            n_tok * 4 * (desc->key_scale == DN_GATE_CHANNEL ? desc->d_k : 1)};
+    for (int i = 0; i < 7; ++i)
+      if (ranges_overlap(S_T, n_S, ins[i], in_n[i])) return DN_ERR_INVALID_ARGUMENT;
+  }
+  {  // in place (S_T == S0) is supported; a partial overlap is not
+    const size_t n_S = (size_t)desc->B * desc->H * desc->d_k * desc->d_v * 4;
+    if (S0 && S0 != S_T && ranges_overlap(S0, n_S, S_T, n_S)) return DN_ERR_INVALID_ARGUMENT;
   }
   if ((st = status_ptr(&a.status)) != DN_OK) return st;
   a.S0 = S0;
@@ -182,6 +213,15 @@ dn_status dn_decode_step(const dn_desc* desc, const void* q, const void* k, cons
   if ((st = fill_args(desc, q, k, v, alpha, beta_k, beta_v, key_scale, &a)) != DN_OK) return st;
   if (!S || !o) return DN_ERR_INVALID_ARGUMENT;
   if (!aligned16(S) || !aligned16(o)) return DN_ERR_MISALIGNED;
+  {  // o is written while S, q, k and v are still read (by the other column slice of the same head)
+    const size_t es = desc->io_dtype == DN_BF16 ? 2 : 4;
+    const size_t nh = (size_t)desc->B * desc->H;
+    const size_t n_o = nh * desc->d_v * es, n_k = nh * desc->d_k * es;
+    const size_t n_S = nh * desc->d_k * desc->d_v * 4;
+    if (ranges_overlap(o, n_o, S, n_S) || ranges_overlap(o, n_o, q, n_k) || ranges_overlap(o, n_o, k, n_k) ||
+        ranges_overlap(o, n_o, v, n_o))
+      return DN_ERR_INVALID_ARGUMENT;
+  }
   if ((st = status_ptr(&a.status)) != DN_OK) return st;
   a.S0 = S;
   a.S = S;
@@ -344,6 +384,7 @@ dn_status dn_chunk_bwd(const dn_desc* desc, const void* q, const void* k, const 
     }
   }
   a.S0 = S0;
+  if ((st = status_ptr(&a.status)) != DN_OK) return st;
   cudaError_t e =
       small_dims(desc)
           ? dn::launch_small_bwd(a, dO, dS_T, dq, dk, dv, d_alpha, d_beta_k, d_beta_v, d_key_scale, dS0,
@@ -365,7 +406,7 @@ dn_status dn_stream_status(void* cuda_stream) {
   if (word != dn::kDevOk) {
     const int zero = 0;
     if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return DN_ERR_CUDA;
-    return DN_ERR_DEVICE_TIMEOUT;
+    return word == dn::kDevGateRange ? DN_ERR_GATE_RANGE : DN_ERR_DEVICE_TIMEOUT;
   }
   return DN_OK;
 }

@@ -57,6 +57,11 @@
  *     split); fp32 io runs an fp32 CUDA-core kernel. Small states (d_k, d_v in
  *     {8, 16}, e.g. the delta-mem page's 8 x 8 memory) run an fp32 CUDA-core
  *     kernel with one warp per head, for the chunked call and the decode step.
+ *   - Gates: alpha >= 0 (0 resets the state), finite. The forward and the decode
+ *     step hold for any such decay, however strong: per-token gates carry the
+ *     chunk's decay products as mantissa and exponent, and a chunk whose
+ *     per-channel decay over half a chunk falls below 2^-50 is evaluated exactly,
+ *     token by token, instead of through the tensor-core factorisation.
  */
 #ifndef DN_H_
 #define DN_H_
@@ -74,7 +79,9 @@ typedef enum {
   DN_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
   DN_ERR_WORKSPACE_TOO_SMALL = 4,
   DN_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
-  DN_ERR_DEVICE_TIMEOUT = 6      /* a kernel's bounded wait gave up (reported by dn_stream_status) */
+  DN_ERR_DEVICE_TIMEOUT = 6,     /* a kernel's bounded wait gave up (reported by dn_stream_status) */
+  DN_ERR_GATE_RANGE = 7          /* dn_chunk_bwd only: a chunk's decay is beyond what its factorisation
+                                    holds in fp32 (reported by dn_stream_status; see dn_chunk_bwd) */
 } dn_status;
 
 typedef enum { DN_F32 = 0, DN_BF16 = 1 } dn_dtype;
@@ -88,7 +95,7 @@ typedef enum { DN_GATE_ONE = 0, DN_GATE_SCALAR = 1, DN_GATE_CHANNEL = 2 } dn_gat
  * the delta-mem page (section 2.C, r_t = S_{t-1} q^m_t). delta-mem's update
  * S_t = lambda_t S_{t-1} + beta_t (v_t - S_{t-1} k_t) k_t^T (section 2.A; undecayed residual) is
  * this recurrence with alpha = lambda, beta^k = beta / lambda, beta^v = lambda (lambda > 0).
- * DN_READ_PRE needs alpha > 0 on the chunk path (it divides by the token's own decay).
+ * The forward takes either read-out for any alpha >= 0; dn_chunk_bwd needs alpha > 0.
  */
 typedef enum { DN_READ_POST = 0, DN_READ_PRE = 1 } dn_readout;
 
@@ -119,8 +126,10 @@ size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc);
  *
  * In:  q, k, v, gates as laid out above; S0 = initial state or NULL (zero).
  * Out: o [B,T,H,d_v] (io dtype), S_T [B,H,d_k,d_v] fp32 (final state).
- * S_T may alias S0 (in-place resume). q, k, v, o must not overlap each other or
- * S_T. `workspace` may be NULL when dn_chunk_fwd_workspace_bytes() is 0.
+ * S_T may alias S0 exactly (in-place resume); any other overlap of S_T with S0
+ * or with an input, and any overlap of o with q, k, v or S_T, is rejected with
+ * DN_ERR_INVALID_ARGUMENT. `workspace` may be NULL when
+ * dn_chunk_fwd_workspace_bytes() is 0.
  * T == 0 copies S0 (or zeros) into S_T and writes no o.
  */
 dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const void* v,
@@ -131,7 +140,8 @@ dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const 
 /*
  * One recurrent step (desc->T must be 1): S <- S_1, o <- S_1^T q, in place.
  * In:  q, k [B,1,H,d_k], v [B,1,H,d_v], gates for one token, S [B,H,d_k,d_v] fp32.
- * Out: S updated in place, o [B,1,H,d_v] (io dtype).
+ * Out: S updated in place, o [B,1,H,d_v] (io dtype); o must not overlap S, q, k
+ * or v (DN_ERR_INVALID_ARGUMENT).
  * Each (b, h) state is read once and written once (HBM-streaming kernel).
  */
 dn_status dn_decode_step(const dn_desc* desc, const void* q, const void* k, const void* v,
@@ -251,7 +261,10 @@ dn_status dn_mc_readout(const dn_mc_desc* desc, const void* q, const float* M, c
  * state and its adjoint (d_k x d_v each), and the residuals and their adjoints (64 x d_v each).
  * Supported: both read-outs (desc->readout as given to the forward); d_k, d_v in {64, 128}
  * (chunked kernels) or both in {8, 16} (small states: one warp per head, sequential, the state
- * entering every token kept in the workspace); alpha > 0. dq, dk, dv must not overlap each other, q, k, v,
+ * entering every token kept in the workspace); alpha > 0. The chunked kernels reference each chunk's
+ * decay to a point inside it, in fp32: a chunk where the decay between that point and any of its
+ * tokens exceeds e^80 per channel (mean log alpha below about -2.5 per token) sets
+ * DN_ERR_GATE_RANGE for dn_stream_status and its gradients are not valid. dq, dk, dv must not overlap each other, q, k, v,
  * dO, S0 or the workspace. fp32 arithmetic throughout. T == 0 writes dS0 = dS_T (or
  * zeros). Asynchronous on the stream.
  */
@@ -266,10 +279,23 @@ dn_status dn_chunk_bwd(const dn_desc* desc, const void* q, const void* k, const 
 
 /*
  * Synchronises `cuda_stream`, then reports (and clears) the device status word
- * that kernels set when a bounded wait gives up (DN_ERR_DEVICE_TIMEOUT), or
+ * that kernels set when a bounded wait gives up (DN_ERR_DEVICE_TIMEOUT) or when
+ * dn_chunk_bwd meets a chunk beyond its range (DN_ERR_GATE_RANGE), or
  * DN_ERR_CUDA if the stream holds a CUDA error. DN_OK otherwise.
+ * The status word's device address is looked up on the first call of any entry
+ * point on each device: make that first call before any stream capture.
  */
 dn_status dn_stream_status(void* cuda_stream);
+
+/*
+ * Diagnostics: the bound of every mbarrier wait in the tensor-core chunk kernels
+ * (default 2 s, far above any legitimate wait). A wait that runs out makes the
+ * kernel leave its loop, drain what it issued (those waits keep the 2 s bound),
+ * free its tensor memory and set DN_ERR_DEVICE_TIMEOUT for dn_stream_status;
+ * 0 makes each wait a single non-blocking probe, so a test can take that path
+ * on purpose. Applies to launches made after the call, process-wide.
+ */
+dn_status dn_set_wait_limit_ns(unsigned long long ns);
 
 /* Static, human-readable name of a status code. Never NULL. */
 const char* dn_status_string(dn_status status);

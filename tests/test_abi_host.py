@@ -234,3 +234,38 @@ def test_binding_bwd_checks_arguments_before_the_library(lib):
         dn.dn_chunk_bwd(q, q, v, a, a, dO=v, out={"q": q, "k": q, "v": v, "alpha": None, "beta_k": a})
     with pytest.raises(TypeError):
         dn.dn_chunk_bwd(q, q.float(), v, a, a, dO=v)
+
+
+def test_decode_rejects_o_overlapping_its_inputs(lib):
+    # o is written by one column slice of a head while the other slice still reads S, q, k, v
+    d = _desc(T=1, alpha=dn.DN_GATE_CHANNEL, beta_k=dn.DN_GATE_CHANNEL)
+    bufs = {n: _Buf(1 << 16) for n in ("q", "k", "v", "a", "bk", "S", "o")}
+
+    def call(**over):
+        p = {n: b.p() for n, b in bufs.items()}
+        p.update(over)
+        return lib.dn_decode_step(ctypes.byref(d), p["q"], p["k"], p["v"], p["a"], p["bk"], None, None, p["S"],
+                                  p["o"], None)
+
+    for name in ("S", "q", "k", "v"):
+        assert call(o=bufs[name].p(32)) == dn.DN_ERR_INVALID_ARGUMENT, name
+
+
+def test_chunk_fwd_rejects_state_overlaps(lib):
+    s = _Buf(1 << 17)
+    nS = 1 * 2 * 64 * 64 * 4
+    # S0 partly overlapping S_T (exact aliasing, S_T == S0, is the supported in-place form)
+    assert _call(lib, _desc(), s0=s.p(0), st=s.p(nS // 2)) == dn.DN_ERR_INVALID_ARGUMENT
+    assert _call(lib, _desc(), s0=s.p(0), st=s.p(0)) != dn.DN_ERR_INVALID_ARGUMENT
+    # S_T overlapping an input it is written while reading
+    q = _Buf(1 << 17)
+    assert _call(lib, _desc(), q=q.p(), st=q.p(64)) == dn.DN_ERR_INVALID_ARGUMENT
+    a = _Buf(1 << 17)
+    assert _call(lib, _desc(), a=a.p(), st=a.p(16)) == dn.DN_ERR_INVALID_ARGUMENT
+
+
+def test_gate_range_status_and_wait_hook(lib):
+    assert dn.dn_status_string(dn.DN_ERR_GATE_RANGE) == "DN_ERR_GATE_RANGE"
+    # the diagnostics hook only records the bound; put the default back
+    dn.dn_set_wait_limit_ns(0)
+    dn.dn_set_wait_limit_ns(dn.DEFAULT_WAIT_NS)
