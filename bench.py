@@ -55,6 +55,19 @@ def algorithmic_bytes(w: di.Workload) -> int:
     return b
 
 
+def chunk_flops(w: di.Workload, C: int = 64) -> int:
+    """Executed flops of one dn_chunk_fwd in chunk form (2 per multiply-add), per head-token:
+    2 C (3 d_k + 2 d_v) for the Gram, scores and WY products, 6 d_k d_v for the three state products
+    (Wk S, Q S, W^T U) and C^2 / 3 for the triangular inverse."""
+    return w.B * w.T * w.H * (2 * C * (3 * w.dk + 2 * w.dv) + 6 * w.dk * w.dv + C * C // 3)
+
+
+def seq_flops(w: di.Workload) -> int:
+    """Flops of the sequential evaluation (fp32 io): per head-token the decay, the two reductions S^T k and
+    S^T q and the rank-1 update, 2 flops each over d_k d_v."""
+    return w.B * w.T * w.H * 8 * w.dk * w.dv
+
+
 def decode_bytes(w: di.Workload) -> int:
     """HBM bytes of one decode step: S read + written once, plus the token's vectors and o."""
     nh = w.B * w.H
@@ -111,6 +124,7 @@ def measured_peaks() -> dict:
 # sources each timed kernel is built from (its recorded DRAM traffic is void once any changes)
 KERNEL_SOURCES = {
     "chunk_fwd": ["dn_chunk_sc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
+    "chunk_tc": ["dn_chunk_tc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
     "decode": ["dn_decode.cu", "dn_common.cuh"],
     "osdn": ["dn_osdn.cu", "dn_tc_ptx.cuh", "dn_common.cuh"],
     "chunk_bwd": ["dn_bwd.cu", "dn_bwd.cuh", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_common.cuh"],
@@ -270,7 +284,8 @@ def run_single_kernel(args):
 
     if not os.path.exists(dnbuild.LIB):
         dnbuild.build()
-    name = {"chunk": WORKLOAD, "decode": DECODE, "osdn": "osdn_phase1", "bwd": WORKLOAD}[args.only]
+    name = {"chunk": WORKLOAD, "decode": DECODE, "osdn": "osdn_phase1", "bwd": WORKLOAD, "kda": "kda",
+            "fg2": "fg2_osdn_long"}[args.only]
     w = di.WORKLOADS[name]
     if args.batch:
         w = w.scaled(B=args.batch)
@@ -298,7 +313,7 @@ def run_single_kernel(args):
                             xd["S0"], dO=gb["dO"], dS_T=gb["dS_T"], workspace=wsb, out=gout)
         elif args.only == "osdn":
             dn.dn_osdn_precond(xd["k"], xd["beta"], xd["retention"], None, eta=eta)
-        elif args.only == "chunk":
+        elif args.only in ("chunk", "kda", "fg2"):
             dn.dn_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
                             xd["S0"])
         else:
@@ -320,6 +335,84 @@ def run_single_kernel(args):
                       "ms_per_launch": e0.elapsed_time(e1) / max(1, args.steps)}))
 
 
+CONFIG_LEGS = {
+    "gdn_fp32_small": "B=1 H=2 T=256 d_k=d_v=64 fp32 q/k/v, alpha~U(0.9,1) and beta per token, S0=0 "
+                      "(sequential fp32 kernel)",
+    "kda": "B=4 H=32 T=8192 d_k=d_v=128 bf16 q/k/v, channel alpha, beta per token, S0~N(0,0.02^2)",
+    "fg2_osdn_long": "B=2 H=16 T=32768 d_k=d_v=128 bf16 q/k/v, channel alpha, beta^k, beta^v, OSDN d, "
+                     "S0~N(0,0.02^2)",
+}
+
+
+def run_config_leg(name, peaks, stream, world, barrier, to_dev, want_cpu, reps):
+    """One dn_chunk_fwd workload of the pages' configurations: ms per call, tokens/s, the HBM and tensor
+    roofline fractions, and (rank 0, one GPU) the fp64 oracle on whole heads of the same workload."""
+    import torch
+
+    import gated_linear_attention_dn_b200 as dn
+    w = di.WORKLOADS[name]
+    x = di.make_inputs(w)
+    xd = {n: to_dev(a) for n, a in x.items()}
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=xd["q"].dtype, device="cuda")
+    ST = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    alg = algorithmic_bytes(w)
+    # inputs smaller than L2 are timed one launch at a time with an L2 flush in between
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if alg < 2 * L2_BYTES else None
+
+    def step():
+        dn.dn_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                        xd["S0"], o=o, S_T=ST, stream=stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    barrier()
+    for e0, e1 in evs:
+        if flush is not None:
+            flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if dn.dn_stream_status(stream) != dn.DN_OK:
+        raise RuntimeError(f"device status after the {name} leg")
+    ms = reduce_max(statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs), world)
+    gbs = alg / (ms * 1e-3) / 1e9
+    leg = {"workload": f"{name}: {CONFIG_LEGS[name]}", "ms_per_call": ms,
+           "tokens_per_s": weak_scaling_rate(w.B * w.T, world, ms),
+           "l2": "flushed (2 x L2 written) before every timed launch" if flush is not None
+                 else f"inputs {alg / 1e6:.0f} MB per call > L2 (no flush)",
+           "hbm": {"achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                   "algorithmic_bytes_per_launch": alg}}
+    if w.io == "bf16":
+        fl = chunk_flops(w)
+        tf = fl / (ms * 1e-3) / 1e12
+        leg["tensor"] = {"achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / peaks["bf16_tflops"], "executed_flops_per_launch": fl,
+                         "peak_source": f"{peaks['source']} bf16 burst"}
+        leg["roofline_time_us"] = 1e6 * max(alg / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+        leg["traffic"] = recorded_traffic("chunk_tc")
+    else:
+        fl = seq_flops(w)
+        tf = fl / (ms * 1e-3) / 1e12
+        fp32_peak = 148 * 4 * 32 * 2 * 1.965e9 / 1e12
+        leg["alu"] = {"achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s", "frac": tf / fp32_peak,
+                      "flops_per_launch": fl, "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flops x 1.965 GHz",
+                      "note": "a sequential chain of T tokens per head: launch and latency bound at this size"}
+    if want_cpu:
+        import oracle
+        oracle.build()
+        nthreads = oracle.max_threads()
+        head_tokens, secs, nheads = oracle_sample(w, x, budget_s=4.0, nthreads=nthreads)
+        leg["cpu_baseline"] = {"value": head_tokens / secs / w.H, "unit": "tokens/s", "cores": nthreads,
+                               "kind": "oracle",
+                               "sample": f"{nheads} of {w.B * w.H} heads, whole T={w.T} each ({secs:.1f} s); "
+                                         "tokens/s = head-tokens/s / H"}
+    del xd, o, ST, flush
+    return leg
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -331,8 +424,10 @@ def main():
     ap.add_argument("--no-osdn", action="store_true", help="skip the OSDN preconditioner scan leg")
     ap.add_argument("--no-mc", action="store_true", help="skip the Memory Caching leg")
     ap.add_argument("--no-bwd", action="store_true", help="skip the chunked backward leg")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the gdn_fp32_small, kda and fg2_osdn_long workload legs")
     ap.add_argument("--decode-steps", type=int, default=100)
-    ap.add_argument("--only", choices=["chunk", "decode", "osdn", "bwd"], default=None,
+    ap.add_argument("--only", choices=["chunk", "decode", "osdn", "bwd", "kda", "fg2"], default=None,
                     help="profiling mode: run just one kernel on the workload with batch --batch")
     ap.add_argument("--batch", type=int, default=0, help="with --only: batch size of the scaled workload")
     args = ap.parse_args()
@@ -418,10 +513,15 @@ def main():
     kern_ms = statistics.mean(per_launch_ms)
     alg = algorithmic_bytes(w)
     achieved = alg / (kern_ms * 1e-3) / 1e9
+    fl = chunk_flops(w)
+    tf = fl / (kern_ms * 1e-3) / 1e12
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": recorded_traffic("chunk_fwd"),
                 "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg,
-                "kernel_ms": kern_ms}
+                "kernel_ms": kern_ms,
+                "tensor": {"achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                           "frac": tf / peaks["bf16_tflops"], "executed_flops_per_launch": fl},
+                "roofline_time_us": 1e6 * max(alg / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))}
 
     # ---- end to end: pinned host buffers, H2D of the step's inputs, D2H of o and S_T
     pin = {n: (None if t is None else t.cpu().pin_memory()) for n, t in xd.items()}
@@ -549,6 +649,16 @@ def main():
         launches += 2 * 10 + 3  # timed: 10 scans of two kernels, 3 chunked passes
         del ko, bo, ro, do, dTo, wso, xf, Sf, of
 
+    # ---- the pages' other configurations, one dn_chunk_fwd workload each
+    configs = None
+    if not args.no_configs:
+        configs = {}
+        for name, reps in (("gdn_fp32_small", 20), ("kda", 10), ("fg2_osdn_long", 5)):
+            configs[name] = run_config_leg(name, peaks, stream, world, barrier, to_dev,
+                                           want_cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline),
+                                           reps=reps)
+            launches += reps
+
     # ---- Memory Caching on the prefill workload: 4 segments of 1024 tokens, residual memory
     mc = None
     if not args.no_mc:
@@ -660,7 +770,7 @@ def main():
             "config": bench_config(world),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clocks.summary(), "gpu_launches": launches, "decode": decode, "osdn_phase1": osdn,
-            "memory_caching": mc, "chunk_bwd": bwd,
+            "memory_caching": mc, "chunk_bwd": bwd, "configs": configs,
             "kernel_source": {k: kernel_source_hash(k) for k in KERNEL_SOURCES},
         }
         print(json.dumps(line), flush=True)
