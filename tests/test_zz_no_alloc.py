@@ -19,6 +19,7 @@ import torch
 import dn_inputs as di
 import gated_linear_attention_dn_b200 as dn
 
+
 def _lib():
     lib = dn.load()
     O = ctypes.POINTER(dn.DnOsdnDesc)
