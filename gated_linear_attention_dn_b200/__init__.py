@@ -178,7 +178,10 @@ def dn_chunk_fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, 
                  S_T=None, stream=None, chunk: int = 0, workspace=None, readout: str = "post"):
     """Chunked prefill. Returns (o [B,T,H,d_v] io dtype, S_T [B,H,d_k,d_v] fp32).
 
-    readout="post": o_t = S_t^T q_t; "pre": o_t = S_{t-1}^T q_t (before the token's update)."""
+    readout="post": o_t = S_t^T q_t; "pre": o_t = S_{t-1}^T q_t (before the token's update).
+    workspace: None allocates the dn_chunk_fwd_workspace_bytes() the problem can use (the split
+    transform + state-chain evaluation); False passes none (the fused one-kernel evaluation); a
+    uint8 CUDA tensor is used as given."""
     lib = load()
     _check_io(q, k, v)
     desc = make_desc(q, v, alpha, beta_k, beta_v, key_scale, chunk, readout)
@@ -189,11 +192,13 @@ def dn_chunk_fwd(q, k, v, alpha=None, beta_k=None, beta_v=None, key_scale=None, 
     if S_T is None:
         S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     ws_bytes = dn_chunk_fwd_workspace_bytes(desc)
-    if ws_bytes and workspace is None:
+    if workspace is False:
+        workspace = None
+    elif ws_bytes and workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     rc = lib.dn_chunk_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k),
                           _ptr(beta_v), _ptr(key_scale), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(workspace),
-                          ws_bytes if workspace is not None else 0, _stream_handle(stream))
+                          workspace.numel() if workspace is not None else 0, _stream_handle(stream))
     if rc != DN_OK:
         raise DnError(rc, "dn_chunk_fwd")
     return o, S_T

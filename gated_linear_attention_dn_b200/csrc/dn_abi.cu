@@ -142,16 +142,20 @@ const char* dn_status_string(dn_status s) {
 }
 
 size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc) {
-  (void)desc;
-  return 0;
+  if (check_desc(desc, false) != DN_OK) return 0;
+  dn::Args a;
+  memset(&a, 0, sizeof(a));
+  a.B = desc->B, a.T = desc->T, a.H = desc->H, a.dk = desc->d_k, a.dv = desc->d_v;
+  a.chunk = desc->chunk == 0 ? 64 : desc->chunk;
+  a.io_bf16 = desc->io_dtype == DN_BF16;
+  a.alpha = desc->alpha, a.beta_k = desc->beta_k, a.beta_v = desc->beta_v, a.key_scale = desc->key_scale;
+  return dn::per_token_tc(a) ? dn::split_sc_workspace_bytes(a) : 0;
 }
 
 dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const void* v,
                        const float* alpha, const float* beta_k, const float* beta_v,
                        const float* key_scale, const float* S0, void* o, float* S_T,
                        void* workspace, size_t workspace_bytes, void* cuda_stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   dn_status st = check_desc(desc, false);
   if (st != DN_OK) return st;
   dn::Args a;
@@ -177,6 +181,19 @@ dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const 
                             n_tok * 4 * (desc->key_scale == DN_GATE_CHANNEL ? desc->d_k : 1)};
     for (int i = 0; i < 7; ++i)
       if (ranges_overlap(S_T, n_S, ins[i], in_n[i])) return DN_ERR_INVALID_ARGUMENT;
+    // a workspace is read and written while every input and output is live
+    if (workspace) {
+      const size_t need = dn_chunk_fwd_workspace_bytes(desc);
+      if (need > 0) {
+        if (workspace_bytes < need) return DN_ERR_WORKSPACE_TOO_SMALL;
+        if (!aligned16(workspace)) return DN_ERR_MISALIGNED;
+        for (int i = 0; i < 7; ++i)
+          if (ranges_overlap(workspace, need, ins[i], in_n[i])) return DN_ERR_INVALID_ARGUMENT;
+        if (ranges_overlap(workspace, need, o, n_o) || ranges_overlap(workspace, need, S_T, n_S) ||
+            ranges_overlap(workspace, need, S0, S0 ? n_S : 0))
+          return DN_ERR_INVALID_ARGUMENT;
+      }
+    }
   }
   {  // in place (S_T == S0) is supported; a partial overlap is not
     const size_t n_S = (size_t)desc->B * desc->H * desc->d_k * desc->d_v * 4;
@@ -196,6 +213,8 @@ dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const 
   cudaError_t e;
   if (dn::small_state_supported(a)) {
     e = dn::launch_small_state(a, s);
+  } else if (workspace && dn::per_token_tc(a)) {
+    e = dn::launch_split_sc(a, workspace, s);
   } else if (a.io_bf16 && dn::chunk_tc_supported(a)) {
     e = dn::launch_chunk_tc(a, s);
   } else {

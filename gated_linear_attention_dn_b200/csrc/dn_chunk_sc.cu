@@ -48,6 +48,7 @@
 // Every mbarrier wait is bounded in time; on expiry both groups leave their loops, the state group
 // drains what it issued (bounded), the CTA sets the status word and frees its tensor memory.
 #include "dn_common.cuh"
+#include "dn_sc_factors.cuh"
 #include "dn_tc_ptx.cuh"
 #include "dn_ut_inverse.cuh"
 
@@ -101,14 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bar_qk[2], bar_k, bar_v, bar_mma, bar_gram, bar_tready, bar_drain;
   __shared__ uint32_t s_tmem;
   __shared__ __align__(16) float s_Y[2048];  // inverse scratch
-  // per-token factors by chunk index mod 4 (gamma_t = rho_t 2^{e_t}, gamma_C / gamma_t = mu_t 2^{n_t}):
-  // rho_t, 1 / rho_t, e_t; the read-out's o scale and Q' exponent (those of gamma_t, or of
-  // gamma_{t-1} before the update); 1 / (rho_t mu_t); c_t = beta^k_t d_t mu_t; n_t; beta^k d;
-  // beta^v; gamma_t as a float; and gamma_C per chunk
-  __shared__ float s_rho[4][C], s_rhoi[4][C], s_orho[4][C], s_pinv[4][C], s_c[4][C], s_ws[4][C], s_bv[4][C],
-      s_gam[4][C];
-  __shared__ int s_ex[4][C], s_oex[4][C], s_n[4][C];
-  __shared__ float s_glast[4];
+  // per-token factors by chunk index mod 4 (dn_sc_factors.cuh)
+  __shared__ scf::Factors s_f[4];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int q4 = warp & 3;  // TMEM lane quadrant this warp may access
@@ -279,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (fp32, where the state update accumulates); rows 32 q4 .. +32, columns of half ch
       {
         const int k = 32 * q4 + lane;
-        const float gl = s_glast[cur];
+        const float gl = s_f[cur].glast;
         uint32_t xr[NCB][32];  // all TMEM loads of this thread in flight at once
         if (c == 0) {
 #pragma unroll
@@ -336,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // transform arrived on tready)
       if (q4 >= 2) {
         const int t = 32 * (q4 - 2) + lane;
-        const float sc = pow2f(s_oex[cur][t]);
+        const float sc = pow2f(s_f[cur].oex[t]);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           uint4* p = reinterpret_cast<uint4*>(kq + canon_chunk(64 + t, 8 * ch + j, 128));
@@ -405,13 +400,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int it = 0; it < 8; ++it) {
             const int e = u + 128 * it, i = e >> 4;
             uint4* p = reinterpret_cast<uint4*>(sm + Ly::STK + canon_chunk(i, e & 15, C));
-            *p = scale_bf16x8(*p, pow2f(s_n[cur][i]));
+            *p = scale_bf16x8(*p, pow2f(s_f[cur].n[i]));
           }
         }
       }
       if (q4 < 2) {
         const int t = 32 * q4 + lane;
-        const float us = s_c[cur][t];
+        const float us = s_f[cur].c[t];
 #pragma unroll
         for (int cb = 0; cb < NV / 64; ++cb) {
           const int col = ch * (NV / 2) + 32 * cb;
@@ -486,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // TMEM load is warp-collective: every lane loads, only rows of real tokens store
       if (q4 >= 2) {
         const int t = 32 * (q4 - 2) + lane, nc = min(C, T - t0);
-        const float os = s_orho[cur][t];  // mantissa of gamma_t (of gamma_{t-1} before the update)
+        const float os = s_f[cur].orho[t];  // mantissa of gamma_t (of gamma_{t-1} before the update)
         __nv_bfloat16* orow =
             reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0 + t) * H + h) * dv + col0;
         uint32_t xr[NCB][32];
@@ -543,83 +538,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ======================================================= transform group
     const int gt = tid - kStateThreads, gw = gt >> 5, gch = gw >> 2;  // q4 == gw & 3
     uint32_t ph_gr = 0;
-    // Thread j < 64 (warps 8, 9) loads token j's gates (alpha, beta^k, d, beta^v) of chunk cn, and
-    // the alpha of token j ^ 32, into registers one chunk ahead of their use; absent gates read as 1,
-    // tokens past the end as alpha 1 and 0 for the others (no decay, no write).
-    float gx[5];
-    auto load_gates = [&](int cn, int j) {
-      const int left = T - cn * C;
-      const bool valid = j < left, valid_p = (j ^ 32) < left;
-      const int64_t tok = ((int64_t)b * T + cn * C + j) * H + h;
-      const int64_t tok_p = ((int64_t)b * T + cn * C + (j ^ 32)) * H + h;
-      gx[0] = (valid && a.alpha == DN_GATE_SCALAR) ? __ldg(a.alpha_p + tok) : 1.f;
-      gx[1] = (valid && a.beta_k == DN_GATE_SCALAR) ? __ldg(a.beta_k_p + tok) : (valid ? 1.f : 0.f);
-      gx[2] = (valid && a.key_scale == DN_GATE_SCALAR) ? __ldg(a.key_scale_p + tok) : 1.f;
-      gx[3] = (valid && a.beta_v == DN_GATE_SCALAR) ? __ldg(a.beta_v_p + tok) : (valid ? 1.f : 0.f);
-      gx[4] = (valid_p && a.alpha == DN_GATE_SCALAR) ? __ldg(a.alpha_p + tok_p) : 1.f;
-    };
-    // Decay factors of chunk cn from the gates in gx (then the next chunk's are loaded). Each of
-    // warps 8 and 9 scans both halves of the chunk (lane l holds tokens l and 32 + l), so neither
-    // waits for the other: inclusive prefix products in mantissa-exponent form give gamma_t, the
-    // previous token's gamma_{t-1} and gamma_C.
-    auto token_prep = [&](int cn, int j) {
-      const int slot = cn & 3;
-      const float ws = gx[1] * gx[2], bv = gx[3];
-      const bool hi = j >= 32;
-      float m1, m2;
-      int e1, e2;
-      split_pow2(hi ? gx[4] : gx[0], m1, e1);  // token lane
-      split_pow2(hi ? gx[0] : gx[4], m2, e2);  // token 32 + lane
-      if (cn + 1 < nchunks) load_gates(cn + 1, j);
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y1 = __shfl_up_sync(0xffffffffu, m1, off), y2 = __shfl_up_sync(0xffffffffu, m2, off);
-        const int f1 = __shfl_up_sync(0xffffffffu, e1, off), f2 = __shfl_up_sync(0xffffffffu, e2, off);
-        if (lane >= off) {
-          mul_pow2(m1, e1, y1, f1);
-          mul_pow2(m2, e2, y2, f2);
-        }
-      }
-      const float t1m = __shfl_sync(0xffffffffu, m1, 31), t2m = __shfl_sync(0xffffffffu, m2, 31);
-      const int t1e = __shfl_sync(0xffffffffu, e1, 31), t2e = __shfl_sync(0xffffffffu, e2, 31);
-      float p1m = __shfl_up_sync(0xffffffffu, m1, 1), p2m = __shfl_up_sync(0xffffffffu, m2, 1);
-      int p1e = __shfl_up_sync(0xffffffffu, e1, 1), p2e = __shfl_up_sync(0xffffffffu, e2, 1);
-      float gm, pm;  // gamma_j and gamma_{j-1}
-      int ge, pe;
-      if (!hi) {
-        gm = m1, ge = e1;
-        if (lane == 0) p1m = 0.5f, p1e = 1;  // gamma_{-1} = 1
-        pm = p1m, pe = p1e;
-      } else {
-        gm = t1m, ge = t1e;
-        mul_pow2(gm, ge, m2, e2);
-        pm = t1m, pe = t1e;
-        if (lane > 0) mul_pow2(pm, pe, p2m, p2e);
-      }
-      float lm = t1m;  // gamma_C
-      int le = t1e;
-      mul_pow2(lm, le, t2m, t2e);
-      float mu = __fdividef(lm, gm);  // gamma_C / gamma_j = mu 2^ne, mu in [0.5, 1)
-      int ne = le - ge;
-      if (mu >= 1.f) mu *= 0.5f, ne += 1;
-      s_rho[slot][j] = gm;
-      s_rhoi[slot][j] = __fdividef(1.f, gm);
-      s_ex[slot][j] = ge;
-      s_orho[slot][j] = pre ? pm : gm;
-      s_oex[slot][j] = pre ? pe : ge;
-      s_pinv[slot][j] = __fdividef(1.f, gm * mu);
-      s_c[slot][j] = ws * mu;
-      s_n[slot][j] = ne;
-      s_gam[slot][j] = gm * pow2f(ge);
-      s_ws[slot][j] = ws;
-      s_bv[slot][j] = bv;
-      if (j == 63) s_glast[slot] = lm * pow2f(le);
-    };
-    if (gt < 64 && nchunks > 0) load_gates(0, gt);
+    // Thread j < 64 (warps 8, 9) holds token j's gates of the next chunk in registers, loaded one
+    // chunk ahead of their use.
+    scf::Gates gx;
+    if (gt < 64 && nchunks > 0) gx = scf::load_gates(a, b, h, 0, gt);
 
     for (int n = 0; n < nchunks; ++n) {
       const int cur = n & 3;
-      if (gt < 64) token_prep(n, gt);
+      if (gt < 64) {
+        const scf::Gates g = gx;
+        if (n + 1 < nchunks) gx = scf::load_gates(a, b, h, n + 1, gt);
+        scf::token_factors(g, gt, lane, pre, s_f[cur]);
+      }
       // ---- X1: the Gram of chunk n has completed, and with it chunk n - 1's Wk / U0 products
       {
         const bool ok = mbar_wait_bounded(&bar_gram, ph_gr, a.wait_ns);
@@ -634,49 +564,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // bf16 P' tile of parity n & 1 (last read by chunk n - 2's O product, long complete)
       float* sL = reinterpret_cast<float*>(sm + Ly::INV);
       float* sT = sL + C * C;
-      if (q4 < 2) {
-        const int t = 32 * q4 + lane;
-        const float rt = s_rho[cur][t];
-        const int et = s_ex[cur][t];
-        float x[32];
-        tmem_ld32(tmem + lane_base + Ly::TM_GR + 32 * gch, x);
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          float y[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 32 * gch + 4 * e4 + e;
-            const float f = s_ws[cur][i] * (rt * s_rhoi[cur][i]) * pow2f(et - s_ex[cur][i]);  // (gamma_t / gamma_i) beta_i d_i
-            y[e] = (i < t) ? x[4 * e4 + e] * f : 0.f;
-          }
-          *reinterpret_cast<float4*>(sL + xi(t, 32 * gch + 4 * e4)) = make_float4(y[0], y[1], y[2], y[3]);
-        }
-      } else {
-        const int t = 32 * (q4 - 2) + lane;
-        const int et = s_oex[cur][t];
-        uint8_t* pt = sm + Ly::TP + (1 + (n & 1)) * (C * C * 2);
-        float x[32];
-        tmem_ld32(tmem + lane_base + Ly::TM_GR + 32 * gch, x);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          float y[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = 32 * gch + 8 * q8 + e;
-            const float f = s_pinv[cur][i] * pow2f(et - s_ex[cur][i]);  // 2^{e_t - e_i} / (rho_i mu_i)
-            y[e] = (i <= t - pre) ? x[8 * q8 + e] * f : 0.f;
-          }
-          *reinterpret_cast<uint4*>(pt + canon_chunk(t, 4 * gch + q8, 64)) =
-              make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]), pack_bf16(y[6], y[7]));
-        }
-      }
+      scf::extract_ap(s_f[cur], tmem + Ly::TM_GR, q4, gch, lane, pre, sL, sm + Ly::TP + (1 + (n & 1)) * (C * C * 2));
       tc_fence_before();
       // ---- X3: T = (I + A)^{-1} -> T Diag(gamma) (TP rows 0..63) and T Diag(beta^v) (STQ rows 0..63)
       if (bv_split)
-        unit_lower_inverse<true, 8, false, true>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_gam[cur], s_bv[cur], gt,
-                                                 kBarXform);
+        unit_lower_inverse<true, 8, false, true>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_f[cur].gam, s_f[cur].bv,
+                                                 gt, kBarXform);
       else
-        unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_gam[cur], s_bv[cur], gt,
+        unit_lower_inverse<true, 8, false>(sL, sT, s_Y, sm + Ly::TP, sm + Ly::STQ, s_f[cur].gam, s_f[cur].bv, gt,
                                            kBarXform);
       fence_proxy_async();
       group_sync(kBarXform, kXformThreads);

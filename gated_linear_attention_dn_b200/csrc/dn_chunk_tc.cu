@@ -835,6 +835,11 @@ bool chunk_tc_supported(const Args& a) {
   return a.io_bf16 && a.dk == 128 && (a.dv == 128 || a.dv == 64) && a.chunk == C && a.T > 0;
 }
 
+bool per_token_tc(const Args& a) {
+  return chunk_tc_supported(a) && a.alpha != DN_GATE_CHANNEL && a.beta_k != DN_GATE_CHANNEL &&
+         a.beta_v != DN_GATE_CHANNEL && a.key_scale != DN_GATE_CHANNEL;
+}
+
 cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s) {
   // per-token gates only -> the pipelined raw-tile kernel (dn_chunk_sc.cu)
   const bool sc = a.alpha != DN_GATE_CHANNEL && a.beta_k != DN_GATE_CHANNEL && a.beta_v != DN_GATE_CHANNEL &&

@@ -44,6 +44,11 @@ cudaError_t launch_seq_fwd(const Args& a, cudaStream_t s);
 cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s);
 // per-token gates only (called by launch_chunk_tc)
 cudaError_t launch_chunk_sc(const Args& a, cudaStream_t s);
+// Whether a problem takes the per-token-gate tensor-core kernels (bf16, d_k = 128, every gate absent or
+// one per token), and the split evaluation of it with a workspace (dn_split_sc.cu): its bytes and launch.
+bool per_token_tc(const Args& a);
+size_t split_sc_workspace_bytes(const Args& a);
+cudaError_t launch_split_sc(const Args& a, void* workspace, cudaStream_t s);
 // OSDN phase 1 (dn_osdn.cu): workspace bytes, and the launch of its two kernels.
 size_t osdn_workspace_bytes(int B, int T, int H);
 cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, const float* d0, float eta, int B,

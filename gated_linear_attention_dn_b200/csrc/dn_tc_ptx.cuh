@@ -60,6 +60,30 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread for up to `hint_ns` while the phase is incomplete.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for threads off the critical path: the thread may sleep between polls, leaving the
+// issue slots of its SM sub-partition to the warps that work.
+__device__ __forceinline__ bool mbar_wait_bounded_idle(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (limit_ns == 0) return mbar_test_wait(bar, parity);
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, 4000u)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // Bounded wait: gives up once `limit_ns` of wall-clock time has passed (each
 // try_wait poll may itself suspend the thread for a while, so the bound is on
 // time, not on polls), returning false so the caller can bail out cleanly.

@@ -112,10 +112,18 @@ typedef struct {
 } dn_desc;
 
 /*
- * Bytes of workspace dn_chunk_fwd needs for this descriptor. The current
- * kernels keep every intermediate on chip and need none (returns 0); the
- * argument is kept so a future path (e.g. a segment-parallel state scan) can
- * ask for scratch without an ABI change. Returns 0 for an invalid descriptor.
+ * Bytes of workspace dn_chunk_fwd can use for this descriptor (0 for an invalid
+ * descriptor, and for problems that have no use for one).
+ *
+ * Problems on the per-token-gate tensor-core path (bf16 io, d_k = 128, d_v in
+ * {64, 128}, every gate absent or one per token: GDN) have two evaluations:
+ *  - with a workspace of at least this size: a chunk-parallel transform kernel
+ *    (decay factors, Gram product, UT inverse of every chunk at once) writes
+ *    ~25 KB per (b, h, chunk of 64 tokens) -- 33 KB when beta^v is given -- and a
+ *    state-chain kernel reads it back; the faster form;
+ *  - with workspace == NULL: one fused kernel per (b, h) that keeps everything on
+ *    chip, at some cost in speed.
+ * Both give the same results up to rounding. Other problems take no workspace.
  */
 size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc);
 
@@ -128,8 +136,12 @@ size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc);
  * Out: o [B,T,H,d_v] (io dtype), S_T [B,H,d_k,d_v] fp32 (final state).
  * S_T may alias S0 exactly (in-place resume); any other overlap of S_T with S0
  * or with an input, and any overlap of o with q, k, v or S_T, is rejected with
- * DN_ERR_INVALID_ARGUMENT. `workspace` may be NULL when
- * dn_chunk_fwd_workspace_bytes() is 0.
+ * DN_ERR_INVALID_ARGUMENT. `workspace`: NULL, or (when
+ * dn_chunk_fwd_workspace_bytes() is not 0) a 16-byte-aligned device buffer of at
+ * least that many bytes, owned by the caller, whose contents on entry do not
+ * matter and which overlaps no input or output (DN_ERR_WORKSPACE_TOO_SMALL,
+ * DN_ERR_MISALIGNED, DN_ERR_INVALID_ARGUMENT otherwise); it is ignored when the
+ * size is 0.
  * T == 0 copies S0 (or zeros) into S_T and writes no o.
  */
 dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const void* v,

@@ -269,3 +269,23 @@ def test_gate_range_status_and_wait_hook(lib):
     # the diagnostics hook only records the bound; put the default back
     dn.dn_set_wait_limit_ns(0)
     dn.dn_set_wait_limit_ns(dn.DEFAULT_WAIT_NS)
+
+
+def test_chunk_fwd_workspace_checks(lib):
+    d = _desc(d_k=128, d_v=128, T=100)
+    need = lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(d))
+    assert need == 2 * 2 * 25616  # B H chunks x record
+    assert lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(_desc(d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL))) == 0
+    assert lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(_desc(d_k=128, d_v=128, io_dtype=dn.DN_F32))) == 0
+    big = np.zeros(1 << 20, dtype=np.uint8)
+    ws = ctypes.c_void_p((big.ctypes.data + 15) & ~15)
+    bufs = {n: _Buf(1 << 18) for n in ("q", "k", "v", "a", "bk", "o", "st")}
+    p = {n: b.p() for n, b in bufs.items()}
+
+    def call(w, nbytes):
+        return lib.dn_chunk_fwd(ctypes.byref(d), p["q"], p["k"], p["v"], p["a"], p["bk"], None, None, None, p["o"],
+                                p["st"], w, nbytes, None)
+
+    assert call(ws, need - 16) == dn.DN_ERR_WORKSPACE_TOO_SMALL
+    assert call(ctypes.c_void_p(ws.value + 8), need) == dn.DN_ERR_MISALIGNED
+    assert call(bufs["q"].p(), need) == dn.DN_ERR_INVALID_ARGUMENT  # overlaps q
