@@ -76,6 +76,10 @@ __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int x, i
                : "memory");
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ void bulk_prefetch(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -97,22 +101,17 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ================================================================== 1. transform kernel
-template <bool BV>
-struct XLayout {
-  static constexpr int KQ = 0;               // [K; Q] bf16 [128][DK] (TMA); after the Gram: fp32 L and T (64 x 64 each)
-  static constexpr int TG = KQ + 128 * DK * 2;  // T Diag(gamma) [64][64]
-  static constexpr int PB = TG + C * C * 2;     // P' [64][64]
-  static constexpr int TB = PB + C * C * 2;     // T Diag(beta^v) [64 or 128][64]
-  static constexpr int TOTAL = TB + tb_bytes(BV);
-  static_assert(TG - KQ >= 2 * C * C * 4, "L and T fit over the [K; Q] tile");
-  static_assert(TOTAL - TG == rec_factor_off(BV), "record tiles are contiguous");
-};
+// Shared memory holds only the [K; Q] tile (TMA), which the fp32 L and T arrays overlay once the
+// Gram is done, and the inverse's scratch; P' and the T tiles go straight to the record, so four
+// CTAs fit on an SM.
+constexpr int kXformSmem = 128 * DK * 2;  // [K; Q] bf16 [128][DK]; after the Gram: fp32 L and T (64 x 64 each)
+static_assert(kXformSmem >= 2 * C * C * 4, "L and T fit over the [K; Q] tile");
+constexpr int kXformPerSm = 4;
 
 template <bool BV>
-__global__ void __launch_bounds__(kThreads) xform_sc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                            const __grid_constant__ CUtensorMap tm_k, const Args a,
-                                                            uint8_t* ws) {
-  using Ly = XLayout<BV>;
+__global__ void __launch_bounds__(kThreads, kXformPerSm) xform_sc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                        const __grid_constant__ CUtensorMap tm_k,
+                                                                        const Args a, uint8_t* ws, int ahead) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   __shared__ __align__(8) uint64_t bar_kq, bar_g;
@@ -124,45 +123,50 @@ __global__ void __launch_bounds__(kThreads) xform_sc_kernel(const __grid_constan
   const int nchunks = (a.T + C - 1) / C;
   const int bh = blockIdx.x / nchunks, c = blockIdx.x % nchunks, b = bh / a.H, h = bh % a.H;
   uint8_t* const rec = ws + (size_t)blockIdx.x * rec_stride(BV);
+  const int64_t nb = (int64_t)blockIdx.x + ahead;  // the block that takes this one's place on its SM
+  const bool pf = ahead > 0 && nb < (int64_t)gridDim.x;
+  const int nbh = (int)(nb / nchunks), nc = (int)(nb % nchunks);
 
+  // thread 0 starts the [K; Q] load at once; warps 2 and 3 load the gates meanwhile (the factor scan
+  // runs there, so that thread 0 is free to issue the Gram as soon as the tile lands)
   if (tid == 0) {
     mbar_init(&bar_kq, 1);
     mbar_init(&bar_g, 1);
     fence_mbar_init();
-  }
-  if (warp == 0) tmem_alloc(&s_tmem, 64);
-  // the 8x8 blocks above the block diagonal of the T tiles (the inverse does not write them)
-  for (int e = tid; e < 64 * 8; e += kThreads) {
-    const int t = e >> 3, x8 = e & 7;
-    if (x8 > (t >> 3)) {
-      *reinterpret_cast<uint4*>(sm + Ly::TG + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(sm + Ly::TB + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
-      if (BV) *reinterpret_cast<uint4*>(sm + Ly::TB + canon_chunk(64 + t, x8, 128)) = make_uint4(0, 0, 0, 0);
+    mbar_expect_tx(&bar_kq, 2u * C * DK * 2);
+#pragma unroll
+    for (int x = 0; x < DK / 64; ++x) {
+      tma_load_4d(sm + x * 128 * 128, &tm_k, &bar_kq, 64 * x, h, c * C, b);
+      tma_load_4d(sm + x * 128 * 128 + 64 * 128, &tm_q, &bar_kq, 64 * x, h, c * C, b);
+    }
+    // the successor block's tiles into L2
+    if (pf) {
+#pragma unroll
+      for (int x = 0; x < DK / 64; ++x) {
+        tma_prefetch_4d(&tm_k, 64 * x, nbh % a.H, nc * C, nbh / a.H);
+        tma_prefetch_4d(&tm_q, 64 * x, nbh % a.H, nc * C, nbh / a.H);
+      }
     }
   }
+  const bool fw = warp == 2 || warp == 3;  // the factor warps
+  const int j = tid - 64;                  // their token
+  scf::Gates g{};
+  if (fw) {
+    if (pf && nc * C + j < a.T) {  // the successor block's gates into L2 too
+      const int64_t tok = ((int64_t)(nbh / a.H) * a.T + nc * C + j) * a.H + nbh % a.H;
+      if (a.alpha == DN_GATE_SCALAR) prefetch_l2(a.alpha_p + tok);
+      if (a.beta_k == DN_GATE_SCALAR) prefetch_l2(a.beta_k_p + tok);
+      if (a.key_scale == DN_GATE_SCALAR) prefetch_l2(a.key_scale_p + tok);
+      if (a.beta_v == DN_GATE_SCALAR) prefetch_l2(a.beta_v_p + tok);
+    }
+    g = scf::load_gates(a, b, h, c, j);
+  }
+  if (warp == 0) tmem_alloc(&s_tmem, 64);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  if (tid == 0) {
-    mbar_expect_tx(&bar_kq, 2u * C * DK * 2);
-#pragma unroll
-    for (int x = 0; x < DK / 64; ++x) {
-      tma_load_4d(sm + Ly::KQ + x * 128 * 128, &tm_k, &bar_kq, 64 * x, h, c * C, b);
-      tma_load_4d(sm + Ly::KQ + x * 128 * 128 + 64 * 128, &tm_q, &bar_kq, 64 * x, h, c * C, b);
-    }
-  }
-  if (tid < 64) scf::token_factors(scf::load_gates(a, b, h, c, tid), tid, lane, pre, s_f);
-  __syncthreads();
-  if (tid < 64) {
-    Rec* r = reinterpret_cast<Rec*>(rec + rec_factor_off(BV));
-    r->c[tid] = s_f.c[tid];
-    r->orho[tid] = s_f.orho[tid];
-    r->oex[tid] = s_f.oex[tid];
-    r->n[tid] = s_f.n[tid];
-    if (tid == 0) r->glast = s_f.glast;
-  }
-  // Gram [K; Q] K^T -> tensor memory (M 128, N 64, K 128)
+  // Gram [K; Q] K^T -> tensor memory (M 128, N 64, K 128), while warps 2 and 3 scan the gates
   bool ok = true, issued = false;
   if (tid == 0) {
     ok = mbar_wait_bounded(&bar_kq, 0, a.wait_ns);
@@ -171,12 +175,22 @@ __global__ void __launch_bounds__(kThreads) xform_sc_kernel(const __grid_constan
       const uint32_t id = idesc_bf16(128, 64, 0, 0);
 #pragma unroll
       for (int kk = 0; kk < DK; kk += 16) {
-        const uint64_t d = sdesc(smem_u32(sm + Ly::KQ) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+        const uint64_t d = sdesc(smem_u32(sm) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
         mma_bf16(tmem, d, d, id, kk > 0);
       }
       mma_commit(&bar_g);
       issued = true;
     }
+  }
+  if (fw) {
+    scf::token_factors(g, j, lane, pre, s_f);
+    // each thread copies the entries it wrote itself
+    Rec* r = reinterpret_cast<Rec*>(rec + rec_factor_off(BV));
+    r->c[j] = s_f.c[j];
+    r->orho[j] = s_f.orho[j];
+    r->oex[j] = s_f.oex[j];
+    r->n[j] = s_f.n[j];
+    if (j == 63) r->glast = s_f.glast;
   }
   if (__syncthreads_or(!ok)) {
     // the [K; Q] load did not land in time: wait for it (bounded), report, free tensor memory
@@ -203,24 +217,53 @@ __global__ void __launch_bounds__(kThreads) xform_sc_kernel(const __grid_constan
     return;
   }
   tc_fence_after();
-  // A and P' (the [K; Q] tile is free now: L and T take its place)
-  float* sL = reinterpret_cast<float*>(sm + Ly::KQ);
+  // A into L (the [K; Q] tile is free now: L and T take its place), and P' into the inverse's
+  // scratch, which warps 2..7 copy to the record with whole-line stores while warps 0 and 1 start
+  // the inverse
+  float* sL = reinterpret_cast<float*>(sm);
   float* sT = sL + C * C;
-  scf::extract_ap(s_f, tmem, q4, gch, lane, pre, sL, sm + Ly::PB);
+  scf::extract_ap(s_f, tmem, q4, gch, lane, pre, sL, reinterpret_cast<uint8_t*>(s_Y));
   tc_fence_before();
   __syncthreads();
-  unit_lower_inverse<true, 8, true, BV>(sL, sT, s_Y, sm + Ly::TG, sm + Ly::TB, s_f.gam, s_f.bv, tid, 0);
-  __syncthreads();
-  // the tiles to the record, 16 bytes per thread and step
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(sm + Ly::TG);
-    uint4* dst = reinterpret_cast<uint4*>(rec);
-    for (int i = tid; i < rec_factor_off(BV) / 16; i += kThreads) dst[i] = src[i];
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  // tensor memory is no longer needed
   if (warp == 0) tmem_dealloc(tmem, 64);
+  if (tid >= 64) {
+    const uint4* src = reinterpret_cast<const uint4*>(s_Y);
+    uint4* dst = reinterpret_cast<uint4*>(rec + kRecP);
+    for (int i = tid - 64; i < C * C * 2 / 16; i += kThreads - 64) dst[i] = src[i];
+  }
+  unit_lower_inverse<false, 8, true, false, false>(sL, sT, s_Y, nullptr, nullptr, nullptr, nullptr, tid, 0);
+  // T Diag(gamma) and T Diag(beta^v) (hi, and lo when beta^v is given) as bf16 operand tiles, one
+  // 16-byte chunk (row t, columns 8 x8 .. +7) per thread and step: eight threads write one
+  // 128-byte row, so the stores are whole lines
+  for (int e = tid; e < C * 8; e += kThreads) {
+    const int t = e >> 3, x8 = e & 7;
+    uint4 tg = make_uint4(0, 0, 0, 0), tb = tg, tl = tg;
+    if (x8 <= (t >> 3)) {
+      const float4 v0 = *reinterpret_cast<const float4*>(sT + xi(t, 8 * x8));
+      const float4 v1 = *reinterpret_cast<const float4*>(sT + xi(t, 8 * x8 + 4));
+      const float y[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      const float* gm = s_f.gam + 8 * x8;
+      const float* bv = s_f.bv + 8 * x8;
+      tg = make_uint4(pack_bf16(y[0] * gm[0], y[1] * gm[1]), pack_bf16(y[2] * gm[2], y[3] * gm[3]),
+                      pack_bf16(y[4] * gm[4], y[5] * gm[5]), pack_bf16(y[6] * gm[6], y[7] * gm[7]));
+      float z[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[e] = y[e] * bv[e];
+      if (BV) {
+        tc::split_bf16(z[0], z[1], tb.x, tl.x);
+        tc::split_bf16(z[2], z[3], tb.y, tl.y);
+        tc::split_bf16(z[4], z[5], tb.z, tl.z);
+        tc::split_bf16(z[6], z[7], tb.w, tl.w);
+      } else {
+        tb = make_uint4(pack_bf16(z[0], z[1]), pack_bf16(z[2], z[3]), pack_bf16(z[4], z[5]), pack_bf16(z[6], z[7]));
+      }
+    }
+    const uint32_t off = canon_chunk(t, x8, 128);
+    *reinterpret_cast<uint4*>(rec + kRecTG + off) = tg;
+    *reinterpret_cast<uint4*>(rec + kRecTB + off) = tb;
+    if (BV) *reinterpret_cast<uint4*>(rec + kRecTB + 64 * 128 + off) = tl;
+  }
 }
 
 // ================================================================== 2. state-chain kernel
@@ -234,17 +277,20 @@ struct CLayout {
   static constexpr int TG = VB + C * NV * 2;       // T Diag(gamma) [64][64]; P' of parity 0 and 1 follow it:
   static constexpr int PB0 = TG + C * C * 2;       // the O product of parity p reads the 128 rows starting
   static constexpr int PB1 = PB0 + C * C * 2;      // 64 rows before PB_p, whose rows 64..127 are P'
-  static constexpr int TB = PB1 + C * C * 2;       // T Diag(beta^v) [128][64] (lo rows 64..127, or zero)
-  static constexpr int OST = TB + 128 * C * 2;     // o rows of a chunk [C][NV] bf16, staged for the TMA store
+  // T Diag(beta^v): hi rows, 64 zero rows, lo rows, 64 zero rows (the U0 product reads 128
+  // rows from the hi or the lo rows, and its rows 64..127 must come out zero)
+  static constexpr int TB = PB1 + C * C * 2;
+  static constexpr int TBLO = TB + 128 * C * 2;
+  static constexpr int OST = TBLO + 128 * C * 2;   // o rows of a chunk [C][NV] bf16, staged for the TMA store
   static constexpr int SMU = OST + C * NV * 2;     // S bf16 [DK][NV]; after D1: U' hi, U' lo [C][NV]
   static constexpr int SMU_BYTES = (DK * NV * 2 > 2 * C * NV * 2) ? DK * NV * 2 : 2 * C * NV * 2;
   static constexpr int FR0 = SMU + SMU_BYTES;      // factor records of parity 0 and 1
   static constexpr int FR1 = FR0 + 1088;
   static constexpr int TOTAL = FR1 + 1088;
-  // the lo operand of T Diag(beta^v) reads 64 rows past TB: they lie in OST
-  static_assert(C * NV * 2 >= 64 * C * 2, "operand overrun stays in shared memory");
   static_assert(TOTAL + 1024 + 4096 <= 227 * 1024, "shared memory budget");
-  static constexpr int TM_S = 0, TM_D1 = NV, TM_U0 = 2 * NV, TM_WK = 3 * NV;
+  // tensor memory: the state; two accumulators (chunk parity) where U0 lands and D1 and the O product
+  // accumulate; Wk
+  static constexpr int TM_S = 0, TM_U = NV, TM_WK = 3 * NV;
   static_assert(TM_WK + DK <= 512, "tensor memory budget");
 };
 
@@ -254,15 +300,18 @@ struct CLayout {
 //    lanes) and meet at a barrier, after which thread 0 issues D1 = [Wk; Q'] S (warp 0 has nothing to
 //    do until D1 is done anyway); quadrants 0 and 1 form U' (rows 0..63 of D1 and U0) and the group
 //    meets again, after which thread 0 issues O += P' U' (rows 64..127 of D1; the o rows leave as soon
-//    as it is done), then the state update (the next chunk's framing waits for it); quadrants 0 and 1
-//    then convert the next chunk's Wk (lanes 0..63) and scale its q rows to Q', while quadrants 2 and 3
-//    store the o rows;
-//  * warp 11 (quadrant 3) scales the k rows of each chunk to K' (shared memory only);
+//    as it is done), then the state update (the next chunk's framing waits for it); quadrants 2 and 3
+//    store the o rows while the state update runs;
+//  * warps 8 and 9 (quadrants 0 and 1) convert each chunk's Wk (lanes 0..63 of its accumulator) to the
+//    bf16 rows 0..63 of its [Wk; Q'] tile, ahead of the chain;
+//  * warp 11 scales the q rows of each chunk to Q' and its k rows to K' (shared memory only);
 //  * lane 0 of warp 10 issues every load (and L2 prefetches further ahead) and the state-independent
-//    products of the next chunk, Wk(c + 1) and U0(c + 1), as soon as thread 0 signals that their
-//    tensor memory is free (so their issue stalls never hold the chain's warps);
-//  * warps 8 and 9 only place warps 10 and 11 on their sub-partitions.
-// Hand-overs across warps go through mbarriers; within warps 0..7 through a named barrier.
+//    products of the next chunk, Wk(c + 1) and U0(c + 1), as soon as their tensor memory is free (so
+//    their issue stalls never hold the chain's warps).
+// Hand-overs across warps go through mbarriers; within warps 0..7 through a named barrier. Each
+// mbarrier that completes once per chunk is waited on for chunk c only by threads whose progress
+// keeps its completion for chunk c + 1 from happening first (a wait by parity cannot tell two
+// completions apart).
 constexpr int kChainThreads = 384;
 constexpr int kLoaderWarp = 10;
 constexpr int kScalerWarp = 11;
@@ -275,15 +324,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const Args a,
                     const uint8_t* ws, int bv_split) {
   using Ly = CLayout<NV>;
-  constexpr int NCB = NV / 64;
+  constexpr int HALVES = 1;  // one state chain per CTA (its per-half barriers use index 0)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   // loads (transaction counts); products (commits); hand-overs (arrivals)
   __shared__ __align__(8) uint64_t bar_kq[2], bar_fr[2], bar_tg, bar_vb, bar_p[2];
   // (the state update, the O product and the o stores of chunk c complete barrier [c & 1]: the loader
   // looks at them a chunk later than the chain, which can never lap it by two chunks)
-  __shared__ __align__(8) uint64_t bar_wk, bar_u0, bar_d1, bar_os[2], bar_o[2], bar_drain, bar_drain2;
-  __shared__ __align__(8) uint64_t bar_kconv, bar_ostored[2], bar_wkfree, bar_ufree;
+  // (per value-column half hf: bar_d1[hf], bar_os[hf][p], bar_o[hf][p], bar_ostored[hf][p], bar_drain[hf])
+  __shared__ __align__(8) uint64_t bar_wk, bar_u0, bar_d1[2], bar_os[2][2], bar_o[2][2], bar_drain[2], bar_drain2;
+  __shared__ __align__(8) uint64_t bar_kconv, bar_ostored[2][2], bar_wkfree, bar_ufree, bar_wkconv;
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, ch = (warp >> 2) & 1;
@@ -302,26 +352,30 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       mbar_init(&bar_kq[j], 1);
       mbar_init(&bar_fr[j], 1);
       mbar_init(&bar_p[j], 1);
-      mbar_init(&bar_os[j], 1);
-      mbar_init(&bar_o[j], 1);
-      mbar_init(&bar_ostored[j], 1);  // the thread that issues the o tile's store
+      mbar_init(&bar_d1[j], 1);
+      mbar_init(&bar_drain[j], 1);
+      for (int hf = 0; hf < 2; ++hf) {
+        mbar_init(&bar_os[hf][j], 1);
+        mbar_init(&bar_o[hf][j], 1);
+        mbar_init(&bar_ostored[hf][j], 1);  // the thread that issues the half's o store
+      }
     }
     mbar_init(&bar_tg, 1);
     mbar_init(&bar_vb, 1);
     mbar_init(&bar_wk, 1);
     mbar_init(&bar_u0, 1);
-    mbar_init(&bar_d1, 1);
-    mbar_init(&bar_drain, 1);
     mbar_init(&bar_drain2, 1);
-    mbar_init(&bar_wkfree, 1);   // thread 0: chunk c's Wk is converted (TM_WK free)
-    mbar_init(&bar_ufree, 1);    // thread 0: chunk c's U' is formed (TM_U0 free)
-    mbar_init(&bar_kconv, 1);    // the k-scaling warp
+    mbar_init(&bar_wkfree, 2);   // warps 8, 9: chunk c's Wk has been read (TM_WK free)
+    mbar_init(&bar_wkconv, 2);   // warps 8, 9: chunk c's Wk rows of the [Wk; Q'] tile are written
+    mbar_init(&bar_ufree, HALVES);  // the halves' issuing threads: chunk c's U' is formed (TM_U0 free)
+    mbar_init(&bar_kconv, 1);    // the scaling warp: chunk c's K' and Q' rows are scaled
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_tmem, 512);
-  if (!bv_split) {  // no lo part: rows 64..127 of the T Diag(beta^v) tile stay zero
-    for (int i = tid; i < 64 * C * 2 / 16; i += kChainThreads)
-      reinterpret_cast<uint4*>(sm + Ly::TB + 64 * 128)[i] = make_uint4(0, 0, 0, 0);
+  // the zero rows after the hi and after the lo rows of T Diag(beta^v)
+  for (int i = tid; i < 64 * C * 2 / 16; i += kChainThreads) {
+    reinterpret_cast<uint4*>(sm + Ly::TB + 64 * 128)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sm + Ly::TBLO + 64 * 128)[i] = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async();
   tc_fence_before();
@@ -342,6 +396,12 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool { return mbar_wait_bounded(bar, parity, a.wait_ns); };
   auto wait_idle = [&](uint64_t* bar, uint32_t parity) -> bool {
     return mbar_wait_bounded_idle(bar, parity, a.wait_ns);
+  };
+  // a per-half, per-parity barrier of every half
+  auto wait_halves = [&](uint64_t (*bars)[2], int j, uint32_t parity) -> bool {
+    for (int hf = 0; hf < HALVES; ++hf)
+      if (!wait_idle(&bars[hf][j], parity)) return false;
+    return true;
   };
 
   bool failed = false;
@@ -376,7 +436,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         mbar_expect_tx(&bar_vb, (uint32_t)C * NV * 2 + tbb);
 #pragma unroll
         for (int x = 0; x < NV / 64; ++x) tma_load_4d(sm + Ly::VB + x * C * 128, &tm_v, &bar_vb, col0 + 64 * x, h, c * C, b);
-        bulk_load(sm + Ly::TB, rec(c) + kRecTB, tbb, &bar_vb);
+        bulk_load(sm + Ly::TB, rec(c) + kRecTB, 8192, &bar_vb);
+        if (bv_split) bulk_load(sm + Ly::TBLO, rec(c) + kRecTB + 8192, 8192, &bar_vb);
         pend_vb = c;
       };
       auto issue_p = [&](int c) {
@@ -408,7 +469,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       for (int c = 2; c < 4 && c < nchunks; ++c) prefetch(c);
       const uint32_t id_wk = idesc_bf16(128, DK, 0, 1);
       const uint32_t id_nv = idesc_bf16(128, NV, 0, 1);
-      // Wk(c) = (T Diag gamma) K(c) -> TM_WK (lanes 0..63); U0(c) = (T Diag beta^v) V(c) -> TM_U0
+      // Wk(c) = (T Diag gamma) K(c) -> TM_WK (lanes 0..63); U0(c) = (T Diag beta^v) V(c) ->
+      // accumulator c & 1 (rows 64..127 zero)
       auto mma_wk = [&](int c) {
 #pragma unroll
         for (int kk = 0; kk < C; kk += 16) {
@@ -419,16 +481,15 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         mma_commit(&bar_wk);
       };
       auto mma_u0 = [&](int c) {
-        const uint32_t tb = smem_u32(sm + Ly::TB), vb = smem_u32(sm + Ly::VB);
-        (void)c;
+        const uint32_t vb = smem_u32(sm + Ly::VB), acc = tmem + Ly::TM_U + (c & 1) * NV;
+        const uint32_t hi = smem_u32(sm + Ly::TB), lo = smem_u32(sm + Ly::TBLO);
 #pragma unroll
         for (int kk = 0; kk < C; kk += 16)
-          mma_bf16(tmem + Ly::TM_U0, sdesc(tb + kk * 2, 16, 1024), sdesc(vb + kk * 128, C * 128, 1024), id_nv, kk > 0);
+          mma_bf16(acc, sdesc(hi + kk * 2, 16, 1024), sdesc(vb + kk * 128, C * 128, 1024), id_nv, kk > 0);
         if (bv_split) {
 #pragma unroll
           for (int kk = 0; kk < C; kk += 16)
-            mma_bf16(tmem + Ly::TM_U0, sdesc(tb + 64 * 128 + kk * 2, 16, 1024), sdesc(vb + kk * 128, C * 128, 1024),
-                     id_nv, 1);
+            mma_bf16(acc, sdesc(lo + kk * 2, 16, 1024), sdesc(vb + kk * 128, C * 128, 1024), id_nv, 1);
         }
         mma_commit(&bar_u0);
       };
@@ -463,7 +524,9 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           issue_tg(1);
         }
         if (more) {
-          ok = wait_idle(&bar_wkfree, par(c)) && wait_idle(&bar_tg, par(c + 1)) && wait_idle(&bar_kq[(c + 1) & 1], par2(c + 1));
+          // (kconv(c) too: the scaling warp must have seen Wk(c) complete before Wk(c + 1) can)
+          ok = wait_idle(&bar_wkfree, par(c)) && wait_idle(&bar_kconv, par(c)) && wait_idle(&bar_tg, par(c + 1)) &&
+               wait_idle(&bar_kq[(c + 1) & 1], par2(c + 1));
           if (!ok) break;
           pend_tg = pend_kq[(c + 1) & 1] = -1;
           tc_fence_after();
@@ -486,13 +549,13 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           }
         }
         if (c + 2 < nchunks) {  // (U0(c) is done: the chain saw it before signalling bar_ufree)
-          ok = wait_idle(&bar_os[c & 1], par2(c));
+          ok = wait_halves(bar_os, c & 1, par2(c));
           if (!ok) break;
           issue_kq(c + 2);
-          ok = wait_idle(&bar_o[c & 1], par2(c));
+          ok = wait_halves(bar_o, c & 1, par2(c));
           if (!ok) break;
           issue_p(c + 2);
-          ok = wait_idle(&bar_ostored[c & 1], par2(c));
+          ok = wait_halves(bar_ostored, c & 1, par2(c));
           if (!ok) break;
           issue_fr(c + 2);
         }
@@ -514,15 +577,10 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       }
     }
   } else if (warp == kScalerWarp) {
-    // ======================================================= k rows of each chunk -> K' = 2^{n} k
-    bool ok = true;
-    for (int c = 0; c < nchunks && ok; ++c) {
-      // its k tile and factors have landed, and Wk(c) has read the raw k rows
-      ok = wait_idle(&bar_kq[c & 1], par2(c)) && wait_idle(&bar_fr[c & 1], par2(c)) && wait_idle(&bar_wk, par(c));
-      if (!ok) break;
-      const Rec* fr = frec(c);
-      uint8_t* const kt = kb(c);
-      // in batches of 8 loads before their stores
+    // ======================================================= q rows -> Q' = 2^{oex} q, k rows -> K' = 2^{n} k
+    // 16-byte chunk e of a 64-row, 128-column tile: row e / 16, chunk e % 16; in batches of 8 loads
+    // before their stores
+    auto scale_rows = [&](uint8_t* tile, int row0, const int* ex) {
 #pragma unroll 1
       for (int j0 = 0; j0 < 32; j0 += 8) {
         uint4 kv[8];
@@ -530,68 +588,95 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int e = lane + 32 * (j0 + j), i = e >> 4;
-          kv[j] = *reinterpret_cast<const uint4*>(kt + canon_chunk(i, e & 15, C));
-          sc[j] = pow2f(fr->n[i]);
+          kv[j] = *reinterpret_cast<const uint4*>(tile + canon_chunk(row0 + i, e & 15, row0 + C));
+          sc[j] = pow2f(ex[i]);
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int e = lane + 32 * (j0 + j), i = e >> 4;
-          *reinterpret_cast<uint4*>(kt + canon_chunk(i, e & 15, C)) = scale_bf16x8(kv[j], sc[j]);
+          *reinterpret_cast<uint4*>(tile + canon_chunk(row0 + i, e & 15, row0 + C)) = scale_bf16x8(kv[j], sc[j]);
         }
       }
+    };
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      // the q and k tiles and the factors of chunk c have landed
+      ok = wait_idle(&bar_kq[c & 1], par2(c)) && wait_idle(&bar_fr[c & 1], par2(c));
+      if (!ok) break;
+      const Rec* fr = frec(c);
+      scale_rows(qb(c), 64, fr->oex);  // rows 64..127 of the [Wk; Q'] tile (the tile has 128 rows)
+      ok = wait_idle(&bar_wk, par(c));   // Wk(c) has read the raw k rows
+      if (!ok) break;
+      scale_rows(kb(c), 0, fr->n);
       fence_proxy_async();
+      // D1(c - 1) is done, so the chain has seen kconv(c - 1) before kconv(c) can complete
+      ok = c == 0 || (wait_idle(&bar_d1[0], par(c - 1)) && (HALVES == 1 || wait_idle(&bar_d1[1], par(c - 1))));
+      if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_kconv);
     }
     if (!ok && nchunks > 0) failed = true;
-  } else if (warp < 8) {
-    // ======================================================= the state chain, warps 0..7
-    const uint32_t id_nv = idesc_bf16(128, NV, 0, 1);
-    const uint32_t id_state = idesc_bf16(128, NV, 1, 1);
-    bool issued = false;  // thread 0 has issued products (the drain then waits for them)
-    // chunk c's Wk (lanes 0..63) -> bf16 rows 0..63 of its [Wk; Q'] tile and its q rows scaled to
-    // Q' = 2^{oex} q (rows 64..127): quadrants 0 and 1, once Wk(c), k, q and the factors are in
-    auto convert = [&](int c) -> bool {
-      if (q4 >= 2) return true;
-      if (!(wait(&bar_wk, par(c)) && wait(&bar_kq[c & 1], par2(c)) && wait(&bar_fr[c & 1], par2(c)))) return false;
+  } else if (warp == 8 || warp == 9) {
+    // ======================================================= Wk(c) (lanes 0..63) -> bf16 rows 0..63 of [Wk; Q'](c)
+    bool ok = true;
+    const int t = 32 * q4 + lane;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      // Wk(c) is done; U'(c - 1) is formed (so D1(c - 1) is done: it read this tile's buffer two chunks
+      // ago, and the chain has seen wkconv(c - 1) before wkconv(c) can complete). Starting only then
+      // keeps these warps off their sub-partitions while quadrants 0 and 1 form U'.
+      ok = wait_idle(&bar_wk, par(c)) && (c == 0 || wait(&bar_ufree, par(c - 1)));
+      if (!ok) break;
       tc_fence_after();
       uint8_t* const qt = qb(c);
-      const int t = 32 * q4 + lane;
-      {
-        uint4 qv[8];  // this thread's half row of q: every load in flight before any store
+      const float nc = -1.f;  // the rows are -Wk: D1 accumulates onto U0
 #pragma unroll
-        for (int j = 0; j < 8; ++j) qv[j] = *reinterpret_cast<const uint4*>(qt + canon_chunk(64 + t, 8 * ch + j, 128));
-        const float sc = pow2f(frec(c)->oex[t]);
+      for (int hb = 0; hb < 2; ++hb) {  // two halves of 64 columns
+        uint32_t xr[2][32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(qt + canon_chunk(64 + t, 8 * ch + j, 128)) = scale_bf16x8(qv[j], sc);
-      }
-      uint32_t xr[DK / 64][32];
+        for (int cb = 0; cb < 2; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_WK + 64 * hb + 32 * cb, xr[cb]);
 #pragma unroll
-      for (int cb = 0; cb < DK / 64; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_WK + ch * (DK / 2) + 32 * cb, xr[cb]);
+        for (int cb = 0; cb < 2; ++cb) tmem_wait_ld(xr[cb]);
+        if (hb == 1) {  // every load of Wk(c) is complete: TM_WK is free for Wk(c + 1)
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_wkfree);
+        }
 #pragma unroll
-      for (int cb = 0; cb < DK / 64; ++cb) tmem_wait_ld(xr[cb]);
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col = 64 * hb + 32 * cb;
+          const float* x = reinterpret_cast<const float*>(xr[cb]);
 #pragma unroll
-      for (int cb = 0; cb < DK / 64; ++cb) {
-        const int col = ch * (DK / 2) + 32 * cb;
-        const uint32_t* x = xr[cb];
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-          uint4 pk = make_uint4(pack_bf16(__uint_as_float(x[8 * q8]), __uint_as_float(x[8 * q8 + 1])),
-                                pack_bf16(__uint_as_float(x[8 * q8 + 2]), __uint_as_float(x[8 * q8 + 3])),
-                                pack_bf16(__uint_as_float(x[8 * q8 + 4]), __uint_as_float(x[8 * q8 + 5])),
-                                pack_bf16(__uint_as_float(x[8 * q8 + 6]), __uint_as_float(x[8 * q8 + 7])));
-          *reinterpret_cast<uint4*>(qt + canon_chunk(t, col / 8 + q8, 128)) = pk;
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const float* y = x + 8 * q8;
+            uint4 pk = make_uint4(pack_bf16(nc * y[0], nc * y[1]), pack_bf16(nc * y[2], nc * y[3]),
+                                  pack_bf16(nc * y[4], nc * y[5]), pack_bf16(nc * y[6], nc * y[7]));
+            *reinterpret_cast<uint4*>(qt + canon_chunk(t, col / 8 + q8, 128)) = pk;
+          }
         }
       }
-      return true;
-    };
-    // o rows of chunk c from rows 64..127 of D1 (quadrants 2, 3, meeting at barrier kBarOut), once O(c)
-    // is done: scaled, rounded and staged in shared memory, then written by one TMA store per 64
-    // columns (the tensor map clips the rows past the sequence's end); thread 64 issues the stores.
-    // Every thread of quadrants 2 and 3 calls it with its failure state (the barrier takes all 128).
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_wkconv);
+    }
+    if (!ok && nchunks > 0) failed = true;
+  } else if (warp < 8) {
+    // ======================================================= the state chain, warps 0..7: warp (q4, ch)
+    // covers lanes 32 q4 .. +31 and value columns ch NV / 2 .. + NV / 2
+    constexpr int NCB = NV / 64;  // 32-column blocks per warp
+    const uint32_t id_nv = idesc_bf16(128, NV, 0, 1);
+    const uint32_t id_state = idesc_bf16(128, NV, 1, 1);
+    const int cw = ch * (NV / 2);  // this warp's first column
+    bool issued = false;           // thread 0 has issued products (the drain then waits for them)
+    // accumulator of chunk c: U0, then U0 - Wk S (rows 0..63; U' = c (U0 - Wk S)) and Q' S + P' U'
+    // (rows 64..127)
+    auto tm_u = [&](int c) -> uint32_t { return tmem + Ly::TM_U + (c & 1) * NV; };
+    // o rows of chunk c from rows 64..127 of its accumulator (quadrants 2, 3, meeting at barrier
+    // kBarOut), once O(c) is done: scaled, rounded and staged in shared memory, then written by one TMA
+    // store per 64 columns (the tensor map clips the rows past the sequence's end); thread 64 issues
+    // the stores. Every thread of quadrants 2 and 3 calls it with its failure state (the barrier takes
+    // all 128).
     auto store_o = [&](int c, bool ok_in) -> bool {
-      bool okw = ok_in && wait(&bar_o[c & 1], par2(c));
+      bool okw = ok_in && wait(&bar_o[0][c & 1], par2(c));
       if (tid == 64) bulk_wait_read_all();  // the previous chunk's store has read the staging tile
       if (group_or(kBarOut, 128, !okw)) return false;
       tc_fence_after();
@@ -599,12 +684,12 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       const float os = frec(c)->orho[t];
       uint32_t xr[NCB][32];
 #pragma unroll
-      for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_D1 + ch * (NV / 2) + 32 * cb, xr[cb]);
+      for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tm_u(c) + lane_base + cw + 32 * cb, xr[cb]);
 #pragma unroll
       for (int cb = 0; cb < NCB; ++cb) tmem_wait_ld(xr[cb]);
 #pragma unroll
       for (int cb = 0; cb < NCB; ++cb) {
-        const int col = ch * (NV / 2) + 32 * cb;
+        const int col = cw + 32 * cb;
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           const float* x = reinterpret_cast<const float*>(xr[cb]) + 8 * q8;
@@ -620,7 +705,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 #pragma unroll
         for (int x = 0; x < NV / 64; ++x) tma_store_4d(&tm_o, sm + Ly::OST + x * C * 128, col0 + 64 * x, h, c * C, b);
         bulk_commit();
-        mbar_arrive(&bar_ostored[c & 1]);  // the factor record's o scales have been read
+        mbar_arrive(&bar_ostored[0][c & 1]);  // the factor record's o scales have been read
       }
       return true;
     };
@@ -629,23 +714,14 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 
     // ok: this thread's waits so far succeeded; run: the group's vote at its last barrier (loops are left
     // only on a vote, so that every thread of the group reaches every barrier)
-    bool ok = nchunks > 0, run = false;
-    // ---- prologue: chunk 0's conversions
-    if (ok) {
-      ok = convert(0);
-      fence_proxy_async();
-      tc_fence_before();
-      run = ok = !chain_sync(!ok);
-      tc_fence_after();
-    }
+    bool ok = nchunks > 0, run = nchunks > 0;
     for (int c = 0; run && c < nchunks; ++c) {
-      const bool more = c + 1 < nchunks;
       // ---- the previous chunk's o rows (quadrants 2, 3): O(c - 1) is done before the state update of
-      // chunk c - 1, which they overlap; D1(c) overwrites their rows after the next barrier
+      // chunk c - 1, which they overlap
       if (c > 0 && q4 >= 2) ok = store_o(c - 1, ok);
       // ---- the state entering chunk c -> bf16 operand tile; gamma_C S -> TM_S (fp32, where the state
       // update accumulates): after the state update of chunk c - 1
-      if (ok && c > 0) ok = wait(&bar_os[(c - 1) & 1], par2(c - 1));
+      if (ok && c > 0) ok = wait(&bar_os[0][(c - 1) & 1], par2(c - 1));
       ok = ok && wait(&bar_fr[c & 1], par2(c));
       if (ok) {
         tc_fence_after();
@@ -655,8 +731,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         if (c == 0) {
 #pragma unroll
           for (int cb = 0; cb < NCB; ++cb) {
-            const int col = ch * (NV / 2) + 32 * cb;
-            const float* src = a.S0 ? a.S0 + ((int64_t)bh * DK + k) * dv + col0 + col : nullptr;
+            const float* src = a.S0 ? a.S0 + ((int64_t)bh * DK + k) * dv + col0 + cw + 32 * cb : nullptr;
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
               const float4 f = src ? *reinterpret_cast<const float4*>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -666,13 +741,13 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           }
         } else {
 #pragma unroll
-          for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_S + ch * (NV / 2) + 32 * cb, xr[cb]);
+          for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tmem + lane_base + Ly::TM_S + cw + 32 * cb, xr[cb]);
 #pragma unroll
           for (int cb = 0; cb < NCB; ++cb) tmem_wait_ld(xr[cb]);
         }
 #pragma unroll
         for (int cb = 0; cb < NCB; ++cb) {
-          const int col = ch * (NV / 2) + 32 * cb;
+          const int col = cw + 32 * cb;
           float x[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(xr[cb][e]);
@@ -695,50 +770,44 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         break;
       }
       tc_fence_after();
-      // ---- D1(c) = [Wk; Q'](c) S (its K' rows are scaled too); TM_WK is free for Wk(c + 1)
+      // ---- D1(c) = [-Wk; Q'](c) S, accumulated onto U0(c), once U0(c) is done, the Wk rows are
+      // converted and the Q' and K' rows scaled
       if (tid == 0) {
-        ok = wait(&bar_kconv, par(c));
+        ok = wait(&bar_kconv, par(c)) && wait(&bar_wkconv, par(c)) && wait(&bar_u0, par(c));
         if (ok) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < DK; kk += 16) {
             const uint64_t ad = sdesc(smem_u32(qb(c)) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
             const uint64_t bd = sdesc(smem_u32(sm + Ly::SMU) + kk * 128, DK * 128, 1024);
-            mma_bf16(tmem + Ly::TM_D1, ad, bd, id_nv, kk > 0);
+            mma_bf16(tm_u(c), ad, bd, id_nv, 1);
           }
-          mma_commit(&bar_d1);
+          mma_commit(&bar_d1[0]);
           issued = true;
-          mbar_arrive(&bar_wkfree);
         }
       }
-      // ---- U' = c (U0 - Wk S) -> hi / lo tiles (the S tile is dead once D1 is done)
-      ok = ok && wait(&bar_d1, par(c)) && wait(&bar_u0, par(c));
+      // ---- U' = c (U0 - Wk S) (rows 0..63 of the accumulator) -> hi / lo tiles (the S tile is dead
+      // once D1 is done)
+      ok = ok && wait(&bar_d1[0], par(c));
       if (ok && q4 < 2) {
         tc_fence_after();
         const int t = 32 * q4 + lane;
         const float us = frec(c)->c[t];
-        uint32_t u0r[NCB][32], d1r[NCB][32];  // every TMEM load of this thread in flight at once
+        uint32_t ur[NCB][32];  // every TMEM load of this thread in flight at once
+#pragma unroll
+        for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tm_u(c) + lane_base + cw + 32 * cb, ur[cb]);
+#pragma unroll
+        for (int cb = 0; cb < NCB; ++cb) tmem_wait_ld(ur[cb]);
 #pragma unroll
         for (int cb = 0; cb < NCB; ++cb) {
-          tmem_ld32_issue(tmem + lane_base + Ly::TM_U0 + ch * (NV / 2) + 32 * cb, u0r[cb]);
-          tmem_ld32_issue(tmem + lane_base + Ly::TM_D1 + ch * (NV / 2) + 32 * cb, d1r[cb]);
-        }
-#pragma unroll
-        for (int cb = 0; cb < NCB; ++cb) {
-          tmem_wait_ld(u0r[cb]);
-          tmem_wait_ld(d1r[cb]);
-        }
-#pragma unroll
-        for (int cb = 0; cb < NCB; ++cb) {
-          const int col = ch * (NV / 2) + 32 * cb;
+          const int col = cw + 32 * cb;
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int i = 8 * q8 + 2 * e;
-              split_bf16(us * (__uint_as_float(u0r[cb][i]) - __uint_as_float(d1r[cb][i])),
-                         us * (__uint_as_float(u0r[cb][i + 1]) - __uint_as_float(d1r[cb][i + 1])), hi[e], lo[e]);
+              split_bf16(us * __uint_as_float(ur[cb][i]), us * __uint_as_float(ur[cb][i + 1]), hi[e], lo[e]);
             }
             const uint32_t off = canon_chunk(t, col / 8 + q8, C);
             *reinterpret_cast<uint4*>(sm + Ly::SMU + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -753,8 +822,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         break;
       }
       tc_fence_after();
-      // ---- O += P' U' (rows 64..127 of D1) -> bar_o; then S_acc += K'^T U' (hi and lo) -> bar_os, which
-      // so also covers O: the next framing overwrites the U' tiles; then U0(c + 1)
+      // ---- O += P' U' (rows 64..127 of the accumulator) -> bar_o; then S_acc += K'^T U' (hi and lo)
+      // -> bar_os, which so also covers O: the next framing overwrites the U' tiles
       if (tid == 0) {
         ok = wait(&bar_p[c & 1], par2(c));
         if (ok) {
@@ -762,9 +831,9 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           const uint32_t pa = smem_u32(pbuf(c)) - C * C * 2;  // rows 64..127 of this operand are P'
 #pragma unroll
           for (int kk = 0; kk < C; kk += 16)
-            mma_bf16(tmem + Ly::TM_D1, sdesc(pa + kk * 2, 16, 1024),
-                     sdesc(smem_u32(sm + Ly::SMU) + kk * 128, C * 128, 1024), id_nv, 1);
-          mma_commit(&bar_o[c & 1]);
+            mma_bf16(tm_u(c), sdesc(pa + kk * 2, 16, 1024), sdesc(smem_u32(sm + Ly::SMU) + kk * 128, C * 128, 1024),
+                     id_nv, 1);
+          mma_commit(&bar_o[0][c & 1]);
           const uint32_t kt = smem_u32(kb(c));
 #pragma unroll
           for (int kk = 0; kk < C; kk += 16) {
@@ -773,24 +842,21 @@ __global__ void __launch_bounds__(kChainThreads, 1)
             mma_bf16(tmem + Ly::TM_S, ak, sdesc(smem_u32(sm + Ly::SMU + C * NV * 2) + kk * 128, C * 128, 1024),
                      id_state, 1);
           }
-          mma_commit(&bar_os[c & 1]);
-          mbar_arrive(&bar_ufree);  // TM_U0 is free: U'(c) has been formed
+          mma_commit(&bar_os[0][c & 1]);
+          mbar_arrive(&bar_ufree);  // U'(c) is formed
         }
       }
-      // ---- chunk c + 1's conversions (quadrants 0, 1) while the products of chunk c run; a failure here
-      // reaches the group at its next barrier
-      if (ok && more) ok = convert(c + 1);
     }
     if (run) {  // (a group decision: every o-storing thread enters the barrier in store_o)
       // the last chunk's o rows and S_T = S_acc
       if (q4 >= 2) ok = store_o(nchunks - 1, ok);
-      ok = ok && wait(&bar_os[(nchunks - 1) & 1], par2(nchunks - 1));
+      ok = ok && wait(&bar_os[0][(nchunks - 1) & 1], par2(nchunks - 1));
       if (ok) {
         tc_fence_after();
         const int k = 32 * q4 + lane;
 #pragma unroll
         for (int cb = 0; cb < NCB; ++cb) {
-          const int col = ch * (NV / 2) + 32 * cb;
+          const int col = cw + 32 * cb;
           float x[32];
           tmem_ld32(tmem + lane_base + Ly::TM_S + col, x);
           float* dst = a.S + ((int64_t)bh * DK + k) * dv + col0 + col;
@@ -804,8 +870,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     if (!ok && nchunks > 0) failed = true;
     if (!ok && tid == 0 && issued) {
       // drain: every tensor-core product thread 0 issued (one commit tracks them all)
-      mma_commit(&bar_drain);
-      mbar_wait_bounded(&bar_drain, 0, kDrainNs);
+      mma_commit(&bar_drain[0]);
+      mbar_wait_bounded(&bar_drain[0], 0, kDrainNs);
     }
   }
   if (failed && (tid & 31) == 0) atomicExch(a.status, kDevTimeout);
@@ -818,11 +884,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 // ------------------------------------------------------------------ host side
 template <bool BV>
 cudaError_t launch_xform(const Args& a, const CUtensorMap& mq, const CUtensorMap& mk, uint8_t* ws, cudaStream_t s) {
-  const int smem = XLayout<BV>::TOTAL + 1024;
+  const int smem = kXformSmem + 1024;
   cudaError_t e = cudaFuncSetAttribute(xform_sc_kernel<BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t nblk = (int64_t)a.B * a.H * ((a.T + C - 1) / C);
-  xform_sc_kernel<BV><<<(unsigned)nblk, kThreads, smem, s>>>(mq, mk, a, ws);
+  // blocks resident at once: a block's successor on its SM slot is about this many blocks later
+  int dev = 0, sms = 148, per_sm = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, xform_sc_kernel<BV>, kThreads, smem) != cudaSuccess)
+    per_sm = 0;
+  xform_sc_kernel<BV><<<(unsigned)nblk, kThreads, smem, s>>>(mq, mk, a, ws, sms * per_sm);
   return cudaGetLastError();
 }
 

@@ -301,12 +301,17 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
   return __bfloat1622float2(h);
 }
 
-// Eight packed bf16 values times a float (a power of two in the callers, so the scaling is exact
-// unless a value leaves the bf16 range).
+// Eight packed bf16 values times a power of two s (0, or 2^k with -126 <= k <= 127, so that s is a
+// bf16 value itself): packed bf16 multiplies, one rounding of the exact product, which is exact
+// unless a value leaves the bf16 range.
 __device__ __forceinline__ uint4 scale_bf16x8(uint4 u, float s) {
-  float2 a = unpack_bf16(u.x), b = unpack_bf16(u.y), c = unpack_bf16(u.z), d = unpack_bf16(u.w);
-  return make_uint4(pack_bf16(a.x * s, a.y * s), pack_bf16(b.x * s, b.y * s), pack_bf16(c.x * s, c.y * s),
-                    pack_bf16(d.x * s, d.y * s));
+  const __nv_bfloat162 s2 = __float2bfloat162_rn(s);
+  auto m = [&](uint32_t x) -> uint32_t {
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&x);
+    h = __hmul2(h, s2);
+    return *reinterpret_cast<uint32_t*>(&h);
+  };
+  return make_uint4(m(u.x), m(u.y), m(u.z), m(u.w));
 }
 
 // Split x into hi = bf16(x) and lo = bf16(x - hi): hi + lo carries ~16 mantissa bits.

@@ -99,10 +99,12 @@ __device__ __forceinline__ void warp_store(const float* d, FW W, int lane) {
 // are not written (their zeros are set once by the caller). The fp32 blocks above the diagonal
 // that the merges read are zeroed here when ZERO (sT shares memory with other data), else the
 // caller keeps them zero. When SC and TT_LO, the bf16 rounding residue of T Diag(cs_v) is written
-// too, into rows 64..127 of tile tt (so that hi + lo carries about 16 mantissa bits). scr: 2048
-// floats of scratch.
+// too, into rows 64..127 of tile tt (so that hi + lo carries about 16 mantissa bits). Without EMIT
+// no tile is written; instead the whole lower triangle of T (8x8 block diagonal included, zeros
+// above the diagonal inside it) is left in sT in fp32, for the caller to convert. scr: 2048 floats
+// of scratch.
 // Not inlined: it gets its own register budget.
-template <bool SC, int NW, bool ZERO = true, bool TT_LO = false>
+template <bool SC, int NW, bool ZERO = true, bool TT_LO = false, bool EMIT = true>
 __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, float* scr, uint8_t* tp, uint8_t* tt,
                                                 const float* cs_c, const float* cs_v, int tid, int bar_id) {
   static_assert(NW >= 4 && NW <= 8, "warp count");
@@ -110,6 +112,7 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
   auto sync = [&] { group_sync(bar_id, 32 * NW); };
   constexpr uint32_t kLoRows = 64 * 128;  // byte offset of row 64 in a 64-column K-major tile
   auto emit1 = [&](int t, int i, float v) {
+    if (!EMIT) return;
     const uint32_t off = canon(t, i, 128);
     *reinterpret_cast<__nv_bfloat16*>(tp + off) = __float2bfloat16_rn(SC ? v * cs_c[i] : v);
     if (SC) {
@@ -120,6 +123,7 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
     }
   };
   auto emit2 = [&](int t, int i, float v0, float v1) {  // columns i, i + 1 (i even)
+    if (!EMIT) return;
     const uint32_t off = canon(t, i, 128);
     *reinterpret_cast<uint32_t*>(tp + off) = pack_bf16(SC ? v0 * cs_c[i] : v0, SC ? v1 * cs_c[i + 1] : v1);
     if (SC && TT_LO) {
@@ -228,8 +232,13 @@ __device__ __noinline__ void unit_lower_inverse(const float* sL, float* sT, floa
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     warp_mm<32>(d, [&](int i, int k) { return sT[xi(32 + 16 * mt + i, 32 + k)]; },
                 [&](int k, int n) { return X[k * 36 + 8 * nt + n]; }, lane);
-    warp_store2(d, [&](int i, int n, float v0, float v1) { emit2(32 + 16 * mt + i, 8 * nt + n, -v0, -v1); },
-                lane);
+    warp_store2(d, [&](int i, int n, float v0, float v1) {
+      if (!EMIT) {
+        sT[xi(32 + 16 * mt + i, 8 * nt + n)] = -v0;
+        sT[xi(32 + 16 * mt + i, 8 * nt + n + 1)] = -v1;
+      }
+      emit2(32 + 16 * mt + i, 8 * nt + n, -v0, -v1);
+    }, lane);
   }
   sync();
 }
