@@ -89,6 +89,10 @@ __device__ __forceinline__ float4 rcp4(float4 a) {
 // load issued before any is used: the mode branch is uniform and outside the loads, and tokens past
 // the end (i >= nvalid) re-read row tok0 + (nvalid - 1) * tstride, or row tok0 when nvalid == 0
 // (the caller points tok0 at a real token then); their values are replaced by `dflt`.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ void gate4x8(float4* out, const float* g, int mode, int64_t tok0, int64_t tstride,
                                         int width, int ch, int nvalid, float dflt) {
   if (mode == DN_GATE_CHANNEL) {
@@ -406,6 +410,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       ph_qk ^= 1;
       ph_v ^= 1;
       qk_pending = v_pending = false;
+    }
+
+    // ---- the next chunk's gate rows into L2 (their loads below are on this loop's critical path):
+    // lane l of warp tg takes the 128-byte line l % 4 of token 8 tg + l / 4 of every per-channel gate
+    if (c + 1 < nchunks) {
+      const int j = 8 * warp + (lane >> 2), line = lane & 3;
+      if (t0 + C + j < T) {
+        const int64_t tok = ((int64_t)b * T + t0 + C + j) * H + h;
+        if (a.alpha == DN_GATE_CHANNEL) prefetch_l2(a.alpha_p + tok * DK + 32 * line);
+        if (a.beta_k == DN_GATE_CHANNEL) prefetch_l2(a.beta_k_p + tok * DK + 32 * line);
+        if (a.key_scale == DN_GATE_CHANNEL) prefetch_l2(a.key_scale_p + tok * DK + 32 * line);
+        if (a.beta_v == DN_GATE_CHANNEL && 32 * line < dv) prefetch_l2(a.beta_v_p + tok * dv + 32 * line);
+      }
     }
 
     // ---- P1: decay factors and the operand tiles (or, for a chunk of too strong a decay, the rows the
