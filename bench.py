@@ -123,7 +123,10 @@ def measured_peaks() -> dict:
 
 # sources each timed kernel is built from (its recorded DRAM traffic is void once any changes)
 KERNEL_SOURCES = {
-    "chunk_fwd": ["dn_chunk_sc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
+    "chunk_fwd": ["dn_split_sc.cu", "dn_sc_factors.cuh", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu",
+                  "dn_common.cuh"],
+    "chunk_sc": ["dn_chunk_sc.cu", "dn_sc_factors.cuh", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu",
+                 "dn_common.cuh"],
     "chunk_tc": ["dn_chunk_tc.cu", "dn_ut_inverse.cuh", "dn_tc_ptx.cuh", "dn_tma.cu", "dn_common.cuh"],
     "decode": ["dn_decode.cu", "dn_common.cuh"],
     "osdn": ["dn_osdn.cu", "dn_tc_ptx.cuh", "dn_common.cuh"],
@@ -141,14 +144,15 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel sources."""
+def recorded_traffic(kernel: str, entry: str = ""):
+    """DRAM bytes per launch from the committed ncu summary (entry `entry`, default the kernel's own
+    name), if taken on the current sources of `kernel`."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kernel)
+    e = d.get(entry or kernel)
     if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
@@ -392,7 +396,7 @@ def run_config_leg(name, peaks, stream, world, barrier, to_dev, want_cpu, reps):
                          "frac": tf / peaks["bf16_tflops"], "executed_flops_per_launch": fl,
                          "peak_source": f"{peaks['source']} bf16 burst"}
         leg["roofline_time_us"] = 1e6 * max(alg / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
-        leg["traffic"] = recorded_traffic("chunk_tc")
+        leg["traffic"] = recorded_traffic("chunk_tc", f"chunk_tc:{name}")
     else:
         fl = seq_flops(w)
         tf = fl / (ms * 1e-3) / 1e12
