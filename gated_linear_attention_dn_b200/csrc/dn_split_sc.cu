@@ -324,16 +324,14 @@ __global__ void __launch_bounds__(kChainThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, const Args a,
                     const uint8_t* ws, int bv_split) {
   using Ly = CLayout<NV>;
-  constexpr int HALVES = 1;  // one state chain per CTA (its per-half barriers use index 0)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   // loads (transaction counts); products (commits); hand-overs (arrivals)
   __shared__ __align__(8) uint64_t bar_kq[2], bar_fr[2], bar_tg, bar_vb, bar_p[2];
   // (the state update, the O product and the o stores of chunk c complete barrier [c & 1]: the loader
   // looks at them a chunk later than the chain, which can never lap it by two chunks)
-  // (per value-column half hf: bar_d1[hf], bar_os[hf][p], bar_o[hf][p], bar_ostored[hf][p], bar_drain[hf])
-  __shared__ __align__(8) uint64_t bar_wk, bar_u0, bar_d1[2], bar_os[2][2], bar_o[2][2], bar_drain[2], bar_drain2;
-  __shared__ __align__(8) uint64_t bar_kconv, bar_ostored[2][2], bar_wkfree, bar_ufree, bar_wkconv;
+  __shared__ __align__(8) uint64_t bar_wk, bar_u0, bar_d1, bar_os[2], bar_o[2], bar_drain, bar_drain2;
+  __shared__ __align__(8) uint64_t bar_kconv, bar_wkfree, bar_ufree, bar_wkconv;
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, ch = (warp >> 2) & 1;
@@ -352,14 +350,11 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       mbar_init(&bar_kq[j], 1);
       mbar_init(&bar_fr[j], 1);
       mbar_init(&bar_p[j], 1);
-      mbar_init(&bar_d1[j], 1);
-      mbar_init(&bar_drain[j], 1);
-      for (int hf = 0; hf < 2; ++hf) {
-        mbar_init(&bar_os[hf][j], 1);
-        mbar_init(&bar_o[hf][j], 1);
-        mbar_init(&bar_ostored[hf][j], 1);  // the thread that issues the half's o store
-      }
+      mbar_init(&bar_os[j], 1);
+      mbar_init(&bar_o[j], 1);
     }
+    mbar_init(&bar_d1, 1);
+    mbar_init(&bar_drain, 1);
     mbar_init(&bar_tg, 1);
     mbar_init(&bar_vb, 1);
     mbar_init(&bar_wk, 1);
@@ -367,7 +362,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     mbar_init(&bar_drain2, 1);
     mbar_init(&bar_wkfree, 2);   // warps 8, 9: chunk c's Wk has been read (TM_WK free)
     mbar_init(&bar_wkconv, 2);   // warps 8, 9: chunk c's Wk rows of the [Wk; Q'] tile are written
-    mbar_init(&bar_ufree, HALVES);  // the halves' issuing threads: chunk c's U' is formed (TM_U0 free)
+    mbar_init(&bar_ufree, 1);    // thread 0: chunk c's U' is formed (the other accumulator is free)
     mbar_init(&bar_kconv, 1);    // the scaling warp: chunk c's K' and Q' rows are scaled
     fence_mbar_init();
   }
@@ -396,12 +391,6 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool { return mbar_wait_bounded(bar, parity, a.wait_ns); };
   auto wait_idle = [&](uint64_t* bar, uint32_t parity) -> bool {
     return mbar_wait_bounded_idle(bar, parity, a.wait_ns);
-  };
-  // a per-half, per-parity barrier of every half
-  auto wait_halves = [&](uint64_t (*bars)[2], int j, uint32_t parity) -> bool {
-    for (int hf = 0; hf < HALVES; ++hf)
-      if (!wait_idle(&bars[hf][j], parity)) return false;
-    return true;
   };
 
   bool failed = false;
@@ -513,9 +502,9 @@ __global__ void __launch_bounds__(kChainThreads, 1)
         }
       }
       // per chunk c: Wk(c + 1) once chunk c's Wk is converted, then T Diag(gamma) of chunk c + 2 once
-      // Wk(c + 1) has read chunk c + 1's; U0(c + 1) once U'(c) is formed; the buffers of chunk c once
-      // its products have read them (k, q: the state update; v, T Diag(beta^v): U0(c); P': the O
-      // product) and its factor record once its o rows are out
+      // Wk(c + 1) has read chunk c + 1's; U0(c + 1) once U'(c) is formed, and then the factor record
+      // of chunk c + 2; the buffers of chunk c once its products have read them (k, q: the state
+      // update; v, T Diag(beta^v): U0(c); P': the O product)
       for (int c = 0; c < nchunks && ok; ++c) {
         const bool more = c + 1 < nchunks;
         if (c == 0 && more) {
@@ -537,6 +526,9 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           pend_vb = -1;
           tc_fence_after();
           mma_u0(c + 1);
+          // chunk c's factor record has been read: by the chain up to U'(c) (its o scales are kept in
+          // registers) and by the scaling warp (kconv(c), seen above)
+          if (c + 2 < nchunks) issue_fr(c + 2);
           if (c + 2 < nchunks) {  // v and T Diag(beta^v) of chunk c + 2 once U0(c + 1) has read chunk c + 1's
             ok = wait_idle(&bar_u0, par(c + 1));
             if (!ok) break;
@@ -549,15 +541,12 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           }
         }
         if (c + 2 < nchunks) {  // (U0(c) is done: the chain saw it before signalling bar_ufree)
-          ok = wait_halves(bar_os, c & 1, par2(c));
+          ok = wait_idle(&bar_os[c & 1], par2(c));
           if (!ok) break;
           issue_kq(c + 2);
-          ok = wait_halves(bar_o, c & 1, par2(c));
+          ok = wait_idle(&bar_o[c & 1], par2(c));
           if (!ok) break;
           issue_p(c + 2);
-          ok = wait_halves(bar_ostored, c & 1, par2(c));
-          if (!ok) break;
-          issue_fr(c + 2);
         }
       }
       if (!ok) {
@@ -610,7 +599,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       scale_rows(kb(c), 0, fr->n);
       fence_proxy_async();
       // D1(c - 1) is done, so the chain has seen kconv(c - 1) before kconv(c) can complete
-      ok = c == 0 || (wait_idle(&bar_d1[0], par(c - 1)) && (HALVES == 1 || wait_idle(&bar_d1[1], par(c - 1))));
+      ok = c == 0 || wait_idle(&bar_d1, par(c - 1));
       if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_kconv);
@@ -671,17 +660,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     // (rows 64..127)
     auto tm_u = [&](int c) -> uint32_t { return tmem + Ly::TM_U + (c & 1) * NV; };
     // o rows of chunk c from rows 64..127 of its accumulator (quadrants 2, 3, meeting at barrier
-    // kBarOut), once O(c) is done: scaled, rounded and staged in shared memory, then written by one TMA
-    // store per 64 columns (the tensor map clips the rows past the sequence's end); thread 64 issues
-    // the stores. Every thread of quadrants 2 and 3 calls it with its failure state (the barrier takes
-    // all 128).
-    auto store_o = [&](int c, bool ok_in) -> bool {
-      bool okw = ok_in && wait(&bar_o[0][c & 1], par2(c));
+    // kBarOut), once O(c) is done: scaled by os (this row's o scale, read while the chunk's factor
+    // record was in), rounded and staged in shared memory, then written by one TMA store per 64
+    // columns (the tensor map clips the rows past the sequence's end); thread 64 issues the stores.
+    // Every thread of quadrants 2 and 3 calls it with its failure state (the barrier takes all 128).
+    auto store_o = [&](int c, bool ok_in, float os) -> bool {
+      bool okw = ok_in && wait(&bar_o[c & 1], par2(c));
       if (tid == 64) bulk_wait_read_all();  // the previous chunk's store has read the staging tile
       if (group_or(kBarOut, 128, !okw)) return false;
       tc_fence_after();
       const int t = 32 * (q4 - 2) + lane;
-      const float os = frec(c)->orho[t];
       uint32_t xr[NCB][32];
 #pragma unroll
       for (int cb = 0; cb < NCB; ++cb) tmem_ld32_issue(tm_u(c) + lane_base + cw + 32 * cb, xr[cb]);
@@ -705,7 +693,6 @@ __global__ void __launch_bounds__(kChainThreads, 1)
 #pragma unroll
         for (int x = 0; x < NV / 64; ++x) tma_store_4d(&tm_o, sm + Ly::OST + x * C * 128, col0 + 64 * x, h, c * C, b);
         bulk_commit();
-        mbar_arrive(&bar_ostored[0][c & 1]);  // the factor record's o scales have been read
       }
       return true;
     };
@@ -715,18 +702,18 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     // ok: this thread's waits so far succeeded; run: the group's vote at its last barrier (loops are left
     // only on a vote, so that every thread of the group reaches every barrier)
     bool ok = nchunks > 0, run = nchunks > 0;
+    float os_prev = 0.f, os_cur = 0.f;  // o scales of this thread's row (quadrants 2, 3) for chunks c - 1, c
     for (int c = 0; run && c < nchunks; ++c) {
-      // ---- the previous chunk's o rows (quadrants 2, 3): O(c - 1) is done before the state update of
-      // chunk c - 1, which they overlap
-      if (c > 0 && q4 >= 2) ok = store_o(c - 1, ok);
       // ---- the state entering chunk c -> bf16 operand tile; gamma_C S -> TM_S (fp32, where the state
       // update accumulates): after the state update of chunk c - 1
-      if (ok && c > 0) ok = wait(&bar_os[0][(c - 1) & 1], par2(c - 1));
+      if (ok && c > 0) ok = wait(&bar_os[(c - 1) & 1], par2(c - 1));
       ok = ok && wait(&bar_fr[c & 1], par2(c));
       if (ok) {
         tc_fence_after();
         const int k = 32 * q4 + lane;
         const float gl = frec(c)->glast;
+        os_prev = os_cur;
+        if (q4 >= 2) os_cur = frec(c)->orho[32 * (q4 - 2) + lane];
         uint32_t xr[NCB][32];  // every TMEM load of this thread in flight at once
         if (c == 0) {
 #pragma unroll
@@ -782,13 +769,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
             const uint64_t bd = sdesc(smem_u32(sm + Ly::SMU) + kk * 128, DK * 128, 1024);
             mma_bf16(tm_u(c), ad, bd, id_nv, 1);
           }
-          mma_commit(&bar_d1[0]);
+          mma_commit(&bar_d1);
           issued = true;
         }
       }
+      // ---- the previous chunk's o rows (quadrants 2, 3, idle until the next barrier): they lie in the
+      // other accumulator, which U0(c + 1) overwrites only after this chunk's U' is formed
+      if (c > 0 && q4 >= 2) ok = store_o(c - 1, ok, os_prev);
       // ---- U' = c (U0 - Wk S) (rows 0..63 of the accumulator) -> hi / lo tiles (the S tile is dead
       // once D1 is done)
-      ok = ok && wait(&bar_d1[0], par(c));
+      ok = ok && wait(&bar_d1, par(c));
       if (ok && q4 < 2) {
         tc_fence_after();
         const int t = 32 * q4 + lane;
@@ -833,7 +823,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           for (int kk = 0; kk < C; kk += 16)
             mma_bf16(tm_u(c), sdesc(pa + kk * 2, 16, 1024), sdesc(smem_u32(sm + Ly::SMU) + kk * 128, C * 128, 1024),
                      id_nv, 1);
-          mma_commit(&bar_o[0][c & 1]);
+          mma_commit(&bar_o[c & 1]);
           const uint32_t kt = smem_u32(kb(c));
 #pragma unroll
           for (int kk = 0; kk < C; kk += 16) {
@@ -842,15 +832,15 @@ __global__ void __launch_bounds__(kChainThreads, 1)
             mma_bf16(tmem + Ly::TM_S, ak, sdesc(smem_u32(sm + Ly::SMU + C * NV * 2) + kk * 128, C * 128, 1024),
                      id_state, 1);
           }
-          mma_commit(&bar_os[0][c & 1]);
+          mma_commit(&bar_os[c & 1]);
           mbar_arrive(&bar_ufree);  // U'(c) is formed
         }
       }
     }
     if (run) {  // (a group decision: every o-storing thread enters the barrier in store_o)
       // the last chunk's o rows and S_T = S_acc
-      if (q4 >= 2) ok = store_o(nchunks - 1, ok);
-      ok = ok && wait(&bar_os[0][(nchunks - 1) & 1], par2(nchunks - 1));
+      if (q4 >= 2) ok = store_o(nchunks - 1, ok, os_cur);
+      ok = ok && wait(&bar_os[(nchunks - 1) & 1], par2(nchunks - 1));
       if (ok) {
         tc_fence_after();
         const int k = 32 * q4 + lane;
@@ -870,8 +860,8 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     if (!ok && nchunks > 0) failed = true;
     if (!ok && tid == 0 && issued) {
       // drain: every tensor-core product thread 0 issued (one commit tracks them all)
-      mma_commit(&bar_drain[0]);
-      mbar_wait_bounded(&bar_drain[0], 0, kDrainNs);
+      mma_commit(&bar_drain);
+      mbar_wait_bounded(&bar_drain, 0, kDrainNs);
     }
   }
   if (failed && (tid & 31) == 0) atomicExch(a.status, kDevTimeout);
