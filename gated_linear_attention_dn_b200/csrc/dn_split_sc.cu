@@ -330,8 +330,12 @@ __global__ void __launch_bounds__(kChainThreads, 1)
   __shared__ __align__(8) uint64_t bar_kq[2], bar_fr[2], bar_tg, bar_vb, bar_p[2];
   // (the state update, the O product and the o stores of chunk c complete barrier [c & 1]: the loader
   // looks at them a chunk later than the chain, which can never lap it by two chunks)
-  __shared__ __align__(8) uint64_t bar_wk, bar_u0, bar_d1, bar_os[2], bar_o[2], bar_drain, bar_drain2;
-  __shared__ __align__(8) uint64_t bar_kconv, bar_wkfree, bar_ufree, bar_wkconv;
+  // (Wk(c) completes both bar_wk and bar_wkp[c & 1]: the scaling warp waits on the latter, which it
+  // cannot fall two completions behind)
+  __shared__ __align__(8) uint64_t bar_wk, bar_wkp[2], bar_u0, bar_d1, bar_os[2], bar_o[2], bar_drain, bar_drain2;
+  // (the scaling warp arrives on bar_kconv and on bar_kconvp[c & 1]: the loader, which reloads chunk
+  // c's factor record after it, waits on the latter)
+  __shared__ __align__(8) uint64_t bar_kconv, bar_kconvp[2], bar_wkfree, bar_ufree, bar_wkconv;
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, ch = (warp >> 2) & 1;
@@ -358,12 +362,16 @@ __global__ void __launch_bounds__(kChainThreads, 1)
     mbar_init(&bar_tg, 1);
     mbar_init(&bar_vb, 1);
     mbar_init(&bar_wk, 1);
+    mbar_init(&bar_wkp[0], 1);
+    mbar_init(&bar_wkp[1], 1);
     mbar_init(&bar_u0, 1);
     mbar_init(&bar_drain2, 1);
     mbar_init(&bar_wkfree, 2);   // warps 8, 9: chunk c's Wk has been read (TM_WK free)
     mbar_init(&bar_wkconv, 2);   // warps 8, 9: chunk c's Wk rows of the [Wk; Q'] tile are written
     mbar_init(&bar_ufree, 1);    // thread 0: chunk c's U' is formed (the other accumulator is free)
     mbar_init(&bar_kconv, 1);    // the scaling warp: chunk c's K' and Q' rows are scaled
+    mbar_init(&bar_kconvp[0], 1);
+    mbar_init(&bar_kconvp[1], 1);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(&s_tmem, 512);
@@ -468,6 +476,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           mma_bf16(tmem + Ly::TM_WK, ad, bk, id_wk, kk > 0);
         }
         mma_commit(&bar_wk);
+        mma_commit(&bar_wkp[c & 1]);
       };
       auto mma_u0 = [&](int c) {
         const uint32_t vb = smem_u32(sm + Ly::VB), acc = tmem + Ly::TM_U + (c & 1) * NV;
@@ -513,8 +522,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           issue_tg(1);
         }
         if (more) {
-          // (kconv(c) too: the scaling warp must have seen Wk(c) complete before Wk(c + 1) can)
-          ok = wait_idle(&bar_wkfree, par(c)) && wait_idle(&bar_kconv, par(c)) && wait_idle(&bar_tg, par(c + 1)) &&
+          ok = wait_idle(&bar_wkfree, par(c)) && wait_idle(&bar_tg, par(c + 1)) &&
                wait_idle(&bar_kq[(c + 1) & 1], par2(c + 1));
           if (!ok) break;
           pend_tg = pend_kq[(c + 1) & 1] = -1;
@@ -527,8 +535,12 @@ __global__ void __launch_bounds__(kChainThreads, 1)
           tc_fence_after();
           mma_u0(c + 1);
           // chunk c's factor record has been read: by the chain up to U'(c) (its o scales are kept in
-          // registers) and by the scaling warp (kconv(c), seen above)
-          if (c + 2 < nchunks) issue_fr(c + 2);
+          // registers) and by the scaling warp
+          if (c + 2 < nchunks) {
+            ok = wait_idle(&bar_kconvp[c & 1], par2(c));
+            if (!ok) break;
+            issue_fr(c + 2);
+          }
           if (c + 2 < nchunks) {  // v and T Diag(beta^v) of chunk c + 2 once U0(c + 1) has read chunk c + 1's
             ok = wait_idle(&bar_u0, par(c + 1));
             if (!ok) break;
@@ -594,7 +606,7 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       if (!ok) break;
       const Rec* fr = frec(c);
       scale_rows(qb(c), 64, fr->oex);  // rows 64..127 of the [Wk; Q'] tile (the tile has 128 rows)
-      ok = wait_idle(&bar_wk, par(c));   // Wk(c) has read the raw k rows
+      ok = wait_idle(&bar_wkp[c & 1], par2(c));  // Wk(c) has read the raw k rows
       if (!ok) break;
       scale_rows(kb(c), 0, fr->n);
       fence_proxy_async();
@@ -602,7 +614,10 @@ __global__ void __launch_bounds__(kChainThreads, 1)
       ok = c == 0 || wait_idle(&bar_d1, par(c - 1));
       if (!ok) break;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_kconv);
+      if (lane == 0) {
+        mbar_arrive(&bar_kconv);
+        mbar_arrive(&bar_kconvp[c & 1]);
+      }
     }
     if (!ok && nchunks > 0) failed = true;
   } else if (warp == 8 || warp == 9) {
