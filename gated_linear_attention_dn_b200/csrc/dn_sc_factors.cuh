@@ -46,17 +46,24 @@ struct Gates {
   float al, bk, d, bv, al_p;
 };
 
+// (Each value is preset and overwritten by a predicated load, so nothing waits for a load before
+// the values are used.)
 __device__ __forceinline__ Gates load_gates(const Args& a, int b, int h, int cn, int j) {
   Gates g;
   const int left = a.T - cn * C;
   const bool valid = j < left, valid_p = (j ^ 32) < left;
   const int64_t tok = ((int64_t)b * a.T + cn * C + j) * a.H + h;
   const int64_t tok_p = ((int64_t)b * a.T + cn * C + (j ^ 32)) * a.H + h;
-  g.al = (valid && a.alpha == DN_GATE_SCALAR) ? __ldg(a.alpha_p + tok) : 1.f;
-  g.bk = (valid && a.beta_k == DN_GATE_SCALAR) ? __ldg(a.beta_k_p + tok) : (valid ? 1.f : 0.f);
-  g.d = (valid && a.key_scale == DN_GATE_SCALAR) ? __ldg(a.key_scale_p + tok) : 1.f;
-  g.bv = (valid && a.beta_v == DN_GATE_SCALAR) ? __ldg(a.beta_v_p + tok) : (valid ? 1.f : 0.f);
-  g.al_p = (valid_p && a.alpha == DN_GATE_SCALAR) ? __ldg(a.alpha_p + tok_p) : 1.f;
+  g.al = 1.f;
+  g.bk = valid ? 1.f : 0.f;
+  g.d = 1.f;
+  g.bv = valid ? 1.f : 0.f;
+  g.al_p = 1.f;
+  if (valid && a.alpha == DN_GATE_SCALAR) g.al = __ldg(a.alpha_p + tok);
+  if (valid && a.beta_k == DN_GATE_SCALAR) g.bk = __ldg(a.beta_k_p + tok);
+  if (valid && a.key_scale == DN_GATE_SCALAR) g.d = __ldg(a.key_scale_p + tok);
+  if (valid && a.beta_v == DN_GATE_SCALAR) g.bv = __ldg(a.beta_v_p + tok);
+  if (valid_p && a.alpha == DN_GATE_SCALAR) g.al_p = __ldg(a.alpha_p + tok_p);
   return g;
 }
 
@@ -155,6 +162,50 @@ __device__ __forceinline__ void extract_ap(const Factors& f, uint32_t tmem_gram,
         const float fp = f.pinv[i] * pow2f(et - f.ex[i]);  // 2^{E_t - e_i} / (rho_i mu_i)
         y[e] = (i <= t - pre) ? x[8 * q8 + e] * fp : 0.f;
       }
+      *reinterpret_cast<uint4*>(pt + tc::canon_chunk(t, 4 * gch + q8, 64)) =
+          make_uint4(tc::pack_bf16(y[0], y[1]), tc::pack_bf16(y[2], y[3]), tc::pack_bf16(y[4], y[5]),
+                     tc::pack_bf16(y[6], y[7]));
+    }
+  }
+}
+
+// The same A and P' as extract_ap for a chunk whose decay exponents (ex and oex of every token) all
+// lie in [-100, 100]: then gamma_t and 1 / gamma_i are plain normal floats and the factors split
+// into a row part and a column part, (gamma_t / gamma_i) beta_i d_i = gamma_t * wg_i and
+// 2^{E_t - e_i} / (rho_i mu_i) = 2^{E_t} * pw_i, with wg_i = beta_i d_i / gamma_i and
+// pw_i = 1 / (gamma_i mu_i) precomputed per token (the powers of two are exact, so only the rounding
+// order of the mantissa products differs from extract_ap).
+__device__ __forceinline__ void extract_ap_fast(const Factors& f, const float* wg, const float* pw, uint32_t tmem_gram,
+                                                int q4, int gch, int lane, int pre, float* sL, uint8_t* pt) {
+  const uint32_t taddr = tmem_gram + ((uint32_t)(32 * q4) << 16) + 32 * gch;
+  if (q4 < 2) {
+    const int t = 32 * q4 + lane;
+    const float gt = f.rho[t] * pow2f(f.ex[t]);
+    float x[32];
+    tc::tmem_ld32(taddr, x);
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+      const int i0 = 32 * gch + 4 * e4;
+      const float4 w = *reinterpret_cast<const float4*>(wg + i0);
+      const float y0 = (i0 < t) ? x[4 * e4] * (gt * w.x) : 0.f;
+      const float y1 = (i0 + 1 < t) ? x[4 * e4 + 1] * (gt * w.y) : 0.f;
+      const float y2 = (i0 + 2 < t) ? x[4 * e4 + 2] * (gt * w.z) : 0.f;
+      const float y3 = (i0 + 3 < t) ? x[4 * e4 + 3] * (gt * w.w) : 0.f;
+      *reinterpret_cast<float4*>(sL + ut::xi(t, i0)) = make_float4(y0, y1, y2, y3);
+    }
+  } else {
+    const int t = 32 * (q4 - 2) + lane;
+    const float et = pow2f(f.oex[t]);
+    float x[32];
+    tc::tmem_ld32(taddr, x);
+#pragma unroll
+    for (int q8 = 0; q8 < 4; ++q8) {
+      const int i0 = 32 * gch + 8 * q8;
+      const float4 p0 = *reinterpret_cast<const float4*>(pw + i0), p1 = *reinterpret_cast<const float4*>(pw + i0 + 4);
+      const float pp[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = (i0 + e <= t - pre) ? x[8 * q8 + e] * (et * pp[e]) : 0.f;
       *reinterpret_cast<uint4*>(pt + tc::canon_chunk(t, 4 * gch + q8, 64)) =
           make_uint4(tc::pack_bf16(y[0], y[1]), tc::pack_bf16(y[2], y[3]), tc::pack_bf16(y[4], y[5]),
                      tc::pack_bf16(y[6], y[7]));

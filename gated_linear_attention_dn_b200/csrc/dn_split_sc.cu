@@ -118,11 +118,14 @@ __global__ void __launch_bounds__(kThreads, kXformPerSm) xform_sc_kernel(const _
   __shared__ uint32_t s_tmem;
   __shared__ __align__(16) float s_Y[2048];
   __shared__ scf::Factors s_f;
+  __shared__ __align__(16) float s_wg[C], s_pw[C];  // column factors of the fast extraction
+  __shared__ int s_wide;                            // a decay exponent of the chunk is beyond +-100
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, gch = warp >> 2;
   const int pre = a.pre_read ? 1 : 0;
   const int nchunks = (a.T + C - 1) / C;
   const int bh = blockIdx.x / nchunks, c = blockIdx.x % nchunks, b = bh / a.H, h = bh % a.H;
   uint8_t* const rec = ws + (size_t)blockIdx.x * rec_stride(BV);
+  if (tid == 0) s_wide = 0;
   const int64_t nb = (int64_t)blockIdx.x + ahead;  // the block that takes this one's place on its SM
   const bool pf = ahead > 0 && nb < (int64_t)gridDim.x;
   const int nbh = (int)(nb / nchunks), nc = (int)(nb % nchunks);
@@ -184,6 +187,11 @@ __global__ void __launch_bounds__(kThreads, kXformPerSm) xform_sc_kernel(const _
   }
   if (fw) {
     scf::token_factors(g, j, lane, pre, s_f);
+    // the column factors of the fast extraction, and whether the chunk may use it
+    const int ej = s_f.ex[j], oj = s_f.oex[j];
+    s_wg[j] = s_f.ws[j] * s_f.rhoi[j] * pow2f(-ej);
+    s_pw[j] = s_f.pinv[j] * pow2f(-ej);
+    if (ej < -100 || ej > 100 || oj < -100 || oj > 100) s_wide = 1;
     // each thread copies the entries it wrote itself
     Rec* r = reinterpret_cast<Rec*>(rec + rec_factor_off(BV));
     r->c[j] = s_f.c[j];
@@ -222,7 +230,10 @@ __global__ void __launch_bounds__(kThreads, kXformPerSm) xform_sc_kernel(const _
   // the inverse
   float* sL = reinterpret_cast<float*>(sm);
   float* sT = sL + C * C;
-  scf::extract_ap(s_f, tmem, q4, gch, lane, pre, sL, reinterpret_cast<uint8_t*>(s_Y));
+  if (s_wide)
+    scf::extract_ap(s_f, tmem, q4, gch, lane, pre, sL, reinterpret_cast<uint8_t*>(s_Y));
+  else
+    scf::extract_ap_fast(s_f, s_wg, s_pw, tmem, q4, gch, lane, pre, sL, reinterpret_cast<uint8_t*>(s_Y));
   tc_fence_before();
   __syncthreads();
   // tensor memory is no longer needed
