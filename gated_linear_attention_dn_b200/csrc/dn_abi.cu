@@ -321,8 +321,12 @@ dn_status dn_mc_readout(const dn_mc_desc* d, const void* q, const float* M, cons
   const size_t n_o = (size_t)d->B * d->T * d->H * d->d_v * es;
   const size_t n_q = (size_t)d->B * d->T * d->H * d->d_k * es;
   if (ranges_overlap(o, n_o, q, n_q)) return DN_ERR_INVALID_ARGUMENT;
+  int* status = nullptr;
+  dn_status st = status_ptr(&status);
+  if (st != DN_OK) return st;
   cudaError_t e = dn::launch_mc_readout(q, M, gates, o, d->B, d->T, d->H, d->d_k, d->d_v, d->seg_len,
-                                        d->io_dtype == DN_BF16, static_cast<cudaStream_t>(cuda_stream));
+                                        d->io_dtype == DN_BF16, status, dn::wait_limit_ns(),
+                                        static_cast<cudaStream_t>(cuda_stream));
   return e == cudaSuccess ? DN_OK : DN_ERR_CUDA;
 }
 

@@ -55,7 +55,7 @@ cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, cons
                         int T, int H, int dk, int io_bf16, float* ws, float* dout, float* dT, cudaStream_t s);
 // Memory Caching read-out (dn_memcache.cu).
 cudaError_t launch_mc_readout(const void* q, const float* M, const float* gates, void* o, int B, int T, int H,
-                              int dk, int dv, int L, int bf16, cudaStream_t s);
+                              int dk, int dv, int L, int bf16, int* status, uint64_t wait_ns, cudaStream_t s);
 // Small states (d_k, d_v in {8, 16}; dn_small.cu): chunk fwd and decode alike.
 bool small_state_supported(const Args& a);
 cudaError_t launch_small_state(const Args& a, cudaStream_t s);

@@ -61,6 +61,37 @@ def test_readout_alone_fp32():
     assert err <= 1e-5
 
 
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64), (64, 128), (64, 64)])
+@pytest.mark.parametrize("L,gated", [(128, False), (64, False), (100, False), (256, True), (100, True)])
+def test_readout_alone_bf16(dk, dv, L, gated):
+    """The tensor-core read-out (bf16 io) by itself against the sum written out in fp64 from the same
+    bf16 inputs: tiles inside one segment (one product of the summed memories), tiles over several
+    segments and ragged segment lengths (a product per memory, rows masked), and gates; the
+    tolerance is the bf16 rounding of the output."""
+    import torch
+    r = np.random.default_rng(11 + dk + dv + L)
+    B, H, T = 2, 3, 640 + 37
+    N = -(-T // L)
+    qb = torch.from_numpy(r.standard_normal((B, T, H, dk)).astype(np.float32)).bfloat16()
+    o0 = torch.from_numpy(r.standard_normal((B, T, H, dv)).astype(np.float32)).bfloat16()
+    M = r.standard_normal((B, N, H, dk, dv)).astype(np.float32) * 0.1
+    g = r.uniform(0, 1, (B, T, H, N)).astype(np.float32) if gated else None
+    o = o0.cuda()
+    dn.dn_mc_readout(qb.cuda(), dev(M), dev(g), o, seg_len=L)
+    assert dn.dn_stream_status() == dn.DN_OK
+    q64 = qb.double().numpy()
+    ref = o0.double().numpy().copy()
+    for t in range(T):
+        for s in range(t // L):
+            w = g[:, t, :, s][..., None] if gated else 1.0
+            ref[:, t] += w * np.einsum("bhk,bhkv->bhv", q64[:, t], M[:, s])
+    err = oracle.rel_l2(host_f64(o), ref)
+    print(f"[parity] mc read-out bf16 d_k={dk} d_v={dv} L={L} gated={gated}: rel-L2 {err:.3e}")
+    assert err <= 5e-3
+    # rows of the first segment are untouched
+    assert torch.equal(o[:, :L].cpu(), o0[:, :L])
+
+
 def test_mc_full_size_sampled_batches():
     """The configuration the benchmark times (GDN prefill B=8, H=16, T=4096, four segments of 1024,
     residual memory): the whole batch on the GPU; the first and last batch rows (all heads, the
