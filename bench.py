@@ -718,17 +718,23 @@ def main():
         rd_ms = timed2(mc_read, 10)
         if dn.dn_stream_status(stream) != dn.DN_OK:
             raise RuntimeError("device status after Memory Caching")
-        # cached reads: a token of segment j reads j memories, 2 d_k d_v flops each
-        flops = B * H * sum(j * L for j in range(nseg)) * 2 * dk * dv
-        fp32_peak = 148 * 4 * 32 * 2 * 1.965e9 / 1e12  # FFMA lanes x 2 flops x max clock, TFLOP/s
+        # the read-out (tensor cores, bf16 io): the rows of the tokens past the first segment read q
+        # once and read and write o once, and the memories 0 .. N-2 are read once; for the residual
+        # memory each 128-token tile multiplies by the sum of the memories it reads, split bf16 hi +
+        # lo: two M 128 x N d_v x K d_k products per tile
+        later = B * H * (T - L)
+        rd_bytes = later * (dk * 2 + 2 * dv * 2) + B * (nseg - 1) * H * dk * dv * 4
+        flops = later * 2 * dk * dv * 2
+        gbs = rd_bytes / (rd_ms * 1e-3) / 1e9
         tf = flops / (rd_ms * 1e-3) / 1e12
         mc = {"workload": "Memory Caching on gdn_prefill: 4 segments of 1024 tokens, residual memory",
               "online_ms": on_ms, "readout_ms": rd_ms, "total_ms": on_ms + rd_ms,
               "tokens_per_s": weak_scaling_rate(B * T, world, on_ms + rd_ms),
-              "readout_roofline": {"bound": "alu", "achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s",
-                                   "frac": tf / fp32_peak, "traffic": None,
-                                   "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flops x 1.965 GHz",
-                                   "algorithmic_flops_per_launch": flops}}
+              "readout_roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                                   "peak_source": peaks["source"], "algorithmic_bytes_per_launch": rd_bytes,
+                                   "tensor": {"achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                              "frac": tf / peaks["bf16_tflops"], "executed_flops_per_launch": flops}}}
         launches += 10 + 10
         del Mc
 
