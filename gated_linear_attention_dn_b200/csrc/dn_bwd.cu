@@ -26,6 +26,8 @@
 //   bwd_local  one CTA per chunk: dq, dk, dv and the gate gradients (key channels in slices of 32)
 // The two chains are sequential over chunks; all elementwise work (gates, logs, exponentials) is done
 // once per chunk by bwd_prep, so a chain step only copies its operands in (cp.async) and multiplies.
+#include <cstring>
+
 #include "dn_bwd.cuh"
 #include "dn_ut_inverse.cuh"
 
@@ -62,6 +64,7 @@ struct BwdArgs {
   float* wU;    // [BH][nc][C][dv]
   float* wdX;   // [BH][nc][dk][dv]
   float* wdVt;  // [BH][nc][C][dv]
+  int* wFlag;   // [BH][nc]: the forward's chunks beyond the factorisation's range (null in the backward)
   int nc;
 };
 
@@ -136,7 +139,7 @@ __device__ __forceinline__ int64_t token(const Args& a, int b, int h, int t) {
 // Called by all kNT threads; returns after a barrier.
 template <int NCH>
 __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, float* hb, float* Kp, float* Qp,
-                           float* Wm, float* er, float* lam, float* ehg, int tid) {
+                           float* Wm, float* er, float* lam, float* ehg, int tid, int* flag) {
   constexpr int LD = NCH + 4, PER = kC * NCH / kNT, BAT = PER < 8 ? PER : 8;
   static_assert(PER * kNT == kC * NCH && PER % BAT == 0, "work split");
   // Every loop below first loads a batch into registers and only then computes and stores to
@@ -164,13 +167,19 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
       if (t == tr) r = run;
     }
     // every exponent of the factorisation within +-80 (e^80 ~ 5.5e34), else the chunk's factors
-    // would over- or underflow fp32: report it instead of returning non-finite gradients
+    // would over- or underflow fp32: report it instead of returning non-finite gradients (the
+    // forward marks the chunk instead, and evaluates it token by token)
     bool ok = fabsf(r) <= 80.f && fabsf(run - r) <= 80.f;
     for (int t = 0; t < kC; ++t) {
       hb[t * LD + i] -= r;
       ok = ok && fabsf(hb[t * LD + i]) <= 80.f;
     }
-    if (!ok && a.status) atomicExch(a.status, kDevGateRange);
+    if (!ok) {
+      if (flag)
+        *flag = 1;
+      else if (a.status)
+        atomicExch(a.status, kDevGateRange);
+    }
     er[i] = expf(r);
     lam[i] = expf(run - r);
   }
@@ -279,7 +288,9 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
   const int c = blockIdx.x % p.nc, bh = blockIdx.x / p.nc, b = bh / a.H, h = bh % a.H;
   const int t0 = c * kC, n = min(kC, a.T - t0);
   const int64_t cb = (int64_t)bh * p.nc + c;
-  prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, p.wEh + cb * kC * DK, tid);
+  if (p.wFlag && tid == 0) p.wFlag[cb] = 0;  // (ordered before any mark by prep_chunk's first barrier)
+  prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, p.wEh + cb * kC * DK, tid,
+                 p.wFlag ? p.wFlag + cb : nullptr);
 
   // warps 0-3: L = strictly-lower(K+ W-^T) (kept in registers); warps 4-7: P = lower(Q+ W-^T), with the
   // diagonal for the post read-out and without it for the pre read-out
@@ -345,6 +356,51 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
     const int t0 = c * kC, n = min(kC, a.T - t0);
     const int64_t cb = (int64_t)bh * p.nc + c;
     __syncthreads();  // the previous chunk is done with every buffer
+    if (p.wFlag && p.wFlag[cb]) {
+      // (forward) a chunk beyond the factorisation's range: its tokens one by one, exactly, on this
+      // CTA's columns; thread (j, part) owns column j and DK / TPC rows of it, so the sums over the
+      // rows take TPC - 1 shuffles. S holds the true state before and after.
+      constexpr int TPC = kNT / DVS, RW = DK / TPC;
+      const int j = tid / TPC, part = tid % TPC, k0 = part * RW;
+      float Sr[RW];
+#pragma unroll
+      for (int r = 0; r < RW; ++r) Sr[r] = S[(k0 + r) * LDS + j];
+      for (int t = 0; t < n; ++t) {
+        const int64_t tok = token(a, b, h, t0 + t);
+        float al[RW], kk[RW], qq[RW], ws[RW];
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+          al[r] = gate_load(a.alpha_p, a.alpha, tok, DK, k0 + r);
+          kk[r] = io_load(a.k, tok * DK + k0 + r, a.io_bf16);
+          qq[r] = io_load(a.q, tok * DK + k0 + r, a.io_bf16);
+          ws[r] = gate_load(a.beta_k_p, a.beta_k, tok, DK, k0 + r) * gate_load(a.key_scale_p, a.key_scale, tok, DK, k0 + r);
+        }
+        const float vt = gate_load(a.beta_v_p, a.beta_v, tok, DV, j0 + j) * io_load(a.v, tok * DV + j0 + j, a.io_bf16);
+        float rr = 0.f, ss = 0.f, wq = 0.f;  // (alpha (.) S)^T k, the read-out's S^T q and w . q over these rows
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+          const float sb = al[r] * Sr[r];
+          rr = fmaf(sb, kk[r], rr);
+          ss = fmaf(a.pre_read ? Sr[r] : sb, qq[r], ss);
+          wq = fmaf(ws[r] * kk[r], qq[r], wq);
+          Sr[r] = sb;
+        }
+#pragma unroll
+        for (int off = 1; off < TPC; off <<= 1) {
+          rr += __shfl_xor_sync(0xffffffffu, rr, off);
+          ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          wq += __shfl_xor_sync(0xffffffffu, wq, off);
+        }
+        const float u = vt - rr;  // u_t = beta^v v_t - S_bar^T k_t
+#pragma unroll
+        for (int r = 0; r < RW; ++r) Sr[r] = fmaf(ws[r] * kk[r], u, Sr[r]);
+        // o_t = S_t^T q_t = S_bar^T q_t + (w . q) u_t; before the update: S_{t-1}^T q_t
+        if (part == 0) io_store(a.o, tok * DV + j0 + j, a.pre_read ? ss : fmaf(wq, u, ss), a.io_bf16);
+      }
+#pragma unroll
+      for (int r = 0; r < RW; ++r) S[(k0 + r) * LDS + j] = Sr[r];
+      continue;
+    }
     async_rows<kC, DK>(Kp, LDK, p.wKp + cb * kC * DK, DK, tid);
     async_rows<kC, DK>(Wm, LDK, p.wWm + cb * kC * DK, DK, tid);
     async_rows<kC, kC>(Tm, kLDC, p.wT + cb * kC * kC, kC, tid);
@@ -415,6 +471,13 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
                       *s = lam[r0 + m] * (*s + v);
                     },
                     lane);
+    }
+  }
+  if (p.wFlag) {  // (forward) S_T
+    __syncthreads();
+    for (int e = tid; e < DK * DVS; e += kNT) {
+      const int i = e / DVS, j = e % DVS;
+      a.S[((int64_t)bh * DK + i) * DV + j0 + j] = S[i * LDS + j];
     }
   }
 }
@@ -797,6 +860,47 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   }
 }
 
+// ------------------------------------------------------------------ forward outputs of the fp32 chunked forward
+// O = Q+ S_m + P U for one chunk (all d_v columns), from the prep and state kernels' workspace; the
+// chunks the state kernel evaluated exactly (marked) already have their o rows.
+template <int DK, int DV>
+__global__ void __launch_bounds__(kNT) fwd_out_kernel(BwdArgs p) {
+  extern __shared__ float4 smem4[];
+  constexpr int LDK = DK + 4, LDV = DV + 4, NI = DV / 16;
+  float* Qp = reinterpret_cast<float*>(smem4);  // [C][LDK]
+  float* Sm = Qp + kC * LDK;                     // [DK][LDV]
+  float* Pm = Sm + DK * LDV;                     // [C][kLDC]
+  float* U = Pm + kC * kLDC;                     // [C][LDV]
+  const Args& a = p.f;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x % p.nc, bh = blockIdx.x / p.nc, b = bh / a.H, h = bh % a.H;
+  const int t0 = c * kC, n = min(kC, a.T - t0);
+  const int64_t cb = (int64_t)bh * p.nc + c;
+  if (p.wFlag[cb]) return;
+  async_rows<kC, DK>(Qp, LDK, p.wQp + cb * kC * DK, DK, tid);
+  async_rows<DK, DV>(Sm, LDV, p.wSm + cb * DK * DV, DV, tid);
+  async_rows<kC, kC>(Pm, kLDC, p.wP + cb * kC * kC, kC, tid);
+  async_rows<kC, DV>(U, LDV, p.wU + cb * kC * DV, DV, tid);
+  tc::cp_async_commit();
+  tc::cp_async_wait_all();
+  __syncthreads();
+  // warp w: rows 16 (w / 2) .. +15, columns (w % 2) DV / 2 .. + DV / 2
+  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * (DV / 2);
+  float acc[1][NI][4] = {};
+  warp_gemm<1, NI, DK>(
+      acc, [&](int m, int k) { return Qp[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return Sm[k * LDV + n0 + nn]; },
+      lane);
+  warp_gemm<1, NI, kC>(
+      acc, [&](int m, int k) { return Pm[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return U[k * LDV + n0 + nn]; },
+      lane);
+  warp_epilogue(acc,
+                [&](int m, int nn, float v) {
+                  const int t = m0 + m;
+                  if (t < n) io_store(a.o, token(a, b, h, t0 + t) * DV + n0 + nn, v, a.io_bf16);
+                },
+                lane);
+}
+
 // ------------------------------------------------------------------ host side
 template <int DK>
 constexpr size_t prep_smem() {
@@ -814,6 +918,11 @@ template <int DV>
 constexpr size_t local_smem() {
   return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 5 * kC * (kDKS + 4) + 4 * kDKS +
                           3 * kC);
+}
+
+template <int DK, int DV>
+constexpr size_t out_smem() {
+  return sizeof(float) * (kC * (DK + 4) + DK * (DV + 4) + kC * kLDC + kC * (DV + 4));
 }
 
 template <class K>
@@ -841,7 +950,63 @@ cudaError_t launch_dims(const BwdArgs& p, cudaStream_t s) {
   return launch(bwd_local_kernel<DK, DV>, chunks, local_smem<DV>(), s, p);
 }
 
+template <int DK, int DV>
+cudaError_t launch_fwd32_dims(const BwdArgs& p, cudaStream_t s) {
+  constexpr int S1 = kDVS_STATE;
+  static_assert(out_smem<DK, DV>() <= 227 * 1024, "shared memory");
+  const int64_t bh = (int64_t)p.f.B * p.f.H;
+  const unsigned chunks = (unsigned)(bh * p.nc);
+  cudaError_t e;
+  if ((e = launch(bwd_prep_kernel<DK>, chunks, prep_smem<DK>(), s, p)) != cudaSuccess) return e;
+  if ((e = launch(bwd_state_kernel<DK, DV, S1>, (unsigned)(bh * (DV / S1)), state_smem<DK, S1>(), s, p)) != cudaSuccess)
+    return e;
+  return launch(fwd_out_kernel<DK, DV>, chunks, out_smem<DK, DV>(), s, p);
+}
+
+// The backward's workspace layout (the forward uses T, P, S_m, U, K+, Q+, W-, e^h, e^r and lam of
+// it), then one int per chunk.
+void set_workspace(BwdArgs& p, const Args& f, float* ws) {
+  p.nc = (f.T + kC - 1) / kC;
+  const int64_t blocks = (int64_t)f.B * f.H * p.nc;
+  p.wT = ws;
+  p.wP = p.wT + blocks * kC * kC;
+  p.wSm = p.wP + blocks * kC * kC;
+  p.wU = p.wSm + blocks * f.dk * f.dv;
+  p.wdX = p.wU + blocks * kC * f.dv;
+  p.wdVt = p.wdX + blocks * f.dk * f.dv;
+  p.wKp = p.wdVt + blocks * kC * f.dv;
+  p.wQp = p.wKp + blocks * kC * f.dk;
+  p.wWm = p.wQp + blocks * kC * f.dk;
+  p.wEh = p.wWm + blocks * kC * f.dk;
+  p.wEr = p.wEh + blocks * kC * f.dk;
+  p.wLam = p.wEr + blocks * f.dk;
+  p.wFlag = nullptr;
+}
+
 }  // namespace
+
+bool chunk_fwd32_supported(const Args& a) {
+  return (a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128) && a.chunk == kC && a.T > 0 &&
+         !(a.io_bf16 && a.dk == 128);  // (bf16 with d_k = 128 has the tcgen05 kernels)
+}
+
+size_t chunk_fwd32_workspace_bytes(const Args& a) {
+  const int64_t blocks = (int64_t)a.B * a.H * ((a.T + kC - 1) / kC);
+  const size_t flags = ((size_t)blocks * sizeof(int) + 15) & ~size_t(15);
+  return chunk_bwd_workspace_bytes(a.B, a.T, a.H, a.dk, a.dv) + flags;
+}
+
+cudaError_t launch_chunk_fwd32(const Args& f, float* ws, cudaStream_t s) {
+  BwdArgs p;
+  memset(&p, 0, sizeof(p));
+  p.f = f;
+  set_workspace(p, f, ws);
+  p.wFlag = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ws) + chunk_bwd_workspace_bytes(f.B, f.T, f.H, f.dk, f.dv));
+  if (f.dk == 128 && f.dv == 128) return launch_fwd32_dims<128, 128>(p, s);
+  if (f.dk == 128 && f.dv == 64) return launch_fwd32_dims<128, 64>(p, s);
+  if (f.dk == 64 && f.dv == 128) return launch_fwd32_dims<64, 128>(p, s);
+  return launch_fwd32_dims<64, 64>(p, s);
+}
 
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
   const int64_t nc = (T + kC - 1) / kC;
@@ -864,20 +1029,7 @@ cudaError_t launch_chunk_bwd(const Args& f, const void* dO, const float* dS_T, v
   p.gbeta_v = gbeta_v;
   p.gkey_scale = gkey_scale;
   p.gS0 = gS0;
-  p.nc = (f.T + kC - 1) / kC;
-  const int64_t blocks = (int64_t)f.B * f.H * p.nc;
-  p.wT = ws;
-  p.wP = p.wT + blocks * kC * kC;
-  p.wSm = p.wP + blocks * kC * kC;
-  p.wU = p.wSm + blocks * f.dk * f.dv;
-  p.wdX = p.wU + blocks * kC * f.dv;
-  p.wdVt = p.wdX + blocks * f.dk * f.dv;
-  p.wKp = p.wdVt + blocks * kC * f.dv;
-  p.wQp = p.wKp + blocks * kC * f.dk;
-  p.wWm = p.wQp + blocks * kC * f.dk;
-  p.wEh = p.wWm + blocks * kC * f.dk;
-  p.wEr = p.wEh + blocks * kC * f.dk;
-  p.wLam = p.wEr + blocks * f.dk;
+  set_workspace(p, f, ws);
   if (f.dk == 128 && f.dv == 128) return launch_dims<128, 128>(p, s);
   if (f.dk == 128 && f.dv == 64) return launch_dims<128, 64>(p, s);
   if (f.dk == 64 && f.dv == 128) return launch_dims<64, 128>(p, s);

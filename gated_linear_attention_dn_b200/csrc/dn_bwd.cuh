@@ -15,6 +15,15 @@ cudaError_t launch_chunk_bwd(const Args& f, const void* dO, const float* dS_T, v
                              float* galpha, float* gbeta_k, float* gbeta_v, float* gkey_scale, float* gS0, float* ws,
                              cudaStream_t s);
 
+// The chunked forward in fp32 (fp32 io, or bf16 with d_k = 64) on the backward's chunk machinery:
+// the prep kernel (every chunk's K+, Q+, W-, T and P), the state chain (S_m and U per chunk, S_T),
+// and the outputs O = Q+ S_m + P U per chunk; a chunk whose decay is beyond the factorisation's
+// range is evaluated token by token in the state chain. Workspace: the backward's plus one int per
+// chunk.
+bool chunk_fwd32_supported(const Args& a);
+size_t chunk_fwd32_workspace_bytes(const Args& a);
+cudaError_t launch_chunk_fwd32(const Args& f, float* ws, cudaStream_t s);
+
 // Small states (d_k, d_v in {8, 16}; dn_small_bwd.cu), either read-out: the state entering every
 // token is kept in the workspace (B * H * T * d_k * d_v fp32).
 size_t small_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);

@@ -120,8 +120,25 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.dn_decode_step(ctypes.byref(d), *bad) == dn.DN_ERR_INVALID_ARGUMENT
 
 
+def _fwd32_bytes(B, T, H, dk, dv):
+    """The fp32 chunked forward's workspace: the backward's chunk quantities (T, P: 64 x 64; S_m, dX:
+    d_k x d_v; U, dV~: 64 x d_v; K+, Q+, W-, e^h: 64 x d_k; e^r, lam: d_k; fp32) per (b, h, chunk), then
+    one int per chunk, rounded up to 16 bytes."""
+    nc = -(-T // 64)
+    per = 2 * 64 * 64 + 2 * dk * dv + 2 * 64 * dv + 4 * 64 * dk + 2 * dk
+    flags = (B * H * nc * 4 + 15) // 16 * 16
+    return B * H * nc * per * 4 + flags
+
+
 def test_workspace_query(lib):
-    assert dn.dn_chunk_fwd_workspace_bytes(_desc()) == 0
+    # bf16 with d_k = 64 and fp32 io take the fp32 chunked forward through a workspace
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc()) == _fwd32_bytes(1, 8, 2, 64, 64)
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(io_dtype=dn.DN_F32, d_k=128, d_v=64, T=130)) == \
+        _fwd32_bytes(1, 130, 2, 128, 64)
+    # small states and per-channel bf16 d_k = 128 take none
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(d_k=8, d_v=8)) == 0
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL)) == 0
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(T=0)) == 0
     assert lib.dn_chunk_fwd_workspace_bytes(None) == 0
 
 
@@ -276,7 +293,8 @@ def test_chunk_fwd_workspace_checks(lib):
     need = lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(d))
     assert need == 2 * 2 * 25616  # B H chunks x record
     assert lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(_desc(d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL))) == 0
-    assert lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(_desc(d_k=128, d_v=128, io_dtype=dn.DN_F32))) == 0
+    assert lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(_desc(d_k=128, d_v=128, io_dtype=dn.DN_F32))) == \
+        _fwd32_bytes(1, 8, 2, 128, 128)
     big = np.zeros(1 << 20, dtype=np.uint8)
     ws = ctypes.c_void_p((big.ctypes.data + 15) & ~15)
     bufs = {n: _Buf(1 << 18) for n in ("q", "k", "v", "a", "bk", "o", "st")}
