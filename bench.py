@@ -341,7 +341,7 @@ def run_single_kernel(args):
 
 CONFIG_LEGS = {
     "gdn_fp32_small": "B=1 H=2 T=256 d_k=d_v=64 fp32 q/k/v, alpha~U(0.9,1) and beta per token, S0=0 "
-                      "(sequential fp32 kernel)",
+                      "(chunk form in fp32: three kernels on split-TF32 warp tensor cores)",
     "kda": "B=4 H=32 T=8192 d_k=d_v=128 bf16 q/k/v, channel alpha, beta per token, S0~N(0,0.02^2)",
     "fg2_osdn_long": "B=2 H=16 T=32768 d_k=d_v=128 bf16 q/k/v, channel alpha, beta^k, beta^v, OSDN d, "
                      "S0~N(0,0.02^2)",
@@ -403,7 +403,7 @@ def run_config_leg(name, peaks, stream, world, barrier, to_dev, want_cpu, reps):
         fp32_peak = 148 * 4 * 32 * 2 * 1.965e9 / 1e12
         leg["alu"] = {"achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s", "frac": tf / fp32_peak,
                       "flops_per_launch": fl, "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flops x 1.965 GHz",
-                      "note": "a sequential chain of T tokens per head: launch and latency bound at this size"}
+                      "note": "4 chunks per head in sequence over 3 kernels: launch and latency bound at this size"}
     if want_cpu:
         import oracle
         oracle.build()

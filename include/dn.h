@@ -123,7 +123,16 @@ typedef struct {
  *    state-chain kernel reads it back; the faster form;
  *  - with workspace == NULL: one fused kernel per (b, h) that keeps everything on
  *    chip, at some cost in speed.
- * Both give the same results up to rounding. Other problems take no workspace.
+ * Problems in fp32 io, and bf16 with d_k = 64 (d_k, d_v in {64, 128}), also have two:
+ *  - with a workspace of at least this size: the chunk form in fp32 (split-TF32 warp
+ *    tensor-core products, about fp32 accuracy): a kernel forms every chunk's decay-scaled
+ *    keys, queries and write keys, UT transform and scores (fp32, ~164 KB per (b, h, chunk)
+ *    at d = 64, ~361 KB at d = 128), the state chain walks the chunks, and a third kernel
+ *    forms the outputs; a chunk whose decay over half a chunk exceeds e^80 per channel is
+ *    evaluated token by token inside the chain;
+ *  - with workspace == NULL: the sequential fp32 kernel, token by token.
+ * Both give the same results up to rounding. Other problems (small states, per-channel
+ * gates at bf16 d_k = 128) take no workspace.
  */
 size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc);
 
