@@ -193,27 +193,48 @@ __global__ void __launch_bounds__(256) mc_readout_tc_kernel(const __grid_constan
   bool ok = true, issued = false, q_seen = false;
   for (int s = 0; s < passes && ok; ++s) {
     // the memory (or the sum of memories 0 .. jmax - 1) as bf16 hi + lo tiles, 16-byte chunks of
-    // 8 columns: consecutive threads take consecutive chunks of a row
-    for (int e = tid; e < DK * DV / 8; e += 256) {
-      const int k = e / (DV / 8), x8 = e % (DV / 8);
-      const float* src = Mb + (int64_t)s * mstride + (int64_t)k * DV + 8 * x8;
-      float4 a0 = *reinterpret_cast<const float4*>(src), a1 = *reinterpret_cast<const float4*>(src + 4);
+    // 8 columns: consecutive threads take consecutive chunks of a row; every load of a memory is in
+    // flight before any of it is used
+    {
+      constexpr int PER = DK * DV / 8 / 256;  // chunks per thread
+      static_assert(PER * 256 * 8 == DK * DV, "work split");
+      float4 m0[PER], m1[PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int e = tid + 256 * i, k = e / (DV / 8), x8 = e % (DV / 8);
+        const float* src = Mb + (int64_t)s * mstride + (int64_t)k * DV + 8 * x8;
+        m0[i] = *reinterpret_cast<const float4*>(src);
+        m1[i] = *reinterpret_cast<const float4*>(src + 4);
+      }
       if (!MASKED) {
         for (int s2 = 1; s2 < jmax; ++s2) {
-          const float4 y0 = *reinterpret_cast<const float4*>(src + s2 * mstride);
-          const float4 y1 = *reinterpret_cast<const float4*>(src + s2 * mstride + 4);
-          a0.x += y0.x, a0.y += y0.y, a0.z += y0.z, a0.w += y0.w;
-          a1.x += y1.x, a1.y += y1.y, a1.z += y1.z, a1.w += y1.w;
+          float4 y0[PER], y1[PER];
+#pragma unroll
+          for (int i = 0; i < PER; ++i) {
+            const int e = tid + 256 * i, k = e / (DV / 8), x8 = e % (DV / 8);
+            const float* src = Mb + s2 * mstride + (int64_t)k * DV + 8 * x8;
+            y0[i] = *reinterpret_cast<const float4*>(src);
+            y1[i] = *reinterpret_cast<const float4*>(src + 4);
+          }
+#pragma unroll
+          for (int i = 0; i < PER; ++i) {
+            m0[i].x += y0[i].x, m0[i].y += y0[i].y, m0[i].z += y0[i].z, m0[i].w += y0[i].w;
+            m1[i].x += y1[i].x, m1[i].y += y1[i].y, m1[i].z += y1[i].z, m1[i].w += y1[i].w;
+          }
         }
       }
-      uint4 hi, lo;
-      split_bf16(a0.x, a0.y, hi.x, lo.x);
-      split_bf16(a0.z, a0.w, hi.y, lo.y);
-      split_bf16(a1.x, a1.y, hi.z, lo.z);
-      split_bf16(a1.z, a1.w, hi.w, lo.w);
-      const uint32_t off = canon_chunk(k, x8, DK);
-      *reinterpret_cast<uint4*>(sm + Ly::BH + off) = hi;
-      *reinterpret_cast<uint4*>(sm + Ly::BL + off) = lo;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int e = tid + 256 * i, k = e / (DV / 8), x8 = e % (DV / 8);
+        uint4 hi, lo;
+        split_bf16(m0[i].x, m0[i].y, hi.x, lo.x);
+        split_bf16(m0[i].z, m0[i].w, hi.y, lo.y);
+        split_bf16(m1[i].x, m1[i].y, hi.z, lo.z);
+        split_bf16(m1[i].z, m1[i].w, hi.w, lo.w);
+        const uint32_t off = canon_chunk(k, x8, DK);
+        *reinterpret_cast<uint4*>(sm + Ly::BH + off) = hi;
+        *reinterpret_cast<uint4*>(sm + Ly::BL + off) = lo;
+      }
     }
     if (MASKED) {
       // this memory's gate of every token of the tile (0 when the token does not read it)
