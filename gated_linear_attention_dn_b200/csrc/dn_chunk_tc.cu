@@ -85,14 +85,14 @@ __device__ __forceinline__ float4 rcp4(float4 a) {
   return make_float4(__fdividef(1.f, a.x), __fdividef(1.f, a.y), __fdividef(1.f, a.z), __fdividef(1.f, a.w));
 }
 
-// Gate values of 8 tokens (rows tok0 + i * tstride, i < 8) for 4 consecutive channels, with every
-// load issued before any is used: the mode branch is uniform and outside the loads, and tokens past
-// the end (i >= nvalid) re-read row tok0 + (nvalid - 1) * tstride, or row tok0 when nvalid == 0
-// (the caller points tok0 at a real token then); their values are replaced by `dflt`.
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
 }
 
+// Gate values of 8 tokens (rows tok0 + i * tstride, i < 8) for 4 consecutive channels, with every
+// load issued before any is used: the mode branch is uniform and outside the loads, and tokens past
+// the end (i >= nvalid) re-read row tok0 + (nvalid - 1) * tstride, or row tok0 when nvalid == 0
+// (the caller points tok0 at a real token then); their values are replaced by `dflt`.
 __device__ __forceinline__ void gate4x8(float4* out, const float* g, int mode, int64_t tok0, int64_t tstride,
                                         int width, int ch, int nvalid, float dflt) {
   if (mode == DN_GATE_CHANNEL) {
@@ -309,6 +309,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, col0 + 64 * x, h, c * C, b);
   };
 
+  // gate values of a chunk for this thread (tokens 8 warp .. + 7, channels 4 lane .. + 3; beta^v for
+  // value columns col0 + 4 lane .. + 3), loaded one chunk ahead so that their latency overlaps the
+  // previous chunk's products
+  // (beta^v too when the value columns are split: with 128 columns the registers are not there)
+  constexpr bool kAheadBv = NV < 128;
+  float4 g_al[8], g_ws[8], g_dd[8], g_bv[8];
+  auto load_gates = [&](int c) {
+    const int nvalid = max(0, min(8, min(C, T - c * C) - 8 * warp));
+    const int64_t tok0 = ((int64_t)b * T + c * C + (nvalid > 0 ? 8 * warp : 0)) * H + h;
+    gate4x8(g_al, a.alpha_p, a.alpha, tok0, H, DK, 4 * lane, nvalid, 1.f);
+    gate4x8(g_ws, a.beta_k_p, a.beta_k, tok0, H, DK, 4 * lane, nvalid, 0.f);
+    gate4x8(g_dd, a.key_scale_p, a.key_scale, tok0, H, DK, 4 * lane, nvalid, 0.f);
+    if (kAheadBv && a.beta_v != DN_GATE_ONE && 4 * lane < NV)
+      gate4x8(g_bv, a.beta_v_p, a.beta_v, tok0, H, dv, col0 + 4 * lane, nvalid, 0.f);
+  };
+  if (nchunks > 0) load_gates(0);
+
   uint32_t ph_qk = 0, ph_v = 0, ph_mma = 0;
   bool qk_pending = false, v_pending = false, mma_pending = false;
   bool o_pending = false;  // the previous chunk's outputs are still in D1 (stored during this chunk)
@@ -412,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       qk_pending = v_pending = false;
     }
 
-    // ---- the next chunk's gate rows into L2 (their loads below are on this loop's critical path):
+    // ---- the next chunk's gate rows into L2, ahead of their loads at the end of this chunk:
     // lane l of warp tg takes the 128-byte line l % 4 of token 8 tg + l / 4 of every per-channel gate
     if (c + 1 < nchunks) {
       const int j = 8 * warp + (lane >> 2), line = lane & 3;
@@ -431,15 +448,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       // per-channel path: thread (g4, tg) owns channels 4g4..4g4+3 of tokens 8tg..8tg+7
       const int g4 = lane, tg = warp, cb0 = 4 * g4;
+      if (bv_split && cb0 < NV) {
+        // V~ = beta^v (.) v, split hi (in place) / lo
+        if (!kAheadBv) {
+          const int nvalid = max(0, min(8, n - 8 * tg));
+          const int64_t tok0 = ((int64_t)b * T + t0 + (nvalid > 0 ? 8 * tg : 0)) * H + h;
+          gate4x8(g_bv, a.beta_v_p, a.beta_v, tok0, H, dv, col0 + cb0, nvalid, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = 8 * tg + i;
+          const float4 bv = g_bv[i];
+          const uint32_t off2 = canon(j, cb0, C);
+          const float4 vv = unpack4(*reinterpret_cast<const uint2*>(sm + Ly::STV + off2));
+          uint2 hi, lo;
+          split4(mul4(vv, bv), hi, lo);
+          *reinterpret_cast<uint2*>(sm + Ly::STV + off2) = hi;
+          *reinterpret_cast<uint2*>(sm + Ly::VLO + off2) = lo;
+        }
+      }
+      // tokens 8 tg .. 8 tg + 7 of this chunk (gates loaded during the previous chunk)
       float4 al[8], ws[8], dd[8];
       uint2 kr[8], qr[8];
-      // tokens 8 tg .. 8 tg + 7 of this chunk; a group wholly past the end reads token 0 of the
-      // chunk (always a real token) and discards it
-      const int nvalid = max(0, min(8, n - 8 * tg));
-      const int64_t tok0 = ((int64_t)b * T + t0 + (nvalid > 0 ? 8 * tg : 0)) * H + h;
-      gate4x8(al, a.alpha_p, a.alpha, tok0, H, DK, cb0, nvalid, 1.f);
-      gate4x8(ws, a.beta_k_p, a.beta_k, tok0, H, DK, cb0, nvalid, 0.f);
-      gate4x8(dd, a.key_scale_p, a.key_scale, tok0, H, DK, cb0, nvalid, 0.f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) al[i] = g_al[i], ws[i] = g_ws[i], dd[i] = g_dd[i];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int j = 8 * tg + i;
@@ -534,22 +566,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint2*>(sm + Ly::WHI + canon(j, cb0, C)) = hi;
         *reinterpret_cast<uint2*>(sm + Ly::WLO + canon(j, cb0, C)) = lo;
       }
-      if (bv_split && cb0 < NV) {
-        // V~ = beta^v (.) v, split hi (in place) / lo
-        float4 bvs[8];
-        gate4x8(bvs, a.beta_v_p, a.beta_v, tok0, H, dv, col0 + cb0, nvalid, 0.f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int j = 8 * tg + i;
-          const float4 bv = bvs[i];
-          const uint32_t off2 = canon(j, cb0, C);
-          const float4 vv = unpack4(*reinterpret_cast<const uint2*>(sm + Ly::STV + off2));
-          uint2 hi, lo;
-          split4(mul4(vv, bv), hi, lo);
-          *reinterpret_cast<uint2*>(sm + Ly::STV + off2) = hi;
-          *reinterpret_cast<uint2*>(sm + Ly::VLO + off2) = lo;
-        }
-      }
     }
     __syncthreads();
 
@@ -576,6 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_v(c + 1);
       }
       if (c + 1 < nchunks) qk_pending = v_pending = true;
+      load_gates(min(c + 1, nchunks - 1));
       continue;
     }
 
@@ -782,6 +799,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bar_mma);
     }
     mma_pending = true;
+    // (unconditional, the last chunk re-reading itself: the arrays are then dead from P1 to here)
+    load_gates(min(c + 1, nchunks - 1));
     {
       bool ok = mbar_wait_bounded(&bar_mma, ph_mma, a.wait_ns);
       if (__syncthreads_or(!ok)) {
