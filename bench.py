@@ -348,6 +348,41 @@ CONFIG_LEGS = {
 }
 
 
+def time_chunk_lengths(w, xd, o, ST, stream, world, chunks, reps, flush=None):
+    """ms per dn_chunk_fwd call for each chunk length in `chunks` on the same device inputs (each with
+    its own workspace): 64 is the tensor-core kernels' tile; 16 and 32 run the chunk form in fp32."""
+    import torch
+
+    import gated_linear_attention_dn_b200 as dn
+    out = {}
+    for C in chunks:
+        desc = dn.make_desc(xd["q"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"], chunk=C)
+        ws = torch.empty(max(dn.dn_chunk_fwd_workspace_bytes(desc), 16), dtype=torch.uint8, device="cuda")
+
+        def call():
+            dn.dn_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
+                            xd["S0"], o=o, S_T=ST, stream=stream, chunk=C, workspace=ws)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(reps):
+            if flush is not None:
+                flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        if dn.dn_stream_status(stream) != dn.DN_OK:
+            raise RuntimeError(f"device status after chunk = {C}")
+        out[str(C)] = reduce_max(tot / reps, world)
+        del ws
+    return out
+
+
 def run_config_leg(name, peaks, stream, world, barrier, to_dev, want_cpu, reps):
     """One dn_chunk_fwd workload of the pages' configurations: ms per call, tokens/s, the HBM and tensor
     roofline fractions, and (rank 0, one GPU) the fp64 oracle on whole heads of the same workload."""
@@ -404,6 +439,13 @@ def run_config_leg(name, peaks, stream, world, barrier, to_dev, want_cpu, reps):
         leg["alu"] = {"achieved": tf, "peak": fp32_peak, "unit": "TFLOP/s", "frac": tf / fp32_peak,
                       "flops_per_launch": fl, "peak_source": "fp32 FFMA: 148 SMs x 128 lanes x 2 flops x 1.965 GHz",
                       "note": "4 chunks per head in sequence over 3 kernels: launch and latency bound at this size"}
+    # the other chunk lengths: 16 and 32 in the chunk form in fp32 (all three for fp32 io)
+    by_chunk = time_chunk_lengths(w, xd, o, ST, stream, world, (16, 32) if w.io == "f32" else (32,),
+                                  reps=reps if w.io == "f32" else 2, flush=flush)
+    by_chunk["64"] = ms
+    leg["chunk_lengths"] = {"ms_per_call": by_chunk, "best": int(min(by_chunk, key=by_chunk.get)),
+                            "note": "64: the default evaluation above; 16 and 32: the chunk form in fp32 "
+                                    "(split-TF32 warp tensor cores) with that chunk length"}
     if want_cpu:
         import oracle
         oracle.build()
@@ -546,6 +588,10 @@ def main():
                 "scope": f"the whole dn_chunk_fwd call ({kernels_per_step} kernels: chunk-parallel transform, then "
                          "the state chain), CUDA events on the launching stream",
                 "fused_ms": fused_ms, "fused_frac": alg / (fused_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    # 32-token chunks on the same inputs (the chunk form in fp32; the tensor-core kernels' tile is 64)
+    by_chunk = time_chunk_lengths(w, xd, o, ST, stream, world, (32,), reps=2)
+    by_chunk["64"] = kern_ms
+    roofline["chunk_lengths"] = {"ms_per_call": by_chunk, "best": int(min(by_chunk, key=by_chunk.get))}
 
     # ---- end to end: pinned host buffers, H2D of the step's inputs, D2H of o and S_T
     pin = {n: (None if t is None else t.cpu().pin_memory()) for n, t in xd.items()}
@@ -615,6 +661,7 @@ def main():
     # ---- decode workload
     decode = None
     launches = kernels_per_step * args.steps
+    launches += 2 * 3  # the two timed calls with 32-token chunks (three kernels each)
     if not args.no_decode:
         wd = di.WORKLOADS[DECODE]
         nd = args.decode_steps
@@ -716,6 +763,8 @@ def main():
                                            want_cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline),
                                            reps=reps)
             launches += reps
+            # the timed calls with other chunk lengths (three kernels each)
+            launches += 3 * (2 * reps if di.WORKLOADS[name].io == "f32" else 2)
 
     # ---- Memory Caching on the prefill workload: 4 segments of 1024 tokens, residual memory
     mc = None

@@ -52,7 +52,7 @@ dn_status check_desc(const dn_desc* d, bool decode) {
   const bool big = (d->d_k == 64 || d->d_k == 128) && (d->d_v == 64 || d->d_v == 128);
   const bool small = (d->d_k == 8 || d->d_k == 16) && (d->d_v == 8 || d->d_v == 16);
   if (!big && !small) return DN_ERR_UNSUPPORTED;
-  if (!(d->chunk == 0 || d->chunk == 64)) return DN_ERR_UNSUPPORTED;
+  if (!(d->chunk == 0 || d->chunk == 16 || d->chunk == 32 || d->chunk == 64)) return DN_ERR_UNSUPPORTED;
   // sizes must stay addressable with 32-bit grid math and 64-bit offsets
   const int64_t heads = (int64_t)d->B * d->H;
   if (heads * 2 >= (int64_t)1 << 31) return DN_ERR_UNSUPPORTED;
@@ -347,6 +347,7 @@ dn_status check_bwd_desc(const dn_desc* d) {
   dn_status st = check_desc(d, false);
   if (st != DN_OK) return st;
   if (small_dims(d)) return DN_OK;
+  if (!(d->chunk == 0 || d->chunk == 64)) return DN_ERR_UNSUPPORTED;  // (its chunks are 64 tokens)
   const int64_t blocks = (int64_t)d->B * d->H * ((d->T + 63) / 64);
   if (blocks >= ((int64_t)1 << 31)) return DN_ERR_UNSUPPORTED;
   return DN_OK;

@@ -137,11 +137,11 @@ __device__ __forceinline__ int64_t token(const Args& a, int b, int h, int t) {
 // Wm itself), er = e^r, lam = e^{g_last - r}; e^h also to global ehg ([C][NCH]) when not null.
 // Tokens past the end have k = q = w = 0 and alpha = 1.
 // Called by all kNT threads; returns after a barrier.
-template <int NCH>
+template <int NCH, int C = kC>
 __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, float* hb, float* Kp, float* Qp,
                            float* Wm, float* er, float* lam, float* ehg, int tid, int* flag) {
-  constexpr int LD = NCH + 4, PER = kC * NCH / kNT, BAT = PER < 8 ? PER : 8;
-  static_assert(PER * kNT == kC * NCH && PER % BAT == 0, "work split");
+  constexpr int LD = NCH + 4, PER = C * NCH / kNT, BAT = PER < 8 ? PER : 8;
+  static_assert(PER * kNT == C * NCH && PER % BAT == 0, "work split");
   // Every loop below first loads a batch into registers and only then computes and stores to
   // shared memory, so a thread's global loads are all in flight at once.
   {
@@ -161,7 +161,7 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
   const int tr = (n - 1) / 2;
   for (int i = tid; i < NCH; i += kNT) {
     float run = 0.f, r = 0.f;
-    for (int t = 0; t < kC; ++t) {
+    for (int t = 0; t < C; ++t) {
       run += hb[t * LD + i];
       hb[t * LD + i] = run;
       if (t == tr) r = run;
@@ -170,7 +170,7 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
     // would over- or underflow fp32: report it instead of returning non-finite gradients (the
     // forward marks the chunk instead, and evaluates it token by token)
     bool ok = fabsf(r) <= 80.f && fabsf(run - r) <= 80.f;
-    for (int t = 0; t < kC; ++t) {
+    for (int t = 0; t < C; ++t) {
       hb[t * LD + i] -= r;
       ok = ok && fabsf(hb[t * LD + i]) <= 80.f;
     }
@@ -228,13 +228,17 @@ __device__ __forceinline__ void async_rows(float* sm, int ss, const float* g, in
   }
 }
 
-// T = (I + L)^-1 for the strictly lower 64 x 64 L in Lm (row stride LDC) into Tm (same stride), fp32.
-// The four 16 x 16 diagonal blocks by forward substitution (one column per thread), then the blocks
-// below the diagonal by block distance d: T_ij = -T_ii sum_{j <= k < i} L_ik T_kj. scr: 768 floats.
-__device__ void inverse64(const float* Lm, float* Tm, float* scr, int tid) {
-  for (int e = tid; e < kC * kC; e += kNT) Tm[(e / kC) * kLDC + e % kC] = 0.f;
+// T = (I + L)^-1 for the strictly lower C x C L in Lm (row stride C + 4) into Tm (same stride), fp32.
+// The C / 16 diagonal blocks of 16 x 16 by forward substitution (one column per thread), then the
+// blocks below the diagonal by block distance d: T_ij = -T_ii sum_{j <= k < i} L_ik T_kj.
+// scr: 768 floats.
+template <int C>
+__device__ void inverse_blocked(const float* Lm, float* Tm, float* scr, int tid) {
+  constexpr int LDC = C + 4, NB = C / 16;
+  static_assert(C % 16 == 0 && NB <= 4, "16-row blocks, scratch for four");
+  for (int e = tid; e < C * C; e += kNT) Tm[(e / C) * LDC + e % C] = 0.f;
   __syncthreads();
-  if (tid < 64) {
+  if (tid < C) {
     const int o = (tid >> 4) * 16, j = tid & 15;
     float x[16];
 #pragma unroll
@@ -243,19 +247,19 @@ __device__ void inverse64(const float* Lm, float* Tm, float* scr, int tid) {
     for (int i = 1; i < 16; ++i) {
       float s = 0.f;
 #pragma unroll
-      for (int k = 0; k < i; ++k) s = fmaf(Lm[(o + i) * kLDC + o + k], x[k], s);
+      for (int k = 0; k < i; ++k) s = fmaf(Lm[(o + i) * LDC + o + k], x[k], s);
       if (i > j) x[i] = -s;
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) Tm[(o + i) * kLDC + o + j] = x[i];
+    for (int i = 0; i < 16; ++i) Tm[(o + i) * LDC + o + j] = x[i];
   }
   __syncthreads();
-  for (int d = 1; d < 4; ++d) {
-    const int np = 4 - d;
+  for (int d = 1; d < NB; ++d) {
+    const int np = NB - d;
     for (int e = tid; e < np * 256; e += kNT) {
       const int bj = e >> 8, bi = bj + d, r = (e >> 4) & 15, col = e & 15;
       float s = 0.f;
-      for (int k = bj * 16; k < bi * 16; ++k) s = fmaf(Lm[(bi * 16 + r) * kLDC + k], Tm[k * kLDC + bj * 16 + col], s);
+      for (int k = bj * 16; k < bi * 16; ++k) s = fmaf(Lm[(bi * 16 + r) * LDC + k], Tm[k * LDC + bj * 16 + col], s);
       scr[e] = s;
     }
     __syncthreads();
@@ -263,22 +267,23 @@ __device__ void inverse64(const float* Lm, float* Tm, float* scr, int tid) {
       const int bj = e >> 8, bi = bj + d, r = (e >> 4) & 15, col = e & 15;
       float s = 0.f;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) s = fmaf(Tm[(bi * 16 + r) * kLDC + bi * 16 + k], scr[(bj << 8) + (k << 4) + col], s);
-      Tm[(bi * 16 + r) * kLDC + bj * 16 + col] = -s;
+      for (int k = 0; k < 16; ++k) s = fmaf(Tm[(bi * 16 + r) * LDC + bi * 16 + k], scr[(bj << 8) + (k << 4) + col], s);
+      Tm[(bi * 16 + r) * LDC + bj * 16 + col] = -s;
     }
     __syncthreads();
   }
 }
 
 // ------------------------------------------------------------------ kernel 1: per-chunk operands
-template <int DK>
+// (C tokens per chunk: 64 for the backward; the forward takes 16, 32 or 64)
+template <int DK, int C = kC>
 __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4;
+  constexpr int LDK = DK + 4, LDC = C + 4;
   float* Kp = reinterpret_cast<float*>(smem4);
-  float* Qp = Kp + kC * LDK;
-  float* Wm = Qp + kC * LDK;
-  float* scr = Wm + kC * LDK;
+  float* Qp = Kp + C * LDK;
+  float* Wm = Qp + C * LDK;
+  float* scr = Wm + C * LDK;
   float* er = scr + 768;
   float* lam = er + DK;
   float* Lm = Kp;  // once K+ and Q+ are consumed, their space holds L and T
@@ -286,26 +291,32 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x % p.nc, bh = blockIdx.x / p.nc, b = bh / a.H, h = bh % a.H;
-  const int t0 = c * kC, n = min(kC, a.T - t0);
+  const int t0 = c * C, n = min(C, a.T - t0);
   const int64_t cb = (int64_t)bh * p.nc + c;
   if (p.wFlag && tid == 0) p.wFlag[cb] = 0;  // (ordered before any mark by prep_chunk's first barrier)
-  prep_chunk<DK>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, p.wEh + cb * kC * DK, tid,
-                 p.wFlag ? p.wFlag + cb : nullptr);
+  prep_chunk<DK, C>(a, b, h, t0, n, 0, Wm, Kp, Qp, Wm, er, lam, p.wEh ? p.wEh + cb * C * DK : nullptr, tid,
+                    p.wFlag ? p.wFlag + cb : nullptr);
 
   // warps 0-3: L = strictly-lower(K+ W-^T) (kept in registers); warps 4-7: P = lower(Q+ W-^T), with the
-  // diagonal for the post read-out and without it for the pre read-out
-  const int m0 = ((warp & 3) >> 1) * 32, n0 = (warp & 1) * 32;
-  float acc[2][4][4] = {};
-  {
+  // diagonal for the post read-out and without it for the pre read-out. Warp tiles of WM x WN: 32 x 32
+  // (C = 64), 16 x 16 (C = 32: four per product; C = 16: one, the other three warps of the four idle)
+  constexpr int MI = C >= 64 ? 2 : 1, NI = C >= 64 ? 4 : 2, WM = 16 * MI, WN = 8 * NI;
+  constexpr int NWN = C / WN, NW = (C / WM) * NWN;
+  static_assert(NW <= 4, "four warps per product");
+  const int wi = warp & 3;
+  const bool gram = wi < NW;
+  const int m0 = (wi / NWN) * WM, n0 = (wi % NWN) * WN;
+  float acc[MI][NI][4] = {};
+  if (gram) {
     const float* X = warp < 4 ? Kp : Qp;
-    warp_gemm<2, 4, DK>(
+    warp_gemm<MI, NI, DK>(
         acc, [&](int m, int k) { return X[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return Wm[(n0 + nn) * LDK + k]; },
         lane);
   }
-  if (warp >= 4) {
-    float* P = p.wP + cb * kC * kC;
+  if (warp >= 4 && gram) {
+    float* P = p.wP + cb * C * C;
     const int diag = a.pre_read ? 0 : 1;  // the pre read-out excludes the token's own write
-    warp_epilogue(acc, [&](int m, int nn, float v) { P[(m0 + m) * kC + n0 + nn] = n0 + nn < m0 + m + diag ? v : 0.f; },
+    warp_epilogue(acc, [&](int m, int nn, float v) { P[(m0 + m) * C + n0 + nn] = n0 + nn < m0 + m + diag ? v : 0.f; },
                   lane);
   }
   if (tid < DK) {
@@ -313,35 +324,38 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
     p.wLam[cb * DK + tid] = lam[tid];
   }
   {  // K+, Q+, W- to the workspace
-    float* dst[3] = {p.wKp + cb * kC * DK, p.wQp + cb * kC * DK, p.wWm + cb * kC * DK};
+    float* dst[3] = {p.wKp + cb * C * DK, p.wQp + cb * C * DK, p.wWm + cb * C * DK};
     const float* src[3] = {Kp, Qp, Wm};
 #pragma unroll
     for (int q = 0; q < 3; ++q)
-      for (int e = tid; e < kC * DK / 4; e += kNT) {
+      for (int e = tid; e < C * DK / 4; e += kNT) {
         const int t = e / (DK / 4), i = (e % (DK / 4)) * 4;
         *reinterpret_cast<float4*>(dst[q] + t * DK + i) = *reinterpret_cast<const float4*>(src[q] + t * LDK + i);
       }
   }
   __syncthreads();  // K+ and Q+ are consumed
-  if (warp < 4)
-    warp_epilogue(acc, [&](int m, int nn, float v) { Lm[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? v : 0.f; }, lane);
+  if (warp < 4 && gram)
+    warp_epilogue(acc, [&](int m, int nn, float v) { Lm[(m0 + m) * LDC + n0 + nn] = n0 + nn < m0 + m ? v : 0.f; }, lane);
   __syncthreads();
-  inverse64(Lm, Tm, scr, tid);
-  float* Tg = p.wT + cb * kC * kC;
-  for (int e = tid; e < kC * kC; e += kNT) Tg[e] = Tm[(e / kC) * kLDC + e % kC];
+  inverse_blocked<C>(Lm, Tm, scr, tid);
+  float* Tg = p.wT + cb * C * C;
+  for (int e = tid; e < C * C; e += kNT) Tg[e] = Tm[(e / C) * LDC + e % C];
 }
 
 // ------------------------------------------------------------------ kernel 2: states, chunks in order
-template <int DK, int DV, int DVS>
+template <int DK, int DV, int DVS, int C = kC>
 __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDS = DVS + 2, NI = DVS / 16;
+  constexpr int LDK = DK + 4, LDS = DVS + 2, LDC = C + 4, NI = DVS / 16;
+  // warp tiles of the C x DVS products: RT x CT tiles of 16 x TW (with C = 16 and 32 columns, four warps)
+  constexpr int RT = C / 16, CT = (8 / RT < DVS / 8) ? 8 / RT : DVS / 8, TW = DVS / CT, NIT = TW / 8;
+  static_assert(RT * CT <= 8 && TW % 8 == 0, "warp tiles");
   float* S = reinterpret_cast<float*>(smem4);  // [DK][LDS]
   float* Kp = S + DK * LDS;                     // [C][LDK]
-  float* Wm = Kp + kC * LDK;                    // [C][LDK]
-  float* Tm = Wm + kC * LDK;                    // [C][kLDC]
-  float* R = Tm + kC * kLDC;                    // [C][LDS]: V~ - K+ S_m, then U
-  float* er = R + kC * LDS;
+  float* Wm = Kp + C * LDK;                     // [C][LDK]
+  float* Tm = Wm + C * LDK;                     // [C][LDC]
+  float* R = Tm + C * LDC;                      // [C][LDS]: V~ - K+ S_m, then U
+  float* er = R + C * LDS;
   float* lam = er + DK;
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -351,9 +365,10 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
     const int i = e / DVS, j = e % DVS;
     S[i * LDS + j] = a.S0 ? a.S0[((int64_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
-  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * (DVS / 2);  // this warp's tile of a 64 x DVS result
+  const bool tiled = warp < RT * CT;
+  const int m0 = (warp / CT) * 16, n0 = (warp % CT) * TW;  // this warp's tile of a C x DVS result
   for (int c = 0; c < p.nc; ++c) {
-    const int t0 = c * kC, n = min(kC, a.T - t0);
+    const int t0 = c * C, n = min(C, a.T - t0);
     const int64_t cb = (int64_t)bh * p.nc + c;
     __syncthreads();  // the previous chunk is done with every buffer
     if (p.wFlag && p.wFlag[cb]) {
@@ -401,14 +416,14 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
       for (int r = 0; r < RW; ++r) S[(k0 + r) * LDS + j] = Sr[r];
       continue;
     }
-    async_rows<kC, DK>(Kp, LDK, p.wKp + cb * kC * DK, DK, tid);
-    async_rows<kC, DK>(Wm, LDK, p.wWm + cb * kC * DK, DK, tid);
-    async_rows<kC, kC>(Tm, kLDC, p.wT + cb * kC * kC, kC, tid);
+    async_rows<C, DK>(Kp, LDK, p.wKp + cb * C * DK, DK, tid);
+    async_rows<C, DK>(Wm, LDK, p.wWm + cb * C * DK, DK, tid);
+    async_rows<C, C>(Tm, LDC, p.wT + cb * C * C, C, tid);
     async_rows<1, DK>(er, 0, p.wEr + cb * DK, 0, tid);
     async_rows<1, DK>(lam, 0, p.wLam + cb * DK, 0, tid);
     tc::cp_async_commit();
     {
-      constexpr int PER = kC * DVS / kNT;
+      constexpr int PER = C * DVS / kNT;
       float x[PER];
 #pragma unroll
       for (int it = 0; it < PER; ++it) {
@@ -435,34 +450,36 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
       Smg[(int64_t)i * DV + j0 + j] = x;
     }
     __syncthreads();
-    {  // R = V~ - K+ S_m (each warp updates only its own tile)
-      float acc[1][NI][4] = {};
-      warp_gemm<1, NI, DK>(
+    if (tiled) {  // R = V~ - K+ S_m (each warp updates only its own tile)
+      float acc[1][NIT][4] = {};
+      warp_gemm<1, NIT, DK>(
           acc, [&](int m, int k) { return Kp[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return S[k * LDS + n0 + nn]; },
           lane);
       warp_epilogue(acc, [&](int m, int nn, float v) { R[(m0 + m) * LDS + n0 + nn] -= v; }, lane);
     }
     __syncthreads();
     {  // U = T R
-      float acc[1][NI][4] = {};
-      warp_gemm<1, NI, kC>(
-          acc, [&](int m, int k) { return Tm[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return R[k * LDS + n0 + nn]; },
-          lane);
+      float acc[1][NIT][4] = {};
+      if (tiled)
+        warp_gemm<1, NIT, C>(
+            acc, [&](int m, int k) { return Tm[(m0 + m) * LDC + k]; }, [&](int k, int nn) { return R[k * LDS + n0 + nn]; },
+            lane);
       __syncthreads();
-      float* Ug = p.wU + cb * kC * DV;
-      warp_epilogue(acc,
-                    [&](int m, int nn, float v) {
-                      R[(m0 + m) * LDS + n0 + nn] = v;
-                      Ug[(int64_t)(m0 + m) * DV + j0 + n0 + nn] = v;
-                    },
-                    lane);
+      float* Ug = p.wU + cb * C * DV;
+      if (tiled)
+        warp_epilogue(acc,
+                      [&](int m, int nn, float v) {
+                        R[(m0 + m) * LDS + n0 + nn] = v;
+                        Ug[(int64_t)(m0 + m) * DV + j0 + n0 + nn] = v;
+                      },
+                      lane);
     }
     __syncthreads();
     // S' = Diag(lam) (S_m + W-^T U): DK x DVS in 16 x DVS/2 tiles
     for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
       const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * (DVS / 2);
       float acc[1][NI][4] = {};
-      warp_gemm<1, NI, kC>(
+      warp_gemm<1, NI, C>(
           acc, [&](int m, int k) { return Wm[k * LDK + r0 + m]; }, [&](int k, int nn) { return R[k * LDS + q0 + nn]; },
           lane);
       warp_epilogue(acc,
@@ -863,35 +880,36 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
 // ------------------------------------------------------------------ forward outputs of the fp32 chunked forward
 // O = Q+ S_m + P U for one chunk (all d_v columns), from the prep and state kernels' workspace; the
 // chunks the state kernel evaluated exactly (marked) already have their o rows.
-template <int DK, int DV>
+template <int DK, int DV, int C>
 __global__ void __launch_bounds__(kNT) fwd_out_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDV = DV + 4, NI = DV / 16;
+  // warp w: rows 16 (w / CT) .. + 15, columns (w % CT) TW .. + TW
+  constexpr int LDK = DK + 4, LDV = DV + 4, LDC = C + 4, RT = C / 16, CT = 8 / RT, TW = DV / CT, NI = TW / 8;
+  static_assert(RT * CT == 8 && TW % 8 == 0, "warp tiles");
   float* Qp = reinterpret_cast<float*>(smem4);  // [C][LDK]
-  float* Sm = Qp + kC * LDK;                     // [DK][LDV]
-  float* Pm = Sm + DK * LDV;                     // [C][kLDC]
-  float* U = Pm + kC * kLDC;                     // [C][LDV]
+  float* Sm = Qp + C * LDK;                      // [DK][LDV]
+  float* Pm = Sm + DK * LDV;                     // [C][LDC]
+  float* U = Pm + C * LDC;                       // [C][LDV]
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x % p.nc, bh = blockIdx.x / p.nc, b = bh / a.H, h = bh % a.H;
-  const int t0 = c * kC, n = min(kC, a.T - t0);
+  const int t0 = c * C, n = min(C, a.T - t0);
   const int64_t cb = (int64_t)bh * p.nc + c;
   if (p.wFlag[cb]) return;
-  async_rows<kC, DK>(Qp, LDK, p.wQp + cb * kC * DK, DK, tid);
+  async_rows<C, DK>(Qp, LDK, p.wQp + cb * C * DK, DK, tid);
   async_rows<DK, DV>(Sm, LDV, p.wSm + cb * DK * DV, DV, tid);
-  async_rows<kC, kC>(Pm, kLDC, p.wP + cb * kC * kC, kC, tid);
-  async_rows<kC, DV>(U, LDV, p.wU + cb * kC * DV, DV, tid);
+  async_rows<C, C>(Pm, LDC, p.wP + cb * C * C, C, tid);
+  async_rows<C, DV>(U, LDV, p.wU + cb * C * DV, DV, tid);
   tc::cp_async_commit();
   tc::cp_async_wait_all();
   __syncthreads();
-  // warp w: rows 16 (w / 2) .. +15, columns (w % 2) DV / 2 .. + DV / 2
-  const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * (DV / 2);
+  const int m0 = (warp / CT) * 16, n0 = (warp % CT) * TW;
   float acc[1][NI][4] = {};
   warp_gemm<1, NI, DK>(
       acc, [&](int m, int k) { return Qp[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return Sm[k * LDV + n0 + nn]; },
       lane);
-  warp_gemm<1, NI, kC>(
-      acc, [&](int m, int k) { return Pm[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return U[k * LDV + n0 + nn]; },
+  warp_gemm<1, NI, C>(
+      acc, [&](int m, int k) { return Pm[(m0 + m) * LDC + k]; }, [&](int k, int nn) { return U[k * LDV + n0 + nn]; },
       lane);
   warp_epilogue(acc,
                 [&](int m, int nn, float v) {
@@ -902,13 +920,13 @@ __global__ void __launch_bounds__(kNT) fwd_out_kernel(BwdArgs p) {
 }
 
 // ------------------------------------------------------------------ host side
-template <int DK>
+template <int DK, int C = kC>
 constexpr size_t prep_smem() {
-  return sizeof(float) * (3 * kC * (DK + 4) + 768 + 2 * DK);
+  return sizeof(float) * (3 * C * (DK + 4) + 768 + 2 * DK);
 }
-template <int DK, int DVS>
+template <int DK, int DVS, int C = kC>
 constexpr size_t state_smem() {
-  return sizeof(float) * (DK * (DVS + 2) + 2 * kC * (DK + 4) + kC * kLDC + kC * (DVS + 2) + 2 * DK);
+  return sizeof(float) * (DK * (DVS + 2) + 2 * C * (DK + 4) + C * (C + 4) + C * (DVS + 2) + 2 * DK);
 }
 template <int DK, int DVS>
 constexpr size_t dstate_smem() {
@@ -920,9 +938,9 @@ constexpr size_t local_smem() {
                           3 * kC);
 }
 
-template <int DK, int DV>
+template <int DK, int DV, int C>
 constexpr size_t out_smem() {
-  return sizeof(float) * (kC * (DK + 4) + DK * (DV + 4) + kC * kLDC + kC * (DV + 4));
+  return sizeof(float) * (C * (DK + 4) + DK * (DV + 4) + C * (C + 4) + C * (DV + 4));
 }
 
 template <class K>
@@ -950,21 +968,54 @@ cudaError_t launch_dims(const BwdArgs& p, cudaStream_t s) {
   return launch(bwd_local_kernel<DK, DV>, chunks, local_smem<DV>(), s, p);
 }
 
-template <int DK, int DV>
+template <int DK, int DV, int C>
 cudaError_t launch_fwd32_dims(const BwdArgs& p, cudaStream_t s) {
   constexpr int S1 = kDVS_STATE;
-  static_assert(out_smem<DK, DV>() <= 227 * 1024, "shared memory");
+  static_assert(out_smem<DK, DV, C>() <= 227 * 1024, "shared memory");
   const int64_t bh = (int64_t)p.f.B * p.f.H;
   const unsigned chunks = (unsigned)(bh * p.nc);
   cudaError_t e;
-  if ((e = launch(bwd_prep_kernel<DK>, chunks, prep_smem<DK>(), s, p)) != cudaSuccess) return e;
-  if ((e = launch(bwd_state_kernel<DK, DV, S1>, (unsigned)(bh * (DV / S1)), state_smem<DK, S1>(), s, p)) != cudaSuccess)
+  if ((e = launch(bwd_prep_kernel<DK, C>, chunks, prep_smem<DK, C>(), s, p)) != cudaSuccess) return e;
+  if ((e = launch(bwd_state_kernel<DK, DV, S1, C>, (unsigned)(bh * (DV / S1)), state_smem<DK, S1, C>(), s, p)) !=
+      cudaSuccess)
     return e;
-  return launch(fwd_out_kernel<DK, DV>, chunks, out_smem<DK, DV>(), s, p);
+  return launch(fwd_out_kernel<DK, DV, C>, chunks, out_smem<DK, DV, C>(), s, p);
 }
 
-// The backward's workspace layout (the forward uses T, P, S_m, U, K+, Q+, W-, e^h, e^r and lam of
-// it), then one int per chunk.
+template <int C>
+cudaError_t launch_fwd32_c(const BwdArgs& p, cudaStream_t s) {
+  const Args& f = p.f;
+  if (f.dk == 128 && f.dv == 128) return launch_fwd32_dims<128, 128, C>(p, s);
+  if (f.dk == 128 && f.dv == 64) return launch_fwd32_dims<128, 64, C>(p, s);
+  if (f.dk == 64 && f.dv == 128) return launch_fwd32_dims<64, 128, C>(p, s);
+  return launch_fwd32_dims<64, 64, C>(p, s);
+}
+
+// The forward's workspace, per (b, h, chunk of C tokens): T and P (C x C), S_m (d_k x d_v), U
+// (C x d_v), K+, Q+ and W- (C x d_k), e^r and lam (d_k), all fp32; then one int per chunk (the
+// marks of the chunks evaluated token by token), the whole rounded up to 16 bytes.
+int64_t fwd32_floats_per_chunk(int C, int dk, int dv) {
+  return 2LL * C * C + (int64_t)dk * dv + (int64_t)C * dv + 3LL * C * dk + 2LL * dk;
+}
+
+void set_fwd_workspace(BwdArgs& p, const Args& f, float* ws) {
+  const int C = f.chunk;
+  p.nc = (f.T + C - 1) / C;
+  const int64_t blocks = (int64_t)f.B * f.H * p.nc;
+  p.wT = ws;
+  p.wP = p.wT + blocks * C * C;
+  p.wSm = p.wP + blocks * C * C;
+  p.wU = p.wSm + blocks * f.dk * f.dv;
+  p.wKp = p.wU + blocks * C * f.dv;
+  p.wQp = p.wKp + blocks * C * f.dk;
+  p.wWm = p.wQp + blocks * C * f.dk;
+  p.wEr = p.wWm + blocks * C * f.dk;
+  p.wLam = p.wEr + blocks * f.dk;
+  p.wEh = nullptr;  // (the backward's e^h is not needed)
+  p.wFlag = reinterpret_cast<int*>(p.wLam + blocks * f.dk);
+}
+
+// The backward's workspace layout, for its chunks of kC tokens.
 void set_workspace(BwdArgs& p, const Args& f, float* ws) {
   p.nc = (f.T + kC - 1) / kC;
   const int64_t blocks = (int64_t)f.B * f.H * p.nc;
@@ -986,26 +1037,28 @@ void set_workspace(BwdArgs& p, const Args& f, float* ws) {
 }  // namespace
 
 bool chunk_fwd32_supported(const Args& a) {
-  return (a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128) && a.chunk == kC && a.T > 0 &&
-         !(a.io_bf16 && a.dk == 128);  // (bf16 with d_k = 128 has the tcgen05 kernels)
+  if (!((a.dk == 64 || a.dk == 128) && (a.dv == 64 || a.dv == 128) && a.T > 0)) return false;
+  if (!(a.chunk == 16 || a.chunk == 32 || a.chunk == kC)) return false;
+  if ((int64_t)a.B * a.H * ((a.T + a.chunk - 1) / a.chunk) >= ((int64_t)1 << 31)) return false;  // (one CTA per chunk)
+  if (a.chunk == 16 || a.chunk == 32) return true;  // (the tcgen05 kernels' tiles are 64 tokens)
+  return a.chunk == kC && !(a.io_bf16 && a.dk == 128);  // (bf16 with d_k = 128 has the tcgen05 kernels)
 }
 
 size_t chunk_fwd32_workspace_bytes(const Args& a) {
-  const int64_t blocks = (int64_t)a.B * a.H * ((a.T + kC - 1) / kC);
-  const size_t flags = ((size_t)blocks * sizeof(int) + 15) & ~size_t(15);
-  return chunk_bwd_workspace_bytes(a.B, a.T, a.H, a.dk, a.dv) + flags;
+  const int64_t blocks = (int64_t)a.B * a.H * ((a.T + a.chunk - 1) / a.chunk);
+  const size_t bytes = (size_t)(blocks * fwd32_floats_per_chunk(a.chunk, a.dk, a.dv)) * sizeof(float) +
+                       (size_t)blocks * sizeof(int);
+  return (bytes + 15) & ~size_t(15);
 }
 
 cudaError_t launch_chunk_fwd32(const Args& f, float* ws, cudaStream_t s) {
   BwdArgs p;
   memset(&p, 0, sizeof(p));
   p.f = f;
-  set_workspace(p, f, ws);
-  p.wFlag = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ws) + chunk_bwd_workspace_bytes(f.B, f.T, f.H, f.dk, f.dv));
-  if (f.dk == 128 && f.dv == 128) return launch_fwd32_dims<128, 128>(p, s);
-  if (f.dk == 128 && f.dv == 64) return launch_fwd32_dims<128, 64>(p, s);
-  if (f.dk == 64 && f.dv == 128) return launch_fwd32_dims<64, 128>(p, s);
-  return launch_fwd32_dims<64, 64>(p, s);
+  set_fwd_workspace(p, f, ws);
+  if (f.chunk == 16) return launch_fwd32_c<16>(p, s);
+  if (f.chunk == 32) return launch_fwd32_c<32>(p, s);
+  return launch_fwd32_c<kC>(p, s);
 }
 
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {

@@ -102,7 +102,9 @@ typedef enum { DN_READ_POST = 0, DN_READ_PRE = 1 } dn_readout;
 typedef struct {
   int B, T, H;        /* batch, tokens per sequence, heads; B, H >= 1, T >= 0 */
   int d_k, d_v;       /* head dims; supported: d_k, d_v in {64, 128}, or both in {8, 16} (small states) */
-  int chunk;          /* chunk length of the WY form; 0 selects the default, 64 (the only value supported) */
+  int chunk;          /* chunk length of the WY form: 16, 32 or 64; 0 selects the default, 64. 16 and 32 run the
+                         chunk form in fp32 (below); small states and the sequential kernel have no chunks;
+                         dn_chunk_bwd takes 0 or 64 */
   dn_dtype io_dtype;  /* dtype of q, k, v and o */
   dn_gate alpha;      /* forget gate: scalar (GDN) or per key channel (KDA) */
   dn_gate beta_k;     /* erase / write strength on the key side (GDN beta; FG2-GDN+ beta^k) */
@@ -123,13 +125,16 @@ typedef struct {
  *    state-chain kernel reads it back; the faster form;
  *  - with workspace == NULL: one fused kernel per (b, h) that keeps everything on
  *    chip, at some cost in speed.
- * Problems in fp32 io, and bf16 with d_k = 64 (d_k, d_v in {64, 128}), also have two:
+ * Problems in fp32 io, and bf16 with d_k = 64 (d_k, d_v in {64, 128}), also have two, and
+ * so does every problem with d_k, d_v in {64, 128} and chunk = 16 or 32:
  *  - with a workspace of at least this size: the chunk form in fp32 (split-TF32 warp
- *    tensor-core products, about fp32 accuracy): a kernel forms every chunk's decay-scaled
- *    keys, queries and write keys, UT transform and scores (fp32, ~164 KB per (b, h, chunk)
- *    at d = 64, ~361 KB at d = 128), the state chain walks the chunks, and a third kernel
- *    forms the outputs; a chunk whose decay over half a chunk exceeds e^80 per channel is
- *    evaluated token by token inside the chain;
+ *    tensor-core products, about fp32 accuracy) with chunks of C = chunk tokens: a kernel
+ *    forms every chunk's decay-scaled keys, queries and write keys, UT transform and scores,
+ *    the state chain walks the chunks, and a third kernel forms the outputs. The workspace
+ *    holds, per (b, h, chunk), 4 * (2 C^2 + d_k d_v + C d_v + 3 C d_k + 2 d_k) bytes (115 KB
+ *    at C = 64 and d = 64, 230 KB at d = 128) plus one int, rounded up to 16 bytes in all; a
+ *    chunk whose decay over half a chunk exceeds e^80 per channel is evaluated token by token
+ *    inside the chain;
  *  - with workspace == NULL: the sequential fp32 kernel, token by token.
  * Both give the same results up to rounding. Other problems (small states, per-channel
  * gates at bf16 d_k = 128) take no workspace.
@@ -281,7 +286,7 @@ dn_status dn_mc_readout(const dn_mc_desc* desc, const void* q, const float* M, c
  * decay-scaled keys, queries and write keys and their decay factors (64 x d_k each), the
  * state and its adjoint (d_k x d_v each), and the residuals and their adjoints (64 x d_v each).
  * Supported: both read-outs (desc->readout as given to the forward); d_k, d_v in {64, 128}
- * (chunked kernels) or both in {8, 16} (small states: one warp per head, sequential, the state
+ * (chunked kernels, chunk 0 or 64; 16 and 32 return DN_ERR_UNSUPPORTED) or both in {8, 16} (small states: one warp per head, sequential, the state
  * entering every token kept in the workspace); alpha > 0. The chunked kernels reference each chunk's
  * decay to a point inside it, in fp32: a chunk where the decay between that point and any of its
  * tokens exceeds e^80 per channel (mean log alpha below about -2.5 per token) sets

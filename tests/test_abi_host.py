@@ -83,7 +83,9 @@ def test_rejects_bad_descriptors(lib):
     assert _call(lib, _desc(alpha=5)) == dn.DN_ERR_INVALID_ARGUMENT
     assert _call(lib, _desc(d_k=96)) == dn.DN_ERR_UNSUPPORTED
     assert _call(lib, _desc(d_v=256)) == dn.DN_ERR_UNSUPPORTED
-    assert _call(lib, _desc(chunk=32)) == dn.DN_ERR_UNSUPPORTED
+    assert _call(lib, _desc(chunk=48)) == dn.DN_ERR_UNSUPPORTED
+    assert _call(lib, _desc(chunk=128)) == dn.DN_ERR_UNSUPPORTED
+    assert _call(lib, _desc(chunk=-1)) == dn.DN_ERR_INVALID_ARGUMENT
     assert _call(lib, _desc(readout=2)) == dn.DN_ERR_INVALID_ARGUMENT
     assert _call(lib, _desc(d_k=8, d_v=64)) == dn.DN_ERR_UNSUPPORTED  # small and large dims do not mix
     assert _call(lib, _desc(d_k=32, d_v=32)) == dn.DN_ERR_UNSUPPORTED
@@ -120,14 +122,13 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.dn_decode_step(ctypes.byref(d), *bad) == dn.DN_ERR_INVALID_ARGUMENT
 
 
-def _fwd32_bytes(B, T, H, dk, dv):
-    """The fp32 chunked forward's workspace: the backward's chunk quantities (T, P: 64 x 64; S_m, dX:
-    d_k x d_v; U, dV~: 64 x d_v; K+, Q+, W-, e^h: 64 x d_k; e^r, lam: d_k; fp32) per (b, h, chunk), then
-    one int per chunk, rounded up to 16 bytes."""
-    nc = -(-T // 64)
-    per = 2 * 64 * 64 + 2 * dk * dv + 2 * 64 * dv + 4 * 64 * dk + 2 * dk
-    flags = (B * H * nc * 4 + 15) // 16 * 16
-    return B * H * nc * per * 4 + flags
+def _fwd32_bytes(B, T, H, dk, dv, C=64):
+    """The fp32 chunked forward's workspace: per (b, h, chunk of C tokens) T, P (C x C), S_m (d_k x d_v),
+    U (C x d_v), K+, Q+, W- (C x d_k), e^r, lam (d_k), fp32; then one int per chunk; the whole rounded
+    up to 16 bytes."""
+    nc = -(-T // C)
+    per = 2 * C * C + dk * dv + C * dv + 3 * C * dk + 2 * dk
+    return (B * H * nc * (per * 4 + 4) + 15) // 16 * 16
 
 
 def test_workspace_query(lib):
@@ -140,6 +141,23 @@ def test_workspace_query(lib):
     assert dn.dn_chunk_fwd_workspace_bytes(_desc(d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL)) == 0
     assert dn.dn_chunk_fwd_workspace_bytes(_desc(T=0)) == 0
     assert lib.dn_chunk_fwd_workspace_bytes(None) == 0
+
+
+def test_chunk_lengths(lib):
+    """chunk in {16, 32}: the chunk form in fp32 with that chunk length, for every d_k, d_v and io dtype
+    (bf16 d_k = 128 included: the tensor-core kernels' tiles are 64 tokens); 0 means 64; small states
+    have no chunks; the backward's chunks are 64 tokens."""
+    for C in (16, 32):
+        for io in (dn.DN_BF16, dn.DN_F32):
+            for dk, dv in ((64, 64), (64, 128), (128, 64), (128, 128)):
+                for al in (dn.DN_GATE_SCALAR, dn.DN_GATE_CHANNEL):
+                    d = _desc(chunk=C, io_dtype=io, d_k=dk, d_v=dv, T=130, alpha=al)
+                    assert dn.dn_chunk_fwd_workspace_bytes(d) == _fwd32_bytes(1, 130, 2, dk, dv, C), (C, io, dk, dv)
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(chunk=64)) == dn.dn_chunk_fwd_workspace_bytes(_desc(chunk=0))
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(chunk=16, d_k=8, d_v=8)) == 0
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(chunk=32))) == 0  # rejected
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(chunk=64))) > 0
+    assert lib.dn_chunk_bwd_workspace_bytes(ctypes.byref(_desc(chunk=16, d_k=8, d_v=8))) > 0
 
 
 def test_binding_has_no_cpu_path(tmp_path):
