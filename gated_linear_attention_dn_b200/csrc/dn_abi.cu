@@ -151,6 +151,7 @@ size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc) {
   a.alpha = desc->alpha, a.beta_k = desc->beta_k, a.beta_v = desc->beta_v, a.key_scale = desc->key_scale;
   if (dn::small_state_supported(a)) return 0;
   if (dn::per_token_tc(a)) return dn::split_sc_workspace_bytes(a);
+  if (dn::split_tc_supported(a)) return dn::split_tc_workspace_bytes(a);
   if (dn::chunk_fwd32_supported(a)) return dn::chunk_fwd32_workspace_bytes(a);
   return 0;
 }
@@ -218,6 +219,8 @@ dn_status dn_chunk_fwd(const dn_desc* desc, const void* q, const void* k, const 
     e = dn::launch_small_state(a, s);
   } else if (workspace && dn::per_token_tc(a)) {
     e = dn::launch_split_sc(a, workspace, s);
+  } else if (workspace && dn::split_tc_supported(a)) {
+    e = dn::launch_split_tc(a, workspace, s);
   } else if (a.io_bf16 && dn::chunk_tc_supported(a)) {
     e = dn::launch_chunk_tc(a, s);
   } else if (workspace && dn::chunk_fwd32_supported(a)) {

@@ -85,10 +85,6 @@ __device__ __forceinline__ float4 rcp4(float4 a) {
   return make_float4(__fdividef(1.f, a.x), __fdividef(1.f, a.y), __fdividef(1.f, a.z), __fdividef(1.f, a.w));
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
-}
-
 // Gate values of 8 tokens (rows tok0 + i * tstride, i < 8) for 4 consecutive channels, with every
 // load issued before any is used: the mode branch is uniform and outside the loads, and tokens past
 // the end (i >= nvalid) re-read row tok0 + (nvalid - 1) * tstride, or row tok0 when nvalid == 0
@@ -115,6 +111,16 @@ __device__ __forceinline__ void gate4x8(float4* out, const float* g, int mode, i
   for (int i = 0; i < 8; ++i)
     if (i >= nvalid) out[i] = f4(dflt);
 }
+
+// shared -> global bulk copy (both addresses 16-byte aligned, bytes a multiple of 16), its group
+// commit, and the wait until the committed copies have completed
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ float4 lds4(const float* p, int idx) { return *reinterpret_cast<const float4*>(p + idx); }
 
@@ -146,7 +152,7 @@ __device__ __forceinline__ void split4(float4 v, uint2& hi, uint2& lo) {
 // (DK x (NV + 1) fp32) transposes the state between the tensor-memory rows and these columns.
 // Called by all 256 threads.
 template <int DK, int NV>
-__device__ __noinline__ void exact_chunk(const Args& a, const uint8_t* sk, const uint8_t* sq, const uint8_t* svhi,
+__device__ __forceinline__ void exact_chunk(const Args& a, const uint8_t* sk, const uint8_t* sq, const uint8_t* svhi,
                                          const uint8_t* svlo, bool v_split, const float* sAl, const float* sWk,
                                          const float* s_wq, float* sX, const float* lam_prev, uint32_t tmem_s,
                                          int c, int n, int b, int h, int bh, int col0, int tid) {
@@ -848,6 +854,718 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ================================================================== split evaluation (workspace)
+// With a workspace, the state-independent part of every chunk -- the decay factors, the operand tiles,
+// the Gram product and the UT inverse -- runs first for all chunks at once (prep_tc_kernel, one CTA
+// per (b, h, chunk)), which writes one record per chunk; chain_tc_kernel then walks each sequence's
+// chunks with the state in tensor memory and bulk-loads each record's parts a step ahead of their
+// use, so that a step of the chain is the Wk / U0 products, the state products and the U conversion.
+// A chunk out of the factors' range is marked in its record, which then carries the exact path's
+// operands instead (raw k and q tiles, alpha and w rows, w . q), and the chain evaluates it token by
+// token as the fused kernel does.
+template <int DK>
+struct XRec {
+  static constexpr uint32_t KQ = 0;                   // [K+; Q+] bf16 [128][DK]; exact: raw k, raw q [C][DK]
+  static constexpr uint32_t TP = KQ + 128 * DK * 2;   // [T; P] bf16 [128][C]
+  static constexpr uint32_t WHI = TP + 128 * C * 2;   // W- hi [C][DK]
+  static constexpr uint32_t WLO = WHI + C * DK * 2;   // W- lo [C][DK]
+  static constexpr uint32_t F = WLO + C * DK * 2;     // gamma_m [DK], gamma_C / gamma_m [DK], w . q [C], flag
+  static constexpr uint32_t F_GM = 0, F_LAM = DK * 4, F_WQ = 2 * DK * 4, F_FLAG = 2 * DK * 4 + C * 4;
+  static constexpr uint32_t FBYTES = 2048;
+  static_assert(F_FLAG + 16 <= FBYTES, "factor block");
+  static constexpr uint32_t V = F + FBYTES;           // V~ hi [C][d_v], then lo [C][d_v] (beta^v given)
+  __host__ __device__ static constexpr size_t vbytes(int dv, bool bv) { return bv ? (size_t)2 * C * dv * 2 : 0; }
+  // alpha rows then w = beta^k d k rows, fp32 [C][DK] each (written for exact chunks only)
+  __host__ __device__ static constexpr size_t x_off(int dv, bool bv) { return V + vbytes(dv, bv); }
+  __host__ __device__ static constexpr size_t stride(int dv, bool bv) { return x_off(dv, bv) + (size_t)2 * C * DK * 4; }
+};
+
+template <int DK>
+struct PLayout {
+  static constexpr int KQ = 0;                  // [K+; Q+] (the Gram's A), then the inverse's fp32 L and T
+  static constexpr int WHI = KQ + 128 * DK * 2;  // W- hi (the Gram's B), then the inverse's scratch
+  static constexpr int TP = WHI + C * DK * 2;    // [T; P]; before P3 the per-8-token decay products
+  static constexpr int TOTAL = TP + 128 * C * 2;
+  static_assert(2 * C * C * 4 <= 128 * DK * 2 && 2048 * 4 <= C * DK * 2 && 8 * DK * 4 <= 128 * C * 2, "overlays");
+};
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads, 2) prep_tc_kernel(const Args a, uint8_t* ws, int nchunks) {
+  using Ly = PLayout<DK>;
+  using R = XRec<DK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_mma;
+  __shared__ uint32_t s_tmem;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, ch = warp >> 2;
+  const int c = blockIdx.x % nchunks, bh = blockIdx.x / nchunks, b = bh / a.H, h = bh % a.H;
+  const int T = a.T, H = a.H, dv = a.dv, t0 = c * C, n = min(C, T - t0);
+  const int pre = a.pre_read ? 1 : 0;
+  const bool bv = a.beta_v != DN_GATE_ONE;
+  uint8_t* const rec = ws + ((size_t)bh * nchunks + c) * R::stride(dv, bv);
+  float* const rf = reinterpret_cast<float*>(rec + R::F);
+  float* const s_grp = reinterpret_cast<float*>(sm + Ly::TP);  // [8][DK]
+  if (tid == 0) {
+    mbar_init(&bar_mma, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&s_tmem, 64);
+  // ---- P1: thread (lane, warp) owns channels 4 lane .. + 3 of tokens 8 warp .. + 7
+  const int tg = warp, cb0 = 4 * lane;
+  const int nvalid = max(0, min(8, n - 8 * tg));
+  const int64_t tok0 = ((int64_t)b * T + t0 + (nvalid > 0 ? 8 * tg : 0)) * H + h;
+  // V~ = beta^v (.) v, split hi / lo, for the value columns 4 lane .. + 3 (both paths read it)
+  if (bv && cb0 < dv) {
+    float4 bvs[8];
+    uint2 vr[8];
+    gate4x8(bvs, a.beta_v_p, a.beta_v, tok0, H, dv, cb0, nvalid, 0.f);
+    const __nv_bfloat16* vp = static_cast<const __nv_bfloat16*>(a.v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ic = i < nvalid ? i : max(nvalid - 1, 0);
+      vr[i] = __ldg(reinterpret_cast<const uint2*>(vp + (tok0 + (int64_t)ic * H) * dv + cb0));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * tg + i;
+      uint2 hi, lo;
+      split4(mul4(unpack4(vr[i]), bvs[i]), hi, lo);
+      const uint32_t o2 = canon(j, cb0, C);
+      *reinterpret_cast<uint2*>(rec + R::V + o2) = hi;
+      *reinterpret_cast<uint2*>(rec + R::V + (uint32_t)(C * dv * 2) + o2) = lo;
+    }
+  }
+
+  float4 al[8], ws4[8], dd[8];
+  uint2 kr[8], qr[8];
+  gate4x8(al, a.alpha_p, a.alpha, tok0, H, DK, cb0, nvalid, 1.f);
+  gate4x8(ws4, a.beta_k_p, a.beta_k, tok0, H, DK, cb0, nvalid, 0.f);
+  gate4x8(dd, a.key_scale_p, a.key_scale, tok0, H, DK, cb0, nvalid, 0.f);
+  {
+    const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(a.k);
+    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(a.q);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ic = i < nvalid ? i : max(nvalid - 1, 0);
+      const int64_t off = (tok0 + (int64_t)ic * H) * DK + cb0;
+      kr[i] = __ldg(reinterpret_cast<const uint2*>(kp + off));
+      qr[i] = __ldg(reinterpret_cast<const uint2*>(qp + off));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (i >= nvalid) kr[i] = qr[i] = make_uint2(0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ws4[i] = mul4(ws4[i], dd[i]);
+  // products inside the group: prefix (second half) or exclusive suffix (first half)
+  float4 loc[8];
+  {
+    float4 p = f4(1.f);
+    if (tg >= 4) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        p = mul4(p, al[i]);
+        loc[i] = p;
+      }
+    } else {
+#pragma unroll
+      for (int i = 7; i >= 0; --i) {
+        loc[i] = p;
+        p = mul4(p, al[i]);
+      }
+    }
+    sts4(s_grp + tg * DK, cb0, p);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  float4 off = f4(1.f);
+  if (tg >= 4) {
+    for (int g = 4; g < tg; ++g) off = mul4(off, lds4(s_grp + g * DK, cb0));
+  } else {
+    for (int g = tg + 1; g < 4; ++g) off = mul4(off, lds4(s_grp + g * DK, cb0));
+  }
+  bool ok = true;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ok = ok && in_range4(mul4(off, loc[i]));
+  if (tg == 0) {
+    float4 gm = f4(1.f), lm = f4(1.f);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) gm = mul4(gm, lds4(s_grp + g * DK, cb0));
+#pragma unroll
+    for (int g = 4; g < 8; ++g) lm = mul4(lm, lds4(s_grp + g * DK, cb0));
+    sts4(rf + R::F_GM / 4, cb0, gm);
+    sts4(rf + R::F_LAM / 4, cb0, lm);
+    ok = ok && in_range4(gm) && in_range4(lm);
+  }
+  const bool extreme = __syncthreads_or(!ok);
+  if (tid == 0) reinterpret_cast<int*>(rf)[R::F_FLAG / 4] = extreme ? 1 : 0;
+
+  if (extreme) {
+    // the exact path's operands: raw k and q tiles, alpha and w rows (fp32), w . q per token
+    float* xa = reinterpret_cast<float*>(rec + R::x_off(dv, bv));
+    float* xw = xa + C * DK;
+    float wq[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * tg + i;
+      *reinterpret_cast<uint2*>(rec + R::KQ + canon(j, cb0, C)) = kr[i];
+      *reinterpret_cast<uint2*>(rec + R::KQ + C * DK * 2 + canon(j, cb0, C)) = qr[i];
+      const float4 kk = unpack4(kr[i]), qq = unpack4(qr[i]);
+      const float4 wv = mul4(ws4[i], kk);
+      sts4(xa, j * DK + cb0, al[i]);
+      sts4(xw, j * DK + cb0, wv);
+      wq[i] = wv.x * qq.x + wv.y * qq.y + wv.z * qq.z + wv.w * qq.w;
+    }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wq[i] += __shfl_xor_sync(0xffffffffu, wq[i], o2);
+    if (lane == 0)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rf[R::F_WQ / 4 + 8 * tg + i] = wq[i];
+  } else {
+    // K+ and Q+ (shared memory, the Gram's A, and the record), W- hi (shared memory, the Gram's B, and
+    // the record), W- lo (the record)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * tg + i;
+      float4 r, rinv;
+      if (tg >= 4) {
+        r = mul4(off, loc[i]);
+        rinv = rcp4(r);
+      } else {
+        rinv = mul4(off, loc[i]);
+        r = rcp4(rinv);
+      }
+      const float4 kk = unpack4(kr[i]), qq = unpack4(qr[i]);
+      const uint2 kpk = pack4(mul4(kk, r));
+      // Q+ = q (.) r_t; for the pre-update read-out q (.) r_{t-1} = q (.) r_t / alpha_t
+      const uint2 qpk = pack4(pre ? mul4(qq, mul4(r, rcp4(al[i]))) : mul4(qq, r));
+      const uint32_t ok_ = canon(j, cb0, 128), oq = canon(64 + j, cb0, 128);
+      *reinterpret_cast<uint2*>(sm + Ly::KQ + ok_) = kpk;
+      *reinterpret_cast<uint2*>(sm + Ly::KQ + oq) = qpk;
+      *reinterpret_cast<uint2*>(rec + R::KQ + ok_) = kpk;
+      *reinterpret_cast<uint2*>(rec + R::KQ + oq) = qpk;
+      uint2 hi, lo;
+      split4(mul4(mul4(ws4[i], kk), rinv), hi, lo);
+      const uint32_t ow = canon(j, cb0, C);
+      *reinterpret_cast<uint2*>(sm + Ly::WHI + ow) = hi;
+      *reinterpret_cast<uint2*>(rec + R::WHI + ow) = hi;
+      *reinterpret_cast<uint2*>(rec + R::WLO + ow) = lo;
+    }
+  }
+  fence_proxy_async();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  bool failed = false;
+  if (!extreme) {
+    // ---- Gram [K+; Q+] W-^T -> tensor memory (64 columns)
+    const uint32_t id_gram = idesc_bf16(128, 64, 0, 0);
+    if (tid == 0) {
+#pragma unroll
+      for (int kk = 0; kk < DK; kk += 16) {
+        const uint64_t ad = sdesc(smem_u32(sm + Ly::KQ) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+        const uint64_t bd = sdesc(smem_u32(sm + Ly::WHI) + (kk >> 6) * (C * 128) + (kk & 63) * 2, 16, 1024);
+        mma_bf16(tmem, ad, bd, id_gram, kk > 0);
+      }
+      mma_commit(&bar_mma);
+    }
+    // rows 0..63 of [T; P]: the 8x8 blocks above the block diagonal of T are zero (the inverse never
+    // writes them; the group products that overlaid the tile are dead)
+    for (int e = tid; e < 64 * 8; e += kThreads) {
+      const int t = e >> 3, x8 = e & 7;
+      if (x8 > (t >> 3)) *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(t, x8, 128)) = make_uint4(0, 0, 0, 0);
+    }
+    const bool okw = mbar_wait_bounded(&bar_mma, 0, a.wait_ns);
+    failed = __syncthreads_or(!okw);
+    if (!failed) {
+      tc_fence_after();
+      // A (strict lower) -> fp32 sL over the [K+; Q+] tile; P (lower incl.) -> bf16 rows 64..127 of [T; P]
+      float* sL = reinterpret_cast<float*>(sm + Ly::KQ);
+      float* sT = sL + C * C;
+      {
+        float x[32];
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        tmem_ld32(tmem + lane_base + 32 * ch, x);
+        const int i0 = 32 * ch;
+        if (q4 < 2) {
+          const int t = 32 * q4 + lane;
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            float y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = i0 + 4 * e4 + e;
+              y[e] = (i < t) ? x[4 * e4 + e] : 0.f;
+            }
+            sts4(sL, xi(t, i0 + 4 * e4), make_float4(y[0], y[1], y[2], y[3]));
+          }
+        } else {
+          const int t = 32 * (q4 - 2) + lane;
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = (i0 + 8 * q8 + e <= t - pre) ? x[8 * q8 + e] : 0.f;
+            uint4 pk = make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
+                                  pack_bf16(y[6], y[7]));
+            *reinterpret_cast<uint4*>(sm + Ly::TP + canon_chunk(64 + t, i0 / 8 + q8, 128)) = pk;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+      unit_lower_inverse<false, 8>(sL, sT, reinterpret_cast<float*>(sm + Ly::WHI), sm + Ly::TP, nullptr, nullptr,
+                                   nullptr, tid, 0);
+      fence_proxy_async();
+      __syncthreads();
+      // [T; P] -> the record
+      if (tid == 0) {
+        bulk_store(rec + R::TP, sm + Ly::TP, 128 * C * 2);
+        bulk_commit();
+      }
+    } else {
+      mbar_wait_bounded(&bar_mma, 0, kWaitNs);  // drain (bounded)
+      if (tid == 0) atomicExch(a.status, kDevTimeout);
+    }
+  }
+  if (tid == 0) bulk_wait_all();  // the record's copies are complete before the block leaves
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+template <int DK, int NV>
+struct XLayout {
+  static constexpr int KQ = 0;                   // [K+; Q+] of the record, then [Wk; Q+]; exact: raw k, raw q
+  static constexpr int TP0 = KQ + 128 * DK * 2;  // [T; P] of even chunks
+  static constexpr int TP1 = TP0 + 128 * C * 2;  // [T; P] of odd chunks
+  static constexpr int WHI = TP1 + 128 * C * 2;  // W- hi
+  static constexpr int WLO = WHI + C * DK * 2;   // W- lo
+  static constexpr int STV = WLO + C * DK * 2;   // V~ hi (the record) or raw v (TMA)
+  static constexpr int VLO = STV + C * NV * 2;   // V~ lo
+  static constexpr int UHI = VLO + C * NV * 2;   // U hi
+  static constexpr int ULO = UHI + C * NV * 2;   // U lo
+  static constexpr int SM = ULO + C * NV * 2;    // S_m bf16 [DK][NV]
+  static constexpr int F0 = SM + DK * NV * 2 + 1024;  // factor blocks of even / odd chunks
+  static constexpr int F1 = F0 + 2048;
+  static constexpr int TOTAL = F1 + 2048;
+  static constexpr int TM_S = 0, TM_D1 = NV, TM_U0 = 2 * NV, TM_SCR = 3 * NV;
+  static_assert(TM_SCR + DK <= (int)kTmemCols, "tensor memory budget");
+  // the exact path's fp32 state transpose (DK x (NV + 1)) overlays the U and S_m tiles
+  static_assert(UHI + DK * (NV + 1) * 4 <= F0, "transpose buffer of the exact path");
+};
+
+template <int DK, int NV>
+__global__ void __launch_bounds__(kThreads, 1)
+    chain_tc_kernel(const __grid_constant__ CUtensorMap tm_v, const Args a, const uint8_t* ws) {
+  using Ly = XLayout<DK, NV>;
+  using R = XRec<DK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_kq, bar_tp[2], bar_w, bar_v, bar_mma;
+  __shared__ uint32_t s_tmem;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, ch = warp >> 2;
+  const int T = a.T, H = a.H, dv = a.dv;
+  const int nslices = dv / NV;
+  const int bh = blockIdx.x / nslices, b = bh / H, h = bh % H;
+  const int col0 = (blockIdx.x % nslices) * NV;
+  const int nchunks = (T + C - 1) / C;
+  const bool bv = a.beta_v != DN_GATE_ONE;
+  const size_t stride = R::stride(dv, bv);
+  auto rec = [&](int c) { return ws + ((size_t)bh * nchunks + c) * stride; };
+  auto fblk = [&](int c) { return reinterpret_cast<float*>(sm + ((c & 1) ? Ly::F1 : Ly::F0)); };
+
+  if (tid == 0) {
+    mbar_init(&bar_kq, 1);
+    mbar_init(&bar_tp[0], 1);
+    mbar_init(&bar_tp[1], 1);
+    mbar_init(&bar_w, 1);
+    mbar_init(&bar_v, 1);
+    mbar_init(&bar_mma, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+  uint8_t* const kq = sm + Ly::KQ;
+  auto tp_of = [&](int c) { return sm + ((c & 1) ? Ly::TP1 : Ly::TP0); };
+
+  // record parts (thread 0): [K+; Q+] and the factors; [T; P]; W- hi and lo; V~ (or raw v)
+  auto issue_kq = [&](int c) {
+    mbar_expect_tx(&bar_kq, 128 * DK * 2 + R::FBYTES);
+    bulk_load(kq, rec(c) + R::KQ, 128 * DK * 2, &bar_kq);
+    bulk_load(fblk(c), rec(c) + R::F, R::FBYTES, &bar_kq);
+  };
+  auto issue_tp = [&](int c) {
+    mbar_expect_tx(&bar_tp[c & 1], 128 * C * 2);
+    bulk_load(tp_of(c), rec(c) + R::TP, 128 * C * 2, &bar_tp[c & 1]);
+  };
+  auto issue_w = [&](int c) {
+    mbar_expect_tx(&bar_w, 2 * C * DK * 2);
+    bulk_load(sm + Ly::WHI, rec(c) + R::WHI, C * DK * 2, &bar_w);
+    bulk_load(sm + Ly::WLO, rec(c) + R::WLO, C * DK * 2, &bar_w);
+  };
+  auto issue_v = [&](int c) {
+    if (bv) {
+      mbar_expect_tx(&bar_v, 2 * C * NV * 2);
+      bulk_load(sm + Ly::STV, rec(c) + R::V + (col0 / 64) * (C * 128), C * NV * 2, &bar_v);
+      bulk_load(sm + Ly::VLO, rec(c) + R::V + C * dv * 2 + (col0 / 64) * (C * 128), C * NV * 2, &bar_v);
+    } else {
+      mbar_expect_tx(&bar_v, (uint32_t)C * NV * 2);
+#pragma unroll
+      for (int x = 0; x < NV / 64; ++x)
+        tma_load_4d(sm + Ly::STV + x * C * 128, &tm_v, &bar_v, col0 + 64 * x, h, c * C, b);
+    }
+  };
+
+  uint32_t ph_kq = 0, ph_tp[2] = {0, 0}, ph_w = 0, ph_v = 0, ph_mma = 0;
+  bool kq_p = false, tp_p[2] = {false, false}, w_p = false, v_p = false, mma_p = false;
+  bool o_pending = false, failed = false;
+  if (nchunks > 0) {
+    if (tid == 0) {
+      issue_kq(0);
+      issue_tp(0);
+      issue_w(0);
+      issue_v(0);
+      if (nchunks > 1) issue_tp(1);
+    }
+    kq_p = w_p = v_p = tp_p[0] = true;
+    tp_p[1] = nchunks > 1;
+  }
+
+  const uint32_t id_wk = idesc_bf16(128, DK, 0, 1);
+  const uint32_t id_nv = idesc_bf16(128, NV, 0, 1);
+  const uint32_t id_state = idesc_bf16(128, NV, 1, 1);
+
+  // S_m = Diag(lambda_prev gamma_m) S (rows 32 q4 .. + 31, columns of half ch): the state in chunk c's
+  // frame, in tensor memory (fp32) and as the bf16 operand tile
+  auto state_to_frame = [&](int c) {
+    const int k = 32 * q4 + lane;
+    const float gm = fblk(c)[R::F_GM / 4 + k];
+    const float mu = (c == 0) ? gm : fblk(c - 1)[R::F_LAM / 4 + k] * gm;
+#pragma unroll
+    for (int cb = 0; cb < NV / 64; ++cb) {
+      const int col = ch * (NV / 2) + 32 * cb;
+      float x[32];
+      if (c == 0) {
+        if (a.S0) {
+          const float* src = a.S0 + ((int64_t)bh * DK + k) * dv + col0 + col;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 f = *reinterpret_cast<const float4*>(src + e);
+            x[e] = f.x, x[e + 1] = f.y, x[e + 2] = f.z, x[e + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] = 0.f;
+        }
+      } else {
+        tmem_ld32(tmem + lane_base + Ly::TM_S + col, x);
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] *= mu;
+      tmem_st32(tmem + lane_base + Ly::TM_S + col, x);
+#pragma unroll
+      for (int q8 = 0; q8 < 4; ++q8) {
+        uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
+                              pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
+        *reinterpret_cast<uint4*>(sm + Ly::SM + canon_chunk(k, col / 8 + q8, DK)) = pk;
+      }
+    }
+  };
+  // o rows of chunk c from rows 64..127 of D1 (quadrants 2 and 3, columns of half ch)
+  auto store_o = [&](int c) {
+    const int t = 32 * (q4 - 2) + lane, t0c = c * C, nc = min(C, T - t0c);
+    __nv_bfloat16* orow =
+        reinterpret_cast<__nv_bfloat16*>(a.o) + (((int64_t)b * T + t0c + t) * H + h) * dv + col0;
+#pragma unroll
+    for (int cb = 0; cb < NV / 64; ++cb) {
+      const int col = ch * (NV / 2) + 32 * cb;
+      float x[32];
+      tmem_ld32(tmem + lane_base + Ly::TM_D1 + col, x);
+      if (t < nc) {
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
+                                pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
+          *reinterpret_cast<uint4*>(orow + col + 8 * q8) = pk;
+        }
+      }
+    }
+  };
+  // a bounded wait by every thread; false (for all) if any thread's wait ran out
+  auto wait_all = [&](uint64_t* bar, uint32_t ph) -> bool {
+    return !__syncthreads_or(!mbar_wait_bounded(bar, ph, a.wait_ns));
+  };
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int n = min(C, T - c * C);
+    // ---- this chunk's [K+; Q+] (or raw k, q) and factors
+    if (!wait_all(&bar_kq, ph_kq)) {
+      failed = true;
+      break;
+    }
+    ph_kq ^= 1;
+    kq_p = false;
+    const float* fc = fblk(c);
+    const bool extreme = reinterpret_cast<const int*>(fc)[R::F_FLAG / 4] != 0;
+    // the next chunk's [T; P] into the buffer chunk c - 1 used (its products are done); the next
+    // record's [K+; Q+] into L2 (it is loaded once this chunk's D1 product has read the tile)
+    if (c + 1 < nchunks) {
+      if (tid == 0) {
+        if (c >= 1) issue_tp(c + 1);
+        bulk_prefetch(rec(c + 1) + R::KQ, 128 * DK * 2);
+        bulk_prefetch(rec(c + 1) + R::F, R::FBYTES);
+      }
+      tp_p[(c + 1) & 1] = true;
+    }
+
+    if (extreme) {
+      // V~ (read by the exact path); [T; P] and W- of the record are not used, their loads are awaited
+      if (!wait_all(&bar_v, ph_v) || !wait_all(&bar_tp[c & 1], ph_tp[c & 1]) || !wait_all(&bar_w, ph_w)) {
+        failed = true;
+        break;
+      }
+      ph_v ^= 1;
+      ph_w ^= 1;
+      ph_tp[c & 1] ^= 1;
+      v_p = w_p = tp_p[c & 1] = false;
+      if (o_pending && q4 >= 2) store_o(c - 1);
+      o_pending = false;
+      tc_fence_before();
+      const float* xa = reinterpret_cast<const float*>(rec(c) + R::x_off(dv, bv));
+      exact_chunk<DK, NV>(a, kq, kq + C * DK * 2, sm + Ly::STV, sm + Ly::VLO, bv, xa, xa + C * DK, fc + R::F_WQ / 4,
+                          reinterpret_cast<float*>(sm + Ly::UHI), fblk(c - 1) + R::F_LAM / 4, tmem + Ly::TM_S, c, n, b,
+                          h, bh, col0, tid);
+      // the state in tensor memory is now the true state: no pending chunk-end factor
+      if (tid < DK) fblk(c)[R::F_LAM / 4 + tid] = 1.f;
+      fence_proxy_async();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (c + 1 < nchunks) {
+        if (tid == 0) {
+          issue_kq(c + 1);
+          issue_w(c + 1);
+          issue_v(c + 1);
+        }
+        kq_p = w_p = v_p = true;
+      }
+      continue;
+    }
+
+    // ---- Wk = [T; P] K+ -> scratch;  U0 = [T; P] V~ -> U0
+    if (!wait_all(&bar_tp[c & 1], ph_tp[c & 1]) || !wait_all(&bar_v, ph_v)) {
+      failed = true;
+      break;
+    }
+    ph_v ^= 1;
+    ph_tp[c & 1] ^= 1;
+    tp_p[c & 1] = v_p = false;
+    if (tid == 0) {
+      const uint32_t tpa = smem_u32(tp_of(c));
+#pragma unroll
+      for (int kk = 0; kk < C; kk += 16) {
+        const uint64_t ad = sdesc(tpa + kk * 2, 16, 1024);
+        const uint64_t bk = sdesc(smem_u32(kq) + kk * 128, 128 * 128, 1024);
+        mma_bf16(tmem + Ly::TM_SCR, ad, bk, id_wk, kk > 0);
+      }
+#pragma unroll
+      for (int kk = 0; kk < C; kk += 16) {
+        const uint64_t ad = sdesc(tpa + kk * 2, 16, 1024);
+        const uint64_t bd = sdesc(smem_u32(sm + Ly::STV) + kk * 128, C * 128, 1024);
+        mma_bf16(tmem + Ly::TM_U0, ad, bd, id_nv, kk > 0);
+      }
+      if (bv) {
+#pragma unroll
+        for (int kk = 0; kk < C; kk += 16) {
+          const uint64_t ad = sdesc(tpa + kk * 2, 16, 1024);
+          const uint64_t bd = sdesc(smem_u32(sm + Ly::VLO) + kk * 128, C * 128, 1024);
+          mma_bf16(tmem + Ly::TM_U0, ad, bd, id_nv, 1);
+        }
+      }
+      mma_commit(&bar_mma);
+    }
+    mma_p = true;
+    // while those run: the previous chunk's outputs and the state in this chunk's frame
+    if (o_pending && q4 >= 2) store_o(c - 1);
+    state_to_frame(c);
+    if (!wait_all(&bar_mma, ph_mma)) {
+      failed = true;
+      break;
+    }
+    ph_mma ^= 1;
+    mma_p = false;
+    tc_fence_after();
+    if (c + 1 < nchunks) {
+      if (tid == 0) issue_v(c + 1);
+      v_p = true;
+    }
+
+    // ---- Wk -> bf16 into rows 0..63 of the [K+; Q+] tile (K+ is dead now)
+    if (q4 < 2) {
+      const int t = 32 * q4 + lane;
+#pragma unroll
+      for (int cb = 0; cb < DK / 64; ++cb) {
+        const int col = ch * (DK / 2) + 32 * cb;
+        float x[32];
+        tmem_ld32(tmem + lane_base + Ly::TM_SCR + col, x);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint4 pk = make_uint4(pack_bf16(x[8 * q8], x[8 * q8 + 1]), pack_bf16(x[8 * q8 + 2], x[8 * q8 + 3]),
+                                pack_bf16(x[8 * q8 + 4], x[8 * q8 + 5]), pack_bf16(x[8 * q8 + 6], x[8 * q8 + 7]));
+          *reinterpret_cast<uint4*>(kq + canon_chunk(t, col / 8 + q8, 128)) = pk;
+        }
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- D1 = [Wk; Q+] S_m
+    if (tid == 0) {
+#pragma unroll
+      for (int kk = 0; kk < DK; kk += 16) {
+        const uint64_t ad = sdesc(smem_u32(kq) + (kk >> 6) * (128 * 128) + (kk & 63) * 2, 16, 1024);
+        const uint64_t bd = sdesc(smem_u32(sm + Ly::SM) + kk * 128, DK * 128, 1024);
+        mma_bf16(tmem + Ly::TM_D1, ad, bd, id_nv, kk > 0);
+      }
+      mma_commit(&bar_mma);
+    }
+    mma_p = true;
+    if (!wait_all(&bar_mma, ph_mma)) {
+      failed = true;
+      break;
+    }
+    ph_mma ^= 1;
+    mma_p = false;
+    tc_fence_after();
+    // the [Wk; Q+] tile and the factor block of chunk c - 1 are free: the next record's tile and factors
+    if (c + 1 < nchunks) {
+      if (tid == 0) issue_kq(c + 1);
+      kq_p = true;
+    }
+
+    // ---- U = U0 - Wk S_m -> hi / lo tiles
+    if (q4 < 2) {
+      const int t = 32 * q4 + lane;
+#pragma unroll
+      for (int cb = 0; cb < NV / 64; ++cb) {
+        const int col = ch * (NV / 2) + 32 * cb;
+        float u0[32], d1[32];
+        tmem_ld32(tmem + lane_base + Ly::TM_U0 + col, u0);
+        tmem_ld32(tmem + lane_base + Ly::TM_D1 + col, d1);
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 8 * q8 + 2 * e;
+            split_bf16(u0[i] - d1[i], u0[i + 1] - d1[i + 1], hi[e], lo[e]);
+          }
+          const uint32_t o2 = canon_chunk(t, col / 8 + q8, C);
+          *reinterpret_cast<uint4*>(sm + Ly::UHI + o2) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(sm + Ly::ULO + o2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- O = Q+ S_m + P U (rows 64..127 of D1); S_acc += W-^T U (split)
+    if (!wait_all(&bar_w, ph_w)) {
+      failed = true;
+      break;
+    }
+    ph_w ^= 1;
+    w_p = false;
+    if (tid == 0) {
+      const uint32_t tpa = smem_u32(tp_of(c));
+#pragma unroll
+      for (int kk = 0; kk < C; kk += 16) {
+        const uint64_t ad = sdesc(tpa + kk * 2, 16, 1024);
+        const uint64_t bd = sdesc(smem_u32(sm + Ly::UHI) + kk * 128, C * 128, 1024);
+        mma_bf16(tmem + Ly::TM_D1, ad, bd, id_nv, 1);
+      }
+#pragma unroll
+      for (int kk = 0; kk < C; kk += 16) {
+        const uint64_t buh = sdesc(smem_u32(sm + Ly::UHI) + kk * 128, C * 128, 1024);
+        const uint64_t bul = sdesc(smem_u32(sm + Ly::ULO) + kk * 128, C * 128, 1024);
+        const uint64_t awh = sdesc(smem_u32(sm + Ly::WHI) + kk * 128, C * 128, 1024);
+        const uint64_t awl = sdesc(smem_u32(sm + Ly::WLO) + kk * 128, C * 128, 1024);
+        mma_bf16(tmem + Ly::TM_S, awh, buh, id_state, 1);
+        mma_bf16(tmem + Ly::TM_S, awh, bul, id_state, 1);
+        mma_bf16(tmem + Ly::TM_S, awl, buh, id_state, 1);
+      }
+      mma_commit(&bar_mma);
+    }
+    mma_p = true;
+    if (!wait_all(&bar_mma, ph_mma)) {
+      failed = true;
+      break;
+    }
+    ph_mma ^= 1;
+    mma_p = false;
+    tc_fence_after();
+    // W- hi and lo are free: the next record's
+    if (c + 1 < nchunks) {
+      if (tid == 0) issue_w(c + 1);
+      w_p = true;
+    }
+    // (this chunk's outputs are stored during the next chunk's first products, or after the loop)
+    o_pending = true;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+
+  if (!failed && nchunks > 0) {
+    if (o_pending && q4 >= 2) store_o(nchunks - 1);
+    // S_T = Diag(gamma_C / gamma_m) S_acc of the last chunk
+    const int k = 32 * q4 + lane;
+    const float lam = fblk(nchunks - 1)[R::F_LAM / 4 + k];
+#pragma unroll
+    for (int cb = 0; cb < NV / 64; ++cb) {
+      const int col = ch * (NV / 2) + 32 * cb;
+      float x[32];
+      tmem_ld32(tmem + lane_base + Ly::TM_S + col, x);
+      float* dst = a.S + ((int64_t)bh * DK + k) * dv + col0 + col;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(lam * x[e], lam * x[e + 1], lam * x[e + 2], lam * x[e + 3]);
+    }
+  }
+  if (failed) {
+    // drain whatever this CTA still has in flight (bounded), then report
+    if (kq_p) mbar_wait_bounded(&bar_kq, ph_kq, kWaitNs);
+    for (int i = 0; i < 2; ++i)
+      if (tp_p[i]) mbar_wait_bounded(&bar_tp[i], ph_tp[i], kWaitNs);
+    if (w_p) mbar_wait_bounded(&bar_w, ph_w, kWaitNs);
+    if (v_p) mbar_wait_bounded(&bar_v, ph_v, kWaitNs);
+    if (mma_p) mbar_wait_bounded(&bar_mma, ph_mma, kWaitNs);
+    if (tid == 0) atomicExch(a.status, kDevTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
 // ---------------------------------------------------------------- host side
 template <int DK, int NV>
 cudaError_t launch_impl(const Args& a, cudaStream_t s) {
@@ -865,7 +1583,47 @@ cudaError_t launch_impl(const Args& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Few sequences: twice their count still fits the SMs (148 when no device can be queried)
+bool few_sequences(const Args& a) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return (int64_t)a.B * a.H * 2 <= sms;
+}
+
+template <int NV>
+cudaError_t launch_split_impl(const Args& a, uint8_t* ws, cudaStream_t s) {
+  const int nc = (a.T + C - 1) / C;
+  const int psmem = PLayout<128>::TOTAL + 1024, csmem = XLayout<128, NV>::TOTAL + 1024;
+  cudaError_t e = cudaFuncSetAttribute(prep_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, psmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(chain_tc_kernel<128, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, csmem);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mv;
+  if (!make_bthd_map(&mv, a.v, a.dv, a.H, a.T, a.B, C)) return cudaErrorInvalidValue;
+  prep_tc_kernel<128><<<(unsigned)((int64_t)a.B * a.H * nc), kThreads, psmem, s>>>(a, ws, nc);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  chain_tc_kernel<128, NV><<<a.B * a.H * (a.dv / NV), kThreads, csmem, s>>>(mv, a, ws);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+// The split evaluation is taken when few sequences leave SMs idle (B H 2 <= SMs, the fused kernel's
+// column split): then the chunk-parallel prep runs on every SM and the chains only walk. With more
+// sequences the fused kernel keeps every SM busy already and the prep's extra work does not pay
+// (measured: kda, 128 sequences, 1.36 ms split against 1.34 ms fused).
+bool split_tc_supported(const Args& a) {
+  return chunk_tc_supported(a) && !per_token_tc(a) && few_sequences(a) &&
+         (int64_t)a.B * a.H * ((a.T + C - 1) / C) < ((int64_t)1 << 31);  // (one prep CTA per chunk)
+}
+
+size_t split_tc_workspace_bytes(const Args& a) {
+  return (size_t)a.B * a.H * ((a.T + C - 1) / C) * XRec<128>::stride(a.dv, a.beta_v != DN_GATE_ONE);
+}
+
+cudaError_t launch_split_tc(const Args& a, void* workspace, cudaStream_t s) {
+  return launch_split_impl<64>(a, static_cast<uint8_t*>(workspace), s);  // 64 value columns per chain
+}
 
 bool chunk_tc_supported(const Args& a) {
   return a.io_bf16 && a.dk == 128 && (a.dv == 128 || a.dv == 64) && a.chunk == C && a.T > 0;
@@ -883,10 +1641,7 @@ cudaError_t launch_chunk_tc(const Args& a, cudaStream_t s) {
   if (sc) return launch_chunk_sc(a, s);
   // few sequences: split the 128 value columns into two 64-column CTAs when that still fits in one
   // wave (each CTA repeats the column-independent prep, Gram and inverse)
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const bool split = a.dv == 128 && (int64_t)a.B * a.H * 2 <= sms;
-  if (a.dv == 128 && !split) return launch_impl<128, 128>(a, s);
+  if (a.dv == 128 && !few_sequences(a)) return launch_impl<128, 128>(a, s);
   return launch_impl<128, 64>(a, s);
 }
 

@@ -49,6 +49,11 @@ cudaError_t launch_chunk_sc(const Args& a, cudaStream_t s);
 bool per_token_tc(const Args& a);
 size_t split_sc_workspace_bytes(const Args& a);
 cudaError_t launch_split_sc(const Args& a, void* workspace, cudaStream_t s);
+// The split evaluation of the per-channel-gate problems (dn_chunk_tc.cu): whether it applies, its
+// workspace bytes, and the launch of its two kernels.
+bool split_tc_supported(const Args& a);
+size_t split_tc_workspace_bytes(const Args& a);
+cudaError_t launch_split_tc(const Args& a, void* workspace, cudaStream_t s);
 // OSDN phase 1 (dn_osdn.cu): workspace bytes, and the launch of its two kernels.
 size_t osdn_workspace_bytes(int B, int T, int H);
 cudaError_t launch_osdn(const void* k, const float* beta, const float* ret, const float* d0, float eta, int B,

@@ -136,9 +136,15 @@ def test_workspace_query(lib):
     assert dn.dn_chunk_fwd_workspace_bytes(_desc()) == _fwd32_bytes(1, 8, 2, 64, 64)
     assert dn.dn_chunk_fwd_workspace_bytes(_desc(io_dtype=dn.DN_F32, d_k=128, d_v=64, T=130)) == \
         _fwd32_bytes(1, 130, 2, 128, 64)
-    # small states and per-channel bf16 d_k = 128 take none
+    # small states take none; per-channel bf16 d_k = 128 takes one record per (b, h, chunk): [K+; Q+],
+    # [T; P], W- hi and lo, the factor block, V~ hi and lo when beta^v is given, alpha and w rows
     assert dn.dn_chunk_fwd_workspace_bytes(_desc(d_k=8, d_v=8)) == 0
-    assert dn.dn_chunk_fwd_workspace_bytes(_desc(d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL)) == 0
+    rec = 32768 + 16384 + 2 * 16384 + 2048 + 2 * 64 * 128 * 4
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL)) == 1 * 2 * 1 * rec
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(d_k=128, d_v=64, T=130, alpha=dn.DN_GATE_CHANNEL,
+                                                 beta_v=dn.DN_GATE_CHANNEL)) == 1 * 2 * 3 * (rec + 2 * 64 * 64 * 2)
+    # (taken for few sequences only, B H 2 <= SMs; more take the fused kernel without a workspace)
+    assert dn.dn_chunk_fwd_workspace_bytes(_desc(B=80, H=1, d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL)) == 0
     assert dn.dn_chunk_fwd_workspace_bytes(_desc(T=0)) == 0
     assert lib.dn_chunk_fwd_workspace_bytes(None) == 0
 
@@ -310,7 +316,6 @@ def test_chunk_fwd_workspace_checks(lib):
     d = _desc(d_k=128, d_v=128, T=100)
     need = lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(d))
     assert need == 2 * 2 * 25616  # B H chunks x record
-    assert lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(_desc(d_k=128, d_v=128, alpha=dn.DN_GATE_CHANNEL))) == 0
     assert lib.dn_chunk_fwd_workspace_bytes(ctypes.byref(_desc(d_k=128, d_v=128, io_dtype=dn.DN_F32))) == \
         _fwd32_bytes(1, 8, 2, 128, 128)
     big = np.zeros(1 << 20, dtype=np.uint8)
