@@ -289,10 +289,12 @@ def run_single_kernel(args):
     if not os.path.exists(dnbuild.LIB):
         dnbuild.build()
     name = {"chunk": WORKLOAD, "decode": DECODE, "osdn": "osdn_phase1", "bwd": WORKLOAD, "kda": "kda",
-            "fg2": "fg2_osdn_long"}[args.only]
+            "fg2": "fg2_osdn_long", "mc": WORKLOAD}[args.only]
     w = di.WORKLOADS[name]
     if args.batch:
         w = w.scaled(B=args.batch)
+    if args.seq:
+        w = w.scaled(T=args.seq)
     x = di.make_osdn_inputs(w) if args.only == "osdn" else di.make_inputs(w)
     eta = x.pop("eta", None)
 
@@ -311,8 +313,21 @@ def run_single_kernel(args):
         gout = dn.dn_chunk_bwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
                                xd["S0"], dO=gb["dO"], dS_T=gb["dS_T"], workspace=wsb)
 
+    if args.only == "mc":
+        # the Memory Caching read-out of the bench's leg: segments of 1024 tokens, their memories (the
+        # chunked pass's S_T of each segment, computed once here), residual gates
+        L = 1024
+        nseg = w.T // L
+        seg = lambda t: None if t is None else t.reshape(w.B * nseg, L, *t.shape[2:])
+        Mc = torch.empty((w.B * nseg, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+        o_mc = torch.empty((w.B, w.T, w.H, w.dv), dtype=xd["q"].dtype, device="cuda")
+        dn.dn_chunk_fwd(seg(xd["q"]), seg(xd["k"]), seg(xd["v"]), seg(xd["alpha"]), seg(xd["beta_k"]),
+                        seg(xd["beta_v"]), seg(xd["key_scale"]), None, o=o_mc.view(w.B * nseg, L, w.H, w.dv), S_T=Mc)
+
     def launch():
-        if args.only == "bwd":
+        if args.only == "mc":
+            dn.dn_mc_readout(xd["q"], Mc.view(w.B, nseg, w.H, w.dk, w.dv), None, o_mc, seg_len=L)
+        elif args.only == "bwd":
             dn.dn_chunk_bwd(xd["q"], xd["k"], xd["v"], xd["alpha"], xd["beta_k"], xd["beta_v"], xd["key_scale"],
                             xd["S0"], dO=gb["dO"], dS_T=gb["dS_T"], workspace=wsb, out=gout)
         elif args.only == "osdn":
@@ -335,16 +350,22 @@ def run_single_kernel(args):
     torch.cuda.synchronize()
     if dn.dn_stream_status() != dn.DN_OK:
         raise RuntimeError("device status")
-    print(json.dumps({"only": args.only, "workload": name, "batch": w.B, "steps": args.steps,
+    print(json.dumps({"only": args.only, "workload": name, "batch": w.B, "seq": w.T, "steps": args.steps,
                       "ms_per_launch": e0.elapsed_time(e1) / max(1, args.steps)}))
 
+
+# kernels per dn_chunk_fwd call of each configuration on a 148-SM B200: the chunk form in fp32 (three);
+# kda's 128 sequences fill the GPU, so the fused per-channel kernel (one); fg2_osdn_long's 32 leave SMs
+# idle, so the split evaluation (the chunk-parallel prep, then the chains: two)
+CONFIG_KERNELS = {"gdn_fp32_small": 3, "kda": 1, "fg2_osdn_long": 2}
 
 CONFIG_LEGS = {
     "gdn_fp32_small": "B=1 H=2 T=256 d_k=d_v=64 fp32 q/k/v, alpha~U(0.9,1) and beta per token, S0=0 "
                       "(chunk form in fp32: three kernels on split-TF32 warp tensor cores)",
-    "kda": "B=4 H=32 T=8192 d_k=d_v=128 bf16 q/k/v, channel alpha, beta per token, S0~N(0,0.02^2)",
+    "kda": "B=4 H=32 T=8192 d_k=d_v=128 bf16 q/k/v, channel alpha, beta per token, S0~N(0,0.02^2) "
+           "(fused per-channel kernel, one CTA per head)",
     "fg2_osdn_long": "B=2 H=16 T=32768 d_k=d_v=128 bf16 q/k/v, channel alpha, beta^k, beta^v, OSDN d, "
-                     "S0~N(0,0.02^2)",
+                     "S0~N(0,0.02^2) (split evaluation: chunk-parallel prep, then 64 chains of 64 columns)",
 }
 
 
@@ -418,7 +439,7 @@ def run_config_leg(name, peaks, stream, world, barrier, to_dev, want_cpu, reps):
         raise RuntimeError(f"device status after the {name} leg")
     ms = reduce_max(statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs), world)
     gbs = alg / (ms * 1e-3) / 1e9
-    leg = {"workload": f"{name}: {CONFIG_LEGS[name]}", "ms_per_call": ms,
+    leg = {"workload": f"{name}: {CONFIG_LEGS[name]}", "ms_per_call": ms, "kernels_per_call": CONFIG_KERNELS[name],
            "tokens_per_s": weak_scaling_rate(w.B * w.T, world, ms),
            "l2": "flushed (2 x L2 written) before every timed launch" if flush is not None
                  else f"inputs {alg / 1e6:.0f} MB per call > L2 (no flush)",
@@ -473,9 +494,10 @@ def main():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the gdn_fp32_small, kda and fg2_osdn_long workload legs")
     ap.add_argument("--decode-steps", type=int, default=100)
-    ap.add_argument("--only", choices=["chunk", "decode", "osdn", "bwd", "kda", "fg2"], default=None,
+    ap.add_argument("--only", choices=["chunk", "decode", "osdn", "bwd", "kda", "fg2", "mc"], default=None,
                     help="profiling mode: run just one kernel on the workload with batch --batch")
     ap.add_argument("--batch", type=int, default=0, help="with --only: batch size of the scaled workload")
+    ap.add_argument("--seq", type=int, default=0, help="with --only: sequence length of the scaled workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -762,7 +784,7 @@ def main():
             configs[name] = run_config_leg(name, peaks, stream, world, barrier, to_dev,
                                            want_cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline),
                                            reps=reps)
-            launches += reps
+            launches += reps * CONFIG_KERNELS[name]
             # the timed calls with other chunk lengths (three kernels each)
             launches += 3 * (2 * reps if di.WORKLOADS[name].io == "f32" else 2)
 
