@@ -136,8 +136,16 @@ typedef struct {
  *    chunk whose decay over half a chunk exceeds e^80 per channel is evaluated token by token
  *    inside the chain;
  *  - with workspace == NULL: the sequential fp32 kernel, token by token.
- * Both give the same results up to rounding. Other problems (small states, per-channel
- * gates at bf16 d_k = 128) take no workspace.
+ * Problems with a per-channel gate at bf16 d_k = 128 (KDA, FG2-GDN+, OSDN) whose sequences
+ * are few (B * H * 2 <= the device's SM count) have two as well:
+ *  - with a workspace of at least this size: a chunk-parallel kernel writes, per (b, h, chunk
+ *    of 64 tokens), the decay-scaled [K+; Q+] tile, the [T; P] tile, W- (bf16 hi and lo), a
+ *    2 KB factor block, V~ (hi and lo, when beta^v is given) and room for a chunk out of the
+ *    factors' range (its raw k, q tiles and fp32 alpha and w rows): 146 KB per chunk, 178 KB
+ *    with beta^v at d_v = 128; state-chain kernels of 64 value columns then read it back;
+ *  - with workspace == NULL, and for more sequences (where this returns 0): one fused kernel
+ *    per (b, h) and slice of value columns.
+ * Both give the same results up to rounding. Other problems (small states) take no workspace.
  */
 size_t dn_chunk_fwd_workspace_bytes(const dn_desc* desc);
 
