@@ -188,3 +188,31 @@ def test_split_wait_timeout_reports_status_and_recovers():
     assert dn.dn_stream_status() == dn.DN_OK
     o_ref, S_ref = oracle.fwd(**x)
     check(o, ST, o_ref, S_ref, "bf16")
+
+
+def test_split_without_start_state():
+    w = di.WORKLOADS["fg2_osdn_long"].scaled(B=1, H=3, T=150)
+    x = di.make_inputs(w)
+    x["S0"] = None
+    _both(w, x)
+
+
+def test_split_resume_in_place():
+    """S_T written over S0 (the caller resumes a sequence): the split evaluation over two pieces equals
+    the oracle over the whole sequence."""
+    w = di.WORKLOADS["kda"].scaled(B=1, H=3, T=300, s0_std=0.5)
+    x = di.make_inputs(w)
+    xd = to_device(x)
+    o_ref, S_ref = oracle.fwd(**x)
+    S = xd["S0"].clone()
+    o_parts = []
+    for lo, hi in ((0, 130), (130, 300)):
+        sl = lambda t: None if t is None else t[:, lo:hi].contiguous()
+        desc = dn.make_desc(sl(xd["q"]), sl(xd["v"]), sl(xd["alpha"]), sl(xd["beta_k"]), sl(xd["beta_v"]),
+                            sl(xd["key_scale"]))
+        assert dn.dn_chunk_fwd_workspace_bytes(desc) > 0
+        o, _ = dn.dn_chunk_fwd(sl(xd["q"]), sl(xd["k"]), sl(xd["v"]), sl(xd["alpha"]), sl(xd["beta_k"]),
+                               sl(xd["beta_v"]), sl(xd["key_scale"]), S, S_T=S)
+        o_parts.append(o)
+    assert dn.dn_stream_status() == dn.DN_OK
+    check(torch.cat(o_parts, dim=1), S, o_ref, S_ref, "bf16")
