@@ -996,8 +996,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep_tc_kernel(const Args a, uint
     for (int g = 0; g < 4; ++g) gm = mul4(gm, lds4(s_grp + g * DK, cb0));
 #pragma unroll
     for (int g = 4; g < 8; ++g) lm = mul4(lm, lds4(s_grp + g * DK, cb0));
-    sts4(rf + R::F_GM / 4, cb0, gm);
-    sts4(rf + R::F_LAM / 4, cb0, lm);
+    *reinterpret_cast<float4*>(rf + R::F_GM / 4 + cb0) = gm;  // (the record, global memory)
+    *reinterpret_cast<float4*>(rf + R::F_LAM / 4 + cb0) = lm;
     ok = ok && in_range4(gm) && in_range4(lm);
   }
   const bool extreme = __syncthreads_or(!ok);
@@ -1015,8 +1015,8 @@ __global__ void __launch_bounds__(kThreads, 2) prep_tc_kernel(const Args a, uint
       *reinterpret_cast<uint2*>(rec + R::KQ + C * DK * 2 + canon(j, cb0, C)) = qr[i];
       const float4 kk = unpack4(kr[i]), qq = unpack4(qr[i]);
       const float4 wv = mul4(ws4[i], kk);
-      sts4(xa, j * DK + cb0, al[i]);
-      sts4(xw, j * DK + cb0, wv);
+      *reinterpret_cast<float4*>(xa + j * DK + cb0) = al[i];
+      *reinterpret_cast<float4*>(xw + j * DK + cb0) = wv;
       wq[i] = wv.x * qq.x + wv.y * qq.y + wv.z * qq.z + wv.w * qq.w;
     }
 #pragma unroll
