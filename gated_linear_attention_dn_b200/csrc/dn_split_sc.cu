@@ -106,12 +106,15 @@ __global__ void __launch_bounds__(kThreads, kXformPerSm) xform_sc_kernel(const _
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q4 = warp & 3, gch = warp >> 2;
   const int pre = a.pre_read ? 1 : 0;
   const int nchunks = (a.T + C - 1) / C;
-  const int bh = blockIdx.x / nchunks, c = blockIdx.x % nchunks, b = bh / a.H, h = bh % a.H;
-  uint8_t* const rec = ws + (size_t)blockIdx.x * rec_stride(BV);
+  // blocks run chunk-major from the last chunk back to the first, so that the records (and q, k
+  // tiles) the state chains read first are the last ones written, still in L2 when the chains start
+  const int nbhs = a.B * a.H;
+  const int c = nchunks - 1 - (int)(blockIdx.x / nbhs), bh = (int)(blockIdx.x % nbhs), b = bh / a.H, h = bh % a.H;
+  uint8_t* const rec = ws + ((size_t)bh * nchunks + c) * rec_stride(BV);
   if (tid == 0) s_wide = 0;
   const int64_t nb = (int64_t)blockIdx.x + ahead;  // the block that takes this one's place on its SM
   const bool pf = ahead > 0 && nb < (int64_t)gridDim.x;
-  const int nbh = (int)(nb / nchunks), nc = (int)(nb % nchunks);
+  const int nc = nchunks - 1 - (int)(nb / nbhs), nbh = (int)(nb % nbhs);
 
   // thread 0 starts the [K; Q] load at once; warps 2 and 3 load the gates meanwhile (the factor scan
   // runs there, so that thread 0 is free to issue the Gram as soon as the tile lands)
