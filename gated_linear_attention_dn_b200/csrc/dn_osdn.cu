@@ -300,24 +300,36 @@ __global__ void __launch_bounds__(2 * DK) osdn_scan_kernel(const void* k, const 
     }
     __syncthreads();
     // d_t for this half's tokens; the second half starts from d_{t0 + 16}
+    // (every operand of the two dependent chains below is loaded first, so that each chain is a run
+    // of fused multiply-adds and not a shared-memory round trip per token)
     float d;
     if (half == 0) {
       d = dstart;
     } else {
-      d = s_rho16 * dstart;
+      float term[HM];
 #pragma unroll
       for (int i = 0; i < HM; ++i) {
         const float x = k_at(st, i);
-        d = fmaf(s_coef[i], x * x, d);
+        term[i] = s_coef[i] * (x * x);
       }
+      d = s_rho16 * dstart;
+#pragma unroll
+      for (int i = 0; i < HM; ++i) d += term[i];
     }
-    float* o = dout + (((int64_t)b * T + t0 + tb) * H + h) * DK + ch;
+    float rt[HM], ea[HM];
     const float* rr = s_r(st);
 #pragma unroll
     for (int t = 0; t < HM; ++t) {
-      if (tb + t < nb) {
+      rt[t] = ret ? rr[tb + t] : 1.f;
+      ea[t] = s_e[tb + t] * a[t];
+    }
+    float* o = dout + (((int64_t)b * T + t0 + tb) * H + h) * DK + ch;
+    const int nt = min(HM, nb - tb);  // this half's real tokens (none past the end)
+#pragma unroll
+    for (int t = 0; t < HM; ++t) {
+      if (t < nt) {
         o[(int64_t)t * H * DK] = d;
-        d = fmaf(ret ? rr[tb + t] : 1.f, d, s_e[tb + t] * a[t]);
+        d = fmaf(rt[t], d, ea[t]);
       }
     }
     // the block's final d: from the second half, or from the first when the block ends by token 16
