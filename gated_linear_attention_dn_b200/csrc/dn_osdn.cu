@@ -253,6 +253,15 @@ __global__ void __launch_bounds__(2 * DK) osdn_scan_kernel(const void* k, const 
       const float x = k_at(st, tb + t);
       a[t] = x * x;
     }
+    // the second half also takes the first half's a (its start d needs them after the last barrier)
+    float a0[HM];
+    if (half == 1) {
+#pragma unroll
+      for (int i = 0; i < HM; ++i) {
+        const float x = k_at(st, i);
+        a0[i] = x * x;
+      }
+    }
     // P_t = <d_{t0}, a_t> for this half's 16 tokens: a transposed butterfly over lanes 0..15's bit
     // pattern, then one exchange across lane bit 4; lane t (mod 16) ends with token t
     {
@@ -308,10 +317,7 @@ __global__ void __launch_bounds__(2 * DK) osdn_scan_kernel(const void* k, const 
     } else {
       float term[HM];
 #pragma unroll
-      for (int i = 0; i < HM; ++i) {
-        const float x = k_at(st, i);
-        term[i] = s_coef[i] * (x * x);
-      }
+      for (int i = 0; i < HM; ++i) term[i] = s_coef[i] * a0[i];
       d = s_rho16 * dstart;
 #pragma unroll
       for (int i = 0; i < HM; ++i) d += term[i];
