@@ -200,7 +200,6 @@ __global__ void __launch_bounds__(2 * DK) osdn_scan_kernel(const void* k, const 
   extern __shared__ __align__(16) float smem_raw[];  // same declaration type as the block kernel's
   uint8_t* const smem = reinterpret_cast<uint8_t*>(smem_raw);
   __shared__ float s_part[2][NW][HM];
-  __shared__ float s_P[kM];
   __shared__ float s_e[kM];
   __shared__ float s_coef[HM];  // R(i + 1, 16) e_i: the first half's writes as seen at token 16
   __shared__ float s_rho16;     // prod_{j < 16} r_j
@@ -284,17 +283,8 @@ __global__ void __launch_bounds__(2 * DK) osdn_scan_kernel(const void* k, const 
     __syncthreads();
     // e = u0 - B P (warp 0, lane t; B column-major), then the second half's start: R(i+1,16) e_i
     if (tid < 32) {
-      float P = 0.f;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) P += s_part[lane / HM][w][lane % HM];
-      s_P[lane] = P;
-      __syncwarp();
-      const float* bu = s_bu(st);
-      float e = bu[kM * kM + lane];
-#pragma unroll
-      for (int s2 = 0; s2 < kM; ++s2) e = fmaf(-bu[s2 * kM + lane], s_P[s2], e);
-      s_e[lane] = e;
       // suffix products over lanes 0..15: suf_i = prod_{i<j<16} r_j (exclusive), rho16 = prod_{j<16} r_j
+      // (they do not depend on P)
       const float rl = (ret && lane < HM) ? s_r(st)[lane] : 1.f;
       float incl = lane < HM ? rl : 1.f;
 #pragma unroll
@@ -304,6 +294,17 @@ __global__ void __launch_bounds__(2 * DK) osdn_scan_kernel(const void* k, const 
       }
       const float nxt = __shfl_down_sync(0xffffffffu, incl, 1);  // every lane takes part
       const float suf = lane == 31 ? 1.f : nxt;
+      float P = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) P += s_part[lane / HM][w][lane % HM];
+      // e_t = u0_t - sum_s B_ts P_s: P_s from lane s, four independent partial sums
+      const float* bu = s_bu(st);
+      float ep[4] = {bu[kM * kM + lane], 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s2 = 0; s2 < kM; ++s2)
+        ep[s2 & 3] = fmaf(-bu[s2 * kM + lane], __shfl_sync(0xffffffffu, P, s2), ep[s2 & 3]);
+      const float e = (ep[0] + ep[1]) + (ep[2] + ep[3]);
+      s_e[lane] = e;
       if (lane < HM) s_coef[lane] = suf * e;
       if (lane == 0) s_rho16 = incl;
     }
