@@ -841,20 +841,24 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
         }
     }
     __syncthreads();
-    // d log alpha_s = sum_{t >= s} dh_t + rowsum(dX (.) X) (the last token's share), per channel
+    // d log alpha_s = sum_{t >= s} dh_t + rowsum(dX (.) X) (the last token's share), per channel: the
+    // suffix sums in shared memory (a dependent chain over the tokens), then d alpha = d log alpha /
+    // alpha for every (token, channel) of the slice at once
     for (int il = tid; il < kDKS; il += kNT) {
       float run = red[il] + red[kDKS + il] + red[2 * kDKS + il] + red[3 * kDKS + il];
       for (int t = kC - 1; t >= 0; --t) {
         run += Wm[t * LDS + il];
-        const float dlog = a.pre_read ? run - Xq[t * LDS + il] : run;
-        if (t < n && a.alpha == DN_GATE_CHANNEL) {
-          const int64_t tok = token(a, b, h, t0 + t);
-          p.galpha[tok * DK + i0 + il] = dlog / gate_load(a.alpha_p, a.alpha, tok, DK, i0 + il);
-        }
-        Wm[t * LDS + il] = dlog;
+        Wm[t * LDS + il] = a.pre_read ? run - Xq[t * LDS + il] : run;
       }
     }
     __syncthreads();
+    if (a.alpha == DN_GATE_CHANNEL) {
+      for (int e = tid; e < n * kDKS; e += kNT) {
+        const int t = e / kDKS, il = e % kDKS;
+        const int64_t tok = token(a, b, h, t0 + t);
+        p.galpha[tok * DK + i0 + il] = Wm[t * LDS + il] / gate_load(a.alpha_p, a.alpha, tok, DK, i0 + il);
+      }
+    }
     // per-token sums over these channels, for gates of width 1
     if (tid < kC) {
       float sa = 0.f, sb = 0.f, sd = 0.f;
