@@ -500,57 +500,88 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
 }
 
 // ------------------------------------------------------------------ kernel 3: state adjoints, chunks in reverse
+// Each chunk's operands are copied in as soon as their buffers are free, so that a step of the chain
+// does not wait for its loads: W- and P (with e^r and lam, double-buffered) after the dU product, T
+// after the dV~ product, Q+ and K+ after the dS product, and dO (double-buffered) through registers
+// during the dV~ and dS products. cp.async groups per step, in issue order: A1 = {W-, P, e^r, lam},
+// A2 = {T}, B = {Q+, K+} (empty groups past the first chunk keep the count).
 template <int DK, int DV, int DVS>
 __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
   constexpr int LDK = DK + 4, LDS = DVS + 2, NI = DVS / 16;
+  constexpr int PER = kC * DVS / kNT;
   float* dS = reinterpret_cast<float*>(smem4);  // [DK][LDS]: dS', then dX, then dS
   float* Qp = dS + DK * LDS;                     // [C][LDK]
   float* Kp = Qp + kC * LDK;
   float* Wm = Kp + kC * LDK;
   float* Tm = Wm + kC * LDK;  // [C][kLDC]
   float* Pm = Tm + kC * kLDC;
-  float* dOs = Pm + kC * kLDC;  // [C][LDS]
-  float* dU = dOs + kC * LDS;   // [C][LDS]: dU, then dV~
-  float* er = dU + kC * LDS;
-  float* lam = er + DK;
+  float* dO0 = Pm + kC * kLDC;  // [C][LDS] x 2 (chunk parity)
+  float* dO1 = dO0 + kC * LDS;
+  float* dU = dO1 + kC * LDS;   // [C][LDS]: dU, then dV~
+  float* erb = dU + kC * LDS;   // [2][DK]
+  float* lamb = erb + 2 * DK;   // [2][DK]
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int NS = DV / DVS;
   const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * DVS, b = bh / a.H, h = bh % a.H;
+  auto cbk = [&](int c) { return (int64_t)bh * p.nc + c; };
+  auto issue_a1 = [&](int c) {
+    if (c >= 0) {
+      async_rows<kC, DK>(Wm, LDK, p.wWm + cbk(c) * kC * DK, DK, tid);
+      async_rows<kC, kC>(Pm, kLDC, p.wP + cbk(c) * kC * kC, kC, tid);
+      async_rows<1, DK>(erb + (c & 1) * DK, 0, p.wEr + cbk(c) * DK, 0, tid);
+      async_rows<1, DK>(lamb + (c & 1) * DK, 0, p.wLam + cbk(c) * DK, 0, tid);
+    }
+    tc::cp_async_commit();
+  };
+  auto issue_a2 = [&](int c) {
+    if (c >= 0) async_rows<kC, kC>(Tm, kLDC, p.wT + cbk(c) * kC * kC, kC, tid);
+    tc::cp_async_commit();
+  };
+  auto issue_b = [&](int c) {
+    if (c >= 0) {
+      async_rows<kC, DK>(Qp, LDK, p.wQp + cbk(c) * kC * DK, DK, tid);
+      async_rows<kC, DK>(Kp, LDK, p.wKp + cbk(c) * kC * DK, DK, tid);
+    }
+    tc::cp_async_commit();
+  };
+  auto load_dO = [&](int c, float* x) {
+    const int t0 = c * kC, n = min(kC, a.T - t0);
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
+      x[it] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j0 + j, a.io_bf16) : 0.f;
+    }
+  };
+  auto store_dO = [&](int c, const float* x) {
+    float* d = (c & 1) ? dO1 : dO0;
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * kNT;
+      d[(e / DVS) * LDS + e % DVS] = x[it];
+    }
+  };
   for (int e = tid; e < DK * DVS; e += kNT) {
     const int i = e / DVS, j = e % DVS;
     dS[i * LDS + j] = p.dS_T ? p.dS_T[((int64_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
+  if (p.nc > 0) {
+    issue_a1(p.nc - 1);
+    issue_a2(p.nc - 1);
+    issue_b(p.nc - 1);
+    float x[PER];
+    load_dO(p.nc - 1, x);
+    store_dO(p.nc - 1, x);
+  }
   const int m0 = (warp >> 1) * 16, n0 = (warp & 1) * (DVS / 2);
   for (int c = p.nc - 1; c >= 0; --c) {
-    const int t0 = c * kC, n = min(kC, a.T - t0);
-    const int64_t cb = (int64_t)bh * p.nc + c;
-    __syncthreads();
-    async_rows<kC, DK>(Qp, LDK, p.wQp + cb * kC * DK, DK, tid);
-    async_rows<kC, DK>(Kp, LDK, p.wKp + cb * kC * DK, DK, tid);
-    async_rows<kC, DK>(Wm, LDK, p.wWm + cb * kC * DK, DK, tid);
-    async_rows<kC, kC>(Tm, kLDC, p.wT + cb * kC * kC, kC, tid);
-    async_rows<kC, kC>(Pm, kLDC, p.wP + cb * kC * kC, kC, tid);
-    async_rows<1, DK>(er, 0, p.wEr + cb * DK, 0, tid);
-    async_rows<1, DK>(lam, 0, p.wLam + cb * DK, 0, tid);
-    tc::cp_async_commit();
-    {
-      constexpr int PER = kC * DVS / kNT;
-      float x[PER];
-#pragma unroll
-      for (int it = 0; it < PER; ++it) {
-        const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
-        x[it] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j0 + j, a.io_bf16) : 0.f;
-      }
-#pragma unroll
-      for (int it = 0; it < PER; ++it) {
-        const int e = tid + it * kNT;
-        dOs[(e / DVS) * LDS + e % DVS] = x[it];
-      }
-    }
-    tc::cp_async_wait_all();
-    __syncthreads();
+    const int64_t cb = cbk(c);
+    const float* dOs = (c & 1) ? dO1 : dO0;
+    const float* er = erb + (c & 1) * DK;
+    const float* lam = lamb + (c & 1) * DK;
+    tc::cp_async_wait_group<1>();  // A1(c) and A2(c) have landed (B(c) may still be in flight)
+    __syncthreads();               // and for every thread; dO(c) is stored; the previous step is done
     float* dXg = p.wdX + cb * DK * DV;
     for (int e = tid; e < DK * DVS; e += kNT) {
       const int i = e / DVS, j = e % DVS;
@@ -570,6 +601,9 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
       warp_epilogue(acc, [&](int m, int nn, float v) { dU[(m0 + m) * LDS + n0 + nn] = v; }, lane);
     }
     __syncthreads();
+    issue_a1(c - 1);  // W- and P are free
+    float xo[PER];
+    if (c > 0) load_dO(c - 1, xo);
     {  // dV~ = T^T dU
       float acc[1][NI][4] = {};
       warp_gemm<1, NI, kC>(
@@ -584,6 +618,8 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
                     },
                     lane);
     }
+    issue_a2(c - 1);               // T is free (every warp passed the barrier inside the product above)
+    tc::cp_async_wait_group<2>();  // B(c) has landed (A1(c - 1), A2(c - 1) may still be in flight)
     __syncthreads();
     // dS = Diag(e^r) (dX + Q+^T dO - K+^T dV~): DK x DVS in 16 x DVS/2 tiles
     for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
@@ -602,7 +638,11 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
                     },
                     lane);
     }
+    __syncthreads();  // Q+, K+ and dO(c + 1)'s buffer are free
+    issue_b(c - 1);
+    if (c > 0) store_dO(c - 1, xo);
   }
+  tc::cp_async_wait_all();
   if (p.gS0) {
     __syncthreads();
     for (int e = tid; e < DK * DVS; e += kNT) {
@@ -934,7 +974,7 @@ constexpr size_t state_smem() {
 }
 template <int DK, int DVS>
 constexpr size_t dstate_smem() {
-  return sizeof(float) * (DK * (DVS + 2) + 3 * kC * (DK + 4) + 2 * kC * kLDC + 2 * kC * (DVS + 2) + 2 * DK);
+  return sizeof(float) * (DK * (DVS + 2) + 3 * kC * (DK + 4) + 2 * kC * kLDC + 3 * kC * (DVS + 2) + 4 * DK);
 }
 template <int DV>
 constexpr size_t local_smem() {
