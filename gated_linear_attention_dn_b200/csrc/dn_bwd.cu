@@ -355,23 +355,67 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   float* Wm = Kp + C * LDK;                     // [C][LDK]
   float* Tm = Wm + C * LDK;                     // [C][LDC]
   float* R = Tm + C * LDC;                      // [C][LDS]: V~ - K+ S_m, then U
-  float* er = R + C * LDS;
-  float* lam = er + DK;
+  float* erb = R + C * LDS;                     // [2][DK] (chunk parity)
+  float* lamb = erb + 2 * DK;                   // [2][DK]
   const Args& a = p.f;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int NS = DV / DVS;
+  constexpr int PER = C * DVS / kNT;
   const int bh = blockIdx.x / NS, j0 = (blockIdx.x % NS) * DVS, b = bh / a.H, h = bh % a.H;
+  // Each chunk's operands are copied in as soon as their buffers are free (K+ with e^r and lam after
+  // the K+ S_m product, T after U = T R, W- after the state update) and V~ comes in through registers
+  // during the state update, so that a step does not wait for its loads. cp.async groups per chunk, in
+  // issue order: A1 = {K+, e^r, lam}, A2 = {T}, B = {W-} (empty past the last chunk).
+  auto cbk = [&](int c) { return (int64_t)bh * p.nc + c; };
+  auto issue_a1 = [&](int c) {
+    if (c < p.nc) {
+      async_rows<C, DK>(Kp, LDK, p.wKp + cbk(c) * C * DK, DK, tid);
+      async_rows<1, DK>(erb + (c & 1) * DK, 0, p.wEr + cbk(c) * DK, 0, tid);
+      async_rows<1, DK>(lamb + (c & 1) * DK, 0, p.wLam + cbk(c) * DK, 0, tid);
+    }
+    tc::cp_async_commit();
+  };
+  auto issue_a2 = [&](int c) {
+    if (c < p.nc) async_rows<C, C>(Tm, LDC, p.wT + cbk(c) * C * C, C, tid);
+    tc::cp_async_commit();
+  };
+  auto issue_b = [&](int c) {
+    if (c < p.nc) async_rows<C, DK>(Wm, LDK, p.wWm + cbk(c) * C * DK, DK, tid);
+    tc::cp_async_commit();
+  };
+  auto load_v = [&](int c, float* x) {  // V~ = beta^v v of chunk c, this thread's elements
+    const int t0 = c * C, n = min(C, a.T - t0);
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
+      x[it] = 0.f;
+      if (t < n) {
+        const int64_t tok = token(a, b, h, t0 + t);
+        x[it] = gate_load(a.beta_v_p, a.beta_v, tok, DV, j0 + j) * io_load(a.v, tok * DV + j0 + j, a.io_bf16);
+      }
+    }
+  };
   for (int e = tid; e < DK * DVS; e += kNT) {
     const int i = e / DVS, j = e % DVS;
     S[i * LDS + j] = a.S0 ? a.S0[((int64_t)bh * DK + i) * DV + j0 + j] : 0.f;
   }
   const bool tiled = warp < RT * CT;
   const int m0 = (warp / CT) * 16, n0 = (warp % CT) * TW;  // this warp's tile of a C x DVS result
+  float xv[PER];
+  if (p.nc > 0) {
+    issue_a1(0);
+    issue_a2(0);
+    issue_b(0);
+    load_v(0, xv);
+  }
   for (int c = 0; c < p.nc; ++c) {
     const int t0 = c * C, n = min(C, a.T - t0);
     const int64_t cb = (int64_t)bh * p.nc + c;
+    const float* er = erb + (c & 1) * DK;
+    const float* lam = lamb + (c & 1) * DK;
     __syncthreads();  // the previous chunk is done with every buffer
     if (p.wFlag && p.wFlag[cb]) {
+      tc::cp_async_wait_all();  // (this chunk's copies are not used; none may still be in flight below)
       // (forward) a chunk beyond the factorisation's range: its tokens one by one, exactly, on this
       // CTA's columns; thread (j, part) owns column j and DK / TPC rows of it, so the sums over the
       // rows take TPC - 1 shuffles. S holds the true state before and after.
@@ -414,33 +458,18 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
       }
 #pragma unroll
       for (int r = 0; r < RW; ++r) S[(k0 + r) * LDS + j] = Sr[r];
+      issue_a1(c + 1);
+      issue_a2(c + 1);
+      issue_b(c + 1);
+      if (c + 1 < p.nc) load_v(c + 1, xv);
       continue;
     }
-    async_rows<C, DK>(Kp, LDK, p.wKp + cb * C * DK, DK, tid);
-    async_rows<C, DK>(Wm, LDK, p.wWm + cb * C * DK, DK, tid);
-    async_rows<C, C>(Tm, LDC, p.wT + cb * C * C, C, tid);
-    async_rows<1, DK>(er, 0, p.wEr + cb * DK, 0, tid);
-    async_rows<1, DK>(lam, 0, p.wLam + cb * DK, 0, tid);
-    tc::cp_async_commit();
-    {
-      constexpr int PER = C * DVS / kNT;
-      float x[PER];
 #pragma unroll
-      for (int it = 0; it < PER; ++it) {
-        const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
-        x[it] = 0.f;
-        if (t < n) {
-          const int64_t tok = token(a, b, h, t0 + t);
-          x[it] = gate_load(a.beta_v_p, a.beta_v, tok, DV, j0 + j) * io_load(a.v, tok * DV + j0 + j, a.io_bf16);
-        }
-      }
-#pragma unroll
-      for (int it = 0; it < PER; ++it) {
-        const int e = tid + it * kNT;
-        R[(e / DVS) * LDS + e % DVS] = x[it];
-      }
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * kNT;
+      R[(e / DVS) * LDS + e % DVS] = xv[it];
     }
-    tc::cp_async_wait_all();
+    tc::cp_async_wait_group<2>();  // A1(c) has landed (A2(c), B(c) may still be in flight)
     __syncthreads();
     float* Smg = p.wSm + cb * DK * DV;
     for (int e = tid; e < DK * DVS; e += kNT) {
@@ -457,7 +486,9 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
           lane);
       warp_epilogue(acc, [&](int m, int nn, float v) { R[(m0 + m) * LDS + n0 + nn] -= v; }, lane);
     }
+    tc::cp_async_wait_group<1>();  // A2(c) has landed (B(c) may still be in flight)
     __syncthreads();
+    issue_a1(c + 1);  // K+ is free
     {  // U = T R
       float acc[1][NIT][4] = {};
       if (tiled)
@@ -465,6 +496,7 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
             acc, [&](int m, int k) { return Tm[(m0 + m) * LDC + k]; }, [&](int k, int nn) { return R[k * LDS + n0 + nn]; },
             lane);
       __syncthreads();
+      issue_a2(c + 1);  // T is free
       float* Ug = p.wU + cb * C * DV;
       if (tiled)
         warp_epilogue(acc,
@@ -474,6 +506,8 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
                       },
                       lane);
     }
+    if (c + 1 < p.nc) load_v(c + 1, xv);
+    tc::cp_async_wait_group<2>();  // B(c) has landed (A1(c + 1), A2(c + 1) may still be in flight)
     __syncthreads();
     // S' = Diag(lam) (S_m + W-^T U): DK x DVS in 16 x DVS/2 tiles
     for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
@@ -489,7 +523,10 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
                     },
                     lane);
     }
+    __syncthreads();  // W- is free
+    issue_b(c + 1);
   }
+  tc::cp_async_wait_all();
   if (p.wFlag) {  // (forward) S_T
     __syncthreads();
     for (int e = tid; e < DK * DVS; e += kNT) {
@@ -970,7 +1007,7 @@ constexpr size_t prep_smem() {
 }
 template <int DK, int DVS, int C = kC>
 constexpr size_t state_smem() {
-  return sizeof(float) * (DK * (DVS + 2) + 2 * C * (DK + 4) + C * (C + 4) + C * (DVS + 2) + 2 * DK);
+  return sizeof(float) * (DK * (DVS + 2) + 2 * C * (DK + 4) + C * (C + 4) + C * (DVS + 2) + 4 * DK);
 }
 template <int DK, int DVS>
 constexpr size_t dstate_smem() {
