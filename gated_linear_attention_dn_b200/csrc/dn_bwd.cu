@@ -132,6 +132,38 @@ __device__ __forceinline__ int64_t token(const Args& a, int b, int h, int t) {
   return ((int64_t)b * a.T + t) * a.H + h;
 }
 
+// Batched loads: N elements (token row tok0 + tt[u] H, channel / column ch[u]) of q, k or v and of a
+// gate, every load issued before any value is used (the dtype and gate-mode branches are uniform and
+// outside the element loop), so that they are all in flight at once. The caller clamps tt to a real
+// token and masks the values of elements past the end.
+template <int N>
+__device__ __forceinline__ void io_load_n(float* out, const void* p, int64_t tok0, const int* tt, int H, const int* ch,
+                                          int width, int bf16) {
+  if (bf16) {
+    const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p);
+#pragma unroll
+    for (int u = 0; u < N; ++u) out[u] = __bfloat162float(q[(tok0 + (int64_t)tt[u] * H) * width + ch[u]]);
+  } else {
+    const float* q = reinterpret_cast<const float*>(p);
+#pragma unroll
+    for (int u = 0; u < N; ++u) out[u] = q[(tok0 + (int64_t)tt[u] * H) * width + ch[u]];
+  }
+}
+template <int N>
+__device__ __forceinline__ void gate_load_n(float* out, const float* g, int mode, int64_t tok0, const int* tt, int H,
+                                            const int* ch, int width) {
+  if (mode == DN_GATE_CHANNEL) {
+#pragma unroll
+    for (int u = 0; u < N; ++u) out[u] = g[(tok0 + (int64_t)tt[u] * H) * width + ch[u]];
+  } else if (mode == DN_GATE_SCALAR) {
+#pragma unroll
+    for (int u = 0; u < N; ++u) out[u] = g[tok0 + (int64_t)tt[u] * H];
+  } else {
+#pragma unroll
+    for (int u = 0; u < N; ++u) out[u] = 1.f;
+  }
+}
+
 // Key channels [i0, i0 + NCH) of the chunk starting at token t0 (n valid tokens) of head (b, h), into
 // [C][NCH + 4] arrays: hb = h_t, Kp = k e^h, Qp = q e^h, Wm = w e^-h (Kp, Qp may be null; hb may be
 // Wm itself), er = e^r, lam = e^{g_last - r}; e^h also to global ehg ([C][NCH]) when not null.
@@ -144,17 +176,23 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
   static_assert(PER * kNT == C * NCH && PER % BAT == 0, "work split");
   // Every loop below first loads a batch into registers and only then computes and stores to
   // shared memory, so a thread's global loads are all in flight at once.
-  {
-    float al[PER];
+  const int64_t tok0 = token(a, b, h, t0);
+  constexpr int BA = PER < 16 ? PER : 16;
+  static_assert(PER % BA == 0, "work split");
+  for (int it0 = 0; it0 < PER; it0 += BA) {
+    float al[BA];
+    int tt[BA], ci[BA];
 #pragma unroll
-    for (int it = 0; it < PER; ++it) {
-      const int e = tid + it * kNT, t = e / NCH, i = e % NCH;
-      al[it] = t < n ? gate_load(a.alpha_p, a.alpha, token(a, b, h, t0 + t), a.dk, i0 + i) : 1.f;
+    for (int u = 0; u < BA; ++u) {
+      const int e = tid + (it0 + u) * kNT, t = e / NCH, i = e % NCH;
+      tt[u] = t < n ? t : 0;
+      ci[u] = i0 + i;
     }
+    gate_load_n<BA>(al, a.alpha_p, a.alpha, tok0, tt, a.H, ci, a.dk);
 #pragma unroll
-    for (int it = 0; it < PER; ++it) {
-      const int e = tid + it * kNT, t = e / NCH, i = e % NCH;
-      hb[t * LD + i] = logf(al[it]);
+    for (int u = 0; u < BA; ++u) {
+      const int e = tid + (it0 + u) * kNT, t = e / NCH, i = e % NCH;
+      hb[t * LD + i] = logf(t < n ? al[u] : 1.f);
     }
   }
   __syncthreads();
@@ -185,20 +223,29 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
   }
   __syncthreads();
   for (int it0 = 0; it0 < PER; it0 += BAT) {
-    float kk[BAT], qq[BAT], ws[BAT];
+    float kk[BAT], qq[BAT], ws[BAT], dd[BAT], al2[BAT];
+    int tt[BAT], ci[BAT];
 #pragma unroll
     for (int u = 0; u < BAT; ++u) {
       const int e = tid + (it0 + u) * kNT, t = e / NCH, i = e % NCH;
-      kk[u] = qq[u] = ws[u] = 0.f;
+      tt[u] = t < n ? t : 0;
+      ci[u] = i0 + i;
+    }
+    io_load_n<BAT>(kk, a.k, tok0, tt, a.H, ci, a.dk, a.io_bf16);
+    if (Qp) io_load_n<BAT>(qq, a.q, tok0, tt, a.H, ci, a.dk, a.io_bf16);
+    gate_load_n<BAT>(ws, a.beta_k_p, a.beta_k, tok0, tt, a.H, ci, a.dk);
+    gate_load_n<BAT>(dd, a.key_scale_p, a.key_scale, tok0, tt, a.H, ci, a.dk);
+    if (Qp && a.pre_read) gate_load_n<BAT>(al2, a.alpha_p, a.alpha, tok0, tt, a.H, ci, a.dk);
+#pragma unroll
+    for (int u = 0; u < BAT; ++u) {
+      const int e = tid + (it0 + u) * kNT, t = e / NCH;
       if (t < n) {
-        const int64_t tok = token(a, b, h, t0 + t);
-        kk[u] = io_load(a.k, tok * a.dk + i0 + i, a.io_bf16);
-        if (Qp) {
-          qq[u] = io_load(a.q, tok * a.dk + i0 + i, a.io_bf16);
-          if (a.pre_read) qq[u] /= gate_load(a.alpha_p, a.alpha, tok, a.dk, i0 + i);  // read before the decay
-        }
-        ws[u] = gate_load(a.beta_k_p, a.beta_k, tok, a.dk, i0 + i) * gate_load(a.key_scale_p, a.key_scale, tok, a.dk, i0 + i);
+        ws[u] *= dd[u];
+        if (Qp && a.pre_read) qq[u] /= al2[u];  // read before the decay
+      } else {
+        kk[u] = qq[u] = ws[u] = 0.f;
       }
+      if (!Qp) qq[u] = 0.f;
     }
 #pragma unroll
     for (int u = 0; u < BAT; ++u) {
@@ -385,14 +432,21 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   };
   auto load_v = [&](int c, float* x) {  // V~ = beta^v v of chunk c, this thread's elements
     const int t0 = c * C, n = min(C, a.T - t0);
+    const int64_t tok0 = token(a, b, h, t0);
+    int tt[PER], cj[PER];
+    float bv[PER];
 #pragma unroll
     for (int it = 0; it < PER; ++it) {
       const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
-      x[it] = 0.f;
-      if (t < n) {
-        const int64_t tok = token(a, b, h, t0 + t);
-        x[it] = gate_load(a.beta_v_p, a.beta_v, tok, DV, j0 + j) * io_load(a.v, tok * DV + j0 + j, a.io_bf16);
-      }
+      tt[it] = t < n ? t : 0;
+      cj[it] = j0 + j;
+    }
+    io_load_n<PER>(x, a.v, tok0, tt, a.H, cj, DV, a.io_bf16);
+    gate_load_n<PER>(bv, a.beta_v_p, a.beta_v, tok0, tt, a.H, cj, DV);
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int t = (tid + it * kNT) / DVS;
+      x[it] = t < n ? x[it] * bv[it] : 0.f;
     }
   };
   for (int e = tid; e < DK * DVS; e += kNT) {
