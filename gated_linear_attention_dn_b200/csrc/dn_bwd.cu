@@ -639,11 +639,18 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   };
   auto load_dO = [&](int c, float* x) {
     const int t0 = c * kC, n = min(kC, a.T - t0);
+    const int64_t tok0 = token(a, b, h, t0);
+    int tt[PER], cj[PER];
 #pragma unroll
     for (int it = 0; it < PER; ++it) {
       const int e = tid + it * kNT, t = e / DVS, j = e % DVS;
-      x[it] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j0 + j, a.io_bf16) : 0.f;
+      tt[it] = t < n ? t : 0;
+      cj[it] = j0 + j;
     }
+    io_load_n<PER>(x, p.dO, tok0, tt, a.H, cj, DV, a.io_bf16);
+#pragma unroll
+    for (int it = 0; it < PER; ++it)
+      if ((tid + it * kNT) / DVS >= n) x[it] = 0.f;
   };
   auto store_dO = [&](int c, const float* x) {
     float* d = (c & 1) ? dO1 : dO0;
@@ -785,17 +792,21 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
       *reinterpret_cast<float4*>(&U[t * LDV + j]) = xu[it];
       *reinterpret_cast<float4*>(&dVt[t * LDV + j]) = xv[it];
     }
+    const int64_t tok0 = token(a, b, h, t0);
     for (int it0 = 0; it0 < kC * DV / kNT; it0 += 8) {
       float x[8];
+      int tt[8], cj[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
-        x[u] = t < n ? io_load(p.dO, token(a, b, h, t0 + t) * DV + j, a.io_bf16) : 0.f;
+        tt[u] = t < n ? t : 0;
+        cj[u] = j;
       }
+      io_load_n<8>(x, p.dO, tok0, tt, a.H, cj, DV, a.io_bf16);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int e = tid + (it0 + u) * kNT;
-        dOs[(e / DV) * LDV + e % DV] = x[u];
+        dOs[(e / DV) * LDV + e % DV] = (e / DV) < n ? x[u] : 0.f;
       }
     }
     if (tid < kC) acc_a[tid] = acc_bk[tid] = acc_d[tid] = 0.f;
@@ -804,15 +815,17 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   // dv = beta^v dV~, and the beta^v gradient v dV~ (summed over channels for a per-token gate)
   for (int it0 = 0; it0 < kC * DV / kNT; it0 += 8) {
     float bv[8], vv[8];
+    int tt[8], cj[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
-      bv[u] = vv[u] = 0.f;
-      if (t < n) {
-        const int64_t tok = token(a, b, h, t0 + t);
-        bv[u] = gate_load(a.beta_v_p, a.beta_v, tok, DV, j);
-        if (a.beta_v == DN_GATE_CHANNEL) vv[u] = io_load(a.v, tok * DV + j, a.io_bf16);
-      }
+      tt[u] = t < n ? t : 0;
+      cj[u] = j;
+    }
+    {
+      const int64_t tok0 = token(a, b, h, t0);
+      gate_load_n<8>(bv, a.beta_v_p, a.beta_v, tok0, tt, a.H, cj, DV);
+      if (a.beta_v == DN_GATE_CHANNEL) io_load_n<8>(vv, a.v, tok0, tt, a.H, cj, DV, a.io_bf16);
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -919,21 +932,32 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
       // thread then reads and writes only its own elements of hb, Qp, Kp, Wm.
       float gq[2][4], gk[2][4], lk[2][4], lb[2][4], ld[2][4], la[2][4];
       const int g = lane >> 2, t4 = lane & 3;
+      {  // the inputs of this thread's elements, every load issued before any is used
+        int tt[8], ci[8];
 #pragma unroll
-      for (int ni = 0; ni < 2; ++ni)
+        for (int ni = 0; ni < 2; ++ni)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {  // the inputs of this thread's elements, loaded up front
-          const int t = m0 + g + (q >> 1) * 8, gi = i0 + n0 + 8 * ni + 2 * t4 + (q & 1);
-          lk[ni][q] = 0.f;
-          lb[ni][q] = ld[ni][q] = la[ni][q] = 1.f;
-          if (t < n) {
-            const int64_t tok = token(a, b, h, t0 + t);
-            lk[ni][q] = io_load(a.k, tok * DK + gi, a.io_bf16);
-            lb[ni][q] = gate_load(a.beta_k_p, a.beta_k, tok, DK, gi);
-            ld[ni][q] = gate_load(a.key_scale_p, a.key_scale, tok, DK, gi);
-            if (a.pre_read) la[ni][q] = gate_load(a.alpha_p, a.alpha, tok, DK, gi);
+          for (int q = 0; q < 4; ++q) {
+            const int t = m0 + g + (q >> 1) * 8;
+            tt[4 * ni + q] = t < n ? t : 0;
+            ci[4 * ni + q] = i0 + n0 + 8 * ni + 2 * t4 + (q & 1);
           }
-        }
+        const int64_t tok0 = token(a, b, h, t0);
+        io_load_n<8>(&lk[0][0], a.k, tok0, tt, a.H, ci, DK, a.io_bf16);
+        gate_load_n<8>(&lb[0][0], a.beta_k_p, a.beta_k, tok0, tt, a.H, ci, DK);
+        gate_load_n<8>(&ld[0][0], a.key_scale_p, a.key_scale, tok0, tt, a.H, ci, DK);
+        if (a.pre_read) gate_load_n<8>(&la[0][0], a.alpha_p, a.alpha, tok0, tt, a.H, ci, DK);
+#pragma unroll
+        for (int ni = 0; ni < 2; ++ni)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (!a.pre_read) la[ni][q] = 1.f;
+            if (m0 + g + (q >> 1) * 8 >= n) {
+              lk[ni][q] = 0.f;
+              lb[ni][q] = ld[ni][q] = la[ni][q] = 1.f;
+            }
+          }
+      }
       auto elem = [&](int ni, int q, int m, int nn, float vq, float vk, float vw) {
         const int t = m0 + m, il = n0 + nn;
         const float eh = Eh[t * LDS + il];
