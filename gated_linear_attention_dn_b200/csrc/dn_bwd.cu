@@ -69,9 +69,13 @@ struct BwdArgs {
 };
 
 // ------------------------------------------------------------------ warp tensor-core products
+// x = hi + lo: hi is x with the 13 low mantissa bits cleared (a TF32 value, taken with one logic op
+// rather than a conversion) and lo = x - hi, exact in fp32. lo goes to the tensor core as it is: a
+// TF32 operand's low 13 bits are not read, so lo enters truncated, off by less than 2^-10 |lo|, that
+// is 2^-20 |x|, the size of the lo * lo product the split leaves out.
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  hi = ut::to_tf32(x);
-  lo = ut::to_tf32(x - __uint_as_float(hi));
+  hi = __float_as_uint(x) & 0xffffe000u;
+  lo = __float_as_uint(x - __uint_as_float(hi));
 }
 
 // acc[MI][NI] (16 x 8 fragments) += sum_{k < K} A(m, k) B(k, n) over the warp tile of 16 MI rows and
