@@ -116,6 +116,68 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, i
   }
 }
 
+// Four 8 x 4 tiles of 32-bit words from shared memory, one register per tile and lane: lane l gives
+// the address of row l % 8 of tile l / 8 and receives word l % 4 of row l / 4 of each tile (the b16
+// matrix load moves every 32-bit word whole, as two adjacent 16-bit elements). For rows of fp32
+// values with k contiguous this is the m16n8k8 TF32 fragment of A, or of B stored n by k.
+__device__ __forceinline__ void ldm_x4(uint32_t (&r)[4], const float* row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(tc::smem_u32(row))
+               : "memory");
+}
+
+__device__ __forceinline__ void split_bits(uint32_t w, uint32_t& hi, uint32_t& lo) {
+  split_tf32(__uint_as_float(w), hi, lo);
+}
+
+// acc[a][MI][NI] += A_a B^T over K for NA operands A_a sharing B: each A_a is a warp tile of 16 MI
+// rows, B one of 8 NI rows (NI even), both fp32 in shared memory with k contiguous (row strides lda,
+// ldb: multiples of 4 floats, 16-byte aligned rows), fragments taken by matrix loads and split as
+// in warp_gemm.
+template <int NA, int MI, int NI, int K>
+__device__ __forceinline__ void warp_gemm_ldm(float (&acc)[NA][MI][NI][4], const float* const (&A)[NA], int lda,
+                                              const float* Bt, int ldb, int lane) {
+  static_assert(NI % 2 == 0 && K % 8 == 0, "tiles");
+  const int j = lane >> 3, r = lane & 7;
+  const int aoff = ((j & 1) * 8 + r) * lda + (j >> 1) * 4;  // tiles: rows 0-7 / 8-15, k 0-3 / 4-7
+  const int boff = ((j >> 1) * 8 + r) * ldb + (j & 1) * 4;  // tiles: n 0-7 / 8-15, k 0-3 / 4-7
+#pragma unroll 4
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t bh[NI][2], bl[NI][2];
+#pragma unroll
+    for (int np = 0; np < NI / 2; ++np) {
+      uint32_t w[4];
+      ldm_x4(w, Bt + 16 * np * ldb + boff + k0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) split_bits(w[q], bh[2 * np + (q >> 1)][q & 1], bl[2 * np + (q >> 1)][q & 1]);
+    }
+#pragma unroll
+    for (int a = 0; a < NA; ++a) {
+      uint32_t ah[MI][4], al[MI][4];
+#pragma unroll
+      for (int mi = 0; mi < MI; ++mi) {
+        uint32_t w[4];
+        ldm_x4(w, A[a] + 16 * mi * lda + aoff + k0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) split_bits(w[q], ah[mi][q], al[mi][q]);
+      }
+#pragma unroll
+      for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[a][mi][ni], al[mi], bh[ni]);
+#pragma unroll
+      for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[a][mi][ni], ah[mi], bl[ni]);
+#pragma unroll
+      for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[a][mi][ni], ah[mi], bh[ni]);
+    }
+  }
+}
+
 // E(m, n, value) for every element of the warp tile's accumulator.
 template <int MI, int NI, class FE>
 __device__ __forceinline__ void warp_epilogue(const float (&acc)[MI][NI][4], FE E, int lane) {
@@ -854,17 +916,15 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   }
   {  // warps 0-3: dP = lower-incl(dO U^T); warps 4-7: dL = -strictly-lower(dV~ U^T); 32 x 32 tiles
     const int m0 = ((warp & 3) >> 1) * 32, n0 = (warp & 1) * 32;
-    const float* X = warp < 4 ? dOs : dVt;
-    float acc[2][4][4] = {};
-    warp_gemm<2, 4, DV>(
-        acc, [&](int m, int k) { return X[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return U[(n0 + nn) * LDV + k]; },
-        lane);
+    const float* const X[1] = {(warp < 4 ? dOs : dVt) + m0 * LDV};
+    float acc[1][2][4][4] = {};
+    warp_gemm_ldm<1, 2, 4, DV>(acc, X, LDV, U + n0 * LDV, LDV, lane);
     const int diag = a.pre_read ? 0 : 1;
     if (warp < 4)
-      warp_epilogue(acc, [&](int m, int nn, float v) { dP[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m + diag ? v : 0.f; },
+      warp_epilogue(acc[0], [&](int m, int nn, float v) { dP[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m + diag ? v : 0.f; },
                     lane);
     else
-      warp_epilogue(acc, [&](int m, int nn, float v) { dL[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? -v : 0.f; }, lane);
+      warp_epilogue(acc[0], [&](int m, int nn, float v) { dL[(m0 + m) * kLDC + n0 + nn] = n0 + nn < m0 + m ? -v : 0.f; }, lane);
   }
   __syncthreads();
 
@@ -883,25 +943,31 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
     tc::cp_async_commit();
     tc::cp_async_wait_all();
     __syncthreads();
-    float aq[1][2][4] = {}, ak[1][2][4] = {}, aw[1][2][4] = {}, ax[1][NIX][4] = {};
+    float aqk[2][1][2][4] = {}, aw1[1][1][2][4] = {}, ax[1][NIX][4] = {};
+    float(&aq)[1][2][4] = aqk[0];
+    float(&ak)[1][2][4] = aqk[1];
+    float(&aw)[1][2][4] = aw1[0];
+    {  // dO S_m^T and dV~ S_m^T in one pass over the shared S_m fragments
+      const float* const X[2] = {dOs + m0 * LDV, dVt + m0 * LDV};
+      warp_gemm_ldm<2, 1, 2, DV>(aqk, X, LDV, Sm + n0 * LDV, LDV, lane);
+    }
+#pragma unroll
+    for (int ni = 0; ni < 2; ++ni)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ak[0][ni][q] = -ak[0][ni][q];
     // dQ+ = dO S_m^T + dP W-
-    warp_gemm<1, 2, DV>(
-        aq, [&](int m, int k) { return dOs[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return Sm[(n0 + nn) * LDV + k]; },
-        lane);
     warp_gemm<1, 2, kC>(
         aq, [&](int m, int k) { return dP[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return Wm[k * LDS + n0 + nn]; },
         lane);
     // dK+ = -dV~ S_m^T + dL W-
-    warp_gemm<1, 2, DV>(
-        ak, [&](int m, int k) { return -dVt[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return Sm[(n0 + nn) * LDV + k]; },
-        lane);
     warp_gemm<1, 2, kC>(
         ak, [&](int m, int k) { return dL[(m0 + m) * kLDC + k]; }, [&](int k, int nn) { return Wm[k * LDS + n0 + nn]; },
         lane);
     // dW- = U dX^T + dP^T Q+ + dL^T K+
-    warp_gemm<1, 2, DV>(
-        aw, [&](int m, int k) { return U[(m0 + m) * LDV + k]; }, [&](int k, int nn) { return dX[(n0 + nn) * LDV + k]; },
-        lane);
+    {
+      const float* const X[1] = {U + m0 * LDV};
+      warp_gemm_ldm<1, 1, 2, DV>(aw1, X, LDV, dX + n0 * LDV, LDV, lane);
+    }
     warp_gemm<1, 2, kC>(
         aw, [&](int m, int k) { return dP[k * kLDC + m0 + m]; }, [&](int k, int nn) { return Qp[k * LDS + n0 + nn]; },
         lane);
