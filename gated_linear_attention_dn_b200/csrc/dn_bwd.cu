@@ -83,6 +83,9 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) 
 template <int MI, int NI, int K, class FA, class FB>
 __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, int lane) {
   const int g = lane >> 2, t = lane & 3;
+  constexpr bool kSplit = MI * NI <= 4;
+  constexpr int AM = kSplit ? MI : 1, AN = kSplit ? NI : 1;
+  float acc_b[AM][AN][4] = {}, acc_c[AM][AN][4] = {};
 #pragma unroll 2
   for (int k0 = 0; k0 < K; k0 += 8) {
     uint32_t ah[MI][4], al[MI][4];
@@ -99,8 +102,8 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, i
       split_tf32(B(k0 + t, 8 * ni + g), bh[ni][0], bl[ni][0]);
       split_tf32(B(k0 + t + 4, 8 * ni + g), bh[ni][1], bl[ni][1]);
     }
-    // the three products of a fragment go to the same accumulator; issuing each round over all
-    // fragments keeps MI * NI independent products in flight instead of one dependent chain
+    // issuing each round over all fragments keeps MI * NI independent products in flight; with
+    // few fragments the three products also go to three accumulators, summed at the end
 #pragma unroll
     for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
@@ -108,11 +111,19 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, i
 #pragma unroll
     for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
-      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[mi][ni], ah[mi], bl[ni]);
+      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(kSplit ? acc_b[mi % AM][ni % AN] : acc[mi][ni], ah[mi], bl[ni]);
 #pragma unroll
     for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
-      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[mi][ni], ah[mi], bh[ni]);
+      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(kSplit ? acc_c[mi % AM][ni % AN] : acc[mi][ni], ah[mi], bh[ni]);
+  }
+  if constexpr (kSplit) {
+#pragma unroll
+    for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+      for (int ni = 0; ni < NI; ++ni)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[mi][ni][q] += acc_b[mi][ni][q] + acc_c[mi][ni][q];
   }
 }
 
@@ -140,6 +151,9 @@ __device__ __forceinline__ void warp_gemm_ldm(float (&acc)[NA][MI][NI][4], const
                                               const float* Bt, int ldb, int lane) {
   static_assert(NI % 2 == 0 && K % 8 == 0, "tiles");
   const int j = lane >> 3, r = lane & 7;
+  constexpr bool kSplit = NA * MI * NI <= 4;  // three accumulators per fragment, as in warp_gemm
+  constexpr int AA = kSplit ? NA : 1, AM = kSplit ? MI : 1, AN = kSplit ? NI : 1;
+  float acc_b[AA][AM][AN][4] = {}, acc_c[AA][AM][AN][4] = {};
   const int aoff = ((j & 1) * 8 + r) * lda + (j >> 1) * 4;  // tiles: rows 0-7 / 8-15, k 0-3 / 4-7
   const int boff = ((j >> 1) * 8 + r) * ldb + (j & 1) * 4;  // tiles: n 0-7 / 8-15, k 0-3 / 4-7
 #pragma unroll 4
@@ -169,12 +183,24 @@ __device__ __forceinline__ void warp_gemm_ldm(float (&acc)[NA][MI][NI][4], const
 #pragma unroll
       for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[a][mi][ni], ah[mi], bl[ni]);
+        for (int ni = 0; ni < NI; ++ni)
+          ut::mma_tf32(kSplit ? acc_b[a % AA][mi % AM][ni % AN] : acc[a][mi][ni], ah[mi], bl[ni]);
 #pragma unroll
       for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
-        for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[a][mi][ni], ah[mi], bh[ni]);
+        for (int ni = 0; ni < NI; ++ni)
+          ut::mma_tf32(kSplit ? acc_c[a % AA][mi % AM][ni % AN] : acc[a][mi][ni], ah[mi], bh[ni]);
     }
+  }
+  if constexpr (kSplit) {
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+      for (int mi = 0; mi < MI; ++mi)
+#pragma unroll
+        for (int ni = 0; ni < NI; ++ni)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[a][mi][ni][q] += acc_b[a][mi][ni][q] + acc_c[a][mi][ni][q];
   }
 }
 
