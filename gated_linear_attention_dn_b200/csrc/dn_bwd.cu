@@ -878,55 +878,118 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
       xu[it] = Ug[tid + it * kNT];
       xv[it] = dVg[tid + it * kNT];
     }
+    // dO rows in 16-byte vectors (8 bf16 or 4 fp32 values), issued with the loads above; rows past the
+    // end read the chunk's first row and are stored as zeros
+    constexpr int VB = DV / 8, PB = kC * VB / kNT, VF = DV / 4, PF = kC * VF / kNT;
+    const int64_t tok0 = token(a, b, h, t0);
+    const uint4* dOg = reinterpret_cast<const uint4*>(p.dO);
+    uint4 xo[PF];
+    if (a.io_bf16) {
+#pragma unroll
+      for (int u = 0; u < PB; ++u) {
+        const int e = tid + u * kNT, t = e / VB;
+        xo[u] = dOg[(tok0 + (int64_t)(t < n ? t : 0) * a.H) * VB + e % VB];
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < PF; ++u) {
+        const int e = tid + u * kNT, t = e / VF;
+        xo[u] = dOg[(tok0 + (int64_t)(t < n ? t : 0) * a.H) * VF + e % VF];
+      }
+    }
 #pragma unroll
     for (int it = 0; it < PER4; ++it) {
       const int e = (tid + it * kNT) * 4, t = e / DV, j = e % DV;
       *reinterpret_cast<float4*>(&U[t * LDV + j]) = xu[it];
       *reinterpret_cast<float4*>(&dVt[t * LDV + j]) = xv[it];
     }
-    const int64_t tok0 = token(a, b, h, t0);
-    for (int it0 = 0; it0 < kC * DV / kNT; it0 += 8) {
-      float x[8];
-      int tt[8], cj[8];
+    if (a.io_bf16) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
-        tt[u] = t < n ? t : 0;
-        cj[u] = j;
+      for (int u = 0; u < PB; ++u) {
+        const int e = tid + u * kNT, t = e / VB, j = (e % VB) * 8;
+        const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xo[u]);
+        float f[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 y = __bfloat1622float2(x2[q]);
+          f[2 * q] = t < n ? y.x : 0.f;
+          f[2 * q + 1] = t < n ? y.y : 0.f;
+        }
+        *reinterpret_cast<float4*>(&dOs[t * LDV + j]) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(&dOs[t * LDV + j + 4]) = make_float4(f[4], f[5], f[6], f[7]);
       }
-      io_load_n<8>(x, p.dO, tok0, tt, a.H, cj, DV, a.io_bf16);
+    } else {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = tid + (it0 + u) * kNT;
-        dOs[(e / DV) * LDV + e % DV] = (e / DV) < n ? x[u] : 0.f;
+      for (int u = 0; u < PF; ++u) {
+        const int e = tid + u * kNT, t = e / VF, j = (e % VF) * 4;
+        const float4 y = *reinterpret_cast<const float4*>(&xo[u]);
+        *reinterpret_cast<float4*>(&dOs[t * LDV + j]) = t < n ? y : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     if (tid < kC) acc_a[tid] = acc_bk[tid] = acc_d[tid] = 0.f;
   }
   __syncthreads();
-  // dv = beta^v dV~, and the beta^v gradient v dV~ (summed over channels for a per-token gate)
-  for (int it0 = 0; it0 < kC * DV / kNT; it0 += 8) {
-    float bv[8], vv[8];
-    int tt[8], cj[8];
+  // dv = beta^v dV~, and the beta^v gradient v dV~ (summed over channels for a per-token gate); eight
+  // columns of a row per vector, every load of the thread issued before any is used
+  {
+    constexpr int V8 = DV / 8, P8 = kC * V8 / kNT;
+    const int64_t tok0 = token(a, b, h, t0);
+    float bv[P8][8], vv[P8][8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
-      tt[u] = t < n ? t : 0;
-      cj[u] = j;
-    }
-    {
-      const int64_t tok0 = token(a, b, h, t0);
-      gate_load_n<8>(bv, a.beta_v_p, a.beta_v, tok0, tt, a.H, cj, DV);
-      if (a.beta_v == DN_GATE_CHANNEL) io_load_n<8>(vv, a.v, tok0, tt, a.H, cj, DV, a.io_bf16);
+    for (int u = 0; u < P8; ++u) {
+      const int e = tid + u * kNT, t = e / V8, j = (e % V8) * 8;
+      const int64_t r = tok0 + (int64_t)(t < n ? t : 0) * a.H;
+      if (a.beta_v == DN_GATE_CHANNEL) {
+        const float4 b0 = *reinterpret_cast<const float4*>(a.beta_v_p + r * DV + j);
+        const float4 b1 = *reinterpret_cast<const float4*>(a.beta_v_p + r * DV + j + 4);
+        bv[u][0] = b0.x, bv[u][1] = b0.y, bv[u][2] = b0.z, bv[u][3] = b0.w;
+        bv[u][4] = b1.x, bv[u][5] = b1.y, bv[u][6] = b1.z, bv[u][7] = b1.w;
+        if (a.io_bf16) {
+          const uint4 x = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + r * DV + j);
+          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 y = __bfloat1622float2(x2[q]);
+            vv[u][2 * q] = y.x, vv[u][2 * q + 1] = y.y;
+          }
+        } else {
+          const float4 v0 = *reinterpret_cast<const float4*>(static_cast<const float*>(a.v) + r * DV + j);
+          const float4 v1 = *reinterpret_cast<const float4*>(static_cast<const float*>(a.v) + r * DV + j + 4);
+          vv[u][0] = v0.x, vv[u][1] = v0.y, vv[u][2] = v0.z, vv[u][3] = v0.w;
+          vv[u][4] = v1.x, vv[u][5] = v1.y, vv[u][6] = v1.z, vv[u][7] = v1.w;
+        }
+      } else {
+        const float x = a.beta_v == DN_GATE_SCALAR ? a.beta_v_p[r] : 1.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) bv[u][q] = x, vv[u][q] = 0.f;
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = tid + (it0 + u) * kNT, t = e / DV, j = e % DV;
+    for (int u = 0; u < P8; ++u) {
+      const int e = tid + u * kNT, t = e / V8, j = (e % V8) * 8;
       if (t < n) {
-        const int64_t tok = token(a, b, h, t0 + t);
-        const float dvt = dVt[t * LDV + j];
-        io_store(p.gv, tok * DV + j, bv[u] * dvt, a.io_bf16);
-        if (a.beta_v == DN_GATE_CHANNEL) p.gbeta_v[tok * DV + j] = vv[u] * dvt;
+        const int64_t r = tok0 + (int64_t)t * a.H;
+        const float4 d0 = *reinterpret_cast<const float4*>(&dVt[t * LDV + j]);
+        const float4 d1 = *reinterpret_cast<const float4*>(&dVt[t * LDV + j + 4]);
+        const float dv8[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+        float g8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) g8[q] = bv[u][q] * dv8[q];
+        if (a.io_bf16) {
+          uint4 o;
+          __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) o2[q] = __floats2bfloat162_rn(g8[2 * q], g8[2 * q + 1]);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.gv) + r * DV + j) = o;
+        } else {
+          float* o = static_cast<float*>(p.gv) + r * DV + j;
+          *reinterpret_cast<float4*>(o) = make_float4(g8[0], g8[1], g8[2], g8[3]);
+          *reinterpret_cast<float4*>(o + 4) = make_float4(g8[4], g8[5], g8[6], g8[7]);
+        }
+        if (a.beta_v == DN_GATE_CHANNEL) {  // (gate gradients need only fp32 alignment: scalar stores)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) p.gbeta_v[r * DV + j + q] = vv[u][q] * dv8[q];
+        }
       }
     }
   }
@@ -1080,14 +1143,27 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
 #pragma unroll
       for (int ni = 0; ni < 2; ++ni)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int t = m0 + g + (q >> 1) * 8, gi = i0 + n0 + 8 * ni + 2 * t4 + (q & 1);
+        for (int q = 0; q < 4; q += 2) {  // elements q and q + 1: the same token, channels gi and gi + 1
+          const int t = m0 + g + (q >> 1) * 8, gi = i0 + n0 + 8 * ni + 2 * t4;
           if (t < n) {
-            const int64_t tok = token(a, b, h, t0 + t);
-            io_store(p.gq, tok * DK + gi, gq[ni][q], a.io_bf16);
-            io_store(p.gk, tok * DK + gi, gk[ni][q], a.io_bf16);
-            if (a.beta_k == DN_GATE_CHANNEL) p.gbeta_k[tok * DK + gi] = Qp[t * LDS + gi - i0];
-            if (a.key_scale == DN_GATE_CHANNEL) p.gkey_scale[tok * DK + gi] = Kp[t * LDS + gi - i0];
+            const int64_t o = token(a, b, h, t0 + t) * DK + gi;
+            if (a.io_bf16) {
+              *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.gq) + o) =
+                  __floats2bfloat162_rn(gq[ni][q], gq[ni][q + 1]);
+              *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.gk) + o) =
+                  __floats2bfloat162_rn(gk[ni][q], gk[ni][q + 1]);
+            } else {
+              *reinterpret_cast<float2*>(static_cast<float*>(p.gq) + o) = make_float2(gq[ni][q], gq[ni][q + 1]);
+              *reinterpret_cast<float2*>(static_cast<float*>(p.gk) + o) = make_float2(gk[ni][q], gk[ni][q + 1]);
+            }
+            if (a.beta_k == DN_GATE_CHANNEL) {
+              p.gbeta_k[o] = Qp[t * LDS + gi - i0];
+              p.gbeta_k[o + 1] = Qp[t * LDS + gi + 1 - i0];
+            }
+            if (a.key_scale == DN_GATE_CHANNEL) {
+              p.gkey_scale[o] = Kp[t * LDS + gi - i0];
+              p.gkey_scale[o + 1] = Kp[t * LDS + gi + 1 - i0];
+            }
           }
         }
     }
@@ -1095,10 +1171,25 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
     // d log alpha_s = sum_{t >= s} dh_t + rowsum(dX (.) X) (the last token's share), per channel: the
     // suffix sums in shared memory (a dependent chain over the tokens), then d alpha = d log alpha /
     // alpha for every (token, channel) of the slice at once
-    for (int il = tid; il < kDKS; il += kNT) {
+    {  // warp w sums tokens 8w .. 8w + 7 of channel (lane); the segments' totals go through S_m's
+       // buffer, free until the next slice's loads
+      static_assert(kNT == 8 * kDKS && kC == 64, "eight segments of eight tokens, one per warp");
+      const int il = tid % kDKS, sg = tid / kDKS;
+      float x[8], tot = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        x[q] = Wm[(8 * sg + q) * LDS + il];
+        tot += x[q];
+      }
+      float* seg = Sm;
+      seg[sg * kDKS + il] = tot;
+      __syncthreads();
       float run = red[il] + red[kDKS + il] + red[2 * kDKS + il] + red[3 * kDKS + il];
-      for (int t = kC - 1; t >= 0; --t) {
-        run += Wm[t * LDS + il];
+      for (int s2 = sg + 1; s2 < 8; ++s2) run += seg[s2 * kDKS + il];
+#pragma unroll
+      for (int q = 7; q >= 0; --q) {
+        const int t = 8 * sg + q;
+        run += x[q];
         Wm[t * LDS + il] = a.pre_read ? run - Xq[t * LDS + il] : run;
       }
     }
