@@ -618,11 +618,15 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
     tc::cp_async_wait_group<2>();  // A1(c) has landed (A2(c), B(c) may still be in flight)
     __syncthreads();
     float* Smg = p.wSm + cb * DK * DV;
-    for (int e = tid; e < DK * DVS; e += kNT) {
-      const int i = e / DVS, j = e % DVS;
-      const float x = S[i * LDS + j] * er[i];
-      S[i * LDS + j] = x;
-      Smg[(int64_t)i * DV + j0 + j] = x;
+    for (int e = tid; e < DK * DVS / 4; e += kNT) {  // four columns per thread: 16-byte stores
+      const int i = e / (DVS / 4), j = (e % (DVS / 4)) * 4;
+      float2* r = reinterpret_cast<float2*>(&S[i * LDS + j]);  // (rows are 8-byte aligned)
+      const float f = er[i];
+      const float2 x0 = r[0], x1 = r[1];
+      const float4 y = make_float4(x0.x * f, x0.y * f, x1.x * f, x1.y * f);
+      r[0] = make_float2(y.x, y.y);
+      r[1] = make_float2(y.z, y.w);
+      *reinterpret_cast<float4*>(&Smg[(int64_t)i * DV + j0 + j]) = y;
     }
     __syncthreads();
     if (tiled) {  // R = V~ - K+ S_m (each warp updates only its own tile)
@@ -773,11 +777,15 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
     tc::cp_async_wait_group<1>();  // A1(c) and A2(c) have landed (B(c) may still be in flight)
     __syncthreads();               // and for every thread; dO(c) is stored; the previous step is done
     float* dXg = p.wdX + cb * DK * DV;
-    for (int e = tid; e < DK * DVS; e += kNT) {
-      const int i = e / DVS, j = e % DVS;
-      const float x = dS[i * LDS + j] * lam[i];
-      dS[i * LDS + j] = x;
-      dXg[(int64_t)i * DV + j0 + j] = x;
+    for (int e = tid; e < DK * DVS / 4; e += kNT) {  // four columns per thread: 16-byte stores
+      const int i = e / (DVS / 4), j = (e % (DVS / 4)) * 4;
+      float2* r = reinterpret_cast<float2*>(&dS[i * LDS + j]);  // (rows are 8-byte aligned)
+      const float f = lam[i];
+      const float2 x0 = r[0], x1 = r[1];
+      const float4 y = make_float4(x0.x * f, x0.y * f, x1.x * f, x1.y * f);
+      r[0] = make_float2(y.x, y.y);
+      r[1] = make_float2(y.z, y.w);
+      *reinterpret_cast<float4*>(&dXg[(int64_t)i * DV + j0 + j]) = y;
     }
     __syncthreads();
     {  // dU = P^T dO + W- dX
