@@ -353,6 +353,10 @@ __device__ void prep_chunk(const Args& a, int b, int h, int t0, int n, int i0, f
 }
 
 constexpr int kLDC = kC + 4;  // row stride of shared 64 x 64 arrays
+template <int DVS>
+constexpr int kLdsState = DVS + 4;
+template <int DVS>
+constexpr int kLdsDstate = DVS + 8;
 
 // cp.async copy of a ROWS x COLS fp32 block (global row stride gs floats) into shared rows of ss
 // floats; 16-byte granules, so COLS, gs, ss and both bases must be multiples of 4 floats. The caller
@@ -485,7 +489,9 @@ __global__ void __launch_bounds__(kNT) bwd_prep_kernel(BwdArgs p) {
 template <int DK, int DV, int DVS, int C = kC>
 __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDS = DVS + 2, LDC = C + 4, NI = DVS / 16;
+  // row stride of the [.][DVS] arrays: = 4 (mod 32) banks, so the lanes of a B fragment (rows t, columns
+  // g) fall on at most two of them, with two CTAs per SM still fitting
+  constexpr int LDK = DK + 4, LDS = kLdsState<DVS>, LDC = C + 4, NI = DVS / 16;
   // warp tiles of the C x DVS products: RT x CT tiles of 16 x TW (with C = 16 and 32 columns, four warps)
   constexpr int RT = C / 16, CT = (8 / RT < DVS / 8) ? 8 / RT : DVS / 8, TW = DVS / CT, NIT = TW / 8;
   static_assert(RT * CT <= 8 && TW % 8 == 0, "warp tiles");
@@ -695,7 +701,9 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
 template <int DK, int DV, int DVS>
 __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDK = DK + 4, LDS = DVS + 2, NI = DVS / 16;
+  // row stride of the [.][DVS] arrays: = 8 (mod 32) banks, so the 32 lanes of a B fragment (rows t,
+  // columns g) fall on 32 different banks
+  constexpr int LDK = DK + 4, LDS = kLdsDstate<DVS>, NI = DVS / 16;
   constexpr int PER = kC * DVS / kNT;
   float* dS = reinterpret_cast<float*>(smem4);  // [DK][LDS]: dS', then dX, then dS
   float* Qp = dS + DK * LDS;                     // [C][LDK]
@@ -1280,11 +1288,11 @@ constexpr size_t prep_smem() {
 }
 template <int DK, int DVS, int C = kC>
 constexpr size_t state_smem() {
-  return sizeof(float) * (DK * (DVS + 2) + 2 * C * (DK + 4) + C * (C + 4) + C * (DVS + 2) + 4 * DK);
+  return sizeof(float) * (DK * kLdsState<DVS> + 2 * C * (DK + 4) + C * (C + 4) + C * kLdsState<DVS> + 4 * DK);
 }
 template <int DK, int DVS>
 constexpr size_t dstate_smem() {
-  return sizeof(float) * (DK * (DVS + 2) + 3 * kC * (DK + 4) + 2 * kC * kLDC + 3 * kC * (DVS + 2) + 4 * DK);
+  return sizeof(float) * (DK * kLdsDstate<DVS> + 3 * kC * (DK + 4) + 2 * kC * kLDC + 3 * kC * kLdsDstate<DVS> + 4 * DK);
 }
 template <int DV>
 constexpr size_t local_smem() {
@@ -1310,6 +1318,7 @@ cudaError_t launch_dims(const BwdArgs& p, cudaStream_t s) {
   constexpr int S1 = kDVS_STATE, S2 = kDVS_DSTATE < DV ? kDVS_DSTATE : DV;
   static_assert(DV % S1 == 0 && DV % S2 == 0, "d_v slices");
   static_assert(local_smem<DV>() <= 227 * 1024 && dstate_smem<DK, S2>() <= 227 * 1024, "shared memory");
+  static_assert(state_smem<DK, S1>() <= 113 * 1024, "two state-chain CTAs per SM");
   const int64_t bh = (int64_t)p.f.B * p.f.H;
   const unsigned chunks = (unsigned)(bh * p.nc);
   cudaError_t e;
