@@ -491,14 +491,15 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
   // row stride of the [.][DVS] arrays: = 4 (mod 32) banks, so the lanes of a B fragment (rows t, columns
   // g) fall on at most two of them, with two CTAs per SM still fitting
-  constexpr int LDK = DK + 4, LDS = kLdsState<DVS>, LDC = C + 4, NI = DVS / 16;
+  // (W- is read only transposed, rows t and columns g of a fragment: its stride is = 8 (mod 32) banks)
+  constexpr int LDK = DK + 4, LDW = DK + 8, LDS = kLdsState<DVS>, LDC = C + 4, NI = DVS / 16;
   // warp tiles of the C x DVS products: RT x CT tiles of 16 x TW (with C = 16 and 32 columns, four warps)
   constexpr int RT = C / 16, CT = (8 / RT < DVS / 8) ? 8 / RT : DVS / 8, TW = DVS / CT, NIT = TW / 8;
   static_assert(RT * CT <= 8 && TW % 8 == 0, "warp tiles");
   float* S = reinterpret_cast<float*>(smem4);  // [DK][LDS]
   float* Kp = S + DK * LDS;                     // [C][LDK]
-  float* Wm = Kp + C * LDK;                     // [C][LDK]
-  float* Tm = Wm + C * LDK;                     // [C][LDC]
+  float* Wm = Kp + C * LDK;                     // [C][LDW]
+  float* Tm = Wm + C * LDW;                     // [C][LDC]
   float* R = Tm + C * LDC;                      // [C][LDS]: V~ - K+ S_m, then U
   float* erb = R + C * LDS;                     // [2][DK] (chunk parity)
   float* lamb = erb + 2 * DK;                   // [2][DK]
@@ -525,7 +526,7 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
     tc::cp_async_commit();
   };
   auto issue_b = [&](int c) {
-    if (c < p.nc) async_rows<C, DK>(Wm, LDK, p.wWm + cbk(c) * C * DK, DK, tid);
+    if (c < p.nc) async_rows<C, DK>(Wm, LDW, p.wWm + cbk(c) * C * DK, DK, tid);
     tc::cp_async_commit();
   };
   auto load_v = [&](int c, float* x) {  // V~ = beta^v v of chunk c, this thread's elements
@@ -670,7 +671,7 @@ __global__ void __launch_bounds__(kNT) bwd_state_kernel(BwdArgs p) {
       const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * (DVS / 2);
       float acc[1][NI][4] = {};
       warp_gemm<1, NI, C>(
-          acc, [&](int m, int k) { return Wm[k * LDK + r0 + m]; }, [&](int k, int nn) { return R[k * LDS + q0 + nn]; },
+          acc, [&](int m, int k) { return Wm[k * LDW + r0 + m]; }, [&](int k, int nn) { return R[k * LDS + q0 + nn]; },
           lane);
       warp_epilogue(acc,
                     [&](int m, int nn, float v) {
@@ -703,12 +704,13 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
   // row stride of the [.][DVS] arrays: = 8 (mod 32) banks, so the 32 lanes of a B fragment (rows t,
   // columns g) fall on 32 different banks
-  constexpr int LDK = DK + 4, LDS = kLdsDstate<DVS>, NI = DVS / 16;
+  // (Q+ and K+ are read only transposed: their stride is = 8 (mod 32) banks; W- is read by rows)
+  constexpr int LDK = DK + 4, LDQ = DK + 8, LDS = kLdsDstate<DVS>, NI = DVS / 16;
   constexpr int PER = kC * DVS / kNT;
   float* dS = reinterpret_cast<float*>(smem4);  // [DK][LDS]: dS', then dX, then dS
-  float* Qp = dS + DK * LDS;                     // [C][LDK]
-  float* Kp = Qp + kC * LDK;
-  float* Wm = Kp + kC * LDK;
+  float* Qp = dS + DK * LDS;                     // [C][LDQ]
+  float* Kp = Qp + kC * LDQ;                     // [C][LDQ]
+  float* Wm = Kp + kC * LDQ;                     // [C][LDK]
   float* Tm = Wm + kC * LDK;  // [C][kLDC]
   float* Pm = Tm + kC * kLDC;
   float* dO0 = Pm + kC * kLDC;  // [C][LDS] x 2 (chunk parity)
@@ -736,8 +738,8 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
   };
   auto issue_b = [&](int c) {
     if (c >= 0) {
-      async_rows<kC, DK>(Qp, LDK, p.wQp + cbk(c) * kC * DK, DK, tid);
-      async_rows<kC, DK>(Kp, LDK, p.wKp + cbk(c) * kC * DK, DK, tid);
+      async_rows<kC, DK>(Qp, LDQ, p.wQp + cbk(c) * kC * DK, DK, tid);
+      async_rows<kC, DK>(Kp, LDQ, p.wKp + cbk(c) * kC * DK, DK, tid);
     }
     tc::cp_async_commit();
   };
@@ -832,10 +834,10 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
       const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * (DVS / 2);
       float acc[1][NI][4] = {};
       warp_gemm<1, NI, kC>(
-          acc, [&](int m, int k) { return Qp[k * LDK + r0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + q0 + nn]; },
+          acc, [&](int m, int k) { return Qp[k * LDQ + r0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + q0 + nn]; },
           lane);
       warp_gemm<1, NI, kC>(
-          acc, [&](int m, int k) { return -Kp[k * LDK + r0 + m]; }, [&](int k, int nn) { return dU[k * LDS + q0 + nn]; },
+          acc, [&](int m, int k) { return -Kp[k * LDQ + r0 + m]; }, [&](int k, int nn) { return dU[k * LDS + q0 + nn]; },
           lane);
       warp_epilogue(acc,
                     [&](int m, int nn, float v) {
@@ -862,7 +864,8 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
 template <int DK, int DV>
 __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
   extern __shared__ float4 smem4[];
-  constexpr int LDV = DV + 4, LDS = kDKS + 4;
+  // LDS: = 8 (mod 32) banks, for the [C][kDKS] tiles read as transposed fragments (rows t, columns g)
+  constexpr int LDV = DV + 4, LDS = kDKS + 8;
   float* U = reinterpret_cast<float*>(smem4);  // [C][LDV]
   float* dVt = U + kC * LDV;
   float* dOs = dVt + kC * LDV;
@@ -1217,17 +1220,28 @@ __global__ void __launch_bounds__(kNT) bwd_local_kernel(BwdArgs p) {
         p.galpha[tok * DK + i0 + il] = Wm[t * LDS + il] / gate_load(a.alpha_p, a.alpha, tok, DK, i0 + il);
       }
     }
-    // per-token sums over these channels, for gates of width 1
-    if (tid < kC) {
+    {  // per-token sums over these channels, for gates of width 1: four threads per token
+      static_assert(kNT == 4 * kC && kDKS % 4 == 0, "four threads per token");
+      const int t = tid >> 2, part = tid & 3;
       float sa = 0.f, sb = 0.f, sd = 0.f;
-      for (int il = 0; il < kDKS; ++il) {
-        sa += Wm[tid * LDS + il];
-        sb += Qp[tid * LDS + il];
-        sd += Kp[tid * LDS + il];
+#pragma unroll
+      for (int q = 0; q < kDKS / 4; ++q) {
+        const int il = 4 * q + part;
+        sa += Wm[t * LDS + il];
+        sb += Qp[t * LDS + il];
+        sd += Kp[t * LDS + il];
       }
-      acc_a[tid] += sa;
-      acc_bk[tid] += sb;
-      acc_d[tid] += sd;
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1) {
+        sa += __shfl_xor_sync(0xffffffffu, sa, off);
+        sb += __shfl_xor_sync(0xffffffffu, sb, off);
+        sd += __shfl_xor_sync(0xffffffffu, sd, off);
+      }
+      if (part == 0) {
+        acc_a[t] += sa;
+        acc_bk[t] += sb;
+        acc_d[t] += sd;
+      }
     }
     __syncthreads();
   }
@@ -1288,15 +1302,16 @@ constexpr size_t prep_smem() {
 }
 template <int DK, int DVS, int C = kC>
 constexpr size_t state_smem() {
-  return sizeof(float) * (DK * kLdsState<DVS> + 2 * C * (DK + 4) + C * (C + 4) + C * kLdsState<DVS> + 4 * DK);
+  return sizeof(float) * (DK * kLdsState<DVS> + C * (DK + 4) + C * (DK + 8) + C * (C + 4) + C * kLdsState<DVS> + 4 * DK);
 }
 template <int DK, int DVS>
 constexpr size_t dstate_smem() {
-  return sizeof(float) * (DK * kLdsDstate<DVS> + 3 * kC * (DK + 4) + 2 * kC * kLDC + 3 * kC * kLdsDstate<DVS> + 4 * DK);
+  return sizeof(float) *
+         (DK * kLdsDstate<DVS> + 2 * kC * (DK + 8) + kC * (DK + 4) + 2 * kC * kLDC + 3 * kC * kLdsDstate<DVS> + 4 * DK);
 }
 template <int DV>
 constexpr size_t local_smem() {
-  return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 5 * kC * (kDKS + 4) + 4 * kDKS +
+  return sizeof(float) * (3 * kC * (DV + 4) + 2 * kC * kLDC + 2 * kDKS * (DV + 4) + 5 * kC * (kDKS + 8) + 4 * kDKS +
                           3 * kC);
 }
 
