@@ -80,7 +80,9 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) 
 
 // acc[MI][NI] (16 x 8 fragments) += sum_{k < K} A(m, k) B(k, n) over the warp tile of 16 MI rows and
 // 8 NI columns, with x = hi + lo split operands: a b ~ a_lo b_hi + a_hi b_lo + a_hi b_hi.
-template <int MI, int NI, int K, class FA, class FB>
+// BEXACT: every B(k, n) is a TF32 value (bf16 data, say), so its lo part is zero and the a_hi b_lo
+// product is left out.
+template <int MI, int NI, int K, bool BEXACT = false, class FA, class FB>
 __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, int lane) {
   const int g = lane >> 2, t = lane & 3;
   constexpr bool kSplit = MI * NI <= 4;
@@ -99,8 +101,13 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, i
     uint32_t bh[NI][2], bl[NI][2];
 #pragma unroll
     for (int ni = 0; ni < NI; ++ni) {
-      split_tf32(B(k0 + t, 8 * ni + g), bh[ni][0], bl[ni][0]);
-      split_tf32(B(k0 + t + 4, 8 * ni + g), bh[ni][1], bl[ni][1]);
+      if constexpr (BEXACT) {
+        bh[ni][0] = __float_as_uint(B(k0 + t, 8 * ni + g));
+        bh[ni][1] = __float_as_uint(B(k0 + t + 4, 8 * ni + g));
+      } else {
+        split_tf32(B(k0 + t, 8 * ni + g), bh[ni][0], bl[ni][0]);
+        split_tf32(B(k0 + t + 4, 8 * ni + g), bh[ni][1], bl[ni][1]);
+      }
     }
     // issuing each round over all fragments keeps MI * NI independent products in flight; with
     // few fragments the three products also go to three accumulators, summed at the end
@@ -108,10 +115,12 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MI][NI][4], FA A, FB B, i
     for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
       for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(acc[mi][ni], al[mi], bh[ni]);
+    if constexpr (!BEXACT) {
 #pragma unroll
-    for (int mi = 0; mi < MI; ++mi)
+      for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
-      for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(kSplit ? acc_b[mi % AM][ni % AN] : acc[mi][ni], ah[mi], bl[ni]);
+        for (int ni = 0; ni < NI; ++ni) ut::mma_tf32(kSplit ? acc_b[mi % AM][ni % AN] : acc[mi][ni], ah[mi], bl[ni]);
+    }
 #pragma unroll
     for (int mi = 0; mi < MI; ++mi)
 #pragma unroll
@@ -798,11 +807,14 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
       *reinterpret_cast<float4*>(&dXg[(int64_t)i * DV + j0 + j]) = y;
     }
     __syncthreads();
-    {  // dU = P^T dO + W- dX
+    {  // dU = P^T dO + W- dX (dO from bf16 io is exact in TF32)
       float acc[1][NI][4] = {};
-      warp_gemm<1, NI, kC>(
-          acc, [&](int m, int k) { return Pm[k * kLDC + m0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + n0 + nn]; },
-          lane);
+      const auto pT = [&](int m, int k) { return Pm[k * kLDC + m0 + m]; };
+      const auto dOb = [&](int k, int nn) { return dOs[k * LDS + n0 + nn]; };
+      if (a.io_bf16)
+        warp_gemm<1, NI, kC, true>(acc, pT, dOb, lane);
+      else
+        warp_gemm<1, NI, kC>(acc, pT, dOb, lane);
       warp_gemm<1, NI, DK>(
           acc, [&](int m, int k) { return Wm[(m0 + m) * LDK + k]; }, [&](int k, int nn) { return dS[k * LDS + n0 + nn]; },
           lane);
@@ -833,9 +845,12 @@ __global__ void __launch_bounds__(kNT) bwd_dstate_kernel(BwdArgs p) {
     for (int tile = warp; tile < (DK / 16) * 2; tile += kNT / 32) {
       const int r0 = (tile >> 1) * 16, q0 = (tile & 1) * (DVS / 2);
       float acc[1][NI][4] = {};
-      warp_gemm<1, NI, kC>(
-          acc, [&](int m, int k) { return Qp[k * LDQ + r0 + m]; }, [&](int k, int nn) { return dOs[k * LDS + q0 + nn]; },
-          lane);
+      const auto qT = [&](int m, int k) { return Qp[k * LDQ + r0 + m]; };
+      const auto dOb = [&](int k, int nn) { return dOs[k * LDS + q0 + nn]; };
+      if (a.io_bf16)
+        warp_gemm<1, NI, kC, true>(acc, qT, dOb, lane);
+      else
+        warp_gemm<1, NI, kC>(acc, qT, dOb, lane);
       warp_gemm<1, NI, kC>(
           acc, [&](int m, int k) { return -Kp[k * LDQ + r0 + m]; }, [&](int k, int nn) { return dU[k * LDS + q0 + nn]; },
           lane);
